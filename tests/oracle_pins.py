@@ -1,0 +1,404 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` function raises ``AssertionError`` when the oracle disagrees
+with what the pages or the mathematics fix.  ``test_oracle_pins.py`` runs them
+on the real oracle; ``test_oracle_mutations.py`` plants plausible mistakes in
+the oracle and checks that at least one pin fails for each.
+
+Independent references used here:
+* torch's ``float8_e4m3fn`` and ``bfloat16`` CPU conversions (library codecs);
+* ``torch.nn.functional.scaled_dot_product_attention`` in float64 on a
+  contiguous ``[heads, seq, dim]`` layout built straight from the generator's
+  values (so the paged write/read path is bypassed);
+* a pure-Python brute force on tiny inputs;
+* closed forms (single token, constant keys, zero query, two tokens, one
+  dominant logit) and the worked block mapping of the TensorRT-LLM deep dive
+  (gentlecold.top, §9: logical blocks 0/1/2 -> physical blocks 17/3/91).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle.pkv_oracle as O
+from paged_kv_attention_block_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------------------
+# Helpers (test side)
+# ---------------------------------------------------------------------------
+
+def oracle_pool_for(w: W.Workload, upto: str = "all"):
+    """Oracle pool holding every token of ``w`` (``upto="all"``) or only history."""
+    pool = O.new_pool(w.num_blocks, w.num_layers, w.num_kv_heads, w.block_size, w.head_dim, w.kv_dtype,
+                      w.k_scale, w.v_scale)
+    k, v, cu, sp = w.packed_kv(upto)
+    O.kv_append(pool, w.layer, k, v, w.kv_in_dtype, cu, sp, w.block_tables)
+    return pool
+
+
+def q64(w: W.Workload) -> np.ndarray:
+    return O.decode_bits(w.q, w.q_dtype) if w.q_dtype != "f32" else w.q.astype(np.float64)
+
+
+def run_oracle(w: W.Workload, pool=None):
+    pool = pool if pool is not None else oracle_pool_for(w)
+    return O.paged_attention(pool, w.layer, q64(w), w.cu_q_lens, w.seq_lens, w.block_tables, w.num_q_heads,
+                             w.softmax_scale, w.causal)
+
+
+def _values64(w: W.Workload, s: int):
+    """Contiguous K/V [seq_len][Hkv][D] of sequence s as the cache holds them (library codecs)."""
+    k, v = w.kv_values(s)
+    if w.kv_dtype == "e4m3":
+        out = []
+        for which, x in ((0, k), (1, v)):
+            sc = (w.k_scale if which == 0 else w.v_scale)[w.layer].astype(np.float32)
+            y = torch.from_numpy(np.ascontiguousarray(x, np.float32) / sc[None, :, None])
+            out.append(y.to(torch.float8_e4m3fn).to(torch.float64).numpy() * sc.astype(np.float64)[None, :, None])
+        return out[0], out[1]
+    if w.kv_dtype == "f32":
+        return k.astype(np.float64), v.astype(np.float64)
+    tdt = torch.bfloat16 if w.kv_dtype == "bf16" else torch.float16
+    conv = lambda x: torch.from_numpy(x.view(np.int16)).view(tdt).to(torch.float64).numpy()  # noqa: E731
+    return conv(k), conv(v)
+
+
+def dense_sdpa(w: W.Workload):
+    """softmax(scale q K^T) V per sequence with torch SDPA, contiguous layout, float64."""
+    qq = q64(w)
+    out = np.full(qq.shape, np.nan)
+    g = w.num_q_heads // w.num_kv_heads
+    cu = w.cu_q_lens
+    for s in range(w.num_seqs):
+        ql, L = int(w.q_lens[s]), int(w.seq_lens[s])
+        if ql == 0:
+            continue
+        k, v = _values64(w, s)
+        K = torch.from_numpy(np.ascontiguousarray(k.transpose(1, 0, 2))).repeat_interleave(g, dim=0)
+        V = torch.from_numpy(np.ascontiguousarray(v.transpose(1, 0, 2))).repeat_interleave(g, dim=0)
+        Q = torch.from_numpy(np.ascontiguousarray(qq[cu[s]:cu[s + 1]].transpose(1, 0, 2)))
+        pos = L - ql + torch.arange(ql)
+        mask = torch.arange(L)[None, :] <= pos[:, None] if w.causal else torch.ones(ql, L, dtype=torch.bool)
+        o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=w.softmax_scale)
+        out[cu[s]:cu[s + 1]] = o.numpy().transpose(1, 0, 2)
+    return out
+
+
+def small_workloads():
+    """Small copies of each workload shape (several tiles, ragged tails)."""
+    return [
+        W.tiny_fp32(seq_lens=(17, 5, 33)),
+        W.llama3_8b_decode_bf16(batch=3, lo=60, hi=200),
+        W.mixed_bf16(n_decode=3, n_prefill=2, chunk=40, dec_lo=30, dec_hi=300, cached_lo_blocks=1,
+                     cached_hi_blocks=3, block_size=16),
+        W.longctx_fp8(batch=2, seq_len=150),
+        W.prefix_reuse_bf16(n_req=3, prefix=256, suf_lo=3, suf_hi=40),
+    ]
+
+
+# ---------------------------------------------------------------------------
+# Number formats
+# ---------------------------------------------------------------------------
+
+def pin_e4m3_decode_table():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin]) and np.array_equal(np.signbit(got[fin]), np.signbit(ref[fin]))
+    # Values the OCP E4M3 definition fixes.
+    assert got[0x7E] == 448.0 and got[0x08] == 2.0 ** -6 and got[0x01] == 2.0 ** -9 and got[0x07] == 7 * 2.0 ** -9
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and got[0x80] == 0.0 and np.signbit(got[0x80])
+
+
+def pin_e4m3_encode():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = O.e4m3_decode(codes)
+    fin = ~np.isnan(vals)
+    # encode(decode(c)) == c for every finite code (including -0).
+    assert np.array_equal(O.e4m3_encode(vals[fin].astype(np.float32)), codes[fin])
+    # Ties go to the even code at every midpoint between neighbouring magnitudes.
+    pos = np.arange(0, 0x7E)
+    lo, hi = O.e4m3_decode(pos), O.e4m3_decode(pos + 1)
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.all(mid.astype(np.float64) == (lo + hi) / 2)
+    want = np.where(pos % 2 == 0, pos, pos + 1)
+    assert np.array_equal(O.e4m3_encode(mid), want.astype(np.uint8))
+    up = np.nextafter(mid, np.float32(np.inf))
+    dn = np.nextafter(mid, np.float32(0))
+    assert np.array_equal(O.e4m3_encode(up), (pos + 1).astype(np.uint8))
+    assert np.array_equal(O.e4m3_encode(dn), pos.astype(np.uint8))
+    # Random values inside the range where torch's (non-saturating) RNE agrees.
+    r = np.random.default_rng(7)
+    x = np.concatenate([r.standard_normal(200000) * 40, r.standard_normal(20000) * 1e-2,
+                        r.uniform(-463.9, 463.9, 20000)]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x), ref)
+    # Saturation to the largest finite value, NaN kept.
+    big = np.array([448, 463.99, 464, 1e6, np.inf, -500, -np.inf, np.nan], np.float32)
+    assert O.e4m3_encode(big).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
+
+
+def pin_bf16_decode():
+    bits = np.arange(0, 65536, 7, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = O.decode_bits(bits, "bf16")
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all()
+
+
+# ---------------------------------------------------------------------------
+# Paged addressing
+# ---------------------------------------------------------------------------
+
+def pin_block_mapping_example():
+    with open(os.path.join(GOLDEN, "block_mapping_example.json")) as f:
+        g = json.load(f)
+    table = np.array(g["block_table"], np.int32)
+    for case in g["cases"]:
+        B = case["block_size"]
+        for p, (phys, slot) in zip(case["positions"], case["expect"]):
+            got = O.block_address(table, p, B)
+            assert (int(got[0]), int(got[1])) == (phys, slot), (p, got, phys, slot)
+    # Append through that table writes exactly those slots and nothing else.
+    B = g["cases"][0]["block_size"]
+    n = 3 * B
+    pool = O.new_pool(100, 1, 1, B, 4, "f32")
+    vals = np.arange(n * 4, dtype=np.float32).reshape(n, 1, 4)
+    O.kv_append(pool, 0, vals, -vals, "f32", np.array([0, n]), np.array([0]), table[None, :])
+    for t in range(n):
+        phys = g["block_table"][t // B]
+        assert np.array_equal(pool.bits[phys, 0, 0, 0, t % B], vals[t, 0])
+        assert np.array_equal(pool.bits[phys, 0, 1, 0, t % B], -vals[t, 0])
+    touched = np.zeros(100, bool)
+    touched[g["block_table"]] = True
+    assert np.isnan(pool.bits[~touched]).all()
+
+
+def pin_append_roundtrip():
+    for w in small_workloads():
+        pool = oracle_pool_for(w)
+        used = np.zeros(w.num_blocks, bool)
+        for s in range(w.num_seqs):
+            k64, v64 = _values64(w, s)
+            L = int(w.seq_lens[s])
+            for h in range(w.num_kv_heads):
+                got_k = O.gather_rows(pool, w.layer, w.block_tables[s], h, 0, L)
+                got_v = O.gather_rows(pool, w.layer, w.block_tables[s], h, 1, L)
+                assert np.array_equal(got_k, k64[:, h, :]) and np.array_equal(got_v, v64[:, h, :]), (w.name, s, h)
+            used[w.block_tables[s][: (L + w.block_size - 1) // w.block_size]] = True
+        sent = O.sentinel_bits(w.kv_dtype)
+        untouched = pool.bits[~used]
+        if w.kv_dtype == "f32":
+            assert np.isnan(untouched).all()
+        else:
+            assert (untouched == sent).all()
+
+
+# ---------------------------------------------------------------------------
+# Attention
+# ---------------------------------------------------------------------------
+
+def pin_dense_equivalence():
+    for w in small_workloads():
+        out, _ = run_oracle(w)
+        ref = dense_sdpa(w)
+        err = np.abs(out - ref).max()
+        assert err <= 1e-12, (w.name, err)
+
+
+def pin_noncausal_dense():
+    w = W.mixed_bf16(n_decode=2, n_prefill=2, chunk=24, dec_lo=20, dec_hi=70, cached_lo_blocks=1,
+                     cached_hi_blocks=2, block_size=16)
+    w.causal = False
+    out, _ = run_oracle(w)
+    assert np.abs(out - dense_sdpa(w)).max() <= 1e-12
+
+
+def pin_brute_force():
+    """Pure-Python loops on a tiny mixed batch (one prefill chunk, one decode)."""
+    w = W.build("brute", seed=5, kv_dtype="f32", num_q_heads=4, num_kv_heads=2, head_dim=3, block_size=2,
+                seq_lens=[5, 4], q_lens=[3, 1], num_blocks=9)
+    out, lse = run_oracle(w)
+    qq = q64(w)
+    cu = w.cu_q_lens
+    for s in range(2):
+        k, v = w.kv_values(s)
+        L, ql = int(w.seq_lens[s]), int(w.q_lens[s])
+        for j in range(ql):
+            p = L - ql + j
+            for h in range(4):
+                kvh = h // 2
+                z = [w.softmax_scale * sum(float(qq[cu[s] + j, h, d]) * float(k[t, kvh, d]) for d in range(3))
+                     for t in range(p + 1)]
+                m = max(z)
+                e = [math.exp(x - m) for x in z]
+                den = sum(e)
+                for d in range(3):
+                    ref = sum(e[t] * float(v[t, kvh, d]) for t in range(p + 1)) / den
+                    assert abs(out[cu[s] + j, h, d] - ref) <= 1e-13, (s, j, h, d)
+                assert abs(lse[cu[s] + j, h] - (m + math.log(den))) <= 1e-13
+
+
+def pin_lse_logsumexp():
+    from scipy.special import logsumexp
+
+    w = W.llama3_8b_decode_bf16(batch=2, lo=30, hi=90)
+    pool = oracle_pool_for(w)
+    _, lse = run_oracle(w, pool)
+    qq = q64(w)
+    for s in range(2):
+        for h in (0, 5, 31):
+            k, _ = _values64(w, s)
+            z = w.softmax_scale * (k[:, h // 4, :] @ qq[s, h])
+            assert abs(lse[s, h] - logsumexp(z)) <= 1e-12
+
+
+def pin_permutation_invariance():
+    base = W.llama3_8b_decode_bf16(batch=3, lo=40, hi=300)
+    w2 = W.llama3_8b_decode_bf16(batch=3, lo=40, hi=300)
+    # Same values, another physical placement: reshuffle the block ids.
+    perm = np.random.default_rng(99).permutation(base.num_blocks).astype(np.int32)
+    w2.block_tables = np.where(base.block_tables >= 0, perm[np.maximum(base.block_tables, 0)], -1)
+    o1, l1 = run_oracle(base)
+    o2, l2 = run_oracle(w2)
+    assert not np.array_equal(base.block_tables, w2.block_tables)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def pin_softmax_rows():
+    w = W.mixed_bf16(n_decode=2, n_prefill=1, chunk=20, dec_lo=20, dec_hi=90, cached_lo_blocks=1,
+                     cached_hi_blocks=2, block_size=16)
+    pool = oracle_pool_for(w)
+    qq = q64(w)
+    for s in range(w.num_seqs):
+        for j in range(int(w.q_lens[s])):
+            for h in (0, 9, 31):
+                p = O.attention_row_probs(pool, 0, qq, w.cu_q_lens, w.seq_lens, w.block_tables, w.num_q_heads,
+                                          w.softmax_scale, True, s, j, h)
+                assert abs(p.sum() - 1.0) <= 1e-12 and (p >= 0).all()
+                lim = int(w.seq_lens[s]) - int(w.q_lens[s]) + j + 1
+                assert (p[lim:] == 0).all() and (p[:lim] > 0).all()
+
+
+def _one_seq(kvals, vvals, qvals, B=4, causal=True, q_len=1):
+    """Oracle on hand-made values: one sequence, Hq=2, Hkv=1, f32."""
+    L, D = kvals.shape
+    nb = (L + B - 1) // B
+    pool = O.new_pool(nb + 3, 1, 1, B, D, "f32")
+    table = (np.arange(nb)[::-1] + 2).astype(np.int32)[None, :]  # reversed, offset placement
+    O.kv_append(pool, 0, kvals[:, None, :].astype(np.float32), vvals[:, None, :].astype(np.float32), "f32",
+                np.array([0, L]), np.array([0]), table)
+    return O.paged_attention(pool, 0, qvals.astype(np.float64), np.array([0, q_len]), np.array([L]), table, 2,
+                             0.125, causal)
+
+
+def pin_closed_forms():
+    r = np.random.default_rng(3)
+    D = 8
+    # seq_len = 1 -> v0 exactly
+    k = r.standard_normal((1, D)).astype(np.float32)
+    v = r.standard_normal((1, D)).astype(np.float32)
+    o, lse = _one_seq(k, v, r.standard_normal((1, 2, D)))
+    assert np.array_equal(o[0, 0], v[0].astype(np.float64)) and np.array_equal(o[0, 1], v[0].astype(np.float64))
+    # q = 0 -> exact mean of V; lse = ln L
+    L = 13
+    k = r.standard_normal((L, D)).astype(np.float32)
+    v = r.standard_normal((L, D)).astype(np.float32)
+    o, lse = _one_seq(k, v, np.zeros((1, 2, D)))
+    assert np.abs(o[0, 0] - v.astype(np.float64).mean(0)).max() <= 1e-15
+    assert abs(lse[0, 0] - math.log(L)) <= 1e-15
+    # all keys equal -> mean of V
+    k = np.tile(r.standard_normal((1, D)).astype(np.float32), (L, 1))
+    o, _ = _one_seq(k, v, r.standard_normal((1, 2, D)))
+    assert np.abs(o[0, 1] - v.astype(np.float64).mean(0)).max() <= 1e-15
+    # two tokens -> (v0 e^z0 + v1 e^z1) / (e^z0 + e^z1)
+    k = r.standard_normal((2, D)).astype(np.float32)
+    v = r.standard_normal((2, D)).astype(np.float32)
+    q = r.standard_normal((1, 2, D))
+    o, _ = _one_seq(k, v, q)
+    z = 0.125 * (k.astype(np.float64) @ q[0, 0])
+    v64 = v.astype(np.float64)
+    ref = (v64[0] * math.exp(z[0]) + v64[1] * math.exp(z[1])) / (math.exp(z[0]) + math.exp(z[1]))
+    assert np.abs(o[0, 0] - ref).max() <= 1e-14
+    # one dominant logit -> v_t
+    L = 9
+    k = r.standard_normal((L, D)).astype(np.float32)
+    v = r.standard_normal((L, D)).astype(np.float32)
+    q = np.zeros((1, 2, D))
+    q[0, :] = 50.0 * 8 * k[4]
+    o, _ = _one_seq(k, v, q)
+    assert np.abs(o[0, 0] - v[4]).max() <= 1e-12
+    # first row of a chunk with nothing cached sees only its own key -> v0
+    L = 6
+    k = r.standard_normal((L, D)).astype(np.float32)
+    v = r.standard_normal((L, D)).astype(np.float32)
+    o, _ = _one_seq(k, v, r.standard_normal((L, 2, D)), q_len=L)
+    assert np.array_equal(o[0, 0], v[0].astype(np.float64))
+    # the last row of that chunk sees every key: it equals the non-causal answer,
+    # while the non-causal first row differs from v0
+    q = r.standard_normal((L, 2, D))
+    oc, _ = _one_seq(k, v, q, q_len=L)
+    on, _ = _one_seq(k, v, q, q_len=L, causal=False)
+    assert np.array_equal(oc[L - 1], on[L - 1]) and not np.allclose(on[0, 0], v[0])
+
+
+def pin_split_reduce():
+    """Partials over arbitrary (some empty) key ranges merge back to the unsplit result."""
+    w = W.llama3_8b_decode_bf16(batch=2, lo=100, hi=300)
+    pool = oracle_pool_for(w)
+    out, lse = run_oracle(w, pool)
+    qq = q64(w)
+    r = np.random.default_rng(11)
+    for s in range(2):
+        L = int(w.seq_lens[s])
+        cuts = np.sort(np.concatenate([[0, L, L, 0], r.integers(0, L, 5)]))
+        for h in (0, 7, 30):
+            k, v = _values64(w, s)
+            K, V = k[:, h // 4], v[:, h // 4]
+            po, pl = [], []
+            for a, b in zip(cuts[:-1], cuts[1:]):
+                if b <= a:
+                    po.append(np.full((1, w.head_dim), 7.0))  # content of an empty part is ignored
+                    pl.append(np.array([-np.inf]))
+                    continue
+                z = w.softmax_scale * (K[a:b] @ qq[s, h])
+                m = z.max()
+                e = np.exp(z - m)
+                po.append(((e @ V[a:b]) / e.sum())[None, :])
+                pl.append(np.array([m + math.log(e.sum())]))
+            o, l = O.split_kv_reduce(np.stack(po), np.stack(pl))
+            assert np.abs(o[0] - out[s, h]).max() <= 1e-13 and abs(l[0] - lse[s, h]) <= 1e-13
+    o, l = O.split_kv_reduce(np.zeros((2, 1, 4)), np.full((2, 1), -np.inf))
+    assert (o == 0).all() and l[0] == -np.inf
+
+
+def pin_prefix_sharing():
+    """Shared prefix blocks give the same result as private copies of them."""
+    w = W.prefix_reuse_bf16(n_req=4, prefix=256, suf_lo=5, suf_hi=60)
+    shared, _ = run_oracle(w)
+    B = w.block_size
+    P = w.shared_prefix_tokens // B
+    assert (w.block_tables[:, :P] == w.block_tables[0, :P]).all()
+    w2 = W.prefix_reuse_bf16(n_req=4, prefix=256, suf_lo=5, suf_hi=60)
+    extra = w2.num_blocks
+    w2.num_blocks = extra + P * w2.num_seqs
+    for s in range(w2.num_seqs):
+        w2.block_tables[s, :P] = extra + s * P + np.arange(P)
+    private, _ = run_oracle(w2)
+    assert np.array_equal(shared, private)
+
+
+ALL_PINS = [
+    pin_e4m3_decode_table, pin_e4m3_encode, pin_bf16_decode, pin_block_mapping_example, pin_append_roundtrip,
+    pin_dense_equivalence, pin_noncausal_dense, pin_brute_force, pin_lse_logsumexp, pin_permutation_invariance,
+    pin_softmax_rows, pin_closed_forms, pin_split_reduce, pin_prefix_sharing,
+]

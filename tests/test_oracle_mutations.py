@@ -1,0 +1,114 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+A pin suite that still passes with a mistake planted would not be pinning
+that part of the oracle.  Every mutation below must make at least one pin in
+``oracle_pins.ALL_PINS`` fail.
+"""
+import numpy as np
+import pytest
+
+import oracle.pkv_oracle as O
+import oracle_pins as P
+
+_orig_block_address = O.block_address
+_orig_softmax_rows = O._softmax_rows
+_orig_gather = O.gather_rows
+_orig_decode = O.decode_bits
+_orig_split = O.split_kv_reduce
+
+
+def _gqa_modulo(h, hq, hkv):
+    return h % hkv
+
+
+def _slot_reversed(row, pos, B):
+    phys, slot = _orig_block_address(row, pos, B)
+    return phys, B - 1 - slot
+
+
+def _block_shifted(row, pos, B):
+    pos = np.asarray(pos)
+    return row[np.minimum(pos // B + (pos % B == B - 1), len(row) - 1)], pos % B
+
+
+def _causal_excludes_self(L, ql, j, causal):
+    j = np.asarray(j)
+    return np.full(j.shape, L) if not causal else L - ql + j
+
+
+def _causal_ignored(L, ql, j, causal):
+    return np.full(np.asarray(j).shape, L)
+
+
+def _truncating_round(x):
+    return np.floor(x)
+
+
+def _half_up_round(x):
+    return np.floor(x + 0.5)
+
+
+def _scale_twice(z):
+    return _orig_softmax_rows(2.0 * z)
+
+
+def _lse_without_max(z):
+    w, m, l = _orig_softmax_rows(z)
+    return w, 0.0 * m, l
+
+
+def _kv_swapped(pool, layer, row, kvh, which, n):
+    return _orig_gather(pool, layer, row, kvh, 1 - which, n)
+
+
+def _e4m3_bias8(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    v = _orig_decode(codes, "e4m3")
+    return np.where((c & 0x78) != 0, v / 2.0, v)
+
+
+def _decode_e4m3_bias8(bits, dtype):
+    return _e4m3_bias8(bits) if dtype == "e4m3" else _orig_decode(bits, dtype)
+
+
+def _bf16_wrong_shift(bits, dtype):
+    if dtype == "bf16":
+        u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(15)
+        return u.view(np.float32).astype(np.float64)
+    return _orig_decode(bits, dtype)
+
+
+def _split_sign(po, pl):
+    return _orig_split(po, -np.asarray(pl))
+
+
+MUTATIONS = {
+    "gqa_modulo_mapping": [("kv_head_of", _gqa_modulo)],
+    "slot_reversed": [("block_address", _slot_reversed)],
+    "block_index_off_by_one": [("block_address", _block_shifted)],
+    "causal_excludes_own_token": [("key_limit", _causal_excludes_self)],
+    "causal_mask_ignored": [("key_limit", _causal_ignored)],
+    "e4m3_truncates": [("rne", _truncating_round)],
+    "e4m3_ties_away": [("rne", _half_up_round)],
+    "softmax_scale_doubled": [("_softmax_rows", _scale_twice)],
+    "lse_drops_max": [("_softmax_rows", _lse_without_max)],
+    "k_v_swapped": [("gather_rows", _kv_swapped)],
+    "e4m3_bias_8": [("e4m3_decode", _e4m3_bias8), ("decode_bits", _decode_e4m3_bias8)],
+    "bf16_decode_shift": [("decode_bits", _bf16_wrong_shift)],
+    "split_merge_sign": [("split_kv_reduce", _split_sign)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    for attr, fn in MUTATIONS[name]:
+        monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin()
+        except Exception as e:  # noqa: BLE001 - any failure of a pin counts
+            caught.append((pin.__name__, type(e).__name__))
+            break
+    assert caught, f"no pin catches the planted mistake {name}"
