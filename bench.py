@@ -1,0 +1,400 @@
+"""Benchmark: one step of paged KV-cache attention on a synthetic in-flight batch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl pkv|reference]
+
+A step is the whole hot path for one layer of one iteration: kv_append of the
+step's new tokens, host planning of the launch, and paged_attention (persistent
+attention kernel plus the merge of split key ranges).  The default workload is
+the Llama-3-8B-shaped decode batch (64 sequences, lengths U[512, 4096], 32/8
+heads, head_dim 128, block 64, bf16 KV).  The pool (~755 MB) is larger than L2
+and L2 is also flushed (a 512 MB write) before every timed step.
+
+Prints ONE JSON line (rank 0).  Under torchrun every rank runs an independent
+replica on its own GPU (the path has no exchange step); time is the max over
+ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode-attention KV GB/s & % of B200 HBM peak; decode tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def elem_bytes(dtype: str) -> int:
+    return {"f32": 4, "bf16": 2, "f16": 2, "e4m3": 1}[dtype]
+
+
+def algorithmic_bytes(w, plan_info=None) -> dict:
+    """Bytes one step must move: distinct K/V bytes read, q, out, tables, scales, partials, appended rows."""
+    eb = elem_bytes(w.kv_dtype)
+    row = w.num_kv_heads * w.head_dim * eb  # one token of one layer, K or V
+    kv = sum(tokens for _, tokens in w.distinct_kv_blocks()) * row * 2
+    qb = elem_bytes(w.q_dtype)
+    q = w.total_q * w.num_q_heads * w.head_dim * qb
+    out = q
+    tables = sum((int(L) + w.block_size - 1) // w.block_size for L in w.seq_lens) * 4 + w.num_seqs * 8
+    scales = 2 * w.num_kv_heads * 4 if w.kv_dtype == "e4m3" else 0
+    parts = 0
+    if plan_info:
+        parts = plan_info["num_partial_rows"] * (w.head_dim + 1) * 4 * 2
+    new_rows = w.total_q * w.num_kv_heads * w.head_dim * 2
+    append = new_rows * elem_bytes(w.kv_in_dtype) + new_rows * eb
+    attn = kv + q + out + tables + scales + parts
+    return {"kv": kv, "attention": attn, "append": append, "step": attn + append}
+
+
+def decode_rows(w) -> int:
+    return int((w.q_lens == 1).sum())
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("attn_mma.cu", "common.cuh", "plan_format.h"):
+        with open(os.path.join(ROOT, "paged_kv_attention_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(config: str):
+    """ncu DRAM bytes per attention launch, if captured on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(config)
+    if not e or e.get("kernel_source") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline figure)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, budget_s: float = 10.0, max_seqs: int | None = None):
+    """Time the oracle on whole-batch steps (or a prefix of sequences) for about budget_s seconds."""
+    import oracle.pkv_oracle as O
+
+    seqs = list(range(w.num_seqs if max_seqs is None else min(max_seqs, w.num_seqs)))
+    pool = O.new_pool(w.num_blocks, w.num_layers, w.num_kv_heads, w.block_size, w.head_dim, w.kv_dtype,
+                      w.k_scale, w.v_scale)
+    k, v, cu, sp = w.packed_kv("history", seqs)
+    O.kv_append(pool, w.layer, k, v, w.kv_in_dtype, cu, sp, w.block_tables[seqs])
+    q = O.decode_bits(w.q, w.q_dtype) if w.q_dtype != "f32" else w.q.astype(np.float64)
+    kn, vn, cun, spn = w.packed_kv("new", seqs)
+    steps, t_wall, t_cpu = 0, 0.0, 0.0
+    while t_wall < budget_s or steps == 0:
+        c0, w0 = time.process_time(), time.perf_counter()
+        O.kv_append(pool, w.layer, kn, vn, w.kv_in_dtype, cun, spn, w.block_tables[seqs])
+        O.paged_attention(pool, w.layer, q, w.cu_q_lens, w.seq_lens, w.block_tables, w.num_q_heads,
+                          w.softmax_scale, w.causal, seqs=seqs)
+        t_wall += time.perf_counter() - w0
+        t_cpu += time.process_time() - c0
+        steps += 1
+    # Bytes of the sampled sequences only.
+    sub = type(w)(**{**w.__dict__})
+    sub.seq_lens, sub.q_lens = w.seq_lens[seqs], w.q_lens[seqs]
+    sub.block_tables = w.block_tables[seqs]
+    b = algorithmic_bytes(sub)
+    per_step = t_wall / steps
+    return {
+        "value": b["step"] / per_step / 1e9,
+        "unit": "GB/s",
+        "cores": max(1, round(t_cpu / t_wall)),
+        "kind": "oracle",
+        "sample": f"{len(seqs)} of {w.num_seqs} sequences of {w.name}, {steps} whole steps "
+                  f"(kv_append + attention, float64 numpy), {t_wall:.1f} s",
+        "ms_per_step": per_step * 1e3,
+        "decode_tok_s": decode_rows(sub) / per_step,
+    }
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    from paged_kv_attention_block_b200 import workloads as W
+
+    w = W.NAMED[args.config]()
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w, budget_s=args.ref_budget, max_seqs=args.ref_seqs)
+        if i >= args.warmup:
+            per_step.append(r["ms_per_step"])
+            base = r
+    ms = float(np.mean(per_step))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
+        "config": {"workload": w.name, "sample": base["sample"]},
+        "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "decode_tok_s": base["decode_tok_s"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# The CUDA path
+# ---------------------------------------------------------------------------
+
+def run_pkv(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_attention_block_b200 import build
+
+    build.build()
+    from paged_kv_attention_block_b200 import api, runner, workloads as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    builder = W.NAMED[args.config]
+    w = builder(seed=builder.__defaults__[0] + 1000 * rank) if rank else builder()
+    dw = runner.DeviceWorkload(w, device=dev)
+    plan_opts = {}
+    if args.kv_split:
+        plan_opts["kv_split"] = args.kv_split
+    plan = dw.plan(**plan_opts)
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(dw.q)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dw.append_new()
+        p = dw.plan(**plan_opts)
+        ev_a = torch.cuda.Event(enable_timing=True)
+        ev_a.record(stream)
+        dw.attention(p, out=out, workspace=ws)
+        return p, ev_a
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    attn_ev = []
+    host_plan_s = 0.0
+    with ClockSampler(local_rank) as clocks:
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(1)
+            ev[i][0].record(stream)
+            dw.append_new()
+            t0 = time.perf_counter()
+            p = dw.plan(**plan_opts)
+            host_plan_s += time.perf_counter() - t0
+            a0 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            dw.attention(p, out=out, workspace=ws)
+            ev[i][1].record(stream)
+            attn_ev.append(a0)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in ev]
+    attn_ms = [a.elapsed_time(e[1]) for a, e in zip(attn_ev, ev)]
+    ms = float(np.mean(step_ms))
+    attn = float(np.mean(attn_ms))
+    if world > 1:
+        t = torch.tensor([ms, attn], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, attn = float(t[0]), float(t[1])
+    assert int(dw.status.item()) == 0, "device status set during the benchmark"
+
+    b = algorithmic_bytes(w, plan.info)
+    value = b["step"] * world / (ms * 1e-3) / 1e9
+    achieved = b["attention"] / (attn * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+
+    # End to end through the public API from pinned host buffers.
+    e2e = run_e2e(args, w, dw, plan_opts, dev, stream, api)
+    if world > 1:
+        t = torch.tensor([e2e["ms"]], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms"] = float(t[0])
+
+    launches_per_step = 2 + (1 if plan.info["num_reduce"] > 0 else 0)
+    if rank == 0:
+        cpu = oracle_sample(w, budget_s=args.ref_budget, max_seqs=args.ref_seqs) if world == 1 and not args.no_cpu else None
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.num_seqs, "kv_tokens": int(w.seq_lens.sum()),
+                       "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                       "block_size": w.block_size, "l2": "flushed before every step (512 MB write); pool > L2",
+                       "parallelism": f"replicas{world}"},
+            "decode_tok_s": decode_rows(w) * world / (ms * 1e-3),
+            "hbm_frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
+            "hbm_frac_of_measured": value / world / peak,
+            "step_bytes": b["step"], "kv_bytes": b["kv"],
+            "attention_ms": attn, "host_plan_us": host_plan_s / args.steps * 1e6,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic_for(w.name), "peak_source": peak_kind,
+                         "kernel": "attn_mma_kernel (+ plan upload and split merge in the timed call)"},
+            "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": b["step"] * world / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms"]},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(),
+            "plan": {k: plan.info[k] for k in ("num_items", "num_reduce", "num_partial_rows", "num_groups", "num_ctas")},
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, dw, plan_opts, dev, stream, api):
+    import torch
+
+    names = {"q": dw.q, "k_new": dw.k_new, "v_new": dw.v_new, "cu_q": dw.cu_q, "seq_lens": dw.seq_lens,
+             "start_pos": dw.start_pos, "block_tables": dw.block_tables}
+    host = {k: v.detach().cpu().pin_memory() for k, v in names.items()}
+    host["out"] = torch.empty(dw.q.shape, dtype=dw.q.dtype).pin_memory()
+    devb = {k: torch.empty_like(v) for k, v in names.items()}
+    devb["out"] = torch.empty_like(dw.q)
+    plan = dw.plan(**plan_opts)
+    devb["workspace"] = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
+    cu, sl, bt = w.cu_q_lens, w.seq_lens, w.block_tables
+
+    def plan_fn():
+        return api.plan_attention(cu, sl, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                                  block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal, block_tables=bt,
+                                  **plan_opts)
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        api.decode_step_e2e(dw.cache, host, devb, plan_fn, w.softmax_scale, w.causal)
+    torch.cuda.synchronize(dev)
+    n = max(1, min(args.steps, 200))
+    tot = 0.0
+    for _ in range(n):
+        flush.fill_(1)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        p = api.decode_step_e2e(dw.cache, host, devb, plan_fn, w.softmax_scale, w.causal)
+        e.record(stream)
+        e.synchronize()
+        tot += s.elapsed_time(e)
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if k != "out") + p.info["plan_bytes"]
+    d2h = host["out"].numel() * host["out"].element_size()
+    return {"ms": tot / n, "h2d": int(h2d), "d2h": int(d2h)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
+    ap.add_argument("--config", default="llama3_8b_decode_bf16")
+    ap.add_argument("--kv-split", type=int, default=0)
+    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference sample")
+    ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample (default all)")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline oracle timing")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_pkv(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

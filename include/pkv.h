@@ -1,0 +1,252 @@
+/*
+ * pkv.h - C ABI of libpkv.so: attention over a paged KV cache on B200 (sm_100a).
+ *
+ * The operations follow the pages on NVIDIA TensorRT-LLM this library is built
+ * from:
+ *   - the KV cache is a pool of fixed-size token blocks, a request reaches its
+ *     blocks through a per-request block table, and the block size is a power
+ *     of two greater than one ("NVIDIA TensorRT-LLM详解", gentlecold.top, §9
+ *     "KV cache系统");
+ *   - new tokens' K/V are written into their pages through a page-table lookup
+ *     (TensorRT-LLM concept explainer, compassingai.com, "技术原理"; deep dive
+ *     §2, decode writes the new token's KV);
+ *   - one batch packs context (prefill) requests before generation (decode)
+ *     requests, without padding, and a long prompt is processed in chunks that
+ *     attend to everything cached so far plus themselves (deep dive §6
+ *     "In-flight batching", §8 "Chunked prefill");
+ *   - the cache may be stored as fp8 (deep dive §13, KvCacheConfig(dtype="fp8")).
+ * The attention itself is softmax(scale * q K^T) V with grouped-query heads:
+ * query head h reads KV head h / (Hq / Hkv).
+ *
+ * Conventions shared by every call:
+ *   - Memory: every pointer named "device" is CUDA device memory owned by the
+ *     caller; "host" pointers are host memory owned by the caller.  The library
+ *     never allocates or frees memory and never synchronises the stream.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued in call order on that stream.
+ *   - Synchronous errors: an invalid argument returns a nonzero pkv_status at
+ *     once and enqueues nothing.  PKV_ERR_CUDA reports a failed launch or copy;
+ *     pkv_last_error() gives a message for the calling thread.
+ *   - Asynchronous errors: a block id outside [0, num_blocks), a logical block
+ *     beyond the table row, or a plan that does not match the lengths on the
+ *     device is recorded by OR-ing a PKV_DEV_* bit into *dev_status (device
+ *     int32, zeroed by the caller, may be NULL); the offending rows or keys are
+ *     skipped.  No kernel traps.
+ *   - Pool layout (row-major):
+ *       pool[num_blocks][num_layers][2][num_kv_heads][block_size][head_dim]
+ *     index 0 of the "2" axis is K, 1 is V; each (block, layer, K|V, head) is
+ *     one contiguous run of block_size * head_dim elements.
+ *   - Token p of sequence s lives in physical block block_tables[s][p / B] at
+ *     slot p % B.  Block tables are int32 [num_seqs][max_blocks] (row stride
+ *     max_blocks); unused entries are ignored.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PKV_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+typedef enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1, /* null pointer, bad shape or dtype, lengths out of range */
+  PKV_ERR_UNSUPPORTED = 2, /* valid but not built: e.g. head_dim outside {64, 128} */
+  PKV_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  PKV_ERR_WORKSPACE = 4,   /* caller buffer smaller than required */
+  PKV_ERR_PLAN = 5         /* plan buffer corrupt or made for other shapes */
+} pkv_status;
+
+typedef enum pkv_dtype {
+  PKV_F32 = 0,
+  PKV_BF16 = 1,
+  PKV_F16 = 2,
+  PKV_FP8_E4M3 = 3 /* OCP E4M3: bias 7, no infinities, max finite 448 */
+} pkv_dtype;
+
+/* Bits OR-ed into *dev_status by kernels. */
+#define PKV_DEV_BAD_BLOCK_ID 0x1      /* block table entry outside [0, num_blocks) */
+#define PKV_DEV_BAD_LOGICAL_BLOCK 0x2 /* position needs a table entry beyond max_blocks */
+#define PKV_DEV_PLAN_MISMATCH 0x4     /* plan item does not fit the device lengths */
+#define PKV_DEV_BAD_APPEND 0x8        /* kv_append position negative */
+
+/* One layer's view of a paged pool (deep dive §9: one block holds a fixed number
+ * of tokens' KV; several layers may be packed in one block). */
+typedef struct pkv_cache {
+  void* pool;             /* device, layout above, element type kv_dtype */
+  int64_t num_blocks;     /* physical blocks in the pool */
+  int32_t num_layers;     /* layers packed per block */
+  int32_t layer;          /* layer this call reads or writes, 0 <= layer < num_layers */
+  int32_t num_kv_heads;   /* Hkv */
+  int32_t head_dim;       /* d: 64 or 128 */
+  int32_t block_size;     /* B: power of two, >= 2 */
+  int32_t kv_dtype;       /* pkv_dtype: F32, BF16, F16 or FP8_E4M3 */
+  const float* k_scale;   /* device float32 [num_layers][Hkv]; FP8_E4M3 only, else NULL */
+  const float* v_scale;   /* device float32 [num_layers][Hkv]; FP8_E4M3 only, else NULL */
+} pkv_cache;
+
+/* Library ABI version (PKV_ABI_VERSION of the build). */
+PKV_API int32_t pkv_abi_version(void);
+
+/* Static description of a status code. */
+PKV_API const char* pkv_status_string(int32_t status);
+
+/* Detail of the last error raised on the calling thread ("" if none). */
+PKV_API const char* pkv_last_error(void);
+
+/*
+ * kv_append - write new tokens' K and V into their pool slots.
+ *
+ * Source: deep dive §2 (decode writes each new token's KV), §8 (a prefill chunk
+ * appends its KV before the next chunk), concept explainer "技术原理" (page-table
+ * lookup on KV writes).
+ *
+ * k_new, v_new: device [total_new][Hkv][head_dim] of in_dtype, packed by
+ *   sequence: sequence s owns rows cu_new[s] .. cu_new[s+1]-1.
+ * cu_new: device int32 [num_seqs+1], cu_new[0] = 0, nondecreasing,
+ *   cu_new[num_seqs] = total_new (total_new also passed by value for the grid).
+ * start_pos: device int32 [num_seqs]: position of sequence s's first new token;
+ *   row cu_new[s]+i goes to position start_pos[s]+i.
+ * block_tables: device int32 [num_seqs][max_blocks].
+ * in_dtype: must equal cache->kv_dtype for F32/BF16/F16 pools.  For an
+ *   FP8_E4M3 pool it is F32, BF16 or F16 and each value x is stored as the
+ *   E4M3 code of the float32 quotient x / scale (IEEE division), rounded to
+ *   nearest even, finite overflow saturated to +-448, with scale =
+ *   k_scale[layer][h] for K and v_scale[layer][h] for V.
+ * Errors: INVALID_ARG for bad shapes/dtypes/null pointers.  Asynchronously,
+ *   rows whose block id is out of range are not written (PKV_DEV_BAD_BLOCK_ID,
+ *   PKV_DEV_BAD_LOGICAL_BLOCK, PKV_DEV_BAD_APPEND).
+ * Stream-ordered; reads no memory after the kernel completes.
+ */
+PKV_API pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, const void* v_new, int32_t in_dtype,
+                         const int32_t* cu_new, const int32_t* start_pos, const int32_t* block_tables,
+                         int32_t max_blocks, int32_t num_seqs, int32_t total_new, int32_t* dev_status,
+                         void* stream);
+
+/*
+ * Planning request for one paged_attention call (a batch of sequences).
+ *
+ * Sequence s processes q_len = cu_q_lens[s+1] - cu_q_lens[s] query tokens this
+ * step (1 for decode, the chunk length for a prefill chunk, 0 = not scheduled)
+ * and attends over seq_lens[s] keys, counting this step's tokens, which must
+ * already be appended.  Query row j of s sits at position seq_lens[s] - q_len
+ * + j; with causal != 0 it attends to keys 0..position (deep dive §8: a chunk
+ * sees the cached KV plus itself), otherwise to all seq_lens[s] keys.
+ */
+typedef struct pkv_plan_request {
+  int32_t num_seqs;
+  int32_t num_q_heads;          /* Hq, a multiple of num_kv_heads */
+  int32_t num_kv_heads;         /* Hkv */
+  int32_t head_dim;             /* 64 or 128 */
+  int32_t block_size;           /* power of two >= 2 */
+  int32_t kv_dtype;             /* pkv_dtype of the pool */
+  int32_t causal;               /* 0 or 1 */
+  int32_t num_ctas;             /* CTAs the launch keeps resident; 0 = ask the current device */
+  int32_t kv_split;             /* 0 = automatic split of long key ranges; >0 = max keys per work
+                                   item (rounded up to 64); <0 = never split */
+  int32_t cascade;              /* nonzero: group consecutive sequences whose tables share leading
+                                   blocks and read those blocks once per group (needs block_tables) */
+  int32_t min_shared_tokens;    /* shortest shared prefix that forms a group (0 = 256) */
+  int32_t max_blocks;           /* row stride of block_tables */
+  const int32_t* cu_q_lens;     /* host int32 [num_seqs+1] */
+  const int32_t* seq_lens;      /* host int32 [num_seqs] */
+  const int32_t* block_tables;  /* host int32 [num_seqs][max_blocks]; NULL disables cascade */
+} pkv_plan_request;
+
+typedef struct pkv_plan_info {
+  size_t plan_bytes;            /* bytes of the plan buffer */
+  size_t workspace_bytes;       /* device workspace paged_attention needs with this plan */
+  int32_t num_items;            /* work items (one CTA-sized tile of rows x key range each) */
+  int32_t num_reduce;           /* output row groups merged from partial states */
+  int32_t num_parts;            /* partial states referenced by the merges */
+  int32_t num_partial_rows;     /* float32 partial rows of head_dim (+1 lse) in the workspace */
+  int32_t num_groups;           /* shared-prefix groups found */
+  int32_t num_ctas;             /* CTAs planned for */
+} pkv_plan_info;
+
+/*
+ * attention_plan - host-only: split the batch into work items for one launch.
+ *
+ * Cuts every (sequence, KV head, query tile) into key ranges so that the work
+ * spreads evenly over num_ctas CTAs, and, with cascade, finds sequences whose
+ * tables share leading physical blocks (deep dive §10: prefix blocks reused
+ * across requests through the radix tree) so that those keys are read once per
+ * group.  The plan depends only on the lengths, the tables' sharing pattern and
+ * the shapes: a runtime plans once per step and reuses the plan for every layer.
+ *
+ * plan: host buffer of `capacity` bytes, or NULL to query sizes only.
+ * info: filled in all cases (required).
+ * Returns WORKSPACE if capacity < info->plan_bytes, INVALID_ARG on bad lengths
+ * (q_len > seq_len, negative values, a table row too short for seq_len, Hq not a
+ * multiple of Hkv, more than 64 query heads per KV head).  Touches no GPU
+ * unless num_ctas == 0.
+ */
+PKV_API pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan, size_t capacity, pkv_plan_info* info);
+
+/* CTAs per launch the attention kernel keeps resident on the current device
+ * for this pool dtype and head_dim (SM count x occupancy). */
+PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int32_t* num_ctas);
+
+/*
+ * paged_attention - out = softmax(scale * q K^T) V over each sequence's paged K/V.
+ *
+ * Source: deep dive §2 (decode reads all history KV to do attention), §6 (one
+ * launch serves a packed mix of prefill and decode requests), §8 (chunked
+ * prefill with causal masking).  One call enqueues one persistent attention
+ * kernel and, when the plan split a key range, one merge kernel (the same
+ * merge pkv_split_kv_reduce performs).
+ *
+ * q: device [total_q][num_q_heads][head_dim], q_dtype F32 (F32 pools only),
+ *   BF16 (BF16 or FP8 pools) or F16 (F16 or FP8 pools).  total_q = cu_q_lens[num_seqs].
+ * cu_q_lens, seq_lens: device int32 copies of the arrays the plan was made from.
+ * block_tables: device int32 [num_seqs][max_blocks].
+ * softmax_scale: scale on q.k (typically 1/sqrt(head_dim)); causal as planned.
+ * plan: host buffer from pkv_attention_plan for these shapes.  It is copied to
+ *   the workspace with cudaMemcpyAsync; use page-locked memory for an
+ *   asynchronous copy and keep it unchanged until the copy has run.
+ * out: device [total_q][num_q_heads][head_dim] in q_dtype.
+ * out_lse: device float32 [total_q][num_q_heads] natural-log sum of exp(scores)
+ *   per row, or NULL.
+ * workspace: device, >= info.workspace_bytes, 256-byte aligned.
+ * Errors: INVALID_ARG/UNSUPPORTED/PLAN/WORKSPACE synchronously; PKV_DEV_* bits
+ *   asynchronously (skipped rows are left unwritten).
+ */
+PKV_API pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                               const int32_t* cu_q_lens, const int32_t* seq_lens, const int32_t* block_tables,
+                               int32_t max_blocks, int32_t num_seqs, float softmax_scale, int32_t causal,
+                               const void* plan, void* out, float* out_lse, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * split_kv_reduce - merge partial softmax states computed over disjoint key sets.
+ *
+ * The pages do not describe split-KV; this is the exact identity that splitting
+ * a softmax over key ranges obeys.  For each row r:
+ *   M = max_i lse[i][r];  w_i = exp(lse[i][r] - M);
+ *   out[r] = sum_i w_i o[i][r] / sum_i w_i;  out_lse[r] = M + ln(sum_i w_i).
+ * A part with lse = -inf (no keys) has weight 0; a row whose parts are all
+ * empty gets out = 0 and out_lse = -inf.
+ *
+ * partial_o: device float32 [n_split][rows][head_dim], each part normalised.
+ * partial_lse: device float32 [n_split][rows], natural log.
+ * out: device [rows][head_dim] in out_dtype (F32, BF16 or F16).
+ * out_lse: device float32 [rows] or NULL.
+ */
+PKV_API pkv_status pkv_split_kv_reduce(const float* partial_o, const float* partial_lse, int32_t n_split, int64_t rows,
+                               int32_t head_dim, void* out, int32_t out_dtype, float* out_lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,259 @@
+"""ctypes binding of libpkv.so (declared in include/pkv.h).
+
+Every function here only converts torch tensors and Python values into the
+pointers and sizes of the C ABI, calls it, and raises ``PkvError`` on a
+nonzero status.  All computation happens in the library's CUDA kernels; if the
+library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.environ.get("PKV_LIBRARY", os.path.join(_HERE, "libpkv.so"))
+
+
+if not os.path.exists(library_path()):
+    raise ImportError(
+        f"{library_path()} is missing: build it with `python -m paged_kv_attention_block_b200.build` "
+        "(the CUDA library is the only implementation)")
+
+_lib = C.CDLL(library_path())
+
+PKV_F32, PKV_BF16, PKV_F16, PKV_FP8_E4M3 = 0, 1, 2, 3
+DTYPE_CODES = {"f32": PKV_F32, "bf16": PKV_BF16, "f16": PKV_F16, "e4m3": PKV_FP8_E4M3}
+_TORCH_CODES = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16,
+                torch.float8_e4m3fn: PKV_FP8_E4M3, torch.uint8: PKV_FP8_E4M3}
+_CODE_TORCH = {PKV_F32: torch.float32, PKV_BF16: torch.bfloat16, PKV_F16: torch.float16,
+               PKV_FP8_E4M3: torch.uint8}
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.pkv_last_error().decode()
+        super().__init__(f"{where}: {_lib.pkv_status_string(status).decode()} ({status}): {msg}")
+
+
+class _Cache(C.Structure):
+    _fields_ = [("pool", C.c_void_p), ("num_blocks", C.c_int64), ("num_layers", C.c_int32), ("layer", C.c_int32),
+                ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("block_size", C.c_int32),
+                ("kv_dtype", C.c_int32), ("k_scale", C.c_void_p), ("v_scale", C.c_void_p)]
+
+
+class _PlanRequest(C.Structure):
+    _fields_ = [("num_seqs", C.c_int32), ("num_q_heads", C.c_int32), ("num_kv_heads", C.c_int32),
+                ("head_dim", C.c_int32), ("block_size", C.c_int32), ("kv_dtype", C.c_int32), ("causal", C.c_int32),
+                ("num_ctas", C.c_int32), ("kv_split", C.c_int32), ("cascade", C.c_int32),
+                ("min_shared_tokens", C.c_int32), ("max_blocks", C.c_int32), ("cu_q_lens", C.c_void_p),
+                ("seq_lens", C.c_void_p), ("block_tables", C.c_void_p)]
+
+
+class _PlanInfo(C.Structure):
+    _fields_ = [("plan_bytes", C.c_size_t), ("workspace_bytes", C.c_size_t), ("num_items", C.c_int32),
+                ("num_reduce", C.c_int32), ("num_parts", C.c_int32), ("num_partial_rows", C.c_int32),
+                ("num_groups", C.c_int32), ("num_ctas", C.c_int32)]
+
+
+_P, _I32, _I64, _SZ, _F = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t, C.c_float
+_lib.pkv_abi_version.restype = _I32
+_lib.pkv_status_string.restype = C.c_char_p
+_lib.pkv_status_string.argtypes = [_I32]
+_lib.pkv_last_error.restype = C.c_char_p
+_lib.pkv_kv_append.restype = _I32
+_lib.pkv_kv_append.argtypes = [C.POINTER(_Cache), _P, _P, _I32, _P, _P, _P, _I32, _I32, _I32, _P, _P]
+_lib.pkv_attention_plan.restype = _I32
+_lib.pkv_attention_plan.argtypes = [C.POINTER(_PlanRequest), _P, _SZ, C.POINTER(_PlanInfo)]
+_lib.pkv_default_num_ctas.restype = _I32
+_lib.pkv_default_num_ctas.argtypes = [_I32, _I32, C.POINTER(_I32)]
+_lib.pkv_paged_attention.restype = _I32
+_lib.pkv_paged_attention.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P, _P, _P,
+                                     _P, _SZ, _P, _P]
+_lib.pkv_split_kv_reduce.restype = _I32
+_lib.pkv_split_kv_reduce.argtypes = [_P, _P, _I32, _I64, _I32, _P, _I32, _P, _P]
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise PkvError(status, where)
+
+
+def status_string(status: int) -> str:
+    return _lib.pkv_status_string(status).decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return _TORCH_CODES[t.dtype]
+
+
+@dataclass
+class Cache:
+    """A paged KV pool ``[num_blocks][num_layers][2][Hkv][B][D]`` on the GPU and the layer a call uses."""
+
+    pool: torch.Tensor
+    kv_dtype: int
+    block_size: int
+    layer: int = 0
+    k_scale: torch.Tensor | None = None  # float32 [num_layers][Hkv], fp8 pools
+    v_scale: torch.Tensor | None = None
+
+    @staticmethod
+    def allocate(num_blocks: int, num_layers: int, num_kv_heads: int, block_size: int, head_dim: int, kv_dtype: str,
+                 device="cuda", fill_nan: bool = True, k_scale=None, v_scale=None) -> "Cache":
+        code = DTYPE_CODES[kv_dtype]
+        shape = (num_blocks, num_layers, 2, num_kv_heads, block_size, head_dim)
+        tdt = _CODE_TORCH[code]
+        pool = torch.empty(shape, dtype=tdt, device=device)
+        if fill_nan:  # sentinel NaNs in every slot no sequence owns
+            if code == PKV_FP8_E4M3:
+                pool.fill_(0x7F)
+            else:
+                pool.fill_(float("nan"))
+        to_dev = lambda s: None if s is None else torch.as_tensor(s, dtype=torch.float32).to(device).contiguous()  # noqa: E731
+        return Cache(pool, code, block_size, 0, to_dev(k_scale), to_dev(v_scale))
+
+    @property
+    def num_kv_heads(self) -> int:
+        return self.pool.shape[3]
+
+    @property
+    def head_dim(self) -> int:
+        return self.pool.shape[5]
+
+    def _c(self) -> _Cache:
+        p = self.pool
+        return _Cache(p.data_ptr(), p.shape[0], p.shape[1], self.layer, p.shape[3], p.shape[5], self.block_size,
+                      self.kv_dtype, _ptr(self.k_scale), _ptr(self.v_scale))
+
+
+def kv_append(cache: Cache, k_new: torch.Tensor, v_new: torch.Tensor, cu_new: torch.Tensor, start_pos: torch.Tensor,
+              block_tables: torch.Tensor, total_new: int | None = None, status: torch.Tensor | None = None,
+              stream=None) -> None:
+    """Write packed new K/V rows ``[total_new][Hkv][D]`` into their pool slots (device tensors)."""
+    num_seqs = start_pos.shape[0]
+    if total_new is None:
+        total_new = k_new.shape[0]
+    c = cache._c()
+    _check(_lib.pkv_kv_append(C.byref(c), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(cu_new),
+                              _ptr(start_pos), _ptr(block_tables), block_tables.shape[1], num_seqs, total_new,
+                              _ptr(status), _stream(stream)), "kv_append")
+
+
+@dataclass
+class Plan:
+    """Host plan buffer (page-locked) and its sizes."""
+
+    buffer: torch.Tensor
+    info: dict
+
+    @property
+    def workspace_bytes(self) -> int:
+        return self.info["workspace_bytes"]
+
+
+def _host_i32(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+                   kv_dtype: int | str, causal: bool = True, block_tables=None, max_blocks: int | None = None,
+                   num_ctas: int = 0, kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0,
+                   pin: bool = True) -> Plan:
+    """Build the work list for one paged_attention call from host copies of the lengths."""
+    cu = _host_i32(cu_q_lens)
+    sl = _host_i32(seq_lens)
+    bt = None if block_tables is None else _host_i32(block_tables)
+    if max_blocks is None:
+        max_blocks = bt.shape[1] if bt is not None else 1
+    code = DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    req = _PlanRequest(sl.shape[0], num_q_heads, num_kv_heads, head_dim, block_size, code, int(bool(causal)), num_ctas,
+                       kv_split, int(bool(cascade)), min_shared_tokens, max_blocks, cu.ctypes.data, sl.ctypes.data,
+                       None if bt is None else bt.ctypes.data)
+    info = _PlanInfo()
+    _check(_lib.pkv_attention_plan(C.byref(req), None, 0, C.byref(info)), "attention_plan")
+    buf = torch.empty(int(info.plan_bytes), dtype=torch.uint8, pin_memory=pin and torch.cuda.is_available())
+    _check(_lib.pkv_attention_plan(C.byref(req), buf.data_ptr(), buf.numel(), C.byref(info)), "attention_plan")
+    return Plan(buf, {f: getattr(info, f) for f, _ in _PlanInfo._fields_})
+
+
+def attention_workspace_bytes(plan: Plan) -> int:
+    return plan.workspace_bytes
+
+
+def default_num_ctas(kv_dtype: int | str, head_dim: int) -> int:
+    code = DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    n = C.c_int32(0)
+    _check(_lib.pkv_default_num_ctas(code, head_dim, C.byref(n)), "default_num_ctas")
+    return n.value
+
+
+def paged_attention(cache: Cache, q: torch.Tensor, cu_q_lens: torch.Tensor, seq_lens: torch.Tensor,
+                    block_tables: torch.Tensor, plan: Plan, softmax_scale: float, causal: bool = True,
+                    out: torch.Tensor | None = None, out_lse: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
+    """out = softmax(scale q K^T) V over the paged cache; returns ``out``."""
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=q.device)
+    c = cache._c()
+    _check(_lib.pkv_paged_attention(C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens), _ptr(seq_lens),
+                                    _ptr(block_tables), block_tables.shape[1], seq_lens.shape[0], float(softmax_scale),
+                                    int(bool(causal)), plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse),
+                                    _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+           "paged_attention")
+    return out
+
+
+def split_kv_reduce(partial_o: torch.Tensor, partial_lse: torch.Tensor, out_dtype=torch.float32,
+                    out: torch.Tensor | None = None, out_lse: torch.Tensor | None = None, stream=None):
+    """Merge ``[n][rows][D]`` partial states into ``[rows][D]``; returns (out, out_lse)."""
+    n, rows, d = partial_o.shape
+    if out is None:
+        out = torch.empty((rows, d), dtype=out_dtype, device=partial_o.device)
+    _check(_lib.pkv_split_kv_reduce(_ptr(partial_o), _ptr(partial_lse), n, rows, d, _ptr(out), _dtype_code(out),
+                                    _ptr(out_lse), _stream(stream)), "split_kv_reduce")
+    return out, out_lse
+
+
+def decode_step_e2e(*args, **kwargs):  # defined in bench-facing helpers below
+    return _decode_step_e2e(*args, **kwargs)
+
+
+def _decode_step_e2e(cache: Cache, host: dict, dev: dict, plan_fn, softmax_scale: float, causal: bool, stream=None):
+    """One step from pinned host inputs: H2D copies, kv_append, plan, attention, D2H of the output.
+
+    ``host`` holds pinned CPU tensors (q, k_new, v_new, cu_q, seq_lens, start_pos,
+    block_tables, out); ``dev`` holds same-shaped device buffers and a workspace.
+    ``plan_fn`` returns the host Plan for this step's lengths.
+    """
+    for name in ("q", "k_new", "v_new", "cu_q", "seq_lens", "start_pos", "block_tables"):
+        dev[name].copy_(host[name], non_blocking=True)
+    kv_append(cache, dev["k_new"], dev["v_new"], dev["cu_q"], dev["start_pos"], dev["block_tables"], stream=stream)
+    plan = plan_fn()
+    paged_attention(cache, dev["q"], dev["cu_q"], dev["seq_lens"], dev["block_tables"], plan, softmax_scale, causal,
+                    out=dev["out"], workspace=dev["workspace"], stream=stream)
+    host["out"].copy_(dev["out"], non_blocking=True)
+    return plan

@@ -1,0 +1,192 @@
+// C ABI: argument checks, plan upload and launches of paged_attention, plus the
+// small shared entry points (version, status strings, error detail, occupancy).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "attn_args.h"
+#include "internal.h"
+#include "plan_format.h"
+
+namespace {
+thread_local char g_last_error[512] = "";
+}
+
+pkv_status pkv_fail(pkv_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+extern "C" int32_t pkv_abi_version(void) { return PKV_ABI_VERSION; }
+
+extern "C" const char* pkv_status_string(int32_t status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_WORKSPACE: return "buffer too small";
+    case PKV_ERR_PLAN: return "plan does not match the call";
+    default: return "unknown status";
+  }
+}
+
+extern "C" const char* pkv_last_error(void) { return g_last_error; }
+
+extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int32_t* num_ctas) {
+  if (!num_ctas) return pkv_fail(PKV_ERR_INVALID_ARG, "default_num_ctas: null output");
+  pkv::AttnKernel k;
+  const int q_dtype = kv_dtype == PKV_F32 ? PKV_F32 : (kv_dtype == PKV_F16 ? PKV_F16 : PKV_BF16);
+  if (!pkv::attn_kernel_for(kv_dtype, q_dtype, head_dim, &k))
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "default_num_ctas: no kernel for kv_dtype %d head_dim %d", kv_dtype, head_dim);
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess && k.smem > 48 * 1024)
+    e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, k.smem);
+  if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "default_num_ctas: %s", cudaGetErrorString(e));
+  *num_ctas = std::max(1, sms * std::max(1, per_sm));
+  return PKV_OK;
+}
+
+// Structural check of a host plan: every index the kernels follow stays inside
+// the plan and the workspace (lengths are checked against the device arrays by
+// the kernels themselves).
+static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv) {
+  const char* base = reinterpret_cast<const char*>(h);
+  const uint64_t bytes = h->bytes;
+  auto inside = [&](uint64_t off, uint64_t n, uint64_t sz) { return off + n * sz <= bytes; };
+  if (h->n_items < 0 || h->n_reduce < 0 || h->n_parts < 0 || h->n_part_rows < 0 || h->total_q < 0 ||
+      !inside(h->items_off, h->n_items, sizeof(PkvItem)) || !inside(h->reduce_off, h->n_reduce, sizeof(PkvReduce)) ||
+      !inside(h->parts_off, h->n_parts, sizeof(int32_t)) || h->num_ctas <= 0)
+    return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan sections out of range");
+  const PkvItem* items = reinterpret_cast<const PkvItem*>(base + h->items_off);
+  for (int i = 0; i < h->n_items; ++i) {
+    const PkvItem& it = items[i];
+    const int64_t rows = int64_t(it.n_q) * g;
+    if (it.n_q <= 0 || rows > PKV_TILE_ROWS || it.kv_head < 0 || it.kv_head >= hkv || it.q_begin < 0 ||
+        int64_t(it.q_begin) + it.n_q > h->total_q || it.k_begin < 0 || it.k_begin > it.k_end ||
+        (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows))
+      return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan item %d out of range", i);
+  }
+  const PkvReduce* reds = reinterpret_cast<const PkvReduce*>(base + h->reduce_off);
+  const int32_t* parts = reinterpret_cast<const int32_t*>(base + h->parts_off);
+  for (int i = 0; i < h->n_reduce; ++i) {
+    const PkvReduce& r = reds[i];
+    const int64_t rows = int64_t(r.n_q) * g;
+    if (r.n_q <= 0 || rows > PKV_TILE_ROWS || r.kv_head < 0 || r.kv_head >= hkv || r.q_begin < 0 ||
+        int64_t(r.q_begin) + r.n_q > h->total_q || r.parts_begin < 0 || r.n_parts < 0 ||
+        int64_t(r.parts_begin) + r.n_parts > h->n_parts)
+      return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan merge %d out of range", i);
+    for (int p = 0; p < r.n_parts; ++p) {
+      const int32_t row = parts[r.parts_begin + p];
+      if (row < 0 || int64_t(row) + rows > h->n_part_rows)
+        return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan merge %d part %d out of range", i, p);
+    }
+  }
+  return PKV_OK;
+}
+
+extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                                          const int32_t* cu_q_lens, const int32_t* seq_lens,
+                                          const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                          float softmax_scale, int32_t causal, const void* plan, void* out,
+                                          float* out_lse, void* workspace, size_t workspace_bytes,
+                                          int32_t* dev_status, void* stream) {
+  if (!cache || !plan) return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: cache and plan are required");
+  const pkv_cache& c = *cache;
+  const PkvPlanHeader* h = static_cast<const PkvPlanHeader*>(plan);
+  if (h->magic != PKV_PLAN_MAGIC) return pkv_fail(PKV_ERR_PLAN, "paged_attention: not a plan buffer");
+  if (c.num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % c.num_kv_heads != 0)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: num_q_heads %d, num_kv_heads %d", num_q_heads, c.num_kv_heads);
+  if (!pkv_is_pow2(c.block_size) || c.block_size < 2)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: block_size %d is not a power of two > 1", c.block_size);
+  if (c.num_layers <= 0 || c.layer < 0 || c.layer >= c.num_layers || c.num_blocks <= 0)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: bad cache shape");
+  if (h->num_seqs != num_seqs || h->num_q_heads != num_q_heads || h->num_kv_heads != c.num_kv_heads ||
+      h->head_dim != c.head_dim || h->block_size != c.block_size || h->kv_dtype != c.kv_dtype ||
+      h->causal != (causal ? 1 : 0))
+    return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan was made for other shapes");
+  pkv::AttnKernel k;
+  if (!pkv::attn_kernel_for(c.kv_dtype, q_dtype, c.head_dim, &k))
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "paged_attention: kv_dtype %d with q_dtype %d, head_dim %d", c.kv_dtype,
+                    q_dtype, c.head_dim);
+  if (c.kv_dtype == PKV_FP8_E4M3 && (!c.k_scale || !c.v_scale))
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: fp8 pool needs k_scale and v_scale");
+  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads); vs != PKV_OK) return vs;
+  const PkvWorkspaceLayout L = pkv_workspace_layout(h->bytes, h->n_part_rows, c.head_dim);
+  if (h->n_items == 0) return PKV_OK;
+  if (!workspace || workspace_bytes < L.total)
+    return pkv_fail(PKV_ERR_WORKSPACE, "paged_attention: workspace %zu < %llu bytes", workspace_bytes,
+                    (unsigned long long)L.total);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: workspace not 256-byte aligned");
+  if (!c.pool || !q || !out || !cu_q_lens || !seq_lens || !block_tables || max_blocks <= 0)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: null pointer or max_blocks <= 0");
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(c.pool)) & 15)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: q and pool must be 16-byte aligned");
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e = cudaMemcpyAsync(ws + L.plan_off, plan, h->bytes, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.counter_off, 0, 256, st);
+  if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: plan upload: %s", cudaGetErrorString(e));
+  if (k.smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: %s", cudaGetErrorString(e));
+  }
+  const char* dplan = ws + L.plan_off;
+  pkv::AttnArgs a{};
+  a.pool = c.pool;
+  a.num_blocks = c.num_blocks;
+  a.num_layers = c.num_layers;
+  a.layer = c.layer;
+  a.hkv = c.num_kv_heads;
+  a.log2_block = pkv_log2(c.block_size);
+  a.k_scale = c.k_scale;
+  a.v_scale = c.v_scale;
+  a.q = q;
+  a.out = out;
+  a.out_lse = out_lse;
+  a.cu_q_lens = cu_q_lens;
+  a.seq_lens = seq_lens;
+  a.block_tables = block_tables;
+  a.max_blocks = max_blocks;
+  a.num_seqs = num_seqs;
+  a.hq = num_q_heads;
+  a.g = num_q_heads / c.num_kv_heads;
+  a.softmax_scale = softmax_scale;
+  a.items = reinterpret_cast<const PkvItem*>(dplan + h->items_off);
+  a.n_items = h->n_items;
+  a.counter = reinterpret_cast<unsigned int*>(ws + L.counter_off);
+  a.part_o = reinterpret_cast<float*>(ws + L.part_o_off);
+  a.part_lse = reinterpret_cast<float*>(ws + L.part_lse_off);
+  a.status = dev_status;
+  const int grid = std::max(1, std::min(h->num_ctas, h->n_items));
+  k.launch(a, grid, st);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: launch failed: %s", cudaGetErrorString(e));
+  if (h->n_reduce > 0) {
+    pkv::ReduceArgs r{};
+    r.reduces = reinterpret_cast<const PkvReduce*>(dplan + h->reduce_off);
+    r.parts = reinterpret_cast<const int32_t*>(dplan + h->parts_off);
+    r.n_reduce = h->n_reduce;
+    r.part_o = a.part_o;
+    r.part_lse = a.part_lse;
+    r.out = out;
+    r.out_lse = out_lse;
+    r.out_dtype = q_dtype;
+    r.hq = num_q_heads;
+    r.g = a.g;
+    r.head_dim = c.head_dim;
+    e = pkv::launch_plan_reduce(r, st);
+    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: merge launch failed: %s", cudaGetErrorString(e));
+  }
+  return PKV_OK;
+}

@@ -1,0 +1,53 @@
+// Launch arguments of the attention and merge kernels (host and device).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "plan_format.h"
+
+namespace pkv {
+
+struct AttnArgs {
+  const void* pool;
+  int64_t num_blocks;
+  int32_t num_layers, layer, hkv, log2_block;
+  const float* k_scale;  // fp8 pools only
+  const float* v_scale;
+  const void* q;
+  void* out;
+  float* out_lse;
+  const int32_t* cu_q_lens;
+  const int32_t* seq_lens;
+  const int32_t* block_tables;
+  int32_t max_blocks, num_seqs, hq, g;
+  float softmax_scale;
+  const PkvItem* items;  // device copy of the plan's items
+  int32_t n_items;
+  unsigned int* counter;  // work counter, zeroed before the launch
+  float* part_o;          // [n_part_rows][head_dim]
+  float* part_lse;        // [n_part_rows]
+  int32_t* status;
+};
+
+struct ReduceArgs {
+  const PkvReduce* reduces;
+  const int32_t* parts;
+  int32_t n_reduce;
+  const float* part_o;
+  const float* part_lse;
+  void* out;
+  float* out_lse;
+  int32_t out_dtype, hq, g, head_dim;
+};
+
+// Kernel selection for one (pool dtype, q dtype, head_dim).
+struct AttnKernel {
+  const void* fn;
+  int threads;
+  int smem;
+  void (*launch)(const AttnArgs&, int grid, cudaStream_t);
+};
+bool attn_kernel_for(int kv_dtype, int q_dtype, int head_dim, AttnKernel* k);
+cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st);
+
+}  // namespace pkv

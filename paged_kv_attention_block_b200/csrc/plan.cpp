@@ -1,0 +1,233 @@
+// Host-side planner: turns one in-flight batch into the work list of a
+// persistent attention launch.
+//
+// Deep dive (gentlecold.top) §6: a batch packs context requests before
+// generation requests, so one launch mixes long causal chunks with one-token
+// decode rows; §8: chunks attend to the cached KV plus themselves; §10:
+// sequences may share prefix blocks through radix-tree reuse.  The planner
+//   1. groups consecutive sequences whose block tables start with the same
+//      physical blocks (cascade): their shared keys become one dense tile per
+//      group and KV head instead of one read per sequence;
+//   2. cuts every (sequence, query tile, KV head) into key ranges small enough
+//      that the persistent CTAs finish together, weighting a tile by its rows
+//      (compute) and keys (bytes);
+//   3. emits the merges that combine split ranges (and group tiles) per row.
+// Items are ordered heaviest first; CTAs pull them from an atomic counter.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "internal.h"
+#include "plan_format.h"
+
+namespace {
+
+struct Unit {
+  int seq, kv_head, q_begin, n_q, k_begin, k_end, pos0, group_part;
+  double weight;
+};
+
+struct Seg {
+  PkvItem it;
+  double cost;
+  int order;
+};
+
+double row_weight(int rows) { return rows <= 16 ? 1.0 : rows / 16.0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan, size_t capacity,
+                                         pkv_plan_info* info) {
+  if (!req || !info) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: req and info are required");
+  std::memset(info, 0, sizeof(*info));
+  const int S = req->num_seqs, Hq = req->num_q_heads, Hkv = req->num_kv_heads, D = req->head_dim;
+  const int B = req->block_size;
+  if (S < 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: num_seqs < 0");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)", Hq, Hkv);
+  const int g = Hq / Hkv;
+  if (g > PKV_TILE_ROWS) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: more than %d query heads per KV head", PKV_TILE_ROWS);
+  if (D != 64 && D != 128) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: head_dim %d (64 or 128)", D);
+  if (!pkv_is_pow2(B) || B < 2) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: block_size %d is not a power of two > 1", B);
+  if (req->kv_dtype < PKV_F32 || req->kv_dtype > PKV_FP8_E4M3) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: kv_dtype");
+  if (S > 0 && (!req->cu_q_lens || !req->seq_lens)) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: null length arrays");
+  if (S > 0 && req->max_blocks <= 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: max_blocks");
+  const int32_t* cu = req->cu_q_lens;
+  const int32_t* L = req->seq_lens;
+  if (S > 0 && cu[0] != 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: cu_q_lens[0] != 0");
+  for (int s = 0; s < S; ++s) {
+    const int ql = cu[s + 1] - cu[s];
+    if (ql < 0 || L[s] < 0 || ql > L[s])
+      return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: sequence %d has q_len %d, seq_len %d", s, ql, L[s]);
+    if ((int64_t(L[s]) + B - 1) / B > req->max_blocks)
+      return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: sequence %d needs %d blocks > max_blocks %d", s,
+                      (L[s] + B - 1) / B, req->max_blocks);
+  }
+  int num_ctas = req->num_ctas;
+  if (num_ctas <= 0) {
+    pkv_status st = pkv_default_num_ctas(req->kv_dtype, D, &num_ctas);
+    if (st != PKV_OK) return st;
+  }
+  const int QT = std::max(1, PKV_TILE_ROWS / g);  // query tokens per tile
+  const bool causal = req->causal != 0;
+  auto q_len = [&](int s) { return cu[s + 1] - cu[s]; };
+
+  // 1. Shared-prefix groups.
+  struct Group { int first, last, tokens; };
+  std::vector<Group> groups;
+  std::vector<int> group_of(S, -1);
+  if (req->cascade && req->block_tables && S > 1) {
+    const int32_t* bt = req->block_tables;
+    const int64_t mb = req->max_blocks;
+    const int min_sh = req->min_shared_tokens > 0 ? req->min_shared_tokens : 256;
+    // Blocks of a sequence every query row may see in full.
+    auto usable = [&](int t) { return (causal ? L[t] - q_len(t) + 1 : L[t]) / B; };
+    int s = 0;
+    while (s < S) {
+      if (q_len(s) < 1 || q_len(s) > QT) { ++s; continue; }
+      int P = usable(s), t = s + 1;
+      while (t < S && q_len(t) >= 1 && q_len(t) <= QT) {
+        const int lim = std::min(P, usable(t));
+        int c = 0;
+        while (c < lim && bt[s * mb + c] == bt[t * mb + c]) ++c;
+        if (int64_t(c) * B < min_sh) break;
+        P = c;
+        ++t;
+      }
+      if (t - s >= 2 && int64_t(P) * B >= min_sh) {
+        for (int m = s; m < t; ++m) group_of[m] = int(groups.size());
+        groups.push_back({s, t - 1, P * B});
+        s = t;
+      } else {
+        ++s;
+      }
+    }
+  }
+
+  std::vector<Seg> segs;
+  std::vector<PkvReduce> reds;
+  std::vector<int32_t> parts;
+  int64_t part_rows = 0;
+  int order = 0;
+  // Partial row of each (group member, KV head) inside its group tile.
+  std::vector<int64_t> gpart(groups.empty() ? 0 : size_t(S) * Hkv, -1);
+  double total_cost = 0;
+  for (const Group& G : groups) {
+    int a = G.first;
+    while (a <= G.last) {
+      int b = a, n = q_len(a);
+      while (b + 1 <= G.last && n + q_len(b + 1) <= QT) n += q_len(++b);
+      for (int h = 0; h < Hkv; ++h) {
+        PkvItem it{G.first, h, cu[a], n, 0, G.tokens, -1, int32_t(part_rows)};
+        for (int m = a; m <= b; ++m) gpart[size_t(m) * Hkv + h] = part_rows + int64_t(cu[m] - cu[a]) * g;
+        part_rows += int64_t(n) * g;
+        const double c = double(G.tokens) * row_weight(n * g);
+        total_cost += c;
+        segs.push_back({it, c, order++});
+      }
+      a = b + 1;
+    }
+  }
+
+  // 2. Units of work.
+  std::vector<Unit> units;
+  for (int s = 0; s < S; ++s) {
+    const int ql = q_len(s);
+    if (ql == 0) continue;
+    const int kb = group_of[s] >= 0 ? groups[group_of[s]].tokens : 0;
+    for (int i0 = 0; i0 < ql; i0 += QT) {
+      const int n = std::min(QT, ql - i0);
+      const int ke = causal ? L[s] - ql + i0 + n : L[s];
+      const int pos0 = causal ? L[s] - ql + i0 : -1;
+      for (int h = 0; h < Hkv; ++h) {
+        const int gp = group_of[s] >= 0 ? int(gpart[size_t(s) * Hkv + h]) : -1;
+        Unit u{s, h, cu[s] + i0, n, kb, ke, pos0, gp, row_weight(n * g)};
+        total_cost += double(std::max(0, ke - kb)) * u.weight;
+        units.push_back(u);
+      }
+    }
+  }
+
+  // 3. Key-range split and merges.
+  const double target = total_cost / (double(num_ctas) * 2.0);
+  for (const Unit& u : units) {
+    const int n = std::max(0, u.k_end - u.k_begin);
+    int64_t max_keys;
+    if (req->kv_split < 0) max_keys = INT32_MAX;
+    else if (req->kv_split > 0) max_keys = round_up(req->kv_split, PKV_TILE_KEYS);
+    else max_keys = std::max<int64_t>(256, round_up(int64_t(std::ceil(target / u.weight)), PKV_TILE_KEYS));
+    const int64_t nseg = n == 0 ? 0 : (n + max_keys - 1) / max_keys;
+    const int rows = u.n_q * g;
+    if (nseg == 1 && u.group_part < 0) {
+      PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, u.k_begin, u.k_end, u.pos0, -1};
+      segs.push_back({it, n * u.weight, order++});
+      continue;
+    }
+    PkvReduce r{u.q_begin, u.n_q, u.kv_head, int32_t(parts.size()), 0, {0, 0, 0}};
+    if (u.group_part >= 0) parts.push_back(u.group_part);
+    if (nseg > 0) {
+      const int64_t seg = round_up((n + nseg - 1) / nseg, PKV_TILE_KEYS);
+      for (int64_t k0 = u.k_begin; k0 < u.k_end; k0 += seg) {
+        const int k1 = int(std::min<int64_t>(u.k_end, k0 + seg));
+        PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, int(k0), k1, u.pos0, int32_t(part_rows)};
+        parts.push_back(int32_t(part_rows));
+        part_rows += rows;
+        segs.push_back({it, (k1 - k0) * u.weight, order++});
+      }
+    }
+    r.n_parts = int32_t(parts.size()) - r.parts_begin;
+    reds.push_back(r);
+  }
+  if (part_rows > INT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: too many partial rows");
+
+  std::stable_sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) { return x.cost > y.cost; });
+
+  const uint64_t items_off = sizeof(PkvPlanHeader);
+  const uint64_t reduce_off = items_off + segs.size() * sizeof(PkvItem);
+  const uint64_t parts_off = reduce_off + reds.size() * sizeof(PkvReduce);
+  const uint64_t bytes = (parts_off + parts.size() * sizeof(int32_t) + 15) & ~uint64_t(15);
+  if (bytes > UINT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: plan too large");
+  info->plan_bytes = bytes;
+  info->workspace_bytes = pkv_workspace_layout(bytes, part_rows, D).total;
+  info->num_items = int32_t(segs.size());
+  info->num_reduce = int32_t(reds.size());
+  info->num_parts = int32_t(parts.size());
+  info->num_partial_rows = int32_t(part_rows);
+  info->num_groups = int32_t(groups.size());
+  info->num_ctas = num_ctas;
+  if (!plan) return PKV_OK;
+  if (capacity < bytes) return pkv_fail(PKV_ERR_WORKSPACE, "attention_plan: capacity %zu < %llu", capacity, (unsigned long long)bytes);
+
+  char* p = static_cast<char*>(plan);
+  std::memset(p, 0, bytes);
+  PkvPlanHeader h{};
+  h.magic = PKV_PLAN_MAGIC;
+  h.bytes = uint32_t(bytes);
+  h.n_items = info->num_items;
+  h.n_reduce = info->num_reduce;
+  h.n_parts = info->num_parts;
+  h.n_part_rows = info->num_partial_rows;
+  h.num_seqs = S;
+  h.total_q = S > 0 ? cu[S] : 0;
+  h.num_q_heads = Hq;
+  h.num_kv_heads = Hkv;
+  h.head_dim = D;
+  h.block_size = B;
+  h.kv_dtype = req->kv_dtype;
+  h.causal = causal ? 1 : 0;
+  h.num_ctas = num_ctas;
+  h.n_groups = info->num_groups;
+  h.items_off = uint32_t(items_off);
+  h.reduce_off = uint32_t(reduce_off);
+  h.parts_off = uint32_t(parts_off);
+  std::memcpy(p, &h, sizeof(h));
+  PkvItem* items = reinterpret_cast<PkvItem*>(p + items_off);
+  for (size_t i = 0; i < segs.size(); ++i) items[i] = segs[i].it;
+  if (!reds.empty()) std::memcpy(p + reduce_off, reds.data(), reds.size() * sizeof(PkvReduce));
+  if (!parts.empty()) std::memcpy(p + parts_off, parts.data(), parts.size() * sizeof(int32_t));
+  return PKV_OK;
+}

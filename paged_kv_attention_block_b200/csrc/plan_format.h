@@ -1,0 +1,85 @@
+// Work-list format shared by the host planner and the attention kernels.
+//
+// A plan is one contiguous buffer: header, items, merges, part list.  The host
+// builds it (plan.cpp), paged_attention copies it into the device workspace,
+// and every CTA of the persistent kernel pulls items from it.
+#pragma once
+#include <stdint.h>
+
+#define PKV_PLAN_MAGIC 0x314e4c50u  // "PLN1"
+
+// Rows of one work item: query tokens x the Hq/Hkv query heads of one KV head.
+#define PKV_TILE_ROWS 64
+// Keys per pipeline stage.
+#define PKV_TILE_KEYS 64
+
+struct PkvPlanHeader {
+  uint32_t magic;
+  uint32_t bytes;        // whole plan, header included
+  int32_t n_items;
+  int32_t n_reduce;
+  int32_t n_parts;
+  int32_t n_part_rows;
+  int32_t num_seqs;
+  int32_t total_q;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t block_size;
+  int32_t kv_dtype;
+  int32_t causal;
+  int32_t num_ctas;
+  int32_t n_groups;
+  uint32_t items_off;    // byte offsets from the start of the plan
+  uint32_t reduce_off;
+  uint32_t parts_off;
+  int32_t pad[13];       // header is 128 bytes
+};
+static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
+
+// One CTA-sized piece of work: rows [q_begin, q_begin + n_q) x the g query
+// heads of kv_head, against keys [k_begin, k_end) read through the block-table
+// row of `seq`.  Row r of the tile is query token q_begin + r / g, head
+// kv_head * g + r % g.  With pos0 >= 0 the tile is causal: token q_begin + i
+// sits at position pos0 + i and sees keys < pos0 + i + 1.  part_row < 0 writes
+// the final output; otherwise the normalised partial state goes to partial
+// rows part_row .. part_row + n_q * g - 1.
+struct PkvItem {
+  int32_t seq;
+  int32_t kv_head;
+  int32_t q_begin;
+  int32_t n_q;
+  int32_t k_begin;
+  int32_t k_end;
+  int32_t pos0;
+  int32_t part_row;
+};
+static_assert(sizeof(PkvItem) == 32, "item size");
+
+// Output rows [q_begin, q_begin + n_q) x heads of kv_head, merged from the
+// partial states listed in parts[parts_begin .. parts_begin + n_parts): entry
+// p names the partial row holding row 0 of this tile.
+struct PkvReduce {
+  int32_t q_begin;
+  int32_t n_q;
+  int32_t kv_head;
+  int32_t parts_begin;
+  int32_t n_parts;
+  int32_t pad[3];
+};
+static_assert(sizeof(PkvReduce) == 32, "reduce size");
+
+// Device workspace layout: [plan copy][counters][partial o][partial lse].
+static inline uint64_t pkv_align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+struct PkvWorkspaceLayout {
+  uint64_t plan_off, counter_off, part_o_off, part_lse_off, total;
+};
+static inline PkvWorkspaceLayout pkv_workspace_layout(uint64_t plan_bytes, int64_t n_part_rows, int head_dim) {
+  PkvWorkspaceLayout L;
+  L.plan_off = 0;
+  L.counter_off = pkv_align256(plan_bytes);
+  L.part_o_off = L.counter_off + 256;
+  L.part_lse_off = pkv_align256(L.part_o_off + uint64_t(n_part_rows) * head_dim * 4);
+  L.total = pkv_align256(L.part_lse_off + uint64_t(n_part_rows) * 4);
+  return L;
+}

@@ -1,0 +1,105 @@
+// split_kv_reduce: merge partial softmax states over disjoint key sets.
+//
+// For one output row with parts (o_i normalised, lse_i natural log):
+//   M = max_i lse_i, w_i = exp(lse_i - M), o = sum w_i o_i / sum w_i,
+//   lse = M + ln sum w_i; parts with lse = -inf weigh nothing.
+// Two launch forms share the per-element merge: the public dense form
+// ([n_split][rows][d] partials) and the plan-driven form that finishes a paged
+// attention launch whose key ranges were split (ragged part lists per tile).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "attn_args.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+PKV_DEVICE void store_any(void* out, int dtype, int64_t idx, float v) {
+  if (dtype == PKV_F32) static_cast<float*>(out)[idx] = v;
+  else if (dtype == PKV_BF16) static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
+  else static_cast<__half*>(out)[idx] = __float2half_rn(v);
+}
+
+// Merge element `d` of a row whose i-th part lives at o_of(i), lse_of(i).
+template <typename LseOf, typename OOf>
+PKV_DEVICE void merge_elem(int n, LseOf lse_of, OOf o_of, float& o, float& lse) {
+  float M = -INFINITY;
+  for (int i = 0; i < n; ++i) M = fmaxf(M, lse_of(i));
+  if (M == -INFINITY) {
+    o = 0.f;
+    lse = -INFINITY;
+    return;
+  }
+  float num = 0.f, den = 0.f;
+  for (int i = 0; i < n; ++i) {
+    const float li = lse_of(i);
+    if (li == -INFINITY) continue;
+    const float w = expf(li - M);
+    den += w;
+    num = fmaf(w, o_of(i), num);
+  }
+  o = num / den;
+  lse = M + logf(den);
+}
+
+__global__ void __launch_bounds__(256) dense_reduce_kernel(const float* __restrict__ po, const float* __restrict__ pl,
+                                                           int n, int64_t rows, int d, void* out, int out_dtype,
+                                                           float* out_lse) {
+  const int64_t total = rows * d;
+  for (int64_t x = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; x < total; x += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = x / d;
+    float o, lse;
+    merge_elem(
+        n, [&](int i) { return pl[i * rows + r]; }, [&](int i) { return po[i * total + x]; }, o, lse);
+    store_any(out, out_dtype, x, o);
+    if (out_lse && x % d == 0) out_lse[r] = lse;
+  }
+}
+
+__global__ void __launch_bounds__(256) plan_reduce_kernel(const ReduceArgs a) {
+  const int d = a.head_dim;
+  for (int e = blockIdx.x; e < a.n_reduce; e += gridDim.x) {
+    const PkvReduce red = a.reduces[e];
+    const int R = red.n_q * a.g;
+    const int32_t* parts = a.parts + red.parts_begin;
+    for (int x = threadIdx.x; x < R * d; x += blockDim.x) {
+      const int r = x / d, k = x % d;
+      float o, lse;
+      merge_elem(
+          red.n_parts, [&](int i) { return a.part_lse[int64_t(parts[i]) + r]; },
+          [&](int i) { return a.part_o[(int64_t(parts[i]) + r) * d + k]; }, o, lse);
+      const int64_t orow = (int64_t(red.q_begin) + r / a.g) * a.hq + red.kv_head * a.g + r % a.g;
+      store_any(a.out, a.out_dtype, orow * d + k, o);
+      if (a.out_lse && k == 0) a.out_lse[orow] = lse;
+    }
+  }
+}
+
+cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st) {
+  if (r.n_reduce <= 0) return cudaSuccess;
+  const int grid = std::min(r.n_reduce, 148 * 8);
+  plan_reduce_kernel<<<grid, 256, 0, st>>>(r);
+  return cudaGetLastError();
+}
+
+}  // namespace pkv
+
+extern "C" pkv_status pkv_split_kv_reduce(const float* partial_o, const float* partial_lse, int32_t n_split,
+                                          int64_t rows, int32_t head_dim, void* out, int32_t out_dtype,
+                                          float* out_lse, void* stream) {
+  if (n_split < 0 || rows < 0 || head_dim <= 0) return pkv_fail(PKV_ERR_INVALID_ARG, "split_kv_reduce: negative sizes");
+  if (out_dtype != PKV_F32 && out_dtype != PKV_BF16 && out_dtype != PKV_F16)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "split_kv_reduce: out_dtype must be F32, BF16 or F16");
+  if (rows == 0) return PKV_OK;
+  if (!out || (n_split > 0 && (!partial_o || !partial_lse)))
+    return pkv_fail(PKV_ERR_INVALID_ARG, "split_kv_reduce: null pointer");
+  const int64_t total = rows * head_dim;
+  const int grid = int(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  pkv::dense_reduce_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(partial_o, partial_lse, n_split, rows,
+                                                                                 head_dim, out, out_dtype, out_lse);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "split_kv_reduce: launch failed: %s", cudaGetErrorString(e));
+  return PKV_OK;
+}

@@ -1,0 +1,87 @@
+"""Decode a plan buffer (host bytes) into numpy records, for tests."""
+import numpy as np
+
+HEADER = np.dtype([("magic", "<u4"), ("bytes", "<u4"), ("n_items", "<i4"), ("n_reduce", "<i4"), ("n_parts", "<i4"),
+                   ("n_part_rows", "<i4"), ("num_seqs", "<i4"), ("total_q", "<i4"), ("num_q_heads", "<i4"),
+                   ("num_kv_heads", "<i4"), ("head_dim", "<i4"), ("block_size", "<i4"), ("kv_dtype", "<i4"),
+                   ("causal", "<i4"), ("num_ctas", "<i4"), ("n_groups", "<i4"), ("items_off", "<u4"),
+                   ("reduce_off", "<u4"), ("parts_off", "<u4"), ("pad", "<i4", 13)])
+ITEM = np.dtype([("seq", "<i4"), ("kv_head", "<i4"), ("q_begin", "<i4"), ("n_q", "<i4"), ("k_begin", "<i4"),
+                 ("k_end", "<i4"), ("pos0", "<i4"), ("part_row", "<i4")])
+REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("parts_begin", "<i4"),
+                   ("n_parts", "<i4"), ("pad", "<i4", 3)])
+assert HEADER.itemsize == 128 and ITEM.itemsize == 32 and REDUCE.itemsize == 32
+
+
+def decode(buf) -> dict:
+    b = np.asarray(buf.cpu().numpy() if hasattr(buf, "cpu") else buf, dtype=np.uint8)
+    h = np.frombuffer(b[:128].tobytes(), HEADER)[0]
+    items = np.frombuffer(b[h["items_off"]:h["items_off"] + 32 * h["n_items"]].tobytes(), ITEM)
+    reds = np.frombuffer(b[h["reduce_off"]:h["reduce_off"] + 32 * h["n_reduce"]].tobytes(), REDUCE)
+    parts = np.frombuffer(b[h["parts_off"]:h["parts_off"] + 4 * h["n_parts"]].tobytes(), "<i4")
+    return {"header": h, "items": items, "reduces": reds, "parts": parts}
+
+
+def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: int, causal: bool, block_tables=None,
+                   block_size=None):
+    """Every (query token, KV head) row group sees exactly its keys once, through one output path."""
+    h, items, reds, parts = plan["header"], plan["items"], plan["reduces"], plan["parts"]
+    g = num_q_heads // num_kv_heads
+    S = len(seq_lens)
+    tok_seq = np.repeat(np.arange(S), np.diff(cu_q))
+    # Partial rows: map part_row -> item, and check items' partial rows don't overlap.
+    used = np.zeros(max(1, int(h["n_part_rows"])), np.int32)
+    by_part = {}
+    for it in items:
+        assert 1 <= it["n_q"] and it["n_q"] * g <= 64 and it["k_begin"] < it["k_end"]
+        if it["part_row"] >= 0:
+            used[it["part_row"]:it["part_row"] + it["n_q"] * g] += 1
+            by_part[int(it["part_row"])] = it
+    assert (used <= 1).all()
+    # Expected key set per (token, kv head): [0, limit).
+    seen = {}
+
+    def add(tok, kvh, a, b, via):
+        seen.setdefault((tok, kvh), []).append((a, b, via))
+
+    direct = items[items["part_row"] < 0]
+    for it in direct:
+        for i in range(it["n_q"]):
+            add(int(it["q_begin"]) + i, int(it["kv_head"]), int(it["k_begin"]), int(it["k_end"]), "direct")
+    for r in reds:
+        for p in parts[r["parts_begin"]:r["parts_begin"] + r["n_parts"]]:
+            # The part is either an item's first row or a row inside a group item.
+            src = None
+            for row0, it in by_part.items():
+                if row0 <= p < row0 + it["n_q"] * g:
+                    src = it
+                    off = (p - row0) // g
+                    break
+            assert src is not None, "part row without an item"
+            assert src["kv_head"] == r["kv_head"]
+            for i in range(r["n_q"]):
+                tok = int(r["q_begin"]) + i
+                assert int(src["q_begin"]) + off + i == tok
+                add(tok, int(r["kv_head"]), int(src["k_begin"]), int(src["k_end"]), "part")
+            if block_tables is not None and src["seq"] != tok_seq[int(r["q_begin"])]:
+                # Group tile: the keys it reads must be identical blocks in both tables.
+                s_own, s_src = tok_seq[int(r["q_begin"])], int(src["seq"])
+                nb = (int(src["k_end"]) + block_size - 1) // block_size
+                assert (block_tables[s_own, :nb] == block_tables[s_src, :nb]).all()
+    for tok in range(int(cu_q[-1])):
+        s = tok_seq[tok]
+        j = tok - int(cu_q[s])
+        ql, L = int(cu_q[s + 1] - cu_q[s]), int(seq_lens[s])
+        lim = L - ql + j + 1 if causal else L
+        for kvh in range(num_kv_heads):
+            ranges = sorted(seen.pop((tok, kvh)))
+            vias = {v for _, _, v in ranges}
+            assert len(vias) == 1, "a row is both written directly and merged"
+            cover = 0
+            for a, b, _ in ranges:
+                assert a == cover, (tok, kvh, ranges)
+                cover = b
+            # Ranges may extend past a causal row's own limit (the kernel masks per row)
+            # but must cover it and stop at the tile's last row limit.
+            assert cover >= lim and cover <= (L if not causal else L)
+    assert not seen

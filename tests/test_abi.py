@@ -1,0 +1,152 @@
+"""The C ABI without a GPU: exports, argument checks, and the host planner (CPU only)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from paged_kv_attention_block_b200 import build as B
+from paged_kv_attention_block_b200 import workloads as W
+import plan_decode as PD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def api():
+    B.build()
+    from paged_kv_attention_block_b200 import api as A
+    return A
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    return sorted(set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(pkv_\w+)\s*\(", text)))
+
+
+def test_exports_match_header(api):
+    names = declared_symbols()
+    assert len(names) >= 8
+    lib = C.CDLL(api.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", api.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (pkv_\w+)", out))
+    assert set(names) == exported, (set(names) ^ exported)
+
+
+def test_version_and_strings(api):
+    assert api._lib.pkv_abi_version() == 1
+    assert api.status_string(0) == "ok" and api.status_string(4) == "buffer too small"
+
+
+def _cache(**kw):
+    from paged_kv_attention_block_b200 import api as A
+    d = dict(pool=0x1000, num_blocks=10, num_layers=1, layer=0, num_kv_heads=2, head_dim=64, block_size=16,
+             kv_dtype=A.PKV_BF16, k_scale=None, v_scale=None)
+    d.update(kw)
+    return A._Cache(**d)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(block_size=24), 1), (dict(block_size=1), 1), (dict(head_dim=96), 2), (dict(layer=1), 1),
+    (dict(kv_dtype=7), 1),
+])
+def test_kv_append_rejects(api, bad, code):
+    c = _cache(**bad)
+    st = api._lib.pkv_kv_append(C.byref(c), 0x1000, 0x1000, c.kv_dtype, 0x1000, 0x1000, 0x1000, 4, 1, 1, None, None)
+    assert st == code, api._lib.pkv_last_error()
+
+
+def test_kv_append_dtype_rules(api):
+    c = _cache()
+    assert api._lib.pkv_kv_append(C.byref(c), 0x1000, 0x1000, api.PKV_F32, 0x1000, 0x1000, 0x1000, 4, 1, 1, None,
+                                  None) == 1
+    c8 = _cache(kv_dtype=api.PKV_FP8_E4M3)
+    assert api._lib.pkv_kv_append(C.byref(c8), 0x1000, 0x1000, api.PKV_F32, 0x1000, 0x1000, 0x1000, 4, 1, 1, None,
+                                  None) == 1  # no scales
+    # Nothing to do is fine and touches no device.
+    assert api._lib.pkv_kv_append(C.byref(c), 0, 0, api.PKV_BF16, 0, 0, 0, 4, 0, 0, None, None) == 0
+
+
+def test_split_reduce_rejects(api):
+    assert api._lib.pkv_split_kv_reduce(0x1000, 0x1000, 2, 4, 64, 0x1000, 3, None, None) == 1  # fp8 output
+    assert api._lib.pkv_split_kv_reduce(0x1000, 0x1000, -1, 4, 64, 0x1000, 0, None, None) == 1
+    assert api._lib.pkv_split_kv_reduce(None, None, 2, 0, 64, None, 0, None, None) == 0
+
+
+def _plan(api, w, **kw):
+    kw.setdefault("num_ctas", 296)
+    return api.plan_attention(w.cu_q_lens, w.seq_lens, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                              head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal,
+                              block_tables=w.block_tables, pin=False, **kw)
+
+
+def test_plan_rejects(api):
+    w = W.llama3_8b_decode_bf16(batch=3, lo=10, hi=50)
+    with pytest.raises(api.PkvError):
+        api.plan_attention(w.cu_q_lens, w.seq_lens, num_q_heads=30, num_kv_heads=8, head_dim=128, block_size=64,
+                           kv_dtype="bf16", num_ctas=10, pin=False)
+    bad = w.seq_lens.copy()
+    bad[1] = 0  # q_len 1 > seq_len 0
+    with pytest.raises(api.PkvError):
+        api.plan_attention(w.cu_q_lens, bad, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=64,
+                           kv_dtype="bf16", num_ctas=10, pin=False)
+    with pytest.raises(api.PkvError):  # table row too short for the length
+        api.plan_attention(w.cu_q_lens, w.seq_lens * 100, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                           block_size=64, kv_dtype="bf16", num_ctas=10, max_blocks=1, pin=False)
+
+
+CASES = [
+    ("decode", lambda: W.llama3_8b_decode_bf16(batch=40, lo=1, hi=5000), {}),
+    ("decode_nosplit", lambda: W.llama3_8b_decode_bf16(batch=9, lo=1, hi=900), {"kv_split": -1}),
+    ("decode_split64", lambda: W.llama3_8b_decode_bf16(batch=9, lo=1, hi=900), {"kv_split": 64}),
+    ("mixed", lambda: W.mixed_bf16(n_decode=30, n_prefill=3, chunk=300, block_size=16, cached_lo_blocks=1,
+                                    cached_hi_blocks=40, aligned=False), {}),
+    ("mixed_split", lambda: W.mixed_bf16(n_decode=5, n_prefill=2, chunk=77), {"kv_split": 128}),
+    ("fp8_long", lambda: W.longctx_fp8(batch=2, seq_len=20000), {"num_ctas": 50}),
+    ("prefix", lambda: W.prefix_reuse_bf16(n_req=37, prefix=512, suf_lo=1, suf_hi=300), {}),
+    ("prefix_split", lambda: W.prefix_reuse_bf16(n_req=11, prefix=256, suf_lo=1, suf_hi=30), {"kv_split": 64}),
+    ("prefix_off", lambda: W.prefix_reuse_bf16(n_req=11, prefix=256), {"cascade": False}),
+    ("tiny", lambda: W.tiny_fp32(), {}),
+]
+
+
+@pytest.mark.parametrize("name,make,opts", CASES, ids=[c[0] for c in CASES])
+def test_plan_covers_every_key_once(api, name, make, opts):
+    w = make()
+    p = _plan(api, w, **opts)
+    d = PD.decode(p.buffer)
+    assert d["header"]["n_items"] == p.info["num_items"]
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
+                      w.block_size)
+    if name == "prefix":
+        assert p.info["num_groups"] >= 1
+    if name == "prefix_off":
+        assert p.info["num_groups"] == 0
+
+
+def test_plan_noncausal_and_empty_rows(api):
+    w = W.build("mix", seed=3, kv_dtype="bf16", num_q_heads=16, num_kv_heads=2, head_dim=64, block_size=32,
+                seq_lens=[40, 7, 300, 1, 90], q_lens=[5, 0, 300, 1, 0], causal=False)
+    d = PD.decode(_plan(api, w).buffer)
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, 16, 2, False)
+
+
+def test_plan_empty_batch(api):
+    p = api.plan_attention(np.zeros(1, np.int32), np.zeros(0, np.int32), num_q_heads=8, num_kv_heads=8,
+                           head_dim=64, block_size=16, kv_dtype="f32", num_ctas=4, pin=False)
+    assert p.info["num_items"] == 0
+
+
+def test_plan_balances_decode(api):
+    """The automatic split keeps every item within ~2x the mean share per CTA."""
+    w = W.llama3_8b_decode_bf16()
+    p = _plan(api, w)
+    items = PD.decode(p.buffer)["items"]
+    keys = (items["k_end"] - items["k_begin"]).astype(np.int64)
+    per_cta = keys.sum() / 296
+    assert keys.max() <= max(256, 2 * per_cta / 2 + 64)
+    assert p.info["num_items"] >= 296

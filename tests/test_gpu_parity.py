@@ -1,0 +1,228 @@
+"""CUDA path against the oracle, through the C ABI (needs a B200).
+
+kv_append: the whole pool, byte for byte (sentinel NaNs included).
+paged_attention: element by element within the stated tolerance, plus the
+log-sum-exp, on scaled-down copies of each workload (several tiles, ragged
+tails) and on edge cases; full-size workloads are checked on sampled
+sequences in test_gpu_fullsize.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.pkv_oracle as O
+from gpu_common import TOL, assert_close, gpu_out_f64, oracle_out, oracle_pool
+from paged_kv_attention_block_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from paged_kv_attention_block_b200 import build
+    build.build()
+    from paged_kv_attention_block_b200 import api, runner
+    return api, runner
+
+
+def run_case(pkv, w, check_pool=True, check_lse=True, **plan_opts):
+    api, runner = pkv
+    dw = runner.DeviceWorkload(w)
+    dw.append_new()
+    plan = dw.plan(**plan_opts)
+    lse = torch.full((w.total_q, w.num_q_heads), float("nan"), device="cuda")
+    out = torch.full_like(dw.q, float("nan"))
+    dw.attention(plan, out=out, out_lse=lse)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) == 0
+    pool = oracle_pool(w)
+    if check_pool:
+        got = dw.pool_bytes()
+        if w.kv_dtype == "f32":
+            same = (got.view(np.uint32) == pool.bits.view(np.uint32))
+        else:
+            same = got == pool.bits
+        assert same.all(), f"kv_append: {int((~same).sum())} pool elements differ"
+    ref, ref_lse = oracle_out(w, pool)
+    err = assert_close(gpu_out_f64(out), ref, w.kv_dtype)
+    if check_lse:
+        lse_err = np.abs(lse.cpu().numpy() - ref_lse).max()
+        assert lse_err <= (1e-5 if w.kv_dtype == "f32" else 2e-3), lse_err
+    return plan, err
+
+
+# ---- the five workload shapes, scaled down -------------------------------
+
+def test_tiny_fp32_exact_config(pkv):
+    run_case(pkv, W.tiny_fp32())
+
+
+def test_tiny_fp32_lengths_before_append_reading(pkv):
+    # The other reading of the tiny config: the listed lengths are the cached
+    # lengths before the appended token.
+    run_case(pkv, W.tiny_fp32(seq_lens=(18, 65, 101, 201)))
+
+
+@pytest.mark.parametrize("split", [0, -1, 64, 192])
+def test_decode_bf16(pkv, split):
+    run_case(pkv, W.llama3_8b_decode_bf16(batch=7, lo=1, hi=1500), kv_split=split, num_ctas=40)
+
+
+@pytest.mark.parametrize("aligned", [True, False])
+def test_mixed_bf16(pkv, aligned):
+    w = W.mixed_bf16(n_decode=9, n_prefill=3, chunk=200, dec_lo=1, dec_hi=1200, cached_lo_blocks=1,
+                     cached_hi_blocks=6, aligned=aligned)
+    run_case(pkv, w, num_ctas=60)
+
+
+def test_mixed_bf16_split_prefill(pkv):
+    w = W.mixed_bf16(n_decode=4, n_prefill=2, chunk=150, dec_lo=100, dec_hi=900, cached_lo_blocks=2,
+                     cached_hi_blocks=5, block_size=32)
+    run_case(pkv, w, kv_split=64)
+
+
+def test_noncausal_chunks(pkv):
+    w = W.mixed_bf16(n_decode=3, n_prefill=2, chunk=70, dec_lo=10, dec_hi=400, cached_lo_blocks=1,
+                     cached_hi_blocks=4, block_size=16)
+    w.causal = False
+    run_case(pkv, w)
+
+
+@pytest.mark.parametrize("split", [0, 256])
+def test_longctx_fp8(pkv, split):
+    run_case(pkv, W.longctx_fp8(batch=3, seq_len=3001), kv_split=split, num_ctas=30)
+
+
+@pytest.mark.parametrize("cascade", [True, False])
+def test_prefix_reuse_bf16(pkv, cascade):
+    w = W.prefix_reuse_bf16(n_req=21, prefix=512, suf_lo=1, suf_hi=300)
+    plan, _ = run_case(pkv, w, cascade=cascade)
+    assert (plan.info["num_groups"] > 0) == cascade
+
+
+# ---- shapes and dtypes ----------------------------------------------------
+
+@pytest.mark.parametrize("B", [2, 4, 16, 32, 64, 128, 256])
+@pytest.mark.parametrize("D", [64, 128])
+def test_block_sizes_and_head_dims(pkv, B, D):
+    w = W.build(f"b{B}d{D}", seed=B * 7 + D, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=D,
+                block_size=B, seq_lens=[1, B - 1 if B > 1 else 1, B, B + 1, 3 * B + 5, 700], q_lens=[1, 1, 1, 1, 4, 33])
+    run_case(pkv, w, num_ctas=16)
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 2), (32, 2), (64, 1)])
+def test_gqa_groups(pkv, hq, hkv):
+    w = W.build(f"g{hq}_{hkv}", seed=hq + hkv, kv_dtype="bf16", num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                block_size=64, seq_lens=[300, 65, 1000, 64], q_lens=[1, 1, 20, 64])
+    run_case(pkv, w, num_ctas=32)
+
+
+@pytest.mark.parametrize("kv,qd", [("f16", "f16"), ("e4m3", "f16"), ("e4m3", "bf16"), ("f32", "f32")])
+@pytest.mark.parametrize("D", [64, 128])
+def test_dtypes(pkv, kv, qd, D):
+    w = W.build(f"{kv}{qd}{D}", seed=D + len(kv), kv_dtype=kv, q_dtype=qd, num_q_heads=16, num_kv_heads=4, head_dim=D,
+                block_size=16, seq_lens=[5, 130, 777, 40], q_lens=[1, 1, 9, 40])
+    run_case(pkv, w, num_ctas=24)
+
+
+def test_fp8_from_bf16_values(pkv):
+    w = W.build("e4m3_bf16in", seed=11, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="bf16", num_q_heads=8,
+                num_kv_heads=2, head_dim=128, block_size=32, seq_lens=[100, 1], q_lens=[1, 1], data_scale=3.0)
+    run_case(pkv, w)
+
+
+# ---- edge cases -------------------------------------------------------------
+
+def test_unscheduled_and_single_token_sequences(pkv):
+    w = W.build("edge", seed=5, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                seq_lens=[1, 50, 9, 1, 17], q_lens=[1, 0, 9, 0, 1])
+    run_case(pkv, w)
+
+
+def test_empty_batch(pkv):
+    api, runner = pkv
+    w = W.build("empty", seed=1, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+                seq_lens=[5], q_lens=[0])
+    dw = runner.DeviceWorkload(w)
+    plan = dw.plan()
+    assert plan.info["num_items"] == 0
+    dw.attention(plan, out=torch.empty(0, 8, 64, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+
+
+def test_large_logits_stay_finite(pkv):
+    w = W.build("big", seed=9, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=64,
+                seq_lens=[500, 90], q_lens=[1, 30], data_scale=8.0)
+    run_case(pkv, w)
+
+
+def test_split_reduce_dense(pkv):
+    api, _ = pkv
+    r = np.random.default_rng(4)
+    n, rows, d = 5, 37, 128
+    po = r.standard_normal((n, rows, d)).astype(np.float32)
+    pl = (r.standard_normal((n, rows)) * 3).astype(np.float32)
+    pl[1, :] = -np.inf
+    pl[:, 3] = -np.inf  # a row with no keys at all
+    o_ref, l_ref = O.split_kv_reduce(po, pl)
+    for dt, tol in ((torch.float32, 1e-6), (torch.bfloat16, 8e-3)):
+        lse = torch.empty(rows, device="cuda")
+        out, _ = api.split_kv_reduce(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda(), out_dtype=dt,
+                                     out_lse=lse)
+        torch.cuda.synchronize()
+        got = out.float().cpu().numpy()
+        assert np.abs(got - o_ref).max() <= tol * max(1.0, np.abs(o_ref).max())
+        gl = lse.cpu().numpy()
+        assert np.isneginf(gl[3]) and np.abs(gl[np.isfinite(l_ref)] - l_ref[np.isfinite(l_ref)]).max() <= 1e-5
+
+
+# ---- errors reported on the device -------------------------------------------
+
+def test_bad_block_id_is_reported_not_faulted(pkv):
+    api, runner = pkv
+    w = W.build("badbt", seed=2, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                seq_lens=[40, 40], q_lens=[1, 1])
+    dw = runner.DeviceWorkload(w)
+    before = dw.cache.pool.clone()
+    bt = dw.block_tables.clone()
+    bt[1, 2] = w.num_blocks + 1000  # corrupt the table on the host side of the call
+    api.kv_append(dw.cache, dw.k_new, dw.v_new, dw.cu_q, dw.start_pos, bt, status=dw.status)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) & 0x1
+    # Sequence 0 was written, the row aimed at the bad block was not; nothing else changed.
+    changed = (dw.cache.pool.view(torch.int16) != before.view(torch.int16)).any(dim=(1, 2, 3, 4, 5))
+    assert int(changed.sum()) == 1
+    dw.status.zero_()
+    plan = dw.plan()
+    out = torch.zeros_like(dw.q)
+    api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, bt, plan, w.softmax_scale, True, out=out,
+                        status=dw.status)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) & 0x1
+
+
+def test_plan_mismatch_is_reported(pkv):
+    api, runner = pkv
+    w = W.build("mism", seed=3, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+                seq_lens=[40, 70], q_lens=[1, 1])
+    dw = runner.DeviceWorkload(w)
+    plan = dw.plan()
+    short = dw.seq_lens.clone()
+    short[1] = 10  # device lengths no longer match the plan
+    api.paged_attention(dw.cache, dw.q, dw.cu_q, short, dw.block_tables, plan, w.softmax_scale, True,
+                        status=dw.status)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) & 0x4
+
+
+def test_repeat_launch_is_deterministic(pkv):
+    api, runner = pkv
+    w = W.llama3_8b_decode_bf16(batch=5, lo=100, hi=3000)
+    dw = runner.DeviceWorkload(w)
+    dw.append_new()
+    plan = dw.plan(num_ctas=20)
+    a = dw.attention(plan).clone()
+    b = dw.attention(plan).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
