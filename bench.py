@@ -218,6 +218,17 @@ def run_reference(args, rank: int, world: int):
 # The CUDA path
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank values (device time: the slowest replica sets the step time)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
 def run_pkv(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -279,10 +290,7 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     attn_ms = [a.elapsed_time(e[1]) for a, e in zip(attn_ev, ev)]
     ms = float(np.mean(step_ms))
     attn = float(np.mean(attn_ms))
-    if world > 1:
-        t = torch.tensor([ms, attn], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, attn = float(t[0]), float(t[1])
+    ms, attn = max_over_ranks([ms, attn], dev)
     assert int(dw.status.item()) == 0, "device status set during the benchmark"
 
     b = algorithmic_bytes(w, plan.info)
@@ -292,10 +300,7 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
 
     # End to end through the public API from pinned host buffers.
     e2e = run_e2e(args, w, dw, plan_opts, dev, stream, api)
-    if world > 1:
-        t = torch.tensor([e2e["ms"]], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms"] = float(t[0])
+    e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
 
     launches_per_step = 2 + (1 if plan.info["num_reduce"] > 0 else 0)
     if rank == 0:
