@@ -245,6 +245,32 @@ PKV_API pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q, in
 PKV_API pkv_status pkv_split_kv_reduce(const float* partial_o, const float* partial_lse, int32_t n_split, int64_t rows,
                                int32_t head_dim, void* out, int32_t out_dtype, float* out_lse, void* stream);
 
+/*
+ * paged_attention_noalloc - paged_attention for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call; it exists for callers that are
+ * handed only input and output buffers and may not allocate device memory
+ * themselves (a plug-in inside a host framework, an allocator-free runtime, or
+ * code whose device memory budget is fixed before it runs).  Arguments and
+ * results are those of pkv_paged_attention without the workspace: the scratch
+ * (plan copy, work counter, split partials) lives in one device array of
+ * PKV_NOALLOC_SCRATCH_BYTES built into the library, which every GPU that loads
+ * the library holds until the process exits.
+ *   - A plan needing more scratch than that returns PKV_ERR_WORKSPACE.
+ *   - The first call on a device looks up the array's address on that device;
+ *     make it outside any stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents (the counter is cleared on the stream by each call).  Calls that
+ *     overlap on the GPU race; order them on one stream.
+ *   - Allocates and frees nothing.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (32ull << 20)
+PKV_API pkv_status pkv_paged_attention_noalloc(const pkv_cache* cache, const void* q, int32_t q_dtype,
+                                       int32_t num_q_heads, const int32_t* cu_q_lens, const int32_t* seq_lens,
+                                       const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                       float softmax_scale, int32_t causal, const void* plan, void* out,
+                                       float* out_lse, int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,6 +77,9 @@ _lib.pkv_default_num_ctas.argtypes = [_I32, _I32, C.POINTER(_I32)]
 _lib.pkv_paged_attention.restype = _I32
 _lib.pkv_paged_attention.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P, _P, _P,
                                      _P, _SZ, _P, _P]
+_lib.pkv_paged_attention_noalloc.restype = _I32
+_lib.pkv_paged_attention_noalloc.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P,
+                                             _P, _P, _P, _P]
 _lib.pkv_split_kv_reduce.restype = _I32
 _lib.pkv_split_kv_reduce.argtypes = [_P, _P, _I32, _I64, _I32, _P, _I32, _P, _P]
 
@@ -224,6 +227,27 @@ def paged_attention(cache: Cache, q: torch.Tensor, cu_q_lens: torch.Tensor, seq_
                                     int(bool(causal)), plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse),
                                     _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
            "paged_attention")
+    return out
+
+
+def paged_attention_noalloc(cache: Cache, q: torch.Tensor, cu_q_lens: torch.Tensor, seq_lens: torch.Tensor,
+                            block_tables: torch.Tensor, plan: Plan, softmax_scale: float, causal: bool = True,
+                            out: torch.Tensor | None = None, out_lse: torch.Tensor | None = None,
+                            status: torch.Tensor | None = None, stream=None):
+    """paged_attention using the library's built-in scratch array instead of a workspace.
+
+    For callers that may not allocate device memory; see pkv_paged_attention_noalloc
+    in include/pkv.h for the size limit and the sharing rules.  ``out`` must be
+    given by such callers (a default is allocated here only for convenience).
+    """
+    if out is None:
+        out = torch.empty_like(q)
+    c = cache._c()
+    _check(_lib.pkv_paged_attention_noalloc(C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens),
+                                            _ptr(seq_lens), _ptr(block_tables), block_tables.shape[1],
+                                            seq_lens.shape[0], float(softmax_scale), int(bool(causal)),
+                                            plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse), _ptr(status),
+                                            _stream(stream)), "paged_attention_noalloc")
     return out
 
 
