@@ -7,7 +7,7 @@ step's new tokens, host planning of the launch, and paged_attention (persistent
 attention kernel plus the merge of split key ranges).  The default workload is
 the Llama-3-8B-shaped decode batch (64 sequences, lengths U[512, 4096], 32/8
 heads, head_dim 128, block 64, bf16 KV).  The pool (~755 MB) is larger than L2
-and L2 is also flushed (a 512 MB write) before every timed step.
+and L2 is also flushed (a 512 MB read) before every timed step.
 
 Prints ONE JSON line (rank 0).  Under torchrun every rank runs an independent
 replica on its own GPU (the path has no exchange step); time is the max over
@@ -89,6 +89,9 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
+            t0 = time.time()  # start timing only once sampling has begun
+            while time.time() - t0 < 10 and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+                time.sleep(0.05)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -126,10 +129,13 @@ class ClockSampler:
 
 
 def kernel_source_hash() -> str:
+    """Hash of every kernel source: a traffic figure is reported only for the sources it was taken on."""
     h = hashlib.sha256()
-    for name in ("attn_mma.cu", "common.cuh", "plan_format.h"):
-        with open(os.path.join(ROOT, "paged_kv_attention_block_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+    csrc = os.path.join(ROOT, "paged_kv_attention_block_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -246,52 +252,83 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     plan_opts = {}
     if args.kv_split:
         plan_opts["kv_split"] = args.kv_split
-    plan = dw.plan(**plan_opts)
+    plan_kw = dict(num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                   block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal, block_tables=w.block_tables,
+                   **plan_opts)
+    plan = api.plan_attention(w.cu_q_lens, w.seq_lens, **plan_kw)
     ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
     out = torch.empty_like(dw.q)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    # L2 is flushed before each step by reading a 512 MB buffer: the KV leaves L2 and the lines
+    # left behind are clean, so no write-back of the flush lands in the timed region.
+    flush = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
 
-    def step():
+    # The GPU side of a step runs from CUDA graphs: one for kv_append and one attention graph per
+    # page-locked plan buffer (double-buffered), so the events below time GPU work only.  The host
+    # plans every step into the buffer whose previous upload has completed.
+    bufs = [api.plan_attention(w.cu_q_lens, w.seq_lens, **plan_kw) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):  # eager warm-up: occupancy queries, tensor-map encoder lookup
+            dw.append_new()
+            api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, bufs[0], w.softmax_scale,
+                                w.causal, out=out, workspace=ws, status=dw.status)
+    torch.cuda.synchronize(dev)
+    g_append = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_append, stream=stream):
         dw.append_new()
-        p = dw.plan(**plan_opts)
-        ev_a = torch.cuda.Event(enable_timing=True)
-        ev_a.record(stream)
-        dw.attention(p, out=out, workspace=ws)
-        return p, ev_a
+    g_attn = []
+    for b in bufs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale, w.causal,
+                                out=out, workspace=ws, status=dw.status)
+        g_attn.append(g)
+    done = [None, None]
+    host_plan_s = 0.0
 
-    for _ in range(max(3, args.warmup)):
-        flush.fill_(1)
-        step()
+    def step(i, evs=None):
+        nonlocal host_plan_s
+        slot = i % 2
+        if done[slot] is not None:
+            done[slot].synchronize()  # the upload that read this buffer has run
+        t0 = time.perf_counter()
+        api.plan_attention(w.cu_q_lens, w.seq_lens, buffer=bufs[slot].buffer, **plan_kw)
+        host_plan_s += time.perf_counter() - t0
+        with torch.cuda.stream(stream):
+            flush.sum()
+            if evs:
+                evs[0].record(stream)
+            g_append.replay()
+            if evs:
+                evs[1].record(stream)
+            g_attn[slot].replay()
+            if evs:
+                evs[2].record(stream)
+            e = torch.cuda.Event()
+            e.record(stream)
+            done[slot] = e
+
+    for i in range(max(3, args.warmup)):
+        step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    attn_ev = []
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     host_plan_s = 0.0
     with ClockSampler(local_rank) as clocks:
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
-            flush.fill_(1)
-            ev[i][0].record(stream)
-            dw.append_new()
-            t0 = time.perf_counter()
-            p = dw.plan(**plan_opts)
-            host_plan_s += time.perf_counter() - t0
-            a0 = torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            dw.attention(p, out=out, workspace=ws)
-            ev[i][1].record(stream)
-            attn_ev.append(a0)
+            step(i, ev[i])
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in ev]
-    attn_ms = [a.elapsed_time(e[1]) for a, e in zip(attn_ev, ev)]
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
     ms = float(np.mean(step_ms))
     attn = float(np.mean(attn_ms))
     ms, attn = max_over_ranks([ms, attn], dev)
     assert int(dw.status.item()) == 0, "device status set during the benchmark"
+    del g_append, g_attn
 
     b = algorithmic_bytes(w, plan.info)
     value = b["step"] * world / (ms * 1e-3) / 1e9
@@ -299,7 +336,7 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     peak, peak_kind = peaks()
 
     # End to end through the public API from pinned host buffers.
-    e2e = run_e2e(args, w, dw, plan_opts, dev, stream, api)
+    e2e = run_e2e(args, w, dw, plan_opts, dev, torch.cuda.current_stream(dev), api)
     e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
 
     launches_per_step = 2 + (1 if plan.info["num_reduce"] > 0 else 0)
@@ -311,7 +348,8 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": w.num_seqs, "kv_tokens": int(w.seq_lens.sum()),
                        "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                       "block_size": w.block_size, "l2": "flushed before every step (512 MB write); pool > L2",
+                       "block_size": w.block_size,
+                       "l2": "flushed before every step by reading a 512 MB buffer; pool larger than L2",
                        "parallelism": f"replicas{world}"},
             "decode_tok_s": decode_rows(w) * world / (ms * 1e-3),
             "hbm_frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
@@ -320,7 +358,7 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             "attention_ms": attn, "host_plan_us": host_plan_s / args.steps * 1e6,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic_for(w.name), "peak_source": peak_kind,
-                         "kernel": "attn_mma_kernel (+ plan upload and split merge in the timed call)"},
+                         "kernel": "attn_tma_kernel (the timed call also uploads the plan and runs the split merge)"},
             "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
             "e2e": {"value": b["step"] * world / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms"]},
@@ -349,14 +387,14 @@ def run_e2e(args, w, dw, plan_opts, dev, stream, api):
                                   block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal, block_tables=bt,
                                   **plan_opts)
 
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.ones(128 << 20, dtype=torch.float32, device=dev)
     for _ in range(3):
         api.decode_step_e2e(dw.cache, host, devb, plan_fn, w.softmax_scale, w.causal)
     torch.cuda.synchronize(dev)
     n = max(1, min(args.steps, 200))
     tot = 0.0
     for _ in range(n):
-        flush.fill_(1)
+        flush.sum()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record(stream)
         p = api.decode_step_e2e(dw.cache, host, devb, plan_fn, w.softmax_scale, w.causal)
@@ -371,7 +409,7 @@ def run_e2e(args, w, dw, plan_opts, dev, stream, api):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--config", default="llama3_8b_decode_bf16")

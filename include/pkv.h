@@ -79,6 +79,7 @@ typedef enum pkv_dtype {
 #define PKV_DEV_BAD_LOGICAL_BLOCK 0x2 /* position needs a table entry beyond max_blocks */
 #define PKV_DEV_PLAN_MISMATCH 0x4     /* plan item does not fit the device lengths */
 #define PKV_DEV_BAD_APPEND 0x8        /* kv_append position negative */
+#define PKV_DEV_TIMEOUT 0x10          /* an internal pipeline wait gave up (about 1 s); results incomplete */
 
 /* One layer's view of a paged pool (deep dive §9: one block holds a fixed number
  * of tokens' KV; several layers may be packed in one block). */
@@ -151,7 +152,8 @@ typedef struct pkv_plan_request {
   int32_t block_size;           /* power of two >= 2 */
   int32_t kv_dtype;             /* pkv_dtype of the pool */
   int32_t causal;               /* 0 or 1 */
-  int32_t num_ctas;             /* CTAs the launch keeps resident; 0 = ask the current device */
+  int32_t num_ctas;             /* CTAs the launch uses (capped at what fits resident); 0 = all that
+                                   fit on the current device */
   int32_t kv_split;             /* 0 = automatic split of long key ranges; >0 = max keys per work
                                    item (rounded up to 64); <0 = never split */
   int32_t cascade;              /* nonzero: group consecutive sequences whose tables share leading
@@ -193,9 +195,9 @@ typedef struct pkv_plan_info {
  */
 PKV_API pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan, size_t capacity, pkv_plan_info* info);
 
-/* CTAs per launch the attention kernel keeps resident on the current device
- * for this pool dtype and head_dim (SM count x occupancy). */
-PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int32_t* num_ctas);
+/* CTAs the attention kernel for this pool dtype, head_dim and block size keeps
+ * resident on the current device (SM count x occupancy). */
+PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int32_t block_size, int32_t* num_ctas);
 
 /*
  * paged_attention - out = softmax(scale * q K^T) V over each sequence's paged K/V.
@@ -210,7 +212,8 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  *   BF16 (BF16 or FP8 pools) or F16 (F16 or FP8 pools).  total_q = cu_q_lens[num_seqs].
  * cu_q_lens, seq_lens: device int32 copies of the arrays the plan was made from.
  * block_tables: device int32 [num_seqs][max_blocks].
- * softmax_scale: scale on q.k (typically 1/sqrt(head_dim)); causal as planned.
+ * softmax_scale: scale on q.k (typically 1/sqrt(head_dim)), positive and finite;
+ *   causal as planned.  fp8 scales must be positive.
  * plan: host buffer from pkv_attention_plan for these shapes.  It is copied to
  *   the workspace with cudaMemcpyAsync; use page-locked memory for an
  *   asynchronous copy and keep it unchanged until the copy has run.

@@ -73,7 +73,7 @@ _lib.pkv_kv_append.argtypes = [C.POINTER(_Cache), _P, _P, _I32, _P, _P, _P, _I32
 _lib.pkv_attention_plan.restype = _I32
 _lib.pkv_attention_plan.argtypes = [C.POINTER(_PlanRequest), _P, _SZ, C.POINTER(_PlanInfo)]
 _lib.pkv_default_num_ctas.restype = _I32
-_lib.pkv_default_num_ctas.argtypes = [_I32, _I32, C.POINTER(_I32)]
+_lib.pkv_default_num_ctas.argtypes = [_I32, _I32, _I32, C.POINTER(_I32)]
 _lib.pkv_paged_attention.restype = _I32
 _lib.pkv_paged_attention.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P, _P, _P,
                                      _P, _SZ, _P, _P]
@@ -183,8 +183,12 @@ def _host_i32(x) -> np.ndarray:
 def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
                    kv_dtype: int | str, causal: bool = True, block_tables=None, max_blocks: int | None = None,
                    num_ctas: int = 0, kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0,
-                   pin: bool = True) -> Plan:
-    """Build the work list for one paged_attention call from host copies of the lengths."""
+                   pin: bool = True, buffer: torch.Tensor | None = None) -> Plan:
+    """Build the work list for one paged_attention call from host copies of the lengths.
+
+    ``buffer`` (uint8, host) is reused when large enough; the caller must not
+    reuse a buffer whose plan upload may still be pending on the GPU.
+    """
     cu = _host_i32(cu_q_lens)
     sl = _host_i32(seq_lens)
     bt = None if block_tables is None else _host_i32(block_tables)
@@ -196,7 +200,10 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
                        None if bt is None else bt.ctypes.data)
     info = _PlanInfo()
     _check(_lib.pkv_attention_plan(C.byref(req), None, 0, C.byref(info)), "attention_plan")
-    buf = torch.empty(int(info.plan_bytes), dtype=torch.uint8, pin_memory=pin and torch.cuda.is_available())
+    if buffer is not None and buffer.numel() >= int(info.plan_bytes):
+        buf = buffer
+    else:
+        buf = torch.empty(int(info.plan_bytes), dtype=torch.uint8, pin_memory=pin and torch.cuda.is_available())
     _check(_lib.pkv_attention_plan(C.byref(req), buf.data_ptr(), buf.numel(), C.byref(info)), "attention_plan")
     return Plan(buf, {f: getattr(info, f) for f, _ in _PlanInfo._fields_})
 
@@ -205,10 +212,10 @@ def attention_workspace_bytes(plan: Plan) -> int:
     return plan.workspace_bytes
 
 
-def default_num_ctas(kv_dtype: int | str, head_dim: int) -> int:
+def default_num_ctas(kv_dtype: int | str, head_dim: int, block_size: int) -> int:
     code = DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
     n = C.c_int32(0)
-    _check(_lib.pkv_default_num_ctas(code, head_dim, C.byref(n)), "default_num_ctas")
+    _check(_lib.pkv_default_num_ctas(code, head_dim, block_size, C.byref(n)), "default_num_ctas")
     return n.value
 
 

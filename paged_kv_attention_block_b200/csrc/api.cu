@@ -6,6 +6,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
+#include <mutex>
 
 #include "attn_args.h"
 #include "internal.h"
@@ -39,20 +41,37 @@ extern "C" const char* pkv_status_string(int32_t status) {
 
 extern "C" const char* pkv_last_error(void) { return g_last_error; }
 
-extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int32_t* num_ctas) {
-  if (!num_ctas) return pkv_fail(PKV_ERR_INVALID_ARG, "default_num_ctas: null output");
-  pkv::AttnKernel k;
-  const int q_dtype = kv_dtype == PKV_F32 ? PKV_F32 : (kv_dtype == PKV_F16 ? PKV_F16 : PKV_BF16);
-  if (!pkv::attn_kernel_for(kv_dtype, q_dtype, head_dim, &k))
-    return pkv_fail(PKV_ERR_UNSUPPORTED, "default_num_ctas: no kernel for kv_dtype %d head_dim %d", kv_dtype, head_dim);
-  int dev = 0, sms = 0, per_sm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+namespace pkv {
+// SM count x occupancy, cached per (device, kernel).
+int resident_ctas(const AttnKernel& k) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({dev, k.fn});
+  if (it != cache.end()) return it->second;
+  int sms = 0, per_sm = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess && k.smem > 48 * 1024)
     e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
   if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, k.smem);
-  if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "default_num_ctas: %s", cudaGetErrorString(e));
-  *num_ctas = std::max(1, sms * std::max(1, per_sm));
+  if (e != cudaSuccess) return -1;
+  const int n = std::max(1, sms * std::max(1, per_sm));
+  cache[{dev, k.fn}] = n;
+  return n;
+}
+}  // namespace pkv
+
+extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int32_t block_size, int32_t* num_ctas) {
+  if (!num_ctas) return pkv_fail(PKV_ERR_INVALID_ARG, "default_num_ctas: null output");
+  pkv::AttnKernel k;
+  const int q_dtype = kv_dtype == PKV_F32 ? PKV_F32 : (kv_dtype == PKV_F16 ? PKV_F16 : PKV_BF16);
+  if (!pkv::attn_kernel_for(kv_dtype, q_dtype, head_dim, block_size, &k))
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "default_num_ctas: no kernel for kv_dtype %d head_dim %d", kv_dtype, head_dim);
+  const int n = pkv::resident_ctas(k);
+  if (n <= 0) return pkv_fail(PKV_ERR_CUDA, "default_num_ctas: occupancy query failed: %s", cudaGetErrorString(cudaGetLastError()));
+  *num_ctas = n;
   return PKV_OK;
 }
 
@@ -115,11 +134,13 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
       h->causal != (causal ? 1 : 0))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan was made for other shapes");
   pkv::AttnKernel k;
-  if (!pkv::attn_kernel_for(c.kv_dtype, q_dtype, c.head_dim, &k))
+  if (!pkv::attn_kernel_for(c.kv_dtype, q_dtype, c.head_dim, c.block_size, &k))
     return pkv_fail(PKV_ERR_UNSUPPORTED, "paged_attention: kv_dtype %d with q_dtype %d, head_dim %d", c.kv_dtype,
                     q_dtype, c.head_dim);
   if (c.kv_dtype == PKV_FP8_E4M3 && (!c.k_scale || !c.v_scale))
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: fp8 pool needs k_scale and v_scale");
+  if (!(softmax_scale > 0.f) || softmax_scale == INFINITY)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: softmax_scale must be positive and finite");
   if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads); vs != PKV_OK) return vs;
   const PkvWorkspaceLayout L = pkv_workspace_layout(h->bytes, h->n_part_rows, c.head_dim);
   if (h->n_items == 0) return PKV_OK;
@@ -135,12 +156,10 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemcpyAsync(ws + L.plan_off, plan, h->bytes, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.counter_off, 0, 256, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.counter_off, 0, L.counter_bytes, st);
   if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: plan upload: %s", cudaGetErrorString(e));
-  if (k.smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
-    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: %s", cudaGetErrorString(e));
-  }
+  const int resident = pkv::resident_ctas(k);  // also sets the kernel's shared-memory limit
+  if (resident <= 0) return pkv_fail(PKV_ERR_CUDA, "paged_attention: occupancy query failed");
   const char* dplan = ws + L.plan_off;
   pkv::AttnArgs a{};
   a.pool = c.pool;
@@ -168,9 +187,8 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
   a.part_o = reinterpret_cast<float*>(ws + L.part_o_off);
   a.part_lse = reinterpret_cast<float*>(ws + L.part_lse_off);
   a.status = dev_status;
-  const int grid = std::max(1, std::min(h->num_ctas, h->n_items));
-  k.launch(a, grid, st);
-  e = cudaGetLastError();
+  const int grid = std::max(1, std::min(std::min(resident, h->num_ctas), h->n_items));
+  e = k.launch(a, grid, st);
   if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: launch failed: %s", cudaGetErrorString(e));
   if (h->n_reduce > 0) {
     pkv::ReduceArgs r{};

@@ -45,9 +45,14 @@ struct AttnKernel {
   const void* fn;
   int threads;
   int smem;
-  void (*launch)(const AttnArgs&, int grid, cudaStream_t);
+  cudaError_t (*launch)(const AttnArgs&, int grid, cudaStream_t);
 };
-bool attn_kernel_for(int kv_dtype, int q_dtype, int head_dim, AttnKernel* k);
+// Picks the TMA kernel where it applies (block size >= 8, 128/256-byte rows),
+// else the cp.async tensor-core kernel, and the CUDA-core kernel for fp32 pools.
+bool attn_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
+bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
+// SM count x occupancy of a kernel on the current device (cached per device).
+int resident_ctas(const AttnKernel& k);
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st);
 
 }  // namespace pkv

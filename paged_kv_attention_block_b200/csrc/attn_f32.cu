@@ -98,8 +98,9 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
 }
 
 template <int D>
-void launch_f32(const AttnArgs& a, int grid, cudaStream_t st) {
+cudaError_t launch_f32(const AttnArgs& a, int grid, cudaStream_t st) {
   attn_f32_kernel<D><<<grid, 128, 0, st>>>(a);
+  return cudaGetLastError();
 }
 
 AttnKernel f32_kernel(int head_dim) {

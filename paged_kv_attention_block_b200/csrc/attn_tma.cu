@@ -1,0 +1,746 @@
+// Paged attention, TMA-fed and warp-specialised (bf16 / f16 / fp8-e4m3 pools,
+// block size >= 8, 128- or 256-byte K/V rows).
+//
+// Same work list and results as attn_mma.cu (deep dive, gentlecold.top: §2
+// decode reads all history KV, §6 one launch for a packed mix of prefill and
+// decode requests, §8 causal chunks, §9 block pool and block tables); the data
+// movement and the decode arithmetic are reorganised for sm_100a:
+//
+//   * Two persistent CTAs per SM: warp 4 is the producer, warps 0-3 consume.
+//     The producer pulls items from the atomic counter (one item ahead),
+//     publishes each item in a 4-slot descriptor ring, and streams the item's
+//     K/V tiles (TK keys: 32 for 256-byte rows, 64 for 128-byte rows) into an
+//     NST-stage shared-memory ring with 5-D TMA loads, 128-byte swizzle,
+//     completion counted on an mbarrier.  Block ids arrive 32 at a time through
+//     shared memory; when a tile lies inside one pool block a single box covers
+//     its K and V rows (they are neighbours on the pool's K|V axis).  The
+//     producer runs ahead across item boundaries, so the HBM queue does not
+//     drain between items.  No load uses cluster multicast.
+//   * Decode items (<= 16 rows): one consumer warp owns a whole tile (tiles go
+//     round-robin over the 4 warps by tile index) and computes S^T = K Q^T and
+//     O^T = V^T P^T, so the keys fill the 16-row MMA dimension and the
+//     query-head group (g = 4 or 8 rows) fills n = 8.  P^T reaches the second
+//     MMA through movmatrix.  Fragment addresses are fixed per lane; masking
+//     runs only on tiles that reach past a row's limit.  The four warps merge
+//     their softmax states at the end of the item.
+//   * Prefill tiles (> 16 rows): every warp reads every tile and owns 16 rows
+//     (the row-split step of attn_tile.cuh).
+//   * Keys past the item's end inside the last tile are masked; their V rows
+//     are zeroed in shared memory before the P V product (0 * NaN would leak).
+//   * Every wait on an mbarrier is bounded; on a timeout the CTA records
+//     PKV_DEV_TIMEOUT, stops issuing work and waits (bounded) for the loads it
+//     has in flight before exiting.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "attn_args.h"
+#include "attn_tile.cuh"
+#include "common.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+template <int D, int KV, bool QBF>
+struct TmaCfg {
+  using L = Cfg<D, KV, QBF>;
+  static constexpr int ELEM = L::ELEM;
+  static constexpr int RB = L::RB;
+  // Keys per tile: 32 for 256-byte rows, 64 for 128-byte rows (16 KB stages).
+  static constexpr int TK = RB == 256 ? 32 : 64;
+  static constexpr int HALVES = RB / 128;  // 128-byte column slabs per row
+  // Stage layout: [slab][K|V][TK rows][128 B]; K tile at +0, V tile at +TK*128.
+  static constexpr int SLAB = 2 * TK * 128;
+  static constexpr int TILE_BYTES = TK * RB;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  // A multiple of 4: decode tiles go round-robin to the 4 consumer warps by tile
+  // index within the item, so within an item every tile that lands in a given
+  // stage belongs to the same warp and the stage's phases are consumed in order;
+  // across items, the end-of-item merge barrier (decode) or every warp reading
+  // every tile (prefill) orders them.
+  // Four 16 KB stages (64 KB) leave room for two CTAs per SM: twice the producers and consumer
+  // warps of one large-ring CTA, which measured faster than a 12-stage ring with one CTA per SM.
+  static constexpr int NST = 4 * std::max(1, std::min(12, (64 * 1024) / STAGE_BYTES) / 4);
+  static constexpr int IR = 4;  // item descriptor slots
+  static constexpr int MERGE_BYTES = 4 * 16 * D * 4 + 2 * 4 * 16 * 4;
+  static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * IR + 1);
+  static constexpr int DESC_BYTES = IR * 64;
+  static constexpr int IDS_BYTES = 32 * 4;
+  static constexpr int SMEM = 1024 + NST * STAGE_BYTES + MERGE_BYTES + BAR_BYTES + DESC_BYTES + IDS_BYTES + 16;
+  static constexpr int THREADS = 160;
+  static_assert(RB == 128 || RB == 256, "TMA path takes 128- or 256-byte rows");
+  static_assert(NST % 4 == 0, "stage count must be a multiple of the consumer warp count");
+  static_assert(2 * SMEM <= 228 * 1024, "two CTAs per SM");
+};
+
+struct ItemDesc {
+  int seq, kv_head, q_begin, n_q, k_begin, k_end, pos0, part_row, ntiles, state;  // state: 0 run, 1 skip, 2 end
+  int pad[6];
+};
+static_assert(sizeof(ItemDesc) == 64, "descriptor slot");
+
+struct TmaArgs {
+  AttnArgs a;
+  int32_t box_rows;  // rows per TMA box: TK when a tile lies inside one block, else the block size
+  int32_t merged;    // 1: one box covers the K and V rows of a tile
+};
+
+// ---- decode-mode per-warp state (S^T / O^T formulation) -------------------
+template <int D, int KV, bool QBF, int NR>
+struct DecState {
+  float acc[NR][D / 16][4];  // O^T fragments: [row group][d m-tile][frag]
+  float m[NR][2], l[NR][2];  // rows 2*t4 + b (+8*group); m in scaled-log2 units
+  uint32_t qb[NR][D / 16][2];
+  int lim[NR][2];
+};
+
+template <int KV>
+PKV_DEVICE int dec_dim(int mt, int e, int g4) {
+  if constexpr (KV == KV_E4M3) return 32 * (mt >> 1) + 2 * g4 + 16 * (e >> 1) + (mt & 1);
+  else return 16 * mt + g4 + 8 * (e >> 1);
+}
+
+// Per-lane shared-memory offsets of the K (A operand) and V (A^T operand)
+// fragments for rows 0..15 of a tile; rows 16 further down add 16 * 128 bytes
+// (the swizzle phase repeats every 8 rows).
+template <int D, int KV, bool QBF>
+struct DecOffsets {
+  static constexpr int N = KV == KV_E4M3 ? D / 32 : D / 16;
+  uint32_t k[N], v[N];
+};
+
+template <int D, int KV, bool QBF>
+PKV_DEVICE void dec_offsets(DecOffsets<D, KV, QBF>& o, int lane) {
+  using T = TmaCfg<D, KV, QBF>;
+  const int mi = lane >> 3, r8 = lane & 7;
+#pragma unroll
+  for (int i = 0; i < DecOffsets<D, KV, QBF>::N; ++i) {
+    if constexpr (KV == KV_E4M3) {
+      o.k[i] = tile_offset<T::RB, T::TK, T::SLAB>((mi & 1) * 8 + r8, 32 * i + (mi >> 1) * 16);
+      o.v[i] = tile_offset<T::RB, T::TK, T::SLAB>((mi >> 1) * 8 + r8, 32 * i + (mi & 1) * 16);
+    } else {
+      o.k[i] = tile_offset<T::RB, T::TK, T::SLAB>((mi & 1) * 8 + r8, 2 * (16 * i + (mi >> 1) * 8));
+      o.v[i] = tile_offset<T::RB, T::TK, T::SLAB>((mi >> 1) * 8 + r8, 2 * (16 * i + (mi & 1) * 8));
+    }
+  }
+}
+
+template <int D, int KV, bool QBF, int NR>
+PKV_DEVICE void dec_load_q(const AttnArgs& a, const ItemDesc& it, int R, DecState<D, KV, QBF, NR>& st, int g4, int t4) {
+  constexpr bool MMA_BF = KV == KV_BF16;
+#pragma unroll
+  for (int nr = 0; nr < NR; ++nr) {
+    const int r = nr * 8 + g4;
+    const bool valid = r < R;
+    const int64_t token = it.q_begin + (valid ? r / a.g : 0);
+    const int head = it.kv_head * a.g + (valid ? r % a.g : 0);
+    const uint16_t* qrow = static_cast<const uint16_t*>(a.q) + (token * a.hq + head) * D;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t w0 = 0, w1 = 0;
+      if (valid) {
+        if constexpr (KV == KV_E4M3) {  // dims permuted to match the fp8 K fragments
+          const uint2 x = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * t4);
+          w0 = x.x;
+          w1 = x.y;
+        } else {
+          w0 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * t4);
+          w1 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * t4);
+        }
+        if constexpr (!MMA_BF && QBF) {
+          w0 = pack_f16x2(bf16_bits_to_float(uint16_t(w0 & 0xffff)), bf16_bits_to_float(uint16_t(w0 >> 16)));
+          w1 = pack_f16x2(bf16_bits_to_float(uint16_t(w1 & 0xffff)), bf16_bits_to_float(uint16_t(w1 >> 16)));
+        }
+      }
+      st.qb[nr][ks][0] = w0;
+      st.qb[nr][ks][1] = w1;
+    }
+  }
+}
+
+// One tile owned by this warp: S^T = K Q^T, online softmax per query row, O^T += V^T P^T.
+// `masked`: some key of the tile is at or past some row's limit.
+template <int D, int KV, bool QBF, int NR>
+PKV_DEVICE void dec_tile(DecState<D, KV, QBF, NR>& st, const DecOffsets<D, KV, QBF>& off, uint32_t kbase,
+                         uint32_t vbase, int key0, int lane, float c, bool masked) {
+  using T = TmaCfg<D, KV, QBF>;
+  constexpr int NKT = T::TK / 16;
+  constexpr bool MMA_BF = KV == KV_BF16;
+  const int g4 = lane >> 2;
+  float s[NR][NKT][4];
+#pragma unroll
+  for (int kt = 0; kt < NKT; ++kt) {
+#pragma unroll
+    for (int nr = 0; nr < NR; ++nr) s[nr][kt][0] = s[nr][kt][1] = s[nr][kt][2] = s[nr][kt][3] = 0.f;
+    const uint32_t kb = kbase + kt * 16 * 128;
+    if constexpr (KV == KV_E4M3) {
+#pragma unroll
+      for (int kp = 0; kp < D / 32; ++kp) {
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4(kb + off.k[kp], r0, r1, r2, r3);
+        const uint32_t a0[4] = {e4m3x2_to_f16x2(uint16_t(r0 & 0xffff)), e4m3x2_to_f16x2(uint16_t(r1 & 0xffff)),
+                                e4m3x2_to_f16x2(uint16_t(r0 >> 16)), e4m3x2_to_f16x2(uint16_t(r1 >> 16))};
+        const uint32_t a1[4] = {e4m3x2_to_f16x2(uint16_t(r2 & 0xffff)), e4m3x2_to_f16x2(uint16_t(r3 & 0xffff)),
+                                e4m3x2_to_f16x2(uint16_t(r2 >> 16)), e4m3x2_to_f16x2(uint16_t(r3 >> 16))};
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr) {
+          mma16816<false>(s[nr][kt], a0, st.qb[nr][2 * kp][0], st.qb[nr][2 * kp][1]);
+          mma16816<false>(s[nr][kt], a1, st.qb[nr][2 * kp + 1][0], st.qb[nr][2 * kp + 1][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(kb + off.k[ks], a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr) mma16816<MMA_BF>(s[nr][kt], a, st.qb[nr][ks][0], st.qb[nr][ks][1]);
+      }
+    }
+  }
+  if (masked) {
+#pragma unroll
+    for (int nr = 0; nr < NR; ++nr)
+#pragma unroll
+      for (int kt = 0; kt < NKT; ++kt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (key0 + kt * 16 + g4 + 8 * (e >> 1) >= st.lim[nr][e & 1]) s[nr][kt][e] = -INFINITY;
+  }
+  // Running max per query row (in raw score units, then scaled), exp2 of the scaled scores.
+#pragma unroll
+  for (int nr = 0; nr < NR; ++nr) {
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int kt = 0; kt < NKT; ++kt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[e & 1] = fmaxf(mx[e & 1], s[nr][kt][e]);
+    float alpha[2], mneg[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float x = mx[b];
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+      const float mnew = fmaxf(st.m[nr][b], x * c);
+      const float muse = mnew == -INFINITY ? 0.f : mnew;
+      alpha[b] = fast_exp2(st.m[nr][b] - muse);
+      st.m[nr][b] = mnew;
+      mneg[b] = -muse;
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int kt = 0; kt < NKT; ++kt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p = fast_exp2(fmaf(s[nr][kt][e], c, mneg[e & 1]));
+        s[nr][kt][e] = p;
+        rs[e & 1] += p;
+      }
+    st.l[nr][0] = st.l[nr][0] * alpha[0] + rs[0];
+    st.l[nr][1] = st.l[nr][1] * alpha[1] + rs[1];
+    // Once the running maxima settle, most tiles leave every alpha at 1: skip the rescale then.
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        st.acc[nr][mt][0] *= alpha[0];
+        st.acc[nr][mt][1] *= alpha[1];
+        st.acc[nr][mt][2] *= alpha[0];
+        st.acc[nr][mt][3] *= alpha[1];
+      }
+    }
+  }
+  // O^T += V^T P^T, 16 keys at a time.
+#pragma unroll
+  for (int kt = 0; kt < NKT; ++kt) {
+    uint32_t pb[NR][2];
+#pragma unroll
+    for (int nr = 0; nr < NR; ++nr) {
+      if constexpr (MMA_BF) {
+        pb[nr][0] = movmatrix_trans(pack_bf16x2(s[nr][kt][0], s[nr][kt][1]));
+        pb[nr][1] = movmatrix_trans(pack_bf16x2(s[nr][kt][2], s[nr][kt][3]));
+      } else {
+        pb[nr][0] = movmatrix_trans(pack_f16x2(s[nr][kt][0], s[nr][kt][1]));
+        pb[nr][1] = movmatrix_trans(pack_f16x2(s[nr][kt][2], s[nr][kt][3]));
+      }
+    }
+    const uint32_t vb = vbase + kt * 16 * 128;
+    if constexpr (KV == KV_E4M3) {
+#pragma unroll
+      for (int c32 = 0; c32 < D / 32; ++c32) {
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4_trans(vb + off.v[c32], r0, r1, r2, r3);
+        const uint32_t p0 = __byte_perm(r0, 0, 0x3120), p1 = __byte_perm(r1, 0, 0x3120);
+        const uint32_t p2 = __byte_perm(r2, 0, 0x3120), p3 = __byte_perm(r3, 0, 0x3120);
+        const uint32_t ae[4] = {e4m3x2_to_f16x2(uint16_t(p0 & 0xffff)), e4m3x2_to_f16x2(uint16_t(p1 & 0xffff)),
+                                e4m3x2_to_f16x2(uint16_t(p2 & 0xffff)), e4m3x2_to_f16x2(uint16_t(p3 & 0xffff))};
+        const uint32_t ao[4] = {e4m3x2_to_f16x2(uint16_t(p0 >> 16)), e4m3x2_to_f16x2(uint16_t(p1 >> 16)),
+                                e4m3x2_to_f16x2(uint16_t(p2 >> 16)), e4m3x2_to_f16x2(uint16_t(p3 >> 16))};
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr) {
+          mma16816<false>(st.acc[nr][2 * c32], ae, pb[nr][0], pb[nr][1]);
+          mma16816<false>(st.acc[nr][2 * c32 + 1], ao, pb[nr][0], pb[nr][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(vb + off.v[mt], a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr) mma16816<MMA_BF>(st.acc[nr][mt], a, pb[nr][0], pb[nr][1]);
+      }
+    }
+  }
+}
+
+// Zero V rows [from, TK) of a staged tile: those keys are past the item's end.
+template <int RB, int TK, int SLAB>
+PKV_DEVICE void zero_v_tail(uint32_t vbase, int from, int lane) {
+  constexpr int CPR = RB / 16;
+  for (int x = lane; x < (TK - from) * CPR; x += 32) {
+    const int r = from + x / CPR, ch = x % CPR;
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(vbase + tile_offset<RB, TK, SLAB>(r, ch * 16)), "r"(0)
+                 : "memory");
+  }
+  __syncwarp();
+}
+
+template <int D, int KV, bool QBF>
+__global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant__ CUtensorMap tmap, const TmaArgs ta) {
+  using T = TmaCfg<D, KV, QBF>;
+  const AttnArgs& a = ta.a;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t stages = base;
+  float* red_o = reinterpret_cast<float*>(base_ptr + T::NST * T::STAGE_BYTES);
+  float* red_m = red_o + 4 * 16 * D;
+  float* red_l = red_m + 4 * 16;
+  const uint32_t bars = base + T::NST * T::STAGE_BYTES + T::MERGE_BYTES;
+  auto full_bar = [&](int i) { return bars + 8 * i; };
+  auto empty_bar = [&](int i) { return bars + 8 * (T::NST + i); };
+  auto ifull_bar = [&](int i) { return bars + 8 * (2 * T::NST + i); };
+  auto iempty_bar = [&](int i) { return bars + 8 * (2 * T::NST + T::IR + i); };
+  const uint32_t merge_bar = bars + 8 * (2 * T::NST + 2 * T::IR);
+  ItemDesc* descs = reinterpret_cast<ItemDesc*>(base_ptr + T::NST * T::STAGE_BYTES + T::MERGE_BYTES + T::BAR_BYTES);
+  volatile int* s_ids = reinterpret_cast<volatile int*>(base_ptr + T::NST * T::STAGE_BYTES + T::MERGE_BYTES +
+                                                        T::BAR_BYTES + T::DESC_BYTES);
+  __shared__ volatile int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < T::NST; ++i) {
+      mbar_init(full_bar(i), 1);
+      mbar_init(empty_bar(i), 4);
+    }
+    for (int i = 0; i < T::IR; ++i) {
+      mbar_init(ifull_bar(i), 1);
+      mbar_init(iempty_bar(i), 4);
+    }
+    mbar_init(merge_bar, 128);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    // The warp fetches item fields and 32 block ids at a time (coalesced);
+    // lane 0 alone runs the tile loop: wait for a free stage, arm its barrier,
+    // issue the boxes.
+    const int total_q = __ldg(a.cu_q_lens + a.num_seqs);
+    const int box_rows = ta.box_rows;
+    const bool merged = ta.merged != 0;
+    const int bmask = (1 << a.log2_block) - 1;
+    const int c3k = 2 * a.layer;
+    int q = 0, it_seq = 0;
+    bool ok = true;
+    // The first item of each CTA is its own index; later ones come from the counter.
+    int next_idx = blockIdx.x;
+    for (;;) {
+      const int slot = it_seq % T::IR;
+      int flag = 1;
+      if (lane == 0) flag = mbar_wait(iempty_bar(slot), ((it_seq / T::IR) & 1) ^ 1) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, flag, 0)) { ok = false; break; }
+      const int idx = __shfl_sync(0xffffffffu, next_idx, 0);
+      ItemDesc& d = descs[slot];
+      if (idx >= a.n_items) {
+        if (lane == 0) {
+          d.state = 2;
+          mbar_arrive(ifull_bar(slot), 1);
+        }
+        break;
+      }
+      if (lane == 0) next_idx = int(gridDim.x + atomicAdd(a.counter, 1u));  // the next item, fetched ahead
+      const int* src = reinterpret_cast<const int*>(a.items + idx);
+      const int field = lane < 8 ? __ldg(src + lane) : 0;
+      PkvItem it;
+      it.seq = __shfl_sync(0xffffffffu, field, 0);
+      it.kv_head = __shfl_sync(0xffffffffu, field, 1);
+      it.q_begin = __shfl_sync(0xffffffffu, field, 2);
+      it.n_q = __shfl_sync(0xffffffffu, field, 3);
+      it.k_begin = __shfl_sync(0xffffffffu, field, 4);
+      it.k_end = __shfl_sync(0xffffffffu, field, 5);
+      it.pos0 = __shfl_sync(0xffffffffu, field, 6);
+      it.part_row = __shfl_sync(0xffffffffu, field, 7);
+      bool valid = it.seq >= 0 && it.seq < a.num_seqs && it.kv_head >= 0 && it.kv_head < a.hkv && it.n_q > 0 &&
+                   it.n_q * a.g <= PKV_TILE_ROWS && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q &&
+                   it.k_begin >= 0 && it.k_begin < it.k_end && (it.k_begin % box_rows) == 0;
+      if (valid) {
+        const int L = __ldg(a.seq_lens + it.seq);
+        valid = it.k_end <= L && ((it.k_end - 1) >> a.log2_block) < a.max_blocks && (it.pos0 < 0 || it.pos0 + it.n_q <= L);
+      }
+      if (!valid && lane == 0) report(a.status, PKV_DEV_PLAN_MISMATCH);
+      const int ntiles = valid ? (it.k_end - it.k_begin + T::TK - 1) / T::TK : 0;
+      if (lane == 0) {
+        d.seq = it.seq; d.kv_head = it.kv_head; d.q_begin = it.q_begin; d.n_q = it.n_q; d.k_begin = it.k_begin;
+        d.k_end = it.k_end; d.pos0 = it.pos0; d.part_row = it.part_row; d.ntiles = ntiles; d.state = valid ? 0 : 1;
+        mbar_arrive(ifull_bar(slot), 1);
+      }
+      ++it_seq;
+      if (ntiles == 0) continue;
+      const int32_t* bt_row = a.block_tables + int64_t(it.seq) * a.max_blocks;
+      const int first_blk = it.k_begin >> a.log2_block;
+      const int nblk_item = ((it.k_end - 1) >> a.log2_block) - first_blk + 1;
+      int t = 0;
+      for (int chunk = 0; chunk < nblk_item && ok; chunk += 32) {
+        s_ids[lane] = chunk + lane < nblk_item ? __ldg(bt_row + first_blk + chunk + lane) : -1;
+        __syncwarp();
+        if (lane == 0) {
+          // Tiles whose first block lies in this chunk (a tile never straddles chunks:
+          // 32 is a multiple of the blocks per tile).
+          for (; t < ntiles; ++t, ++q) {
+            const int key0 = it.k_begin + t * T::TK;
+            const int rel = (key0 >> a.log2_block) - first_blk - chunk;
+            if (rel >= 32) break;
+            const int stg = q % T::NST;
+            if (s_abort || !mbar_wait(empty_bar(stg), ((q / T::NST) & 1) ^ 1)) { flag = 0; break; }
+            const uint32_t sdst = stages + stg * T::STAGE_BYTES;
+            if (merged) {
+              int phys = s_ids[rel];
+              if (phys < 0 || phys >= a.num_blocks) {
+                report(a.status, PKV_DEV_BAD_BLOCK_ID);
+                phys = int(a.num_blocks);  // out of the tensor: the load fills zeros
+              }
+              mbar_arrive_expect_tx(full_bar(stg), T::HALVES * 2 * T::TK * 128);
+#pragma unroll
+              for (int h = 0; h < T::HALVES; ++h)
+                tma_load_5d(sdst + h * T::SLAB, &tmap, full_bar(stg), h * (128 / T::ELEM), key0 & bmask, it.kv_head,
+                            c3k, phys);
+            } else {
+              int nb = 0;
+              while (nb < T::TK / box_rows && key0 + nb * box_rows < it.k_end) ++nb;
+              mbar_arrive_expect_tx(full_bar(stg), uint32_t(nb) * T::HALVES * 2 * box_rows * 128);
+              for (int j = 0; j < nb; ++j) {
+                int phys = s_ids[rel + j];
+                if (phys < 0 || phys >= a.num_blocks) {
+                  report(a.status, PKV_DEV_BAD_BLOCK_ID);
+                  phys = int(a.num_blocks);
+                }
+#pragma unroll
+                for (int h = 0; h < T::HALVES; ++h) {
+                  const uint32_t dst = sdst + h * T::SLAB + uint32_t(j * box_rows) * 128;
+                  tma_load_5d(dst, &tmap, full_bar(stg), h * (128 / T::ELEM), 0, it.kv_head, c3k, phys);
+                  tma_load_5d(dst + T::TK * 128, &tmap, full_bar(stg), h * (128 / T::ELEM), 0, it.kv_head, c3k + 1,
+                              phys);
+                }
+              }
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, flag, 0)) ok = false;  // also orders s_ids reuse
+      }
+      q = __shfl_sync(0xffffffffu, q, 0);
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      report(a.status, PKV_DEV_TIMEOUT);
+      s_abort = 1;
+      // Let loads already issued land before the CTA's shared memory goes away.
+      for (int k = 1; k <= T::NST && q - k >= 0; ++k) mbar_wait(full_bar((q - k) % T::NST), ((q - k) / T::NST) & 1);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int g4 = lane >> 2, t4 = lane & 3;
+  DecOffsets<D, KV, QBF> offs;
+  dec_offsets<D, KV, QBF>(offs, lane);
+  int q = 0, it_seq = 0, merge_phase = 0;
+  bool ok = true;
+  for (;;) {
+    const int slot = it_seq % T::IR;
+    if (s_abort || !mbar_wait(ifull_bar(slot), (it_seq / T::IR) & 1)) { ok = false; break; }
+    const ItemDesc d = descs[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(iempty_bar(slot), 1);
+    ++it_seq;
+    if (d.state == 2) break;
+    if (d.state == 1) continue;
+    const int R = d.n_q * a.g;
+    const int ntiles = d.ntiles;
+    float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
+    float vscale = 1.f;
+    if constexpr (KV == KV_E4M3) {
+      c *= __ldg(a.k_scale + a.layer * a.hkv + d.kv_head);
+      vscale = __ldg(a.v_scale + a.layer * a.hkv + d.kv_head);
+    }
+    const bool to_part = d.part_row >= 0;
+    const int last_valid = d.k_end - (d.k_begin + (ntiles - 1) * T::TK);  // rows of the last tile in range
+
+    if (R <= 16) {
+      // ---- decode: warps take whole tiles round-robin, S^T / O^T formulation.
+      auto run = [&](auto nr_tag) {
+        constexpr int NR = decltype(nr_tag)::value;
+        DecState<D, KV, QBF, NR> st;
+        dec_load_q<D, KV, QBF, NR>(a, d, R, st, g4, t4);
+        int lim_min = d.k_end;
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int r = nr * 8 + 2 * t4 + b;
+            st.lim[nr][b] = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / a.g + 1) : d.k_end;
+            lim_min = min(lim_min, st.lim[nr][b]);
+            st.m[nr][b] = -INFINITY;
+            st.l[nr][b] = 0.f;
+          }
+        lim_min = __reduce_min_sync(0xffffffffu, lim_min);
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr)
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) st.acc[nr][mt][0] = st.acc[nr][mt][1] = st.acc[nr][mt][2] = st.acc[nr][mt][3] = 0.f;
+        for (int t = warp; t < ntiles; t += 4) {
+          // Owner by tile index within the item: the split of keys over warps (and so the
+          // rounding of the merge) does not depend on which items this CTA ran before.
+          const int qq = q + t;
+          const int stg = qq % T::NST;
+          if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1)) { ok = false; continue; }
+          const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::TK * 128;
+          if (t == ntiles - 1 && last_valid < T::TK) {
+            zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);
+            fence_proxy_async_smem();
+          }
+          const int key0 = d.k_begin + t * T::TK;
+          dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, key0, lane, c, key0 + T::TK > lim_min);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty_bar(stg), 4);
+        }
+        // Row sums over the eight lanes that share a row.
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float x = st.l[nr][b];
+            x += __shfl_xor_sync(0xffffffffu, x, 4);
+            x += __shfl_xor_sync(0xffffffffu, x, 8);
+            x += __shfl_xor_sync(0xffffffffu, x, 16);
+            st.l[nr][b] = x;
+          }
+#pragma unroll
+        for (int nr = 0; nr < NR; ++nr)
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int r = nr * 8 + 2 * t4 + (e & 1);
+              if (r < R) red_o[(warp * 16 + r) * D + dec_dim<KV>(mt, e, g4)] = st.acc[nr][mt][e];
+            }
+        if (g4 == 0) {
+#pragma unroll
+          for (int nr = 0; nr < NR; ++nr)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              const int r = nr * 8 + 2 * t4 + b;
+              red_m[warp * 16 + r] = st.m[nr][b];
+              red_l[warp * 16 + r] = st.l[nr][b];
+            }
+        }
+      };
+      if (R <= 8) run(std::integral_constant<int, 1>{});
+      else run(std::integral_constant<int, 2>{});
+      mbar_arrive(merge_bar, 1);
+      if (!mbar_wait(merge_bar, merge_phase)) ok = false;
+      merge_phase ^= 1;
+      for (int x = tid; x < R * D; x += 128) {
+        const int r = x / D, dd = x % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * 16 + r]);
+        float o = 0.f, lsum = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float f = fast_exp2(red_m[w * 16 + r] - M);
+            lsum += red_l[w * 16 + r] * f;
+            o += red_o[(w * 16 + r) * D + dd] * f;
+          }
+        }
+        const float inv = lsum > 0.f ? vscale / lsum : 0.f;
+        const int64_t orow = to_part ? int64_t(d.part_row) + r : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
+        if (to_part) a.part_o[orow * D + dd] = o * inv;
+        else store_q_dtype<QBF>(a.out, orow * D + dd, o * inv);
+        if (dd == 0) {
+          const float lse = lsum > 0.f ? (M + __log2f(lsum)) * kLn2 : -INFINITY;
+          if (to_part) a.part_lse[orow] = lse;
+          else if (a.out_lse) a.out_lse[orow] = lse;
+        }
+      }
+      mbar_arrive(merge_bar, 1);
+      if (!mbar_wait(merge_bar, merge_phase)) ok = false;
+      merge_phase ^= 1;
+    } else {
+      // ---- prefill tile: every warp reads every tile, 16 rows per warp.
+      ItemCtx<D, KV, QBF> cx;
+      cx.g = a.g;
+      cx.R = R;
+      cx.row_base = 16 * warp;
+      const bool active = cx.row_base < R;
+      PkvItem it{d.seq, d.kv_head, d.q_begin, d.n_q, d.k_begin, d.k_end, d.pos0, d.part_row};
+      load_q<D, KV, QBF>(a, it, cx, g4, t4);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = cx.row_base + g4 + 8 * hh;
+        cx.lim[hh] = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / cx.g + 1) : d.k_end;
+        cx.m[hh] = -INFINITY;
+        cx.l[hh] = 0.f;
+      }
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt) cx.acc[nt][0] = cx.acc[nt][1] = cx.acc[nt][2] = cx.acc[nt][3] = 0.f;
+      for (int t = 0; t < ntiles; ++t) {
+        const int qq = q + t;
+        const int stg = qq % T::NST;
+        if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1)) { ok = false; continue; }
+        const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::TK * 128;
+        if (t == ntiles - 1 && last_valid < T::TK) {
+          zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);  // each warp writes the same zeros
+          fence_proxy_async_smem();
+        }
+        if (active)
+          compute_keys<T::TK / 16, D, KV, QBF, T::TK, T::SLAB>(a, cx, kb, vb, 0, d.k_begin + t * T::TK, g4, t4, lane, c);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(stg), 1);
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        cx.l[hh] += __shfl_xor_sync(0xffffffffu, cx.l[hh], 1);
+        cx.l[hh] += __shfl_xor_sync(0xffffffffu, cx.l[hh], 2);
+      }
+      if (active) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = cx.row_base + g4 + 8 * hh;
+          if (r >= R) continue;
+          const float inv = cx.l[hh] > 0.f ? vscale / cx.l[hh] : 0.f;
+          const float lse = cx.l[hh] > 0.f ? (cx.m[hh] + __log2f(cx.l[hh])) * kLn2 : -INFINITY;
+          const int64_t orow = to_part ? int64_t(d.part_row) + r : (int64_t(d.q_begin) + r / cx.g) * a.hq + d.kv_head * cx.g + r % cx.g;
+#pragma unroll
+          for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+            for (int e = 2 * hh; e < 2 * hh + 2; ++e) {
+              const int dd = acc_dim<KV>(nt, e, t4);
+              const float v = cx.acc[nt][e] * inv;
+              if (to_part) a.part_o[orow * D + dd] = v;
+              else store_q_dtype<QBF>(a.out, orow * D + dd, v);
+            }
+          if (t4 == 0) {
+            if (to_part) a.part_lse[orow] = lse;
+            else if (a.out_lse) a.out_lse[orow] = lse;
+          }
+        }
+      }
+    }
+    q += ntiles;
+    if (!ok) break;
+  }
+  if (!ok) {
+    report(a.status, PKV_DEV_TIMEOUT);
+    s_abort = 1;
+  }
+}
+
+// ---- host side -------------------------------------------------------------
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+// The pool as a 5-D tensor (innermost first): head_dim, slot, kv head, 2*layer + K|V, block.
+// A box is 128 bytes of one row x box_rows slots x 1 head x box_kv (1: K or V; 2: K and V) x 1 block.
+static bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataType dt, int box_rows, int box_kv,
+                          CUtensorMap* map) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t B = uint64_t(1) << a.log2_block;
+  cuuint64_t dims[5] = {cuuint64_t(head_dim), B, cuuint64_t(a.hkv), cuuint64_t(2 * a.num_layers), cuuint64_t(a.num_blocks)};
+  const uint64_t row = uint64_t(head_dim) * elem;
+  cuuint64_t strides[4] = {row, row * B, row * B * a.hkv, row * B * a.hkv * 2 * a.num_layers};
+  cuuint32_t box[5] = {cuuint32_t(128 / elem), cuuint32_t(box_rows), 1, cuuint32_t(box_kv), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(map, dt, 5, const_cast<void*>(a.pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int KV, bool QBF>
+cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
+  using T = TmaCfg<D, KV, QBF>;
+  CUtensorMap map;
+  const CUtensorMapDataType dt = KV == KV_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : KV == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const int B = 1 << a.log2_block;
+  const bool merged = B >= T::TK;
+  const int box_rows = merged ? T::TK : B;
+  if (!make_pool_map(a, D, T::ELEM, dt, box_rows, merged ? 2 : 1, &map)) return cudaErrorInvalidValue;
+  attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, TmaArgs{a, box_rows, merged ? 1 : 0});
+  return cudaGetLastError();
+}
+
+template <int D, int KV, bool QBF>
+AttnKernel tma_kernel() {
+  using T = TmaCfg<D, KV, QBF>;
+  return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF>), T::THREADS, T::SMEM,
+                    &launch_tma<D, KV, QBF>};
+}
+
+bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {
+  if (block_size < 8) return false;
+  const bool d128 = head_dim == 128;
+  if (head_dim != 64 && head_dim != 128) return false;
+  switch (kv_dtype) {
+    case PKV_BF16:
+      if (q_dtype != PKV_BF16) return false;
+      *k = d128 ? tma_kernel<128, KV_BF16, true>() : tma_kernel<64, KV_BF16, true>();
+      return true;
+    case PKV_F16:
+      if (q_dtype != PKV_F16) return false;
+      *k = d128 ? tma_kernel<128, KV_F16, false>() : tma_kernel<64, KV_F16, false>();
+      return true;
+    case PKV_FP8_E4M3:
+      if (!d128) return false;  // 64-byte rows stay on the cp.async kernel
+      if (q_dtype == PKV_BF16) *k = tma_kernel<128, KV_E4M3, true>();
+      else if (q_dtype == PKV_F16) *k = tma_kernel<128, KV_E4M3, false>();
+      else return false;
+      return true;
+  }
+  return false;
+}
+
+}  // namespace pkv

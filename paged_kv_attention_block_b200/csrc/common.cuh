@@ -39,16 +39,18 @@ PKV_DEVICE uint32_t e4m3x2_to_f16x2(uint16_t two) {
 }
 
 // ---- shared-memory tile layout -------------------------------------------
-// A K or V tile is PKV_TILE_KEYS rows of RB = head_dim * elem bytes.  Rows
+// A K or V tile is TK rows (keys) of RB = head_dim * elem bytes.  Rows
 // wider than 128 B are split into 128-B column slabs, each slab rows x 128 B,
 // and 16-byte chunks are XOR-swizzled with address bits 7..9 (the 128-byte
 // swizzle pattern), which makes the 8-row ldmatrix / LDS.128 phases of the MMA
 // fragment loads bank-conflict free.
-template <int RB>
+// SLAB is the distance between column slabs (TK * 128 when a tile's slabs are
+// adjacent; larger when K and V slabs interleave).
+template <int RB, int TK = PKV_TILE_KEYS, int SLAB = TK * 128>
 PKV_DEVICE uint32_t tile_offset(int row, int byte) {
   uint32_t lin;
   if constexpr (RB >= 128) {
-    lin = uint32_t(byte >> 7) * (PKV_TILE_KEYS * 128) + uint32_t(row) * 128 + uint32_t(byte & 127);
+    lin = uint32_t(byte >> 7) * SLAB + uint32_t(row) * 128 + uint32_t(byte & 127);
   } else {
     lin = uint32_t(row) * RB + uint32_t(byte);
   }
@@ -101,4 +103,103 @@ PKV_DEVICE float fast_exp2(float x) {
   return y;
 }
 
+}  // namespace pkv
+
+// ---- mbarriers, TMA, warp-level matrix moves (sm_90+ PTX) -----------------
+namespace pkv {
+
+PKV_DEVICE void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+PKV_DEVICE void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
+PKV_DEVICE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+PKV_DEVICE void mbar_arrive(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+PKV_DEVICE void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+PKV_DEVICE bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase with the given parity: false after about 4e9 SM
+// cycles (1-3 s at B200 clocks); the caller records an error and stops waiting.
+// The deadline uses the SM-local cycle counter, which is cheap to read.
+constexpr long long kWaitLimitCycles = 4000000000ll;
+PKV_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  }
+}
+
+// 5-D tiled TMA load into shared memory, completion counted on `bar` (no multicast).
+PKV_DEVICE void tma_load_5d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], "
+      "[%2];\n" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
+PKV_DEVICE void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one row pair per thread.
+PKV_DEVICE uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  return d;
+}
+
+PKV_DEVICE void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
+}  // namespace pkv
+
+namespace pkv {
+// Merge element of a row whose n partial states sit at o_of(i), lse_of(i)
+// (normalised o, natural-log lse; lse = -inf marks an empty part):
+//   M = max lse_i, w_i = exp(lse_i - M), o = sum w_i o_i / sum w_i, lse = M + ln sum w_i.
+template <typename LseOf, typename OOf>
+PKV_DEVICE void merge_elem(int n, LseOf lse_of, OOf o_of, float& o, float& lse) {
+  float M = -INFINITY;
+  for (int i = 0; i < n; ++i) M = fmaxf(M, lse_of(i));
+  if (M == -INFINITY) {
+    o = 0.f;
+    lse = -INFINITY;
+    return;
+  }
+  float num = 0.f, den = 0.f;
+  for (int i = 0; i < n; ++i) {
+    const float li = lse_of(i);
+    if (li == -INFINITY) continue;
+    const float w = expf(li - M);
+    den += w;
+    num = fmaf(w, o_of(i), num);
+  }
+  o = num / den;
+  lse = M + logf(den);
+}
+
+PKV_DEVICE void store_any(void* out, int dtype, int64_t idx, float v) {
+  if (dtype == 0) static_cast<float*>(out)[idx] = v;
+  else if (dtype == 1) static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
+  else static_cast<__half*>(out)[idx] = __float2half_rn(v);
+}
 }  // namespace pkv

@@ -2,7 +2,7 @@
 #pragma once
 #include <stdint.h>
 
-#include "../../include/pkv.h"
+#include "pkv.h"
 
 // Record a message for pkv_last_error() on this thread and return `s`.
 pkv_status pkv_fail(pkv_status s, const char* fmt, ...);

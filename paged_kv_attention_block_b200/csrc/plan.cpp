@@ -69,7 +69,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   }
   int num_ctas = req->num_ctas;
   if (num_ctas <= 0) {
-    pkv_status st = pkv_default_num_ctas(req->kv_dtype, D, &num_ctas);
+    pkv_status st = pkv_default_num_ctas(req->kv_dtype, D, B, &num_ctas);
     if (st != PKV_OK) return st;
   }
   const int QT = std::max(1, PKV_TILE_ROWS / g);  // query tokens per tile

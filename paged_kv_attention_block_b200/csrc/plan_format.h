@@ -69,16 +69,18 @@ struct PkvReduce {
 };
 static_assert(sizeof(PkvReduce) == 32, "reduce size");
 
-// Device workspace layout: [plan copy][counters][partial o][partial lse].
+// Device workspace layout: [plan copy][work counter][partial o][partial lse].
+// The counter is cleared on the stream before every launch.
 static inline uint64_t pkv_align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 struct PkvWorkspaceLayout {
-  uint64_t plan_off, counter_off, part_o_off, part_lse_off, total;
+  uint64_t plan_off, counter_off, counter_bytes, part_o_off, part_lse_off, total;
 };
 static inline PkvWorkspaceLayout pkv_workspace_layout(uint64_t plan_bytes, int64_t n_part_rows, int head_dim) {
   PkvWorkspaceLayout L;
   L.plan_off = 0;
   L.counter_off = pkv_align256(plan_bytes);
-  L.part_o_off = L.counter_off + 256;
+  L.counter_bytes = 256;
+  L.part_o_off = L.counter_off + L.counter_bytes;
   L.part_lse_off = pkv_align256(L.part_o_off + uint64_t(n_part_rows) * head_dim * 4);
   L.total = pkv_align256(L.part_lse_off + uint64_t(n_part_rows) * 4);
   return L;

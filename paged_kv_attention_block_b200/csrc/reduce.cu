@@ -16,34 +16,6 @@
 
 namespace pkv {
 
-PKV_DEVICE void store_any(void* out, int dtype, int64_t idx, float v) {
-  if (dtype == PKV_F32) static_cast<float*>(out)[idx] = v;
-  else if (dtype == PKV_BF16) static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-  else static_cast<__half*>(out)[idx] = __float2half_rn(v);
-}
-
-// Merge element `d` of a row whose i-th part lives at o_of(i), lse_of(i).
-template <typename LseOf, typename OOf>
-PKV_DEVICE void merge_elem(int n, LseOf lse_of, OOf o_of, float& o, float& lse) {
-  float M = -INFINITY;
-  for (int i = 0; i < n; ++i) M = fmaxf(M, lse_of(i));
-  if (M == -INFINITY) {
-    o = 0.f;
-    lse = -INFINITY;
-    return;
-  }
-  float num = 0.f, den = 0.f;
-  for (int i = 0; i < n; ++i) {
-    const float li = lse_of(i);
-    if (li == -INFINITY) continue;
-    const float w = expf(li - M);
-    den += w;
-    num = fmaf(w, o_of(i), num);
-  }
-  o = num / den;
-  lse = M + logf(den);
-}
-
 __global__ void __launch_bounds__(256) dense_reduce_kernel(const float* __restrict__ po, const float* __restrict__ pl,
                                                            int n, int64_t rows, int d, void* out, int out_dtype,
                                                            float* out_lse) {

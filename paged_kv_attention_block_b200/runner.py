@@ -40,6 +40,10 @@ class DeviceWorkload:
         self.k_new = to_device(k, w.kv_in_dtype, self.device)
         self.v_new = to_device(v, w.kv_in_dtype, self.device)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        # Pinned plan buffers reused round-robin; an event per slot marks when its upload was enqueued.
+        self._plan_bufs = [None] * 4
+        self._plan_events = [None] * 4
+        self._plan_slot = 0
         if history:
             self.append_history(seq_chunk_tokens)
 
@@ -67,15 +71,28 @@ class DeviceWorkload:
 
     def plan(self, **opts) -> api.Plan:
         w = self.w
-        return api.plan_attention(w.cu_q_lens, w.seq_lens, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
-                                  head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal,
-                                  block_tables=w.block_tables, **opts)
+        i = self._plan_slot
+        if self._plan_events[i] is not None:
+            self._plan_events[i].synchronize()  # that buffer's upload has run
+        p = api.plan_attention(w.cu_q_lens, w.seq_lens, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                               head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal,
+                               block_tables=w.block_tables, buffer=self._plan_bufs[i], **opts)
+        self._plan_bufs[i] = p.buffer
+        p.slot = i
+        self._plan_slot = (i + 1) % len(self._plan_bufs)
+        return p
 
     def attention(self, plan: api.Plan, out=None, out_lse=None, workspace=None, stream=None):
         w = self.w
-        return api.paged_attention(self.cache, self.q, self.cu_q, self.seq_lens, self.block_tables, plan,
-                                   w.softmax_scale, w.causal, out=out, out_lse=out_lse, workspace=workspace,
-                                   status=self.status, stream=stream)
+        out = api.paged_attention(self.cache, self.q, self.cu_q, self.seq_lens, self.block_tables, plan,
+                                  w.softmax_scale, w.causal, out=out, out_lse=out_lse, workspace=workspace,
+                                  status=self.status, stream=stream)
+        slot = getattr(plan, "slot", None)
+        if slot is not None:
+            ev = torch.cuda.Event()
+            ev.record(torch.cuda.current_stream(self.device) if stream is None else stream)
+            self._plan_events[slot] = ev
+        return out
 
     def pool_bytes(self) -> np.ndarray:
         p = self.cache.pool

@@ -101,9 +101,23 @@ def test_prefix_reuse_bf16(pkv, cascade):
     assert (plan.info["num_groups"] > 0) == cascade
 
 
+@pytest.mark.parametrize("ctas", [1, 2, 3, 5])
+def test_few_ctas_many_items(pkv, ctas):
+    """Few persistent CTAs working through many items: the stage and item rings wrap many times,
+    alternating decode items (warps own whole tiles) and prefill tiles (warps share every tile)."""
+    w = W.mixed_bf16(n_decode=40, n_prefill=3, chunk=100, dec_lo=1, dec_hi=900, cached_lo_blocks=1,
+                     cached_hi_blocks=4, block_size=64)
+    run_case(pkv, w, num_ctas=ctas, kv_split=128)
+
+
+@pytest.mark.parametrize("ctas", [1, 3])
+def test_few_ctas_decode_fp8(pkv, ctas):
+    run_case(pkv, W.longctx_fp8(batch=5, seq_len=2000), num_ctas=ctas, kv_split=192)
+
+
 # ---- shapes and dtypes ----------------------------------------------------
 
-@pytest.mark.parametrize("B", [2, 4, 16, 32, 64, 128, 256])
+@pytest.mark.parametrize("B", [2, 4, 8, 16, 32, 64, 128, 256])
 @pytest.mark.parametrize("D", [64, 128])
 def test_block_sizes_and_head_dims(pkv, B, D):
     w = W.build(f"b{B}d{D}", seed=B * 7 + D, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=D,
