@@ -205,8 +205,10 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  * Source: deep dive §2 (decode reads all history KV to do attention), §6 (one
  * launch serves a packed mix of prefill and decode requests), §8 (chunked
  * prefill with causal masking).  One call enqueues one persistent attention
- * kernel and, when the plan split a key range, one merge kernel (the same
- * merge pkv_split_kv_reduce performs).
+ * kernel for the decode-sized tiles, one tcgen05 kernel for the tiles of more
+ * than 16 rows of a bf16/f16 pool (when the plan has such tiles) and, when the
+ * plan split a key range, one merge kernel (the same merge
+ * pkv_split_kv_reduce performs), in that order on `stream`.
  *
  * q: device [total_q][num_q_heads][head_dim], q_dtype F32 (F32 pools only),
  *   BF16 (BF16 or FP8 pools) or F16 (F16 or FP8 pools).  total_q = cu_q_lens[num_seqs].
@@ -220,6 +222,7 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  * out: device [total_q][num_q_heads][head_dim] in q_dtype.
  * out_lse: device float32 [total_q][num_q_heads] natural-log sum of exp(scores)
  *   per row, or NULL.
+ * q, out and the pool must be 16-byte aligned.
  * workspace: device, >= info.workspace_bytes, 256-byte aligned.
  * Errors: INVALID_ARG/UNSUPPORTED/PLAN/WORKSPACE synchronously; PKV_DEV_* bits
  *   asynchronously (skipped rows are left unwritten).

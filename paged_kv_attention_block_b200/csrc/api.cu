@@ -78,29 +78,38 @@ extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, i
 // Structural check of a host plan: every index the kernels follow stays inside
 // the plan and the workspace (lengths are checked against the device arrays by
 // the kernels themselves).
-static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv) {
+static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_rows, bool tc) {
   const char* base = reinterpret_cast<const char*>(h);
   const uint64_t bytes = h->bytes;
   auto inside = [&](uint64_t off, uint64_t n, uint64_t sz) { return off + n * sz <= bytes; };
-  if (h->n_items < 0 || h->n_reduce < 0 || h->n_parts < 0 || h->n_part_rows < 0 || h->total_q < 0 ||
-      !inside(h->items_off, h->n_items, sizeof(PkvItem)) || !inside(h->reduce_off, h->n_reduce, sizeof(PkvReduce)) ||
-      !inside(h->parts_off, h->n_parts, sizeof(int32_t)) || h->num_ctas <= 0)
+  if (h->n_items < 0 || h->n_tc_items < 0 || h->n_reduce < 0 || h->n_parts < 0 || h->n_part_rows < 0 ||
+      h->total_q < 0 || !inside(h->items_off, h->n_items, sizeof(PkvItem)) ||
+      !inside(h->tc_items_off, h->n_tc_items, sizeof(PkvItem)) || !inside(h->reduce_off, h->n_reduce, sizeof(PkvReduce)) ||
+      !inside(h->parts_off, h->n_parts, sizeof(int32_t)) || h->num_ctas <= 0 || (h->n_tc_items > 0 && h->tc_num_ctas <= 0))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan sections out of range");
-  const PkvItem* items = reinterpret_cast<const PkvItem*>(base + h->items_off);
-  for (int i = 0; i < h->n_items; ++i) {
-    const PkvItem& it = items[i];
-    const int64_t rows = int64_t(it.n_q) * g;
-    if (it.n_q <= 0 || rows > PKV_TILE_ROWS || it.kv_head < 0 || it.kv_head >= hkv || it.q_begin < 0 ||
-        int64_t(it.q_begin) + it.n_q > h->total_q || it.k_begin < 0 || it.k_begin > it.k_end ||
-        (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows))
-      return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan item %d out of range", i);
-  }
+  if (h->n_tc_items > 0 && !tc) return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan has tcgen05 items for a pool without that kernel");
+  auto check_items = [&](uint32_t off, int n, int lo, int hi, const char* what) -> pkv_status {
+    const PkvItem* items = reinterpret_cast<const PkvItem*>(base + off);
+    for (int i = 0; i < n; ++i) {
+      const PkvItem& it = items[i];
+      const int64_t rows = int64_t(it.n_q) * g;
+      if (it.n_q <= 0 || rows < lo || rows > hi || it.kv_head < 0 || it.kv_head >= hkv || it.q_begin < 0 ||
+          int64_t(it.q_begin) + it.n_q > h->total_q || it.k_begin < 0 || it.k_begin > it.k_end ||
+          (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows))
+        return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d out of range", what, i);
+    }
+    return PKV_OK;
+  };
+  if (pkv_status s = check_items(h->items_off, h->n_items, 1, max_rows, "item"); s != PKV_OK) return s;
+  if (pkv_status s = check_items(h->tc_items_off, h->n_tc_items, PKV_DECODE_ROWS + 1, PKV_TILE_ROWS_TC, "tcgen05 item");
+      s != PKV_OK)
+    return s;
   const PkvReduce* reds = reinterpret_cast<const PkvReduce*>(base + h->reduce_off);
   const int32_t* parts = reinterpret_cast<const int32_t*>(base + h->parts_off);
   for (int i = 0; i < h->n_reduce; ++i) {
     const PkvReduce& r = reds[i];
     const int64_t rows = int64_t(r.n_q) * g;
-    if (r.n_q <= 0 || rows > PKV_TILE_ROWS || r.kv_head < 0 || r.kv_head >= hkv || r.q_begin < 0 ||
+    if (r.n_q <= 0 || rows > PKV_TILE_ROWS_TC || r.kv_head < 0 || r.kv_head >= hkv || r.q_begin < 0 ||
         int64_t(r.q_begin) + r.n_q > h->total_q || r.parts_begin < 0 || r.n_parts < 0 ||
         int64_t(r.parts_begin) + r.n_parts > h->n_parts)
       return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan merge %d out of range", i);
@@ -141,17 +150,20 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: fp8 pool needs k_scale and v_scale");
   if (!(softmax_scale > 0.f) || softmax_scale == INFINITY)
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: softmax_scale must be positive and finite");
-  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads); vs != PKV_OK) return vs;
+  pkv::AttnKernel ktc{};
+  const bool tc = pkv::attn_tc_kernel_for(c.kv_dtype, q_dtype, c.head_dim, c.block_size, &ktc);
+  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads, k.max_rows, tc); vs != PKV_OK)
+    return vs;
   const PkvWorkspaceLayout L = pkv_workspace_layout(h->bytes, h->n_part_rows, c.head_dim);
-  if (h->n_items == 0) return PKV_OK;
+  if (h->n_items == 0 && h->n_tc_items == 0) return PKV_OK;
   if (!workspace || workspace_bytes < L.total)
     return pkv_fail(PKV_ERR_WORKSPACE, "paged_attention: workspace %zu < %llu bytes", workspace_bytes,
                     (unsigned long long)L.total);
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: workspace not 256-byte aligned");
   if (!c.pool || !q || !out || !cu_q_lens || !seq_lens || !block_tables || max_blocks <= 0)
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: null pointer or max_blocks <= 0");
-  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(c.pool)) & 15)
-    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: q and pool must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(c.pool)) & 15)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: q, out and pool must be 16-byte aligned");
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -159,7 +171,8 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
   if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.counter_off, 0, L.counter_bytes, st);
   if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: plan upload: %s", cudaGetErrorString(e));
   const int resident = pkv::resident_ctas(k);  // also sets the kernel's shared-memory limit
-  if (resident <= 0) return pkv_fail(PKV_ERR_CUDA, "paged_attention: occupancy query failed");
+  const int tc_resident = h->n_tc_items > 0 ? pkv::resident_ctas(ktc) : 1;
+  if (resident <= 0 || tc_resident <= 0) return pkv_fail(PKV_ERR_CUDA, "paged_attention: occupancy query failed");
   const char* dplan = ws + L.plan_off;
   pkv::AttnArgs a{};
   a.pool = c.pool;
@@ -187,9 +200,22 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
   a.part_o = reinterpret_cast<float*>(ws + L.part_o_off);
   a.part_lse = reinterpret_cast<float*>(ws + L.part_lse_off);
   a.status = dev_status;
-  const int grid = std::max(1, std::min(std::min(resident, h->num_ctas), h->n_items));
-  e = k.launch(a, grid, st);
-  if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: launch failed: %s", cudaGetErrorString(e));
+  a.max_rows = k.max_rows;
+  if (h->n_items > 0) {
+    const int grid = std::max(1, std::min(std::min(resident, h->num_ctas), h->n_items));
+    e = k.launch(a, grid, st);
+    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: launch failed: %s", cudaGetErrorString(e));
+  }
+  if (h->n_tc_items > 0) {
+    pkv::AttnArgs t = a;
+    t.items = reinterpret_cast<const PkvItem*>(dplan + h->tc_items_off);
+    t.n_items = h->n_tc_items;
+    t.counter = a.counter + 32;  // 128 bytes on
+    t.max_rows = ktc.max_rows;
+    const int grid = std::max(1, std::min(std::min(tc_resident, h->tc_num_ctas), h->n_tc_items));
+    e = ktc.launch(t, grid, st);
+    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: tcgen05 launch failed: %s", cudaGetErrorString(e));
+  }
   if (h->n_reduce > 0) {
     pkv::ReduceArgs r{};
     r.reduces = reinterpret_cast<const PkvReduce*>(dplan + h->reduce_off);

@@ -1,5 +1,6 @@
 // Launch arguments of the attention and merge kernels (host and device).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,6 +28,7 @@ struct AttnArgs {
   float* part_o;          // [n_part_rows][head_dim]
   float* part_lse;        // [n_part_rows]
   int32_t* status;
+  int32_t max_rows;       // rows per item this kernel accepts
 };
 
 struct ReduceArgs {
@@ -46,13 +48,20 @@ struct AttnKernel {
   int threads;
   int smem;
   cudaError_t (*launch)(const AttnArgs&, int grid, cudaStream_t);
+  int max_rows;  // rows per item the kernel accepts
 };
 // Picks the TMA kernel where it applies (block size >= 8, 128/256-byte rows),
 // else the cp.async tensor-core kernel, and the CUDA-core kernel for fp32 pools.
 bool attn_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
+// tcgen05 kernel for the tiles of more than 16 rows of a 16-bit pool (attn_tc.cu).
+bool attn_tc_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
 // SM count x occupancy of a kernel on the current device (cached per device).
 int resident_ctas(const AttnKernel& k);
+// The pool as a 5-D TMA tensor (attn_tma.cu): head_dim, slot, kv head, 2*layer + K|V, block;
+// boxes of 128 bytes x box_rows slots x 1 head x box_kv x 1 block, 128-byte swizzle.
+bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataType dt, int box_rows, int box_kv,
+                   CUtensorMap* map);
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st);
 
 }  // namespace pkv

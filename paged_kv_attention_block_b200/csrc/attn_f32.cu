@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
     if (idx >= a.n_items) break;
     const PkvItem it = a.items[idx];
     bool ok = it.seq >= 0 && it.seq < a.num_seqs && it.kv_head >= 0 && it.kv_head < a.hkv && it.n_q > 0 &&
-              it.n_q * a.g <= PKV_TILE_ROWS && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q && it.k_begin >= 0 &&
+              it.n_q * a.g <= a.max_rows && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q && it.k_begin >= 0 &&
               it.k_begin <= it.k_end;
     if (ok) {
       const int L = __ldg(a.seq_lens + it.seq);
@@ -104,8 +104,8 @@ cudaError_t launch_f32(const AttnArgs& a, int grid, cudaStream_t st) {
 }
 
 AttnKernel f32_kernel(int head_dim) {
-  if (head_dim == 128) return AttnKernel{reinterpret_cast<const void*>(&attn_f32_kernel<128>), 128, 0, &launch_f32<128>};
-  return AttnKernel{reinterpret_cast<const void*>(&attn_f32_kernel<64>), 128, 0, &launch_f32<64>};
+  if (head_dim == 128) return AttnKernel{reinterpret_cast<const void*>(&attn_f32_kernel<128>), 128, 0, &launch_f32<128>, PKV_TILE_ROWS};
+  return AttnKernel{reinterpret_cast<const void*>(&attn_f32_kernel<64>), 128, 0, &launch_f32<64>, PKV_TILE_ROWS};
 }
 
 }  // namespace pkv

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(128, 2) attn_mma_kernel(const AttnArgs a) {
     if (idx >= a.n_items) break;
     const PkvItem it = a.items[idx];
     bool ok = it.seq >= 0 && it.seq < a.num_seqs && it.kv_head >= 0 && it.kv_head < a.hkv && it.n_q > 0 &&
-              it.n_q * a.g <= PKV_TILE_ROWS && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q && it.k_begin >= 0 &&
+              it.n_q * a.g <= a.max_rows && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q && it.k_begin >= 0 &&
               it.k_begin <= it.k_end;
     if (ok) {
       const int L = __ldg(a.seq_lens + it.seq);
@@ -235,7 +235,7 @@ template <int D, int KV, bool QBF>
 AttnKernel mma_kernel() {
   using C = Cfg<D, KV, QBF>;
   return AttnKernel{reinterpret_cast<const void*>(&attn_mma_kernel<D, KV, QBF>), C::THREADS, C::SMEM,
-                    &launch_mma<D, KV, QBF>};
+                    &launch_mma<D, KV, QBF>, PKV_TILE_ROWS};
 }
 
 AttnKernel f32_kernel(int head_dim);  // attn_f32.cu

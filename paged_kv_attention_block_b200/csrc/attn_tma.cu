@@ -23,8 +23,9 @@
 //     MMA through movmatrix.  Fragment addresses are fixed per lane; masking
 //     runs only on tiles that reach past a row's limit.  The four warps merge
 //     their softmax states at the end of the item.
-//   * Prefill tiles (> 16 rows): every warp reads every tile and owns 16 rows
-//     (the row-split step of attn_tile.cuh).
+//   * Prefill tiles (> 16 rows; fp8 pools, since 16-bit pools send them to the
+//     tcgen05 kernel of attn_tc.cu): every warp reads every tile and owns 16
+//     rows (the row-split step of attn_tile.cuh).
 //   * Keys past the item's end inside the last tile are masked; their V rows
 //     are zeroed in shared memory before the P V product (0 * NaN would leak).
 //   * Every wait on an mbarrier is bounded; on a timeout the CTA records
@@ -389,7 +390,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       it.pos0 = __shfl_sync(0xffffffffu, field, 6);
       it.part_row = __shfl_sync(0xffffffffu, field, 7);
       bool valid = it.seq >= 0 && it.seq < a.num_seqs && it.kv_head >= 0 && it.kv_head < a.hkv && it.n_q > 0 &&
-                   it.n_q * a.g <= PKV_TILE_ROWS && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q &&
+                   it.n_q * a.g <= a.max_rows && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q &&
                    it.k_begin >= 0 && it.k_begin < it.k_end && (it.k_begin % box_rows) == 0;
       if (valid) {
         const int L = __ldg(a.seq_lens + it.seq);
@@ -683,8 +684,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // The pool as a 5-D tensor (innermost first): head_dim, slot, kv head, 2*layer + K|V, block.
 // A box is 128 bytes of one row x box_rows slots x 1 head x box_kv (1: K or V; 2: K and V) x 1 block.
-static bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataType dt, int box_rows, int box_kv,
-                          CUtensorMap* map) {
+bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataType dt, int box_rows, int box_kv,
+                   CUtensorMap* map) {
   auto fn = encode_fn();
   if (!fn) return false;
   const uint64_t B = uint64_t(1) << a.log2_block;
@@ -717,7 +718,7 @@ template <int D, int KV, bool QBF>
 AttnKernel tma_kernel() {
   using T = TmaCfg<D, KV, QBF>;
   return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF>), T::THREADS, T::SMEM,
-                    &launch_tma<D, KV, QBF>};
+                    &launch_tma<D, KV, QBF>, PKV_TILE_ROWS};
 }
 
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {

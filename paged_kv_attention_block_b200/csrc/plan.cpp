@@ -12,7 +12,11 @@
 //      that the persistent CTAs finish together, weighting a tile by its rows
 //      (compute) and keys (bytes);
 //   3. emits the merges that combine split ranges (and group tiles) per row.
-// Items are ordered heaviest first; CTAs pull them from an atomic counter.
+// On 16-bit pools tiles of more than 16 rows (prefill chunks, shared-prefix
+// groups) go to a second list served by the tcgen05 kernel, 128 rows a tile,
+// and are split and balanced over that kernel's CTAs on their own.  Items are
+// ordered heaviest first within each list; CTAs pull them from an atomic
+// counter.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -31,7 +35,7 @@ struct Unit {
 struct Seg {
   PkvItem it;
   double cost;
-  int order;
+  bool tc;  // tensor-memory list
 };
 
 double row_weight(int rows) { return rows <= 16 ? 1.0 : rows / 16.0; }
@@ -67,12 +71,18 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: sequence %d needs %d blocks > max_blocks %d", s,
                       (L[s] + B - 1) / B, req->max_blocks);
   }
+  const bool tc = pkv_tc_capable(req->kv_dtype, D, B);
   int num_ctas = req->num_ctas;
+  int tc_ctas = req->num_ctas;
   if (num_ctas <= 0) {
     pkv_status st = pkv_default_num_ctas(req->kv_dtype, D, B, &num_ctas);
     if (st != PKV_OK) return st;
+    tc_ctas = tc ? pkv_tc_resident_ctas(req->kv_dtype, D, B) : num_ctas;
+    if (tc_ctas <= 0) return pkv_fail(PKV_ERR_CUDA, "attention_plan: occupancy query of the tcgen05 kernel failed");
   }
-  const int QT = std::max(1, PKV_TILE_ROWS / g);  // query tokens per tile
+  const int rows_cap = tc ? PKV_TILE_ROWS_TC : PKV_TILE_ROWS;
+  const int QT = std::max(1, rows_cap / g);  // query tokens per tile
+  auto is_tc = [&](int rows) { return tc && rows > PKV_DECODE_ROWS; };
   const bool causal = req->causal != 0;
   auto q_len = [&](int s) { return cu[s + 1] - cu[s]; };
 
@@ -112,10 +122,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   std::vector<PkvReduce> reds;
   std::vector<int32_t> parts;
   int64_t part_rows = 0;
-  int order = 0;
   // Partial row of each (group member, KV head) inside its group tile.
   std::vector<int64_t> gpart(groups.empty() ? 0 : size_t(S) * Hkv, -1);
-  double total_cost = 0;
+  double total_cost[2] = {0, 0};  // register-tile list, tensor-memory list
   for (const Group& G : groups) {
     int a = G.first;
     while (a <= G.last) {
@@ -126,8 +135,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
         for (int m = a; m <= b; ++m) gpart[size_t(m) * Hkv + h] = part_rows + int64_t(cu[m] - cu[a]) * g;
         part_rows += int64_t(n) * g;
         const double c = double(G.tokens) * row_weight(n * g);
-        total_cost += c;
-        segs.push_back({it, c, order++});
+        total_cost[is_tc(n * g)] += c;
+        segs.push_back({it, c, is_tc(n * g)});
       }
       a = b + 1;
     }
@@ -146,37 +155,40 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       for (int h = 0; h < Hkv; ++h) {
         const int gp = group_of[s] >= 0 ? int(gpart[size_t(s) * Hkv + h]) : -1;
         Unit u{s, h, cu[s] + i0, n, kb, ke, pos0, gp, row_weight(n * g)};
-        total_cost += double(std::max(0, ke - kb)) * u.weight;
+        total_cost[is_tc(n * g)] += double(std::max(0, ke - kb)) * u.weight;
         units.push_back(u);
       }
     }
   }
 
   // 3. Key-range split and merges.
-  const double target = total_cost / (double(num_ctas) * 2.0);
+  const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 2.0)};
   for (const Unit& u : units) {
     const int n = std::max(0, u.k_end - u.k_begin);
+    const int rows = u.n_q * g;
+    const bool t = is_tc(rows);
+    const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     int64_t max_keys;
     if (req->kv_split < 0) max_keys = INT32_MAX;
-    else if (req->kv_split > 0) max_keys = round_up(req->kv_split, PKV_TILE_KEYS);
-    else max_keys = std::max<int64_t>(256, round_up(int64_t(std::ceil(target / u.weight)), PKV_TILE_KEYS));
+    else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
+    else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
+                                      round_up(int64_t(std::ceil(target[t] / u.weight)), tile_keys));
     const int64_t nseg = n == 0 ? 0 : (n + max_keys - 1) / max_keys;
-    const int rows = u.n_q * g;
     if (nseg == 1 && u.group_part < 0) {
       PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, u.k_begin, u.k_end, u.pos0, -1};
-      segs.push_back({it, n * u.weight, order++});
+      segs.push_back({it, n * u.weight, t});
       continue;
     }
     PkvReduce r{u.q_begin, u.n_q, u.kv_head, int32_t(parts.size()), 0, {0, 0, 0}};
     if (u.group_part >= 0) parts.push_back(u.group_part);
     if (nseg > 0) {
-      const int64_t seg = round_up((n + nseg - 1) / nseg, PKV_TILE_KEYS);
+      const int64_t seg = round_up((n + nseg - 1) / nseg, tile_keys);
       for (int64_t k0 = u.k_begin; k0 < u.k_end; k0 += seg) {
         const int k1 = int(std::min<int64_t>(u.k_end, k0 + seg));
         PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, int(k0), k1, u.pos0, int32_t(part_rows)};
         parts.push_back(int32_t(part_rows));
         part_rows += rows;
-        segs.push_back({it, (k1 - k0) * u.weight, order++});
+        segs.push_back({it, (k1 - k0) * u.weight, t});
       }
     }
     r.n_parts = int32_t(parts.size()) - r.parts_begin;
@@ -184,16 +196,21 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   }
   if (part_rows > INT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: too many partial rows");
 
-  std::stable_sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) { return x.cost > y.cost; });
+  // Register-tile items first, then tensor-memory items; heaviest first within each list.
+  std::stable_sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) {
+    return x.tc != y.tc ? y.tc : x.cost > y.cost;
+  });
+  const int64_t n_tc = std::count_if(segs.begin(), segs.end(), [](const Seg& s) { return s.tc; });
 
   const uint64_t items_off = sizeof(PkvPlanHeader);
+  const uint64_t tc_items_off = items_off + (segs.size() - n_tc) * sizeof(PkvItem);
   const uint64_t reduce_off = items_off + segs.size() * sizeof(PkvItem);
   const uint64_t parts_off = reduce_off + reds.size() * sizeof(PkvReduce);
   const uint64_t bytes = (parts_off + parts.size() * sizeof(int32_t) + 15) & ~uint64_t(15);
   if (bytes > UINT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: plan too large");
   info->plan_bytes = bytes;
   info->workspace_bytes = pkv_workspace_layout(bytes, part_rows, D).total;
-  info->num_items = int32_t(segs.size());
+  info->num_items = int32_t(segs.size());  // both lists
   info->num_reduce = int32_t(reds.size());
   info->num_parts = int32_t(parts.size());
   info->num_partial_rows = int32_t(part_rows);
@@ -207,7 +224,10 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   PkvPlanHeader h{};
   h.magic = PKV_PLAN_MAGIC;
   h.bytes = uint32_t(bytes);
-  h.n_items = info->num_items;
+  h.n_items = int32_t(segs.size() - n_tc);
+  h.n_tc_items = int32_t(n_tc);
+  h.tc_items_off = uint32_t(tc_items_off);
+  h.tc_num_ctas = tc_ctas;
   h.n_reduce = info->num_reduce;
   h.n_parts = info->num_parts;
   h.n_part_rows = info->num_partial_rows;

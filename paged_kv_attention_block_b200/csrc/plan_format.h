@@ -1,17 +1,25 @@
 // Work-list format shared by the host planner and the attention kernels.
 //
-// A plan is one contiguous buffer: header, items, merges, part list.  The host
-// builds it (plan.cpp), paged_attention copies it into the device workspace,
-// and every CTA of the persistent kernel pulls items from it.
+// A plan is one contiguous buffer: header, items, tensor-memory items, merges,
+// part list.  The host builds it (plan.cpp), paged_attention copies it into
+// the device workspace, and the CTAs of each persistent kernel pull items
+// from their own list.
 #pragma once
 #include <stdint.h>
 
 #define PKV_PLAN_MAGIC 0x314e4c50u  // "PLN1"
 
-// Rows of one work item: query tokens x the Hq/Hkv query heads of one KV head.
+// Rows of one work item (query tokens x the Hq/Hkv query heads of one KV
+// head) for the register-tile kernels.
 #define PKV_TILE_ROWS 64
-// Keys per pipeline stage.
+// Keys per pipeline stage of the register-tile kernels.
 #define PKV_TILE_KEYS 64
+// Tensor-memory items (16-bit pools): more than PKV_DECODE_ROWS and at most
+// PKV_TILE_ROWS_TC rows (one tensor-memory lane per row), keys in tiles of
+// PKV_TC_TILE_KEYS; a split key range starts on a multiple of that.
+#define PKV_DECODE_ROWS 16
+#define PKV_TILE_ROWS_TC 128
+#define PKV_TC_TILE_KEYS 128
 
 struct PkvPlanHeader {
   uint32_t magic;
@@ -33,7 +41,10 @@ struct PkvPlanHeader {
   uint32_t items_off;    // byte offsets from the start of the plan
   uint32_t reduce_off;
   uint32_t parts_off;
-  int32_t pad[13];       // header is 128 bytes
+  int32_t n_tc_items;    // tensor-memory items (attn_tc kernel), after the others
+  uint32_t tc_items_off;
+  int32_t tc_num_ctas;   // CTAs planned for the tensor-memory kernel
+  int32_t pad[10];       // header is 128 bytes
 };
 static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 
@@ -69,8 +80,9 @@ struct PkvReduce {
 };
 static_assert(sizeof(PkvReduce) == 32, "reduce size");
 
-// Device workspace layout: [plan copy][work counter][partial o][partial lse].
-// The counter is cleared on the stream before every launch.
+// Device workspace layout: [plan copy][work counters][partial o][partial lse].
+// The counters (one per kernel, 128 bytes apart) are cleared on the stream
+// before every call.
 static inline uint64_t pkv_align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 struct PkvWorkspaceLayout {
   uint64_t plan_off, counter_off, counter_bytes, part_o_off, part_lse_off, total;
@@ -79,7 +91,7 @@ static inline PkvWorkspaceLayout pkv_workspace_layout(uint64_t plan_bytes, int64
   PkvWorkspaceLayout L;
   L.plan_off = 0;
   L.counter_off = pkv_align256(plan_bytes);
-  L.counter_bytes = 256;
+  L.counter_bytes = 256;  // counter of the register-tile kernel at +0, tensor-memory kernel at +128
   L.part_o_off = L.counter_off + L.counter_bytes;
   L.part_lse_off = pkv_align256(L.part_o_off + uint64_t(n_part_rows) * head_dim * 4);
   L.total = pkv_align256(L.part_lse_off + uint64_t(n_part_rows) * 4);

@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(256) dense_reduce_kernel(const float* __restri
 }
 
 __global__ void __launch_bounds__(256) plan_reduce_kernel(const ReduceArgs a) {
+  // Rows per merge come from the plan (up to PKV_TILE_ROWS_TC).
   const int d = a.head_dim;
   for (int e = blockIdx.x; e < a.n_reduce; e += gridDim.x) {
     const PkvReduce red = a.reduces[e];

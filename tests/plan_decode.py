@@ -5,7 +5,8 @@ HEADER = np.dtype([("magic", "<u4"), ("bytes", "<u4"), ("n_items", "<i4"), ("n_r
                    ("n_part_rows", "<i4"), ("num_seqs", "<i4"), ("total_q", "<i4"), ("num_q_heads", "<i4"),
                    ("num_kv_heads", "<i4"), ("head_dim", "<i4"), ("block_size", "<i4"), ("kv_dtype", "<i4"),
                    ("causal", "<i4"), ("num_ctas", "<i4"), ("n_groups", "<i4"), ("items_off", "<u4"),
-                   ("reduce_off", "<u4"), ("parts_off", "<u4"), ("pad", "<i4", 13)])
+                   ("reduce_off", "<u4"), ("parts_off", "<u4"), ("n_tc_items", "<i4"), ("tc_items_off", "<u4"),
+                   ("tc_num_ctas", "<i4"), ("pad", "<i4", 10)])
 ITEM = np.dtype([("seq", "<i4"), ("kv_head", "<i4"), ("q_begin", "<i4"), ("n_q", "<i4"), ("k_begin", "<i4"),
                  ("k_end", "<i4"), ("pos0", "<i4"), ("part_row", "<i4")])
 REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("parts_begin", "<i4"),
@@ -13,13 +14,19 @@ REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("par
 assert HEADER.itemsize == 128 and ITEM.itemsize == 32 and REDUCE.itemsize == 32
 
 
+TILE_ROWS, DECODE_ROWS, TILE_ROWS_TC, TC_TILE_KEYS = 64, 16, 128, 128
+
+
 def decode(buf) -> dict:
+    """Header, both item lists (items: register-tile list then tensor-memory list), merges, parts."""
     b = np.asarray(buf.cpu().numpy() if hasattr(buf, "cpu") else buf, dtype=np.uint8)
     h = np.frombuffer(b[:128].tobytes(), HEADER)[0]
-    items = np.frombuffer(b[h["items_off"]:h["items_off"] + 32 * h["n_items"]].tobytes(), ITEM)
+    reg = np.frombuffer(b[h["items_off"]:h["items_off"] + 32 * h["n_items"]].tobytes(), ITEM)
+    tc = np.frombuffer(b[h["tc_items_off"]:h["tc_items_off"] + 32 * h["n_tc_items"]].tobytes(), ITEM)
+    items = np.concatenate([reg, tc])
     reds = np.frombuffer(b[h["reduce_off"]:h["reduce_off"] + 32 * h["n_reduce"]].tobytes(), REDUCE)
     parts = np.frombuffer(b[h["parts_off"]:h["parts_off"] + 4 * h["n_parts"]].tobytes(), "<i4")
-    return {"header": h, "items": items, "reduces": reds, "parts": parts}
+    return {"header": h, "items": items, "reg_items": reg, "tc_items": tc, "reduces": reds, "parts": parts}
 
 
 def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: int, causal: bool, block_tables=None,
@@ -27,13 +34,22 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
     """Every (query token, KV head) row group sees exactly its keys once, through one output path."""
     h, items, reds, parts = plan["header"], plan["items"], plan["reduces"], plan["parts"]
     g = num_q_heads // num_kv_heads
+    # List membership: tensor-memory items carry more than 16 and at most 128 rows and
+    # start their key range on a multiple of the 128-key tile (or of the block size when
+    # smaller); register-tile items carry at most 64 rows.
+    for it in plan["reg_items"]:
+        assert it["n_q"] * g <= TILE_ROWS
+    for it in plan["tc_items"]:
+        assert DECODE_ROWS < it["n_q"] * g <= TILE_ROWS_TC
+        if block_size is not None:
+            assert it["k_begin"] % min(block_size, TC_TILE_KEYS) == 0
     S = len(seq_lens)
     tok_seq = np.repeat(np.arange(S), np.diff(cu_q))
     # Partial rows: map part_row -> item, and check items' partial rows don't overlap.
     used = np.zeros(max(1, int(h["n_part_rows"])), np.int32)
     by_part = {}
     for it in items:
-        assert 1 <= it["n_q"] and it["n_q"] * g <= 64 and it["k_begin"] < it["k_end"]
+        assert 1 <= it["n_q"] and it["k_begin"] < it["k_end"]
         if it["part_row"] >= 0:
             used[it["part_row"]:it["part_row"] + it["n_q"] * g] += 1
             by_part[int(it["part_row"])] = it

@@ -119,13 +119,28 @@ def test_plan_covers_every_key_once(api, name, make, opts):
     w = make()
     p = _plan(api, w, **opts)
     d = PD.decode(p.buffer)
-    assert d["header"]["n_items"] == p.info["num_items"]
+    assert d["header"]["n_items"] + d["header"]["n_tc_items"] == p.info["num_items"]
     PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
                       w.block_size)
     if name == "prefix":
         assert p.info["num_groups"] >= 1
     if name == "prefix_off":
         assert p.info["num_groups"] == 0
+
+
+def test_plan_routes_prefill_tiles_to_tensor_memory_list(api):
+    """16-bit pools: tiles of more than 16 rows go to the tcgen05 list in 128-row tiles;
+    fp8 pools keep 64-row tiles in the register-tile list."""
+    w = W.mixed_bf16(n_decode=6, n_prefill=2, chunk=300, block_size=16, cached_lo_blocks=1, cached_hi_blocks=20)
+    d = PD.decode(_plan(api, w).buffer)
+    g = w.num_q_heads // w.num_kv_heads
+    tc, reg = d["tc_items"], d["reg_items"]
+    assert len(tc) > 0 and (tc["n_q"] * g > 16).all() and (tc["n_q"] * g).max() == 128
+    assert (reg["n_q"] * g <= 16).all()
+    w8 = W.build("f8", seed=2, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32, num_kv_heads=8,
+                 head_dim=128, block_size=16, seq_lens=[400, 50], q_lens=[200, 1])
+    d8 = PD.decode(_plan(api, w8).buffer)
+    assert d8["header"]["n_tc_items"] == 0 and (d8["items"]["n_q"] * 4).max() == 64
 
 
 def test_plan_noncausal_and_empty_rows(api):
@@ -145,7 +160,9 @@ def test_plan_balances_decode(api):
     """The automatic split keeps every item within ~2x the mean share per CTA."""
     w = W.llama3_8b_decode_bf16()
     p = _plan(api, w)
-    items = PD.decode(p.buffer)["items"]
+    d = PD.decode(p.buffer)
+    assert d["header"]["n_tc_items"] == 0  # one-token rows: every item stays in the decode list
+    items = d["items"]
     keys = (items["k_end"] - items["k_begin"]).astype(np.int64)
     per_cta = keys.sum() / 296
     assert keys.max() <= max(256, 2 * per_cta / 2 + 64)

@@ -171,6 +171,17 @@ def test_large_logits_stay_finite(pkv):
     run_case(pkv, w)
 
 
+@pytest.mark.parametrize("kv", ["bf16", "f16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_running_max_jumps(pkv, kv, D):
+    # Logits spread over hundreds of log2 units: a row's running max keeps
+    # jumping by more than 2^8 from tile to tile, so the output accumulator is
+    # rescaled many times; long causal chunks span many key tiles.
+    w = W.build("jumps", seed=11, kv_dtype=kv, num_q_heads=8, num_kv_heads=2, head_dim=D, block_size=16,
+                seq_lens=[700, 333], q_lens=[200, 77], data_scale=6.0)
+    run_case(pkv, w)
+
+
 def test_split_reduce_dense(pkv):
     api, _ = pkv
     r = np.random.default_rng(4)
