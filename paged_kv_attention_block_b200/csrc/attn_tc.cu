@@ -7,21 +7,35 @@
 // the plan's second item list; one persistent CTA per SM runs 128-row tiles,
 // one tensor-memory lane and one softmax thread per row:
 //
-//   warp 4     TMA producer: pulls items from its atomic counter, publishes each
+//   warp 8     TMA producer: pulls items from its atomic counter, publishes each
 //              in a 4-slot descriptor ring and streams K and V tiles of 128 keys
 //              into two separate rings (a K stage is released as soon as S has
 //              been computed from it, a V stage once P V has), 128-byte swizzle,
 //              completion counted on mbarriers.  No load uses cluster multicast.
-//   warp 5     MMA issuer (one thread): S = Q K^T into one of two tensor-memory S
-//              buffers, O += P V into the tensor-memory O (V read as an MN-major
-//              operand straight from its ring); completions are signalled with
-//              tcgen05.commit on mbarriers.  S of tile t+2 is issued as soon as
-//              the softmax threads are done with S of tile t.
-//   warps 0-3  softmax: stage Q once per item (K-major, 128-byte swizzle); per
-//              tile load this thread's row of S, mask it, keep the row's running
-//              max and sum in registers (no shuffles) and write the row of P
-//              (16-bit) to shared memory; the epilogue reads the row of O from
-//              tensor memory, divides by the sum and stores it.
+//   warps 9, 10 MMA issuers (one thread each): warp 10 issues S = Q K^T into one
+//              of two tensor-memory S buffers, as soon as the tile's K has landed
+//              and the softmax threads are done with the buffer's previous tile;
+//              warp 9 issues O += P V into the tensor-memory O once a tile's P is
+//              written.  Q and P are the A operands straight from tensor memory,
+//              K and V the B operands from their rings (V as an MN-major operand),
+//              so shared memory only carries K and V.  Completions are signalled
+//              with tcgen05.commit on mbarriers; with two issuers one thread's
+//              commits and waits overlap the other's MMAs.
+//   warps 0-7  softmax, two threads per row: warps w and w + 4 share the
+//              tensor-memory lanes of rows 32 (w % 4) .. + 31 and split every row's
+//              columns in halves.  Once per item each thread writes its half of the
+//              row of Q into tensor memory; per tile it loads its half of the row
+//              of S, masks it, swaps its partial max with its partner through
+//              shared memory, keeps the running max and its partial sum in
+//              registers and writes its half of the row of P (16-bit) back to
+//              tensor memory; the epilogue reads its half of the row of O, divides
+//              by the row's sum and stores it.
+//
+// Tensor memory (512 columns, one CTA per SM): O at 0, S buffers at 128 and
+// 256, Q at 384.  P of a tile overwrites the first half of its own S buffer
+// (both threads of every row have loaded their S by then: the max swap sits in
+// between), so P is double-buffered with S and a tile's softmax never waits for
+// the previous P V unless it has to rescale O.
 //
 // The running max of a row only moves when the row max exceeds it by more than
 // 2^8 (log2 units), so P stays <= 256 and the row of O in tensor memory is
@@ -48,22 +62,29 @@ struct TcCfg {
   static constexpr int ROWS = PKV_TILE_ROWS_TC;  // rows per item: tensor-memory lanes
   static constexpr int SLAB = TK * 128;          // one column slab of a K or V tile
   static constexpr int TILE = HALVES * SLAB;     // one K or V tile
-  static constexpr int NST = D == 128 ? 2 : 4;   // stages of each ring
-  static constexpr int QSLAB = ROWS * 128;
-  static constexpr int Q_BYTES = HALVES * QSLAB;
-  static constexpr int PSLAB = ROWS * 128;       // 64 keys of P
-  static constexpr int P_BYTES = (TK / 64) * PSLAB;
+  static constexpr int NST = (192 * 1024) / (2 * TILE);  // stages of each ring: 3 (d 128), 6 (d 64)
   static constexpr int IR = 4;                   // item descriptor slots
   // mbarrier indices
+  // Warp roles: 0-7 softmax (two threads per row), 8 TMA producer, 9 P V issuer, 10 S issuer.
+  static constexpr int SM_WARPS = 8, SM_THREADS = 32 * SM_WARPS, PROD_WARP = 8, PV_WARP = 9, S_WARP = 10;
+  static constexpr int CONSUMER_WARPS = SM_WARPS + 2;
+  static constexpr int HALF = TK / 2;  // keys of a tile per softmax thread
+  // Every POLY_EVERY-th pair of a thread's scores takes its exp2 on the FMA pipe
+  // (exp2_fma2), the rest on the exp unit: the split that balances the two.
+  static constexpr int POLY_EVERY = 3;
+  // S, P and exchange barriers come in pairs by parity, so that a waiter is never two phases behind.
   static constexpr int KFULL = 0, KEMPTY = NST, VFULL = 2 * NST, VEMPTY = 3 * NST, IFULL = 4 * NST,
-                       IEMPTY = IFULL + IR, SBAR = IEMPTY + IR, PBAR = SBAR + 2, OBAR = PBAR + 1, QBAR = OBAR + 1,
-                       FIN = QBAR + 1, END = FIN + 1, NBAR = END + 1;
-  static constexpr int K_OFF = 0, V_OFF = NST * TILE, Q_OFF = 2 * NST * TILE, P_OFF = Q_OFF + Q_BYTES,
-                       BAR_OFF = P_OFF + P_BYTES, DESC_OFF = BAR_OFF + (8 * NBAR + 63) / 64 * 64;
+                       IEMPTY = IFULL + IR, SBAR = IEMPTY + IR, PBAR = SBAR + 2, XBAR = PBAR + 2, OBAR = XBAR + 2,
+                       QBAR = OBAR + 2, FIN = QBAR + 1, END = FIN + 1, NBAR = END + 1;
+  // XCHG: partial row maxima / sums swapped between the two threads of a row, [2 parities][2 halves][128 rows].
+  static constexpr int K_OFF = 0, V_OFF = NST * TILE, XCHG_OFF = 2 * NST * TILE, BAR_OFF = XCHG_OFF + 2 * 2 * ROWS * 4,
+                       DESC_OFF = BAR_OFF + (8 * NBAR + 63) / 64 * 64;
   static constexpr int SMEM = 1024 + DESC_OFF + IR * 64;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 32 * (S_WARP + 1);
   static constexpr int TMEM_COLS = 512;
-  static constexpr int S_COL = 128;  // S buffers at columns 128 and 256, O at column 0
+  // Tensor-memory columns: O, two S buffers (fp32; P in the first half of each), Q (16-bit pairs).
+  static constexpr int O_COL = 0, S_COL = 128, Q_COL = 384;
+  static_assert(Q_COL + D / 2 <= TMEM_COLS, "tensor-memory map");
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   // The CTA takes all 512 tensor-memory columns: shared memory must rule out a second CTA on the SM.
@@ -87,55 +108,63 @@ PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
-// Row r of the item (query token q_begin + r / g, head kv_head * g + r % g) into
-// the staged Q: [D / 64 column slabs][128 rows][128 B], 16-byte chunks
-// XOR-swizzled by the row's low three bits (the 128-byte swizzle, K-major).
+// Half hf of row r of the item (query token q_begin + r / g, head kv_head * g +
+// r % g): head dims [hf * D / 2, (hf + 1) * D / 2) into this thread's
+// tensor-memory lane at q_tmem, two 16-bit values per column (the pairs are
+// the row's bytes in memory order).  Rows past R are zero.
 template <int D>
-PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t qbase, int r) {
+PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_tmem, int r, int hf) {
   const bool valid = r < R;
   const uint4* src = reinterpret_cast<const uint4*>(
       static_cast<const uint16_t*>(a.q) +
-      ((int64_t(d.q_begin) + (valid ? r / a.g : 0)) * a.hq + d.kv_head * a.g + (valid ? r % a.g : 0)) * D);
+      ((int64_t(d.q_begin) + (valid ? r / a.g : 0)) * a.hq + d.kv_head * a.g + (valid ? r % a.g : 0)) * D +
+      hf * (D / 2));
+  uint32_t w[D / 4];
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-    sts128(qbase + uint32_t(c >> 3) * (128 * 128) + uint32_t(r) * 128 + (uint32_t((c & 7) ^ (r & 7)) << 4), v);
+  for (int i = 0; i < D / 16; ++i) {
+    const uint4 v = valid ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    w[4 * i] = v.x;
+    w[4 * i + 1] = v.y;
+    w[4 * i + 2] = v.z;
+    w[4 * i + 3] = v.w;
   }
+  if constexpr (D == 128) tc::st32_nowait(q_tmem, w);
+  else tc::st16_nowait(q_tmem, w);
+  tc::wait_st();
 }
 
-// S[128 x TK] = Q K^T, one thread: D/16 MMAs of K = 16.  Q and K are K-major
-// with the 128-byte swizzle: 8-row groups 1024 bytes apart, the k-step moving
-// 32 bytes inside a 128-byte row, then to the next 64-element column slab.
+// S[128 x TK] = Q K^T, one thread: D/16 MMAs of K = 16.  Q comes from tensor
+// memory (8 columns per step); K is K-major with the 128-byte swizzle: 8-row
+// groups 1024 bytes apart, the k-step moving 32 bytes inside a 128-byte row,
+// then to the next 64-element column slab.
 template <int D, bool BF>
-PKV_DEVICE void tc_mma_s(uint32_t s_tmem, uint32_t qbase, uint32_t kbase) {
+PKV_DEVICE void tc_mma_s(uint32_t s_tmem, uint32_t q_tmem, uint32_t kbase) {
   using T = TcCfg<D>;
   constexpr uint32_t IDESC = tc::idesc_f16(BF, 128, T::TK, false, false);
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
-    const uint64_t ad = tc::smem_desc(qbase + (ks >> 2) * T::QSLAB + (ks & 3) * 32, 16, 1024, tc::SW128);
     const uint64_t bd = tc::smem_desc(kbase + (ks >> 2) * T::SLAB + (ks & 3) * 32, 16, 1024, tc::SW128);
-    tc::mma_ss(s_tmem, ad, bd, IDESC, ks > 0);
+    tc::mma_ts(s_tmem, q_tmem + 8 * ks, bd, IDESC, ks > 0);
   }
 }
 
-// O[128 x D] (+)= P V, one thread: TK/16 MMAs of K = 16.  P is K-major (two
-// 64-key slabs); V is the B operand in MN-major form: 64 head dims contiguous
-// (128 bytes, 128-byte swizzle), the next 64 dims one column slab further, 8
-// keys per 1024-byte swizzle atom, so each 16-key step advances 2048 bytes.
+// O[128 x D] (+)= P V, one thread: TK/16 MMAs of K = 16.  P comes from tensor
+// memory; V is the B operand in MN-major form: 64 head dims contiguous (128
+// bytes, 128-byte swizzle), the next 64 dims one column slab further, 8 keys
+// per 1024-byte swizzle atom, so each 16-key step advances 2048 bytes.
 template <int D, bool BF>
-PKV_DEVICE void tc_mma_o(uint32_t o_tmem, uint32_t pbase, uint32_t vbase, bool accumulate) {
+PKV_DEVICE void tc_mma_o(uint32_t o_tmem, uint32_t p_tmem, uint32_t vbase, bool accumulate) {
   using T = TcCfg<D>;
   constexpr uint32_t IDESC = tc::idesc_f16(BF, 128, D, false, true);
 #pragma unroll
   for (int ks = 0; ks < T::TK / 16; ++ks) {
-    const uint64_t ad = tc::smem_desc(pbase + (ks >> 2) * T::PSLAB + (ks & 3) * 32, 16, 1024, tc::SW128);
     const uint64_t bd = tc::smem_desc(vbase + ks * 2048, T::SLAB, 1024, tc::SW128);
-    tc::mma_ss(o_tmem, ad, bd, IDESC, accumulate || ks > 0);
+    tc::mma_ts(o_tmem, p_tmem + 8 * ks, bd, IDESC, accumulate || ks > 0);
   }
 }
 
 template <int D, bool BF>
-__global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcArgs ta) {
+__global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcArgs ta) {
   using T = TcCfg<D>;
   constexpr unsigned FULL = 0xffffffffu;
   const AttnArgs& a = ta.a;
@@ -143,7 +172,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t kring = base + T::K_OFF, vring = base + T::V_OFF, qbuf = base + T::Q_OFF, pbuf = base + T::P_OFF;
+  const uint32_t kring = base + T::K_OFF, vring = base + T::V_OFF;
   const uint32_t bars = base + T::BAR_OFF;
   auto bar = [&](int i) { return bars + 8 * i; };
   TcDesc* descs = reinterpret_cast<TcDesc*>(base_ptr + T::DESC_OFF);
@@ -152,6 +181,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (warp == 0) tc::alloc(smem_addr(&s_tmem), T::TMEM_COLS);
+  float* xchg = reinterpret_cast<float*>(base_ptr + T::XCHG_OFF);
   if (tid == 32) {
     for (int i = 0; i < T::NST; ++i) {
       mbar_init(bar(T::KFULL + i), 1);
@@ -161,15 +191,17 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     }
     for (int i = 0; i < T::IR; ++i) {
       mbar_init(bar(T::IFULL + i), 1);
-      mbar_init(bar(T::IEMPTY + i), 5);  // four softmax warps and the issuer
+      mbar_init(bar(T::IEMPTY + i), T::CONSUMER_WARPS);
     }
-    mbar_init(bar(T::SBAR), 1);
-    mbar_init(bar(T::SBAR + 1), 1);
-    mbar_init(bar(T::PBAR), 128);
-    mbar_init(bar(T::OBAR), 1);
-    mbar_init(bar(T::QBAR), 128);
-    mbar_init(bar(T::FIN), 1);
-    mbar_init(bar(T::END), 5);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(T::SBAR + b), 1);
+      mbar_init(bar(T::PBAR + b), T::SM_THREADS);
+      mbar_init(bar(T::XBAR + b), T::SM_THREADS);
+      mbar_init(bar(T::OBAR + b), 1);
+    }
+    mbar_init(bar(T::QBAR), T::SM_THREADS);
+    mbar_init(bar(T::FIN), 2);
+    mbar_init(bar(T::END), T::CONSUMER_WARPS);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -178,7 +210,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   tc::fence_after_sync();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 4) {
+  if (warp == T::PROD_WARP) {
     // ------------------------------------------------------------ producer
     const int total_q = __ldg(a.cu_q_lens + a.num_seqs);
     const int box_rows = ta.box_rows;
@@ -280,10 +312,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     return;
   }
 
-  if (warp == 5) {
-    // ---------------------------------------------------------- MMA issuer
+  if (warp > T::PROD_WARP) {
+    // ------------------------------------------- MMA issuers (9: P V, 10: S)
+    // Tile qq (counted over the CTA's items) uses ring stage qq % NST, S buffer and
+    // S / P / O barriers qq & 1, whose phases for that tile have parity (qq >> 1) & 1.
+    const bool s_side = warp == T::S_WARP;
     int q = 0, it_seq = 0;
-    uint32_t q_ph = 0, p_ph = 0;
+    uint32_t q_ph = 0;
     bool ok = true;
     for (;;) {
       const int slot = it_seq % T::IR;
@@ -298,28 +333,33 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       if (d.state == 1) continue;
       const int n = d.ntiles;
       if (lane == 0) {
-        auto issue_s = [&](int t) -> bool {
-          const int qq = q + t, stg = qq % T::NST;
-          if (s_abort || !mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1)) return false;
-          tc_mma_s<D, BF>(tmem + T::S_COL + (t & 1) * T::TK, qbuf, kring + stg * T::TILE);
-          tc::commit(bar(T::SBAR + (t & 1)));
-          tc::commit(bar(T::KEMPTY + stg));
-          return true;
-        };
-        bool good = !s_abort && mbar_wait(bar(T::QBAR), q_ph);
-        if (good) tc::fence_after_sync();
-        for (int t = 0; t < min(2, n) && good; ++t) good = issue_s(t);
-        for (int t = 0; t < n && good; ++t) {
-          const int qq = q + t, stg = qq % T::NST;
-          good = !s_abort && mbar_wait(bar(T::PBAR), p_ph);
-          p_ph ^= 1;
-          if (good) good = mbar_wait(bar(T::VFULL + stg), (qq / T::NST) & 1);
-          if (!good) break;
-          tc::fence_after_sync();
-          tc_mma_o<D, BF>(tmem, pbuf, vring + stg * T::TILE, t > 0);
-          tc::commit(bar(T::OBAR));
-          tc::commit(bar(T::VEMPTY + stg));
-          if (t + 2 < n) good = issue_s(t + 2);
+        bool good = true;
+        if (s_side) {
+          // Q staged means every earlier item is finished (its epilogue waited for its last P V).
+          good = !s_abort && mbar_wait(bar(T::QBAR), q_ph);
+          if (good) tc::fence_after_sync();
+          for (int t = 0; t < n && good; ++t) {
+            const int qq = q + t, stg = qq % T::NST;
+            // The buffer's previous tile: its P (in the buffer) has been read by P V.
+            if (t >= 2) good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1);
+            if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1);
+            if (!good) break;
+            tc::fence_after_sync();
+            tc_mma_s<D, BF>(tmem + T::S_COL + (qq & 1) * T::TK, tmem + T::Q_COL, kring + stg * T::TILE);
+            tc::commit(bar(T::SBAR + (qq & 1)));
+            tc::commit(bar(T::KEMPTY + stg));
+          }
+        } else {
+          for (int t = 0; t < n && good; ++t) {
+            const int qq = q + t, stg = qq % T::NST;
+            good = !s_abort && mbar_wait(bar(T::PBAR + (qq & 1)), (qq >> 1) & 1);
+            if (good) good = mbar_wait(bar(T::VFULL + stg), (qq / T::NST) & 1);
+            if (!good) break;
+            tc::fence_after_sync();
+            tc_mma_o<D, BF>(tmem + T::O_COL, tmem + T::S_COL + (qq & 1) * T::TK, vring + stg * T::TILE, t > 0);
+            tc::commit(bar(T::OBAR + (qq & 1)));
+            tc::commit(bar(T::VEMPTY + stg));
+          }
         }
         if (!good) {
           ok = false;
@@ -332,7 +372,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     }
     if (lane == 0) {
       if (!ok) report(a.status, PKV_DEV_TIMEOUT);
-      // Every MMA this CTA issued has completed before tensor memory is released.
+      // Every MMA this thread issued has completed before tensor memory is released.
       tc::commit(bar(T::FIN));
       mbar_wait(bar(T::FIN), 0);
       tc::fence_before_sync();
@@ -342,12 +382,25 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   }
 
   // ---------------------------------------------------------------- softmax
-  const int r = tid;  // row of the tile and tensor-memory lane
-  const uint32_t lane_base = uint32_t(warp * 32) << 16;
-  const uint32_t o_tm = tmem + lane_base, s_tm = tmem + lane_base + T::S_COL;
-  int q = 0, it_seq = 0;
-  uint32_t s_ph = 0, o_ph = 0;  // s_ph bit b: parity to wait for on S buffer b
+  const int lq = warp & 3, hf = warp >> 2;  // lane quarter and column half
+  const int r = 32 * lq + lane;             // row of the tile and tensor-memory lane
+  const int stid = tid;                     // 0 .. SM_THREADS - 1
+  const uint32_t lane_base = uint32_t(lq * 32) << 16;
+  const uint32_t o_tm = tmem + lane_base + T::O_COL + hf * (D / 2), s_tm = tmem + lane_base + T::S_COL + hf * T::HALF;
+  const uint32_t q_tm = tmem + lane_base + T::Q_COL + hf * (D / 4);
+  const uint32_t p_tm = tmem + lane_base + T::S_COL + hf * (T::HALF / 2);  // + S buffer offset
+  int q = 0, it_seq = 0, xc = 0;  // xc: exchanges so far (barrier XBAR + (xc & 1), parity (xc >> 1) & 1)
   bool ok = true;
+  // Swap a value with the row's other thread through shared memory (bounded wait).
+  auto exchange = [&](float mine, float& other) -> bool {
+    float* buf = xchg + (xc & 1) * 2 * T::ROWS;
+    buf[hf * T::ROWS + r] = mine;
+    mbar_arrive(bar(T::XBAR + (xc & 1)), 1);
+    const bool done = warp_wait(bar(T::XBAR + (xc & 1)), (xc >> 1) & 1);
+    other = buf[(hf ^ 1) * T::ROWS + r];
+    ++xc;
+    return done;
+  };
   for (;;) {
     const int slot = it_seq % T::IR;
     bool go = __all_sync(FULL, ok && !s_abort);
@@ -367,32 +420,44 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     const int lim = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / a.g + 1) : d.k_end;
 
     // The previous item's MMAs are complete (its epilogue waited for the last P V): Q is free.
-    tc_stage_q<D>(a, d, R, qbuf, r);
-    fence_proxy_async_smem();
+    tc_stage_q<D>(a, d, R, q_tm, r, hf);
     tc::fence_before_sync();
     mbar_arrive(bar(T::QBAR), 1);
 
-    float m_run = -INFINITY, l_run = 0.f;  // running max (log2 units) and sum of this row
+    float m_run = -INFINITY, l_run = 0.f;  // running max of the row (log2 units), sum of this half
     for (int t = 0; t < ntiles; ++t) {
-      const int qq = q + t, stg = qq % T::NST, sb = t & 1;
+      const int qq = q + t, stg = qq % T::NST, sb = qq & 1;
       go = __all_sync(FULL, ok && !s_abort);
-      if (go) go = warp_wait(bar(T::SBAR + sb), (s_ph >> sb) & 1);
-      s_ph ^= 1u << sb;
+      if (go) go = warp_wait(bar(T::SBAR + sb), (qq >> 1) & 1);
       if (!go) { ok = false; continue; }
       tc::fence_after_sync();
-      float s[T::TK];
+      float s[T::HALF];
+      {
+        uint32_t* u = reinterpret_cast<uint32_t*>(s);
 #pragma unroll
-      for (int c0 = 0; c0 < T::TK; c0 += 32) tc::ld32(s_tm + sb * T::TK + c0, s + c0);
-      const int key0 = d.k_begin + t * T::TK;
-      if (key0 + T::TK > lim) {
+        for (int c0 = 0; c0 < T::HALF; c0 += 32) tc::ld32_nowait(s_tm + sb * T::TK + c0, u + c0);
+        tc::wait_ld();
+        tc::keep_after_wait<T::HALF>(u);
+      }
+      const int key0 = d.k_begin + t * T::TK + hf * T::HALF;
+      if (key0 + T::HALF > lim) {
 #pragma unroll
-        for (int j = 0; j < T::TK; ++j)
+        for (int j = 0; j < T::HALF; ++j)
           if (key0 + j >= lim) s[j] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // Max of this half over 8 independent chains, then of the row with the partner's.
+      float mx8[8];
 #pragma unroll
-      for (int j = 0; j < T::TK; ++j) mx = fmaxf(mx, s[j]);
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int j = 8; j < T::HALF; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      float mx_other;
+      if (!exchange(mx, mx_other)) { ok = false; continue; }
+      mx = fmaxf(mx, mx_other);
       const float mnew = mx * c;
+      // Both threads of the row take the same decisions from the same values.
       float alpha = 1.f;
       bool rescale = false;
       if (mnew > m_run + 8.f) {
@@ -402,18 +467,24 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         l_run *= alpha;
       }
       const float mneg = m_run == -INFINITY ? 0.f : -m_run;
-      float rs = 0.f;
+      // p = 2^(s c - m) in pairs; partial sums over four pair chains.
+      const float2 c2 = make_float2(c, c), m2 = make_float2(mneg, mneg);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int j = 0; j < T::TK; ++j) {
-        s[j] = fast_exp2(fmaf(s[j], c, mneg));
-        rs += s[j];
+      for (int i = 0; i < T::HALF / 2; ++i) {
+        const float2 x = ffma2(make_float2(s[2 * i], s[2 * i + 1]), c2, m2);
+        const float2 p = (i % T::POLY_EVERY) == 0 ? exp2_fma2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        acc[i & 3] = fadd2(acc[i & 3], p);
+        s[2 * i] = p.x;
+        s[2 * i + 1] = p.y;
       }
-      l_run += rs;
+      acc[0] = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      l_run += acc[0].x + acc[0].y;
       if (t == ntiles - 1 && last_valid < T::TK) {
         // Keys past the item's end: zero their V rows before P V reads them (0 * NaN would leak).
         if (warp_wait(bar(T::VFULL + stg), (qq / T::NST) & 1)) {
           const uint32_t vt = vring + stg * T::TILE;
-          for (int x = tid; x < (T::TK - last_valid) * T::HALVES * 8; x += 128) {
+          for (int x = stid; x < (T::TK - last_valid) * T::HALVES * 8; x += T::SM_THREADS) {
             const int row = last_valid + x / (T::HALVES * 8), h = (x / 8) % T::HALVES, ch = x % 8;
             sts128(vt + h * T::SLAB + row * 128 + (uint32_t(ch ^ (row & 7)) << 4), make_uint4(0, 0, 0, 0));
           }
@@ -421,16 +492,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           ok = false;
         }
       }
-      if (t > 0) {  // P V of the previous tile has read P and updated O
-        const bool done = warp_wait(bar(T::OBAR), o_ph);
-        o_ph ^= 1;
-        if (!done) { ok = false; continue; }
-        tc::fence_after_sync();
-      }
       if (__any_sync(FULL, rescale)) {
+        // O must hold the previous tile's P V before it is rescaled (t > 0 here).
+        if (!warp_wait(bar(T::OBAR + ((qq - 1) & 1)), ((qq - 1) >> 1) & 1)) { ok = false; continue; }
+        tc::fence_after_sync();
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
           float o[32];
           tc::ld32(o_tm + c0, o);
 #pragma unroll
@@ -438,44 +506,43 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           tc::st32(o_tm + c0, o);
         }
       }
+      // This half of the row of P (16-bit pairs) into tensor memory for the P V step.
+      {
+        uint32_t w[T::HALF / 2];
 #pragma unroll
-      for (int ch = 0; ch < T::TK / 8; ++ch) {
-        const float* x = s + 8 * ch;
-        uint4 v;
-        if constexpr (BF) {
-          v = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                         pack_bf16x2(x[6], x[7]));
-        } else {
-          v = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]), pack_f16x2(x[4], x[5]),
-                         pack_f16x2(x[6], x[7]));
-        }
-        sts128(pbuf + (ch >> 3) * T::PSLAB + uint32_t(r) * 128 + (uint32_t((ch & 7) ^ (r & 7)) << 4), v);
+        for (int i = 0; i < T::HALF / 2; ++i)
+          w[i] = BF ? pack_bf16x2(s[2 * i], s[2 * i + 1]) : pack_f16x2(s[2 * i], s[2 * i + 1]);
+        tc::st32_nowait(p_tm + sb * T::TK, w);
       }
-      fence_proxy_async_smem();
+      tc::wait_st();
+      if (t == ntiles - 1 && last_valid < T::TK) fence_proxy_async_smem();  // the zeroed V rows
       tc::fence_before_sync();
-      mbar_arrive(bar(T::PBAR), 1);
+      mbar_arrive(bar(T::PBAR + sb), 1);
     }
-    // Epilogue: O / l for this thread's row, straight from tensor memory.
+    // Epilogue: this half of O / l, straight from tensor memory; l is the sum of both halves.
     go = __all_sync(FULL, ok);
-    if (go) go = warp_wait(bar(T::OBAR), o_ph);
-    o_ph ^= 1;
+    float l_other = 0.f;
+    if (go) go = exchange(l_run, l_other);
+    if (go) go = warp_wait(bar(T::OBAR + ((q + ntiles - 1) & 1)), ((q + ntiles - 1) >> 1) & 1);
     if (go) {
       tc::fence_after_sync();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float l = l_run + l_other;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       const int64_t orow = to_part ? int64_t(d.part_row) + r
                                    : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
         float o[32];
         tc::ld32(o_tm + c0, o);
+        const int col = hf * (D / 2) + c0;
         if (r < R) {
           if (to_part) {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + orow * D + c0);
+            float4* dst = reinterpret_cast<float4*>(a.part_o + orow * D + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               dst[i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c0);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float* x = o + 8 * i;
@@ -489,8 +556,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           }
         }
       }
-      if (r < R) {
-        const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      if (r < R && hf == 0) {
+        const float lse = l > 0.f ? (m_run + __log2f(l)) * kLn2 : -INFINITY;
         if (to_part) a.part_lse[orow] = lse;
         else if (a.out_lse) a.out_lse[orow] = lse;
       }
@@ -504,7 +571,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     report(a.status, PKV_DEV_TIMEOUT);
     s_abort = 1;
   }
-  // Release tensor memory once the issuer's MMAs are done and every softmax
+  // Release tensor memory once the issuers' MMAs are done and every softmax
   // warp has finished with its lanes (bounded waits; freed on every path).
   tc::fence_before_sync();
   __syncwarp();

@@ -106,6 +106,51 @@ PKV_DEVICE float fast_exp2(float x) {
   return y;
 }
 
+// ---- packed float pairs (sm_100 f32x2 arithmetic) and an FMA-pipe exp2 -----
+
+PKV_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 pa, pb, pc, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n mov.b64 pc, {%6, %7};\n"
+      " fma.rn.f32x2 pd, pa, pb, pc;\n mov.b64 {%0, %1}, pd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+PKV_DEVICE float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 pa, pb, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n"
+      " add.rn.f32x2 pd, pa, pb;\n mov.b64 {%0, %1}, pd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe (the softmax is bound by the exp unit, so a
+// share of its exponentials is computed here instead).  Range reduction: adding
+// 1.5 * 2^23 rounds x to the nearest integer j, held in the low mantissa bits of
+// the sum; f = x - j lies in [-1/2, 1/2].  2^f is a cubic fitted to 2^f on
+// [-1/2, 1/2] by weighted least squares iterated towards equal relative error
+// (csrc/exp2_poly_fit.py); its largest relative error is 7.5e-5, below the
+// rounding of P to 16 bits.  2^j is added to the exponent field: the sum's bits
+// are 0x4B400000 + j, and (0x4B400000 << 23) is 0 modulo 2^32, so shifting the
+// sum's bits left by 23 gives j << 23.  x is clamped at -125, where the result
+// is still a normal number; exact values below that are < 2^-125 and do not
+// matter next to the row maximum's 2^0.
+constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f, kExp2C3 = 0.055171665f;
+constexpr float kRoundShift = 12582912.f;  // 1.5 * 2^23
+PKV_DEVICE float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(kRoundShift, kRoundShift));
+  const float2 j = fadd2(t, make_float2(-kRoundShift, -kRoundShift));
+  const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 }  // namespace pkv
 
 // ---- mbarriers, TMA, warp-level matrix moves (sm_90+ PTX) -----------------
