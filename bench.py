@@ -63,7 +63,26 @@ def algorithmic_bytes(w, plan_info=None) -> dict:
     new_rows = w.total_q * w.num_kv_heads * w.head_dim * 2
     append = new_rows * elem_bytes(w.kv_in_dtype) + new_rows * eb
     attn = kv + q + out + tables + scales + parts
-    return {"kv": kv, "attention": attn, "append": append, "step": attn + append}
+    # The attention kernels alone: everything but the merge's read of the partials and its output.
+    kernels = kv + q + out + tables + scales + parts // 2
+    return {"kv": kv, "attention": attn, "kernels": kernels, "append": append, "step": attn + append}
+
+
+def prefill_flops(w) -> float:
+    """4 d Hq per causal-valid (query, key) pair of the prefill chunks (q_len > 1)."""
+    pairs = 0
+    for L, ql in zip(w.seq_lens.astype(np.int64), w.q_lens.astype(np.int64)):
+        if ql > 1:
+            pairs += ql * (L - ql) + ql * (ql + 1) // 2 if w.causal else ql * L
+    return 4.0 * w.head_dim * w.num_q_heads * float(pairs)
+
+
+def bf16_peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
 
 
 def decode_rows(w) -> int:
@@ -262,6 +281,12 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     # left behind are clean, so no write-back of the flush lands in the timed region.
     flush = torch.ones(128 << 20, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
+    # Events recorded by the library right before and after the attention kernels (inside the
+    # graphs): the dominant kernels' own duration, read back one step at a time after the timed run.
+    kev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    with torch.cuda.stream(stream):
+        for e in kev:
+            e.record(stream)  # creates the CUDA events
 
     # The GPU side of a step runs from CUDA graphs: one for kv_append and one attention graph per
     # page-locked plan buffer (double-buffered), so the events below time GPU work only.  The host
@@ -276,18 +301,22 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     g_append = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_append, stream=stream):
         dw.append_new()
-    g_attn = []
-    for b in bufs:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale, w.causal,
-                                out=out, workspace=ws, status=dw.status)
-        g_attn.append(g)
+    # Two sets of attention graphs: the timed steps run graphs without the kernel events (their
+    # record nodes would add latency to the step); the kernel-only timing runs graphs with them.
+    g_attn, g_attn_ev = [], []
+    for evs_, graphs in ((None, g_attn), (kev, g_attn_ev)):
+        for b in bufs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
+                                    w.causal, out=out, workspace=ws, status=dw.status, kernel_events=evs_)
+            graphs.append(g)
     done = [None, None]
     host_plan_s = 0.0
 
-    def step(i, evs=None):
+    def step(i, evs=None, graphs=None):
         nonlocal host_plan_s
+        graphs = graphs or g_attn
         slot = i % 2
         if done[slot] is not None:
             done[slot].synchronize()  # the upload that read this buffer has run
@@ -301,7 +330,7 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             g_append.replay()
             if evs:
                 evs[1].record(stream)
-            g_attn[slot].replay()
+            graphs[slot].replay()
             if evs:
                 evs[2].record(stream)
             e = torch.cuda.Event()
@@ -326,20 +355,31 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     attn_ms = [b.elapsed_time(c) for _, b, c in ev]
     ms = float(np.mean(step_ms))
     attn = float(np.mean(attn_ms))
-    ms, attn = max_over_ranks([ms, attn], dev)
+    # The attention kernels' own duration: the same steps, one at a time, each read back after it ran.
+    kern_ms = []
+    for i in range(min(args.steps, 300)):
+        step(i, graphs=g_attn_ev)
+        torch.cuda.synchronize(dev)
+        kern_ms.append(kev[0].elapsed_time(kev[1]))
+    kern = float(np.mean(kern_ms))
+    ms, attn, kern = max_over_ranks([ms, attn, kern], dev)
     assert int(dw.status.item()) == 0, "device status set during the benchmark"
-    del g_append, g_attn
+    del g_append, g_attn, g_attn_ev
+    prefill = run_prefill_only(w, dev, api, runner, plan_kw) if rank == 0 and prefill_flops(w) > 0 else None
 
     b = algorithmic_bytes(w, plan.info)
     value = b["step"] * world / (ms * 1e-3) / 1e9
-    achieved = b["attention"] / (attn * 1e-3) / 1e9
+    achieved = b["kernels"] / (kern * 1e-3) / 1e9
     peak, peak_kind = peaks()
 
     # End to end through the public API from pinned host buffers.
     e2e = run_e2e(args, w, dw, plan_opts, dev, torch.cuda.current_stream(dev), api)
     e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
 
-    launches_per_step = 2 + (1 if plan.info["num_reduce"] > 0 else 0)
+    n_tc = plan.info["num_tc_items"]
+    launches_per_step = (1 + (plan.info["num_items"] > n_tc) + (n_tc > 0) + (plan.info["num_reduce"] > 0))
+    kernels = " + ".join(k for k, on in (("attn_tma_kernel", plan.info["num_items"] > n_tc),
+                                          ("attn_tc_kernel", n_tc > 0)) if on)
     if rank == 0:
         cpu = oracle_sample(w, budget_s=args.ref_budget, max_seqs=args.ref_seqs) if world == 1 and not args.no_cpu else None
         line = {
@@ -355,18 +395,60 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             "hbm_frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
             "hbm_frac_of_measured": value / world / peak,
             "step_bytes": b["step"], "kv_bytes": b["kv"],
-            "attention_ms": attn, "host_plan_us": host_plan_s / args.steps * 1e6,
+            "attention_ms": attn, "attention_kernels_ms": kern, "host_plan_us": host_plan_s / args.steps * 1e6,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic_for(w.name), "peak_source": peak_kind,
-                         "kernel": "attn_tma_kernel (the timed call also uploads the plan and runs the split merge)"},
+                         "kernel": kernels, "timed": "kernel-only CUDA events around the attention kernels, "
+                                                     "L2 flushed before each of up to 300 steps"},
             "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
             "e2e": {"value": b["step"] * world / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms"]},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
-            "plan": {k: plan.info[k] for k in ("num_items", "num_reduce", "num_partial_rows", "num_groups", "num_ctas")},
+            "plan": {k: plan.info[k] for k in ("num_items", "num_tc_items", "num_reduce", "num_partial_rows",
+                                               "num_groups", "num_ctas")},
         }
+        if prefill is not None:
+            line["prefill"] = prefill
         print(json.dumps(line), flush=True)
+
+
+def run_prefill_only(w, dev, api, runner, plan_kw, steps: int = 100):
+    """The prefill chunks of the batch alone (same lengths, same cached prefixes): tensor TFLOP/s
+    of the tcgen05 kernel, from kernel-only events, L2 flushed before each launch."""
+    import torch
+    from paged_kv_attention_block_b200 import workloads as W
+
+    idx = [i for i in range(w.num_seqs) if int(w.q_lens[i]) > 1]
+    sub = W.build(w.name + "_prefill_only", seed=7, kv_dtype=w.kv_dtype, num_q_heads=w.num_q_heads,
+                  num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=w.block_size,
+                  seq_lens=w.seq_lens[idx], q_lens=w.q_lens[idx], causal=w.causal)
+    dw = runner.DeviceWorkload(sub, device=dev)
+    dw.append_new()
+    kw = {k: v for k, v in plan_kw.items() if k != "block_tables"}
+    plan = api.plan_attention(sub.cu_q_lens, sub.seq_lens, **{**kw, "block_tables": sub.block_tables})
+    out = torch.empty_like(dw.q)
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
+    flush = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+    kev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    for e in kev:
+        e.record()
+    times = []
+    for i in range(steps + 3):
+        flush.sum()
+        api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, plan, sub.softmax_scale, sub.causal,
+                            out=out, workspace=ws, status=dw.status, kernel_events=kev)
+        torch.cuda.synchronize(dev)
+        if i >= 3:
+            times.append(kev[0].elapsed_time(kev[1]))
+    assert int(dw.status.item()) == 0
+    us = float(np.mean(times)) * 1e3
+    flops = prefill_flops(sub)
+    peak, kind = bf16_peak_tflops()
+    tflops = flops / (us * 1e-6) / 1e12
+    return {"workload": f"the {len(idx)} prefill chunks of {w.name} alone", "flops": flops, "us": us,
+            "tflops": tflops, "peak_tflops": peak, "peak_source": kind, "frac": tflops / peak,
+            "kernel": "attn_tc_kernel" if plan.info["num_tc_items"] else "attn_tma_kernel"}
 
 
 def run_e2e(args, w, dw, plan_opts, dev, stream, api):

@@ -174,6 +174,7 @@ typedef struct pkv_plan_info {
   int32_t num_partial_rows;     /* float32 partial rows of head_dim (+1 lse) in the workspace */
   int32_t num_groups;           /* shared-prefix groups found */
   int32_t num_ctas;             /* CTAs planned for */
+  int32_t num_tc_items;         /* of num_items: tiles of more than 16 rows for the tcgen05 kernel */
 } pkv_plan_info;
 
 /*
@@ -234,6 +235,22 @@ PKV_API pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q, in
                                size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * paged_attention_timed - pkv_paged_attention that also records two CUDA
+ * events (cudaEvent_t, created by the caller; either may be NULL) on `stream`:
+ * kernels_begin right before the attention kernels and kernels_end right after
+ * them, before the merge of split key ranges.  With events created for timing,
+ * cudaEventElapsedTime gives the attention kernels' own duration (also inside a
+ * captured graph).  Arguments, results and errors are otherwise those of
+ * pkv_paged_attention.
+ */
+PKV_API pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const void* q, int32_t q_dtype,
+                               int32_t num_q_heads, const int32_t* cu_q_lens, const int32_t* seq_lens,
+                               const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                               float softmax_scale, int32_t causal, const void* plan, void* out, float* out_lse,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream,
+                               void* kernels_begin, void* kernels_end);
+
+/*
  * split_kv_reduce - merge partial softmax states computed over disjoint key sets.
  *
  * The pages do not describe split-KV; this is the exact identity that splitting
@@ -266,7 +283,7 @@ PKV_API pkv_status pkv_split_kv_reduce(const float* partial_o, const float* part
  *   - The first call on a device looks up the array's address on that device;
  *     make it outside any stream capture.
  *   - All calls on a device share the array and it keeps the last call's
- *     contents (the counter is cleared on the stream by each call).  Calls that
+ *     contents (the work counters are cleared by each call's plan upload).  Calls that
  *     overlap on the GPU race; order them on one stream.
  *   - Allocates and frees nothing.
  */

@@ -60,7 +60,7 @@ class _PlanRequest(C.Structure):
 class _PlanInfo(C.Structure):
     _fields_ = [("plan_bytes", C.c_size_t), ("workspace_bytes", C.c_size_t), ("num_items", C.c_int32),
                 ("num_reduce", C.c_int32), ("num_parts", C.c_int32), ("num_partial_rows", C.c_int32),
-                ("num_groups", C.c_int32), ("num_ctas", C.c_int32)]
+                ("num_groups", C.c_int32), ("num_ctas", C.c_int32), ("num_tc_items", C.c_int32)]
 
 
 _P, _I32, _I64, _SZ, _F = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t, C.c_float
@@ -77,6 +77,9 @@ _lib.pkv_default_num_ctas.argtypes = [_I32, _I32, _I32, C.POINTER(_I32)]
 _lib.pkv_paged_attention.restype = _I32
 _lib.pkv_paged_attention.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P, _P, _P,
                                      _P, _SZ, _P, _P]
+_lib.pkv_paged_attention_timed.restype = _I32
+_lib.pkv_paged_attention_timed.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P, _P,
+                                           _P, _P, _SZ, _P, _P, _P, _P]
 _lib.pkv_paged_attention_noalloc.restype = _I32
 _lib.pkv_paged_attention_noalloc.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P,
                                              _P, _P, _P, _P]
@@ -222,18 +225,28 @@ def default_num_ctas(kv_dtype: int | str, head_dim: int, block_size: int) -> int
 def paged_attention(cache: Cache, q: torch.Tensor, cu_q_lens: torch.Tensor, seq_lens: torch.Tensor,
                     block_tables: torch.Tensor, plan: Plan, softmax_scale: float, causal: bool = True,
                     out: torch.Tensor | None = None, out_lse: torch.Tensor | None = None,
-                    workspace: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
-    """out = softmax(scale q K^T) V over the paged cache; returns ``out``."""
+                    workspace: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None,
+                    kernel_events=None):
+    """out = softmax(scale q K^T) V over the paged cache; returns ``out``.
+
+    ``kernel_events``: optional (begin, end) torch.cuda.Event pair recorded right
+    before and right after the attention kernels (pkv_paged_attention_timed).
+    """
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=q.device)
     c = cache._c()
-    _check(_lib.pkv_paged_attention(C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens), _ptr(seq_lens),
-                                    _ptr(block_tables), block_tables.shape[1], seq_lens.shape[0], float(softmax_scale),
-                                    int(bool(causal)), plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse),
-                                    _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
-           "paged_attention")
+    args = (C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens), _ptr(seq_lens), _ptr(block_tables),
+            block_tables.shape[1], seq_lens.shape[0], float(softmax_scale), int(bool(causal)), plan.buffer.data_ptr(),
+            _ptr(out), _ptr(out_lse), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    if kernel_events is None:
+        _check(_lib.pkv_paged_attention(*args), "paged_attention")
+    else:
+        handles = [e.cuda_event for e in kernel_events]
+        if not all(handles):
+            raise ValueError("kernel_events: record each event once before use (torch creates CUDA events lazily)")
+        _check(_lib.pkv_paged_attention_timed(*args, *handles), "paged_attention")
     return out
 
 

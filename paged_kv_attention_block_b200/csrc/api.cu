@@ -81,7 +81,9 @@ extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, i
 static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_rows, bool tc) {
   const char* base = reinterpret_cast<const char*>(h);
   const uint64_t bytes = h->bytes;
-  auto inside = [&](uint64_t off, uint64_t n, uint64_t sz) { return off + n * sz <= bytes; };
+  if (bytes < sizeof(PkvPlanHeader) + PKV_PLAN_COUNTER_BYTES || (bytes & 255))
+    return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan size %llu", (unsigned long long)bytes);
+  auto inside = [&](uint64_t off, uint64_t n, uint64_t sz) { return off + n * sz <= bytes - PKV_PLAN_COUNTER_BYTES; };
   if (h->n_items < 0 || h->n_tc_items < 0 || h->n_reduce < 0 || h->n_parts < 0 || h->n_part_rows < 0 ||
       h->total_q < 0 || !inside(h->items_off, h->n_items, sizeof(PkvItem)) ||
       !inside(h->tc_items_off, h->n_tc_items, sizeof(PkvItem)) || !inside(h->reduce_off, h->n_reduce, sizeof(PkvReduce)) ||
@@ -122,12 +124,23 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
   return PKV_OK;
 }
 
-extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
-                                          const int32_t* cu_q_lens, const int32_t* seq_lens,
-                                          const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
-                                          float softmax_scale, int32_t causal, const void* plan, void* out,
-                                          float* out_lse, void* workspace, size_t workspace_bytes,
-                                          int32_t* dev_status, void* stream) {
+// Under stream capture the record must be external, so that the graph records
+// the event each time it runs; outside capture it is a plain record.
+static cudaError_t record_event(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal)
+                                             : cudaEventRecord(ev, st);
+}
+
+extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const void* q, int32_t q_dtype,
+                                                int32_t num_q_heads, const int32_t* cu_q_lens,
+                                                const int32_t* seq_lens, const int32_t* block_tables,
+                                                int32_t max_blocks, int32_t num_seqs, float softmax_scale,
+                                                int32_t causal, const void* plan, void* out, float* out_lse,
+                                                void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                                void* stream, void* kernels_begin, void* kernels_end) {
   if (!cache || !plan) return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: cache and plan are required");
   const pkv_cache& c = *cache;
   const PkvPlanHeader* h = static_cast<const PkvPlanHeader*>(plan);
@@ -167,8 +180,8 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
+  // One copy uploads the plan and clears the work counters at its end.
   cudaError_t e = cudaMemcpyAsync(ws + L.plan_off, plan, h->bytes, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.counter_off, 0, L.counter_bytes, st);
   if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: plan upload: %s", cudaGetErrorString(e));
   const int resident = pkv::resident_ctas(k);  // also sets the kernel's shared-memory limit
   const int tc_resident = h->n_tc_items > 0 ? pkv::resident_ctas(ktc) : 1;
@@ -201,6 +214,10 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
   a.part_lse = reinterpret_cast<float*>(ws + L.part_lse_off);
   a.status = dev_status;
   a.max_rows = k.max_rows;
+  if (kernels_begin) {
+    e = record_event(static_cast<cudaEvent_t>(kernels_begin), st);
+    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));
+  }
   if (h->n_items > 0) {
     const int grid = std::max(1, std::min(std::min(resident, h->num_ctas), h->n_items));
     e = k.launch(a, grid, st);
@@ -215,6 +232,10 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
     const int grid = std::max(1, std::min(std::min(tc_resident, h->tc_num_ctas), h->n_tc_items));
     e = ktc.launch(t, grid, st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: tcgen05 launch failed: %s", cudaGetErrorString(e));
+  }
+  if (kernels_end) {
+    e = record_event(static_cast<cudaEvent_t>(kernels_end), st);
+    if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));
   }
   if (h->n_reduce > 0) {
     pkv::ReduceArgs r{};
@@ -233,4 +254,15 @@ extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q,
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: merge launch failed: %s", cudaGetErrorString(e));
   }
   return PKV_OK;
+}
+
+extern "C" pkv_status pkv_paged_attention(const pkv_cache* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                                          const int32_t* cu_q_lens, const int32_t* seq_lens,
+                                          const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                          float softmax_scale, int32_t causal, const void* plan, void* out,
+                                          float* out_lse, void* workspace, size_t workspace_bytes,
+                                          int32_t* dev_status, void* stream) {
+  return pkv_paged_attention_timed(cache, q, q_dtype, num_q_heads, cu_q_lens, seq_lens, block_tables, max_blocks,
+                                   num_seqs, softmax_scale, causal, plan, out, out_lse, workspace, workspace_bytes,
+                                   dev_status, stream, nullptr, nullptr);
 }

@@ -4,10 +4,15 @@
 // page-table lookup on KV writes).  fp8 pools store E4M3(x / scale) with
 // round-to-nearest-even and saturation (deep dive §13, fp8 KV cache).
 //
-// One thread moves one 8-element chunk of one (token, K|V, head) row: the
-// bytes are tiny next to attention, so the kernel only needs coalesced 8..32 B
-// accesses and a grid sized from the element count.
+// One warp per (token, K|V): lane 0 resolves the destination slot once (the
+// token's sequence by binary search over cu_new staged in shared memory, its
+// position, the block table entry), then the lanes move the token's rows for
+// every KV head in 16-byte (8-byte for fp8) pieces.  The bytes are tiny next
+// to attention; what costs is the chain of dependent index loads, kept to
+// three per unit.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
@@ -58,77 +63,105 @@ PKV_DEVICE void load8<__half>(const __half* src, float* x) {
   }
 }
 
-// Find s with cu[s] <= t < cu[s+1] (cu nondecreasing, cu[0] = 0).
+// Packed token t belongs to sequence s with cu[s] <= t < cu[s + 1] (binary search;
+// cu is in shared memory when the batch is small enough, else global memory).
 PKV_DEVICE int find_seq(const int32_t* cu, int n, int t) {
   int lo = 0, hi = n;  // invariant: cu[lo] <= t < cu[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(cu + mid) <= t) lo = mid; else hi = mid;
+    if (cu[mid] <= t) lo = mid; else hi = mid;
   }
   return lo;
 }
 
-// Same dtype in and out: move 16 bytes per thread.  ElemT is the element
-// type; the chunk holds 16 / sizeof(ElemT) elements.
+constexpr int kCuCache = 2048;  // sequences whose cu_new entries are staged in shared memory
+
+// One warp per (new token, K|V): lane 0 resolves the destination slot (sequence,
+// position, block table entry) once, then the warp moves the token's rows for
+// every KV head.  Returns the pool element offset of head 0's row, or -1 after
+// recording a device error.
+PKV_DEVICE int64_t append_target(const AppendArgs& a, const int32_t* cu, int t, int which, int lane) {
+  int64_t base = -1;
+  if (lane == 0) {
+    const int s = find_seq(cu, a.num_seqs, t);
+    const int p = __ldg(a.start_pos + s) + (t - cu[s]);
+    const int lb = p >> a.log2_block;
+    if (p < 0) {
+      report(a.status, PKV_DEV_BAD_APPEND);
+    } else if (lb >= a.max_blocks) {
+      report(a.status, PKV_DEV_BAD_LOGICAL_BLOCK);
+    } else {
+      const int phys = __ldg(a.block_tables + int64_t(s) * a.max_blocks + lb);
+      if (phys < 0 || phys >= a.num_blocks) {
+        report(a.status, PKV_DEV_BAD_BLOCK_ID);
+      } else {
+        const int slot = p & ((1 << a.log2_block) - 1);
+        base = ((((int64_t(phys) * a.num_layers + a.layer) * 2 + which) * a.hkv) << a.log2_block) + slot;
+        base *= a.head_dim;
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, base, 0);
+}
+
+PKV_DEVICE const int32_t* stage_cu(const AppendArgs& a, int32_t* s_cu) {
+  const bool cached = a.num_seqs < kCuCache;
+  if (cached)
+    for (int i = threadIdx.x; i <= a.num_seqs; i += blockDim.x) s_cu[i] = __ldg(a.cu_new + i);
+  __syncthreads();
+  return cached ? s_cu : a.cu_new;
+}
+
 template <int ELEM>
 __global__ void __launch_bounds__(256) kv_append_copy_kernel(AppendArgs a) {
-  constexpr int PER = 16 / ELEM;
-  const int chunks = a.head_dim / PER;
-  const int64_t total = int64_t(a.total_new) * 2 * a.hkv * chunks;
-  for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total; idx += int64_t(gridDim.x) * blockDim.x) {
-    int64_t r = idx;
-    const int c = int(r % chunks); r /= chunks;
-    const int h = int(r % a.hkv); r /= a.hkv;
-    const int which = int(r % 2);
-    const int t = int(r / 2);
-    const int s = find_seq(a.cu_new, a.num_seqs, t);
-    const int p = __ldg(a.start_pos + s) + (t - __ldg(a.cu_new + s));
-    if (p < 0) { report(a.status, PKV_DEV_BAD_APPEND); continue; }
-    const int lb = p >> a.log2_block;
-    if (lb >= a.max_blocks) { report(a.status, PKV_DEV_BAD_LOGICAL_BLOCK); continue; }
-    const int phys = __ldg(a.block_tables + int64_t(s) * a.max_blocks + lb);
-    if (phys < 0 || phys >= a.num_blocks) { report(a.status, PKV_DEV_BAD_BLOCK_ID); continue; }
-    const int slot = p & ((1 << a.log2_block) - 1);
-    const int64_t row = (((int64_t(phys) * a.num_layers + a.layer) * 2 + which) * a.hkv + h) * (int64_t(1) << a.log2_block) + slot;
-    const char* src = static_cast<const char*>(which ? a.v_new : a.k_new) + ((int64_t(t) * a.hkv + h) * a.head_dim + c * PER) * ELEM;
-    char* dst = static_cast<char*>(a.pool) + (row * a.head_dim + c * PER) * ELEM;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+  __shared__ int32_t s_cu[kCuCache + 1];
+  const int32_t* cu = stage_cu(a, s_cu);
+  constexpr int PER = 16 / ELEM;  // elements per 16-byte chunk
+  const int row_chunks = a.head_dim / PER;
+  const int chunks = a.hkv * row_chunks;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int u = blockIdx.x * 8 + warp; u < 2 * a.total_new; u += gridDim.x * 8) {
+    const int t = u >> 1, which = u & 1;
+    const int64_t base = append_target(a, cu, t, which, lane);
+    if (base < 0) continue;
+    const char* src = static_cast<const char*>(which ? a.v_new : a.k_new) + int64_t(t) * a.hkv * a.head_dim * ELEM;
+    char* dst = static_cast<char*>(a.pool) + base * ELEM;
+    for (int x = lane; x < chunks; x += 32) {
+      const int h = x / row_chunks, c = x % row_chunks;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (int64_t(h) * a.head_dim + c * PER) * ELEM));
+      *reinterpret_cast<uint4*>(dst + ((int64_t(h) << a.log2_block) * a.head_dim + c * PER) * ELEM) = v;
+    }
   }
 }
 
-// fp8 pool: 8 values per thread, quotient x / scale in float32, E4M3 RNE satfinite.
 template <typename Tin>
 __global__ void __launch_bounds__(256) kv_append_e4m3_kernel(AppendArgs a) {
-  const int chunks = a.head_dim / 8;
-  const int64_t total = int64_t(a.total_new) * 2 * a.hkv * chunks;
-  for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total; idx += int64_t(gridDim.x) * blockDim.x) {
-    int64_t r = idx;
-    const int c = int(r % chunks); r /= chunks;
-    const int h = int(r % a.hkv); r /= a.hkv;
-    const int which = int(r % 2);
-    const int t = int(r / 2);
-    const int s = find_seq(a.cu_new, a.num_seqs, t);
-    const int p = __ldg(a.start_pos + s) + (t - __ldg(a.cu_new + s));
-    if (p < 0) { report(a.status, PKV_DEV_BAD_APPEND); continue; }
-    const int lb = p >> a.log2_block;
-    if (lb >= a.max_blocks) { report(a.status, PKV_DEV_BAD_LOGICAL_BLOCK); continue; }
-    const int phys = __ldg(a.block_tables + int64_t(s) * a.max_blocks + lb);
-    if (phys < 0 || phys >= a.num_blocks) { report(a.status, PKV_DEV_BAD_BLOCK_ID); continue; }
-    const int slot = p & ((1 << a.log2_block) - 1);
-    const int64_t row = (((int64_t(phys) * a.num_layers + a.layer) * 2 + which) * a.hkv + h) * (int64_t(1) << a.log2_block) + slot;
-    const Tin* src = static_cast<const Tin*>(which ? a.v_new : a.k_new) + (int64_t(t) * a.hkv + h) * a.head_dim + c * 8;
-    const float scale = __ldg((which ? a.v_scale : a.k_scale) + a.layer * a.hkv + h);
-    float x[8];
-    load8<Tin>(src, x);
-    uint32_t lo = 0, hi = 0;
+  __shared__ int32_t s_cu[kCuCache + 1];
+  const int32_t* cu = stage_cu(a, s_cu);
+  const int row_chunks = a.head_dim / 8;  // 8 values -> 8 bytes
+  const int chunks = a.hkv * row_chunks;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int u = blockIdx.x * 8 + warp; u < 2 * a.total_new; u += gridDim.x * 8) {
+    const int t = u >> 1, which = u & 1;
+    const int64_t base = append_target(a, cu, t, which, lane);
+    if (base < 0) continue;
+    const Tin* src = static_cast<const Tin*>(which ? a.v_new : a.k_new) + int64_t(t) * a.hkv * a.head_dim;
+    uint8_t* dst = static_cast<uint8_t*>(a.pool) + base;
+    const float* scales = (which ? a.v_scale : a.k_scale) + a.layer * a.hkv;
+    for (int x = lane; x < chunks; x += 32) {
+      const int h = x / row_chunks, c = x % row_chunks;
+      const float scale = __ldg(scales + h);
+      float v[8];
+      load8<Tin>(src + int64_t(h) * a.head_dim + c * 8, v);
+      uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 v = make_float2(__fdiv_rn(x[2 * i], scale), __fdiv_rn(x[2 * i + 1], scale));
-      const uint32_t two = uint32_t(__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3));
-      if (i < 2) lo |= two << (16 * i); else hi |= two << (16 * (i - 2));
+      for (int i = 0; i < 4; ++i) {
+        const float2 q = make_float2(__fdiv_rn(v[2 * i], scale), __fdiv_rn(v[2 * i + 1], scale));
+        const uint32_t two = uint32_t(__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3));
+        if (i < 2) lo |= two << (16 * i); else hi |= two << (16 * (i - 2));
+      }
+      *reinterpret_cast<uint2*>(dst + (int64_t(h) << a.log2_block) * a.head_dim + c * 8) = make_uint2(lo, hi);
     }
-    uint8_t* dst = static_cast<uint8_t*>(a.pool) + row * a.head_dim + c * 8;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
   }
 }
 
@@ -165,9 +198,8 @@ extern "C" pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, c
                k_new, v_new, cu_new, start_pos, block_tables, max_blocks, num_seqs, total_new,
                c.k_scale, c.v_scale, dev_status};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int per = c.kv_dtype == PKV_FP8_E4M3 ? 8 : 16 / (c.kv_dtype == PKV_F32 ? 4 : 2);
-  const int64_t work = int64_t(total_new) * 2 * c.num_kv_heads * (c.head_dim / per);
-  const int grid = int(std::min<int64_t>((work + 255) / 256, 148 * 16));
+  // Eight (token, K|V) units per 256-thread block, one per warp.
+  const int grid = int(std::min<int64_t>((int64_t(total_new) * 2 + 7) / 8, 148 * 16));
   switch (c.kv_dtype) {
     case PKV_F32: kv_append_copy_kernel<4><<<grid, 256, 0, st>>>(a); break;
     case PKV_BF16:

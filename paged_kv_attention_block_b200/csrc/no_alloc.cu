@@ -17,8 +17,8 @@
 //     device (cudaGetSymbolAddress, with that device current).  Make that first
 //     call outside any stream capture.
 //   * Every call on a device uses the same array, and the array keeps whatever
-//     the last call left there.  The work counter is cleared on the stream at the
-//     start of each call; partial states are fully written before they are read.
+//     the last call left there.  The work counters are cleared by each call's plan
+//     upload; partial states are fully written before they are read.
 //     Calls whose work overlaps on the GPU (other streams, other host threads
 //     without ordering) race on the array: order them on one stream.
 //   * Nothing here allocates or frees memory.

@@ -206,7 +206,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   const uint64_t tc_items_off = items_off + (segs.size() - n_tc) * sizeof(PkvItem);
   const uint64_t reduce_off = items_off + segs.size() * sizeof(PkvItem);
   const uint64_t parts_off = reduce_off + reds.size() * sizeof(PkvReduce);
-  const uint64_t bytes = (parts_off + parts.size() * sizeof(int32_t) + 15) & ~uint64_t(15);
+  const uint64_t bytes = pkv_plan_bytes(parts_off + parts.size() * sizeof(int32_t));
   if (bytes > UINT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: plan too large");
   info->plan_bytes = bytes;
   info->workspace_bytes = pkv_workspace_layout(bytes, part_rows, D).total;
@@ -216,6 +216,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   info->num_partial_rows = int32_t(part_rows);
   info->num_groups = int32_t(groups.size());
   info->num_ctas = num_ctas;
+  info->num_tc_items = int32_t(n_tc);
   if (!plan) return PKV_OK;
   if (capacity < bytes) return pkv_fail(PKV_ERR_WORKSPACE, "attention_plan: capacity %zu < %llu", capacity, (unsigned long long)bytes);
 

@@ -80,19 +80,24 @@ struct PkvReduce {
 };
 static_assert(sizeof(PkvReduce) == 32, "reduce size");
 
-// Device workspace layout: [plan copy][work counters][partial o][partial lse].
-// The counters (one per kernel, 128 bytes apart) are cleared on the stream
-// before every call.
+// The plan buffer ends in a 256-byte block of zeros, 256-byte aligned: the
+// kernels' work counters (the register-tile kernel's at +0, the tensor-memory
+// kernel's at +128).  Uploading the plan therefore also clears the counters.
+#define PKV_PLAN_COUNTER_BYTES 256
 static inline uint64_t pkv_align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+// Plan bytes for a body (header, items, merges, parts) of `body` bytes.
+static inline uint64_t pkv_plan_bytes(uint64_t body) { return pkv_align256(body) + PKV_PLAN_COUNTER_BYTES; }
+
+// Device workspace layout: [plan copy with its counters][partial o][partial lse].
 struct PkvWorkspaceLayout {
   uint64_t plan_off, counter_off, counter_bytes, part_o_off, part_lse_off, total;
 };
 static inline PkvWorkspaceLayout pkv_workspace_layout(uint64_t plan_bytes, int64_t n_part_rows, int head_dim) {
   PkvWorkspaceLayout L;
   L.plan_off = 0;
-  L.counter_off = pkv_align256(plan_bytes);
-  L.counter_bytes = 256;  // counter of the register-tile kernel at +0, tensor-memory kernel at +128
-  L.part_o_off = L.counter_off + L.counter_bytes;
+  L.counter_off = plan_bytes - PKV_PLAN_COUNTER_BYTES;
+  L.counter_bytes = PKV_PLAN_COUNTER_BYTES;
+  L.part_o_off = pkv_align256(plan_bytes);
   L.part_lse_off = pkv_align256(L.part_o_off + uint64_t(n_part_rows) * head_dim * 4);
   L.total = pkv_align256(L.part_lse_off + uint64_t(n_part_rows) * 4);
   return L;

@@ -30,30 +30,65 @@ __global__ void __launch_bounds__(256) dense_reduce_kernel(const float* __restri
   }
 }
 
-__global__ void __launch_bounds__(256) plan_reduce_kernel(const ReduceArgs a) {
-  // Rows per merge come from the plan (up to PKV_TILE_ROWS_TC).
-  const int d = a.head_dim;
+// One warp per output row of a merge (a merge covers n_q tokens x g heads);
+// lane j merges head dims [VEC j, VEC (j + 1)) with the same per-element
+// arithmetic as merge_elem, so each lane issues VEC-wide loads of the parts.
+template <int D>
+__global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
+  constexpr int VEC = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = blockIdx.x; e < a.n_reduce; e += gridDim.x) {
     const PkvReduce red = a.reduces[e];
     const int R = red.n_q * a.g;
     const int32_t* parts = a.parts + red.parts_begin;
-    for (int x = threadIdx.x; x < R * d; x += blockDim.x) {
-      const int r = x / d, k = x % d;
-      float o, lse;
-      merge_elem(
-          red.n_parts, [&](int i) { return a.part_lse[int64_t(parts[i]) + r]; },
-          [&](int i) { return a.part_o[(int64_t(parts[i]) + r) * d + k]; }, o, lse);
+    const int n = red.n_parts;
+    for (int r = warp; r < R; r += 4) {
+      float M = -INFINITY;
+      for (int i = 0; i < n; ++i) M = fmaxf(M, __ldg(a.part_lse + int64_t(__ldg(parts + i)) + r));
+      float o[VEC], lse;
+      if (M == -INFINITY) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) o[v] = 0.f;
+        lse = -INFINITY;
+      } else {
+        float num[VEC], den = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) num[v] = 0.f;
+        for (int i = 0; i < n; ++i) {
+          const int64_t prow = int64_t(__ldg(parts + i)) + r;
+          const float li = __ldg(a.part_lse + prow);
+          if (li == -INFINITY) continue;
+          const float w = expf(li - M);
+          den += w;
+          const float* src = a.part_o + prow * D + lane * VEC;
+          float x[VEC];
+          if constexpr (VEC == 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(src));
+            x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+          } else {
+            const float2 f = __ldg(reinterpret_cast<const float2*>(src));
+            x[0] = f.x; x[1] = f.y;
+          }
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) num[v] = fmaf(w, x[v], num[v]);
+        }
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) o[v] = num[v] / den;
+        lse = M + logf(den);
+      }
       const int64_t orow = (int64_t(red.q_begin) + r / a.g) * a.hq + red.kv_head * a.g + r % a.g;
-      store_any(a.out, a.out_dtype, orow * d + k, o);
-      if (a.out_lse && k == 0) a.out_lse[orow] = lse;
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) store_any(a.out, a.out_dtype, orow * D + lane * VEC + v, o[v]);
+      if (a.out_lse && lane == 0) a.out_lse[orow] = lse;
     }
   }
 }
 
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st) {
   if (r.n_reduce <= 0) return cudaSuccess;
-  const int grid = std::min(r.n_reduce, 148 * 8);
-  plan_reduce_kernel<<<grid, 256, 0, st>>>(r);
+  const int grid = std::min(r.n_reduce, 148 * 16);
+  if (r.head_dim == 128) plan_reduce_kernel<128><<<grid, 128, 0, st>>>(r);
+  else plan_reduce_kernel<64><<<grid, 128, 0, st>>>(r);
   return cudaGetLastError();
 }
 
