@@ -298,25 +298,36 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, bufs[0], w.softmax_scale,
                                 w.causal, out=out, workspace=ws, status=dw.status)
     torch.cuda.synchronize(dev)
+    # The timed steps replay one graph per step (kv_append then paged_attention), one graph per
+    # plan buffer.  A second set splits the step into an append graph and an attention graph
+    # whose library call also records events around the attention kernels: the per-phase and
+    # kernel-only times come from replaying those one step at a time after the timed run (event
+    # record nodes inside the timed graphs would add latency to the step).
+    g_step = []
+    for b in bufs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            dw.append_new()
+            api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
+                                w.causal, out=out, workspace=ws, status=dw.status)
+        g_step.append(g)
     g_append = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_append, stream=stream):
         dw.append_new()
-    # Two sets of attention graphs: the timed steps run graphs without the kernel events (their
-    # record nodes would add latency to the step); the kernel-only timing runs graphs with them.
-    g_attn, g_attn_ev = [], []
-    for evs_, graphs in ((None, g_attn), (kev, g_attn_ev)):
-        for b in bufs:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
-                                    w.causal, out=out, workspace=ws, status=dw.status, kernel_events=evs_)
-            graphs.append(g)
+    g_attn_ev = []
+    for b in bufs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
+                                w.causal, out=out, workspace=ws, status=dw.status, kernel_events=kev)
+        g_attn_ev.append(g)
     done = [None, None]
     host_plan_s = 0.0
 
-    def step(i, evs=None, graphs=None):
+    def step(i, evs=None, split=False):
+        """One step; `evs` = (start, after append, end) events; split: the append and attention
+        graphs (the latter with kernel events) instead of the one-graph step."""
         nonlocal host_plan_s
-        graphs = graphs or g_attn
         slot = i % 2
         if done[slot] is not None:
             done[slot].synchronize()  # the upload that read this buffer has run
@@ -327,10 +338,13 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             flush.sum()
             if evs:
                 evs[0].record(stream)
-            g_append.replay()
-            if evs:
-                evs[1].record(stream)
-            graphs[slot].replay()
+            if split:
+                g_append.replay()
+                if evs:
+                    evs[1].record(stream)
+                g_attn_ev[slot].replay()
+            else:
+                g_step[slot].replay()
             if evs:
                 evs[2].record(stream)
             e = torch.cuda.Event()
@@ -343,6 +357,8 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    nsplit = min(args.steps, 300)
+    ev_split = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(nsplit)]
     host_plan_s = 0.0
     with ClockSampler(local_rank) as clocks:
         torch.cuda.synchronize(dev)
@@ -352,19 +368,19 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
         if world > 1:
             dist.barrier()
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
-    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
     ms = float(np.mean(step_ms))
-    attn = float(np.mean(attn_ms))
-    # The attention kernels' own duration: the same steps, one at a time, each read back after it ran.
+    # Per phase and the attention kernels' own duration: the same steps from the split graphs,
+    # one at a time, each read back after it ran.
     kern_ms = []
-    for i in range(min(args.steps, 300)):
-        step(i, graphs=g_attn_ev)
+    for i in range(nsplit):
+        step(i, ev_split[i], split=True)
         torch.cuda.synchronize(dev)
         kern_ms.append(kev[0].elapsed_time(kev[1]))
+    attn = float(np.mean([b.elapsed_time(c) for _, b, c in ev_split]))
     kern = float(np.mean(kern_ms))
     ms, attn, kern = max_over_ranks([ms, attn, kern], dev)
     assert int(dw.status.item()) == 0, "device status set during the benchmark"
-    del g_append, g_attn, g_attn_ev
+    del g_step, g_append, g_attn_ev
     prefill = run_prefill_only(w, dev, api, runner, plan_kw) if rank == 0 and prefill_flops(w) > 0 else None
 
     b = algorithmic_bytes(w, plan.info)

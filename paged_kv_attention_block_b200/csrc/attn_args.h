@@ -64,4 +64,22 @@ bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataTyp
                    CUtensorMap* map);
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st);
 
+// Launch `kernel` with programmatic stream serialization: it may begin while the
+// kernel ahead of it on the stream is still running (and must call pdl_wait
+// before it depends on that kernel's results).
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace pkv

@@ -180,6 +180,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // This kernel may start while the decode-tile kernel ahead of it is still running: it reads
+  // nothing that kernel writes (and waits for it before finishing, below).
   if (warp == 0) tc::alloc(smem_addr(&s_tmem), T::TMEM_COLS);
   float* xchg = reinterpret_cast<float*>(base_ptr + T::XCHG_OFF);
   if (tid == 32) {
@@ -299,6 +301,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       }
       if (!ok) break;
     }
+    pdl_trigger();  // every item of this CTA is claimed: the split merge may be scheduled
     if (!ok && lane == 0) {
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;
@@ -581,6 +584,9 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     __syncwarp();
     tc::fence_after_sync();
     tc::dealloc(tmem, T::TMEM_COLS);
+    // The grid finishes only after the kernel ahead of it, so the merge that waits for this
+    // grid also sees that kernel's partial states.
+    if (lane == 0) pdl_wait();
   }
 }
 
@@ -594,8 +600,9 @@ cudaError_t launch_tc(const AttnArgs& a, int grid, cudaStream_t st) {
   if (!make_pool_map(a, D, 2, BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, box_rows, 1,
                      &map))
     return cudaErrorInvalidValue;
-  attn_tc_kernel<D, BF><<<grid, T::THREADS, T::SMEM, st>>>(map, TcArgs{a, box_rows});
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(attn_tc_kernel<D, BF>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map,
+                                   TcArgs{a, box_rows});
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D, bool BF>

@@ -459,6 +459,10 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       q = __shfl_sync(0xffffffffu, q, 0);
       if (!ok) break;
     }
+    // Every item of this CTA is claimed: the kernels after this one on the stream (tcgen05
+    // tiles, split merge) may be scheduled as the CTAs drain.  The tcgen05 kernel reads nothing
+    // this one writes, and the merge waits for it to finish.
+    pdl_trigger();
     if (!ok && lane == 0) {
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;

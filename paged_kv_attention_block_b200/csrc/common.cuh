@@ -106,6 +106,15 @@ PKV_DEVICE float fast_exp2(float x) {
   return y;
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+// A grid launched with programmatic stream serialization may start before the
+// kernel ahead of it on the stream has finished.  pdl_wait blocks until that
+// kernel has completed and its memory operations are visible; pdl_trigger lets
+// this grid's dependent be scheduled before this grid finishes (each CTA
+// triggers; a CTA that exits counts as triggered).
+PKV_DEVICE void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+PKV_DEVICE void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- packed float pairs (sm_100 f32x2 arithmetic) and an FMA-pipe exp2 -----
 
 PKV_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {

@@ -37,6 +37,7 @@ template <int D>
 __global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
   constexpr int VEC = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();  // launched as a dependent of the attention kernels: their partial states are complete
   for (int e = blockIdx.x; e < a.n_reduce; e += gridDim.x) {
     const PkvReduce red = a.reduces[e];
     const int R = red.n_q * a.g;
@@ -87,8 +88,9 @@ __global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st) {
   if (r.n_reduce <= 0) return cudaSuccess;
   const int grid = std::min(r.n_reduce, 148 * 16);
-  if (r.head_dim == 128) plan_reduce_kernel<128><<<grid, 128, 0, st>>>(r);
-  else plan_reduce_kernel<64><<<grid, 128, 0, st>>>(r);
+  const cudaError_t e = r.head_dim == 128 ? launch_pdl(plan_reduce_kernel<128>, dim3(grid), dim3(128), 0, st, r)
+                                           : launch_pdl(plan_reduce_kernel<64>, dim3(grid), dim3(128), 0, st, r);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
