@@ -163,6 +163,10 @@ typedef struct pkv_plan_request {
   const int32_t* cu_q_lens;     /* host int32 [num_seqs+1] */
   const int32_t* seq_lens;      /* host int32 [num_seqs] */
   const int32_t* block_tables;  /* host int32 [num_seqs][max_blocks]; NULL disables cascade */
+  int32_t window;               /* limited attention window (deep dive §11: tokens outside the window
+                                   no longer take part in attention): query row at position p sees keys
+                                   p - window < t <= p.  0 = no limit.  Needs causal; disables cascade.
+                                   The plan carries it to pkv_paged_attention. */
 } pkv_plan_request;
 
 typedef struct pkv_plan_info {

@@ -28,6 +28,9 @@ What it computes, step by step, with the passage each step follows:
   for keys ``t <= p`` (all ``t < seq_len`` when not causal), then the plain
   softmax ``w = exp(z - max z) / sum`` and ``o = sum_t w_t v_t``; also
   ``lse = max z + ln sum exp(z - max z)``.  No tiling, no online softmax.
+  With a limited attention window ``W`` (deep dive §11, "有限attention window":
+  tokens outside the window no longer take part in attention), row ``j`` sees
+  only the ``W`` most recent positions up to its own: keys ``p - W < t <= p``.
 * ``split_kv_reduce``: partial states over disjoint key sets ``(o_i, lse_i)``
   (``o_i`` normalised, natural-log ``lse_i``; an empty set has ``lse = -inf``)
   merge as ``M = max lse_i``, ``w_i = exp(lse_i - M)``, ``o = sum w_i o_i / sum
@@ -48,7 +51,7 @@ import numpy as np
 
 __all__ = [
     "E4M3_MAX", "e4m3_decode", "e4m3_encode", "decode_bits", "kv_head_of", "block_address",
-    "key_limit", "OraclePool", "new_pool", "kv_append", "gather_rows", "paged_attention",
+    "key_limit", "key_start", "OraclePool", "new_pool", "kv_append", "gather_rows", "paged_attention",
     "attention_row_probs", "split_kv_reduce", "sentinel_bits",
 ]
 
@@ -158,6 +161,14 @@ def key_limit(seq_len: int, q_len: int, j, causal: bool):
     return seq_len - q_len + j + 1
 
 
+def key_start(seq_len: int, q_len: int, j, window: int):
+    """First key query row ``j`` may attend to: 0, or ``p - W + 1`` under a window ``W``."""
+    j = np.asarray(j)
+    if window <= 0:
+        return np.zeros(j.shape, dtype=np.int64)
+    return np.maximum(0, seq_len - q_len + j + 1 - window)
+
+
 class OraclePool:
     """Host copy of a pool: ``bits[num_blocks][num_layers][2][Hkv][B][D]`` in storage bits."""
 
@@ -238,13 +249,16 @@ def _softmax_rows(z: np.ndarray):
 
 
 def paged_attention(pool: OraclePool, layer: int, q: np.ndarray, cu_q_lens, seq_lens, block_tables,
-                    num_q_heads: int, softmax_scale: float, causal: bool = True, seqs=None):
+                    num_q_heads: int, softmax_scale: float, causal: bool = True, seqs=None, window: int = 0):
     """softmax(scale * q K^T) V over each sequence's paged K/V.
 
     ``q`` is float64 ``[T_q][Hq][D]`` (already decoded).  Returns ``(out, lse)``
     with ``out`` float64 ``[T_q][Hq][D]`` and ``lse`` float64 ``[T_q][Hq]``; rows
-    of sequences outside ``seqs`` stay NaN.
+    of sequences outside ``seqs`` stay NaN.  ``window`` > 0 (causal only) limits
+    every row to its ``window`` most recent positions.
     """
+    if window > 0 and not causal:
+        raise ValueError("a window needs causal positions")
     T, Hq, D = q.shape
     Hkv = pool.num_kv_heads
     out = np.full((T, Hq, D), np.nan)
@@ -256,6 +270,7 @@ def paged_attention(pool: OraclePool, layer: int, q: np.ndarray, cu_q_lens, seq_
         if ql == 0:
             continue
         lim = key_limit(L, ql, np.arange(ql), causal)
+        lo = key_start(L, ql, np.arange(ql), window)
         kv_cache = {}
         for h in range(Hq):
             kvh = int(kv_head_of(h, num_q_heads, Hkv))
@@ -264,7 +279,8 @@ def paged_attention(pool: OraclePool, layer: int, q: np.ndarray, cu_q_lens, seq_
                                  gather_rows(pool, layer, block_tables[s], kvh, 1, L))
             K, V = kv_cache[kvh]
             z = softmax_scale * (q[q0:q1, h, :] @ K.T)
-            z = np.where(np.arange(L)[None, :] < lim[:, None], z, -np.inf)
+            t = np.arange(L)[None, :]
+            z = np.where((t < lim[:, None]) & (t >= lo[:, None]), z, -np.inf)
             w, m, l = _softmax_rows(z)
             out[q0:q1, h, :] = (w @ V) / l[:, None]
             lse[q0:q1, h] = m + np.log(l)
@@ -272,14 +288,16 @@ def paged_attention(pool: OraclePool, layer: int, q: np.ndarray, cu_q_lens, seq_
 
 
 def attention_row_probs(pool: OraclePool, layer: int, q: np.ndarray, cu_q_lens, seq_lens, block_tables,
-                        num_q_heads: int, softmax_scale: float, causal: bool, s: int, j: int, h: int):
+                        num_q_heads: int, softmax_scale: float, causal: bool, s: int, j: int, h: int,
+                        window: int = 0):
     """The probability row of one query (sequence ``s``, row ``j``, head ``h``), float64 [seq_len]."""
     L = int(seq_lens[s])
     ql = int(cu_q_lens[s + 1] - cu_q_lens[s])
     kvh = int(kv_head_of(h, num_q_heads, pool.num_kv_heads))
     K = gather_rows(pool, layer, block_tables[s], kvh, 0, L)
     z = softmax_scale * (K @ q[int(cu_q_lens[s]) + j, h, :])
-    z = np.where(np.arange(L) < key_limit(L, ql, j, causal), z, -np.inf)
+    t = np.arange(L)
+    z = np.where((t < key_limit(L, ql, j, causal)) & (t >= key_start(L, ql, j, window)), z, -np.inf)
     w = np.exp(z - z.max())
     return w / w.sum()
 

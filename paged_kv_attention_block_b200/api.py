@@ -54,7 +54,7 @@ class _PlanRequest(C.Structure):
                 ("head_dim", C.c_int32), ("block_size", C.c_int32), ("kv_dtype", C.c_int32), ("causal", C.c_int32),
                 ("num_ctas", C.c_int32), ("kv_split", C.c_int32), ("cascade", C.c_int32),
                 ("min_shared_tokens", C.c_int32), ("max_blocks", C.c_int32), ("cu_q_lens", C.c_void_p),
-                ("seq_lens", C.c_void_p), ("block_tables", C.c_void_p)]
+                ("seq_lens", C.c_void_p), ("block_tables", C.c_void_p), ("window", C.c_int32)]
 
 
 class _PlanInfo(C.Structure):
@@ -186,8 +186,11 @@ def _host_i32(x) -> np.ndarray:
 def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
                    kv_dtype: int | str, causal: bool = True, block_tables=None, max_blocks: int | None = None,
                    num_ctas: int = 0, kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0,
-                   pin: bool = True, buffer: torch.Tensor | None = None) -> Plan:
+                   pin: bool = True, buffer: torch.Tensor | None = None, window: int = 0) -> Plan:
     """Build the work list for one paged_attention call from host copies of the lengths.
+
+    ``window`` > 0 limits every (causal) row to its ``window`` most recent positions; the
+    plan carries it to ``paged_attention``.
 
     ``buffer`` (uint8, host) is reused when large enough; the caller must not
     reuse a buffer whose plan upload may still be pending on the GPU.
@@ -200,7 +203,7 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
     code = DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
     req = _PlanRequest(sl.shape[0], num_q_heads, num_kv_heads, head_dim, block_size, code, int(bool(causal)), num_ctas,
                        kv_split, int(bool(cascade)), min_shared_tokens, max_blocks, cu.ctypes.data, sl.ctypes.data,
-                       None if bt is None else bt.ctypes.data)
+                       None if bt is None else bt.ctypes.data, int(window))
     info = _PlanInfo()
     _check(_lib.pkv_attention_plan(C.byref(req), None, 0, C.byref(info)), "attention_plan")
     if buffer is not None and buffer.numel() >= int(info.plan_bytes):

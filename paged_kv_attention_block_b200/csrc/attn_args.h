@@ -29,6 +29,7 @@ struct AttnArgs {
   float* part_lse;        // [n_part_rows]
   int32_t* status;
   int32_t max_rows;       // rows per item this kernel accepts
+  int32_t window;         // limited attention window (causal rows see keys pos - window < t <= pos); 0 = none
 };
 
 struct ReduceArgs {

@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
       }
       const int lim = it.pos0 >= 0 ? min(it.k_end, it.pos0 + r / a.g + 1) : it.k_end;
       float m = -INFINITY, l = 0.f;
-      for (int t = it.k_begin; t < lim; ++t) {
+      for (int t = max(it.k_begin, window_start(a.window, it.pos0 >= 0 ? it.pos0 + r / a.g : -1)); t < lim; ++t) {
         const int phys = __ldg(bt_row + (t >> a.log2_block));
         if (phys < 0 || phys >= a.num_blocks) {
           if (lane == 0) report(a.status, PKV_DEV_BAD_BLOCK_ID);

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(128, 2) attn_mma_kernel(const AttnArgs a) {
     for (int hh = 0; hh < 2; ++hh) {
       const int r = c.row_base + g4 + 8 * hh;
       c.lim[hh] = (it.pos0 >= 0 && r < c.R) ? min(it.k_end, it.pos0 + r / c.g + 1) : it.k_end;
+      c.lo[hh] = window_start(a.window, (it.pos0 >= 0 && r < c.R) ? it.pos0 + r / c.g : -1);
       c.m[hh] = -INFINITY;
       c.l[hh] = 0.f;
     }

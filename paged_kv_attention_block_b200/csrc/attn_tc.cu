@@ -421,6 +421,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     const bool to_part = d.part_row >= 0;
     const int last_valid = d.k_end - (d.k_begin + (ntiles - 1) * T::TK);  // keys of the last tile in range
     const int lim = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / a.g + 1) : d.k_end;
+    const int lo = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / a.g : -1);
 
     // The previous item's MMAs are complete (its epilogue waited for the last P V): Q is free.
     tc_stage_q<D>(a, d, R, q_tm, r, hf);
@@ -443,10 +444,10 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         tc::keep_after_wait<T::HALF>(u);
       }
       const int key0 = d.k_begin + t * T::TK + hf * T::HALF;
-      if (key0 + T::HALF > lim) {
+      if (key0 + T::HALF > lim || key0 < lo) {
 #pragma unroll
         for (int j = 0; j < T::HALF; ++j)
-          if (key0 + j >= lim) s[j] = -INFINITY;
+          if (key0 + j >= lim || key0 + j < lo) s[j] = -INFINITY;
       }
       // Max of this half over 8 independent chains, then of the row with the partner's.
       float mx8[8];

@@ -33,6 +33,7 @@ struct ItemCtx {
   using C = Cfg<D, KV, QBF>;
   int R, row_base, g;
   int lim[2];          // exclusive key bound of rows g4 and g4 + 8
+  int lo[2];           // first key of rows g4 and g4 + 8 (limited attention window)
   float m[2], l[2];    // running max (log2 domain) and partial sum per row
   float acc[C::NNT][4];
   uint32_t qf[C::NKS][4];
@@ -112,7 +113,7 @@ PKV_DEVICE void compute_keys(const AttnArgs& a, ItemCtx<D, KV, QBF>& c, uint32_t
     for (int e = 0; e < 4; ++e) {
       const int hh = e >> 1;
       const int key = key0 + kt0 + 8 * nt + 2 * t4 + (e & 1);
-      const float v = key < c.lim[hh] ? s[nt][e] * scale_log2 : -INFINITY;
+      const float v = (key < c.lim[hh] && key >= c.lo[hh]) ? s[nt][e] * scale_log2 : -INFINITY;
       s[nt][e] = v;
       mx[hh] = fmaxf(mx[hh], v);
     }

@@ -96,6 +96,7 @@ struct DecState {
   float m[NR][2], l[NR][2];  // rows 2*t4 + b (+8*group); m in scaled-log2 units
   uint32_t qb[NR][D / 16][2];
   int lim[NR][2];
+  int lo[NR][2];  // first visible key (limited attention window)
 };
 
 template <int KV>
@@ -209,7 +210,10 @@ PKV_DEVICE void dec_tile(DecState<D, KV, QBF, NR>& st, const DecOffsets<D, KV, Q
       for (int kt = 0; kt < NKT; ++kt)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (key0 + kt * 16 + g4 + 8 * (e >> 1) >= st.lim[nr][e & 1]) s[nr][kt][e] = -INFINITY;
+        {
+          const int key = key0 + kt * 16 + g4 + 8 * (e >> 1);
+          if (key >= st.lim[nr][e & 1] || key < st.lo[nr][e & 1]) s[nr][kt][e] = -INFINITY;
+        }
   }
   // Running max per query row (in raw score units, then scaled), exp2 of the scaled scores.
 #pragma unroll
@@ -504,18 +508,21 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
         constexpr int NR = decltype(nr_tag)::value;
         DecState<D, KV, QBF, NR> st;
         dec_load_q<D, KV, QBF, NR>(a, d, R, st, g4, t4);
-        int lim_min = d.k_end;
+        int lim_min = d.k_end, lo_max = 0;
 #pragma unroll
         for (int nr = 0; nr < NR; ++nr)
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             const int r = nr * 8 + 2 * t4 + b;
             st.lim[nr][b] = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / a.g + 1) : d.k_end;
+            st.lo[nr][b] = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / a.g : -1);
             lim_min = min(lim_min, st.lim[nr][b]);
+            lo_max = max(lo_max, st.lo[nr][b]);
             st.m[nr][b] = -INFINITY;
             st.l[nr][b] = 0.f;
           }
         lim_min = __reduce_min_sync(0xffffffffu, lim_min);
+        lo_max = __reduce_max_sync(0xffffffffu, lo_max);
 #pragma unroll
         for (int nr = 0; nr < NR; ++nr)
 #pragma unroll
@@ -532,7 +539,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             fence_proxy_async_smem();
           }
           const int key0 = d.k_begin + t * T::TK;
-          dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, key0, lane, c, key0 + T::TK > lim_min);
+          dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, key0, lane, c, key0 + T::TK > lim_min || key0 < lo_max);
           __syncwarp();
           if (lane == 0) mbar_arrive(empty_bar(stg), 4);
         }
@@ -599,8 +606,9 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       mbar_arrive(merge_bar, 1);
       if (!mbar_wait(merge_bar, merge_phase)) ok = false;
       merge_phase ^= 1;
-    } else {
-      // ---- prefill tile: every warp reads every tile, 16 rows per warp.
+    } else if constexpr (KV == KV_E4M3) {
+      // ---- prefill tile (fp8 pools; 16-bit pools send these to the tcgen05 kernel):
+      // every warp reads every tile, 16 rows per warp.
       ItemCtx<D, KV, QBF> cx;
       cx.g = a.g;
       cx.R = R;
@@ -612,6 +620,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       for (int hh = 0; hh < 2; ++hh) {
         const int r = cx.row_base + g4 + 8 * hh;
         cx.lim[hh] = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / cx.g + 1) : d.k_end;
+        cx.lo[hh] = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / cx.g : -1);
         cx.m[hh] = -INFINITY;
         cx.l[hh] = 0.f;
       }
@@ -721,8 +730,9 @@ cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
 template <int D, int KV, bool QBF>
 AttnKernel tma_kernel() {
   using T = TmaCfg<D, KV, QBF>;
+  // 16-bit pools: only decode-sized tiles (larger ones are tcgen05 items); fp8: up to 64 rows.
   return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF>), T::THREADS, T::SMEM,
-                    &launch_tma<D, KV, QBF>, PKV_TILE_ROWS};
+                    &launch_tma<D, KV, QBF>, KV == KV_E4M3 ? PKV_TILE_ROWS : PKV_DECODE_ROWS};
 }
 
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {

@@ -106,6 +106,11 @@ PKV_DEVICE float fast_exp2(float x) {
   return y;
 }
 
+// First key a causal row at position pos may see under a limited attention
+// window (keys pos - window < t <= pos); 0 without a window or for rows that
+// have no position (non-causal, padding).
+PKV_DEVICE int window_start(int window, int pos) { return (window > 0 && pos >= 0) ? pos + 1 - window : 0; }
+
 // ---- programmatic dependent launch -------------------------------------------
 // A grid launched with programmatic stream serialization may start before the
 // kernel ahead of it on the stream has finished.  pdl_wait blocks until that

@@ -60,6 +60,10 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (req->kv_dtype < PKV_F32 || req->kv_dtype > PKV_FP8_E4M3) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: kv_dtype");
   if (S > 0 && (!req->cu_q_lens || !req->seq_lens)) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: null length arrays");
   if (S > 0 && req->max_blocks <= 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: max_blocks");
+  const int window = req->window;
+  if (window < 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: window %d < 0", window);
+  if (window > 0 && !req->causal)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: a limited attention window needs causal rows");
   const int32_t* cu = req->cu_q_lens;
   const int32_t* L = req->seq_lens;
   if (S > 0 && cu[0] != 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: cu_q_lens[0] != 0");
@@ -90,7 +94,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   struct Group { int first, last, tokens; };
   std::vector<Group> groups;
   std::vector<int> group_of(S, -1);
-  if (req->cascade && req->block_tables && S > 1) {
+  // A window would cut the shared prefix differently for every member: no groups then.
+  if (req->cascade && req->block_tables && S > 1 && window == 0) {
     const int32_t* bt = req->block_tables;
     const int64_t mb = req->max_blocks;
     const int min_sh = req->min_shared_tokens > 0 ? req->min_shared_tokens : 256;
@@ -152,10 +157,13 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       const int n = std::min(QT, ql - i0);
       const int ke = causal ? L[s] - ql + i0 + n : L[s];
       const int pos0 = causal ? L[s] - ql + i0 : -1;
+      // Under a window the tile's first row sees keys from pos0 - window + 1 on; the range starts
+      // there, rounded down to 128 keys (the kernels' tile alignment), and rows mask the rest.
+      const int k0 = window > 0 ? std::max(kb, int(std::max(0, pos0 - window + 1) / 128 * 128)) : kb;
       for (int h = 0; h < Hkv; ++h) {
         const int gp = group_of[s] >= 0 ? int(gpart[size_t(s) * Hkv + h]) : -1;
-        Unit u{s, h, cu[s] + i0, n, kb, ke, pos0, gp, row_weight(n * g)};
-        total_cost[is_tc(n * g)] += double(std::max(0, ke - kb)) * u.weight;
+        Unit u{s, h, cu[s] + i0, n, k0, ke, pos0, gp, row_weight(n * g)};
+        total_cost[is_tc(n * g)] += double(std::max(0, ke - k0)) * u.weight;
         units.push_back(u);
       }
     }
@@ -229,6 +237,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.n_tc_items = int32_t(n_tc);
   h.tc_items_off = uint32_t(tc_items_off);
   h.tc_num_ctas = tc_ctas;
+  h.window = window;
   h.n_reduce = info->num_reduce;
   h.n_parts = info->num_parts;
   h.n_part_rows = info->num_partial_rows;

@@ -44,7 +44,8 @@ struct PkvPlanHeader {
   int32_t n_tc_items;    // tensor-memory items (attn_tc kernel), after the others
   uint32_t tc_items_off;
   int32_t tc_num_ctas;   // CTAs planned for the tensor-memory kernel
-  int32_t pad[10];       // header is 128 bytes
+  int32_t window;        // limited attention window in positions; 0 = none
+  int32_t pad[9];        // header is 128 bytes
 };
 static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 

@@ -76,7 +76,8 @@ class DeviceWorkload:
             self._plan_events[i].synchronize()  # that buffer's upload has run
         p = api.plan_attention(w.cu_q_lens, w.seq_lens, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
                                head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal,
-                               block_tables=w.block_tables, buffer=self._plan_bufs[i], **opts)
+                               block_tables=w.block_tables, buffer=self._plan_bufs[i],
+                               **({"window": w.window} if w.window else {}), **opts)
         self._plan_bufs[i] = p.buffer
         p.slot = i
         self._plan_slot = (i + 1) % len(self._plan_bufs)

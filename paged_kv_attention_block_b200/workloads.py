@@ -92,6 +92,7 @@ class Workload:
     shared_prefix_tokens: int
     k_scale: np.ndarray | None = None  # [num_layers][Hkv] float32, fp8 only
     v_scale: np.ndarray | None = None
+    window: int = 0  # limited attention window (positions); 0 = every cached key
     _kv_cache: dict = field(default_factory=dict, repr=False)
     _q: np.ndarray | None = field(default=None, repr=False)
 
@@ -249,6 +250,7 @@ def build(
     num_layers: int = 1,
     layer: int = 0,
     causal: bool = True,
+    window: int = 0,
     softmax_scale: float | None = None,
     table_slack: int = 0,
     threads: int | None = None,
@@ -287,7 +289,7 @@ def build(
         name=name, seed=seed, kv_dtype=kv_dtype, q_dtype=q_dtype, kv_in_dtype=kv_in_dtype,
         num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B,
         num_blocks=int(num_blocks), num_layers=num_layers, layer=layer, seq_lens=seq_lens,
-        q_lens=q_lens, block_tables=bt, softmax_scale=float(softmax_scale), causal=causal,
+        q_lens=q_lens, block_tables=bt, softmax_scale=float(softmax_scale), causal=causal, window=int(window),
         data_scale=data_scale, shared_prefix_tokens=shared_prefix_tokens,
     )
     if kv_dtype == "e4m3":

@@ -25,7 +25,7 @@ def oracle_pool(w: W.Workload, seqs=None) -> O.OraclePool:
 def oracle_out(w: W.Workload, pool: O.OraclePool, seqs=None):
     q = O.decode_bits(w.q, w.q_dtype) if w.q_dtype != "f32" else w.q.astype(np.float64)
     return O.paged_attention(pool, w.layer, q, w.cu_q_lens, w.seq_lens, w.block_tables, w.num_q_heads,
-                             w.softmax_scale, w.causal, seqs=seqs)
+                             w.softmax_scale, w.causal, seqs=seqs, window=w.window)
 
 
 def gpu_out_f64(t: torch.Tensor) -> np.ndarray:

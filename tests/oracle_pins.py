@@ -50,7 +50,7 @@ def q64(w: W.Workload) -> np.ndarray:
 def run_oracle(w: W.Workload, pool=None):
     pool = pool if pool is not None else oracle_pool_for(w)
     return O.paged_attention(pool, w.layer, q64(w), w.cu_q_lens, w.seq_lens, w.block_tables, w.num_q_heads,
-                             w.softmax_scale, w.causal)
+                             w.softmax_scale, w.causal, window=w.window)
 
 
 def _values64(w: W.Workload, s: int):
@@ -86,6 +86,8 @@ def dense_sdpa(w: W.Workload):
         Q = torch.from_numpy(np.ascontiguousarray(qq[cu[s]:cu[s + 1]].transpose(1, 0, 2)))
         pos = L - ql + torch.arange(ql)
         mask = torch.arange(L)[None, :] <= pos[:, None] if w.causal else torch.ones(ql, L, dtype=torch.bool)
+        if w.window:
+            mask &= torch.arange(L)[None, :] > pos[:, None] - w.window
         o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=w.softmax_scale)
         out[cu[s]:cu[s + 1]] = o.numpy().transpose(1, 0, 2)
     return out
@@ -397,8 +399,72 @@ def pin_prefix_sharing():
     assert np.array_equal(shared, private)
 
 
+# ---------------------------------------------------------------------------
+# Limited attention window (deep dive §11)
+# ---------------------------------------------------------------------------
+
+def pin_window_dense():
+    """Banded causal mask on the contiguous layout (torch SDPA) for several windows."""
+    for W_ in (1, 3, 17, 70):
+        for w in (W.mixed_bf16(n_decode=3, n_prefill=2, chunk=40, dec_lo=30, dec_hi=300, cached_lo_blocks=1,
+                               cached_hi_blocks=3, block_size=16),
+                  W.longctx_fp8(batch=2, seq_len=150)):
+            w.window = W_
+            out, _ = run_oracle(w)
+            assert np.abs(out - dense_sdpa(w)).max() <= 1e-12, (w.name, W_)
+
+
+def pin_window_limits():
+    """A window of one position leaves only the row's own token (o = v_p exactly); a window at
+    least as long as the sequence changes nothing, bit for bit."""
+    w = W.mixed_bf16(n_decode=3, n_prefill=2, chunk=24, dec_lo=20, dec_hi=90, cached_lo_blocks=1,
+                     cached_hi_blocks=2, block_size=16)
+    pool = oracle_pool_for(w)
+    full, full_lse = run_oracle(w, pool)
+    w.window = int(w.seq_lens.max())
+    same, same_lse = run_oracle(w, pool)
+    assert np.array_equal(full, same) and np.array_equal(full_lse, same_lse)
+    w.window = 1
+    one, _ = run_oracle(w, pool)
+    g = w.num_q_heads // w.num_kv_heads
+    for s in range(w.num_seqs):
+        k, v = _values64(w, s)
+        L, ql = int(w.seq_lens[s]), int(w.q_lens[s])
+        for j in range(ql):
+            tok = int(w.cu_q_lens[s]) + j
+            for h in range(w.num_q_heads):
+                assert np.array_equal(one[tok, h], v[L - ql + j, h // g]), (s, j, h)
+
+
+def pin_window_brute_force():
+    """Pure-Python loops with a window of 3 on a tiny mixed batch."""
+    w = W.build("brute_w", seed=6, kv_dtype="f32", num_q_heads=4, num_kv_heads=2, head_dim=3, block_size=2,
+                seq_lens=[7, 5], q_lens=[4, 1], num_blocks=12, window=3)
+    out, lse = run_oracle(w)
+    qq = q64(w)
+    cu = w.cu_q_lens
+    for s in range(2):
+        k, v = w.kv_values(s)
+        L, ql = int(w.seq_lens[s]), int(w.q_lens[s])
+        for j in range(ql):
+            p = L - ql + j
+            keys = range(max(0, p - 2), p + 1)
+            for h in range(4):
+                kvh = h // 2
+                z = {t: w.softmax_scale * sum(float(qq[cu[s] + j, h, d]) * float(k[t, kvh, d]) for d in range(3))
+                     for t in keys}
+                m = max(z.values())
+                e = {t: math.exp(x - m) for t, x in z.items()}
+                den = sum(e.values())
+                for d in range(3):
+                    ref = sum(e[t] * float(v[t, kvh, d]) for t in keys) / den
+                    assert abs(out[cu[s] + j, h, d] - ref) <= 1e-13, (s, j, h, d)
+                assert abs(lse[cu[s] + j, h] - (m + math.log(den))) <= 1e-13
+
+
 ALL_PINS = [
     pin_e4m3_decode_table, pin_e4m3_encode, pin_bf16_decode, pin_block_mapping_example, pin_append_roundtrip,
     pin_dense_equivalence, pin_noncausal_dense, pin_brute_force, pin_lse_logsumexp, pin_permutation_invariance,
-    pin_softmax_rows, pin_closed_forms, pin_split_reduce, pin_prefix_sharing,
+    pin_softmax_rows, pin_closed_forms, pin_split_reduce, pin_prefix_sharing, pin_window_dense, pin_window_limits,
+    pin_window_brute_force,
 ]

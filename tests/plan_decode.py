@@ -6,7 +6,7 @@ HEADER = np.dtype([("magic", "<u4"), ("bytes", "<u4"), ("n_items", "<i4"), ("n_r
                    ("num_kv_heads", "<i4"), ("head_dim", "<i4"), ("block_size", "<i4"), ("kv_dtype", "<i4"),
                    ("causal", "<i4"), ("num_ctas", "<i4"), ("n_groups", "<i4"), ("items_off", "<u4"),
                    ("reduce_off", "<u4"), ("parts_off", "<u4"), ("n_tc_items", "<i4"), ("tc_items_off", "<u4"),
-                   ("tc_num_ctas", "<i4"), ("pad", "<i4", 10)])
+                   ("tc_num_ctas", "<i4"), ("window", "<i4"), ("pad", "<i4", 9)])
 ITEM = np.dtype([("seq", "<i4"), ("kv_head", "<i4"), ("q_begin", "<i4"), ("n_q", "<i4"), ("k_begin", "<i4"),
                  ("k_end", "<i4"), ("pos0", "<i4"), ("part_row", "<i4")])
 REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("parts_begin", "<i4"),
@@ -30,8 +30,11 @@ def decode(buf) -> dict:
 
 
 def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: int, causal: bool, block_tables=None,
-                   block_size=None):
-    """Every (query token, KV head) row group sees exactly its keys once, through one output path."""
+                   block_size=None, window: int = 0):
+    """Every (query token, KV head) row group sees exactly its keys once, through one output path.
+
+    Under a window the key ranges may start below a row's first visible key (the kernels mask
+    per row) but not past it."""
     h, items, reds, parts = plan["header"], plan["items"], plan["reduces"], plan["parts"]
     g = num_q_heads // num_kv_heads
     # List membership: tensor-memory items carry more than 16 and at most 128 rows and
@@ -93,7 +96,9 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
             ranges = sorted(seen.pop((tok, kvh)))
             vias = {v for _, _, v in ranges}
             assert len(vias) == 1, "a row is both written directly and merged"
-            cover = 0
+            start = max(0, L - ql + j + 1 - window) if window > 0 else 0
+            cover = ranges[0][0]
+            assert cover <= start and (window > 0 or cover == 0), (tok, kvh, ranges)
             for a, b, _ in ranges:
                 assert a == cover, (tok, kvh, ranges)
                 cover = b

@@ -143,6 +143,34 @@ def test_plan_routes_prefill_tiles_to_tensor_memory_list(api):
     assert d8["header"]["n_tc_items"] == 0 and (d8["items"]["n_q"] * 4).max() == 64
 
 
+@pytest.mark.parametrize("window", [1, 5, 64, 200, 100000])
+@pytest.mark.parametrize("split", [0, 64])
+def test_plan_window_ranges(api, window, split):
+    """Under a limited window every row still sees all its visible keys once, and key ranges start
+    no later than (and at most a 128-key tile before) the tile's first visible key."""
+    w = W.mixed_bf16(n_decode=20, n_prefill=3, chunk=300, block_size=16, cached_lo_blocks=1, cached_hi_blocks=40,
+                     aligned=False)
+    w.window = window
+    p = _plan(api, w, window=window, kv_split=split)
+    d = PD.decode(p.buffer)
+    assert d["header"]["window"] == window
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
+                      w.block_size, window=window)
+    if window < 1000:  # the planner skips keys no row of a tile can see
+        base = _plan(api, w, kv_split=split)
+        keys = lambda pl: int((pl["items"]["k_end"] - pl["items"]["k_begin"]).sum())  # noqa: E731
+        assert keys(d) < keys(PD.decode(base.buffer))
+
+
+def test_plan_window_rejects(api):
+    w = W.llama3_8b_decode_bf16(batch=3, lo=10, hi=50)
+    with pytest.raises(api.PkvError):
+        _plan(api, w, window=-1)
+    w.causal = False
+    with pytest.raises(api.PkvError):
+        _plan(api, w, window=8)
+
+
 def test_plan_noncausal_and_empty_rows(api):
     w = W.build("mix", seed=3, kv_dtype="bf16", num_q_heads=16, num_kv_heads=2, head_dim=64, block_size=32,
                 seq_lens=[40, 7, 300, 1, 90], q_lens=[5, 0, 300, 1, 0], causal=False)

@@ -171,6 +171,45 @@ def test_large_logits_stay_finite(pkv):
     run_case(pkv, w)
 
 
+@pytest.mark.parametrize("kv,qd", [("bf16", "bf16"), ("e4m3", "bf16")])
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (64, 8)])
+def test_multi_token_causal_decode(pkv, kv, qd, hq, hkv):
+    # Speculative verification: 2..8 new tokens per sequence, causal among themselves; with g = 4
+    # rows stay decode-sized (<= 16) up to 4 tokens and become tensor-memory tiles past that.
+    r = np.random.default_rng(5)
+    q_lens = r.integers(2, 9, size=24)
+    seq_lens = q_lens + r.integers(30, 1500, size=24)
+    w = W.build("spec", seed=12, kv_dtype=kv, q_dtype=qd, kv_in_dtype="f32" if kv == "e4m3" else None,
+                num_q_heads=hq, num_kv_heads=hkv, head_dim=128, block_size=64, seq_lens=seq_lens, q_lens=q_lens)
+    run_case(pkv, w)
+
+
+@pytest.mark.parametrize("window", [1, 7, 100, 1000])
+@pytest.mark.parametrize("kind", ["mixed_bf16", "decode_f16_d64", "fp8", "block4", "f32"])
+def test_limited_attention_window(pkv, window, kind):
+    # Every kernel path under a window: decode tiles and tcgen05 prefill tiles (bf16 / f16),
+    # fp8 decode and row-split prefill, the cp.async kernel (block 4), the fp32 kernel.
+    r = np.random.default_rng(window)
+    if kind == "mixed_bf16":
+        w = W.build("win", seed=13, kv_dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                    seq_lens=[700, 333, 90, 1500, 41], q_lens=[300, 77, 1, 1, 1], window=window)
+    elif kind == "decode_f16_d64":
+        w = W.build("win", seed=14, kv_dtype="f16", num_q_heads=16, num_kv_heads=4, head_dim=64, block_size=64,
+                    seq_lens=r.integers(1, 3000, size=9), q_lens=[1] * 9, window=window)
+    elif kind == "fp8":
+        w = W.build("win", seed=15, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                    num_kv_heads=8, head_dim=128, block_size=128, seq_lens=[2000, 400, 77], q_lens=[1, 150, 1],
+                    window=window)
+    elif kind == "block4":
+        w = W.build("win", seed=16, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=4,
+                    seq_lens=[300, 45, 180], q_lens=[20, 1, 1], window=window)
+    else:
+        w = W.build("win", seed=17, kv_dtype="f32", num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+                    seq_lens=[300, 45, 180], q_lens=[20, 1, 1], window=window)
+    run_case(pkv, w, kv_split=64)
+    run_case(pkv, w, check_pool=False)
+
+
 @pytest.mark.parametrize("kv", ["bf16", "f16"])
 @pytest.mark.parametrize("D", [64, 128])
 def test_prefill_running_max_jumps(pkv, kv, D):

@@ -15,6 +15,7 @@ _orig_softmax_rows = O._softmax_rows
 _orig_gather = O.gather_rows
 _orig_decode = O.decode_bits
 _orig_split = O.split_kv_reduce
+_orig_start = O.key_start
 
 
 def _gqa_modulo(h, hq, hkv):
@@ -78,6 +79,10 @@ def _bf16_wrong_shift(bits, dtype):
     return _orig_decode(bits, dtype)
 
 
+def _window_one_too_wide(L, ql, j, window):
+    return np.maximum(0, _orig_start(L, ql, j, window) - (1 if window > 0 else 0))
+
+
 def _split_sign(po, pl):
     return _orig_split(po, -np.asarray(pl))
 
@@ -96,6 +101,7 @@ MUTATIONS = {
     "e4m3_bias_8": [("e4m3_decode", _e4m3_bias8), ("decode_bits", _decode_e4m3_bias8)],
     "bf16_decode_shift": [("decode_bits", _bf16_wrong_shift)],
     "split_merge_sign": [("split_kv_reduce", _split_sign)],
+    "window_one_too_wide": [("key_start", _window_one_too_wide)],
 }
 
 
