@@ -147,14 +147,19 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# The sources the decode-tile attention kernel (the roofline kernel of the default workload) is
+# built from: a traffic figure is reported only for the sources it was taken on.
+TRAFFIC_SOURCES = ("attn_tma.cu", "attn_tile.cuh", "attn_args.h", "common.cuh", "internal.h", "plan_format.h")
+
+
 def kernel_source_hash() -> str:
-    """Hash of every kernel source: a traffic figure is reported only for the sources it was taken on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_attention_block_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in TRAFFIC_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    with open(os.path.join(ROOT, "include", "pkv.h"), "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 

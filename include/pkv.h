@@ -80,6 +80,7 @@ typedef enum pkv_dtype {
 #define PKV_DEV_PLAN_MISMATCH 0x4     /* plan item does not fit the device lengths */
 #define PKV_DEV_BAD_APPEND 0x8        /* kv_append position negative */
 #define PKV_DEV_TIMEOUT 0x10          /* an internal pipeline wait gave up (about 1 s); results incomplete */
+#define PKV_DEV_BAD_COPY 0x20         /* copy_block_prefix: token count outside [0, block_size] */
 
 /* One layer's view of a paged pool (deep dive §9: one block holds a fixed number
  * of tokens' KV; several layers may be packed in one block). */
@@ -133,6 +134,30 @@ PKV_API pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, cons
                          const int32_t* cu_new, const int32_t* start_pos, const int32_t* block_tables,
                          int32_t max_blocks, int32_t num_seqs, int32_t total_new, int32_t* dev_status,
                          void* stream);
+
+/*
+ * copy_block_prefix - copy the first tokens of pool blocks into other blocks.
+ *
+ * Source: deep dive §11 (partial reuse: when a new request matches only part of
+ * a cached block, copy_on_partial_reuse copies the matched tokens of that block
+ * into a new block, so that several requests can reuse the same block
+ * partially while each appends its own tokens after the copy).
+ *
+ * For i in [0, count): slots 0 .. n_tokens[i]-1 of block src_blocks[i] are
+ * copied into the same slots of block dst_blocks[i], for every layer, K and
+ * V, and every KV head; slots n_tokens[i] .. block_size-1 of the destination
+ * are left as they were.  n_tokens[i] = block_size copies the whole block.
+ * src_blocks, dst_blocks, n_tokens: device int32 [count].
+ * A destination must not be the source or destination of another copy of the
+ * same call (such copies race); src == dst is a no-op.
+ * Errors: INVALID_ARG for bad shapes / null pointers.  Asynchronously, copies
+ *   with a block id outside [0, num_blocks) (PKV_DEV_BAD_BLOCK_ID) or a token
+ *   count outside [0, block_size] (PKV_DEV_BAD_COPY) are skipped.
+ * Stream-ordered; bit-exact (a byte copy, any pool dtype).
+ */
+PKV_API pkv_status pkv_copy_block_prefix(const pkv_cache* cache, const int32_t* src_blocks,
+                                         const int32_t* dst_blocks, const int32_t* n_tokens, int32_t count,
+                                         int32_t* dev_status, void* stream);
 
 /*
  * Planning request for one paged_attention call (a batch of sequences).

@@ -28,6 +28,9 @@ What it computes, step by step, with the passage each step follows:
   for keys ``t <= p`` (all ``t < seq_len`` when not causal), then the plain
   softmax ``w = exp(z - max z) / sum`` and ``o = sum_t w_t v_t``; also
   ``lse = max z + ln sum exp(z - max z)``.  No tiling, no online softmax.
+  ``copy_block_prefix`` (deep dive §11, partial reuse with
+  ``copy_on_partial_reuse``): the first ``n`` slots of a block, every layer, K
+  and V and KV head, copied into the same slots of another block.
   With a limited attention window ``W`` (deep dive §11, "有限attention window":
   tokens outside the window no longer take part in attention), row ``j`` sees
   only the ``W`` most recent positions up to its own: keys ``p - W < t <= p``.
@@ -51,7 +54,7 @@ import numpy as np
 
 __all__ = [
     "E4M3_MAX", "e4m3_decode", "e4m3_encode", "decode_bits", "kv_head_of", "block_address",
-    "key_limit", "key_start", "OraclePool", "new_pool", "kv_append", "gather_rows", "paged_attention",
+    "key_limit", "key_start", "copy_block_prefix", "OraclePool", "new_pool", "kv_append", "gather_rows", "paged_attention",
     "attention_row_probs", "split_kv_reduce", "sentinel_bits",
 ]
 
@@ -229,6 +232,14 @@ def kv_append(pool: OraclePool, layer: int, k_new, v_new, in_dtype: str, cu_new,
             raise IndexError(f"sequence {s}: block id out of range")
         for which, src in ((0, k_new), (1, v_new)):
             pool.bits[phys, layer, which, :, slot, :] = _store(pool, which, layer, src[lo:hi], in_dtype)
+
+
+def copy_block_prefix(pool: OraclePool, src_blocks, dst_blocks, n_tokens):
+    """Partial reuse (deep dive §11, copy_on_partial_reuse): slots ``0 .. n-1`` of block ``src``
+    go to the same slots of block ``dst``, for every layer, K and V and KV head; in order, as a
+    plain copy of the stored values."""
+    for src, dst, n in zip(np.asarray(src_blocks), np.asarray(dst_blocks), np.asarray(n_tokens)):
+        pool.bits[int(dst), :, :, :, :int(n), :] = pool.bits[int(src), :, :, :, :int(n), :]
 
 
 def gather_rows(pool: OraclePool, layer: int, table_row, kvh: int, which: int, n: int) -> np.ndarray:

@@ -68,6 +68,8 @@ _lib.pkv_abi_version.restype = _I32
 _lib.pkv_status_string.restype = C.c_char_p
 _lib.pkv_status_string.argtypes = [_I32]
 _lib.pkv_last_error.restype = C.c_char_p
+_lib.pkv_copy_block_prefix.restype = _I32
+_lib.pkv_copy_block_prefix.argtypes = [C.POINTER(_Cache), _P, _P, _P, _I32, _P, _P]
 _lib.pkv_kv_append.restype = _I32
 _lib.pkv_kv_append.argtypes = [C.POINTER(_Cache), _P, _P, _I32, _P, _P, _P, _I32, _I32, _I32, _P, _P]
 _lib.pkv_attention_plan.restype = _I32
@@ -163,6 +165,15 @@ def kv_append(cache: Cache, k_new: torch.Tensor, v_new: torch.Tensor, cu_new: to
     _check(_lib.pkv_kv_append(C.byref(c), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(cu_new),
                               _ptr(start_pos), _ptr(block_tables), block_tables.shape[1], num_seqs, total_new,
                               _ptr(status), _stream(stream)), "kv_append")
+
+
+def copy_block_prefix(cache: Cache, src_blocks: torch.Tensor, dst_blocks: torch.Tensor, n_tokens: torch.Tensor,
+                      status: torch.Tensor | None = None, stream=None) -> None:
+    """Copy slots [0, n_tokens[i]) of block src_blocks[i] into block dst_blocks[i] (device int32 tensors),
+    every layer, K and V, every head (partial reuse of a cached block)."""
+    c = cache._c()
+    _check(_lib.pkv_copy_block_prefix(C.byref(c), _ptr(src_blocks), _ptr(dst_blocks), _ptr(n_tokens),
+                                      src_blocks.shape[0], _ptr(status), _stream(stream)), "copy_block_prefix")
 
 
 @dataclass

@@ -462,9 +462,55 @@ def pin_window_brute_force():
                 assert abs(lse[cu[s] + j, h] - (m + math.log(den))) <= 1e-13
 
 
+# ---------------------------------------------------------------------------
+# Partial reuse: block prefix copy (deep dive §11)
+# ---------------------------------------------------------------------------
+
+def pin_block_copy():
+    """Copy a sequence's blocks, whole and in part, into free blocks: a table pointing at the
+    copies gathers the same rows bit for bit up to the copied length; the rest of a partially
+    copied block keeps its sentinels; attention of a request that reuses the copied prefix equals
+    attention over the original tokens."""
+    w = W.build("copy", seed=19, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=16, block_size=8,
+                seq_lens=[61, 20, 35], q_lens=[1, 1, 1], pool_factor=3.0)
+    pool = oracle_pool_for(w)
+    B = w.block_size
+    used = set(int(b) for b in w.block_tables.ravel() if b >= 0)
+    free = [b for b in range(w.num_blocks) if b not in used]
+    s, L = 0, int(w.seq_lens[0])
+    nblk = (L + B - 1) // B
+    n_last = L - (nblk - 1) * B
+    src = w.block_tables[s, :nblk].copy()
+    dst = np.array(free[:nblk], np.int32)
+    ns = np.array([B] * (nblk - 1) + [max(1, n_last // 2)], np.int32)
+    before = pool.bits.copy()
+    O.copy_block_prefix(pool, src, dst, ns)
+    table = w.block_tables[s].copy()
+    table[:nblk] = dst
+    n_copied = (nblk - 1) * B + int(ns[-1])
+    for kvh in range(w.num_kv_heads):
+        for which in (0, 1):
+            a = O.gather_rows(pool, w.layer, w.block_tables[s], kvh, which, n_copied)
+            b = O.gather_rows(pool, w.layer, table, kvh, which, n_copied)
+            assert np.array_equal(a, b)
+    # Untouched: slots past the copied prefix of the last block, and every other block.
+    last = int(dst[-1])
+    assert np.array_equal(pool.bits[last, :, :, :, int(ns[-1]):], before[last, :, :, :, int(ns[-1]):])
+    others = np.ones(w.num_blocks, bool)
+    others[dst] = False
+    assert np.array_equal(pool.bits[others], before[others])
+    # A request reusing the copied prefix (its own table) attends like the original over those tokens.
+    q = q64(w)[:1]
+    o1, l1 = O.paged_attention(pool, w.layer, q, np.array([0, 1]), np.array([n_copied]),
+                               w.block_tables[s:s + 1], w.num_q_heads, w.softmax_scale, True)
+    o2, l2 = O.paged_attention(pool, w.layer, q, np.array([0, 1]), np.array([n_copied]), table[None, :],
+                               w.num_q_heads, w.softmax_scale, True)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
 ALL_PINS = [
     pin_e4m3_decode_table, pin_e4m3_encode, pin_bf16_decode, pin_block_mapping_example, pin_append_roundtrip,
     pin_dense_equivalence, pin_noncausal_dense, pin_brute_force, pin_lse_logsumexp, pin_permutation_invariance,
     pin_softmax_rows, pin_closed_forms, pin_split_reduce, pin_prefix_sharing, pin_window_dense, pin_window_limits,
-    pin_window_brute_force,
+    pin_window_brute_force, pin_block_copy,
 ]

@@ -16,6 +16,8 @@ from paged_kv_attention_block_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
+O_DEV_BAD_BLOCK_ID, O_DEV_BAD_COPY = 0x1, 0x20  # PKV_DEV_* bits of include/pkv.h
+
 
 @pytest.fixture(scope="module")
 def pkv():
@@ -208,6 +210,45 @@ def test_limited_attention_window(pkv, window, kind):
                     seq_lens=[300, 45, 180], q_lens=[20, 1, 1], window=window)
     run_case(pkv, w, kv_split=64)
     run_case(pkv, w, check_pool=False)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3", "f32"])
+def test_copy_block_prefix_bit_exact(pkv, kv):
+    # Partial reuse: copies of whole and partial block prefixes into free blocks, the whole pool
+    # compared byte for byte with the oracle's copy; bad ids and counts are reported, not written.
+    api, runner = pkv
+    if kv == "e4m3":
+        w = W.build("copy", seed=18, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=8,
+                    num_kv_heads=2, head_dim=128, block_size=16, seq_lens=[100, 37, 64], q_lens=[1, 1, 1],
+                    num_layers=2, layer=1, pool_factor=3.0)
+    else:
+        w = W.build("copy", seed=18, kv_dtype=kv, num_q_heads=8, num_kv_heads=2, head_dim=64 if kv == "f32" else 128,
+                    block_size=16, seq_lens=[100, 37, 64], q_lens=[1, 1, 1], num_layers=2, layer=1, pool_factor=3.0)
+    dw = runner.DeviceWorkload(w)
+    dw.append_new()
+    used = set(int(b) for b in w.block_tables.ravel() if b >= 0)
+    free = [b for b in range(w.num_blocks) if b not in used]
+    src = w.block_tables[0, :7]
+    ns = [16, 1, 8, 0, 15, 16, 4]
+    dst = free[:7]
+    pool = oracle_pool(w)
+    O.copy_block_prefix(pool, src, dst, ns)
+    dev = lambda x: torch.tensor(np.asarray(x, np.int32), device="cuda")  # noqa: E731
+    api.copy_block_prefix(dw.cache, dev(src), dev(dst), dev(ns), status=dw.status)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) == 0
+    got = dw.pool_bytes()
+    if kv == "f32":
+        assert (got.view(np.uint32) == pool.bits.view(np.uint32)).all()
+    else:
+        assert (got == pool.bits).all()
+    before = dw.pool_bytes().copy()
+    api.copy_block_prefix(dw.cache, dev([src[0], w.num_blocks]), dev([free[8], free[9]]), dev([17, 4]),
+                          status=dw.status)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) == (O_DEV_BAD_BLOCK_ID | O_DEV_BAD_COPY)
+    after = dw.pool_bytes()
+    assert (after.view(np.uint8) == before.view(np.uint8)).all()
 
 
 @pytest.mark.parametrize("kv", ["bf16", "f16"])

@@ -16,6 +16,7 @@ _orig_gather = O.gather_rows
 _orig_decode = O.decode_bits
 _orig_split = O.split_kv_reduce
 _orig_start = O.key_start
+_orig_copy = O.copy_block_prefix
 
 
 def _gqa_modulo(h, hq, hkv):
@@ -83,6 +84,14 @@ def _window_one_too_wide(L, ql, j, window):
     return np.maximum(0, _orig_start(L, ql, j, window) - (1 if window > 0 else 0))
 
 
+def _copy_whole_block(pool, src, dst, n):
+    return _orig_copy(pool, src, dst, [pool.block_size] * len(list(n)))
+
+
+def _copy_off_by_one(pool, src, dst, n):
+    return _orig_copy(pool, src, dst, [max(0, int(x) - 1) for x in n])
+
+
 def _split_sign(po, pl):
     return _orig_split(po, -np.asarray(pl))
 
@@ -102,6 +111,8 @@ MUTATIONS = {
     "bf16_decode_shift": [("decode_bits", _bf16_wrong_shift)],
     "split_merge_sign": [("split_kv_reduce", _split_sign)],
     "window_one_too_wide": [("key_start", _window_one_too_wide)],
+    "copy_whole_block": [("copy_block_prefix", _copy_whole_block)],
+    "copy_one_token_short": [("copy_block_prefix", _copy_off_by_one)],
 }
 
 
