@@ -473,40 +473,70 @@ def run_prefill_only(w, dev, api, runner, plan_kw, steps: int = 100):
 
 
 def run_e2e(args, w, dw, plan_opts, dev, stream, api):
+    """The step end to end through the public API, as a serving loop runs it: every step copies
+    its inputs (q, new K/V, lengths, positions, tables) from pinned host memory, appends, plans on
+    the host, uploads the plan, runs attention and copies the output back to pinned host memory.
+    Two input/output buffer sets and plan buffers alternate, the copies run on their own stream,
+    so step i+1's copies and host planning overlap step i's kernels.  Time = events around n
+    back-to-back steps (all copies inside), divided by n."""
     import torch
 
     names = {"q": dw.q, "k_new": dw.k_new, "v_new": dw.v_new, "cu_q": dw.cu_q, "seq_lens": dw.seq_lens,
              "start_pos": dw.start_pos, "block_tables": dw.block_tables}
     host = {k: v.detach().cpu().pin_memory() for k, v in names.items()}
-    host["out"] = torch.empty(dw.q.shape, dtype=dw.q.dtype).pin_memory()
-    devb = {k: torch.empty_like(v) for k, v in names.items()}
-    devb["out"] = torch.empty_like(dw.q)
-    plan = dw.plan(**plan_opts)
-    devb["workspace"] = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
+    outs_h = [torch.empty(dw.q.shape, dtype=dw.q.dtype).pin_memory() for _ in range(2)]
+    devb = [{k: torch.empty_like(v) for k, v in names.items()} for _ in range(2)]
+    outs_d = [torch.empty_like(dw.q) for _ in range(2)]
     cu, sl, bt = w.cu_q_lens, w.seq_lens, w.block_tables
+    kw = dict(num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=w.block_size,
+              kv_dtype=w.kv_dtype, causal=w.causal, block_tables=bt, **plan_opts)
+    plans = [api.plan_attention(cu, sl, **kw) for _ in range(2)]
+    ws = torch.empty(max(plans[0].workspace_bytes, 256), dtype=torch.uint8, device=dev)
+    copy = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(2)]     # inputs of a slot copied in
+    consumed = [torch.cuda.Event() for _ in range(2)]  # kernels of a slot done with its inputs and plan
+    fetched = [torch.cuda.Event() for _ in range(2)]   # output of a slot copied out
+    pending = [False, False]
 
-    def plan_fn():
-        return api.plan_attention(cu, sl, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
-                                  block_size=w.block_size, kv_dtype=w.kv_dtype, causal=w.causal, block_tables=bt,
-                                  **plan_opts)
+    def step(i):
+        b = i % 2
+        if pending[b]:
+            consumed[b].synchronize()  # the plan buffer's last upload has run: it may be rewritten
+        api.plan_attention(cu, sl, buffer=plans[b].buffer, **kw)
+        with torch.cuda.stream(copy):
+            copy.wait_event(consumed[b])
+            copy.wait_event(fetched[b])
+            for name in names:
+                devb[b][name].copy_(host[name], non_blocking=True)
+            ready[b].record(copy)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ready[b])
+            d = devb[b]
+            api.kv_append(dw.cache, d["k_new"], d["v_new"], d["cu_q"], d["start_pos"], d["block_tables"])
+            api.paged_attention(dw.cache, d["q"], d["cu_q"], d["seq_lens"], d["block_tables"], plans[b],
+                                w.softmax_scale, w.causal, out=outs_d[b], workspace=ws)
+            consumed[b].record(stream)
+        with torch.cuda.stream(copy):
+            copy.wait_event(consumed[b])
+            outs_h[b].copy_(outs_d[b], non_blocking=True)
+            fetched[b].record(copy)
+        pending[b] = True
 
-    flush = torch.ones(128 << 20, dtype=torch.float32, device=dev)
-    for _ in range(3):
-        api.decode_step_e2e(dw.cache, host, devb, plan_fn, w.softmax_scale, w.causal)
+    for i in range(4):
+        step(i)
     torch.cuda.synchronize(dev)
-    n = max(1, min(args.steps, 200))
-    tot = 0.0
-    for _ in range(n):
-        flush.sum()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record(stream)
-        p = api.decode_step_e2e(dw.cache, host, devb, plan_fn, w.softmax_scale, w.causal)
-        e.record(stream)
-        e.synchronize()
-        tot += s.elapsed_time(e)
-    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if k != "out") + p.info["plan_bytes"]
-    d2h = host["out"].numel() * host["out"].element_size()
-    return {"ms": tot / n, "h2d": int(h2d), "d2h": int(d2h)}
+    n = max(2, min(args.steps, 500))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    copy.wait_event(s)
+    for i in range(n):
+        step(i)
+    stream.wait_event(fetched[(n - 1) % 2])
+    e.record(stream)
+    e.synchronize()
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + plans[0].info["plan_bytes"]
+    d2h = outs_h[0].numel() * outs_h[0].element_size()
+    return {"ms": s.elapsed_time(e) / n, "h2d": int(h2d), "d2h": int(d2h)}
 
 
 def main():

@@ -49,6 +49,9 @@ class _Cache(C.Structure):
                 ("kv_dtype", C.c_int32), ("k_scale", C.c_void_p), ("v_scale", C.c_void_p)]
 
 
+_WORKSPACE_TOO_SMALL = 4  # PKV_ERR_WORKSPACE
+
+
 class _PlanRequest(C.Structure):
     _fields_ = [("num_seqs", C.c_int32), ("num_q_heads", C.c_int32), ("num_kv_heads", C.c_int32),
                 ("head_dim", C.c_int32), ("block_size", C.c_int32), ("kv_dtype", C.c_int32), ("causal", C.c_int32),
@@ -216,12 +219,18 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
                        kv_split, int(bool(cascade)), min_shared_tokens, max_blocks, cu.ctypes.data, sl.ctypes.data,
                        None if bt is None else bt.ctypes.data, int(window))
     info = _PlanInfo()
-    _check(_lib.pkv_attention_plan(C.byref(req), None, 0, C.byref(info)), "attention_plan")
-    if buffer is not None and buffer.numel() >= int(info.plan_bytes):
+    # With a buffer given, plan straight into it (one call); only a buffer too small costs a
+    # size query and a new buffer.
+    st = (_lib.pkv_attention_plan(C.byref(req), buffer.data_ptr(), buffer.numel(), C.byref(info))
+          if buffer is not None else _WORKSPACE_TOO_SMALL)
+    if st == 0:
         buf = buffer
     else:
+        if st != _WORKSPACE_TOO_SMALL:
+            _check(st, "attention_plan")
+        _check(_lib.pkv_attention_plan(C.byref(req), None, 0, C.byref(info)), "attention_plan")
         buf = torch.empty(int(info.plan_bytes), dtype=torch.uint8, pin_memory=pin and torch.cuda.is_available())
-    _check(_lib.pkv_attention_plan(C.byref(req), buf.data_ptr(), buf.numel(), C.byref(info)), "attention_plan")
+        _check(_lib.pkv_attention_plan(C.byref(req), buf.data_ptr(), buf.numel(), C.byref(info)), "attention_plan")
     return Plan(buf, {f: getattr(info, f) for f, _ in _PlanInfo._fields_})
 
 

@@ -38,9 +38,42 @@ struct Seg {
   bool tc;  // tensor-memory list
 };
 
+// Register-tile items first, then tensor-memory items; heaviest first within each list, ties in
+// creation order (the order a stable sort by cost would keep).  A cost is keys x max(1, rows/16),
+// so c = 16 x cost is an integer (clamped to 32 bits past 2^25 keys).  Each item gets the key
+// [list bit][c_max - c, `bits` wide][creation index, 20 bits] (the planner refuses 2^20 items or
+// more), and a stable least-significant-digit radix sort over the bits above the index, in
+// 11-bit digits, orders them: the indices start ascending and stability keeps ties that way.
+void order_segments(const std::vector<Seg>& segs, std::vector<uint64_t>& keys, std::vector<uint64_t>& tmp) {
+  const size_t n = segs.size();
+  keys.resize(n);
+  tmp.resize(n);
+  uint64_t c_max = 0;
+  for (size_t i = 0; i < n; ++i) {
+    keys[i] = std::min<uint64_t>(uint64_t(segs[i].cost * 16.0 + 0.5), 0xFFFFFFFFull);
+    c_max = std::max(c_max, keys[i]);
+  }
+  int bits = 0;
+  while (bits < 32 && (c_max >> bits) != 0) ++bits;
+  for (size_t i = 0; i < n; ++i)
+    keys[i] = (((uint64_t(segs[i].tc) << bits) | (c_max - keys[i])) << 20) | uint64_t(i);
+  if (n < 2) return;
+  uint32_t count[2048];
+  for (int shift = 20; shift < 21 + bits; shift += 11) {
+    std::memset(count, 0, sizeof(count));
+    for (size_t i = 0; i < n; ++i) ++count[(keys[i] >> shift) & 2047];
+    if (count[(keys[0] >> shift) & 2047] == n) continue;  // one digit value: order unchanged
+    uint32_t sum = 0;
+    for (int d = 0; d < 2048; ++d) { const uint32_t c = count[d]; count[d] = sum; sum += c; }
+    for (size_t i = 0; i < n; ++i) tmp[count[(keys[i] >> shift) & 2047]++] = keys[i];
+    keys.swap(tmp);
+  }
+}
+
 double row_weight(int rows) { return rows <= 16 ? 1.0 : rows / 16.0; }
 
-int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+// m a power of two
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) & ~(m - 1); }
 
 }  // namespace
 
@@ -126,6 +159,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   std::vector<Seg> segs;
   std::vector<PkvReduce> reds;
   std::vector<int32_t> parts;
+  segs.reserve(size_t(S) * Hkv * 2 + 64);
+  reds.reserve(size_t(S) * Hkv);
+  parts.reserve(size_t(S) * Hkv * 2);
   int64_t part_rows = 0;
   // Partial row of each (group member, KV head) inside its group tile.
   std::vector<int64_t> gpart(groups.empty() ? 0 : size_t(S) * Hkv, -1);
@@ -149,6 +185,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
 
   // 2. Units of work.
   std::vector<Unit> units;
+  units.reserve(size_t(S) * Hkv);
   for (int s = 0; s < S; ++s) {
     const int ql = q_len(s);
     if (ql == 0) continue;
@@ -171,17 +208,25 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
 
   // 3. Key-range split and merges.
   const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 2.0)};
+  // Units come in runs of one row count (every KV head of a tile): the split length is computed
+  // once per run.
+  int last_rows = -1;
+  int32_t mk = 0;
   for (const Unit& u : units) {
     const int n = std::max(0, u.k_end - u.k_begin);
     const int rows = u.n_q * g;
     const bool t = is_tc(rows);
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
-    int64_t max_keys;
-    if (req->kv_split < 0) max_keys = INT32_MAX;
-    else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
-    else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
-                                      round_up(int64_t(std::ceil(target[t] / u.weight)), tile_keys));
-    const int64_t nseg = n == 0 ? 0 : (n + max_keys - 1) / max_keys;
+    if (rows != last_rows) {
+      int64_t max_keys;
+      if (req->kv_split < 0) max_keys = INT32_MAX;
+      else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
+      else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
+                                        round_up(int64_t(std::ceil(target[t] / u.weight)), tile_keys));
+      mk = int32_t(std::min<int64_t>(max_keys, INT32_MAX / 2));
+      last_rows = rows;
+    }
+    const int32_t nseg = n == 0 ? 0 : int32_t((uint32_t(n) + uint32_t(mk) - 1u) / uint32_t(mk));
     if (nseg == 1 && u.group_part < 0) {
       PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, u.k_begin, u.k_end, u.pos0, -1};
       segs.push_back({it, n * u.weight, t});
@@ -190,7 +235,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     PkvReduce r{u.q_begin, u.n_q, u.kv_head, int32_t(parts.size()), 0, {0, 0, 0}};
     if (u.group_part >= 0) parts.push_back(u.group_part);
     if (nseg > 0) {
-      const int64_t seg = round_up((n + nseg - 1) / nseg, tile_keys);
+      const int64_t seg = round_up(int64_t((uint32_t(n) + uint32_t(nseg) - 1u) / uint32_t(nseg)), tile_keys);
       for (int64_t k0 = u.k_begin; k0 < u.k_end; k0 += seg) {
         const int k1 = int(std::min<int64_t>(u.k_end, k0 + seg));
         PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, int(k0), k1, u.pos0, int32_t(part_rows)};
@@ -203,11 +248,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     reds.push_back(r);
   }
   if (part_rows > INT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: too many partial rows");
+  if (segs.size() >= (size_t(1) << 20)) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: more than 2^20 work items");
 
-  // Register-tile items first, then tensor-memory items; heaviest first within each list.
-  std::stable_sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) {
-    return x.tc != y.tc ? y.tc : x.cost > y.cost;
-  });
   const int64_t n_tc = std::count_if(segs.begin(), segs.end(), [](const Seg& s) { return s.tc; });
 
   const uint64_t items_off = sizeof(PkvPlanHeader);
@@ -256,7 +298,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.parts_off = uint32_t(parts_off);
   std::memcpy(p, &h, sizeof(h));
   PkvItem* items = reinterpret_cast<PkvItem*>(p + items_off);
-  for (size_t i = 0; i < segs.size(); ++i) items[i] = segs[i].it;
+  std::vector<uint64_t> order, scratch;
+  order_segments(segs, order, scratch);
+  for (size_t i = 0; i < segs.size(); ++i) items[i] = segs[size_t(order[i] & 0xFFFFF)].it;
   if (!reds.empty()) std::memcpy(p + reduce_off, reds.data(), reds.size() * sizeof(PkvReduce));
   if (!parts.empty()) std::memcpy(p + parts_off, parts.data(), parts.size() * sizeof(int32_t));
   return PKV_OK;

@@ -195,3 +195,24 @@ def test_plan_balances_decode(api):
     per_cta = keys.sum() / 296
     assert keys.max() <= max(256, 2 * per_cta / 2 + 64)
     assert p.info["num_items"] >= 296
+
+
+@pytest.mark.parametrize("name,make,opts", CASES, ids=[c[0] for c in CASES])
+def test_plan_orders_heaviest_first(api, name, make, opts):
+    """Each list runs heaviest item first (cost = keys x max(1, rows / 16)), so the last items
+    the CTAs claim are the short ones; equal costs keep creation order, which for items outside
+    shared-prefix groups is (first token, KV head, first key) ascending."""
+    w = make()
+    p = _plan(api, w, **opts)
+    d = PD.decode(p.buffer)
+    g = w.num_q_heads // w.num_kv_heads
+    for lst in (d["reg_items"], d["tc_items"]):
+        if len(lst) == 0:
+            continue
+        cost = (lst["k_end"] - lst["k_begin"]).astype(np.float64) * np.maximum(1.0, lst["n_q"] * g / 16.0)
+        assert (np.diff(cost) <= 0).all()
+        if p.info["num_groups"] == 0:
+            for i in range(1, len(lst)):
+                if cost[i] == cost[i - 1]:
+                    a, b = lst[i - 1], lst[i]
+                    assert (a["q_begin"], a["kv_head"], a["k_begin"]) < (b["q_begin"], b["kv_head"], b["k_begin"])
