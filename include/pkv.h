@@ -14,7 +14,8 @@
  *     requests, without padding, and a long prompt is processed in chunks that
  *     attend to everything cached so far plus themselves (deep dive §6
  *     "In-flight batching", §8 "Chunked prefill");
- *   - the cache may be stored as fp8 (deep dive §13, KvCacheConfig(dtype="fp8")).
+ *   - the cache may be stored as fp8 or as NVFP4 (deep dive §13 "量化：FP8、FP4与
+ *     KV cache dtype": KvCacheConfig(dtype="fp8") and dtype="nvfp4").
  * The attention itself is softmax(scale * q K^T) V with grouped-query heads:
  * query head h reads KV head h / (Hq / Hkv).
  *
@@ -35,7 +36,12 @@
  *   - Pool layout (row-major):
  *       pool[num_blocks][num_layers][2][num_kv_heads][block_size][head_dim]
  *     index 0 of the "2" axis is K, 1 is V; each (block, layer, K|V, head) is
- *     one contiguous run of block_size * head_dim elements.
+ *     one contiguous run of block_size * head_dim elements.  An NVFP4 pool
+ *     keeps the same order with a different run: block_size rows of
+ *     head_dim / 2 bytes of packed E2M1 codes (dimension 2i in the low nibble
+ *     of byte i, 2i+1 in the high nibble), then block_size rows of
+ *     head_dim / 16 bytes of E4M3 block scales (byte j scales dimensions
+ *     16j .. 16j+15 of its row): block_size * head_dim * 9 / 16 bytes per run.
  *   - Token p of sequence s lives in physical block block_tables[s][p / B] at
  *     slot p % B.  Block tables are int32 [num_seqs][max_blocks] (row stride
  *     max_blocks); unused entries are ignored.
@@ -71,7 +77,11 @@ typedef enum pkv_dtype {
   PKV_F32 = 0,
   PKV_BF16 = 1,
   PKV_F16 = 2,
-  PKV_FP8_E4M3 = 3 /* OCP E4M3: bias 7, no infinities, max finite 448 */
+  PKV_FP8_E4M3 = 3, /* OCP E4M3: bias 7, no infinities, max finite 448 */
+  PKV_NVFP4 = 4     /* KV pools only: E2M1 codes (1 sign, 2 exponent, 1 mantissa bit:
+                       0, 0.5, 1, 1.5, 2, 3, 4, 6) with an E4M3 scale per 16 values and a
+                       float32 scale per (layer, KV head, K|V); value = code * block scale
+                       * k_scale or v_scale.  head_dim 128, block_size >= 16. */
 } pkv_dtype;
 
 /* Bits OR-ed into *dev_status by kernels. */
@@ -92,9 +102,9 @@ typedef struct pkv_cache {
   int32_t num_kv_heads;   /* Hkv */
   int32_t head_dim;       /* d: 64 or 128 */
   int32_t block_size;     /* B: power of two, >= 2 */
-  int32_t kv_dtype;       /* pkv_dtype: F32, BF16, F16 or FP8_E4M3 */
-  const float* k_scale;   /* device float32 [num_layers][Hkv]; FP8_E4M3 only, else NULL */
-  const float* v_scale;   /* device float32 [num_layers][Hkv]; FP8_E4M3 only, else NULL */
+  int32_t kv_dtype;       /* pkv_dtype: F32, BF16, F16, FP8_E4M3 or NVFP4 */
+  const float* k_scale;   /* device float32 [num_layers][Hkv], positive and finite; FP8_E4M3 and NVFP4 only */
+  const float* v_scale;   /* device float32 [num_layers][Hkv], positive and finite; FP8_E4M3 and NVFP4 only */
 } pkv_cache;
 
 /* Library ABI version (PKV_ABI_VERSION of the build). */
@@ -124,7 +134,13 @@ PKV_API const char* pkv_last_error(void);
  *   FP8_E4M3 pool it is F32, BF16 or F16 and each value x is stored as the
  *   E4M3 code of the float32 quotient x / scale (IEEE division), rounded to
  *   nearest even, finite overflow saturated to +-448, with scale =
- *   k_scale[layer][h] for K and v_scale[layer][h] for V.
+ *   k_scale[layer][h] for K and v_scale[layer][h] for V.  For an NVFP4 pool it
+ *   is F32, BF16 or F16 (finite values); each row's 16-value group x with
+ *   global scale g = k_scale[layer][h] (K) or v_scale[layer][h] (V) is stored,
+ *   all in float32 with IEEE rounding, as: a = max |x_i|; block scale code
+ *   c = E4M3(a / (6 * g)) (nearest even, saturating); s = value of c; codes
+ *   E2M1(x_i / (s * g)), nearest even, saturating to +-6, the sign kept (all
+ *   codes 0 when s = 0).
  * Errors: INVALID_ARG for bad shapes/dtypes/null pointers.  Asynchronously,
  *   rows whose block id is out of range are not written (PKV_DEV_BAD_BLOCK_ID,
  *   PKV_DEV_BAD_LOGICAL_BLOCK, PKV_DEV_BAD_APPEND).

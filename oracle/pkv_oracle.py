@@ -19,7 +19,14 @@ What it computes, step by step, with the passage each step follows:
   cache (deep dive §13, ``KvCacheConfig(dtype="fp8")``) the stored byte is the
   E4M3 encoding, round-to-nearest-even with saturation to +-448, of
   ``x / scale`` computed in float32, with one scale per (layer, KV head) for K
-  and one for V.
+  and one for V.  With an NVFP4 cache (deep dive §13, ``NVFP4 KV cache`` and
+  ``KvCacheConfig(dtype="nvfp4")``; the pages name the format but print none
+  of it, so the reading is the published NVFP4 definition: 4-bit E2M1 values in
+  groups of 16 sharing an E4M3 scale, under a float32 scale per tensor, here
+  per (layer, KV head, K|V)), each 16-value group ``x`` of a row with global
+  scale ``g`` stores the block scale code ``c = E4M3(max|x| / (6 g))`` and the
+  element codes ``E2M1(x_i / (value(c) g))`` (nearest even, saturating at 6;
+  all zero when the block scale is 0), every quotient and product in float32.
 * ``paged_attention`` (deep dive §2: decode reads the whole KV history of the
   request to do attention; §6: context and generation requests in one packed
   batch; §8: a chunk attends to the cached KV plus itself): for sequence ``s``,
@@ -41,8 +48,9 @@ What it computes, step by step, with the passage each step follows:
   a softmax over key ranges; the pages do not print it (they never describe
   split-KV), so it is pinned against the unsplit computation.
 
-Every floating-point step is float64 except the one the fp8 encoding decides:
-``x / scale`` is taken in float32 because the stored byte depends on it.
+Every floating-point step is float64 except the ones the fp8 and NVFP4
+encodings decide: their quotients and products are taken in float32 because the
+stored bytes depend on them.
 
 Helper functions (``kv_head_of``, ``block_address``, ``key_limit``,
 ``rne``) are module-level so that tests can plant a mistake in one of them and
@@ -53,12 +61,14 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "E4M3_MAX", "e4m3_decode", "e4m3_encode", "decode_bits", "kv_head_of", "block_address",
+    "E4M3_MAX", "e4m3_decode", "e4m3_encode", "e2m1_decode", "e2m1_encode", "nvfp4_quantize", "nvfp4_pool_bytes",
+    "NVFP4_GROUP", "decode_bits", "kv_head_of", "block_address",
     "key_limit", "key_start", "copy_block_prefix", "OraclePool", "new_pool", "kv_append", "gather_rows", "paged_attention",
     "attention_row_probs", "split_kv_reduce", "sentinel_bits",
 ]
 
 E4M3_MAX = 448.0
+NVFP4_GROUP = 16  # values sharing one E4M3 block scale
 
 
 # ---------------------------------------------------------------------------
@@ -116,6 +126,57 @@ def e4m3_encode(x32: np.ndarray) -> np.ndarray:
     return out.astype(np.uint8)
 
 
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """4-bit E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; no infinity or NaN.
+
+    Exponent field 0 is subnormal ``m * 0.5``; otherwise ``(1 + m/2) * 2^(e-1)``, so the
+    magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+    """
+    c = np.asarray(codes, dtype=np.int64)
+    sign = (c >> 3) & 1
+    e = (c >> 1) & 3
+    m = (c & 1).astype(np.float64)
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.exp2(e.astype(np.float64) - 1.0))
+    return np.where(sign == 1, -mag, mag)
+
+
+def e2m1_encode(y32: np.ndarray) -> np.ndarray:
+    """float32 (finite) -> E2M1 code: the nearest of the eight magnitudes, a tie going to the
+    code with mantissa bit 0 (round half to even), beyond 6 saturating to 6; the sign bit is
+    the sign of the input (so -0.1 gives the code of -0)."""
+    y = np.asarray(y32, dtype=np.float32).astype(np.float64)
+    mags = e2m1_decode(np.arange(8))
+    a = np.minimum(np.abs(y), mags[-1])  # saturation first: huge inputs are 6, not a far tie
+    dist = np.abs(a[..., None] - mags)  # [..., 8]
+    best = dist.min(axis=-1, keepdims=True)
+    tied = dist == best
+    # Among the nearest codes take the even one (mantissa bit 0); at most two are nearest.
+    even = tied & ((np.arange(8) & 1) == 0)
+    pick = np.where(even.any(axis=-1), even.argmax(axis=-1), tied.argmax(axis=-1))
+    return (pick | np.where(np.signbit(y), 8, 0)).astype(np.uint8)
+
+
+def nvfp4_quantize(x32: np.ndarray, g) -> tuple[np.ndarray, np.ndarray]:
+    """Rows ``x32`` [..., D] (float32) with global scale ``g`` (float32, broadcast over [...]) ->
+    (E2M1 codes uint8 [..., D], E4M3 block scale codes uint8 [..., D / 16]).
+
+    Per 16-value group: ``a = max |x|``, ``c = E4M3(a / (6 g))``, ``s = value(c)``; codes
+    ``E2M1(x / (s g))``, all zero when ``s`` is 0.  Products and quotients in float32."""
+    x = np.asarray(x32, dtype=np.float32)
+    D = x.shape[-1]
+    grp = x.reshape(x.shape[:-1] + (D // NVFP4_GROUP, NVFP4_GROUP))
+    gg = np.asarray(g, dtype=np.float32)[..., None]  # broadcast over the group axis
+    amax = np.abs(grp).max(axis=-1)
+    six_g = (np.float32(6.0) * gg).astype(np.float32)
+    scale_codes = e4m3_encode((amax / six_g).astype(np.float32))
+    s = e4m3_decode(scale_codes).astype(np.float32)
+    denom = (s * gg).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = (grp / denom[..., None]).astype(np.float32)
+    codes = np.where((s == 0)[..., None], np.uint8(0), e2m1_encode(np.where((s == 0)[..., None], 0, y)))
+    return codes.reshape(x.shape).astype(np.uint8), scale_codes
+
+
 def decode_bits(bits: np.ndarray, dtype: str) -> np.ndarray:
     """Stored bits -> float64, exactly."""
     if dtype == "f32":
@@ -138,7 +199,7 @@ def _to_f32(bits: np.ndarray, dtype: str) -> np.ndarray:
 def sentinel_bits(dtype: str):
     """NaN pattern that fills pool slots no sequence owns."""
     return {"f32": np.float32(np.nan), "bf16": np.uint16(0x7FC0), "f16": np.uint16(0x7E00),
-            "e4m3": np.uint8(0x7F)}[dtype]
+            "e4m3": np.uint8(0x7F), "nvfp4": np.uint8(0x7F)}[dtype]
 
 
 # ---------------------------------------------------------------------------
@@ -173,11 +234,16 @@ def key_start(seq_len: int, q_len: int, j, window: int):
 
 
 class OraclePool:
-    """Host copy of a pool: ``bits[num_blocks][num_layers][2][Hkv][B][D]`` in storage bits."""
+    """Host copy of a pool: ``bits[num_blocks][num_layers][2][Hkv][B][D]`` in storage bits.
 
-    def __init__(self, bits: np.ndarray, dtype: str, k_scale=None, v_scale=None):
+    NVFP4 pools hold one E2M1 code per element in ``bits`` and the E4M3 block scale codes in
+    ``block_scales[num_blocks][num_layers][2][Hkv][B][D / 16]``; ``nvfp4_pool_bytes`` packs
+    both into the pool's byte image."""
+
+    def __init__(self, bits: np.ndarray, dtype: str, k_scale=None, v_scale=None, block_scales=None):
         self.bits = bits
         self.dtype = dtype
+        self.block_scales = block_scales
         self.k_scale = None if k_scale is None else np.asarray(k_scale, np.float32)
         self.v_scale = None if v_scale is None else np.asarray(v_scale, np.float32)
 
@@ -199,13 +265,34 @@ class OraclePool:
 
 
 def new_pool(num_blocks, num_layers, num_kv_heads, block_size, head_dim, dtype, k_scale=None, v_scale=None):
+    shape = (num_blocks, num_layers, 2, num_kv_heads, block_size, head_dim)
+    if dtype == "nvfp4":
+        # The 0x7F fill byte: codes 0xF (dimension 2i) and 0x7 (2i+1), block scales E4M3 NaN.
+        bits = np.empty(shape, np.uint8)
+        bits[..., 0::2] = 0xF
+        bits[..., 1::2] = 0x7
+        scales = np.full(shape[:-1] + (head_dim // NVFP4_GROUP,), 0x7F, np.uint8)
+        return OraclePool(bits, dtype, k_scale, v_scale, scales)
     storage = {"f32": np.float32, "bf16": np.uint16, "f16": np.uint16, "e4m3": np.uint8}[dtype]
-    bits = np.full((num_blocks, num_layers, 2, num_kv_heads, block_size, head_dim), sentinel_bits(dtype), storage)
+    bits = np.full(shape, sentinel_bits(dtype), storage)
     return OraclePool(bits, dtype, k_scale, v_scale)
 
 
-def _store(pool: OraclePool, which: int, layer: int, x_bits: np.ndarray, in_dtype: str) -> np.ndarray:
-    """Values [n][Hkv][D] in ``in_dtype`` -> stored bits for the pool dtype."""
+def nvfp4_pool_bytes(pool: OraclePool) -> np.ndarray:
+    """The pool's byte image: per (block, layer, K|V, head), B rows of D/2 bytes (dimension 2i in
+    the low nibble of byte i, 2i+1 in the high one) then B rows of D/16 block scale bytes."""
+    c = pool.bits
+    packed = (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+    lead = c.shape[:4]
+    return np.concatenate([packed.reshape(lead + (-1,)), pool.block_scales.reshape(lead + (-1,))], axis=-1)
+
+
+def _store(pool: OraclePool, which: int, layer: int, x_bits: np.ndarray, in_dtype: str):
+    """Values [n][Hkv][D] in ``in_dtype`` -> stored bits for the pool dtype (NVFP4: codes and
+    block scale codes)."""
+    if pool.dtype == "nvfp4":
+        x32 = _to_f32(x_bits, in_dtype)
+        return nvfp4_quantize(x32, pool.scale(which, layer).astype(np.float32)[None, :])
     if pool.dtype == "e4m3":
         x32 = _to_f32(x_bits, in_dtype)
         scale = pool.scale(which, layer).astype(np.float32)[None, :, None]
@@ -231,7 +318,12 @@ def kv_append(pool: OraclePool, layer: int, k_new, v_new, in_dtype: str, cu_new,
         if np.any(phys < 0) or np.any(phys >= pool.bits.shape[0]):
             raise IndexError(f"sequence {s}: block id out of range")
         for which, src in ((0, k_new), (1, v_new)):
-            pool.bits[phys, layer, which, :, slot, :] = _store(pool, which, layer, src[lo:hi], in_dtype)
+            stored = _store(pool, which, layer, src[lo:hi], in_dtype)
+            if pool.dtype == "nvfp4":
+                pool.bits[phys, layer, which, :, slot, :] = stored[0]
+                pool.block_scales[phys, layer, which, :, slot, :] = stored[1]
+            else:
+                pool.bits[phys, layer, which, :, slot, :] = stored
 
 
 def copy_block_prefix(pool: OraclePool, src_blocks, dst_blocks, n_tokens):
@@ -240,12 +332,19 @@ def copy_block_prefix(pool: OraclePool, src_blocks, dst_blocks, n_tokens):
     plain copy of the stored values."""
     for src, dst, n in zip(np.asarray(src_blocks), np.asarray(dst_blocks), np.asarray(n_tokens)):
         pool.bits[int(dst), :, :, :, :int(n), :] = pool.bits[int(src), :, :, :, :int(n), :]
+        if pool.block_scales is not None:
+            pool.block_scales[int(dst), :, :, :, :int(n), :] = pool.block_scales[int(src), :, :, :, :int(n), :]
 
 
 def gather_rows(pool: OraclePool, layer: int, table_row, kvh: int, which: int, n: int) -> np.ndarray:
     """Dequantised K (which=0) or V (which=1) of tokens ``0..n-1`` for one KV head, float64 [n][D]."""
     t = np.arange(n)
     phys, slot = block_address(table_row, t, pool.block_size)
+    if pool.dtype == "nvfp4":
+        codes = pool.bits[phys, layer, which, kvh, slot, :]
+        block = e4m3_decode(pool.block_scales[phys, layer, which, kvh, slot, :])  # [n][D/16]
+        vals = e2m1_decode(codes) * np.repeat(block, NVFP4_GROUP, axis=-1)
+        return vals * np.float64(pool.scale(which, layer)[kvh])
     vals = decode_bits(pool.bits[phys, layer, which, kvh, slot, :], pool.dtype)
     if pool.dtype == "e4m3":
         vals = vals * np.float64(pool.scale(which, layer)[kvh])

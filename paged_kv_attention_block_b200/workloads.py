@@ -23,7 +23,9 @@ Recipe (all draws from numpy PCG64 streams keyed by (seed, stream id)):
   ``ceil(pool_factor * need)`` blocks (or an explicit ``num_blocks``);
   block-table padding is -1;
 * fp8 scales are calibration inputs: ``amax / 448`` per (layer, KV head) and
-  separately for K and V, over every token of that head.
+  separately for K and V, over every token of that head; NVFP4 global scales
+  are ``amax / (6 * 448)`` on the same footing (the largest E2M1 value times
+  the largest E4M3 block scale), so no block scale saturates.
 """
 from __future__ import annotations
 
@@ -35,8 +37,15 @@ import os
 import numpy as np
 
 # Storage dtype names shared by the binding and the tests.
-DTYPES = ("f32", "bf16", "f16", "e4m3")
-ELEM_BYTES = {"f32": 4, "bf16": 2, "f16": 2, "e4m3": 1}
+DTYPES = ("f32", "bf16", "f16", "e4m3", "nvfp4")
+
+
+def kv_row_bytes(dtype: str, head_dim: int) -> float:
+    """Bytes of one token's K (or V) row of one head in a pool of ``dtype`` (NVFP4: head_dim / 2
+    bytes of codes and head_dim / 16 bytes of block scales)."""
+    if dtype == "nvfp4":
+        return head_dim // 2 + head_dim // 16
+    return head_dim * {"f32": 4, "bf16": 2, "f16": 2, "e4m3": 1}[dtype]
 
 _STREAM_LENS, _STREAM_PERM, _STREAM_Q, _STREAM_PREFIX = 1, 2, 3, 4
 _STREAM_SEQ_BASE = 1000
@@ -90,7 +99,7 @@ class Workload:
     causal: bool
     data_scale: float
     shared_prefix_tokens: int
-    k_scale: np.ndarray | None = None  # [num_layers][Hkv] float32, fp8 only
+    k_scale: np.ndarray | None = None  # [num_layers][Hkv] float32, fp8 and NVFP4 only
     v_scale: np.ndarray | None = None
     window: int = 0  # limited attention window (positions); 0 = every cached key
     _kv_cache: dict = field(default_factory=dict, repr=False)
@@ -209,8 +218,9 @@ class Workload:
         return sorted(used.items())
 
 
-def _calibrate_fp8(w: Workload, threads: int) -> None:
-    """amax/448 scales per (layer, KV head), separately for K and V."""
+def _calibrate_fp8(w: Workload, threads: int, top: float = 448.0) -> None:
+    """amax / top scales per (layer, KV head), separately for K and V (top: 448 for fp8,
+    6 * 448 for NVFP4 global scales)."""
     H = w.num_kv_heads
 
     def one(s):
@@ -225,8 +235,8 @@ def _calibrate_fp8(w: Workload, threads: int) -> None:
             amax_v = np.maximum(amax_v, av)
     ks = np.ones((w.num_layers, H), np.float32)
     vs = np.ones((w.num_layers, H), np.float32)
-    ks[w.layer] = (np.maximum(amax_k, 1e-12) / 448.0).astype(np.float32)
-    vs[w.layer] = (np.maximum(amax_v, 1e-12) / 448.0).astype(np.float32)
+    ks[w.layer] = (np.maximum(amax_k, 1e-12) / top).astype(np.float32)
+    vs[w.layer] = (np.maximum(amax_v, 1e-12) / top).astype(np.float32)
     w.k_scale, w.v_scale = ks, vs
 
 
@@ -263,7 +273,7 @@ def build(
     if q_dtype is None:
         q_dtype = "f32" if kv_dtype == "f32" else ("f16" if kv_dtype == "f16" else "bf16")
     if kv_in_dtype is None:
-        kv_in_dtype = "f32" if kv_dtype in ("f32", "e4m3") else kv_dtype
+        kv_in_dtype = "f32" if kv_dtype in ("f32", "e4m3", "nvfp4") else kv_dtype
     S = len(seq_lens)
     nblk = [(int(L) + B - 1) // B for L in seq_lens]
     P_blocks = shared_prefix_tokens // B
@@ -292,8 +302,8 @@ def build(
         q_lens=q_lens, block_tables=bt, softmax_scale=float(softmax_scale), causal=causal, window=int(window),
         data_scale=data_scale, shared_prefix_tokens=shared_prefix_tokens,
     )
-    if kv_dtype == "e4m3":
-        _calibrate_fp8(w, threads or min(32, os.cpu_count() or 1))
+    if kv_dtype in ("e4m3", "nvfp4"):
+        _calibrate_fp8(w, threads or min(32, os.cpu_count() or 1), 448.0 if kv_dtype == "e4m3" else 6.0 * 448.0)
     return w
 
 
@@ -340,6 +350,14 @@ def mixed_bf16(seed: int = 1003, n_decode: int = 120, n_prefill: int = 4, chunk:
                  block_size=block_size, seq_lens=seq_lens, q_lens=q_lens)
 
 
+def llama3_8b_decode_nvfp4(seed: int = 1002, batch: int = 64, lo: int = 512, hi: int = 4096) -> Workload:
+    """The Llama-3-8B decode batch (same lengths and values as the bf16 one) over an NVFP4 cache:
+    Hq 32 / Hkv 8, d 128, block 64, q bf16, K/V appended from float32."""
+    return build("llama3_8b_decode_nvfp4", seed=seed, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32",
+                 num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=64, seq_lens=_lens(seed, batch, lo, hi),
+                 q_lens=[1] * batch, data_scale=0.5)
+
+
 def longctx_fp8(seed: int = 1004, batch: int = 8, seq_len: int = 131072) -> Workload:
     """Long-context decode, e4m3 KV with per-(layer, KV-head) scales, q bf16, block 128."""
     return build("longctx_fp8", seed=seed, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32",
@@ -361,5 +379,6 @@ NAMED = {
     "llama3_8b_decode_bf16": llama3_8b_decode_bf16,
     "mixed_bf16": mixed_bf16,
     "longctx_fp8": longctx_fp8,
+    "llama3_8b_decode_nvfp4": llama3_8b_decode_nvfp4,
     "prefix_reuse_bf16": prefix_reuse_bf16,
 }

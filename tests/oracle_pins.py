@@ -7,6 +7,8 @@ the oracle and checks that at least one pin fails for each.
 
 Independent references used here:
 * torch's ``float8_e4m3fn`` and ``bfloat16`` CPU conversions (library codecs);
+* the E2M1 value table (the eight magnitudes the 4-bit format defines) and a
+  rounding written here as scaled round-half-even per binade, for NVFP4;
 * ``torch.nn.functional.scaled_dot_product_attention`` in float64 on a
   contiguous ``[heads, seq, dim]`` layout built straight from the generator's
   values (so the paged write/read path is bypassed);
@@ -62,6 +64,17 @@ def _values64(w: W.Workload, s: int):
             sc = (w.k_scale if which == 0 else w.v_scale)[w.layer].astype(np.float32)
             y = torch.from_numpy(np.ascontiguousarray(x, np.float32) / sc[None, :, None])
             out.append(y.to(torch.float8_e4m3fn).to(torch.float64).numpy() * sc.astype(np.float64)[None, :, None])
+        return out[0], out[1]
+    if w.kv_dtype == "nvfp4":
+        # Codes from the (separately pinned) quantiser, values through the E2M1 table and torch's
+        # E4M3 conversion: the paged write and read paths are bypassed.
+        out = []
+        for which, x in ((0, k), (1, v)):
+            g = (w.k_scale if which == 0 else w.v_scale)[w.layer].astype(np.float32)
+            codes, sc = O.nvfp4_quantize(np.ascontiguousarray(x, np.float32), g[None, :])
+            mag = np.array(E2M1_MAGNITUDES)[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+            blk = torch.from_numpy(sc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+            out.append(mag * np.repeat(blk, 16, axis=-1) * g.astype(np.float64)[None, :, None])
         return out[0], out[1]
     if w.kv_dtype == "f32":
         return k.astype(np.float64), v.astype(np.float64)
@@ -149,6 +162,108 @@ def pin_e4m3_encode():
     assert O.e4m3_encode(big).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
 
 
+# The eight E2M1 magnitudes (codes 0..7); code | 8 is the negative.
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def _e2m1_round_here(y):
+    """Nearest E2M1 value with ties to even, written independently of the oracle: spacing 0.5
+    below 2, 1 in [2, 4), 2 from 4; np.rint breaks ties to the even multiple; clamp at 6."""
+    y = np.asarray(y, np.float64)
+    a = np.abs(y)
+    r = np.where(a < 2, np.rint(a * 2) / 2, np.where(a < 4, np.rint(a), 2 * np.rint(a / 2)))
+    r = np.minimum(r, 6.0)
+    return np.where(np.signbit(y), -r, r)
+
+
+def pin_e2m1_table():
+    got = O.e2m1_decode(np.arange(16))
+    assert np.array_equal(got[:8], np.array(E2M1_MAGNITUDES))
+    assert np.array_equal(got[8:], -np.array(E2M1_MAGNITUDES)) and np.signbit(got[8])
+
+
+def pin_e2m1_encode():
+    codes = np.arange(16)
+    vals = np.array(E2M1_MAGNITUDES + tuple(-m for m in E2M1_MAGNITUDES), np.float32)
+    vals[8] = -0.0
+    assert np.array_equal(O.e2m1_encode(vals), codes.astype(np.uint8))
+    # Midpoints: 0.25 -> 0, 0.75 -> 1, 1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4 (even codes).
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    assert O.e2m1_encode(mids).tolist() == [0, 2, 2, 4, 4, 6, 6]
+    assert O.e2m1_encode(-mids).tolist() == [8, 10, 10, 12, 12, 14, 14]
+    up = np.nextafter(mids, np.float32(np.inf))
+    dn = np.nextafter(mids, np.float32(0))
+    assert O.e2m1_encode(up).tolist() == [1, 2, 3, 4, 5, 6, 7]
+    assert O.e2m1_encode(dn).tolist() == [0, 1, 2, 3, 4, 5, 6]
+    assert O.e2m1_encode(np.array([6.0, 6.5, 100.0, -1e30], np.float32)).tolist() == [7, 7, 7, 15]
+    r = np.random.default_rng(5)
+    y = np.concatenate([r.uniform(-7, 7, 100000), r.standard_normal(20000) * 0.3]).astype(np.float32)
+    got = O.e2m1_decode(O.e2m1_encode(y))
+    assert np.array_equal(got, _e2m1_round_here(y))
+
+
+def pin_nvfp4_worked_group():
+    """Groups worked by hand from the format: with g = 1 and max |x| = 6 the block scale is 1.0
+    (E4M3 code 0x38) and each value on the E2M1 grid keeps its own code; 0.25 is a tie that goes
+    to the even code 0.  Doubling g halves the block scale (0x30); an all-zero group stores
+    zero codes and a zero scale.  The byte image puts dimension 2i in the low nibble."""
+    x = np.array([-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6, 0.25], np.float32)
+    want = [0xF, 0xE, 0xD, 0xC, 0xB, 0xA, 0x9, 0x0, 0x1, 0x2, 0x3, 0x4, 0x5, 0x6, 0x7, 0x0]
+    codes, sc = O.nvfp4_quantize(x[None, :], np.float32(1.0))
+    assert codes[0].tolist() == want and sc[0].tolist() == [0x38]
+    codes, sc = O.nvfp4_quantize(x[None, :], np.float32(2.0))
+    assert codes[0].tolist() == want and sc[0].tolist() == [0x30]
+    codes, sc = O.nvfp4_quantize(np.zeros((1, 32), np.float32), np.float32(0.01))
+    assert not codes.any() and not sc.any()
+    # amax 3 with g = 1: scale 0.5 (0x30), so 3 -> 6 (code 7) and 0.2 / 0.5 = 0.4 -> 0.5 (code 1).
+    y = np.zeros(16, np.float32)
+    y[0], y[1], y[2] = 3.0, -0.2, 0.7
+    codes, sc = O.nvfp4_quantize(y[None, :], np.float32(1.0))
+    assert sc[0].tolist() == [0x30] and codes[0, :3].tolist() == [0x7, 0x9, 0x3]
+    # Byte image of a 1-block, 1-head, 2-slot pool of head_dim 32 (64 bytes per run of K or V).
+    pool = O.new_pool(1, 1, 1, 2, 32, "nvfp4", np.ones((1, 1), np.float32), np.ones((1, 1), np.float32))
+    row = np.array([1, 2, 3, 4, 6, 0.5, 1.5, 0] * 4, np.float32).reshape(1, 1, 32)
+    O.kv_append(pool, 0, row, row, "f32", np.array([0, 1]), np.array([1]), np.array([[0]]))
+    img = O.nvfp4_pool_bytes(pool)
+    assert img.shape == (1, 1, 2, 1, 2 * 16 + 2 * 2)
+    # Slot 1 of K: codes 2, 4, 5, 6 | 7, 1, 3, 0 (scale 1.0: max 6) -> bytes 0x42, 0x65, 0x17, 0x03.
+    assert img[0, 0, 0, 0, 16:20].tolist() == [0x42, 0x65, 0x17, 0x03]
+    assert img[0, 0, 0, 0, 32 + 2:32 + 4].tolist() == [0x38, 0x38]
+    assert img[0, 0, 0, 0, 0:16].tolist() == [0x7F] * 16  # slot 0 untouched
+
+
+def pin_nvfp4_scale_invariance():
+    """Scaling the values and the global scale by the same power of two changes no stored code
+    (all quantities stay exact and inside the E4M3 normal range)."""
+    r = np.random.default_rng(9)
+    x = (r.standard_normal((50, 4, 128)) * 0.7).astype(np.float32)
+    g = (np.abs(x).max(axis=(0, 2)) / (6 * 448)).astype(np.float32)[None, :]
+    c0, s0 = O.nvfp4_quantize(x, g)
+    for k in (-3, 2, 5):
+        c1, s1 = O.nvfp4_quantize(x * np.float32(2.0 ** k), g * np.float32(2.0 ** k))
+        assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+
+
+def pin_nvfp4_error_bound():
+    """Dequantised values stay within half an E2M1 step (at most 1, at the top binade) of
+    x / (s g), and the block scale is E4M3's rounding of max |x| / (6 g): relative error at
+    most 2^-4 in the normal range."""
+    r = np.random.default_rng(10)
+    x = (r.standard_normal((200, 2, 128)) * r.uniform(0.01, 3, (200, 2, 1))).astype(np.float32)
+    g = (np.abs(x).max(axis=(0, 2)) / (6 * 448)).astype(np.float32)[None, :]
+    codes, sc = O.nvfp4_quantize(x, g)
+    s = torch.from_numpy(sc).view(torch.float8_e4m3fn).to(torch.float64).numpy()  # [n][H][8]
+    gg = g.astype(np.float64)[..., None]
+    amax = np.abs(x.astype(np.float64)).reshape(200, 2, 8, 16).max(axis=-1)
+    target = amax / (6 * gg)
+    normal = target >= 2.0 ** -6
+    assert (np.abs(s - target)[normal] <= target[normal] * 2.0 ** -4 * (1 + 1e-12)).all()
+    mag = np.array(E2M1_MAGNITUDES)[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    y = x.astype(np.float64) / (np.repeat(s, 16, axis=-1) * gg)
+    step = np.where(np.abs(y) < 2, 0.25, np.where(np.abs(y) < 4, 0.5, 1.0))
+    assert (np.abs(mag - np.clip(y, -6, 6)) <= step * (1 + 1e-6)).all()
+
+
 def pin_bf16_decode():
     bits = np.arange(0, 65536, 7, dtype=np.uint32).astype(np.uint16)
     ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
@@ -215,6 +330,15 @@ def pin_dense_equivalence():
         ref = dense_sdpa(w)
         err = np.abs(out - ref).max()
         assert err <= 1e-12, (w.name, err)
+
+
+def pin_nvfp4_dense():
+    """An NVFP4 cache: the paged oracle against SDPA over values dequantised here (E2M1 table,
+    torch's E4M3 conversion), prefill chunk and decode rows, several blocks and a ragged tail."""
+    w = W.build("nv", seed=21, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=8,
+                num_kv_heads=2, head_dim=128, block_size=16, seq_lens=[70, 33, 5], q_lens=[20, 1, 1])
+    out, _ = run_oracle(w)
+    assert np.abs(out - dense_sdpa(w)).max() <= 1e-12
 
 
 def pin_noncausal_dense():
@@ -512,5 +636,6 @@ ALL_PINS = [
     pin_e4m3_decode_table, pin_e4m3_encode, pin_bf16_decode, pin_block_mapping_example, pin_append_roundtrip,
     pin_dense_equivalence, pin_noncausal_dense, pin_brute_force, pin_lse_logsumexp, pin_permutation_invariance,
     pin_softmax_rows, pin_closed_forms, pin_split_reduce, pin_prefix_sharing, pin_window_dense, pin_window_limits,
-    pin_window_brute_force, pin_block_copy,
+    pin_window_brute_force, pin_block_copy, pin_e2m1_table, pin_e2m1_encode, pin_nvfp4_worked_group,
+    pin_nvfp4_scale_invariance, pin_nvfp4_error_bound, pin_nvfp4_dense,
 ]

@@ -17,6 +17,10 @@ _orig_decode = O.decode_bits
 _orig_split = O.split_kv_reduce
 _orig_start = O.key_start
 _orig_copy = O.copy_block_prefix
+_orig_e2m1_encode = O.e2m1_encode
+_orig_e2m1_decode = O.e2m1_decode
+_orig_pool_bytes = O.nvfp4_pool_bytes
+_orig_quantize = O.nvfp4_quantize
 
 
 def _gqa_modulo(h, hq, hkv):
@@ -92,6 +96,59 @@ def _copy_off_by_one(pool, src, dst, n):
     return _orig_copy(pool, src, dst, [max(0, int(x) - 1) for x in n])
 
 
+def _e2m1_ties_up(y32):
+    """Ties of the E2M1 rounding go to the larger magnitude instead of the even code."""
+    y = np.asarray(y32, np.float32)
+    a = np.abs(y)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    bump = np.isin(a, mids)
+    return _orig_e2m1_encode(np.where(bump, np.nextafter(a, np.float32(np.inf)) * np.sign(y), y).astype(np.float32))
+
+
+def _e2m1_exponent_bias_0(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    v = _orig_e2m1_decode(codes)
+    return np.where(((c >> 1) & 3) != 0, 2.0 * v, v)
+
+
+def _nibbles_swapped(pool):
+    img = _orig_pool_bytes(pool).copy()
+    n = pool.bits.shape[4] * pool.bits.shape[5] // 2
+    img[..., :n] = ((img[..., :n] >> 4) | (img[..., :n] << 4)) & 0xFF
+    return img
+
+
+def _quantize_scale_over_4(x32, g):
+    """Block scale max / (4 g) instead of max / (6 g); element codes against that scale."""
+    x = np.asarray(x32, np.float32)
+    D = x.shape[-1]
+    grp = x.reshape(x.shape[:-1] + (D // 16, 16))
+    gg = np.asarray(g, np.float32)[..., None]
+    sc = O.e4m3_encode((np.abs(grp).max(axis=-1) / (np.float32(4.0) * gg)).astype(np.float32))
+    s = O.e4m3_decode(sc).astype(np.float32)
+    denom = np.where(s == 0, 1, s * gg).astype(np.float32)
+    codes = O.e2m1_encode((grp / denom[..., None]).astype(np.float32))
+    return np.where((s == 0)[..., None], 0, codes).reshape(x.shape).astype(np.uint8), sc
+
+
+def _quantize_without_global(x32, g):
+    """Element codes from x / s, dropping the global scale."""
+    codes, sc = _orig_quantize(x32, g)
+    x = np.asarray(x32, np.float32)
+    D = x.shape[-1]
+    s = O.e4m3_decode(sc).astype(np.float32)
+    y = x.reshape(x.shape[:-1] + (D // 16, 16)) / np.where(s == 0, 1, s)[..., None]
+    return O.e2m1_encode(y.astype(np.float32)).reshape(x.shape), sc
+
+
+def _gather_without_block_scale(pool, layer, row, kvh, which, n):
+    if pool.dtype != "nvfp4":
+        return _orig_gather(pool, layer, row, kvh, which, n)
+    t = np.arange(n)
+    phys, slot = O.block_address(row, t, pool.block_size)
+    return O.e2m1_decode(pool.bits[phys, layer, which, kvh, slot, :]) * np.float64(pool.scale(which, layer)[kvh])
+
+
 def _split_sign(po, pl):
     return _orig_split(po, -np.asarray(pl))
 
@@ -113,6 +170,13 @@ MUTATIONS = {
     "window_one_too_wide": [("key_start", _window_one_too_wide)],
     "copy_whole_block": [("copy_block_prefix", _copy_whole_block)],
     "copy_one_token_short": [("copy_block_prefix", _copy_off_by_one)],
+    "e2m1_ties_up": [("e2m1_encode", _e2m1_ties_up)],
+    "e2m1_exponent_bias_0": [("e2m1_decode", _e2m1_exponent_bias_0)],
+    "nvfp4_nibbles_swapped": [("nvfp4_pool_bytes", _nibbles_swapped)],
+    "nvfp4_block_scale_over_4": [("nvfp4_quantize", _quantize_scale_over_4)],
+    "nvfp4_codes_without_global_scale": [("nvfp4_quantize", _quantize_without_global)],
+    "nvfp4_gather_drops_block_scale": [("gather_rows", _gather_without_block_scale)],
+    "nvfp4_group_32": [("NVFP4_GROUP", 32)],
 }
 
 
