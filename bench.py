@@ -49,19 +49,20 @@ def elem_bytes(dtype: str) -> int:
 
 def algorithmic_bytes(w, plan_info=None) -> dict:
     """Bytes one step must move: distinct K/V bytes read, q, out, tables, scales, partials, appended rows."""
-    eb = elem_bytes(w.kv_dtype)
-    row = w.num_kv_heads * w.head_dim * eb  # one token of one layer, K or V
+    from paged_kv_attention_block_b200.workloads import kv_row_bytes
+
+    row = w.num_kv_heads * kv_row_bytes(w.kv_dtype, w.head_dim)  # one token of one layer, K or V (NVFP4: + block scales)
     kv = sum(tokens for _, tokens in w.distinct_kv_blocks()) * row * 2
     qb = elem_bytes(w.q_dtype)
     q = w.total_q * w.num_q_heads * w.head_dim * qb
     out = q
     tables = sum((int(L) + w.block_size - 1) // w.block_size for L in w.seq_lens) * 4 + w.num_seqs * 8
-    scales = 2 * w.num_kv_heads * 4 if w.kv_dtype == "e4m3" else 0
+    scales = 2 * w.num_kv_heads * 4 if w.kv_dtype in ("e4m3", "nvfp4") else 0
     parts = 0
     if plan_info:
         parts = plan_info["num_partial_rows"] * (w.head_dim + 1) * 4 * 2
-    new_rows = w.total_q * w.num_kv_heads * w.head_dim * 2
-    append = new_rows * elem_bytes(w.kv_in_dtype) + new_rows * eb
+    new_rows = w.total_q * w.num_kv_heads * 2  # (token, head) rows of K and V
+    append = new_rows * (w.head_dim * elem_bytes(w.kv_in_dtype) + kv_row_bytes(w.kv_dtype, w.head_dim))
     attn = kv + q + out + tables + scales + parts
     # The attention kernels alone: everything but the merge's read of the partials and its output.
     kernels = kv + q + out + tables + scales + parts // 2
@@ -473,70 +474,36 @@ def run_prefill_only(w, dev, api, runner, plan_kw, steps: int = 100):
 
 
 def run_e2e(args, w, dw, plan_opts, dev, stream, api):
-    """The step end to end through the public API, as a serving loop runs it: every step copies
-    its inputs (q, new K/V, lengths, positions, tables) from pinned host memory, appends, plans on
-    the host, uploads the plan, runs attention and copies the output back to pinned host memory.
-    Two input/output buffer sets and plan buffers alternate, the copies run on their own stream,
-    so step i+1's copies and host planning overlap step i's kernels.  Time = events around n
-    back-to-back steps (all copies inside), divided by n."""
+    """The step end to end through the public API as a serving loop runs it (api.GraphStep):
+    every step plans on the host, copies its packed inputs (q, new K/V, lengths, positions,
+    tables) and its plan from page-locked host memory, appends, runs attention and copies the
+    output back to page-locked host memory, as one graph replay per step; two buffer slots let
+    the host plan step i+1 while the GPU runs step i.  Time = events around n back-to-back steps
+    (every copy inside), divided by n."""
     import torch
 
     names = {"q": dw.q, "k_new": dw.k_new, "v_new": dw.v_new, "cu_q": dw.cu_q, "seq_lens": dw.seq_lens,
              "start_pos": dw.start_pos, "block_tables": dw.block_tables}
-    host = {k: v.detach().cpu().pin_memory() for k, v in names.items()}
-    outs_h = [torch.empty(dw.q.shape, dtype=dw.q.dtype).pin_memory() for _ in range(2)]
-    devb = [{k: torch.empty_like(v) for k, v in names.items()} for _ in range(2)]
-    outs_d = [torch.empty_like(dw.q) for _ in range(2)]
-    cu, sl, bt = w.cu_q_lens, w.seq_lens, w.block_tables
     kw = dict(num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=w.block_size,
-              kv_dtype=w.kv_dtype, causal=w.causal, block_tables=bt, **plan_opts)
-    plans = [api.plan_attention(cu, sl, **kw) for _ in range(2)]
-    ws = torch.empty(max(plans[0].workspace_bytes, 256), dtype=torch.uint8, device=dev)
-    copy = torch.cuda.Stream(dev)
-    ready = [torch.cuda.Event() for _ in range(2)]     # inputs of a slot copied in
-    consumed = [torch.cuda.Event() for _ in range(2)]  # kernels of a slot done with its inputs and plan
-    fetched = [torch.cuda.Event() for _ in range(2)]   # output of a slot copied out
-    pending = [False, False]
-
-    def step(i):
-        b = i % 2
-        if pending[b]:
-            consumed[b].synchronize()  # the plan buffer's last upload has run: it may be rewritten
-        api.plan_attention(cu, sl, buffer=plans[b].buffer, **kw)
-        with torch.cuda.stream(copy):
-            copy.wait_event(consumed[b])
-            copy.wait_event(fetched[b])
-            for name in names:
-                devb[b][name].copy_(host[name], non_blocking=True)
-            ready[b].record(copy)
-        with torch.cuda.stream(stream):
-            stream.wait_event(ready[b])
-            d = devb[b]
-            api.kv_append(dw.cache, d["k_new"], d["v_new"], d["cu_q"], d["start_pos"], d["block_tables"])
-            api.paged_attention(dw.cache, d["q"], d["cu_q"], d["seq_lens"], d["block_tables"], plans[b],
-                                w.softmax_scale, w.causal, out=outs_d[b], workspace=ws)
-            consumed[b].record(stream)
-        with torch.cuda.stream(copy):
-            copy.wait_event(consumed[b])
-            outs_h[b].copy_(outs_d[b], non_blocking=True)
-            fetched[b].record(copy)
-        pending[b] = True
-
-    for i in range(4):
-        step(i)
-    torch.cuda.synchronize(dev)
+              kv_dtype=w.kv_dtype, causal=w.causal, **plan_opts)
+    gs = api.GraphStep(dw.cache, names, kw, w.softmax_scale, w.causal, stream=torch.cuda.Stream(dev))
+    for views in gs.host:
+        for k, v in names.items():
+            views[k].copy_(v.cpu())
+    for _ in range(4):
+        gs.wait(gs.run())
     n = max(2, min(args.steps, 500))
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    copy.wait_event(s)
-    for i in range(n):
-        step(i)
-    stream.wait_event(fetched[(n - 1) % 2])
-    e.record(stream)
+    s.record(gs.stream)
+    slot = None
+    for _ in range(n):
+        slot = gs.run()
+    e.record(gs.stream)
+    out = gs.wait(slot)
     e.synchronize()
-    h2d = sum(v.numel() * v.element_size() for v in host.values()) + plans[0].info["plan_bytes"]
-    d2h = outs_h[0].numel() * outs_h[0].element_size()
-    return {"ms": s.elapsed_time(e) / n, "h2d": int(h2d), "d2h": int(d2h)}
+    assert torch.isfinite(out.float()).all(), "non-finite output in the end-to-end loop"
+    plan_bytes = gs._plans[0].info["plan_bytes"]
+    return {"ms": s.elapsed_time(e) / n, "h2d": int(gs.h2d_bytes + plan_bytes), "d2h": int(gs.d2h_bytes)}
 
 
 def main():

@@ -13,7 +13,7 @@ from importlib import import_module
 _API = (
     "PkvError", "Cache", "Plan", "kv_append", "plan_attention", "paged_attention", "split_kv_reduce",
     "attention_workspace_bytes", "default_num_ctas", "library_path", "status_string", "DTYPE_CODES",
-    "decode_step_e2e", "paged_attention_noalloc",
+    "GraphStep", "paged_attention_noalloc",
 )
 
 __all__ = list(_API) + ["workloads"]

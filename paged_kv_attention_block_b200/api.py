@@ -28,12 +28,12 @@ if not os.path.exists(library_path()):
 
 _lib = C.CDLL(library_path())
 
-PKV_F32, PKV_BF16, PKV_F16, PKV_FP8_E4M3 = 0, 1, 2, 3
-DTYPE_CODES = {"f32": PKV_F32, "bf16": PKV_BF16, "f16": PKV_F16, "e4m3": PKV_FP8_E4M3}
+PKV_F32, PKV_BF16, PKV_F16, PKV_FP8_E4M3, PKV_NVFP4 = 0, 1, 2, 3, 4
+DTYPE_CODES = {"f32": PKV_F32, "bf16": PKV_BF16, "f16": PKV_F16, "e4m3": PKV_FP8_E4M3, "nvfp4": PKV_NVFP4}
 _TORCH_CODES = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16,
                 torch.float8_e4m3fn: PKV_FP8_E4M3, torch.uint8: PKV_FP8_E4M3}
 _CODE_TORCH = {PKV_F32: torch.float32, PKV_BF16: torch.bfloat16, PKV_F16: torch.float16,
-               PKV_FP8_E4M3: torch.uint8}
+               PKV_FP8_E4M3: torch.uint8, PKV_NVFP4: torch.uint8}
 
 
 class PkvError(RuntimeError):
@@ -119,13 +119,16 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 @dataclass
 class Cache:
-    """A paged KV pool ``[num_blocks][num_layers][2][Hkv][B][D]`` on the GPU and the layer a call uses."""
+    """A paged KV pool ``[num_blocks][num_layers][2][Hkv][B][D]`` on the GPU and the layer a call uses.
+
+    An NVFP4 pool is ``[num_blocks][num_layers][2][Hkv][B * D * 9 / 16]`` bytes: per run, B rows
+    of D/2 bytes of E2M1 codes, then B rows of D/16 bytes of E4M3 block scales."""
 
     pool: torch.Tensor
     kv_dtype: int
     block_size: int
     layer: int = 0
-    k_scale: torch.Tensor | None = None  # float32 [num_layers][Hkv], fp8 pools
+    k_scale: torch.Tensor | None = None  # float32 [num_layers][Hkv], fp8 and NVFP4 pools
     v_scale: torch.Tensor | None = None
 
     @staticmethod
@@ -133,10 +136,12 @@ class Cache:
                  device="cuda", fill_nan: bool = True, k_scale=None, v_scale=None) -> "Cache":
         code = DTYPE_CODES[kv_dtype]
         shape = (num_blocks, num_layers, 2, num_kv_heads, block_size, head_dim)
+        if code == PKV_NVFP4:
+            shape = (num_blocks, num_layers, 2, num_kv_heads, block_size * (head_dim // 2 + head_dim // 16))
         tdt = _CODE_TORCH[code]
         pool = torch.empty(shape, dtype=tdt, device=device)
-        if fill_nan:  # sentinel NaNs in every slot no sequence owns
-            if code == PKV_FP8_E4M3:
+        if fill_nan:  # sentinel NaNs in every slot no sequence owns (NVFP4: NaN block scales)
+            if code in (PKV_FP8_E4M3, PKV_NVFP4):
                 pool.fill_(0x7F)
             else:
                 pool.fill_(float("nan"))
@@ -149,11 +154,13 @@ class Cache:
 
     @property
     def head_dim(self) -> int:
+        if self.kv_dtype == PKV_NVFP4:
+            return self.pool.shape[4] // self.block_size * 16 // 9
         return self.pool.shape[5]
 
     def _c(self) -> _Cache:
         p = self.pool
-        return _Cache(p.data_ptr(), p.shape[0], p.shape[1], self.layer, p.shape[3], p.shape[5], self.block_size,
+        return _Cache(p.data_ptr(), p.shape[0], p.shape[1], self.layer, p.shape[3], self.head_dim, self.block_size,
                       self.kv_dtype, _ptr(self.k_scale), _ptr(self.v_scale))
 
 
@@ -305,22 +312,99 @@ def split_kv_reduce(partial_o: torch.Tensor, partial_lse: torch.Tensor, out_dtyp
     return out, out_lse
 
 
-def decode_step_e2e(*args, **kwargs):  # defined in bench-facing helpers below
-    return _decode_step_e2e(*args, **kwargs)
+class GraphStep:
+    """One serving step from page-locked host inputs, replayed as a CUDA graph per buffer slot.
 
+    A step is: one host-to-device copy of the packed inputs (q, new K/V rows, cu_q_lens,
+    seq_lens, start_pos, block tables) and of the step's plan, ``kv_append``,
+    ``paged_attention``, and one device-to-host copy of the output.  Every call of
+    :meth:`run` re-plans on the host (into the slot's page-locked plan buffer, which the
+    graph uploads) and replays the slot's graph; with two slots the host plans step i+1
+    while the GPU runs step i.  The graph is captured again whenever a new plan differs
+    from the captured one in a launch-shaping field (item and merge counts, CTA counts).
 
-def _decode_step_e2e(cache: Cache, host: dict, dev: dict, plan_fn, softmax_scale: float, causal: bool, stream=None):
-    """One step from pinned host inputs: H2D copies, kv_append, plan, attention, D2H of the output.
-
-    ``host`` holds pinned CPU tensors (q, k_new, v_new, cu_q, seq_lens, start_pos,
-    block_tables, out); ``dev`` holds same-shaped device buffers and a workspace.
-    ``plan_fn`` returns the host Plan for this step's lengths.
+    Callers write each step's inputs into :attr:`host` (named page-locked views of one
+    buffer) before :meth:`run`, and read the output from the tensor that :meth:`wait`
+    returns.
     """
-    for name in ("q", "k_new", "v_new", "cu_q", "seq_lens", "start_pos", "block_tables"):
-        dev[name].copy_(host[name], non_blocking=True)
-    kv_append(cache, dev["k_new"], dev["v_new"], dev["cu_q"], dev["start_pos"], dev["block_tables"], stream=stream)
-    plan = plan_fn()
-    paged_attention(cache, dev["q"], dev["cu_q"], dev["seq_lens"], dev["block_tables"], plan, softmax_scale, causal,
-                    out=dev["out"], workspace=dev["workspace"], stream=stream)
-    host["out"].copy_(dev["out"], non_blocking=True)
-    return plan
+
+    _FIELDS = ("q", "k_new", "v_new", "cu_q", "seq_lens", "start_pos", "block_tables")
+    _SHAPE_KEYS = ("plan_bytes", "workspace_bytes", "num_items", "num_tc_items", "num_reduce", "num_parts",
+                   "num_partial_rows", "num_ctas")
+
+    def __init__(self, cache: Cache, like: dict, plan_kwargs: dict, softmax_scale: float, causal: bool = True,
+                 slots: int = 2, stream=None):
+        self.cache, self.plan_kwargs, self.scale, self.causal = cache, dict(plan_kwargs), float(softmax_scale), causal
+        self.stream = stream if stream is not None else torch.cuda.Stream()
+        dev = self.stream.device
+        # One page-locked buffer and one device buffer per slot, each field 256-byte aligned.
+        offs, total = {}, 0
+        for name in self._FIELDS:
+            t = like[name]
+            offs[name] = (total, t.dtype, tuple(t.shape))
+            total = (total + t.numel() * t.element_size() + 255) // 256 * 256
+
+        def views(buf):
+            return {n: buf[o:o + int(np.prod(sh)) * torch.empty((), dtype=dt).element_size()].view(dt).view(sh)
+                    for n, (o, dt, sh) in offs.items()}
+
+        self.h2d_bytes = total
+        self._hbuf = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(slots)]
+        self._dbuf = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(slots)]
+        self.host = [views(b) for b in self._hbuf]
+        self._dev = [views(b) for b in self._dbuf]
+        q = like["q"]
+        self._out_d = [torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(slots)]
+        self._out_h = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(slots)]
+        self.d2h_bytes = q.numel() * q.element_size()
+        self._plans = [None] * slots
+        self._graphs = [None] * slots
+        self._shape = [None] * slots
+        self._done = [torch.cuda.Event() for _ in range(slots)]
+        self._pending = [False] * slots
+        self._ws = None
+        self._slot = 0
+
+    def _plan_into(self, b: int) -> Plan:
+        h = self.host[b]
+        buf = None if self._plans[b] is None else self._plans[b].buffer
+        return plan_attention(h["cu_q"].numpy(), h["seq_lens"].numpy(), block_tables=h["block_tables"].numpy(),
+                              buffer=buf, **self.plan_kwargs)
+
+    def _capture(self, b: int, plan: Plan) -> None:
+        if self._ws is None or self._ws.numel() < plan.workspace_bytes:
+            self._ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=self.stream.device)
+        d = self._dev[b]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self._dbuf[b].copy_(self._hbuf[b], non_blocking=True)
+            kv_append(self.cache, d["k_new"], d["v_new"], d["cu_q"], d["start_pos"], d["block_tables"])
+            paged_attention(self.cache, d["q"], d["cu_q"], d["seq_lens"], d["block_tables"], plan, self.scale,
+                            self.causal, out=self._out_d[b], workspace=self._ws)
+            self._out_h[b].copy_(self._out_d[b], non_blocking=True)
+        self._graphs[b] = g
+
+    def run(self) -> int:
+        """Plan and launch one step on the next slot; returns the slot (pass it to :meth:`wait`)."""
+        b = self._slot
+        self._slot = (b + 1) % len(self._graphs)
+        if self._pending[b]:
+            self._done[b].synchronize()  # the slot's last replay has read its inputs and plan
+        plan = self._plan_into(b)
+        self._plans[b] = plan
+        shape = tuple(plan.info[k] for k in self._SHAPE_KEYS)
+        if self._graphs[b] is None or shape != self._shape[b]:
+            torch.cuda.synchronize(self.stream.device)
+            self._capture(b, plan)
+            self._shape[b] = shape
+        with torch.cuda.stream(self.stream):
+            self._graphs[b].replay()
+            self._done[b].record(self.stream)
+        self._pending[b] = True
+        return b
+
+    def wait(self, slot: int) -> torch.Tensor:
+        """Block until the slot's step has finished; returns its page-locked host output."""
+        self._done[slot].synchronize()
+        self._pending[slot] = False
+        return self._out_h[slot]

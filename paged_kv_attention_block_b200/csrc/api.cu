@@ -159,8 +159,8 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   if (!pkv::attn_kernel_for(c.kv_dtype, q_dtype, c.head_dim, c.block_size, &k))
     return pkv_fail(PKV_ERR_UNSUPPORTED, "paged_attention: kv_dtype %d with q_dtype %d, head_dim %d", c.kv_dtype,
                     q_dtype, c.head_dim);
-  if (c.kv_dtype == PKV_FP8_E4M3 && (!c.k_scale || !c.v_scale))
-    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: fp8 pool needs k_scale and v_scale");
+  if ((c.kv_dtype == PKV_FP8_E4M3 || c.kv_dtype == PKV_NVFP4) && (!c.k_scale || !c.v_scale))
+    return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: fp8 and NVFP4 pools need k_scale and v_scale");
   if (!(softmax_scale > 0.f) || softmax_scale == INFINITY)
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: softmax_scale must be positive and finite");
   pkv::AttnKernel ktc{};

@@ -48,15 +48,22 @@ namespace pkv {
 template <int D, int KV, bool QBF>
 struct TmaCfg {
   using L = Cfg<D, KV, QBF>;
+  static constexpr bool FP4 = KV == KV_NVFP4;
   static constexpr int ELEM = L::ELEM;
-  static constexpr int RB = L::RB;
-  // Keys per tile: 32 for 256-byte rows, 64 for 128-byte rows (16 KB stages).
+  // Bytes per K or V row (NVFP4: the packed codes; the block scales travel separately).
+  static constexpr int RB = FP4 ? D / 2 : L::RB;
+  // Keys per tile: 32 for 256-byte rows, 64 for 128- and 64-byte rows.
   static constexpr int TK = RB == 256 ? 32 : 64;
-  static constexpr int HALVES = RB / 128;  // 128-byte column slabs per row
-  // Stage layout: [slab][K|V][TK rows][128 B]; K tile at +0, V tile at +TK*128.
+  static constexpr int HALVES = FP4 ? 1 : RB / 128;  // 128-byte column slabs per row
+  // Stage layout: [slab][K|V][TK rows][128 B]; K tile at +0, V tile at +TK*128.  NVFP4:
+  // K codes [TK][64 B] (64-byte swizzle), V codes, then K and V block scales [TK][D/16 B].
   static constexpr int SLAB = 2 * TK * 128;
   static constexpr int TILE_BYTES = TK * RB;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int V_OFF = FP4 ? TILE_BYTES : TK * 128;
+  static constexpr int SCALE_ROW = FP4 ? D / 16 : 0;
+  static constexpr int KS_OFF = 2 * TILE_BYTES;
+  static constexpr int VS_OFF = KS_OFF + TK * SCALE_ROW;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES + 2 * TK * SCALE_ROW;
   // A multiple of 4: decode tiles go round-robin to the 4 consumer warps by tile
   // index within the item, so within an item every tile that lands in a given
   // stage belongs to the same warp and the stage's phases are consumed in order;
@@ -64,7 +71,7 @@ struct TmaCfg {
   // every tile (prefill) orders them.
   // Four 16 KB stages (64 KB) leave room for two CTAs per SM: twice the producers and consumer
   // warps of one large-ring CTA, which measured faster than a 12-stage ring with one CTA per SM.
-  static constexpr int NST = 4 * std::max(1, std::min(12, (64 * 1024) / STAGE_BYTES) / 4);
+  static constexpr int NST = FP4 ? 8 : 4 * std::max(1, std::min(12, (64 * 1024) / STAGE_BYTES) / 4);
   static constexpr int IR = 4;  // item descriptor slots
   static constexpr int MERGE_BYTES = 4 * 16 * D * 4 + 2 * 4 * 16 * 4;
   static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * IR + 1);
@@ -72,7 +79,8 @@ struct TmaCfg {
   static constexpr int IDS_BYTES = 32 * 4;
   static constexpr int SMEM = 1024 + NST * STAGE_BYTES + MERGE_BYTES + BAR_BYTES + DESC_BYTES + IDS_BYTES + 16;
   static constexpr int THREADS = 160;
-  static_assert(RB == 128 || RB == 256, "TMA path takes 128- or 256-byte rows");
+  static_assert(RB == 128 || RB == 256 || (FP4 && D == 128), "TMA path takes 128- or 256-byte rows, or NVFP4 d 128");
+  static_assert(STAGE_BYTES % 1024 == 0, "stages keep the swizzle atoms aligned");
   static_assert(NST % 4 == 0, "stage count must be a multiple of the consumer warp count");
   static_assert(2 * SMEM <= 228 * 1024, "two CTAs per SM");
 };
@@ -102,7 +110,24 @@ struct DecState {
 template <int KV>
 PKV_DEVICE int dec_dim(int mt, int e, int g4) {
   if constexpr (KV == KV_E4M3) return 32 * (mt >> 1) + 2 * g4 + 16 * (e >> 1) + (mt & 1);
+  else if constexpr (KV == KV_NVFP4) return 64 * (mt >> 2) + 32 * (e >> 1) + 4 * g4 + (mt & 3);
   else return 16 * mt + g4 + 8 * (e >> 1);
+}
+
+// The decode tiles of fp8 and NVFP4 pools hold values times 2^-8 (E4M3) or 2^-7 (E2M1 code
+// times block scale): x times the power of two back (exact).
+template <int KV>
+PKV_DEVICE float deq_undo(float x) {
+  if constexpr (KV == KV_E4M3) return x * 256.f;
+  else if constexpr (KV == KV_NVFP4) return x * 128.f;
+  else return x;
+}
+
+// NVFP4 rows are 64 bytes; TMA's 64-byte swizzle XORs address bits 7..8 into the
+// 16-byte chunk index (bits 4..5), so the 8-row ldmatrix phases hit distinct banks.
+PKV_DEVICE uint32_t sw64(int row, int byte) {
+  const uint32_t lin = uint32_t(row) * 64 + uint32_t(byte);
+  return lin ^ (((lin >> 7) & 3) << 4);
 }
 
 // Per-lane shared-memory offsets of the K (A operand) and V (A^T operand)
@@ -110,7 +135,7 @@ PKV_DEVICE int dec_dim(int mt, int e, int g4) {
 // (the swizzle phase repeats every 8 rows).
 template <int D, int KV, bool QBF>
 struct DecOffsets {
-  static constexpr int N = KV == KV_E4M3 ? D / 32 : D / 16;
+  static constexpr int N = KV == KV_NVFP4 ? 2 : (KV == KV_E4M3 ? D / 32 : D / 16);
   uint32_t k[N], v[N];
 };
 
@@ -120,7 +145,13 @@ PKV_DEVICE void dec_offsets(DecOffsets<D, KV, QBF>& o, int lane) {
   const int mi = lane >> 3, r8 = lane & 7;
 #pragma unroll
   for (int i = 0; i < DecOffsets<D, KV, QBF>::N; ++i) {
-    if constexpr (KV == KV_E4M3) {
+    if constexpr (KV == KV_NVFP4) {
+      // Column pair i = 16-byte chunks 2i, 2i+1 (dims 64i .. 64i+63).  K: matrix mi holds rows
+      // 8*(mi & 1) .. +7 of chunk 2i + (mi >> 1); V (transposed): keys 8*(mi >> 1) .. +7 of
+      // chunk 2i + (mi & 1).
+      o.k[i] = sw64((mi & 1) * 8 + r8, 16 * (2 * i + (mi >> 1)));
+      o.v[i] = sw64((mi >> 1) * 8 + r8, 16 * (2 * i + (mi & 1)));
+    } else if constexpr (KV == KV_E4M3) {
       o.k[i] = tile_offset<T::RB, T::TK, T::SLAB>((mi & 1) * 8 + r8, 32 * i + (mi >> 1) * 16);
       o.v[i] = tile_offset<T::RB, T::TK, T::SLAB>((mi >> 1) * 8 + r8, 32 * i + (mi & 1) * 16);
     } else {
@@ -144,10 +175,18 @@ PKV_DEVICE void dec_load_q(const AttnArgs& a, const ItemDesc& it, int R, DecStat
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t w0 = 0, w1 = 0;
       if (valid) {
-        if constexpr (KV == KV_E4M3) {  // dims permuted to match the fp8 K fragments
+        if constexpr (KV == KV_NVFP4) {
+          // k-step 2c + h pairs dims (b + 2h, b + 2h + 4) and (b + 2h + 1, b + 2h + 5), b = 32c + 8 t4:
+          // the nibble pairs (i, i + 4) of the lane's K word.
+          const uint4 x = *reinterpret_cast<const uint4*>(qrow + 32 * (ks >> 1) + 8 * t4);
+          const uint32_t lo = (ks & 1) ? x.y : x.x, hi = (ks & 1) ? x.w : x.z;
+          w0 = __byte_perm(lo, hi, 0x5410);
+          w1 = __byte_perm(lo, hi, 0x7632);
+        } else if constexpr (KV == KV_E4M3) {
+          // dims 16 ks + 4 t4 + {0, 2} and + {1, 3}: the byte pairs (0, 2), (1, 3) of the K word.
           const uint2 x = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * t4);
-          w0 = x.x;
-          w1 = x.y;
+          w0 = __byte_perm(x.x, x.y, 0x5410);
+          w1 = __byte_perm(x.x, x.y, 0x7632);
         } else {
           w0 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * t4);
           w1 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * t4);
@@ -164,29 +203,64 @@ PKV_DEVICE void dec_load_q(const AttnArgs& a, const ItemDesc& it, int R, DecStat
 }
 
 // One tile owned by this warp: S^T = K Q^T, online softmax per query row, O^T += V^T P^T.
-// `masked`: some key of the tile is at or past some row's limit.
+// `masked`: some key of the tile is at or past some row's limit.  ksc / vsc: the tile's K and
+// V block scales (NVFP4 pools only).
 template <int D, int KV, bool QBF, int NR>
 PKV_DEVICE void dec_tile(DecState<D, KV, QBF, NR>& st, const DecOffsets<D, KV, QBF>& off, uint32_t kbase,
-                         uint32_t vbase, int key0, int lane, float c, bool masked) {
+                         uint32_t vbase, uint32_t ksc, uint32_t vsc, int key0, int lane, float c, bool masked) {
   using T = TmaCfg<D, KV, QBF>;
   constexpr int NKT = T::TK / 16;
   constexpr bool MMA_BF = KV == KV_BF16;
+  constexpr int ROW = KV == KV_NVFP4 ? 64 : 128;  // bytes between rows of a slab
   const int g4 = lane >> 2;
   float s[NR][NKT][4];
 #pragma unroll
   for (int kt = 0; kt < NKT; ++kt) {
 #pragma unroll
     for (int nr = 0; nr < NR; ++nr) s[nr][kt][0] = s[nr][kt][1] = s[nr][kt][2] = s[nr][kt][3] = 0.f;
-    const uint32_t kb = kbase + kt * 16 * 128;
-    if constexpr (KV == KV_E4M3) {
+    const uint32_t kb = kbase + kt * 16 * ROW;
+    if constexpr (KV == KV_NVFP4) {
+      // Block scales of keys g4 and g4 + 8 (eight bytes each: groups 0-3, 4-7); the lane's
+      // eight dims of chunk c lie in group 2c + (t4 >> 1).
+      const int t4 = lane & 3;
+      const uint2 s0 = lds64(ksc + uint32_t(kt * 16 + g4) * 8);
+      const uint2 s1 = lds64(ksc + uint32_t(kt * 16 + g4 + 8) * 8);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        uint32_t r[4];  // key g4 chunk 2p, key g4+8 chunk 2p, key g4 chunk 2p+1, key g4+8 chunk 2p+1
+        ldmatrix_x4(kb + off.k[p], r[0], r[1], r[2], r[3]);
+        const uint32_t w0 = p ? s0.y : s0.x, w1 = p ? s1.y : s1.x;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          // Block scale byte b of keys g4 and g4 + 8 into bytes 1 and 3, as f16x2 (s, s) * 2^7.
+          const uint32_t b = uint32_t(2 * cc + (t4 >> 1));
+          const uint32_t sel = (b << 4) | (b << 12);
+          const uint32_t sg = hmul2(e4m3_b13_f16x2(__byte_perm(w0, 0, sel)), kF16Pow2_15x2);
+          const uint32_t sg8 = hmul2(e4m3_b13_f16x2(__byte_perm(w1, 0, sel)), kF16Pow2_15x2);
+          const uint32_t lo = r[2 * cc], hi = r[2 * cc + 1];
+          // Nibble pairs (i, i+4) of each word as f16x2 values * 2^-14; times the scales: * 2^-7.
+          const uint32_t l0 = hmul2(e2m1_pair_f16x2<0>(lo), sg), l1 = hmul2(e2m1_pair_f16x2<1>(lo), sg);
+          const uint32_t l2 = hmul2(e2m1_pair_f16x2<2>(lo), sg), l3 = hmul2(e2m1_pair_f16x2<3>(lo), sg);
+          const uint32_t h0 = hmul2(e2m1_pair_f16x2<0>(hi), sg8), h1 = hmul2(e2m1_pair_f16x2<1>(hi), sg8);
+          const uint32_t h2 = hmul2(e2m1_pair_f16x2<2>(hi), sg8), h3 = hmul2(e2m1_pair_f16x2<3>(hi), sg8);
+          // k-step 2c + h: k (2t, 2t+1) = dims (b + 2h, b + 2h + 4), (2t+8, 2t+9) = (b + 2h + 1, b + 2h + 5).
+          const uint32_t k0[4] = {l0, h0, l1, h1}, k1[4] = {l2, h2, l3, h3};
+          const int ks = 2 * (2 * p + cc);
+#pragma unroll
+          for (int nr = 0; nr < NR; ++nr) {
+            mma16816<false>(s[nr][kt], k0, st.qb[nr][ks][0], st.qb[nr][ks][1]);
+            mma16816<false>(s[nr][kt], k1, st.qb[nr][ks + 1][0], st.qb[nr][ks + 1][1]);
+          }
+        }
+      }
+    } else if constexpr (KV == KV_E4M3) {
 #pragma unroll
       for (int kp = 0; kp < D / 32; ++kp) {
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4(kb + off.k[kp], r0, r1, r2, r3);
-        const uint32_t a0[4] = {e4m3x2_to_f16x2(uint16_t(r0 & 0xffff)), e4m3x2_to_f16x2(uint16_t(r1 & 0xffff)),
-                                e4m3x2_to_f16x2(uint16_t(r0 >> 16)), e4m3x2_to_f16x2(uint16_t(r1 >> 16))};
-        const uint32_t a1[4] = {e4m3x2_to_f16x2(uint16_t(r2 & 0xffff)), e4m3x2_to_f16x2(uint16_t(r3 & 0xffff)),
-                                e4m3x2_to_f16x2(uint16_t(r2 >> 16)), e4m3x2_to_f16x2(uint16_t(r3 >> 16))};
+        // Values times 2^-8 (undone in the softmax scale).
+        const uint32_t a0[4] = {e4m3_b02_f16x2(r0), e4m3_b02_f16x2(r1), e4m3_b13_f16x2(r0), e4m3_b13_f16x2(r1)};
+        const uint32_t a1[4] = {e4m3_b02_f16x2(r2), e4m3_b02_f16x2(r3), e4m3_b13_f16x2(r2), e4m3_b13_f16x2(r3)};
 #pragma unroll
         for (int nr = 0; nr < NR; ++nr) {
           mma16816<false>(s[nr][kt], a0, st.qb[nr][2 * kp][0], st.qb[nr][2 * kp][1]);
@@ -272,18 +346,50 @@ PKV_DEVICE void dec_tile(DecState<D, KV, QBF, NR>& st, const DecOffsets<D, KV, Q
         pb[nr][1] = movmatrix_trans(pack_f16x2(s[nr][kt][2], s[nr][kt][3]));
       }
     }
-    const uint32_t vb = vbase + kt * 16 * 128;
-    if constexpr (KV == KV_E4M3) {
+    const uint32_t vb = vbase + kt * 16 * ROW;
+    if constexpr (KV == KV_NVFP4) {
+      // V block scales of keys (2t4, 2t4+1) and (2t4+8, 2t4+9): two adjacent 8-byte rows each.
+      // The lane's dims of chunk c lie in group 2c + (g4 >> 2).
+      const int t4 = lane & 3;
+      const uint4 v0 = lds128(vsc + uint32_t(kt * 16 + 2 * t4) * 8);
+      const uint4 v1 = lds128(vsc + uint32_t(kt * 16 + 8 + 2 * t4) * 8);
+      const uint32_t bA = uint32_t(g4 >> 2), bB = bA + 2;
+      const uint32_t selA = (bA << 4) | ((bA + 4) << 12), selB = (bB << 4) | ((bB + 4) << 12);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        uint32_t x[4];  // keys 0-7 chunk 2p, keys 0-7 chunk 2p+1, keys 8-15 chunk 2p, keys 8-15 chunk 2p+1
+        ldmatrix_x4_trans(vb + off.v[p], x[0], x[1], x[2], x[3]);
+        const uint32_t a0w = p ? v0.y : v0.x, a1w = p ? v0.w : v0.z;  // keys 2t4, 2t4+1
+        const uint32_t b0w = p ? v1.y : v1.x, b1w = p ? v1.w : v1.z;  // keys 2t4+8, 2t4+9
+        // (key 2t, key 2t+1) scale pairs in bytes 1 and 3, as f16x2 * 2^7.
+        const uint32_t sc[4] = {hmul2(e4m3_b13_f16x2(__byte_perm(a0w, a1w, selA)), kF16Pow2_15x2),
+                                hmul2(e4m3_b13_f16x2(__byte_perm(a0w, a1w, selB)), kF16Pow2_15x2),
+                                hmul2(e4m3_b13_f16x2(__byte_perm(b0w, b1w, selA)), kF16Pow2_15x2),
+                                hmul2(e4m3_b13_f16x2(__byte_perm(b0w, b1w, selB)), kF16Pow2_15x2)};
+        // Each word: key 2t's codes of dims 4 g4 + 0..3 (bits 0..15), key 2t+1's (bits 16..31): nibble
+        // pair (i, i+4) is the key pair of dim 4 g4 + i, as f16x2 * 2^-14; times the scales: * 2^-7.
+#define PKV_FP4_V_MTILE(I)                                                                                        \
+  {                                                                                                               \
+    const uint32_t a[4] = {hmul2(e2m1_pair_f16x2<I>(x[0]), sc[0]), hmul2(e2m1_pair_f16x2<I>(x[1]), sc[1]),       \
+                           hmul2(e2m1_pair_f16x2<I>(x[2]), sc[2]), hmul2(e2m1_pair_f16x2<I>(x[3]), sc[3])};      \
+    _Pragma("unroll") for (int nr = 0; nr < NR; ++nr) mma16816<false>(st.acc[nr][4 * p + I], a, pb[nr][0], pb[nr][1]); \
+  }
+        // m-tile 4p + i: rows g4 -> dim 64p + 4 g4 + i, rows g4 + 8 -> dim 64p + 32 + 4 g4 + i.
+        PKV_FP4_V_MTILE(0)
+        PKV_FP4_V_MTILE(1)
+        PKV_FP4_V_MTILE(2)
+        PKV_FP4_V_MTILE(3)
+#undef PKV_FP4_V_MTILE
+      }
+    } else if constexpr (KV == KV_E4M3) {
 #pragma unroll
       for (int c32 = 0; c32 < D / 32; ++c32) {
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4_trans(vb + off.v[c32], r0, r1, r2, r3);
-        const uint32_t p0 = __byte_perm(r0, 0, 0x3120), p1 = __byte_perm(r1, 0, 0x3120);
-        const uint32_t p2 = __byte_perm(r2, 0, 0x3120), p3 = __byte_perm(r3, 0, 0x3120);
-        const uint32_t ae[4] = {e4m3x2_to_f16x2(uint16_t(p0 & 0xffff)), e4m3x2_to_f16x2(uint16_t(p1 & 0xffff)),
-                                e4m3x2_to_f16x2(uint16_t(p2 & 0xffff)), e4m3x2_to_f16x2(uint16_t(p3 & 0xffff))};
-        const uint32_t ao[4] = {e4m3x2_to_f16x2(uint16_t(p0 >> 16)), e4m3x2_to_f16x2(uint16_t(p1 >> 16)),
-                                e4m3x2_to_f16x2(uint16_t(p2 >> 16)), e4m3x2_to_f16x2(uint16_t(p3 >> 16))};
+        // Each word holds (key 2t: dims d, d+1)(key 2t+1: dims d, d+1): bytes (0, 2) are the key
+        // pair of dim d, bytes (1, 3) of dim d+1.  Values times 2^-8 (undone in the output scale).
+        const uint32_t ae[4] = {e4m3_b02_f16x2(r0), e4m3_b02_f16x2(r1), e4m3_b02_f16x2(r2), e4m3_b02_f16x2(r3)};
+        const uint32_t ao[4] = {e4m3_b13_f16x2(r0), e4m3_b13_f16x2(r1), e4m3_b13_f16x2(r2), e4m3_b13_f16x2(r3)};
 #pragma unroll
         for (int nr = 0; nr < NR; ++nr) {
           mma16816<false>(st.acc[nr][2 * c32], ae, pb[nr][0], pb[nr][1]);
@@ -302,6 +408,17 @@ PKV_DEVICE void dec_tile(DecState<D, KV, QBF, NR>& st, const DecOffsets<D, KV, Q
   }
 }
 
+// NVFP4: zero V code rows [from, TK) (64 bytes each; the swizzle only permutes chunks within a
+// row) and their block scale rows (D/16 bytes each) of a staged tile.
+template <int TK, int SROW>
+PKV_DEVICE void zero_v_tail_fp4(uint32_t vbase, uint32_t vscale, int from, int lane) {
+  for (int x = lane; x < (TK - from) * 4; x += 32)
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(vbase + uint32_t(from * 64 + x * 16)), "r"(0) : "memory");
+  for (int x = lane; x < (TK - from) * SROW / 8; x += 32)
+    asm volatile("st.shared.v2.u32 [%0], {%1,%1};\n" ::"r"(vscale + uint32_t(from * SROW + x * 8)), "r"(0) : "memory");
+  __syncwarp();
+}
+
 // Zero V rows [from, TK) of a staged tile: those keys are past the item's end.
 template <int RB, int TK, int SLAB>
 PKV_DEVICE void zero_v_tail(uint32_t vbase, int from, int lane) {
@@ -315,7 +432,8 @@ PKV_DEVICE void zero_v_tail(uint32_t vbase, int from, int lane) {
 }
 
 template <int D, int KV, bool QBF>
-__global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant__ CUtensorMap tmap, const TmaArgs ta) {
+__global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                          const __grid_constant__ CUtensorMap smap, const TmaArgs ta) {
   using T = TmaCfg<D, KV, QBF>;
   const AttnArgs& a = ta.a;
   extern __shared__ uint8_t smem_raw[];
@@ -426,7 +544,32 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             const int stg = q % T::NST;
             if (s_abort || !mbar_wait(empty_bar(stg), ((q / T::NST) & 1) ^ 1)) { flag = 0; break; }
             const uint32_t sdst = stages + stg * T::STAGE_BYTES;
-            if (merged) {
+            if constexpr (T::FP4) {
+              // Codes through `tmap`, block scales through `smap` (16-byte rows of two slots).
+              int nb = 1;
+              if (!merged)
+                for (nb = 0; nb < T::TK / box_rows && key0 + nb * box_rows < it.k_end;) ++nb;
+              const int rows = merged ? T::TK : box_rows;
+              mbar_arrive_expect_tx(full_bar(stg), uint32_t(nb * rows) * 2 * (T::RB + T::SCALE_ROW));
+              for (int j = 0; j < nb; ++j) {
+                int phys = s_ids[rel + j];
+                if (phys < 0 || phys >= a.num_blocks) {
+                  report(a.status, PKV_DEV_BAD_BLOCK_ID);
+                  phys = int(a.num_blocks);  // out of the tensor: the loads fill zeros
+                }
+                if (merged) {
+                  tma_load_5d(sdst, &tmap, full_bar(stg), 0, key0 & bmask, it.kv_head, c3k, phys);
+                  tma_load_5d(sdst + T::KS_OFF, &smap, full_bar(stg), 0, (key0 & bmask) >> 1, it.kv_head, c3k, phys);
+                } else {
+                  const uint32_t r0 = uint32_t(j * box_rows);
+                  tma_load_5d(sdst + r0 * T::RB, &tmap, full_bar(stg), 0, 0, it.kv_head, c3k, phys);
+                  tma_load_5d(sdst + T::V_OFF + r0 * T::RB, &tmap, full_bar(stg), 0, 0, it.kv_head, c3k + 1, phys);
+                  tma_load_5d(sdst + T::KS_OFF + r0 * T::SCALE_ROW, &smap, full_bar(stg), 0, 0, it.kv_head, c3k, phys);
+                  tma_load_5d(sdst + T::VS_OFF + r0 * T::SCALE_ROW, &smap, full_bar(stg), 0, 0, it.kv_head, c3k + 1,
+                              phys);
+                }
+              }
+            } else if (merged) {
               int phys = s_ids[rel];
               if (phys < 0 || phys >= a.num_blocks) {
                 report(a.status, PKV_DEV_BAD_BLOCK_ID);
@@ -495,7 +638,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     const int ntiles = d.ntiles;
     float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
     float vscale = 1.f;
-    if constexpr (KV == KV_E4M3) {
+    if constexpr (KV == KV_E4M3 || KV == KV_NVFP4) {
       c *= __ldg(a.k_scale + a.layer * a.hkv + d.kv_head);
       vscale = __ldg(a.v_scale + a.layer * a.hkv + d.kv_head);
     }
@@ -504,6 +647,8 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
 
     if (R <= 16) {
       // ---- decode: warps take whole tiles round-robin, S^T / O^T formulation.
+      // fp8 and NVFP4 tiles dequantise to value * 2^-8 (E4M3) or * 2^-7 (E2M1 times its
+      // block scale); the scores and the output scale take the power of two back, exactly.
       auto run = [&](auto nr_tag) {
         constexpr int NR = decltype(nr_tag)::value;
         DecState<D, KV, QBF, NR> st;
@@ -533,13 +678,15 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
           const int qq = q + t;
           const int stg = qq % T::NST;
           if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1)) { ok = false; continue; }
-          const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::TK * 128;
+          const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::V_OFF;
           if (t == ntiles - 1 && last_valid < T::TK) {
-            zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);
+            if constexpr (T::FP4) zero_v_tail_fp4<T::TK, T::SCALE_ROW>(vb, kb + T::VS_OFF, last_valid, lane);
+            else zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);
             fence_proxy_async_smem();
           }
           const int key0 = d.k_begin + t * T::TK;
-          dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, key0, lane, c, key0 + T::TK > lim_min || key0 < lo_max);
+          dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, kb + T::KS_OFF, kb + T::VS_OFF, key0, lane, deq_undo<KV>(c),
+                                   key0 + T::TK > lim_min || key0 < lo_max);
           __syncwarp();
           if (lane == 0) mbar_arrive(empty_bar(stg), 4);
         }
@@ -574,8 +721,12 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             }
         }
       };
-      if (R <= 8) run(std::integral_constant<int, 1>{});
-      else run(std::integral_constant<int, 2>{});
+      if constexpr (T::FP4) {
+        run(std::integral_constant<int, 1>{});  // NVFP4 items carry at most 8 rows
+      } else {
+        if (R <= 8) run(std::integral_constant<int, 1>{});
+        else run(std::integral_constant<int, 2>{});
+      }
       mbar_arrive(merge_bar, 1);
       if (!mbar_wait(merge_bar, merge_phase)) ok = false;
       merge_phase ^= 1;
@@ -593,7 +744,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             o += red_o[(w * 16 + r) * D + dd] * f;
           }
         }
-        const float inv = lsum > 0.f ? vscale / lsum : 0.f;
+        const float inv = lsum > 0.f ? deq_undo<KV>(vscale) / lsum : 0.f;
         const int64_t orow = to_part ? int64_t(d.part_row) + r : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
         if (to_part) a.part_o[orow * D + dd] = o * inv;
         else store_q_dtype<QBF>(a.out, orow * D + dd, o * inv);
@@ -712,10 +863,49 @@ bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataTyp
   return r == CUDA_SUCCESS;
 }
 
+// An NVFP4 pool as two 5-D tensors over the same (block, layer, K|V, head) runs of
+// B * head_dim * 9/16 bytes: the E2M1 codes (rows of head_dim/2 bytes, 64-byte swizzle) and the
+// E4M3 block scales (which start B * head_dim/2 bytes into each run; viewed as 16-byte rows of
+// 16 / (head_dim/16) slots, no swizzle).  Boxes: box_rows slots x 1 head x box_kv x 1 block.
+bool make_fp4_maps(const AttnArgs& a, int head_dim, int box_rows, int box_kv, CUtensorMap* codes,
+                   CUtensorMap* scales) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t B = uint64_t(1) << a.log2_block;
+  const uint64_t rowb = uint64_t(head_dim) / 2, srow = uint64_t(head_dim) / 16;
+  const uint64_t run = B * (rowb + srow);
+  const uint64_t per = 16 / srow;  // slots per 16-byte scale row
+  if ((B * srow) % 16 || box_rows % per) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  cuuint64_t dims[5] = {rowb, B, cuuint64_t(a.hkv), cuuint64_t(2 * a.num_layers), cuuint64_t(a.num_blocks)};
+  cuuint64_t strides[4] = {rowb, run, run * a.hkv, run * a.hkv * 2 * a.num_layers};
+  cuuint32_t box[5] = {cuuint32_t(rowb), cuuint32_t(box_rows), 1, cuuint32_t(box_kv), 1};
+  CUresult r = fn(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(a.pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  void* sbase = static_cast<char*>(const_cast<void*>(a.pool)) + B * rowb;
+  cuuint64_t sdims[5] = {16, B / per, cuuint64_t(a.hkv), cuuint64_t(2 * a.num_layers), cuuint64_t(a.num_blocks)};
+  cuuint64_t sstrides[4] = {16, run, run * a.hkv, run * a.hkv * 2 * a.num_layers};
+  cuuint32_t sbox[5] = {16, cuuint32_t(box_rows / per), 1, cuuint32_t(box_kv), 1};
+  r = fn(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, sbase, sdims, sstrides, sbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int KV, bool QBF>
 cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
   using T = TmaCfg<D, KV, QBF>;
   CUtensorMap map;
+  if constexpr (T::FP4) {
+    const int B = 1 << a.log2_block;
+    const bool merged = B >= T::TK;
+    const int box_rows = merged ? T::TK : B;
+    CUtensorMap smap;
+    if (!make_fp4_maps(a, D, box_rows, merged ? 2 : 1, &map, &smap)) return cudaErrorInvalidValue;
+    attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, smap, TmaArgs{a, box_rows, merged ? 1 : 0});
+    return cudaGetLastError();
+  }
   const CUtensorMapDataType dt = KV == KV_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : KV == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -723,7 +913,7 @@ cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
   const bool merged = B >= T::TK;
   const int box_rows = merged ? T::TK : B;
   if (!make_pool_map(a, D, T::ELEM, dt, box_rows, merged ? 2 : 1, &map)) return cudaErrorInvalidValue;
-  attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, TmaArgs{a, box_rows, merged ? 1 : 0});
+  attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, map, TmaArgs{a, box_rows, merged ? 1 : 0});
   return cudaGetLastError();
 }
 
@@ -732,7 +922,8 @@ AttnKernel tma_kernel() {
   using T = TmaCfg<D, KV, QBF>;
   // 16-bit pools: only decode-sized tiles (larger ones are tcgen05 items); fp8: up to 64 rows.
   return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF>), T::THREADS, T::SMEM,
-                    &launch_tma<D, KV, QBF>, KV == KV_E4M3 ? PKV_TILE_ROWS : PKV_DECODE_ROWS};
+                    &launch_tma<D, KV, QBF>,
+                    KV == KV_E4M3 ? PKV_TILE_ROWS : (KV == KV_NVFP4 ? PKV_FP4_ROWS : PKV_DECODE_ROWS)};
 }
 
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {
@@ -752,6 +943,14 @@ bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size
       if (!d128) return false;  // 64-byte rows stay on the cp.async kernel
       if (q_dtype == PKV_BF16) *k = tma_kernel<128, KV_E4M3, true>();
       else if (q_dtype == PKV_F16) *k = tma_kernel<128, KV_E4M3, false>();
+      else return false;
+      return true;
+    case PKV_NVFP4:
+      // Decode tiles only (<= 8 rows); 16-byte block-scale rows need two slots per row and
+      // 128-byte aligned scale boxes, so blocks of at least 16 slots.
+      if (!d128 || block_size < 16) return false;
+      if (q_dtype == PKV_BF16) *k = tma_kernel<128, KV_NVFP4, true>();
+      else if (q_dtype == PKV_F16) *k = tma_kernel<128, KV_NVFP4, false>();
       else return false;
       return true;
   }

@@ -6,7 +6,9 @@
 // of head_dim values, so slots 0 .. n-1 of one (block, layer, K|V, head) are
 // one contiguous run of n * head_dim elements.  One warp per (copy, layer,
 // K|V, head) run moves it in 16-byte pieces (row bytes are multiples of 16 for
-// head_dim 64 / 128 and every pool dtype).
+// head_dim 64 / 128 and every pool dtype).  An NVFP4 run holds block_size rows of
+// codes and then block_size rows of block scales: the first n of each are copied
+// (the scale rows in 8-byte pieces).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -21,7 +23,8 @@ struct CopyArgs {
   int64_t num_blocks;
   int32_t runs_per_block;  // num_layers * 2 * Hkv
   int32_t log2_block;
-  int32_t row_bytes;       // head_dim * element size
+  int32_t row_bytes;       // head_dim * element size (NVFP4: head_dim / 2 bytes of codes)
+  int32_t scale_row_bytes; // NVFP4: head_dim / 16 bytes of block scales per row, else 0
   const int32_t* src;
   const int32_t* dst;
   const int32_t* n_tokens;
@@ -44,12 +47,20 @@ __global__ void __launch_bounds__(256) copy_block_prefix_kernel(CopyArgs a) {
       continue;
     }
     if (src == dst || n == 0) continue;
-    const int64_t run_bytes = int64_t(a.row_bytes) << a.log2_block;  // one (layer, K|V, head) of a block
+    const int64_t codes_bytes = int64_t(a.row_bytes) << a.log2_block;
+    const int64_t run_bytes = codes_bytes + (int64_t(a.scale_row_bytes) << a.log2_block);  // one (layer, K|V, head)
     const int64_t block_bytes = run_bytes * a.runs_per_block;
-    const uint4* s = reinterpret_cast<const uint4*>(a.pool + src * block_bytes + run * run_bytes);
-    uint4* d = reinterpret_cast<uint4*>(a.pool + dst * block_bytes + run * run_bytes);
+    const uint8_t* sbase = a.pool + src * block_bytes + run * run_bytes;
+    uint8_t* dbase = a.pool + dst * block_bytes + run * run_bytes;
+    const uint4* s = reinterpret_cast<const uint4*>(sbase);
+    uint4* d = reinterpret_cast<uint4*>(dbase);
     const int chunks = n * a.row_bytes / 16;
     for (int c = lane; c < chunks; c += 32) d[c] = __ldg(s + c);
+    if (a.scale_row_bytes) {
+      const uint2* ss = reinterpret_cast<const uint2*>(sbase + codes_bytes);
+      uint2* ds = reinterpret_cast<uint2*>(dbase + codes_bytes);
+      for (int c = lane; c < n * a.scale_row_bytes / 8; c += 32) ds[c] = __ldg(ss + c);
+    }
   }
 }
 
@@ -67,14 +78,18 @@ extern "C" pkv_status pkv_copy_block_prefix(const pkv_cache* cache, const int32_
   if (c.head_dim != 64 && c.head_dim != 128) return pkv_fail(PKV_ERR_UNSUPPORTED, "copy_block_prefix: head_dim %d", c.head_dim);
   if (c.num_kv_heads <= 0 || c.num_layers <= 0 || c.num_blocks <= 0)
     return pkv_fail(PKV_ERR_INVALID_ARG, "copy_block_prefix: bad cache shape");
-  if (c.kv_dtype < PKV_F32 || c.kv_dtype > PKV_FP8_E4M3) return pkv_fail(PKV_ERR_INVALID_ARG, "copy_block_prefix: kv_dtype");
+  if (c.kv_dtype < PKV_F32 || c.kv_dtype > PKV_NVFP4) return pkv_fail(PKV_ERR_INVALID_ARG, "copy_block_prefix: kv_dtype");
+  if (c.kv_dtype == PKV_NVFP4 && c.head_dim != 128)
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "copy_block_prefix: NVFP4 pools take head_dim 128");
   if (count == 0) return PKV_OK;
   if (!c.pool || !src_blocks || !dst_blocks || !n_tokens)
     return pkv_fail(PKV_ERR_INVALID_ARG, "copy_block_prefix: null pointer");
   if (reinterpret_cast<uintptr_t>(c.pool) & 15) return pkv_fail(PKV_ERR_INVALID_ARG, "copy_block_prefix: pool not 16-byte aligned");
+  const bool fp4 = c.kv_dtype == PKV_NVFP4;
   const int elem = c.kv_dtype == PKV_F32 ? 4 : (c.kv_dtype == PKV_FP8_E4M3 ? 1 : 2);
   CopyArgs a{static_cast<uint8_t*>(c.pool), c.num_blocks, c.num_layers * 2 * c.num_kv_heads, pkv_log2(c.block_size),
-             c.head_dim * elem, src_blocks, dst_blocks, n_tokens, count, dev_status};
+             fp4 ? c.head_dim / 2 : c.head_dim * elem, fp4 ? c.head_dim / 16 : 0, src_blocks, dst_blocks, n_tokens,
+             count, dev_status};
   const int64_t runs = int64_t(count) * a.runs_per_block;
   const int grid = int(std::min<int64_t>((runs + 7) / 8, 148 * 16));
   copy_block_prefix_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);

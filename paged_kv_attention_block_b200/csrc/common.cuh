@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -11,7 +12,7 @@
 
 namespace pkv {
 
-enum KvKind { KV_BF16 = 0, KV_F16 = 1, KV_E4M3 = 2 };
+enum KvKind { KV_BF16 = 0, KV_F16 = 1, KV_E4M3 = 2, KV_NVFP4 = 3 };
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -36,6 +37,30 @@ PKV_DEVICE uint32_t pack_f16x2(float lo, float hi) {
 PKV_DEVICE uint32_t e4m3x2_to_f16x2(uint16_t two) {
   __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
   return uint32_t(r.x) | (uint32_t(r.y) << 16);
+}
+
+// Integer dequantisation into f16 bit patterns, for the decode tiles where conversion
+// instructions would be the bottleneck.  Placing a code's exponent and mantissa bits into the
+// low bits of the f16 exponent and the top of its mantissa (sign to bit 15) yields the code's
+// value times a fixed power of two, subnormals included: 2^-8 for E4M3 (exponent bias 15
+// against 7), 2^-14 for E2M1 (bias 15 against 1).  NaN codes come out finite.
+//
+// E4M3 codes in bytes 0 and 2 of w -> f16x2 (byte 0, byte 2) * 2^-8; bytes 1, 3 are ignored.
+PKV_DEVICE uint32_t e4m3_b02_f16x2(uint32_t w) { return ((w << 7) & 0x3F803F80u) | ((w << 8) & 0x80008000u); }
+// E4M3 codes in bytes 1 and 3 of w -> f16x2 (byte 1, byte 3) * 2^-8; bytes 0, 2 are ignored.
+PKV_DEVICE uint32_t e4m3_b13_f16x2(uint32_t w) { return ((w >> 1) & 0x3F803F80u) | (w & 0x80008000u); }
+// E2M1 codes in nibbles I and I + 4 of w -> f16x2 (nibble I, nibble I+4) * 2^-14.
+template <int I>
+PKV_DEVICE uint32_t e2m1_pair_f16x2(uint32_t w) {
+  const uint32_t x = w << (12 - 4 * I);  // nibble I -> bits 12..15, nibble I+4 -> bits 28..31
+  return ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
+}
+constexpr uint32_t kF16Pow2_15x2 = 0x78007800u;  // f16x2 (2^15, 2^15)
+// f16x2 product, round to nearest (exact for the scaled E2M1 and E4M3 values multiplied here).
+PKV_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 // ---- shared-memory tile layout -------------------------------------------
@@ -70,6 +95,12 @@ PKV_DEVICE void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"
 PKV_DEVICE uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+PKV_DEVICE uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 

@@ -2,7 +2,10 @@
 // block tables (deep dive §2: decode writes the new token's KV; §8: a prefill
 // chunk appends its KV before the next chunk; concept explainer "技术原理":
 // page-table lookup on KV writes).  fp8 pools store E4M3(x / scale) with
-// round-to-nearest-even and saturation (deep dive §13, fp8 KV cache).
+// round-to-nearest-even and saturation (deep dive §13, fp8 KV cache); NVFP4
+// pools (deep dive §13, NVFP4 KV cache) store per 16-value group an E4M3 block
+// scale of max|x| / (6 g) and E2M1 codes of x / (scale g), g the float32 scale
+// of the (layer, KV head, K|V).
 //
 // One warp per (token, K|V): lane 0 resolves the destination slot once (the
 // token's sequence by binary search over cu_new staged in shared memory, its
@@ -165,6 +168,76 @@ __global__ void __launch_bounds__(256) kv_append_e4m3_kernel(AppendArgs a) {
   }
 }
 
+// float -> E2M1 code: nearest of 0, 0.5, 1, 1.5, 2, 3, 4, 6, ties to the even code (the
+// thresholds alternate strict and non-strict accordingly), saturating at 6; the sign bit is
+// the input's.
+PKV_DEVICE uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  const uint32_t c = uint32_t(a > 0.25f) + uint32_t(a >= 0.75f) + uint32_t(a > 1.25f) + uint32_t(a >= 1.75f) +
+                     uint32_t(a > 2.5f) + uint32_t(a >= 3.5f) + uint32_t(a > 5.0f);
+  return c | ((__float_as_uint(y) >> 31) << 3);
+}
+
+template <typename Tin>
+PKV_DEVICE void load4(const Tin* src, float* x);
+template <>
+PKV_DEVICE void load4<float>(const float* src, float* x) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+template <>
+PKV_DEVICE void load4<__nv_bfloat16>(const __nv_bfloat16* src, float* x) {
+  const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+  x[0] = bf16_bits_to_float(uint16_t(a.x & 0xffff)); x[1] = bf16_bits_to_float(uint16_t(a.x >> 16));
+  x[2] = bf16_bits_to_float(uint16_t(a.y & 0xffff)); x[3] = bf16_bits_to_float(uint16_t(a.y >> 16));
+}
+template <>
+PKV_DEVICE void load4<__half>(const __half* src, float* x) {
+  const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+  x[0] = f16_bits_to_float(uint16_t(a.x & 0xffff)); x[1] = f16_bits_to_float(uint16_t(a.x >> 16));
+  x[2] = f16_bits_to_float(uint16_t(a.y & 0xffff)); x[3] = f16_bits_to_float(uint16_t(a.y >> 16));
+}
+
+// NVFP4 (head_dim 128): one warp per (token, K|V); per KV head each lane quantises four
+// consecutive dims, the four lanes of a 16-value group share its max through shuffles, and
+// lane 4j writes the group's block scale.
+template <typename Tin>
+__global__ void __launch_bounds__(256) kv_append_nvfp4_kernel(AppendArgs a) {
+  __shared__ int32_t s_cu[kCuCache + 1];
+  const int32_t* cu = stage_cu(a, s_cu);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t run_bytes = int64_t(128 / 2 + 128 / 16) << a.log2_block;
+  for (int u = blockIdx.x * 8 + warp; u < 2 * a.total_new; u += gridDim.x * 8) {
+    const int t = u >> 1, which = u & 1;
+    const int64_t base = append_target(a, cu, t, which, lane);  // element offset of head 0's row
+    if (base < 0) continue;
+    const int64_t row = base >> 7;  // (run of head 0) * B + slot
+    const int64_t run0 = row >> a.log2_block;
+    const int slot = int(row & ((1 << a.log2_block) - 1));
+    const Tin* src = static_cast<const Tin*>(which ? a.v_new : a.k_new) + int64_t(t) * a.hkv * 128;
+    const float* gs = (which ? a.v_scale : a.k_scale) + a.layer * a.hkv;
+    for (int h = 0; h < a.hkv; ++h) {
+      float x[4];
+      load4<Tin>(src + h * 128 + lane * 4, x);
+      float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const float g = __ldg(gs + h);
+      const __nv_fp8_storage_t sc = __nv_cvt_float_to_fp8(__fdiv_rn(amax, __fmul_rn(6.0f, g)), __NV_SATFINITE, __NV_E4M3);
+      const float s = __half2float(__half(__nv_cvt_fp8_to_halfraw(sc, __NV_E4M3)));
+      uint32_t codes = 0;
+      if (s != 0.f) {
+        const float den = __fmul_rn(s, g);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) codes |= e2m1_code(__fdiv_rn(x[i], den)) << (4 * i);
+      }
+      uint8_t* run = static_cast<uint8_t*>(a.pool) + (run0 + h) * run_bytes;
+      *reinterpret_cast<uint16_t*>(run + slot * 64 + lane * 2) = uint16_t(codes);
+      if ((lane & 3) == 0) run[(int64_t(64) << a.log2_block) + slot * 8 + (lane >> 2)] = sc;
+    }
+  }
+}
+
 }  // namespace pkv
 
 extern "C" pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, const void* v_new, int32_t in_dtype,
@@ -180,11 +253,14 @@ extern "C" pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, c
   if (c.head_dim != 64 && c.head_dim != 128) return pkv_fail(PKV_ERR_UNSUPPORTED, "kv_append: head_dim %d", c.head_dim);
   if (c.num_kv_heads <= 0 || c.num_layers <= 0 || c.layer < 0 || c.layer >= c.num_layers || c.num_blocks <= 0)
     return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: bad cache shape");
-  if (c.kv_dtype < PKV_F32 || c.kv_dtype > PKV_FP8_E4M3) return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: kv_dtype");
-  if (c.kv_dtype == PKV_FP8_E4M3) {
+  if (c.kv_dtype < PKV_F32 || c.kv_dtype > PKV_NVFP4) return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: kv_dtype");
+  if (c.kv_dtype == PKV_NVFP4 && c.head_dim != 128)
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "kv_append: NVFP4 pools take head_dim 128");
+  if (c.kv_dtype == PKV_FP8_E4M3 || c.kv_dtype == PKV_NVFP4) {
     if (in_dtype != PKV_F32 && in_dtype != PKV_BF16 && in_dtype != PKV_F16)
-      return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: fp8 pool takes F32, BF16 or F16 values");
-    if (!c.k_scale || !c.v_scale) return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: fp8 pool needs k_scale and v_scale");
+      return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: fp8 and NVFP4 pools take F32, BF16 or F16 values");
+    if (!c.k_scale || !c.v_scale)
+      return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: fp8 and NVFP4 pools need k_scale and v_scale");
   } else if (in_dtype != c.kv_dtype) {
     return pkv_fail(PKV_ERR_INVALID_ARG, "kv_append: in_dtype %d must equal the pool dtype %d", in_dtype, c.kv_dtype);
   }
@@ -204,6 +280,11 @@ extern "C" pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, c
     case PKV_F32: kv_append_copy_kernel<4><<<grid, 256, 0, st>>>(a); break;
     case PKV_BF16:
     case PKV_F16: kv_append_copy_kernel<2><<<grid, 256, 0, st>>>(a); break;
+    case PKV_NVFP4:
+      if (in_dtype == PKV_F32) kv_append_nvfp4_kernel<float><<<grid, 256, 0, st>>>(a);
+      else if (in_dtype == PKV_BF16) kv_append_nvfp4_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+      else kv_append_nvfp4_kernel<__half><<<grid, 256, 0, st>>>(a);
+      break;
     default:
       if (in_dtype == PKV_F32) kv_append_e4m3_kernel<float><<<grid, 256, 0, st>>>(a);
       else if (in_dtype == PKV_BF16) kv_append_e4m3_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);

@@ -90,7 +90,12 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (g > PKV_TILE_ROWS) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: more than %d query heads per KV head", PKV_TILE_ROWS);
   if (D != 64 && D != 128) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: head_dim %d (64 or 128)", D);
   if (!pkv_is_pow2(B) || B < 2) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: block_size %d is not a power of two > 1", B);
-  if (req->kv_dtype < PKV_F32 || req->kv_dtype > PKV_FP8_E4M3) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: kv_dtype");
+  if (req->kv_dtype < PKV_F32 || req->kv_dtype > PKV_NVFP4) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: kv_dtype");
+  // NVFP4 pools run on the decode kernel alone: tiles of at most 8 rows, head_dim 128, blocks of 16+ slots.
+  const bool fp4 = req->kv_dtype == PKV_NVFP4;
+  if (fp4 && (D != 128 || B < 16 || g > PKV_FP4_ROWS))
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: NVFP4 pools take head_dim 128, block_size >= 16 and at most %d "
+                    "query heads per KV head", PKV_FP4_ROWS);
   if (S > 0 && (!req->cu_q_lens || !req->seq_lens)) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: null length arrays");
   if (S > 0 && req->max_blocks <= 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: max_blocks");
   const int window = req->window;
@@ -117,7 +122,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     tc_ctas = tc ? pkv_tc_resident_ctas(req->kv_dtype, D, B) : num_ctas;
     if (tc_ctas <= 0) return pkv_fail(PKV_ERR_CUDA, "attention_plan: occupancy query of the tcgen05 kernel failed");
   }
-  const int rows_cap = tc ? PKV_TILE_ROWS_TC : PKV_TILE_ROWS;
+  const int rows_cap = tc ? PKV_TILE_ROWS_TC : (fp4 ? PKV_FP4_ROWS : PKV_TILE_ROWS);
   const int QT = std::max(1, rows_cap / g);  // query tokens per tile
   auto is_tc = [&](int rows) { return tc && rows > PKV_DECODE_ROWS; };
   const bool causal = req->causal != 0;

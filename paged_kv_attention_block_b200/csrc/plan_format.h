@@ -18,6 +18,7 @@
 // PKV_TILE_ROWS_TC rows (one tensor-memory lane per row), keys in tiles of
 // PKV_TC_TILE_KEYS; a split key range starts on a multiple of that.
 #define PKV_DECODE_ROWS 16
+#define PKV_FP4_ROWS 8     /* rows per tile on NVFP4 pools (one register tile of query rows) */
 #define PKV_TILE_ROWS_TC 128
 #define PKV_TC_TILE_KEYS 128
 

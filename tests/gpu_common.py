@@ -9,7 +9,9 @@ from paged_kv_attention_block_b200 import workloads as W
 
 # Tolerances on the attention output (relative to the output magnitude for
 # 16-bit and fp8 pools, absolute for float32 pools).
-TOL = {"f32": 1e-5, "bf16": 2e-2, "f16": 2e-2, "e4m3": 6e-2}
+# NVFP4 values are exact in f16 (an E2M1 value times an E4M3 scale), so after the shared stored
+# codes its arithmetic is the fp8 path's: f16 operands rounded once (q, P), float32 sums.
+TOL = {"f32": 1e-5, "bf16": 2e-2, "f16": 2e-2, "e4m3": 6e-2, "nvfp4": 2e-2}
 
 
 def oracle_pool(w: W.Workload, seqs=None) -> O.OraclePool:
@@ -20,6 +22,11 @@ def oracle_pool(w: W.Workload, seqs=None) -> O.OraclePool:
         rows = w.block_tables if seqs is None else w.block_tables[list(seqs)]
         O.kv_append(pool, w.layer, k, v, w.kv_in_dtype, cu, sp, rows)
     return pool
+
+
+def oracle_pool_bytes(pool: O.OraclePool) -> np.ndarray:
+    """The oracle pool as the device holds it (NVFP4: the packed byte image)."""
+    return O.nvfp4_pool_bytes(pool) if pool.dtype == "nvfp4" else pool.bits
 
 
 def oracle_out(w: W.Workload, pool: O.OraclePool, seqs=None):

@@ -67,6 +67,16 @@ def test_kv_append_dtype_rules(api):
     c8 = _cache(kv_dtype=api.PKV_FP8_E4M3)
     assert api._lib.pkv_kv_append(C.byref(c8), 0x1000, 0x1000, api.PKV_F32, 0x1000, 0x1000, 0x1000, 4, 1, 1, None,
                                   None) == 1  # no scales
+    # NVFP4: head_dim 128 only, scales required, float inputs only.
+    c4 = _cache(kv_dtype=api.PKV_NVFP4, head_dim=64, k_scale=0x1000, v_scale=0x1000)
+    assert api._lib.pkv_kv_append(C.byref(c4), 0x1000, 0x1000, api.PKV_F32, 0x1000, 0x1000, 0x1000, 4, 1, 1, None,
+                                  None) == 2
+    c4 = _cache(kv_dtype=api.PKV_NVFP4, head_dim=128)
+    assert api._lib.pkv_kv_append(C.byref(c4), 0x1000, 0x1000, api.PKV_F32, 0x1000, 0x1000, 0x1000, 4, 1, 1, None,
+                                  None) == 1  # no scales
+    c4 = _cache(kv_dtype=api.PKV_NVFP4, head_dim=128, k_scale=0x1000, v_scale=0x1000)
+    assert api._lib.pkv_kv_append(C.byref(c4), 0x1000, 0x1000, api.PKV_NVFP4, 0x1000, 0x1000, 0x1000, 4, 1, 1, None,
+                                  None) == 1  # codes are not an input dtype
     # Nothing to do is fine and touches no device.
     assert api._lib.pkv_kv_append(C.byref(c), 0, 0, api.PKV_BF16, 0, 0, 0, 4, 0, 0, None, None) == 0
 
@@ -160,6 +170,24 @@ def test_plan_window_ranges(api, window, split):
         base = _plan(api, w, kv_split=split)
         keys = lambda pl: int((pl["items"]["k_end"] - pl["items"]["k_begin"]).sum())  # noqa: E731
         assert keys(d) < keys(PD.decode(base.buffer))
+
+
+def test_plan_nvfp4_rules(api):
+    """NVFP4 pools: decode-kernel tiles of at most 8 rows, head_dim 128, blocks of 16+ slots,
+    at most 8 query heads per KV head."""
+    w = W.build("nv", seed=3, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32, num_kv_heads=8,
+                head_dim=128, block_size=16, seq_lens=[300, 40, 9], q_lens=[37, 2, 1])
+    d = PD.decode(_plan(api, w).buffer)
+    g = w.num_q_heads // w.num_kv_heads
+    assert d["header"]["n_tc_items"] == 0 and (d["items"]["n_q"] * g <= 8).all()
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
+                      w.block_size)
+    for kw in (dict(head_dim=64), dict(block_size=8), dict(num_q_heads=128)):
+        args = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16, kv_dtype="nvfp4", num_ctas=10,
+                    pin=False)
+        args.update(kw)
+        with pytest.raises(api.PkvError):
+            api.plan_attention(np.array([0, 1], np.int32), np.array([5], np.int32), **args)
 
 
 def test_plan_window_rejects(api):

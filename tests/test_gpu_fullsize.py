@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import assert_close, gpu_out_f64, oracle_out, oracle_pool
+from gpu_common import assert_close, gpu_out_f64, oracle_out, oracle_pool, oracle_pool_bytes
 from paged_kv_attention_block_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -19,6 +19,7 @@ SAMPLES = {
     "mixed_bf16": [0, 3, 4, 123],
     "longctx_fp8": [5],
     "prefix_reuse_bf16": [0, 128, 255],
+    "llama3_8b_decode_nvfp4": [0, 17, 63],
 }
 
 
@@ -48,7 +49,7 @@ def test_fullsize_sampled(name):
         ids = torch.from_numpy(w.block_tables[s, :nb].astype(np.int64)).cuda()
         g = got.index_select(0, ids)
         g = (g.view(torch.int16) if g.dtype in (torch.bfloat16, torch.float16) else g).cpu().numpy()
-        want = pool.bits[w.block_tables[s, :nb]]
+        want = oracle_pool_bytes(pool)[w.block_tables[s, :nb]]
         if w.kv_dtype == "f32":
             assert (g.view(np.uint32) == want.view(np.uint32)).all()
         else:

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle.pkv_oracle as O
-from gpu_common import TOL, assert_close, gpu_out_f64, oracle_out, oracle_pool
+from gpu_common import TOL, assert_close, gpu_out_f64, oracle_out, oracle_pool, oracle_pool_bytes
 from paged_kv_attention_block_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +44,7 @@ def run_case(pkv, w, check_pool=True, check_lse=True, **plan_opts):
         if w.kv_dtype == "f32":
             same = (got.view(np.uint32) == pool.bits.view(np.uint32))
         else:
-            same = got == pool.bits
+            same = got == oracle_pool_bytes(pool)
         assert same.all(), f"kv_append: {int((~same).sum())} pool elements differ"
     ref, ref_lse = oracle_out(w, pool)
     err = assert_close(gpu_out_f64(out), ref, w.kv_dtype)
@@ -212,13 +212,13 @@ def test_limited_attention_window(pkv, window, kind):
     run_case(pkv, w, check_pool=False)
 
 
-@pytest.mark.parametrize("kv", ["bf16", "e4m3", "f32"])
+@pytest.mark.parametrize("kv", ["bf16", "e4m3", "f32", "nvfp4"])
 def test_copy_block_prefix_bit_exact(pkv, kv):
     # Partial reuse: copies of whole and partial block prefixes into free blocks, the whole pool
     # compared byte for byte with the oracle's copy; bad ids and counts are reported, not written.
     api, runner = pkv
-    if kv == "e4m3":
-        w = W.build("copy", seed=18, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=8,
+    if kv in ("e4m3", "nvfp4"):
+        w = W.build("copy", seed=18, kv_dtype=kv, q_dtype="bf16", kv_in_dtype="f32", num_q_heads=8,
                     num_kv_heads=2, head_dim=128, block_size=16, seq_lens=[100, 37, 64], q_lens=[1, 1, 1],
                     num_layers=2, layer=1, pool_factor=3.0)
     else:
@@ -241,7 +241,7 @@ def test_copy_block_prefix_bit_exact(pkv, kv):
     if kv == "f32":
         assert (got.view(np.uint32) == pool.bits.view(np.uint32)).all()
     else:
-        assert (got == pool.bits).all()
+        assert (got == oracle_pool_bytes(pool)).all()
     before = dw.pool_bytes().copy()
     api.copy_block_prefix(dw.cache, dev([src[0], w.num_blocks]), dev([free[8], free[9]]), dev([17, 4]),
                           status=dw.status)
@@ -353,3 +353,46 @@ def test_graph_step_matches_oracle(pkv):
         got = gs.wait(s).float().numpy().astype(np.float64)
         assert_close(got, ref, w.kv_dtype, what=f"slot {s}")
     assert gs.h2d_bytes >= sum(t.numel() * t.element_size() for t in names.values())
+
+
+
+# ---- NVFP4 KV cache (E2M1 codes, E4M3 block scales, float32 scale per (layer, head, K|V)) ----
+
+@pytest.mark.parametrize("B", [16, 32, 64, 128])
+@pytest.mark.parametrize("hq", [32, 64])
+def test_nvfp4_decode(pkv, B, hq):
+    """kv_append byte for byte (codes and block scales) and decode attention, Hkv 8, d 128,
+    ragged lengths over several 64-key tiles, blocks smaller and larger than a tile."""
+    w = W.build("nv_dec", seed=30 + B, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=hq,
+                num_kv_heads=8, head_dim=128, block_size=B, seq_lens=[1, 63, 64, 65, 300, 777, 2049],
+                q_lens=[1] * 7, data_scale=0.5)
+    run_case(pkv, w)
+
+
+@pytest.mark.parametrize("split", [-1, 64, 0])
+def test_nvfp4_llama3_8b_decode_shape(pkv, split):
+    run_case(pkv, W.llama3_8b_decode_nvfp4(batch=9, lo=1, hi=3000), kv_split=split)
+
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "f16"])
+def test_nvfp4_from_16bit_values(pkv, in_dtype):
+    w = W.build("nv_in", seed=33, kv_dtype="nvfp4", q_dtype="bf16" if in_dtype == "bf16" else "f16",
+                kv_in_dtype=in_dtype, num_q_heads=16, num_kv_heads=4, head_dim=128, block_size=64,
+                seq_lens=[130, 5, 700], q_lens=[1, 1, 1])
+    run_case(pkv, w)
+
+
+def test_nvfp4_chunks_and_multi_token(pkv):
+    """Prefill chunks and multi-token decode rows over an NVFP4 cache (8-row tiles, causal)."""
+    w = W.build("nv_mix", seed=34, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                num_kv_heads=8, head_dim=128, block_size=16, seq_lens=[300, 90, 41, 17], q_lens=[45, 4, 2, 1])
+    run_case(pkv, w)
+
+
+@pytest.mark.parametrize("window", [1, 50, 200])
+def test_nvfp4_limited_window(pkv, window):
+    w = W.build("nv_win", seed=35, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                num_kv_heads=8, head_dim=128, block_size=32, seq_lens=[700, 64, 250], q_lens=[3, 1, 1],
+                window=window)
+    run_case(pkv, w)
+
