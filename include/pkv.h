@@ -189,8 +189,8 @@ typedef struct pkv_plan_request {
   int32_t num_seqs;
   int32_t num_q_heads;          /* Hq, a multiple of num_kv_heads */
   int32_t num_kv_heads;         /* Hkv */
-  int32_t head_dim;             /* 64 or 128 */
-  int32_t block_size;           /* power of two >= 2 */
+  int32_t head_dim;             /* 64 or 128 (128 for NVFP4 pools) */
+  int32_t block_size;           /* power of two >= 2 (>= 16 for NVFP4 pools) */
   int32_t kv_dtype;             /* pkv_dtype of the pool */
   int32_t causal;               /* 0 or 1 */
   int32_t num_ctas;             /* CTAs the launch uses (capped at what fits resident); 0 = all that
@@ -257,11 +257,13 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  * pkv_split_kv_reduce performs), in that order on `stream`.
  *
  * q: device [total_q][num_q_heads][head_dim], q_dtype F32 (F32 pools only),
- *   BF16 (BF16 or FP8 pools) or F16 (F16 or FP8 pools).  total_q = cu_q_lens[num_seqs].
+ *   BF16 (BF16, FP8 or NVFP4 pools) or F16 (F16, FP8 or NVFP4 pools).
+ *   total_q = cu_q_lens[num_seqs].  NVFP4 pools: head_dim 128, block_size >= 16,
+ *   at most 8 query heads per KV head (else UNSUPPORTED, from the planner too).
  * cu_q_lens, seq_lens: device int32 copies of the arrays the plan was made from.
  * block_tables: device int32 [num_seqs][max_blocks].
  * softmax_scale: scale on q.k (typically 1/sqrt(head_dim)), positive and finite;
- *   causal as planned.  fp8 scales must be positive.
+ *   causal as planned.  fp8 and NVFP4 scales must be positive.
  * plan: host buffer from pkv_attention_plan for these shapes.  It is copied to
  *   the workspace with cudaMemcpyAsync; use page-locked memory for an
  *   asynchronous copy and keep it unchanged until the copy has run.
