@@ -19,6 +19,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -153,14 +154,21 @@ class ClockSampler:
 TRAFFIC_SOURCES = ("attn_tma.cu", "attn_tile.cuh", "attn_args.h", "common.cuh", "internal.h", "plan_format.h")
 
 
+def _code_only(src: str) -> str:
+    """C/C++ source without comments or blank lines: a comment edit does not change the kernel."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_attention_block_b200", "csrc")
     for name in TRAFFIC_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
-    with open(os.path.join(ROOT, "include", "pkv.h"), "rb") as f:
-        h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
+    with open(os.path.join(ROOT, "include", "pkv.h"), encoding="utf-8") as f:
+        h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
