@@ -485,9 +485,10 @@ def run_e2e(args, w, dw, plan_opts, dev, stream, api):
     """The step end to end through the public API as a serving loop runs it (api.GraphStep):
     every step plans on the host, copies its packed inputs (q, new K/V, lengths, positions,
     tables) and its plan from page-locked host memory, appends, runs attention and copies the
-    output back to page-locked host memory, as one graph replay per step; two buffer slots let
-    the host plan step i+1 while the GPU runs step i.  Time = events around n back-to-back steps
-    (every copy inside), divided by n."""
+    output back to page-locked host memory: three graph replays per step (copy in, kernels, copy
+    out) on three streams, two buffer slots, so copies overlap the neighbouring steps' kernels and
+    the host plans step i+1 while the GPU runs step i.  Time = events from before the first input
+    copy to after the last output copy of n back-to-back steps, divided by n."""
     import torch
 
     names = {"q": dw.q, "k_new": dw.k_new, "v_new": dw.v_new, "cu_q": dw.cu_q, "seq_lens": dw.seq_lens,
@@ -501,12 +502,13 @@ def run_e2e(args, w, dw, plan_opts, dev, stream, api):
     for _ in range(4):
         gs.wait(gs.run())
     n = max(2, min(args.steps, 500))
+    torch.cuda.synchronize(dev)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(gs.stream)
+    s.record(gs.copy_in_stream)  # before the first input copy
     slot = None
     for _ in range(n):
         slot = gs.run()
-    e.record(gs.stream)
+    e.record(gs.copy_out_stream)  # after the last output copy
     out = gs.wait(slot)
     e.synchronize()
     assert torch.isfinite(out.float()).all(), "non-finite output in the end-to-end loop"

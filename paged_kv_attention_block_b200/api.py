@@ -313,19 +313,21 @@ def split_kv_reduce(partial_o: torch.Tensor, partial_lse: torch.Tensor, out_dtyp
 
 
 class GraphStep:
-    """One serving step from page-locked host inputs, replayed as a CUDA graph per buffer slot.
+    """One serving step from page-locked host inputs, as three CUDA graphs per buffer slot.
 
     A step is: one host-to-device copy of the packed inputs (q, new K/V rows, cu_q_lens,
-    seq_lens, start_pos, block tables) and of the step's plan, ``kv_append``,
-    ``paged_attention``, and one device-to-host copy of the output.  Every call of
-    :meth:`run` re-plans on the host (into the slot's page-locked plan buffer, which the
-    graph uploads) and replays the slot's graph; with two slots the host plans step i+1
-    while the GPU runs step i.  The graph is captured again whenever a new plan differs
+    seq_lens, start_pos, block tables); ``kv_append`` and ``paged_attention`` (which uploads
+    the step's plan from its page-locked buffer); one device-to-host copy of the output.
+    The copies run on their own streams, so with two slots the inputs of step i+1 travel
+    while step i computes and the output of step i travels while step i+1 computes; the
+    host plans step i+1 meanwhile.  Every call of :meth:`run` re-plans on the host into the
+    slot's plan buffer; the slot's graphs are captured again whenever a new plan differs
     from the captured one in a launch-shaping field (item and merge counts, CTA counts).
 
-    Callers write each step's inputs into :attr:`host` (named page-locked views of one
-    buffer) before :meth:`run`, and read the output from the tensor that :meth:`wait`
-    returns.
+    Callers write a step's inputs into :attr:`host` ``[slot]`` (named page-locked views of
+    one buffer) before :meth:`run` takes that slot and after :meth:`wait` has returned for
+    the slot's previous step, and read the output from the tensor that :meth:`wait` returns
+    before the slot's next step is launched.
     """
 
     _FIELDS = ("q", "k_new", "v_new", "cu_q", "seq_lens", "start_pos", "block_tables")
@@ -335,8 +337,10 @@ class GraphStep:
     def __init__(self, cache: Cache, like: dict, plan_kwargs: dict, softmax_scale: float, causal: bool = True,
                  slots: int = 2, stream=None):
         self.cache, self.plan_kwargs, self.scale, self.causal = cache, dict(plan_kwargs), float(softmax_scale), causal
-        self.stream = stream if stream is not None else torch.cuda.Stream()
+        self.stream = stream if stream is not None else torch.cuda.Stream()  # kernels
         dev = self.stream.device
+        self.copy_in_stream = torch.cuda.Stream(dev)
+        self.copy_out_stream = torch.cuda.Stream(dev)
         # One page-locked buffer and one device buffer per slot, each field 256-byte aligned.
         offs, total = {}, 0
         for name in self._FIELDS:
@@ -358,9 +362,11 @@ class GraphStep:
         self._out_h = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(slots)]
         self.d2h_bytes = q.numel() * q.element_size()
         self._plans = [None] * slots
-        self._graphs = [None] * slots
+        self._graphs = [None] * slots  # (copy in, compute, copy out) per slot
         self._shape = [None] * slots
-        self._done = [torch.cuda.Event() for _ in range(slots)]
+        self._ready = [torch.cuda.Event() for _ in range(slots)]     # inputs of the slot on the device
+        self._consumed = [torch.cuda.Event() for _ in range(slots)]  # kernels done with inputs, plan, output buffer
+        self._fetched = [torch.cuda.Event() for _ in range(slots)]   # output of the slot on the host
         self._pending = [False] * slots
         self._ws = None
         self._slot = 0
@@ -375,21 +381,23 @@ class GraphStep:
         if self._ws is None or self._ws.numel() < plan.workspace_bytes:
             self._ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=self.stream.device)
         d = self._dev[b]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=self.stream):
+        g_in, g_run, g_out = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_in, stream=self.copy_in_stream):
             self._dbuf[b].copy_(self._hbuf[b], non_blocking=True)
+        with torch.cuda.graph(g_run, stream=self.stream):
             kv_append(self.cache, d["k_new"], d["v_new"], d["cu_q"], d["start_pos"], d["block_tables"])
             paged_attention(self.cache, d["q"], d["cu_q"], d["seq_lens"], d["block_tables"], plan, self.scale,
                             self.causal, out=self._out_d[b], workspace=self._ws)
+        with torch.cuda.graph(g_out, stream=self.copy_out_stream):
             self._out_h[b].copy_(self._out_d[b], non_blocking=True)
-        self._graphs[b] = g
+        self._graphs[b] = (g_in, g_run, g_out)
 
     def run(self) -> int:
         """Plan and launch one step on the next slot; returns the slot (pass it to :meth:`wait`)."""
         b = self._slot
         self._slot = (b + 1) % len(self._graphs)
         if self._pending[b]:
-            self._done[b].synchronize()  # the slot's last replay has read its inputs and plan
+            self._consumed[b].synchronize()  # the slot's last kernels have read its inputs and plan
         plan = self._plan_into(b)
         self._plans[b] = plan
         shape = tuple(plan.info[k] for k in self._SHAPE_KEYS)
@@ -397,14 +405,25 @@ class GraphStep:
             torch.cuda.synchronize(self.stream.device)
             self._capture(b, plan)
             self._shape[b] = shape
+        g_in, g_run, g_out = self._graphs[b]
+        with torch.cuda.stream(self.copy_in_stream):
+            self.copy_in_stream.wait_event(self._consumed[b])  # device inputs of the slot free
+            g_in.replay()
+            self._ready[b].record(self.copy_in_stream)
         with torch.cuda.stream(self.stream):
-            self._graphs[b].replay()
-            self._done[b].record(self.stream)
+            self.stream.wait_event(self._ready[b])
+            self.stream.wait_event(self._fetched[b])  # the slot's previous output has left
+            g_run.replay()
+            self._consumed[b].record(self.stream)
+        with torch.cuda.stream(self.copy_out_stream):
+            self.copy_out_stream.wait_event(self._consumed[b])
+            g_out.replay()
+            self._fetched[b].record(self.copy_out_stream)
         self._pending[b] = True
         return b
 
     def wait(self, slot: int) -> torch.Tensor:
         """Block until the slot's step has finished; returns its page-locked host output."""
-        self._done[slot].synchronize()
+        self._fetched[slot].synchronize()
         self._pending[slot] = False
         return self._out_h[slot]
