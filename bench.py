@@ -161,6 +161,26 @@ def _code_only(src: str) -> str:
     return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
 
 
+def read_stream_gbs(buf, reps: int = 10):
+    """A plain read-only stream as the practical HBM ceiling: torch's sum over ``buf`` (larger
+    than L2), CUDA events around each pass, the median pass.  None if it cannot be taken."""
+    import torch
+
+    try:
+        times = []
+        for _ in range(reps + 2):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            buf.sum()
+            e.record()
+            e.synchronize()
+            times.append(s.elapsed_time(e))
+        ms = statistics.median(times[2:])
+        return buf.numel() * buf.element_size() / (ms * 1e-3) / 1e9
+    except Exception:  # noqa: BLE001 - a missing ceiling must not cost the benchmark line
+        return None
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_attention_block_b200", "csrc")
@@ -402,6 +422,8 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     achieved = b["kernels"] / (kern * 1e-3) / 1e9
     peak, peak_kind = peaks()
 
+    read_ceiling = read_stream_gbs(flush)
+
     # End to end through the public API from pinned host buffers.
     e2e = run_e2e(args, w, dw, plan_opts, dev, torch.cuda.current_stream(dev), api)
     e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
@@ -424,6 +446,9 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
             "decode_tok_s": decode_rows(w) * world / (ms * 1e-3),
             "hbm_frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
             "hbm_frac_of_measured": value / world / peak,
+            "read_stream_ceiling": None if read_ceiling is None else {
+                "value": read_ceiling, "unit": "GB/s", "kernels_frac": achieved / read_ceiling,
+                "how": "torch sum over a 512 MB float32 buffer, CUDA events, median of 10 passes"},
             "step_bytes": b["step"], "kv_bytes": b["kv"],
             "attention_ms": attn, "attention_kernels_ms": kern, "host_plan_us": host_plan_s / args.steps * 1e6,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
