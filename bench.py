@@ -23,6 +23,7 @@ import re
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -101,7 +102,9 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # The raw samples go to $PKV_BENCH_OUT (default: the system temp directory).
+        out = os.environ.get("PKV_BENCH_OUT") or tempfile.gettempdir()
+        self.path = os.path.join(out, f"pkv_clocks_rank{index}.csv")
 
     def __enter__(self):
         try:
