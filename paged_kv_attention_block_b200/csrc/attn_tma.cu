@@ -1,5 +1,6 @@
 // Paged attention, TMA-fed and warp-specialised (bf16 / f16 / fp8-e4m3 pools,
-// block size >= 8, 128- or 256-byte K/V rows).
+// block size >= 8, 128- or 256-byte K/V rows; NVFP4 pools, d 128, block size
+// >= 16).
 //
 // Same work list and results as attn_mma.cu (deep dive, gentlecold.top: §2
 // decode reads all history KV, §6 one launch for a packed mix of prefill and
@@ -26,6 +27,12 @@
 //   * Prefill tiles (> 16 rows; fp8 pools, since 16-bit pools send them to the
 //     tcgen05 kernel of attn_tc.cu): every warp reads every tile and owns 16
 //     rows (the row-split step of attn_tile.cuh).
+//   * fp8 and NVFP4 tiles widen to f16 in registers with integer operations
+//     (exact; values times a power of two taken back in the score and output
+//     scales).  NVFP4 tiles arrive as two TMA boxes, E2M1 codes (64-byte rows,
+//     64-byte swizzle) and E4M3 block scales, and each E2M1 value is multiplied
+//     by its block scale in f16 (exact) before the MMA.  deep dive §13 (NVFP4
+//     KV cache).
 //   * Keys past the item's end inside the last tile are masked; their V rows
 //     are zeroed in shared memory before the P V product (0 * NaN would leak).
 //   * Every wait on an mbarrier is bounded; on a timeout the CTA records
