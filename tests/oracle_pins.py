@@ -300,6 +300,32 @@ def pin_block_mapping_example():
     assert np.isnan(pool.bits[~touched]).all()
 
 
+def pin_partial_reuse_example():
+    """The deep dive's partial-reuse example: block [A, B, C, D], a new request [A, B, X, Y] matching two
+    tokens; the matched tokens are copied into a new block, the request appends X and Y after them, and the
+    existing block is left as it was (tests/golden/partial_reuse_example.json)."""
+    with open(os.path.join(GOLDEN, "partial_reuse_example.json")) as f:
+        g = json.load(f)
+    B, n = g["block_size"], g["matched_tokens"]
+    labels = sorted(set(g["existing_block"]) | set(g["new_request"]))
+    row = {lab: np.full((1, 8), 10.0 * (i + 1), np.float32) + np.arange(8, dtype=np.float32) for i, lab in enumerate(labels)}
+    kv = lambda toks, sign: np.stack([sign * row[t] for t in toks])  # noqa: E731  [T][Hkv=1][D=8]
+    pool = O.new_pool(6, 1, 1, B, 8, "f32")
+    old, new = 1, 4  # physical blocks
+    O.kv_append(pool, 0, kv(g["existing_block"], 1), kv(g["existing_block"], -1), "f32", np.array([0, B]),
+                np.array([0]), np.array([[old]]))
+    O.copy_block_prefix(pool, [old], [new], [n])
+    tail = g["new_request"][n:]
+    O.kv_append(pool, 0, kv(tail, 1), kv(tail, -1), "f32", np.array([0, len(tail)]), np.array([n]),
+                np.array([[new]]))
+    for blk, want in ((old, g["expect_existing"]), (new, g["expect_new"])):
+        for which, sign in ((0, 1), (1, -1)):
+            got = O.gather_rows(pool, 0, np.array([blk]), 0, which, B)
+            assert np.array_equal(got, kv(want, sign)[:, 0, :].astype(np.float64)), (blk, which)
+    others = [b for b in range(6) if b not in (old, new)]
+    assert np.isnan(pool.bits[others]).all()
+
+
 def pin_append_roundtrip():
     for w in small_workloads():
         pool = oracle_pool_for(w)
@@ -633,7 +659,8 @@ def pin_block_copy():
 
 
 ALL_PINS = [
-    pin_e4m3_decode_table, pin_e4m3_encode, pin_bf16_decode, pin_block_mapping_example, pin_append_roundtrip,
+    pin_e4m3_decode_table, pin_e4m3_encode, pin_bf16_decode, pin_block_mapping_example, pin_partial_reuse_example,
+    pin_append_roundtrip,
     pin_dense_equivalence, pin_noncausal_dense, pin_brute_force, pin_lse_logsumexp, pin_permutation_invariance,
     pin_softmax_rows, pin_closed_forms, pin_split_reduce, pin_prefix_sharing, pin_window_dense, pin_window_limits,
     pin_window_brute_force, pin_block_copy, pin_e2m1_table, pin_e2m1_encode, pin_nvfp4_worked_group,

@@ -1,0 +1,48 @@
+"""The benchmark's byte and flop accounting against first principles (CPU only).
+
+KV bytes follow the static source audit's sizing (kkqc.cn, §四 "KV Cache"): layers x tokens x KV
+width x bytes per element, counted once per distinct physical block (deep dive §10: shared prefix
+blocks are stored once).  Prefill flops count 4 d Hq per causal-valid (query, key) pair, here by
+enumerating the pairs.
+"""
+import numpy as np
+
+import bench
+from paged_kv_attention_block_b200 import workloads as W
+
+
+def _row_bytes(w):
+    # K or V of one token, all KV heads: d values per head (NVFP4: d/2 code bytes + d/16 scale bytes).
+    per_head = {"f32": 4 * w.head_dim, "bf16": 2 * w.head_dim, "f16": 2 * w.head_dim, "e4m3": w.head_dim,
+                "nvfp4": w.head_dim // 2 + w.head_dim // 16}[w.kv_dtype]
+    return w.num_kv_heads * per_head
+
+
+def test_kv_bytes_private_sequences():
+    for w in (W.llama3_8b_decode_bf16(batch=7, lo=1, hi=900), W.longctx_fp8(batch=2, seq_len=300),
+              W.llama3_8b_decode_nvfp4(batch=5, lo=3, hi=500), W.tiny_fp32()):
+        want = int(w.seq_lens.sum()) * 2 * _row_bytes(w)  # one layer, K and V
+        assert bench.algorithmic_bytes(w)["kv"] == want, w.name
+
+
+def test_kv_bytes_shared_prefix_counted_once():
+    w = W.prefix_reuse_bf16(n_req=9, prefix=256, suf_lo=1, suf_hi=70)
+    unique_tokens = 256 + int((w.seq_lens - 256).sum())
+    assert bench.algorithmic_bytes(w)["kv"] == unique_tokens * 2 * _row_bytes(w)
+
+
+def test_append_bytes():
+    w = W.llama3_8b_decode_nvfp4(batch=4, lo=3, hi=100)
+    rows = int(w.q_lens.sum()) * w.num_kv_heads * 2
+    assert bench.algorithmic_bytes(w)["append"] == rows * (w.head_dim * 4 + w.head_dim // 2 + w.head_dim // 16)
+
+
+def test_prefill_flops_by_enumeration():
+    w = W.build("pf", seed=3, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+                seq_lens=[40, 9, 30, 5], q_lens=[17, 1, 30, 2])
+    pairs = 0
+    for L, ql in zip(w.seq_lens, w.q_lens):
+        if ql > 1:  # prefill chunks only
+            for j in range(ql):
+                pairs += sum(1 for t in range(L) if t <= L - ql + j)
+    assert bench.prefill_flops(w) == 4.0 * w.head_dim * w.num_q_heads * pairs
