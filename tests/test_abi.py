@@ -6,6 +6,7 @@ import subprocess
 
 import numpy as np
 import pytest
+import torch
 
 from paged_kv_attention_block_b200 import build as B
 from paged_kv_attention_block_b200 import workloads as W
@@ -244,3 +245,19 @@ def test_plan_orders_heaviest_first(api, name, make, opts):
                 if cost[i] == cost[i - 1]:
                     a, b = lst[i - 1], lst[i]
                     assert (a["q_begin"], a["kv_head"], a["k_begin"]) < (b["q_begin"], b["kv_head"], b["k_begin"])
+
+
+def test_plan_is_deterministic_and_reuses_buffers(api):
+    """The same request gives the same bytes; a large enough buffer is planned into in place, a
+    too small one is replaced by a fresh buffer holding the same plan."""
+    w = W.mixed_bf16(n_decode=12, n_prefill=2, chunk=100, block_size=16, cached_lo_blocks=1, cached_hi_blocks=9)
+    a = _plan(api, w)
+    b = _plan(api, w)
+    n = a.info["plan_bytes"]
+    assert torch.equal(a.buffer[:n], b.buffer[:n])
+    big = torch.zeros(n + 4096, dtype=torch.uint8)
+    c = _plan(api, w, buffer=big)
+    assert c.buffer is big and torch.equal(big[:n], a.buffer[:n]) and c.info == a.info
+    small = torch.zeros(64, dtype=torch.uint8)
+    d = _plan(api, w, buffer=small)
+    assert d.buffer is not small and torch.equal(d.buffer[:n], a.buffer[:n]) and not small.any()
