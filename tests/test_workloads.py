@@ -46,3 +46,16 @@ def test_fp8_scales_are_amax_over_448():
     for h in range(w.num_kv_heads):
         amax = max(np.abs(w.kv_values(s)[0][:, h]).max() for s in range(2))
         assert w.k_scale[0, h] == np.float32(amax / 448.0)
+
+
+def test_nvfp4_global_scales_and_shared_values():
+    """NVFP4 global scales are amax / (6 * 448) per (layer, KV head), K and V apart; the NVFP4 decode
+    batch draws the same lengths, tables and values as the bf16 one."""
+    w = W.llama3_8b_decode_nvfp4(batch=3, lo=20, hi=90)
+    for h in range(w.num_kv_heads):
+        for which, sc in ((0, w.k_scale), (1, w.v_scale)):
+            amax = max(np.abs(w.kv_values(s)[which][:, h]).max() for s in range(3))
+            assert sc[0, h] == np.float32(amax / (6.0 * 448.0))
+    b = W.llama3_8b_decode_bf16(batch=3, lo=20, hi=90)
+    assert np.array_equal(w.seq_lens, b.seq_lens) and np.array_equal(w.block_tables, b.block_tables)
+    assert w.kv_in_dtype == "f32" and w.q_dtype == "bf16" and w.block_size == 64
