@@ -20,6 +20,8 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <functional>
+#include <queue>
 #include <vector>
 
 #include "internal.h"
@@ -213,6 +215,72 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
 
   // 3. Key-range split and merges.
   const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 2.0)};
+  // Longest key range of one item of a unit's list; the automatic length (about two items per
+  // CTA) is scaled by `mult`.
+  auto max_keys_for = [&](const Unit& u, bool t, double mult) -> int32_t {
+    const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
+    int64_t max_keys;
+    if (req->kv_split < 0) max_keys = INT32_MAX;
+    else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
+    else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
+                                      round_up(int64_t(std::ceil(target[t] * mult / u.weight)), tile_keys));
+    return int32_t(std::min<int64_t>(max_keys, INT32_MAX / 2));
+  };
+  // Tail check of the register-tile list.  The CTAs take items heaviest first from a counter, so
+  // when the item count only just passes a multiple of the CTA count (a batch of equal long
+  // ranges split into equal pieces), a few CTAs run one extra round while the rest idle.  Then
+  // longer pieces are tried, and the one with the shortest simulated schedule (the greedy
+  // assignment the counter produces, constant per-CTA speed) is kept if it is 2 % shorter.
+  double reg_mult = 1.0;
+  if (req->kv_split == 0) {
+    std::vector<double> costs;
+    auto list_costs = [&](double mult) {
+      costs.clear();
+      for (const Seg& s : segs)
+        if (!s.tc) costs.push_back(s.cost);  // shared-prefix group items, never split
+      int last = -1;
+      int32_t m = 0;
+      for (const Unit& u : units) {
+        const int rows = u.n_q * g;
+        if (is_tc(rows)) continue;
+        if (rows != last) {
+          m = max_keys_for(u, false, mult);
+          last = rows;
+        }
+        const int n = std::max(0, u.k_end - u.k_begin);
+        if (n == 0) continue;
+        const uint32_t nseg = (uint32_t(n) + uint32_t(m) - 1u) / uint32_t(m);
+        const int64_t seg = round_up(int64_t((uint32_t(n) + nseg - 1u) / nseg), PKV_TILE_KEYS);
+        for (int64_t k0 = 0; k0 < n; k0 += seg) costs.push_back(double(std::min<int64_t>(n, k0 + seg) - k0) * u.weight);
+      }
+    };
+    auto makespan = [&]() {
+      std::sort(costs.begin(), costs.end(), std::greater<double>());
+      std::priority_queue<double, std::vector<double>, std::greater<double>> load;
+      for (int i = 0; i < num_ctas; ++i) load.push(0.0);
+      double worst = 0.0;
+      for (double c : costs) {
+        const double t = load.top() + c;
+        load.pop();
+        load.push(t);
+        worst = std::max(worst, t);
+      }
+      return worst;
+    };
+    list_costs(1.0);
+    const size_t N = costs.size(), C = size_t(num_ctas);
+    if (N > C && N < 4 * C && (N % C) * 4 < C) {
+      double best = makespan();
+      for (double mult : {1.125, 1.25, 1.375, 1.5}) {
+        list_costs(mult);
+        const double t = makespan();
+        if (t < best * 0.98) {
+          best = t;
+          reg_mult = mult;
+        }
+      }
+    }
+  }
   // Units come in runs of one row count (every KV head of a tile): the split length is computed
   // once per run.
   int last_rows = -1;
@@ -223,12 +291,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     const bool t = is_tc(rows);
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     if (rows != last_rows) {
-      int64_t max_keys;
-      if (req->kv_split < 0) max_keys = INT32_MAX;
-      else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
-      else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
-                                        round_up(int64_t(std::ceil(target[t] / u.weight)), tile_keys));
-      mk = int32_t(std::min<int64_t>(max_keys, INT32_MAX / 2));
+      mk = max_keys_for(u, t, t ? 1.0 : reg_mult);
       last_rows = rows;
     }
     const int32_t nseg = n == 0 ? 0 : int32_t((uint32_t(n) + uint32_t(mk) - 1u) / uint32_t(mk));

@@ -261,3 +261,23 @@ def test_plan_is_deterministic_and_reuses_buffers(api):
     small = torch.zeros(64, dtype=torch.uint8)
     d = _plan(api, w, buffer=small)
     assert d.buffer is not small and torch.equal(d.buffer[:n], a.buffer[:n]) and not small.any()
+
+
+def test_plan_avoids_a_tail_round(api):
+    """Eight equal 131072-key sequences on 296 CTAs: about two items per CTA would be 640 pieces
+    of 13120 keys, leaving 48 CTAs a third round; the planner takes 9 pieces per (sequence, KV
+    head) instead (576 items, no CTA beyond two rounds).  Batches of unequal lengths keep the
+    two-items-per-CTA split."""
+    w = W.longctx_fp8()
+    d = PD.decode(_plan(api, w).buffer)
+    items = d["items"]
+    assert len(items) <= 2 * 296 and len(items) == 8 * 8 * 9
+    assert set((items["k_end"] - items["k_begin"]).tolist()) == {14592, 131072 - 8 * 14592}
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
+                      w.block_size)
+    explicit = PD.decode(_plan(api, w, kv_split=14592).buffer)
+    assert np.array_equal(explicit["items"], items)
+    dec = W.llama3_8b_decode_bf16()
+    two_per_cta = -(-int(dec.seq_lens.sum()) * dec.num_kv_heads // (2 * 296))  # keys, one-row-group weight 1
+    auto, fixed = _plan(api, dec), _plan(api, dec, kv_split=-(-two_per_cta // 64) * 64)
+    assert torch.equal(auto.buffer[:auto.info["plan_bytes"]], fixed.buffer[:fixed.info["plan_bytes"]])
