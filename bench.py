@@ -158,10 +158,11 @@ TRAFFIC_SOURCES = ("attn_tma.cu", "attn_tile.cuh", "attn_args.h", "common.cuh", 
 
 
 def _code_only(src: str) -> str:
-    """C/C++ source without comments or blank lines: a comment edit does not change the kernel."""
+    """C/C++ source without comments, blank lines or runs of spaces: a comment edit does not change
+    the kernel."""
     src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
-    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return "\n".join(" ".join(line.split()) for line in src.splitlines() if line.strip())
 
 
 def read_stream_gbs(buf, reps: int = 10):

@@ -46,3 +46,13 @@ def test_prefill_flops_by_enumeration():
             for j in range(ql):
                 pairs += sum(1 for t in range(L) if t <= L - ql + j)
     assert bench.prefill_flops(w) == 4.0 * w.head_dim * w.num_q_heads * pairs
+
+
+def test_traffic_key_ignores_comments_only():
+    """The key that ties an ncu traffic figure to the decode kernel's code: comment and blank-line
+    edits keep it, a code edit changes it."""
+    src = "int f(int x) {  // doubles\n  /* body */ return 2 * x;\n}\n"
+    same = "// a header\nint f(int x) {\n\n  return 2 * x;  /* still doubles */\n}\n"
+    other = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench._code_only(src) == bench._code_only(same)
+    assert bench._code_only(src) != bench._code_only(other)
