@@ -169,7 +169,8 @@ PKV_API pkv_status pkv_kv_append(const pkv_cache* cache, const void* k_new, cons
  * Errors: INVALID_ARG for bad shapes / null pointers.  Asynchronously, copies
  *   with a block id outside [0, num_blocks) (PKV_DEV_BAD_BLOCK_ID) or a token
  *   count outside [0, block_size] (PKV_DEV_BAD_COPY) are skipped.
- * Stream-ordered; bit-exact (a byte copy, any pool dtype).
+ * Stream-ordered; bit-exact (a byte copy, any pool dtype; for NVFP4 pools, head_dim
+ *   128, the slots' codes and their block scales).
  */
 PKV_API pkv_status pkv_copy_block_prefix(const pkv_cache* cache, const int32_t* src_blocks,
                                          const int32_t* dst_blocks, const int32_t* n_tokens, int32_t count,
