@@ -317,6 +317,25 @@ PKV_API pkv_status pkv_split_kv_reduce(const float* partial_o, const float* part
                                int32_t head_dim, void* out, int32_t out_dtype, float* out_lse, void* stream);
 
 /*
+ * stream_read - a plain read-only stream over device memory (a measurement aid).
+ *
+ * Decode attention reads every cached K/V byte once per step (deep dive §2:
+ * decode reads all history KV), so the fastest plain read of HBM is the
+ * practical ceiling its bandwidth is judged against.  This reads `bytes`
+ * bytes at `src` once and XOR-folds them into *sink (device uint32, any
+ * initial value) so that no load is dead.
+ * mode 0: every thread issues 16-byte non-caching loads over a grid-strided
+ *   range (4 CTAs of 512 threads per SM);
+ * mode 1: one elected thread per CTA copies 32 KB chunks into a 4-stage
+ *   shared-memory ring with 1-D bulk async copies counted on mbarriers, as the
+ *   attention kernels' TMA producers do (one CTA per SM, no multicast).
+ * src and bytes: multiples of 16.  dev_status: PKV_DEV_TIMEOUT if a ring wait
+ *   of mode 1 gives up (may be NULL).  Stream-ordered; allocates nothing.
+ */
+PKV_API pkv_status pkv_stream_read(const void* src, size_t bytes, int32_t mode, uint32_t* sink,
+                                   int32_t* dev_status, void* stream);
+
+/*
  * paged_attention_noalloc - paged_attention for callers that cannot allocate.
  *
  * The pages have no counterpart to this call; it exists for callers that are

@@ -88,6 +88,8 @@ _lib.pkv_paged_attention_timed.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P
 _lib.pkv_paged_attention_noalloc.restype = _I32
 _lib.pkv_paged_attention_noalloc.argtypes = [C.POINTER(_Cache), _P, _I32, _I32, _P, _P, _P, _I32, _I32, _F, _I32, _P,
                                              _P, _P, _P, _P]
+_lib.pkv_stream_read.restype = _I32
+_lib.pkv_stream_read.argtypes = [_P, _SZ, _I32, _P, _P, _P]
 _lib.pkv_split_kv_reduce.restype = _I32
 _lib.pkv_split_kv_reduce.argtypes = [_P, _P, _I32, _I64, _I32, _P, _I32, _P, _P]
 
@@ -241,6 +243,67 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
     return Plan(buf, {f: getattr(info, f) for f, _ in _PlanInfo._fields_})
 
 
+class Planner:
+    """A reusable host planner for batches of one size: the planning request and the host int32
+    arrays it points at are built once, so each :meth:`plan` is a single call into the library.
+
+    ``cu_q_lens`` ``[num_seqs + 1]``, ``seq_lens`` ``[num_seqs]`` and ``block_tables``
+    ``[num_seqs][max_blocks]`` are the host arrays the planner reads; contiguous int32 arrays
+    given here (numpy, or CPU torch tensors, page-locked ones included) are used in place, so a
+    caller that updates them between steps re-plans without any copy; others are copied once.
+    ``block_tables`` may be None (no shared-prefix grouping).
+    """
+
+    def __init__(self, cu_q_lens, seq_lens, block_tables=None, *, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, block_size: int, kv_dtype: int | str, causal: bool = True, num_ctas: int = 0,
+                 kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0, window: int = 0,
+                 max_blocks: int | None = None):
+        self.cu_q_lens = self._host(cu_q_lens)
+        self.seq_lens = self._host(seq_lens)
+        self.block_tables = None if block_tables is None else self._host(block_tables)
+        if max_blocks is None:
+            max_blocks = self.block_tables.shape[1] if self.block_tables is not None else 1
+        code = DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+        self._req = _PlanRequest(self.seq_lens.shape[0], num_q_heads, num_kv_heads, head_dim, block_size, code,
+                                 int(bool(causal)), num_ctas, kv_split, int(bool(cascade)), min_shared_tokens,
+                                 max_blocks, self.cu_q_lens.ctypes.data, self.seq_lens.ctypes.data,
+                                 None if self.block_tables is None else self.block_tables.ctypes.data, int(window))
+        self._req_ref = C.byref(self._req)
+        self._info = _PlanInfo()
+        self._info_ref = C.byref(self._info)
+
+    @staticmethod
+    def _host(x) -> np.ndarray:
+        if isinstance(x, torch.Tensor):
+            if x.device.type != "cpu":
+                raise ValueError("the planner reads host arrays")
+            if x.dtype == torch.int32 and x.is_contiguous():
+                return x.numpy()  # shares the tensor's memory
+            x = x.numpy()
+        return np.ascontiguousarray(x, dtype=np.int32)
+
+    def plan(self, buffer: torch.Tensor | None = None, pin: bool = True) -> Plan:
+        """Plan into ``buffer`` (uint8 host; a new page-locked one when missing or too small)."""
+        st = (_lib.pkv_attention_plan(self._req_ref, buffer.data_ptr(), buffer.numel(), self._info_ref)
+              if buffer is not None else _WORKSPACE_TOO_SMALL)
+        if st != 0:
+            if st != _WORKSPACE_TOO_SMALL:
+                _check(st, "attention_plan")
+            _check(_lib.pkv_attention_plan(self._req_ref, None, 0, self._info_ref), "attention_plan")
+            buffer = torch.empty(int(self._info.plan_bytes), dtype=torch.uint8,
+                                 pin_memory=pin and torch.cuda.is_available())
+            _check(_lib.pkv_attention_plan(self._req_ref, buffer.data_ptr(), buffer.numel(), self._info_ref),
+                   "attention_plan")
+        return Plan(buffer, {f: getattr(self._info, f) for f, _ in _PlanInfo._fields_})
+
+    def plan_into(self, buffer: torch.Tensor) -> int:
+        """Plan into ``buffer`` (large enough, as a previous :meth:`plan` of these shapes returned it);
+        returns the plan's bytes.  The cheapest form: one library call, no result dictionary."""
+        _check(_lib.pkv_attention_plan(self._req_ref, buffer.data_ptr(), buffer.numel(), self._info_ref),
+               "attention_plan")
+        return self._info.plan_bytes
+
+
 def attention_workspace_bytes(plan: Plan) -> int:
     return plan.workspace_bytes
 
@@ -312,6 +375,13 @@ def split_kv_reduce(partial_o: torch.Tensor, partial_lse: torch.Tensor, out_dtyp
     return out, out_lse
 
 
+def stream_read(buf: torch.Tensor, sink: torch.Tensor, mode: int = 0, status: torch.Tensor | None = None,
+                stream=None) -> None:
+    """Read every byte of device tensor ``buf`` once (pkv_stream_read); ``sink``: device int32 [1]."""
+    _check(_lib.pkv_stream_read(buf.data_ptr(), buf.numel() * buf.element_size(), int(mode), sink.data_ptr(),
+                                _ptr(status), _stream(stream)), "stream_read")
+
+
 class GraphStep:
     """One serving step from page-locked host inputs, as three CUDA graphs per buffer slot.
 
@@ -362,6 +432,7 @@ class GraphStep:
         self._out_h = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(slots)]
         self.d2h_bytes = q.numel() * q.element_size()
         self._plans = [None] * slots
+        self._planners = [None] * slots
         self._graphs = [None] * slots  # (copy in, compute, copy out) per slot
         self._shape = [None] * slots
         self._ready = [torch.cuda.Event() for _ in range(slots)]     # inputs of the slot on the device
@@ -372,10 +443,12 @@ class GraphStep:
         self._slot = 0
 
     def _plan_into(self, b: int) -> Plan:
-        h = self.host[b]
+        # One planner per slot reads the slot's page-locked lengths and tables in place.
+        if self._planners[b] is None:
+            h = self.host[b]
+            self._planners[b] = Planner(h["cu_q"], h["seq_lens"], h["block_tables"], **self.plan_kwargs)
         buf = None if self._plans[b] is None else self._plans[b].buffer
-        return plan_attention(h["cu_q"].numpy(), h["seq_lens"].numpy(), block_tables=h["block_tables"].numpy(),
-                              buffer=buf, **self.plan_kwargs)
+        return self._planners[b].plan(buf)
 
     def _capture(self, b: int, plan: Plan) -> None:
         if self._ws is None or self._ws.numel() < plan.workspace_bytes:

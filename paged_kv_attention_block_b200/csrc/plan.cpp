@@ -8,15 +8,20 @@
 //   1. groups consecutive sequences whose block tables start with the same
 //      physical blocks (cascade): their shared keys become one dense tile per
 //      group and KV head instead of one read per sequence;
-//   2. cuts every (sequence, query tile, KV head) into key ranges small enough
-//      that the persistent CTAs finish together, weighting a tile by its rows
-//      (compute) and keys (bytes);
+//   2. cuts every (sequence, query tile) into key pieces small enough that the
+//      persistent CTAs finish together, weighting a tile by its rows (compute)
+//      and keys (bytes); every KV head of a tile gets the same pieces;
 //   3. emits the merges that combine split ranges (and group tiles) per row.
 // On 16-bit pools tiles of more than 16 rows (prefill chunks, shared-prefix
 // groups) go to a second list served by the tcgen05 kernel, 128 rows a tile,
 // and are split and balanced over that kernel's CTAs on their own.  Items are
 // ordered heaviest first within each list; CTAs pull them from an atomic
 // counter.
+//
+// The work is done once per (query tile, key piece) -- a "piece" below -- and
+// expanded over the KV heads only when the items are written: a decode batch of
+// S sequences plans S tiles, not S x Hkv.  Scratch vectors live per thread and
+// keep their capacity across calls, so a steady-state plan allocates nothing.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -29,50 +34,69 @@
 
 namespace {
 
-struct Unit {
-  int seq, kv_head, q_begin, n_q, k_begin, k_end, pos0, group_part;
-  double weight;
+// One (query tile, key piece): every KV head h of it becomes an item (and, when the tile's
+// keys are split or it belongs to a shared-prefix group, a merge per head).
+struct Piece {
+  int32_t seq, q_begin, n_q, k_begin, k_end, pos0;
+  int32_t part0;     // partial row of head 0 (head h: part0 + h * part_stride); -1: final output
+  int32_t part_stride;
+  uint64_t cost16;   // 16 x keys x max(1, rows / 16)
+  bool tc;           // tensor-memory list
 };
 
-struct Seg {
-  PkvItem it;
-  double cost;
-  bool tc;  // tensor-memory list
+// A (query tile) whose keys were split or that also reads a group tile: one merge per KV head.
+struct Merge {
+  int32_t q_begin, n_q;
+  int32_t group_part0, group_stride;  // partial row of head 0 in its group tile; -1: none
+  int32_t first_piece, n_pieces;      // pieces of this tile (consecutive in the piece list)
 };
 
-// Register-tile items first, then tensor-memory items; heaviest first within each list, ties in
-// creation order (the order a stable sort by cost would keep).  A cost is keys x max(1, rows/16),
-// so c = 16 x cost is an integer (clamped to 32 bits past 2^25 keys).  Each item gets the key
-// [list bit][c_max - c, `bits` wide][creation index, 20 bits] (the planner refuses 2^20 items or
-// more), and a stable least-significant-digit radix sort over the bits above the index, in
-// 11-bit digits, orders them: the indices start ascending and stability keeps ties that way.
-void order_segments(const std::vector<Seg>& segs, std::vector<uint64_t>& keys, std::vector<uint64_t>& tmp) {
-  const size_t n = segs.size();
+struct Scratch {
+  std::vector<Piece> pieces;
+  std::vector<Merge> merges;
+  std::vector<int32_t> group_of;
+  std::vector<int64_t> member_part;  // per sequence: partial row of head 0 in its group tile
+  std::vector<int32_t> member_stride;
+  std::vector<uint64_t> keys, tmp;
+  std::vector<double> costs;
+};
+
+Scratch& scratch() {
+  thread_local Scratch s;
+  return s;
+}
+
+// Pieces ordered register-tile list first, then tensor-memory list; heaviest first within each
+// list, ties in creation order.  Each piece gets the key [list bit][c_max - c, `bits` wide]
+// [creation index, 20 bits] (the planner refuses 2^20 pieces or more), and a stable
+// least-significant-digit radix sort over the bits above the index, in 8-bit digits, orders them:
+// the indices start ascending and stability keeps ties that way.
+void order_pieces(const std::vector<Piece>& ps, std::vector<uint64_t>& keys, std::vector<uint64_t>& tmp) {
+  const size_t n = ps.size();
   keys.resize(n);
   tmp.resize(n);
   uint64_t c_max = 0;
-  for (size_t i = 0; i < n; ++i) {
-    keys[i] = std::min<uint64_t>(uint64_t(segs[i].cost * 16.0 + 0.5), 0xFFFFFFFFull);
-    c_max = std::max(c_max, keys[i]);
-  }
+  for (size_t i = 0; i < n; ++i) c_max = std::max(c_max, std::min<uint64_t>(ps[i].cost16, 0xFFFFFFFFull));
   int bits = 0;
   while (bits < 32 && (c_max >> bits) != 0) ++bits;
   for (size_t i = 0; i < n; ++i)
-    keys[i] = (((uint64_t(segs[i].tc) << bits) | (c_max - keys[i])) << 20) | uint64_t(i);
+    keys[i] = (((uint64_t(ps[i].tc) << bits) | (c_max - std::min<uint64_t>(ps[i].cost16, 0xFFFFFFFFull))) << 20) |
+              uint64_t(i);
   if (n < 2) return;
-  uint32_t count[2048];
-  for (int shift = 20; shift < 21 + bits; shift += 11) {
+  uint32_t count[256];
+  for (int shift = 20; shift < 21 + bits; shift += 8) {
     std::memset(count, 0, sizeof(count));
-    for (size_t i = 0; i < n; ++i) ++count[(keys[i] >> shift) & 2047];
-    if (count[(keys[0] >> shift) & 2047] == n) continue;  // one digit value: order unchanged
+    for (size_t i = 0; i < n; ++i) ++count[(keys[i] >> shift) & 255];
+    if (count[(keys[0] >> shift) & 255] == n) continue;  // one digit value: order unchanged
     uint32_t sum = 0;
-    for (int d = 0; d < 2048; ++d) { const uint32_t c = count[d]; count[d] = sum; sum += c; }
-    for (size_t i = 0; i < n; ++i) tmp[count[(keys[i] >> shift) & 2047]++] = keys[i];
+    for (int d = 0; d < 256; ++d) { const uint32_t c = count[d]; count[d] = sum; sum += c; }
+    for (size_t i = 0; i < n; ++i) tmp[count[(keys[i] >> shift) & 255]++] = keys[i];
     keys.swap(tmp);
   }
 }
 
-double row_weight(int rows) { return rows <= 16 ? 1.0 : rows / 16.0; }
+// 16 x the cost weight of a tile of `rows` rows: max(1, rows / 16) x 16.
+inline uint64_t weight16(int rows) { return uint64_t(std::max(16, rows)); }
 
 // m a power of two
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) & ~(m - 1); }
@@ -133,7 +157,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   // 1. Shared-prefix groups.
   struct Group { int first, last, tokens; };
   std::vector<Group> groups;
-  std::vector<int> group_of(S, -1);
+  Scratch& sc = scratch();
+  sc.group_of.assign(size_t(S), -1);
   // A window would cut the shared prefix differently for every member: no groups then.
   if (req->cascade && req->block_tables && S > 1 && window == 0) {
     const int32_t* bt = req->block_tables;
@@ -154,7 +179,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
         ++t;
       }
       if (t - s >= 2 && int64_t(P) * B >= min_sh) {
-        for (int m = s; m < t; ++m) group_of[m] = int(groups.size());
+        for (int m = s; m < t; ++m) sc.group_of[m] = int(groups.size());
         groups.push_back({s, t - 1, P * B});
         s = t;
       } else {
@@ -163,40 +188,46 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     }
   }
 
-  std::vector<Seg> segs;
-  std::vector<PkvReduce> reds;
-  std::vector<int32_t> parts;
-  segs.reserve(size_t(S) * Hkv * 2 + 64);
-  reds.reserve(size_t(S) * Hkv);
-  parts.reserve(size_t(S) * Hkv * 2);
+  std::vector<Piece>& pieces = sc.pieces;
+  std::vector<Merge>& merges = sc.merges;
+  pieces.clear();
+  merges.clear();
   int64_t part_rows = 0;
-  // Partial row of each (group member, KV head) inside its group tile.
-  std::vector<int64_t> gpart(groups.empty() ? 0 : size_t(S) * Hkv, -1);
-  double total_cost[2] = {0, 0};  // register-tile list, tensor-memory list
+  double total_cost[2] = {0, 0};  // register-tile list, tensor-memory list (keys x weight, all heads)
+  if (!groups.empty()) {
+    sc.member_part.assign(size_t(S), -1);
+    sc.member_stride.assign(size_t(S), 0);
+  }
+  // Group tiles: consecutive members packed into tiles of at most QT query tokens; the tile of
+  // head h writes its partial rows at part0 + h * n * g.
   for (const Group& G : groups) {
     int a = G.first;
     while (a <= G.last) {
       int b = a, n = q_len(a);
       while (b + 1 <= G.last && n + q_len(b + 1) <= QT) n += q_len(++b);
-      for (int h = 0; h < Hkv; ++h) {
-        PkvItem it{G.first, h, cu[a], n, 0, G.tokens, -1, int32_t(part_rows)};
-        for (int m = a; m <= b; ++m) gpart[size_t(m) * Hkv + h] = part_rows + int64_t(cu[m] - cu[a]) * g;
-        part_rows += int64_t(n) * g;
-        const double c = double(G.tokens) * row_weight(n * g);
-        total_cost[is_tc(n * g)] += c;
-        segs.push_back({it, c, is_tc(n * g)});
+      const int rows = n * g;
+      for (int m = a; m <= b; ++m) {
+        sc.member_part[m] = part_rows + int64_t(cu[m] - cu[a]) * g;
+        sc.member_stride[m] = rows;
       }
+      const bool t = is_tc(rows);
+      pieces.push_back({G.first, cu[a], n, 0, G.tokens, -1, int32_t(part_rows), rows,
+                        uint64_t(G.tokens) * weight16(rows), t});
+      part_rows += int64_t(rows) * Hkv;
+      total_cost[t] += double(G.tokens) * double(weight16(rows)) / 16.0 * Hkv;
       a = b + 1;
     }
   }
+  const size_t n_group_pieces = pieces.size();
 
-  // 2. Units of work.
-  std::vector<Unit> units;
-  units.reserve(size_t(S) * Hkv);
+  // 2. Query tiles: (sequence, first token, tokens, keys [k0, ke), first position).
+  struct Tile { int32_t seq, q_begin, n_q, k0, ke, pos0; };
+  std::vector<Tile> tiles;
+  tiles.reserve(size_t(S));
   for (int s = 0; s < S; ++s) {
     const int ql = q_len(s);
     if (ql == 0) continue;
-    const int kb = group_of[s] >= 0 ? groups[group_of[s]].tokens : 0;
+    const int kb = sc.group_of[s] >= 0 ? groups[sc.group_of[s]].tokens : 0;
     for (int i0 = 0; i0 < ql; i0 += QT) {
       const int n = std::min(QT, ql - i0);
       const int ke = causal ? L[s] - ql + i0 + n : L[s];
@@ -204,27 +235,30 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       // Under a window the tile's first row sees keys from pos0 - window + 1 on; the range starts
       // there, rounded down to 128 keys (the kernels' tile alignment), and rows mask the rest.
       const int k0 = window > 0 ? std::max(kb, int(std::max(0, pos0 - window + 1) / 128 * 128)) : kb;
-      for (int h = 0; h < Hkv; ++h) {
-        const int gp = group_of[s] >= 0 ? int(gpart[size_t(s) * Hkv + h]) : -1;
-        Unit u{s, h, cu[s] + i0, n, k0, ke, pos0, gp, row_weight(n * g)};
-        total_cost[is_tc(n * g)] += double(std::max(0, ke - k0)) * u.weight;
-        units.push_back(u);
-      }
+      tiles.push_back({s, cu[s] + i0, n, k0, ke, pos0});
+      total_cost[is_tc(n * g)] += double(std::max(0, ke - k0)) * double(weight16(n * g)) / 16.0 * Hkv;
     }
   }
 
   // 3. Key-range split and merges.
   const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 2.0)};
-  // Longest key range of one item of a unit's list; the automatic length (about two items per
+  // Longest key range of one item of a tile's list; the automatic length (about two items per
   // CTA) is scaled by `mult`.
-  auto max_keys_for = [&](const Unit& u, bool t, double mult) -> int32_t {
+  auto max_keys_for = [&](int rows, bool t, double mult) -> int32_t {
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     int64_t max_keys;
     if (req->kv_split < 0) max_keys = INT32_MAX;
     else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
     else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
-                                      round_up(int64_t(std::ceil(target[t] * mult / u.weight)), tile_keys));
+                                      round_up(int64_t(std::ceil(target[t] * mult * 16.0 / double(weight16(rows)))),
+                                               tile_keys));
     return int32_t(std::min<int64_t>(max_keys, INT32_MAX / 2));
+  };
+  // Pieces of a range of n keys split into pieces of at most mk keys: nseg pieces of `seg` keys
+  // (a multiple of the tile), the last one shorter.
+  auto split = [](int n, int32_t mk, int64_t tile_keys, int32_t& nseg, int64_t& seg) {
+    nseg = n == 0 ? 0 : int32_t((uint32_t(n) + uint32_t(mk) - 1u) / uint32_t(mk));
+    seg = nseg == 0 ? 0 : round_up(int64_t((uint32_t(n) + uint32_t(nseg) - 1u) / uint32_t(nseg)), tile_keys);
   };
   // Tail check of the register-tile list.  The CTAs take items heaviest first from a counter, so
   // when the item count only just passes a multiple of the CTA count (a batch of equal long
@@ -233,47 +267,58 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   // assignment the counter produces, constant per-CTA speed) is kept if it is 2 % shorter.
   double reg_mult = 1.0;
   if (req->kv_split == 0) {
-    std::vector<double> costs;
-    auto list_costs = [&](double mult) {
-      costs.clear();
-      for (const Seg& s : segs)
-        if (!s.tc) costs.push_back(s.cost);  // shared-prefix group items, never split
+    auto count_items = [&](double mult) {
+      size_t n_items = 0;
+      for (size_t i = 0; i < n_group_pieces; ++i) n_items += pieces[i].tc ? 0 : size_t(Hkv);
       int last = -1;
       int32_t m = 0;
-      for (const Unit& u : units) {
-        const int rows = u.n_q * g;
+      for (const Tile& t : tiles) {
+        const int rows = t.n_q * g;
         if (is_tc(rows)) continue;
-        if (rows != last) {
-          m = max_keys_for(u, false, mult);
-          last = rows;
-        }
-        const int n = std::max(0, u.k_end - u.k_begin);
-        if (n == 0) continue;
-        const uint32_t nseg = (uint32_t(n) + uint32_t(m) - 1u) / uint32_t(m);
-        const int64_t seg = round_up(int64_t((uint32_t(n) + nseg - 1u) / nseg), PKV_TILE_KEYS);
-        for (int64_t k0 = 0; k0 < n; k0 += seg) costs.push_back(double(std::min<int64_t>(n, k0 + seg) - k0) * u.weight);
+        if (rows != last) { m = max_keys_for(rows, false, mult); last = rows; }
+        int32_t nseg;
+        int64_t seg;
+        split(std::max(0, t.ke - t.k0), m, PKV_TILE_KEYS, nseg, seg);
+        n_items += size_t(nseg) * size_t(Hkv);
       }
+      return n_items;
     };
-    auto makespan = [&]() {
-      std::sort(costs.begin(), costs.end(), std::greater<double>());
-      std::priority_queue<double, std::vector<double>, std::greater<double>> load;
-      for (int i = 0; i < num_ctas; ++i) load.push(0.0);
-      double worst = 0.0;
-      for (double c : costs) {
-        const double t = load.top() + c;
-        load.pop();
-        load.push(t);
-        worst = std::max(worst, t);
-      }
-      return worst;
-    };
-    list_costs(1.0);
-    const size_t N = costs.size(), C = size_t(num_ctas);
+    const size_t N = count_items(1.0), C = size_t(num_ctas);
     if (N > C && N < 4 * C && (N % C) * 4 < C) {
-      double best = makespan();
+      std::vector<double>& costs = sc.costs;
+      auto makespan = [&](double mult) {
+        costs.clear();
+        for (size_t i = 0; i < n_group_pieces; ++i)  // shared-prefix group items, never split
+          if (!pieces[i].tc) costs.insert(costs.end(), size_t(Hkv), double(pieces[i].cost16) / 16.0);
+        int last = -1;
+        int32_t m = 0;
+        for (const Tile& t : tiles) {
+          const int rows = t.n_q * g;
+          if (is_tc(rows)) continue;
+          if (rows != last) { m = max_keys_for(rows, false, mult); last = rows; }
+          const int n = std::max(0, t.ke - t.k0);
+          int32_t nseg;
+          int64_t seg;
+          split(n, m, PKV_TILE_KEYS, nseg, seg);
+          const double w = double(weight16(rows)) / 16.0;
+          for (int64_t k0 = 0; k0 < n; k0 += seg)
+            costs.insert(costs.end(), size_t(Hkv), double(std::min<int64_t>(n, k0 + seg) - k0) * w);
+        }
+        std::sort(costs.begin(), costs.end(), std::greater<double>());
+        std::priority_queue<double, std::vector<double>, std::greater<double>> load;
+        for (int i = 0; i < num_ctas; ++i) load.push(0.0);
+        double worst = 0.0;
+        for (double c : costs) {
+          const double t = load.top() + c;
+          load.pop();
+          load.push(t);
+          worst = std::max(worst, t);
+        }
+        return worst;
+      };
+      double best = makespan(1.0);
       for (double mult : {1.125, 1.25, 1.375, 1.5}) {
-        list_costs(mult);
-        const double t = makespan();
+        const double t = makespan(mult);
         if (t < best * 0.98) {
           best = t;
           reg_mult = mult;
@@ -281,56 +326,62 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       }
     }
   }
-  // Units come in runs of one row count (every KV head of a tile): the split length is computed
-  // once per run.
+  // Tiles come in runs of one row count: the split length is computed once per run.
   int last_rows = -1;
   int32_t mk = 0;
-  for (const Unit& u : units) {
-    const int n = std::max(0, u.k_end - u.k_begin);
-    const int rows = u.n_q * g;
+  int64_t n_parts = 0;
+  for (const Tile& tl : tiles) {
+    const int n = std::max(0, tl.ke - tl.k0);
+    const int rows = tl.n_q * g;
     const bool t = is_tc(rows);
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     if (rows != last_rows) {
-      mk = max_keys_for(u, t, t ? 1.0 : reg_mult);
+      mk = max_keys_for(rows, t, t ? 1.0 : reg_mult);
       last_rows = rows;
     }
-    const int32_t nseg = n == 0 ? 0 : int32_t((uint32_t(n) + uint32_t(mk) - 1u) / uint32_t(mk));
-    if (nseg == 1 && u.group_part < 0) {
-      PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, u.k_begin, u.k_end, u.pos0, -1};
-      segs.push_back({it, n * u.weight, t});
+    int32_t nseg;
+    int64_t seg;
+    split(n, mk, tile_keys, nseg, seg);
+    const uint64_t w16 = weight16(rows);
+    const int32_t gp = sc.group_of[tl.seq] >= 0 ? int32_t(sc.member_part[tl.seq]) : -1;
+    if (nseg == 1 && gp < 0) {
+      pieces.push_back({tl.seq, tl.q_begin, tl.n_q, tl.k0, tl.ke, tl.pos0, -1, 0, uint64_t(n) * w16, t});
       continue;
     }
-    PkvReduce r{u.q_begin, u.n_q, u.kv_head, int32_t(parts.size()), 0, {0, 0, 0}};
-    if (u.group_part >= 0) parts.push_back(u.group_part);
-    if (nseg > 0) {
-      const int64_t seg = round_up(int64_t((uint32_t(n) + uint32_t(nseg) - 1u) / uint32_t(nseg)), tile_keys);
-      for (int64_t k0 = u.k_begin; k0 < u.k_end; k0 += seg) {
-        const int k1 = int(std::min<int64_t>(u.k_end, k0 + seg));
-        PkvItem it{u.seq, u.kv_head, u.q_begin, u.n_q, int(k0), k1, u.pos0, int32_t(part_rows)};
-        parts.push_back(int32_t(part_rows));
-        part_rows += rows;
-        segs.push_back({it, (k1 - k0) * u.weight, t});
-      }
+    Merge mg{tl.q_begin, tl.n_q, gp, gp >= 0 ? sc.member_stride[tl.seq] : 0, int32_t(pieces.size()), nseg};
+    // Partial rows of the tile's pieces: head h, piece p at base + (h * nseg + p) * rows.
+    const int64_t base = part_rows;
+    int p = 0;
+    for (int64_t k0 = tl.k0; k0 < tl.ke; k0 += seg, ++p) {
+      const int k1 = int(std::min<int64_t>(tl.ke, k0 + seg));
+      pieces.push_back({tl.seq, tl.q_begin, tl.n_q, int32_t(k0), k1, tl.pos0, int32_t(base + int64_t(p) * rows),
+                        int32_t(int64_t(nseg) * rows), uint64_t(k1 - k0) * w16, t});
     }
-    r.n_parts = int32_t(parts.size()) - r.parts_begin;
-    reds.push_back(r);
+    part_rows += int64_t(nseg) * rows * Hkv;
+    n_parts += int64_t(nseg + (gp >= 0 ? 1 : 0)) * Hkv;
+    merges.push_back(mg);
+    if (part_rows > INT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: too many partial rows");
   }
   if (part_rows > INT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: too many partial rows");
-  if (segs.size() >= (size_t(1) << 20)) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: more than 2^20 work items");
+  if (pieces.size() >= (size_t(1) << 20) || pieces.size() * size_t(Hkv) >= (size_t(1) << 26))
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: too many work items");
 
-  const int64_t n_tc = std::count_if(segs.begin(), segs.end(), [](const Seg& s) { return s.tc; });
+  size_t n_tc_pieces = 0;
+  for (const Piece& pc : pieces) n_tc_pieces += pc.tc ? 1 : 0;
+  const int64_t n_items = int64_t(pieces.size()) * Hkv, n_tc = int64_t(n_tc_pieces) * Hkv;
+  const int64_t n_reduce = int64_t(merges.size()) * Hkv;
 
   const uint64_t items_off = sizeof(PkvPlanHeader);
-  const uint64_t tc_items_off = items_off + (segs.size() - n_tc) * sizeof(PkvItem);
-  const uint64_t reduce_off = items_off + segs.size() * sizeof(PkvItem);
-  const uint64_t parts_off = reduce_off + reds.size() * sizeof(PkvReduce);
-  const uint64_t bytes = pkv_plan_bytes(parts_off + parts.size() * sizeof(int32_t));
+  const uint64_t tc_items_off = items_off + uint64_t(n_items - n_tc) * sizeof(PkvItem);
+  const uint64_t reduce_off = items_off + uint64_t(n_items) * sizeof(PkvItem);
+  const uint64_t parts_off = reduce_off + uint64_t(n_reduce) * sizeof(PkvReduce);
+  const uint64_t bytes = pkv_plan_bytes(parts_off + uint64_t(n_parts) * sizeof(int32_t));
   if (bytes > UINT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: plan too large");
   info->plan_bytes = bytes;
   info->workspace_bytes = pkv_workspace_layout(bytes, part_rows, D).total;
-  info->num_items = int32_t(segs.size());  // both lists
-  info->num_reduce = int32_t(reds.size());
-  info->num_parts = int32_t(parts.size());
+  info->num_items = int32_t(n_items);  // both lists
+  info->num_reduce = int32_t(n_reduce);
+  info->num_parts = int32_t(n_parts);
   info->num_partial_rows = int32_t(part_rows);
   info->num_groups = int32_t(groups.size());
   info->num_ctas = num_ctas;
@@ -339,11 +390,10 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (capacity < bytes) return pkv_fail(PKV_ERR_WORKSPACE, "attention_plan: capacity %zu < %llu", capacity, (unsigned long long)bytes);
 
   char* p = static_cast<char*>(plan);
-  std::memset(p, 0, bytes);
   PkvPlanHeader h{};
   h.magic = PKV_PLAN_MAGIC;
   h.bytes = uint32_t(bytes);
-  h.n_items = int32_t(segs.size() - n_tc);
+  h.n_items = int32_t(n_items - n_tc);
   h.n_tc_items = int32_t(n_tc);
   h.tc_items_off = uint32_t(tc_items_off);
   h.tc_num_ctas = tc_ctas;
@@ -365,11 +415,32 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.reduce_off = uint32_t(reduce_off);
   h.parts_off = uint32_t(parts_off);
   std::memcpy(p, &h, sizeof(h));
+  // Items: pieces heaviest first, each expanded over the KV heads.
   PkvItem* items = reinterpret_cast<PkvItem*>(p + items_off);
-  std::vector<uint64_t> order, scratch;
-  order_segments(segs, order, scratch);
-  for (size_t i = 0; i < segs.size(); ++i) items[i] = segs[size_t(order[i] & 0xFFFFF)].it;
-  if (!reds.empty()) std::memcpy(p + reduce_off, reds.data(), reds.size() * sizeof(PkvReduce));
-  if (!parts.empty()) std::memcpy(p + parts_off, parts.data(), parts.size() * sizeof(int32_t));
+  order_pieces(pieces, sc.keys, sc.tmp);
+  for (size_t i = 0; i < pieces.size(); ++i) {
+    const Piece& pc = pieces[size_t(sc.keys[i] & 0xFFFFF)];
+    for (int hh = 0; hh < Hkv; ++hh)
+      *items++ = PkvItem{pc.seq, hh, pc.q_begin, pc.n_q, pc.k_begin, pc.k_end, pc.pos0,
+                         pc.part0 < 0 ? -1 : pc.part0 + hh * pc.part_stride};
+  }
+  // Merges and their part lists, per tile and KV head: the group part first, then the pieces.
+  PkvReduce* reds = reinterpret_cast<PkvReduce*>(p + reduce_off);
+  int32_t* parts = reinterpret_cast<int32_t*>(p + parts_off);
+  int32_t np = 0;
+  for (const Merge& mg : merges) {
+    for (int hh = 0; hh < Hkv; ++hh) {
+      const int32_t begin = np;
+      if (mg.group_part0 >= 0) parts[np++] = mg.group_part0 + hh * mg.group_stride;
+      for (int k = 0; k < mg.n_pieces; ++k) {
+        const Piece& pc = pieces[size_t(mg.first_piece + k)];
+        parts[np++] = pc.part0 + hh * pc.part_stride;
+      }
+      *reds++ = PkvReduce{mg.q_begin, mg.n_q, hh, begin, np - begin, {0, 0, 0}};
+    }
+  }
+  // Zero the tail: alignment padding and the work counters.
+  const uint64_t used = parts_off + uint64_t(np) * sizeof(int32_t);
+  std::memset(p + used, 0, bytes - used);
   return PKV_OK;
 }

@@ -230,7 +230,8 @@ def test_plan_balances_decode(api):
 def test_plan_orders_heaviest_first(api, name, make, opts):
     """Each list runs heaviest item first (cost = keys x max(1, rows / 16)), so the last items
     the CTAs claim are the short ones; equal costs keep creation order, which for items outside
-    shared-prefix groups is (first token, KV head, first key) ascending."""
+    shared-prefix groups is (first token, first key, KV head) ascending: the planner splits each
+    query tile once and gives every KV head of it the same key pieces."""
     w = make()
     p = _plan(api, w, **opts)
     d = PD.decode(p.buffer)
@@ -244,7 +245,7 @@ def test_plan_orders_heaviest_first(api, name, make, opts):
             for i in range(1, len(lst)):
                 if cost[i] == cost[i - 1]:
                     a, b = lst[i - 1], lst[i]
-                    assert (a["q_begin"], a["kv_head"], a["k_begin"]) < (b["q_begin"], b["kv_head"], b["k_begin"])
+                    assert (a["q_begin"], a["k_begin"], a["kv_head"]) < (b["q_begin"], b["k_begin"], b["kv_head"])
 
 
 def test_plan_is_deterministic_and_reuses_buffers(api):
