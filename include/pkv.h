@@ -31,8 +31,11 @@
  *   - Asynchronous errors: a block id outside [0, num_blocks), a logical block
  *     beyond the table row, or a plan that does not match the lengths on the
  *     device is recorded by OR-ing a PKV_DEV_* bit into *dev_status (device
- *     int32, zeroed by the caller, may be NULL); the offending rows or keys are
- *     skipped.  No kernel traps.
+ *     int32, zeroed by the caller, may be NULL).  kv_append and copy_block_prefix
+ *     skip the offending rows; paged_attention skips work items that do not fit
+ *     the device lengths and reads the keys of an out-of-range block as zeros
+ *     (no memory outside the pool is read; the affected rows' outputs are not
+ *     meaningful, every other row is unaffected).  No kernel traps.
  *   - Pool layout (row-major):
  *       pool[num_blocks][num_layers][2][num_kv_heads][block_size][head_dim]
  *     index 0 of the "2" axis is K, 1 is V; each (block, layer, K|V, head) is
@@ -56,7 +59,7 @@
 extern "C" {
 #endif
 
-#define PKV_ABI_VERSION 1
+#define PKV_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define PKV_API __attribute__((visibility("default")))
@@ -89,7 +92,8 @@ typedef enum pkv_dtype {
 #define PKV_DEV_BAD_LOGICAL_BLOCK 0x2 /* position needs a table entry beyond max_blocks */
 #define PKV_DEV_PLAN_MISMATCH 0x4     /* plan item does not fit the device lengths */
 #define PKV_DEV_BAD_APPEND 0x8        /* kv_append position negative */
-#define PKV_DEV_TIMEOUT 0x10          /* an internal pipeline wait gave up (about 1 s); results incomplete */
+#define PKV_DEV_TIMEOUT 0x10          /* an internal pipeline wait gave up (after the plan's wait limit: by default
+                                         4e9 SM cycles, 2.0 s at 1965 MHz); results incomplete */
 #define PKV_DEV_BAD_COPY 0x20         /* copy_block_prefix: token count outside [0, block_size] */
 
 /* One layer's view of a paged pool (deep dive §9: one block holds a fixed number
@@ -209,7 +213,20 @@ typedef struct pkv_plan_request {
                                    no longer take part in attention): query row at position p sees keys
                                    p - window < t <= p.  0 = no limit.  Needs causal; disables cascade.
                                    The plan carries it to pkv_paged_attention. */
+  int32_t wait_limit_kcycles;   /* limit on every internal pipeline wait of the attention kernels, in
+                                   thousands of SM cycles; 0 = the default 4e6 (4e9 cycles: 2.0 s at 1965
+                                   MHz, about 3 s at 1.3 GHz).  A wait that runs out sets PKV_DEV_TIMEOUT,
+                                   and the kernel stops issuing work, waits (bounded) for its own copies
+                                   in flight, frees its tensor memory and exits.  >= 0. */
+  int32_t debug_flags;          /* 0 in normal use.  PKV_DEBUG_WITHHOLD_LOADS: the producers of the
+                                   TMA-fed decode kernel and of the tcgen05 kernel publish every work
+                                   item but load no K/V tile, so every consumer wait runs out: a way to
+                                   test the timeout path (with a short wait_limit_kcycles) without a
+                                   fault.  Outputs are then incomplete.  Kernels without a TMA producer
+                                   (block sizes below 8, 64-byte fp8 rows, fp32 pools) ignore it. */
 } pkv_plan_request;
+
+#define PKV_DEBUG_WITHHOLD_LOADS 0x1
 
 typedef struct pkv_plan_info {
   size_t plan_bytes;            /* bytes of the plan buffer */

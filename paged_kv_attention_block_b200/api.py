@@ -57,7 +57,10 @@ class _PlanRequest(C.Structure):
                 ("head_dim", C.c_int32), ("block_size", C.c_int32), ("kv_dtype", C.c_int32), ("causal", C.c_int32),
                 ("num_ctas", C.c_int32), ("kv_split", C.c_int32), ("cascade", C.c_int32),
                 ("min_shared_tokens", C.c_int32), ("max_blocks", C.c_int32), ("cu_q_lens", C.c_void_p),
-                ("seq_lens", C.c_void_p), ("block_tables", C.c_void_p), ("window", C.c_int32)]
+                ("seq_lens", C.c_void_p), ("block_tables", C.c_void_p), ("window", C.c_int32),
+                ("wait_limit_kcycles", C.c_int32), ("debug_flags", C.c_int32)]
+
+PKV_DEBUG_WITHHOLD_LOADS = 0x1
 
 
 class _PlanInfo(C.Structure):
@@ -135,14 +138,18 @@ class Cache:
 
     @staticmethod
     def allocate(num_blocks: int, num_layers: int, num_kv_heads: int, block_size: int, head_dim: int, kv_dtype: str,
-                 device="cuda", fill_nan: bool = True, k_scale=None, v_scale=None) -> "Cache":
+                 device="cuda", fill_nan: bool = True, k_scale=None, v_scale=None,
+                 fill_byte: int | None = None) -> "Cache":
+        """``fill_byte`` (0..255) fills every pool byte with that value instead of the NaN sentinels."""
         code = DTYPE_CODES[kv_dtype]
         shape = (num_blocks, num_layers, 2, num_kv_heads, block_size, head_dim)
         if code == PKV_NVFP4:
             shape = (num_blocks, num_layers, 2, num_kv_heads, block_size * (head_dim // 2 + head_dim // 16))
         tdt = _CODE_TORCH[code]
         pool = torch.empty(shape, dtype=tdt, device=device)
-        if fill_nan:  # sentinel NaNs in every slot no sequence owns (NVFP4: NaN block scales)
+        if fill_byte is not None:
+            pool.view(torch.uint8).fill_(int(fill_byte))
+        elif fill_nan:  # sentinel NaNs in every slot no sequence owns (NVFP4: NaN block scales)
             if code in (PKV_FP8_E4M3, PKV_NVFP4):
                 pool.fill_(0x7F)
             else:
@@ -209,11 +216,14 @@ def _host_i32(x) -> np.ndarray:
 def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
                    kv_dtype: int | str, causal: bool = True, block_tables=None, max_blocks: int | None = None,
                    num_ctas: int = 0, kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0,
-                   pin: bool = True, buffer: torch.Tensor | None = None, window: int = 0) -> Plan:
+                   pin: bool = True, buffer: torch.Tensor | None = None, window: int = 0,
+                   wait_limit_kcycles: int = 0, debug_flags: int = 0) -> Plan:
     """Build the work list for one paged_attention call from host copies of the lengths.
 
     ``window`` > 0 limits every (causal) row to its ``window`` most recent positions; the
-    plan carries it to ``paged_attention``.
+    plan carries it to ``paged_attention``, as it does ``wait_limit_kcycles`` (limit of every
+    pipeline wait, thousands of SM cycles, 0 = default) and ``debug_flags``
+    (``PKV_DEBUG_WITHHOLD_LOADS`` makes every wait run out, to test the timeout path).
 
     ``buffer`` (uint8, host) is reused when large enough; the caller must not
     reuse a buffer whose plan upload may still be pending on the GPU.
@@ -226,7 +236,7 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
     code = DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
     req = _PlanRequest(sl.shape[0], num_q_heads, num_kv_heads, head_dim, block_size, code, int(bool(causal)), num_ctas,
                        kv_split, int(bool(cascade)), min_shared_tokens, max_blocks, cu.ctypes.data, sl.ctypes.data,
-                       None if bt is None else bt.ctypes.data, int(window))
+                       None if bt is None else bt.ctypes.data, int(window), int(wait_limit_kcycles), int(debug_flags))
     info = _PlanInfo()
     # With a buffer given, plan straight into it (one call); only a buffer too small costs a
     # size query and a new buffer.
@@ -257,7 +267,7 @@ class Planner:
     def __init__(self, cu_q_lens, seq_lens, block_tables=None, *, num_q_heads: int, num_kv_heads: int,
                  head_dim: int, block_size: int, kv_dtype: int | str, causal: bool = True, num_ctas: int = 0,
                  kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0, window: int = 0,
-                 max_blocks: int | None = None):
+                 max_blocks: int | None = None, wait_limit_kcycles: int = 0, debug_flags: int = 0):
         self.cu_q_lens = self._host(cu_q_lens)
         self.seq_lens = self._host(seq_lens)
         self.block_tables = None if block_tables is None else self._host(block_tables)
@@ -267,7 +277,8 @@ class Planner:
         self._req = _PlanRequest(self.seq_lens.shape[0], num_q_heads, num_kv_heads, head_dim, block_size, code,
                                  int(bool(causal)), num_ctas, kv_split, int(bool(cascade)), min_shared_tokens,
                                  max_blocks, self.cu_q_lens.ctypes.data, self.seq_lens.ctypes.data,
-                                 None if self.block_tables is None else self.block_tables.ctypes.data, int(window))
+                                 None if self.block_tables is None else self.block_tables.ctypes.data, int(window),
+                                 int(wait_limit_kcycles), int(debug_flags))
         self._req_ref = C.byref(self._req)
         self._info = _PlanInfo()
         self._info_ref = C.byref(self._info)

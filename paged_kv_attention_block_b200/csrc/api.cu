@@ -153,7 +153,8 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: bad cache shape");
   if (h->num_seqs != num_seqs || h->num_q_heads != num_q_heads || h->num_kv_heads != c.num_kv_heads ||
       h->head_dim != c.head_dim || h->block_size != c.block_size || h->kv_dtype != c.kv_dtype ||
-      h->causal != (causal ? 1 : 0) || h->window < 0 || (h->window > 0 && !causal))
+      h->causal != (causal ? 1 : 0) || h->window < 0 || (h->window > 0 && !causal) || h->wait_limit_kcycles < 0 ||
+      (h->debug_flags & ~PKV_DEBUG_WITHHOLD_LOADS))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan was made for other shapes");
   pkv::AttnKernel k;
   if (!pkv::attn_kernel_for(c.kv_dtype, q_dtype, c.head_dim, c.block_size, &k))
@@ -215,6 +216,8 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   a.status = dev_status;
   a.max_rows = k.max_rows;
   a.window = h->window;
+  a.debug_flags = h->debug_flags;
+  a.wait_limit = h->wait_limit_kcycles > 0 ? 1000ll * h->wait_limit_kcycles : PKV_DEFAULT_WAIT_CYCLES;
   if (kernels_begin) {
     e = record_event(static_cast<cudaEvent_t>(kernels_begin), st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));

@@ -103,8 +103,8 @@ struct TcArgs {
 };
 
 // Every lane waits; the warp agrees on the outcome (tcgen05.ld / st are warp-wide).
-PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity) {
-  const bool ok = mbar_wait(bar, parity);
+PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity, const long long* wl) {
+  const bool ok = mbar_wait(bar, parity, wl);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   TcDesc* descs = reinterpret_cast<TcDesc*>(base_ptr + T::DESC_OFF);
   __shared__ volatile int s_abort;
   __shared__ uint32_t s_tmem;
+  __shared__ long long s_wl;  // SM cycles any one wait may take
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // This kernel may start while the decode-tile kernel ahead of it is still running: it reads
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     mbar_init(bar(T::FIN), 2);
     mbar_init(bar(T::END), T::CONSUMER_WARPS);
     s_abort = 0;
+    s_wl = a.wait_limit;
     fence_mbar_init();
   }
   tc::fence_before_sync();
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     for (;;) {
       const int slot = it_seq % T::IR;
       int flag = 1;
-      if (lane == 0) flag = mbar_wait(bar(T::IEMPTY + slot), ((it_seq / T::IR) & 1) ^ 1) ? 1 : 0;
+      if (lane == 0) flag = mbar_wait(bar(T::IEMPTY + slot), ((it_seq / T::IR) & 1) ^ 1, &s_wl) ? 1 : 0;
       if (!__shfl_sync(FULL, flag, 0)) { ok = false; break; }
       const int idx = __shfl_sync(FULL, next_idx, 0);
       TcDesc& d = descs[slot];
@@ -264,6 +266,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         mbar_arrive(bar(T::IFULL + slot), 1);
       }
       ++it_seq;
+      // Test switch: publish the item but load none of its tiles, so every consumer wait runs out.
+      if (a.debug_flags & PKV_DEBUG_WITHHOLD_LOADS) continue;
       const int32_t* bt_row = a.block_tables + int64_t(it.seq) * a.max_blocks;
       for (int t = 0; t < ntiles && ok; ++t, ++q) {
         const int key0 = it.k_begin + t * T::TK;
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         for (int kv = 0; kv < 2; ++kv) {  // K tile, then V tile
           int f = 1;
           if (lane == 0) {
-            f = (!s_abort && mbar_wait(bar((kv ? T::VEMPTY : T::KEMPTY) + stg), par)) ? 1 : 0;
+            f = (!s_abort && mbar_wait(bar((kv ? T::VEMPTY : T::KEMPTY) + stg), par, &s_wl)) ? 1 : 0;
             if (f) mbar_arrive_expect_tx(bar((kv ? T::VFULL : T::KFULL) + stg), bytes);
           }
           if (!__shfl_sync(FULL, f, 0)) { ok = false; break; }
@@ -306,10 +310,10 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;
       // Let loads already issued land before the CTA's shared memory goes away.
-      if (k_armed) mbar_wait(bar(T::KFULL + q % T::NST), (q / T::NST) & 1);
+      if (k_armed) mbar_wait(bar(T::KFULL + q % T::NST), (q / T::NST) & 1, &s_wl);
       for (int k = 1; k <= T::NST && q - k >= 0; ++k) {
-        mbar_wait(bar(T::KFULL + (q - k) % T::NST), ((q - k) / T::NST) & 1);
-        mbar_wait(bar(T::VFULL + (q - k) % T::NST), ((q - k) / T::NST) & 1);
+        mbar_wait(bar(T::KFULL + (q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
+        mbar_wait(bar(T::VFULL + (q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
       }
     }
     return;
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     for (;;) {
       const int slot = it_seq % T::IR;
       int f = 1;
-      if (lane == 0) f = (!s_abort && mbar_wait(bar(T::IFULL + slot), (it_seq / T::IR) & 1)) ? 1 : 0;
+      if (lane == 0) f = (!s_abort && mbar_wait(bar(T::IFULL + slot), (it_seq / T::IR) & 1, &s_wl)) ? 1 : 0;
       if (!__shfl_sync(FULL, f, 0)) { ok = false; break; }
       const TcDesc d = descs[slot];
       __syncwarp();
@@ -339,13 +343,13 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         bool good = true;
         if (s_side) {
           // Q staged means every earlier item is finished (its epilogue waited for its last P V).
-          good = !s_abort && mbar_wait(bar(T::QBAR), q_ph);
+          good = !s_abort && mbar_wait(bar(T::QBAR), q_ph, &s_wl);
           if (good) tc::fence_after_sync();
           for (int t = 0; t < n && good; ++t) {
             const int qq = q + t, stg = qq % T::NST;
             // The buffer's previous tile: its P (in the buffer) has been read by P V.
-            if (t >= 2) good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1);
-            if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1);
+            if (t >= 2) good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
+            if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1, &s_wl);
             if (!good) break;
             tc::fence_after_sync();
             tc_mma_s<D, BF>(tmem + T::S_COL + (qq & 1) * T::TK, tmem + T::Q_COL, kring + stg * T::TILE);
@@ -355,8 +359,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         } else {
           for (int t = 0; t < n && good; ++t) {
             const int qq = q + t, stg = qq % T::NST;
-            good = !s_abort && mbar_wait(bar(T::PBAR + (qq & 1)), (qq >> 1) & 1);
-            if (good) good = mbar_wait(bar(T::VFULL + stg), (qq / T::NST) & 1);
+            good = !s_abort && mbar_wait(bar(T::PBAR + (qq & 1)), (qq >> 1) & 1, &s_wl);
+            if (good) good = mbar_wait(bar(T::VFULL + stg), (qq / T::NST) & 1, &s_wl);
             if (!good) break;
             tc::fence_after_sync();
             tc_mma_o<D, BF>(tmem + T::O_COL, tmem + T::S_COL + (qq & 1) * T::TK, vring + stg * T::TILE, t > 0);
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       if (!ok) report(a.status, PKV_DEV_TIMEOUT);
       // Every MMA this thread issued has completed before tensor memory is released.
       tc::commit(bar(T::FIN));
-      mbar_wait(bar(T::FIN), 0);
+      mbar_wait(bar(T::FIN), 0, &s_wl);
       tc::fence_before_sync();
       mbar_arrive(bar(T::END), 1);
     }
@@ -399,7 +403,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     float* buf = xchg + (xc & 1) * 2 * T::ROWS;
     buf[hf * T::ROWS + r] = mine;
     mbar_arrive(bar(T::XBAR + (xc & 1)), 1);
-    const bool done = warp_wait(bar(T::XBAR + (xc & 1)), (xc >> 1) & 1);
+    const bool done = warp_wait(bar(T::XBAR + (xc & 1)), (xc >> 1) & 1, &s_wl);
     other = buf[(hf ^ 1) * T::ROWS + r];
     ++xc;
     return done;
@@ -407,7 +411,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   for (;;) {
     const int slot = it_seq % T::IR;
     bool go = __all_sync(FULL, ok && !s_abort);
-    if (go) go = warp_wait(bar(T::IFULL + slot), (it_seq / T::IR) & 1);
+    if (go) go = warp_wait(bar(T::IFULL + slot), (it_seq / T::IR) & 1, &s_wl);
     if (!go) { ok = false; break; }
     const TcDesc d = descs[slot];
     __syncwarp();
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     for (int t = 0; t < ntiles; ++t) {
       const int qq = q + t, stg = qq % T::NST, sb = qq & 1;
       go = __all_sync(FULL, ok && !s_abort);
-      if (go) go = warp_wait(bar(T::SBAR + sb), (qq >> 1) & 1);
+      if (go) go = warp_wait(bar(T::SBAR + sb), (qq >> 1) & 1, &s_wl);
       if (!go) { ok = false; continue; }
       tc::fence_after_sync();
       float s[T::HALF];
@@ -486,7 +490,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       l_run += acc[0].x + acc[0].y;
       if (t == ntiles - 1 && last_valid < T::TK) {
         // Keys past the item's end: zero their V rows before P V reads them (0 * NaN would leak).
-        if (warp_wait(bar(T::VFULL + stg), (qq / T::NST) & 1)) {
+        if (warp_wait(bar(T::VFULL + stg), (qq / T::NST) & 1, &s_wl)) {
           const uint32_t vt = vring + stg * T::TILE;
           for (int x = stid; x < (T::TK - last_valid) * T::HALVES * 8; x += T::SM_THREADS) {
             const int row = last_valid + x / (T::HALVES * 8), h = (x / 8) % T::HALVES, ch = x % 8;
@@ -498,7 +502,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       }
       if (__any_sync(FULL, rescale)) {
         // O must hold the previous tile's P V before it is rescaled (t > 0 here).
-        if (!warp_wait(bar(T::OBAR + ((qq - 1) & 1)), ((qq - 1) >> 1) & 1)) { ok = false; continue; }
+        if (!warp_wait(bar(T::OBAR + ((qq - 1) & 1)), ((qq - 1) >> 1) & 1, &s_wl)) { ok = false; continue; }
         tc::fence_after_sync();
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
@@ -527,7 +531,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     go = __all_sync(FULL, ok);
     float l_other = 0.f;
     if (go) go = exchange(l_run, l_other);
-    if (go) go = warp_wait(bar(T::OBAR + ((q + ntiles - 1) & 1)), ((q + ntiles - 1) >> 1) & 1);
+    if (go) go = warp_wait(bar(T::OBAR + ((q + ntiles - 1) & 1)), ((q + ntiles - 1) >> 1) & 1, &s_wl);
     if (go) {
       tc::fence_after_sync();
       const float l = l_run + l_other;
@@ -581,7 +585,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   __syncwarp();
   if (lane == 0) mbar_arrive(bar(T::END), 1);
   if (warp == 0) {
-    if (lane == 0 && !mbar_wait(bar(T::END), 0)) mbar_wait(bar(T::END), 0);
+    if (lane == 0 && !mbar_wait(bar(T::END), 0, &s_wl)) mbar_wait(bar(T::END), 0, &s_wl);
     __syncwarp();
     tc::fence_after_sync();
     tc::dealloc(tmem, T::TMEM_COLS);

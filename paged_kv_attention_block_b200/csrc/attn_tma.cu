@@ -461,6 +461,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
   volatile int* s_ids = reinterpret_cast<volatile int*>(base_ptr + T::NST * T::STAGE_BYTES + T::MERGE_BYTES +
                                                         T::BAR_BYTES + T::DESC_BYTES);
   __shared__ volatile int s_abort;
+  __shared__ long long s_wl;  // SM cycles any one wait may take
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -474,6 +475,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     }
     mbar_init(merge_bar, 128);
     s_abort = 0;
+    s_wl = a.wait_limit;
     fence_mbar_init();
   }
   __syncthreads();
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     for (;;) {
       const int slot = it_seq % T::IR;
       int flag = 1;
-      if (lane == 0) flag = mbar_wait(iempty_bar(slot), ((it_seq / T::IR) & 1) ^ 1) ? 1 : 0;
+      if (lane == 0) flag = mbar_wait(iempty_bar(slot), ((it_seq / T::IR) & 1) ^ 1, &s_wl) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, flag, 0)) { ok = false; break; }
       const int idx = __shfl_sync(0xffffffffu, next_idx, 0);
       ItemDesc& d = descs[slot];
@@ -534,6 +536,8 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       }
       ++it_seq;
       if (ntiles == 0) continue;
+      // Test switch: publish the item but load none of its tiles, so every consumer wait runs out.
+      if (a.debug_flags & PKV_DEBUG_WITHHOLD_LOADS) continue;
       const int32_t* bt_row = a.block_tables + int64_t(it.seq) * a.max_blocks;
       const int first_blk = it.k_begin >> a.log2_block;
       const int nblk_item = ((it.k_end - 1) >> a.log2_block) - first_blk + 1;
@@ -549,7 +553,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             const int rel = (key0 >> a.log2_block) - first_blk - chunk;
             if (rel >= 32) break;
             const int stg = q % T::NST;
-            if (s_abort || !mbar_wait(empty_bar(stg), ((q / T::NST) & 1) ^ 1)) { flag = 0; break; }
+            if (s_abort || !mbar_wait(empty_bar(stg), ((q / T::NST) & 1) ^ 1, &s_wl)) { flag = 0; break; }
             const uint32_t sdst = stages + stg * T::STAGE_BYTES;
             if constexpr (T::FP4) {
               // Codes through `tmap`, block scales through `smap` (16-byte rows of two slots).
@@ -621,7 +625,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;
       // Let loads already issued land before the CTA's shared memory goes away.
-      for (int k = 1; k <= T::NST && q - k >= 0; ++k) mbar_wait(full_bar((q - k) % T::NST), ((q - k) / T::NST) & 1);
+      for (int k = 1; k <= T::NST && q - k >= 0; ++k) mbar_wait(full_bar((q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
     }
     return;
   }
@@ -634,7 +638,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
   bool ok = true;
   for (;;) {
     const int slot = it_seq % T::IR;
-    if (s_abort || !mbar_wait(ifull_bar(slot), (it_seq / T::IR) & 1)) { ok = false; break; }
+    if (s_abort || !mbar_wait(ifull_bar(slot), (it_seq / T::IR) & 1, &s_wl)) { ok = false; break; }
     const ItemDesc d = descs[slot];
     __syncwarp();
     if (lane == 0) mbar_arrive(iempty_bar(slot), 1);
@@ -684,7 +688,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
           // rounding of the merge) does not depend on which items this CTA ran before.
           const int qq = q + t;
           const int stg = qq % T::NST;
-          if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1)) { ok = false; continue; }
+          if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1, &s_wl)) { ok = false; continue; }
           const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::V_OFF;
           if (t == ntiles - 1 && last_valid < T::TK) {
             if constexpr (T::FP4) zero_v_tail_fp4<T::TK, T::SCALE_ROW>(vb, kb + T::VS_OFF, last_valid, lane);
@@ -735,7 +739,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
         else run(std::integral_constant<int, 2>{});
       }
       mbar_arrive(merge_bar, 1);
-      if (!mbar_wait(merge_bar, merge_phase)) ok = false;
+      if (!mbar_wait(merge_bar, merge_phase, &s_wl)) ok = false;
       merge_phase ^= 1;
       for (int x = tid; x < R * D; x += 128) {
         const int r = x / D, dd = x % D;
@@ -762,7 +766,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
         }
       }
       mbar_arrive(merge_bar, 1);
-      if (!mbar_wait(merge_bar, merge_phase)) ok = false;
+      if (!mbar_wait(merge_bar, merge_phase, &s_wl)) ok = false;
       merge_phase ^= 1;
     } else if constexpr (KV == KV_E4M3) {
       // ---- prefill tile (fp8 pools; 16-bit pools send these to the tcgen05 kernel):
@@ -787,7 +791,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       for (int t = 0; t < ntiles; ++t) {
         const int qq = q + t;
         const int stg = qq % T::NST;
-        if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1)) { ok = false; continue; }
+        if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1, &s_wl)) { ok = false; continue; }
         const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::TK * 128;
         if (t == ntiles - 1 && last_valid < T::TK) {
           zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);  // each warp writes the same zeros

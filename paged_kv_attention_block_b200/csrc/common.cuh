@@ -223,18 +223,25 @@ PKV_DEVICE bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity: false after about 4e9 SM
-// cycles (1-3 s at B200 clocks); the caller records an error and stops waiting.
-// The deadline uses the SM-local cycle counter, which is cheap to read.
-constexpr long long kWaitLimitCycles = 4000000000ll;
-PKV_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity: false once `limit` SM cycles
+// have passed (by default 4e9: 2.0 s at 1965 MHz, about 3 s at 1.3 GHz); the
+// caller records an error and stops waiting.  The deadline uses the SM-local
+// cycle counter, which is cheap to read.
+PKV_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = PKV_DEFAULT_WAIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
     for (int i = 0; i < 16; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
+}
+// The same wait with the limit read from shared memory (where a kernel keeps its per-launch
+// limit), only once the first try has failed: the hot path holds no register for it.
+PKV_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, const long long* limit_smem) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long limit = *static_cast<const volatile long long*>(limit_smem);
+  return mbar_wait(bar, parity, limit);
 }
 
 // 5-D tiled TMA load into shared memory, completion counted on `bar` (no multicast).

@@ -128,6 +128,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (window < 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: window %d < 0", window);
   if (window > 0 && !req->causal)
     return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: a limited attention window needs causal rows");
+  if (req->wait_limit_kcycles < 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: wait_limit_kcycles < 0");
+  if (req->debug_flags & ~PKV_DEBUG_WITHHOLD_LOADS)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: unknown debug_flags 0x%x", req->debug_flags);
   const int32_t* cu = req->cu_q_lens;
   const int32_t* L = req->seq_lens;
   if (S > 0 && cu[0] != 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: cu_q_lens[0] != 0");
@@ -398,6 +401,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.tc_items_off = uint32_t(tc_items_off);
   h.tc_num_ctas = tc_ctas;
   h.window = window;
+  h.wait_limit_kcycles = req->wait_limit_kcycles;
+  h.debug_flags = req->debug_flags;
   h.n_reduce = info->num_reduce;
   h.n_parts = info->num_parts;
   h.n_part_rows = info->num_partial_rows;

@@ -21,6 +21,9 @@
 #define PKV_FP4_ROWS 8     /* rows per tile on NVFP4 pools (one register tile of query rows) */
 #define PKV_TILE_ROWS_TC 128
 #define PKV_TC_TILE_KEYS 128
+// Limit of every pipeline wait of the attention kernels when the plan gives none, in SM cycles
+// (2.0 s at 1965 MHz, about 3 s at 1.3 GHz).
+#define PKV_DEFAULT_WAIT_CYCLES 4000000000ll
 
 struct PkvPlanHeader {
   uint32_t magic;
@@ -46,7 +49,9 @@ struct PkvPlanHeader {
   uint32_t tc_items_off;
   int32_t tc_num_ctas;   // CTAs planned for the tensor-memory kernel
   int32_t window;        // limited attention window in positions; 0 = none
-  int32_t pad[9];        // header is 128 bytes
+  int32_t wait_limit_kcycles;  // limit on every pipeline wait, thousands of SM cycles; 0 = default
+  int32_t debug_flags;   // PKV_DEBUG_* (0 in normal use)
+  int32_t pad[7];        // header is 128 bytes
 };
 static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 

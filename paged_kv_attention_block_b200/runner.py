@@ -25,11 +25,13 @@ def to_device(x: np.ndarray, dtype: str, device) -> torch.Tensor:
 
 
 class DeviceWorkload:
-    def __init__(self, w: Workload, device="cuda", history: bool = True, seq_chunk_tokens: int = 1 << 21):
+    def __init__(self, w: Workload, device="cuda", history: bool = True, seq_chunk_tokens: int = 1 << 21,
+                 fill_byte: int | None = None):
         self.w = w
         self.device = torch.device(device)
         self.cache = api.Cache.allocate(w.num_blocks, w.num_layers, w.num_kv_heads, w.block_size, w.head_dim,
-                                        w.kv_dtype, device=self.device, k_scale=w.k_scale, v_scale=w.v_scale)
+                                        w.kv_dtype, device=self.device, k_scale=w.k_scale, v_scale=w.v_scale,
+                                        fill_byte=fill_byte)
         self.cache.layer = w.layer
         self.block_tables = torch.from_numpy(w.block_tables).to(self.device)
         self.seq_lens = torch.from_numpy(w.seq_lens).to(self.device)

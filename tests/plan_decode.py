@@ -6,7 +6,8 @@ HEADER = np.dtype([("magic", "<u4"), ("bytes", "<u4"), ("n_items", "<i4"), ("n_r
                    ("num_kv_heads", "<i4"), ("head_dim", "<i4"), ("block_size", "<i4"), ("kv_dtype", "<i4"),
                    ("causal", "<i4"), ("num_ctas", "<i4"), ("n_groups", "<i4"), ("items_off", "<u4"),
                    ("reduce_off", "<u4"), ("parts_off", "<u4"), ("n_tc_items", "<i4"), ("tc_items_off", "<u4"),
-                   ("tc_num_ctas", "<i4"), ("window", "<i4"), ("pad", "<i4", 9)])
+                   ("tc_num_ctas", "<i4"), ("window", "<i4"), ("wait_limit_kcycles", "<i4"), ("debug_flags", "<i4"),
+                   ("pad", "<i4", 7)])
 ITEM = np.dtype([("seq", "<i4"), ("kv_head", "<i4"), ("q_begin", "<i4"), ("n_q", "<i4"), ("k_begin", "<i4"),
                  ("k_end", "<i4"), ("pos0", "<i4"), ("part_row", "<i4")])
 REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("parts_begin", "<i4"),

@@ -39,7 +39,7 @@ def test_exports_match_header(api):
 
 
 def test_version_and_strings(api):
-    assert api._lib.pkv_abi_version() == 1
+    assert api._lib.pkv_abi_version() == 2
     assert api.status_string(0) == "ok" and api.status_string(4) == "buffer too small"
 
 
@@ -282,3 +282,17 @@ def test_plan_avoids_a_tail_round(api):
     two_per_cta = -(-int(dec.seq_lens.sum()) * dec.num_kv_heads // (2 * 296))  # keys, one-row-group weight 1
     auto, fixed = _plan(api, dec), _plan(api, dec, kv_split=-(-two_per_cta // 64) * 64)
     assert torch.equal(auto.buffer[:auto.info["plan_bytes"]], fixed.buffer[:fixed.info["plan_bytes"]])
+
+
+def test_plan_carries_wait_limit_and_debug_flags(api):
+    """The plan header carries the per-launch wait limit and the test switch to the kernels;
+    negative limits and unknown flags are refused."""
+    w = W.llama3_8b_decode_bf16(batch=3, lo=10, hi=500)
+    d = PD.decode(_plan(api, w).buffer)
+    assert d["header"]["wait_limit_kcycles"] == 0 and d["header"]["debug_flags"] == 0
+    d = PD.decode(_plan(api, w, wait_limit_kcycles=200, debug_flags=api.PKV_DEBUG_WITHHOLD_LOADS).buffer)
+    assert d["header"]["wait_limit_kcycles"] == 200 and d["header"]["debug_flags"] == api.PKV_DEBUG_WITHHOLD_LOADS
+    with pytest.raises(api.PkvError):
+        _plan(api, w, wait_limit_kcycles=-1)
+    with pytest.raises(api.PkvError):
+        _plan(api, w, debug_flags=0x2)

@@ -307,6 +307,65 @@ def test_bad_block_id_is_reported_not_faulted(pkv):
     assert int(dw.status.item()) & 0x1
 
 
+STRAY_CASES = {
+    "bf16": lambda: W.build("stray", seed=41, kv_dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                            block_size=64, seq_lens=[1, 63, 65, 700, 2049], q_lens=[1, 1, 1, 30, 1]),
+    "e4m3": lambda: W.build("stray", seed=42, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                            num_kv_heads=8, head_dim=128, block_size=64, seq_lens=[1, 63, 65, 700, 2049],
+                            q_lens=[1, 1, 1, 30, 1]),
+    "nvfp4": lambda: W.build("stray", seed=43, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                             num_kv_heads=8, head_dim=128, block_size=64, seq_lens=[1, 63, 65, 700, 2049],
+                             q_lens=[1, 1, 1, 5, 1]),
+}
+
+
+@pytest.mark.parametrize("kv", list(STRAY_CASES))
+def test_unowned_slots_do_not_reach_the_output(pkv, kv):
+    """Stray reads, for every pool type, including fp8 and NVFP4 whose integer dequantisation turns
+    the NaN sentinel into a finite value: the pool bytes no sequence owns are filled with two
+    different values (0x7F and 0x3C) before the same appends; the outputs of the same plan must be
+    bit-identical, so no byte outside a sequence's slots (tails of partly filled blocks, blocks of
+    other sequences, unused blocks) reaches any output, and the result matches the oracle."""
+    api, runner = pkv
+    w = STRAY_CASES[kv]()
+    outs = []
+    for fill in (0x7F, 0x3C):
+        dw = runner.DeviceWorkload(w, fill_byte=fill)
+        dw.append_new()
+        out = torch.full_like(dw.q, float("nan"))
+        dw.attention(dw.plan(kv_split=64), out=out)
+        torch.cuda.synchronize()
+        assert int(dw.status.item()) == 0
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1]), "a pool byte outside the sequences reached the output"
+    ref, _ = oracle_out(w, oracle_pool(w))
+    assert_close(gpu_out_f64(outs[0]), ref, w.kv_dtype)
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "nvfp4"])
+def test_bad_block_id_in_quantised_pools(pkv, kv):
+    """fp8 and NVFP4 decode tiles: a block id outside the pool inside a sequence's range is
+    reported (PKV_DEV_BAD_BLOCK_ID), its keys read as zeros rather than from any memory, the
+    output stays finite, and every other sequence still matches the oracle."""
+    api, runner = pkv
+    w = STRAY_CASES[kv]()
+    dw = runner.DeviceWorkload(w)
+    dw.append_new()
+    bt = dw.block_tables.clone()
+    bad_seq = 3
+    bt[bad_seq, 5] = w.num_blocks + 77
+    out = torch.full_like(dw.q, float("nan"))
+    api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, bt, dw.plan(), w.softmax_scale, w.causal, out=out,
+                        status=dw.status)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) & 0x1
+    got = gpu_out_f64(out)
+    assert np.isfinite(got).all()
+    ref, _ = oracle_out(w, oracle_pool(w))
+    rows = np.concatenate([np.arange(w.cu_q_lens[s], w.cu_q_lens[s + 1]) for s in range(w.num_seqs) if s != bad_seq])
+    assert_close(got, ref, w.kv_dtype, rows=rows)
+
+
 def test_plan_mismatch_is_reported(pkv):
     api, runner = pkv
     w = W.build("mism", seed=3, kv_dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
@@ -319,6 +378,40 @@ def test_plan_mismatch_is_reported(pkv):
                         status=dw.status)
     torch.cuda.synchronize()
     assert int(dw.status.item()) & 0x4
+
+
+TIMEOUT_CASES = {
+    # decode tiles (TMA-fed kernel), bf16 and fp8 pools
+    "decode_bf16": lambda: W.llama3_8b_decode_bf16(batch=5, lo=100, hi=2000),
+    "decode_fp8": lambda: W.longctx_fp8(batch=2, seq_len=3000),
+    # a prefill chunk (tcgen05 kernel) beside decode rows
+    "mixed_bf16": lambda: W.mixed_bf16(n_decode=3, n_prefill=1, chunk=150, dec_lo=50, dec_hi=900, cached_lo_blocks=1,
+                                       cached_hi_blocks=3),
+}
+
+
+@pytest.mark.parametrize("kind", list(TIMEOUT_CASES))
+def test_wait_timeout_is_reported(pkv, kind):
+    """The bounded waits' timeout path: with PKV_DEBUG_WITHHOLD_LOADS the producers publish the
+    work but load nothing, so with a short wait limit (2e5 SM cycles, about 0.1 ms) every
+    consumer wait runs out; the kernels record PKV_DEV_TIMEOUT, drain, free tensor memory and
+    return.  The context stays usable: a normal launch on the same pool then matches the oracle."""
+    api, runner = pkv
+    w = TIMEOUT_CASES[kind]()
+    dw = runner.DeviceWorkload(w)
+    dw.append_new()
+    plan = dw.plan(num_ctas=16, wait_limit_kcycles=200, debug_flags=api.PKV_DEBUG_WITHHOLD_LOADS)
+    out = torch.zeros_like(dw.q)
+    dw.attention(plan, out=out)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) & 0x10, "PKV_DEV_TIMEOUT not reported"
+    dw.status.zero_()
+    out = torch.full_like(dw.q, float("nan"))
+    dw.attention(dw.plan(num_ctas=16), out=out)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) == 0
+    ref, _ = oracle_out(w, oracle_pool(w))
+    assert_close(gpu_out_f64(out), ref, w.kv_dtype)
 
 
 def test_repeat_launch_is_deterministic(pkv):
