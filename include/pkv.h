@@ -365,7 +365,10 @@ PKV_API pkv_status pkv_stream_read(const void* src, size_t bytes, int32_t mode, 
  * the library holds until the process exits.
  *   - A plan needing more scratch than that returns PKV_ERR_WORKSPACE.
  *   - The first call on a device looks up the array's address on that device;
- *     make it outside any stream capture.
+ *     make it outside any stream capture.  After the device's context changes
+ *     (cudaDeviceReset, a context destroyed and created again) the array may
+ *     move: the next call notices the new context and looks the address up
+ *     again, so make that call outside stream capture as well.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents (the work counters are cleared by each call's plan upload).  Calls that
  *     overlap on the GPU race; order them on one stream.

@@ -341,16 +341,19 @@ def paged_attention(cache: Cache, q: torch.Tensor, cu_q_lens: torch.Tensor, seq_
     if workspace is None:
         workspace = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=q.device)
     c = cache._c()
-    args = (C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens), _ptr(seq_lens), _ptr(block_tables),
-            block_tables.shape[1], seq_lens.shape[0], float(softmax_scale), int(bool(causal)), plan.buffer.data_ptr(),
-            _ptr(out), _ptr(out_lse), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
-    if kernel_events is None:
-        _check(_lib.pkv_paged_attention(*args), "paged_attention")
-    else:
-        handles = [e.cuda_event for e in kernel_events]
-        if not all(handles):
-            raise ValueError("kernel_events: record each event once before use (torch creates CUDA events lazily)")
-        _check(_lib.pkv_paged_attention_timed(*args, *handles), "paged_attention")
+    # The library launches on (and sizes its grids for) the current device: make it q's.
+    with torch.cuda.device(q.device):
+        args = (C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens), _ptr(seq_lens), _ptr(block_tables),
+                block_tables.shape[1], seq_lens.shape[0], float(softmax_scale), int(bool(causal)),
+                plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse), _ptr(workspace), workspace.numel(), _ptr(status),
+                _stream(stream))
+        if kernel_events is None:
+            _check(_lib.pkv_paged_attention(*args), "paged_attention")
+        else:
+            handles = [e.cuda_event for e in kernel_events]
+            if not all(handles):
+                raise ValueError("kernel_events: record each event once before use (torch creates CUDA events lazily)")
+            _check(_lib.pkv_paged_attention_timed(*args, *handles), "paged_attention")
     return out
 
 
@@ -367,11 +370,13 @@ def paged_attention_noalloc(cache: Cache, q: torch.Tensor, cu_q_lens: torch.Tens
     if out is None:
         out = torch.empty_like(q)
     c = cache._c()
-    _check(_lib.pkv_paged_attention_noalloc(C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens),
-                                            _ptr(seq_lens), _ptr(block_tables), block_tables.shape[1],
-                                            seq_lens.shape[0], float(softmax_scale), int(bool(causal)),
-                                            plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse), _ptr(status),
-                                            _stream(stream)), "paged_attention_noalloc")
+    # The built-in scratch array is chosen by the current device: make it q's.
+    with torch.cuda.device(q.device):
+        _check(_lib.pkv_paged_attention_noalloc(C.byref(c), _ptr(q), _dtype_code(q), q.shape[1], _ptr(cu_q_lens),
+                                                _ptr(seq_lens), _ptr(block_tables), block_tables.shape[1],
+                                                seq_lens.shape[0], float(softmax_scale), int(bool(causal)),
+                                                plan.buffer.data_ptr(), _ptr(out), _ptr(out_lse), _ptr(status),
+                                                _stream(stream)), "paged_attention_noalloc")
     return out
 
 

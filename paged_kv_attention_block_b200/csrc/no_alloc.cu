@@ -15,13 +15,18 @@
 //     pkv_paged_attention with a workspace of your own).
 //   * The first call on a device looks up the array's device address on that
 //     device (cudaGetSymbolAddress, with that device current).  Make that first
-//     call outside any stream capture.
+//     call outside any stream capture.  The address is kept per device together
+//     with the identity of the device's current CUDA context; when the context
+//     changes (cudaDeviceReset, or a context destroyed and made again) the
+//     module is loaded anew and the array may move, so the next call looks the
+//     address up again -- that call, too, must be made outside stream capture.
 //   * Every call on a device uses the same array, and the array keeps whatever
 //     the last call left there.  The work counters are cleared by each call's plan
 //     upload; partial states are fully written before they are read.
 //     Calls whose work overlaps on the GPU (other streams, other host threads
 //     without ordering) race on the array: order them on one stream.
 //   * Nothing here allocates or frees memory.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -36,8 +41,34 @@ static __device__ __align__(256) unsigned char pkv_noalloc_scratch[PKV_NOALLOC_S
 namespace {
 std::mutex g_setup_mutex;
 void* g_scratch_ptr[PKV_NOALLOC_MAX_DEVICES] = {};
+unsigned long long g_scratch_ctx[PKV_NOALLOC_MAX_DEVICES] = {};  // context the address belongs to
 
-// Device address of the scratch array on the current device, looked up once per device.
+// Identity of the calling thread's current CUDA context (0 if the driver cannot say): the
+// driver's unique context id, reached through the runtime's driver entry points.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
+
+// Device address of the scratch array on the current device, looked up on the first call per
+// device and again whenever that device's context has changed since.
 pkv_status scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -45,12 +76,14 @@ pkv_status scratch_for_current_device(void** out) {
   if (dev < 0 || dev >= PKV_NOALLOC_MAX_DEVICES)
     return pkv_fail(PKV_ERR_UNSUPPORTED, "paged_attention_noalloc: device %d beyond %d", dev, PKV_NOALLOC_MAX_DEVICES);
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
+  const unsigned long long ctx = g_scratch_ptr[dev] ? current_context_id() : 0;
+  if (!g_scratch_ptr[dev] || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, pkv_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return pkv_fail(PKV_ERR_CUDA, "paged_attention_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();  // the symbol lookup made the context current if needed
   }
   *out = g_scratch_ptr[dev];
   return PKV_OK;

@@ -10,9 +10,6 @@ array holds must be refused before anything is launched.
 This file is collected last so that a run stopping at the first failure has
 already run every other test.
 """
-import ctypes as C
-
-import numpy as np
 import pytest
 import torch
 
@@ -62,16 +59,18 @@ def test_noalloc_matches_workspace_entry(pkv, name, make, opts):
 
 
 def test_noalloc_refuses_oversized_plan(pkv):
-    api, _ = pkv
-    S = 64
-    cu = np.arange(S + 1, dtype=np.int32)
-    lens = np.full(S, 4096, np.int32)
-    plan = api.plan_attention(cu, lens, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=64,
-                              kv_dtype="bf16", max_blocks=64, num_ctas=296, kv_split=64, pin=False)
+    """A plan whose scratch exceeds the built-in array is refused before any launch.  Every
+    argument is a real device buffer of the right shape, so a regression that let the call
+    through would show as a wrong status or output, not as a stray memory access."""
+    api, runner = pkv
+    w = W.llama3_8b_decode_bf16(batch=64, lo=4096, hi=4096)
+    dw = runner.DeviceWorkload(w, history=False)
+    plan = dw.plan(num_ctas=296, kv_split=64)
     assert plan.workspace_bytes > 32 << 20
-    cache = api.Cache.allocate(4, 1, 8, 64, 128, "bf16", device="cuda")
-    c = cache._c()
-    st = api._lib.pkv_paged_attention_noalloc(C.byref(c), 0x1000, api.PKV_BF16, 32, 0x1000, 0x1000, 0x1000, 64, S,
-                                              0.1, 1, plan.buffer.data_ptr(), 0x1000, None, None, None)
-    assert st == 4, api._lib.pkv_last_error()
-    assert b"scratch" in api._lib.pkv_last_error()
+    out = torch.full_like(dw.q, float("nan"))
+    with pytest.raises(api.PkvError) as e:
+        api.paged_attention_noalloc(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, plan, w.softmax_scale,
+                                    w.causal, out=out, status=dw.status)
+    assert e.value.status == 4 and "scratch" in str(e.value)
+    torch.cuda.synchronize()
+    assert int(dw.status.item()) == 0 and torch.isnan(out.float()).all()  # nothing ran
