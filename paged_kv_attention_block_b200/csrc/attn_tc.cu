@@ -216,6 +216,9 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
 
   if (warp == T::PROD_WARP) {
     // ------------------------------------------------------------ producer
+    // Ahead of the decode-tile kernel (PKV_PLAN_TC_FIRST): let it start at once on the SMs this
+    // grid leaves free; it waits for this grid before it reads the partial states written here.
+    if (a.plan_flags & PKV_PLAN_TC_FIRST) pdl_trigger();
     const int total_q = __ldg(a.cu_q_lens + a.num_seqs);
     const int box_rows = ta.box_rows;
     const int lb = a.log2_block;

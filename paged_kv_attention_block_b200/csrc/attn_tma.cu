@@ -627,6 +627,10 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       // Let loads already issued land before the CTA's shared memory goes away.
       for (int k = 1; k <= T::NST && q - k >= 0; ++k) mbar_wait(full_bar((q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
     }
+    // Launched behind the tcgen05 kernel (PKV_PLAN_TC_FIRST), this grid finishes only after it,
+    // so the merge that waits for this grid also sees that kernel's partial states.  (A no-op
+    // when this grid was launched without a programmatic dependency.)
+    if (lane == 0) pdl_wait();
     return;
   }
 
@@ -741,6 +745,10 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       mbar_arrive(merge_bar, 1);
       if (!mbar_wait(merge_bar, merge_phase, &s_wl)) ok = false;
       merge_phase ^= 1;
+      // A decode row of a shared-prefix group also takes the group tile's partial state, which
+      // the tcgen05 kernel ahead of this one (PKV_PLAN_TC_FIRST) writes: wait for it first.
+      const bool group_merge = d.part_row <= -2;
+      if (group_merge) pdl_wait();
       for (int x = tid; x < R * D; x += 128) {
         const int r = x / D, dd = x % D;
         float M = -INFINITY;
@@ -756,11 +764,26 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
           }
         }
         const float inv = lsum > 0.f ? deq_undo<KV>(vscale) / lsum : 0.f;
+        float val = o * inv;
+        float lse2 = lsum > 0.f ? M + __log2f(lsum) : -INFINITY;  // log2 of the row's sum of exp2 scores
+        if (group_merge) {
+          // The shared-prefix group tile's state for this row (natural-log lse): the same merge as
+          // the split merge, M = max, w = 2^(lse - M), o = sum w o / sum w.
+          const int64_t grow = int64_t(-2 - d.part_row) + r;
+          const float lg = a.part_lse[grow] * kLog2e;
+          const float og = a.part_o[grow * D + dd];
+          const float mx = fmaxf(lse2, lg);
+          if (mx != -INFINITY) {
+            const float wo = fast_exp2(lse2 - mx), wg = fast_exp2(lg - mx);
+            val = (wo * val + wg * og) / (wo + wg);
+            lse2 = mx + __log2f(wo + wg);
+          }
+        }
         const int64_t orow = to_part ? int64_t(d.part_row) + r : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
-        if (to_part) a.part_o[orow * D + dd] = o * inv;
-        else store_q_dtype<QBF>(a.out, orow * D + dd, o * inv);
+        if (to_part) a.part_o[orow * D + dd] = val;
+        else store_q_dtype<QBF>(a.out, orow * D + dd, val);
         if (dd == 0) {
-          const float lse = lsum > 0.f ? (M + __log2f(lsum)) * kLn2 : -INFINITY;
+          const float lse = lse2 * kLn2;
           if (to_part) a.part_lse[orow] = lse;
           else if (a.out_lse) a.out_lse[orow] = lse;
         }
@@ -904,6 +927,22 @@ bool make_fp4_maps(const AttnArgs& a, int head_dim, int box_rows, int box_kv, CU
   return r == CUDA_SUCCESS;
 }
 
+// Behind the tcgen05 kernel (PKV_PLAN_TC_FIRST) the decode-tile kernel is a programmatic
+// dependent: its CTAs start on the SMs the tcgen05 kernel leaves free.
+template <int D, int KV, bool QBF>
+cudaError_t launch_tma_grid(const AttnArgs& a, int grid, cudaStream_t st, const CUtensorMap& map,
+                            const CUtensorMap& smap, const TmaArgs& ta) {
+  using T = TmaCfg<D, KV, QBF>;
+  cudaError_t e;
+  if (a.plan_flags & PKV_PLAN_TC_FIRST)
+    e = launch_pdl(attn_tma_kernel<D, KV, QBF>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, smap, ta);
+  else {
+    attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, smap, ta);
+    e = cudaSuccess;
+  }
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int D, int KV, bool QBF>
 cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
   using T = TmaCfg<D, KV, QBF>;
@@ -914,8 +953,7 @@ cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
     const int box_rows = merged ? T::TK : B;
     CUtensorMap smap;
     if (!make_fp4_maps(a, D, box_rows, merged ? 2 : 1, &map, &smap)) return cudaErrorInvalidValue;
-    attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, smap, TmaArgs{a, box_rows, merged ? 1 : 0});
-    return cudaGetLastError();
+    return launch_tma_grid<D, KV, QBF>(a, grid, st, map, smap, TmaArgs{a, box_rows, merged ? 1 : 0});
   }
   const CUtensorMapDataType dt = KV == KV_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : KV == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -924,8 +962,7 @@ cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
   const bool merged = B >= T::TK;
   const int box_rows = merged ? T::TK : B;
   if (!make_pool_map(a, D, T::ELEM, dt, box_rows, merged ? 2 : 1, &map)) return cudaErrorInvalidValue;
-  attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, map, TmaArgs{a, box_rows, merged ? 1 : 0});
-  return cudaGetLastError();
+  return launch_tma_grid<D, KV, QBF>(a, grid, st, map, map, TmaArgs{a, box_rows, merged ? 1 : 0});
 }
 
 template <int D, int KV, bool QBF>

@@ -38,7 +38,8 @@ namespace {
 // keys are split or it belongs to a shared-prefix group, a merge per head).
 struct Piece {
   int32_t seq, q_begin, n_q, k_begin, k_end, pos0;
-  int32_t part0;     // partial row of head 0 (head h: part0 + h * part_stride); -1: final output
+  int32_t part0;     // partial row of head 0 (head h: part0 + h * part_stride); -1: final output;
+                     // <= -2: final output merged with a group's partial rows (the same formula)
   int32_t part_stride;
   uint64_t cost16;   // 16 x keys x max(1, rows / 16)
   bool tc;           // tensor-memory list
@@ -57,6 +58,7 @@ struct Scratch {
   std::vector<int32_t> group_of;
   std::vector<int64_t> member_part;  // per sequence: partial row of head 0 in its group tile
   std::vector<int32_t> member_stride;
+  std::vector<uint8_t> member_tc;    // per sequence: its group tile runs on the tcgen05 kernel
   std::vector<uint64_t> keys, tmp;
   std::vector<double> costs;
 };
@@ -200,7 +202,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (!groups.empty()) {
     sc.member_part.assign(size_t(S), -1);
     sc.member_stride.assign(size_t(S), 0);
+    sc.member_tc.assign(size_t(S), 0);
   }
+  bool tc_first = false;  // some decode item merges a group partial the tcgen05 kernel writes
   // Group tiles: consecutive members packed into tiles of at most QT query tokens; the tile of
   // head h writes its partial rows at part0 + h * n * g.
   for (const Group& G : groups) {
@@ -209,11 +213,12 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       int b = a, n = q_len(a);
       while (b + 1 <= G.last && n + q_len(b + 1) <= QT) n += q_len(++b);
       const int rows = n * g;
+      const bool t = is_tc(rows);
       for (int m = a; m <= b; ++m) {
         sc.member_part[m] = part_rows + int64_t(cu[m] - cu[a]) * g;
         sc.member_stride[m] = rows;
+        sc.member_tc[m] = t;
       }
-      const bool t = is_tc(rows);
       pieces.push_back({G.first, cu[a], n, 0, G.tokens, -1, int32_t(part_rows), rows,
                         uint64_t(G.tokens) * weight16(rows), t});
       part_rows += int64_t(rows) * Hkv;
@@ -351,6 +356,15 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       pieces.push_back({tl.seq, tl.q_begin, tl.n_q, tl.k0, tl.ke, tl.pos0, -1, 0, uint64_t(n) * w16, t});
       continue;
     }
+    if (nseg == 1 && !t && sc.member_tc[tl.seq]) {
+      // A decode-tile member of a group whose tile runs on the tcgen05 kernel: that kernel goes
+      // first, and this item merges the group's partial state into its own in its epilogue and
+      // writes the final rows (part_row -2 - r: merge with the group partial rows r ..).
+      pieces.push_back({tl.seq, tl.q_begin, tl.n_q, tl.k0, tl.ke, tl.pos0, -2 - gp, -sc.member_stride[tl.seq],
+                        uint64_t(n) * w16, t});
+      tc_first = true;
+      continue;
+    }
     Merge mg{tl.q_begin, tl.n_q, gp, gp >= 0 ? sc.member_stride[tl.seq] : 0, int32_t(pieces.size()), nseg};
     // Partial rows of the tile's pieces: head h, piece p at base + (h * nseg + p) * rows.
     const int64_t base = part_rows;
@@ -403,6 +417,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.window = window;
   h.wait_limit_kcycles = req->wait_limit_kcycles;
   h.debug_flags = req->debug_flags;
+  h.flags = tc_first ? PKV_PLAN_TC_FIRST : 0;
   h.n_reduce = info->num_reduce;
   h.n_parts = info->num_parts;
   h.n_part_rows = info->num_partial_rows;
@@ -427,7 +442,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     const Piece& pc = pieces[size_t(sc.keys[i] & 0xFFFFF)];
     for (int hh = 0; hh < Hkv; ++hh)
       *items++ = PkvItem{pc.seq, hh, pc.q_begin, pc.n_q, pc.k_begin, pc.k_end, pc.pos0,
-                         pc.part0 < 0 ? -1 : pc.part0 + hh * pc.part_stride};
+                         pc.part0 == -1 ? -1 : pc.part0 + hh * pc.part_stride};
   }
   // Merges and their part lists, per tile and KV head: the group part first, then the pieces.
   PkvReduce* reds = reinterpret_cast<PkvReduce*>(p + reduce_off);

@@ -7,7 +7,7 @@ HEADER = np.dtype([("magic", "<u4"), ("bytes", "<u4"), ("n_items", "<i4"), ("n_r
                    ("causal", "<i4"), ("num_ctas", "<i4"), ("n_groups", "<i4"), ("items_off", "<u4"),
                    ("reduce_off", "<u4"), ("parts_off", "<u4"), ("n_tc_items", "<i4"), ("tc_items_off", "<u4"),
                    ("tc_num_ctas", "<i4"), ("window", "<i4"), ("wait_limit_kcycles", "<i4"), ("debug_flags", "<i4"),
-                   ("pad", "<i4", 7)])
+                   ("flags", "<i4"), ("pad", "<i4", 6)])
 ITEM = np.dtype([("seq", "<i4"), ("kv_head", "<i4"), ("q_begin", "<i4"), ("n_q", "<i4"), ("k_begin", "<i4"),
                  ("k_end", "<i4"), ("pos0", "<i4"), ("part_row", "<i4")])
 REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("parts_begin", "<i4"),
@@ -64,30 +64,46 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
     def add(tok, kvh, a, b, via):
         seen.setdefault((tok, kvh), []).append((a, b, via))
 
-    direct = items[items["part_row"] < 0]
+    def group_source(p):
+        """The item whose partial rows hold row p, and p's token offset inside it."""
+        for row0, it in by_part.items():
+            if row0 <= p < row0 + it["n_q"] * g:
+                return it, (p - row0) // g
+        raise AssertionError("part row without an item")
+
+    def check_shared_blocks(tok, src):
+        if block_tables is not None and src["seq"] != tok_seq[tok]:
+            # Group tile: the keys it reads must be identical blocks in both tables.
+            s_own, s_src = tok_seq[tok], int(src["seq"])
+            nb = (int(src["k_end"]) + block_size - 1) // block_size
+            assert (block_tables[s_own, :nb] == block_tables[s_src, :nb]).all()
+
+    direct = items[items["part_row"] == -1]
     for it in direct:
         for i in range(it["n_q"]):
             add(int(it["q_begin"]) + i, int(it["kv_head"]), int(it["k_begin"]), int(it["k_end"]), "direct")
+    # Items that merge a group tile's partial rows in their epilogue (after that tile's kernel).
+    merged = items[items["part_row"] <= -2]
+    assert len(merged) == 0 or h["flags"] & 1, "epilogue merges need the tcgen05 kernel first"
+    for it in merged:
+        src, off = group_source(-2 - int(it["part_row"]))
+        assert src["kv_head"] == it["kv_head"] and src["n_q"] * g > 16
+        for i in range(it["n_q"]):
+            tok = int(it["q_begin"]) + i
+            assert int(src["q_begin"]) + off + i == tok
+            add(tok, int(it["kv_head"]), int(src["k_begin"]), int(src["k_end"]), "epilogue")
+            add(tok, int(it["kv_head"]), int(it["k_begin"]), int(it["k_end"]), "epilogue")
+        check_shared_blocks(int(it["q_begin"]), src)
     for r in reds:
         for p in parts[r["parts_begin"]:r["parts_begin"] + r["n_parts"]]:
             # The part is either an item's first row or a row inside a group item.
-            src = None
-            for row0, it in by_part.items():
-                if row0 <= p < row0 + it["n_q"] * g:
-                    src = it
-                    off = (p - row0) // g
-                    break
-            assert src is not None, "part row without an item"
+            src, off = group_source(p)
             assert src["kv_head"] == r["kv_head"]
             for i in range(r["n_q"]):
                 tok = int(r["q_begin"]) + i
                 assert int(src["q_begin"]) + off + i == tok
                 add(tok, int(r["kv_head"]), int(src["k_begin"]), int(src["k_end"]), "part")
-            if block_tables is not None and src["seq"] != tok_seq[int(r["q_begin"])]:
-                # Group tile: the keys it reads must be identical blocks in both tables.
-                s_own, s_src = tok_seq[int(r["q_begin"])], int(src["seq"])
-                nb = (int(src["k_end"]) + block_size - 1) // block_size
-                assert (block_tables[s_own, :nb] == block_tables[s_src, :nb]).all()
+            check_shared_blocks(int(r["q_begin"]), src)
     for tok in range(int(cu_q[-1])):
         s = tok_seq[tok]
         j = tok - int(cu_q[s])

@@ -101,6 +101,26 @@ def test_prefix_reuse_bf16(pkv, cascade):
     w = W.prefix_reuse_bf16(n_req=21, prefix=512, suf_lo=1, suf_hi=300)
     plan, _ = run_case(pkv, w, cascade=cascade)
     assert (plan.info["num_groups"] > 0) == cascade
+    # With the group tiles on the tcgen05 kernel, every member's decode item merges the group's
+    # state in its own epilogue: no merge pass.
+    assert (plan.info["num_reduce"] == 0) == cascade
+
+
+@pytest.mark.parametrize("kv", ["bf16", "f16"])
+@pytest.mark.parametrize("split", [0, 64])
+def test_prefix_reuse_member_paths(pkv, kv, split):
+    """Shared-prefix members on every path: one-token and two-token members (8 and 16 rows, decode
+    tiles that merge the group state in their epilogue, or through the merge pass when their
+    suffix is split) and three-token members (24 rows: tcgen05 tiles merged by the merge pass);
+    Hq 64 / Hkv 8, block 16."""
+    r = np.random.default_rng(23)
+    n = 19
+    q_lens = r.integers(1, 4, size=n)
+    seq_lens = 256 + q_lens + r.integers(0, 200, size=n)
+    w = W.build("members", seed=24, kv_dtype=kv, num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=16,
+                seq_lens=seq_lens, q_lens=q_lens, shared_prefix_tokens=256)
+    plan, _ = run_case(pkv, w, kv_split=split)
+    assert plan.info["num_groups"] >= 1
 
 
 @pytest.mark.parametrize("ctas", [1, 2, 3, 5])
