@@ -415,6 +415,121 @@ PKV_DEVICE void dec_tile(DecState<D, KV, QBF, NR>& st, const DecOffsets<D, KV, Q
   }
 }
 
+// NVFP4 tile, 16 keys at a time: S^T for 16 keys, the online-softmax update, then O^T += V^T P^T
+// for those keys.  The dequantisation roughly triples the instruction count of a tile, so the
+// loop over the tile's 16-key steps is kept rolled: its body stays small enough for the
+// instruction cache (a fully unrolled 64-key tile was stalled on instruction fetch).
+template <int D, bool QBF>
+PKV_DEVICE void dec_tile_fp4(DecState<D, KV_NVFP4, QBF, 1>& st, const DecOffsets<D, KV_NVFP4, QBF>& off, uint32_t kbase,
+                             uint32_t vbase, uint32_t ksc, uint32_t vsc, int key0, int lane, float c, bool masked) {
+  using T = TmaCfg<D, KV_NVFP4, QBF>;
+  constexpr int NKT = T::TK / 16;
+  constexpr int ROW = 64;  // bytes between rows of codes
+  const int g4 = lane >> 2, t4 = lane & 3;
+#pragma unroll 1
+  for (int kt = 0; kt < NKT; ++kt) {
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t kb = kbase + kt * 16 * ROW;
+    {
+      // Block scales of keys g4 and g4 + 8 (eight bytes each: groups 0-3, 4-7); the lane's eight
+      // dims of chunk c lie in group 2c + (t4 >> 1).
+      const uint2 s0 = lds64(ksc + uint32_t(kt * 16 + g4) * 8);
+      const uint2 s1 = lds64(ksc + uint32_t(kt * 16 + g4 + 8) * 8);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        uint32_t r[4];  // key g4 chunk 2p, key g4+8 chunk 2p, key g4 chunk 2p+1, key g4+8 chunk 2p+1
+        ldmatrix_x4(kb + off.k[p], r[0], r[1], r[2], r[3]);
+        const uint32_t w0 = p ? s0.y : s0.x, w1 = p ? s1.y : s1.x;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          // Block scale byte b of keys g4 and g4 + 8 into bytes 1 and 3, as f16x2 (s, s) * 2^7.
+          const uint32_t b = uint32_t(2 * cc + (t4 >> 1));
+          const uint32_t sel = (b << 4) | (b << 12);
+          const uint32_t sg = hmul2(e4m3_b13_f16x2(__byte_perm(w0, 0, sel)), kF16Pow2_15x2);
+          const uint32_t sg8 = hmul2(e4m3_b13_f16x2(__byte_perm(w1, 0, sel)), kF16Pow2_15x2);
+          const uint32_t lo = r[2 * cc], hi = r[2 * cc + 1];
+          const uint32_t k0[4] = {hmul2(e2m1_pair_f16x2<0>(lo), sg), hmul2(e2m1_pair_f16x2<0>(hi), sg8),
+                                  hmul2(e2m1_pair_f16x2<1>(lo), sg), hmul2(e2m1_pair_f16x2<1>(hi), sg8)};
+          const uint32_t k1[4] = {hmul2(e2m1_pair_f16x2<2>(lo), sg), hmul2(e2m1_pair_f16x2<2>(hi), sg8),
+                                  hmul2(e2m1_pair_f16x2<3>(lo), sg), hmul2(e2m1_pair_f16x2<3>(hi), sg8)};
+          const int ks = 2 * (2 * p + cc);
+          mma16816<false>(s4, k0, st.qb[0][ks][0], st.qb[0][ks][1]);
+          mma16816<false>(s4, k1, st.qb[0][ks + 1][0], st.qb[0][ks + 1][1]);
+        }
+      }
+    }
+    if (masked) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = key0 + kt * 16 + g4 + 8 * (e >> 1);
+        if (key >= st.lim[0][e & 1] || key < st.lo[0][e & 1]) s4[e] = -INFINITY;
+      }
+    }
+    // Online softmax over these 16 keys for the lane's two query rows.
+    float alpha[2], mneg[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float x = fmaxf(s4[b], s4[b + 2]);
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+      const float mnew = fmaxf(st.m[0][b], x * c);
+      const float muse = mnew == -INFINITY ? 0.f : mnew;
+      alpha[b] = fast_exp2(st.m[0][b] - muse);
+      st.m[0][b] = mnew;
+      mneg[b] = -muse;
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s4[e] = fast_exp2(fmaf(s4[e], c, mneg[e & 1]));
+      rs[e & 1] += s4[e];
+    }
+    st.l[0][0] = st.l[0][0] * alpha[0] + rs[0];
+    st.l[0][1] = st.l[0][1] * alpha[1] + rs[1];
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        st.acc[0][mt][0] *= alpha[0];
+        st.acc[0][mt][1] *= alpha[1];
+        st.acc[0][mt][2] *= alpha[0];
+        st.acc[0][mt][3] *= alpha[1];
+      }
+    }
+    const uint32_t pb0 = movmatrix_trans(pack_f16x2(s4[0], s4[1]));
+    const uint32_t pb1 = movmatrix_trans(pack_f16x2(s4[2], s4[3]));
+    // O^T += V^T P^T for these keys.  V block scales of keys (2t4, 2t4+1) and (2t4+8, 2t4+9): two
+    // adjacent 8-byte rows each; the lane's dims of chunk c lie in group 2c + (g4 >> 2).
+    const uint32_t vb = vbase + kt * 16 * ROW;
+    const uint4 v0 = lds128(vsc + uint32_t(kt * 16 + 2 * t4) * 8);
+    const uint4 v1 = lds128(vsc + uint32_t(kt * 16 + 8 + 2 * t4) * 8);
+    const uint32_t bA = uint32_t(g4 >> 2), bB = bA + 2;
+    const uint32_t selA = (bA << 4) | ((bA + 4) << 12), selB = (bB << 4) | ((bB + 4) << 12);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      uint32_t x[4];  // keys 0-7 chunk 2p, keys 0-7 chunk 2p+1, keys 8-15 chunk 2p, keys 8-15 chunk 2p+1
+      ldmatrix_x4_trans(vb + off.v[p], x[0], x[1], x[2], x[3]);
+      const uint32_t a0w = p ? v0.y : v0.x, a1w = p ? v0.w : v0.z;  // keys 2t4, 2t4+1
+      const uint32_t b0w = p ? v1.y : v1.x, b1w = p ? v1.w : v1.z;  // keys 2t4+8, 2t4+9
+      // (key 2t, key 2t+1) scale pairs in bytes 1 and 3, as f16x2 * 2^7.
+      const uint32_t sc[4] = {hmul2(e4m3_b13_f16x2(__byte_perm(a0w, a1w, selA)), kF16Pow2_15x2),
+                              hmul2(e4m3_b13_f16x2(__byte_perm(a0w, a1w, selB)), kF16Pow2_15x2),
+                              hmul2(e4m3_b13_f16x2(__byte_perm(b0w, b1w, selA)), kF16Pow2_15x2),
+                              hmul2(e4m3_b13_f16x2(__byte_perm(b0w, b1w, selB)), kF16Pow2_15x2)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // m-tile 4p + i: rows g4 -> dim 64p + 4 g4 + i, rows g4 + 8 -> dim 64p + 32 + 4 g4 + i.
+        uint32_t a[4];
+        a[0] = hmul2(e2m1_pair_f16x2_dyn(x[0], i), sc[0]);
+        a[1] = hmul2(e2m1_pair_f16x2_dyn(x[1], i), sc[1]);
+        a[2] = hmul2(e2m1_pair_f16x2_dyn(x[2], i), sc[2]);
+        a[3] = hmul2(e2m1_pair_f16x2_dyn(x[3], i), sc[3]);
+        mma16816<false>(st.acc[0][4 * p + i], a, pb0, pb1);
+      }
+    }
+  }
+}
+
 // NVFP4: zero V code rows [from, TK) (64 bytes each; the swizzle only permutes chunks within a
 // row) and their block scale rows (D/16 bytes each) of a staged tile.
 template <int TK, int SROW>
@@ -700,8 +815,12 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             fence_proxy_async_smem();
           }
           const int key0 = d.k_begin + t * T::TK;
-          dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, kb + T::KS_OFF, kb + T::VS_OFF, key0, lane, deq_undo<KV>(c),
-                                   key0 + T::TK > lim_min || key0 < lo_max);
+          if constexpr (T::FP4)
+            dec_tile_fp4<D, QBF>(st, offs, kb, vb, kb + T::KS_OFF, kb + T::VS_OFF, key0, lane, deq_undo<KV>(c),
+                                 key0 + T::TK > lim_min || key0 < lo_max);
+          else
+            dec_tile<D, KV, QBF, NR>(st, offs, kb, vb, kb + T::KS_OFF, kb + T::VS_OFF, key0, lane, deq_undo<KV>(c),
+                                     key0 + T::TK > lim_min || key0 < lo_max);
           __syncwarp();
           if (lane == 0) mbar_arrive(empty_bar(stg), 4);
         }

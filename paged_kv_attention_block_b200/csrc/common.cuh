@@ -55,6 +55,11 @@ PKV_DEVICE uint32_t e2m1_pair_f16x2(uint32_t w) {
   const uint32_t x = w << (12 - 4 * I);  // nibble I -> bits 12..15, nibble I+4 -> bits 28..31
   return ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
 }
+// The same for a pair index known only at run time (I in 0..3).
+PKV_DEVICE uint32_t e2m1_pair_f16x2_dyn(uint32_t w, int I) {
+  const uint32_t x = w << (12 - 4 * I);
+  return ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
+}
 constexpr uint32_t kF16Pow2_15x2 = 0x78007800u;  // f16x2 (2^15, 2^15)
 // f16x2 product, round to nearest (exact for the scaled E2M1 and E4M3 values multiplied here).
 PKV_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {

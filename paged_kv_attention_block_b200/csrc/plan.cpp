@@ -25,8 +25,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
-#include <functional>
-#include <queue>
+#include <iterator>
 #include <vector>
 
 #include "internal.h"
@@ -52,6 +51,11 @@ struct Merge {
   int32_t first_piece, n_pieces;      // pieces of this tile (consecutive in the piece list)
 };
 
+struct CostRun {
+  uint64_t cost16;
+  uint32_t count;
+};
+
 struct Scratch {
   std::vector<Piece> pieces;
   std::vector<Merge> merges;
@@ -60,7 +64,8 @@ struct Scratch {
   std::vector<int32_t> member_stride;
   std::vector<uint8_t> member_tc;    // per sequence: its group tile runs on the tcgen05 kernel
   std::vector<uint64_t> keys, tmp;
-  std::vector<double> costs;
+  std::vector<CostRun> runs;                       // tail check: runs of equal-cost items
+  std::vector<uint64_t> loads_a, loads_b, merged;  // tail check: CTA loads
 };
 
 Scratch& scratch() {
@@ -293,11 +298,17 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     };
     const size_t N = count_items(1.0), C = size_t(num_ctas);
     if (N > C && N < 4 * C && (N % C) * 4 < C) {
-      std::vector<double>& costs = sc.costs;
+      // The counter's greedy assignment, simulated over runs of equal-cost items: items come
+      // heaviest first and each goes to the least loaded CTA.  Within a run the loads an item
+      // lands on only grow, so the updated loads form a second ascending queue beside the
+      // untouched ones; a run is O(items) and the two queues are merged between runs.
+      std::vector<CostRun>& runs = sc.runs;
+      std::vector<uint64_t>& A = sc.loads_a;
+      std::vector<uint64_t>& Bq = sc.loads_b;
       auto makespan = [&](double mult) {
-        costs.clear();
+        runs.clear();
         for (size_t i = 0; i < n_group_pieces; ++i)  // shared-prefix group items, never split
-          if (!pieces[i].tc) costs.insert(costs.end(), size_t(Hkv), double(pieces[i].cost16) / 16.0);
+          if (!pieces[i].tc) runs.push_back({pieces[i].cost16, uint32_t(Hkv)});
         int last = -1;
         int32_t m = 0;
         for (const Tile& t : tiles) {
@@ -308,21 +319,28 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
           int32_t nseg;
           int64_t seg;
           split(n, m, PKV_TILE_KEYS, nseg, seg);
-          const double w = double(weight16(rows)) / 16.0;
-          for (int64_t k0 = 0; k0 < n; k0 += seg)
-            costs.insert(costs.end(), size_t(Hkv), double(std::min<int64_t>(n, k0 + seg) - k0) * w);
+          if (nseg == 0) continue;
+          const uint64_t w16 = weight16(rows);
+          if (nseg > 1) runs.push_back({uint64_t(seg) * w16, uint32_t(nseg - 1) * uint32_t(Hkv)});
+          runs.push_back({uint64_t(n - (nseg - 1) * seg) * w16, uint32_t(Hkv)});
         }
-        std::sort(costs.begin(), costs.end(), std::greater<double>());
-        std::priority_queue<double, std::vector<double>, std::greater<double>> load;
-        for (int i = 0; i < num_ctas; ++i) load.push(0.0);
-        double worst = 0.0;
-        for (double c : costs) {
-          const double t = load.top() + c;
-          load.pop();
-          load.push(t);
-          worst = std::max(worst, t);
+        std::sort(runs.begin(), runs.end(), [](const CostRun& x, const CostRun& y) { return x.cost16 > y.cost16; });
+        A.assign(size_t(num_ctas), 0);
+        for (size_t r = 0; r < runs.size();) {
+          const uint64_t c = runs[r].cost16;
+          uint64_t cnt = 0;
+          for (; r < runs.size() && runs[r].cost16 == c; ++r) cnt += runs[r].count;
+          Bq.clear();
+          size_t ia = 0, ib = 0;
+          for (uint64_t k = 0; k < cnt; ++k) {
+            const bool from_a = ia < A.size() && (ib >= Bq.size() || A[ia] <= Bq[ib]);
+            Bq.push_back((from_a ? A[ia++] : Bq[ib++]) + c);
+          }
+          sc.merged.clear();
+          std::merge(A.begin() + long(ia), A.end(), Bq.begin() + long(ib), Bq.end(), std::back_inserter(sc.merged));
+          A.swap(sc.merged);
         }
-        return worst;
+        return A.empty() ? 0.0 : double(A.back());
       };
       double best = makespan(1.0);
       for (double mult : {1.125, 1.25, 1.375, 1.5}) {
