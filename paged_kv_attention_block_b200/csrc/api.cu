@@ -93,14 +93,29 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
   if (h->flags & ~PKV_PLAN_TC_FIRST) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
   // group_merge: decode items may merge a group's partial rows (part_row <= -2) written by the
   // tcgen05 kernel, which then runs first.
-  auto check_items = [&](uint32_t off, int n, int lo, int hi, bool group_merge, const char* what) -> pkv_status {
+  if (h->n_rows < 0 || !inside(h->rows_off, h->n_rows, sizeof(int32_t)))
+    return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan token list out of range");
+  const int32_t* rows_list = reinterpret_cast<const int32_t*>(base + h->rows_off);
+  auto check_items = [&](uint32_t off, int n, int lo, int hi, bool group_merge, bool tc_list,
+                         const char* what) -> pkv_status {
     const PkvItem* items = reinterpret_cast<const PkvItem*>(base + off);
     for (int i = 0; i < n; ++i) {
       const PkvItem& it = items[i];
       const int64_t rows = int64_t(it.n_q) * g;
       const int64_t grow = -2 - int64_t(it.part_row);
+      // Listed query tokens (shared-prefix group tiles, tensor-memory list, partial rows only).
+      const bool listed = it.pos0 <= -2;
+      const int64_t loff = -2 - int64_t(it.pos0);
+      if (listed) {
+        if (!tc_list || it.part_row < 0 || loff + it.n_q > h->n_rows)
+          return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d lists bad tokens", what, i);
+        for (int k = 0; k < it.n_q; ++k) {
+          const int32_t tok = rows_list[loff + k];
+          if (tok < 0 || tok >= h->total_q) return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d lists bad tokens", what, i);
+        }
+      }
       if (it.n_q <= 0 || rows < lo || rows > hi || it.kv_head < 0 || it.kv_head >= hkv || it.q_begin < 0 ||
-          int64_t(it.q_begin) + it.n_q > h->total_q || it.k_begin < 0 || it.k_begin > it.k_end ||
+          (!listed && int64_t(it.q_begin) + it.n_q > h->total_q) || it.k_begin < 0 || it.k_begin > it.k_end ||
           (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows) ||
           (it.part_row <= -2 && (!group_merge || rows > PKV_DECODE_ROWS || grow + rows > h->n_part_rows)))
         return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d out of range", what, i);
@@ -108,8 +123,9 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
     return PKV_OK;
   };
   const bool group_merge = (h->flags & PKV_PLAN_TC_FIRST) && h->n_tc_items > 0;
-  if (pkv_status s = check_items(h->items_off, h->n_items, 1, max_rows, group_merge, "item"); s != PKV_OK) return s;
-  if (pkv_status s = check_items(h->tc_items_off, h->n_tc_items, PKV_DECODE_ROWS + 1, PKV_TILE_ROWS_TC, false,
+  if (pkv_status s = check_items(h->items_off, h->n_items, 1, max_rows, group_merge, false, "item"); s != PKV_OK)
+    return s;
+  if (pkv_status s = check_items(h->tc_items_off, h->n_tc_items, PKV_DECODE_ROWS + 1, PKV_TILE_ROWS_TC, false, true,
                                  "tcgen05 item");
       s != PKV_OK)
     return s;
@@ -188,8 +204,21 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  // One copy uploads the plan and clears the work counters at its end.
-  cudaError_t e = cudaMemcpyAsync(ws + L.plan_off, plan, h->bytes, cudaMemcpyHostToDevice, st);
+  // One copy stages the plan in the workspace and clears the work counters at its end.  A
+  // page-locked plan is read by a kernel straight from host memory (launched as a programmatic
+  // dependent of whatever precedes it, so it overlaps that work, and finishing only after it);
+  // any other plan goes through cudaMemcpyAsync.
+  cudaError_t e;
+  cudaPointerAttributes pa{};
+  const void* plan_dev = nullptr;
+  if (cudaPointerGetAttributes(&pa, plan) == cudaSuccess && pa.type == cudaMemoryTypeHost && pa.devicePointer)
+    plan_dev = pa.devicePointer;
+  else
+    cudaGetLastError();  // a failed query leaves no sticky error; take the copy path
+  if (plan_dev)
+    e = pkv::launch_plan_stage(plan_dev, ws + L.plan_off, h->bytes, st);
+  else
+    e = cudaMemcpyAsync(ws + L.plan_off, plan, h->bytes, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: plan upload: %s", cudaGetErrorString(e));
   const int resident = pkv::resident_ctas(k);  // also sets the kernel's shared-memory limit
   const int tc_resident = h->n_tc_items > 0 ? pkv::resident_ctas(ktc) : 1;
@@ -216,6 +245,7 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   a.g = num_q_heads / c.num_kv_heads;
   a.softmax_scale = softmax_scale;
   a.items = reinterpret_cast<const PkvItem*>(dplan + h->items_off);
+  a.row_tokens = reinterpret_cast<const int32_t*>(dplan + h->rows_off);
   a.n_items = h->n_items;
   a.counter = reinterpret_cast<unsigned int*>(ws + L.counter_off);
   a.part_o = reinterpret_cast<float*>(ws + L.part_o_off);

@@ -23,6 +23,7 @@ struct AttnArgs {
   int32_t max_blocks, num_seqs, hq, g;
   float softmax_scale;
   const PkvItem* items;  // device copy of the plan's items
+  const int32_t* row_tokens;  // device copy of the plan's listed query tokens (group tiles)
   int32_t n_items;
   unsigned int* counter;  // work counter, zeroed before the launch
   float* part_o;          // [n_part_rows][head_dim]
@@ -67,6 +68,10 @@ int resident_ctas(const AttnKernel& k);
 bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataType dt, int box_rows, int box_kv,
                    CUtensorMap* map);
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st);
+// Copy `bytes` (a multiple of 16) of a page-locked host plan, addressed through its device
+// alias, into the workspace (reduce.cu).  Launched as a programmatic dependent; the grid
+// completes only after the work ahead of it on the stream.
+cudaError_t launch_plan_stage(const void* plan_dev, void* dst, uint64_t bytes, cudaStream_t st);
 
 // Launch `kernel` with programmatic stream serialization: it may begin while the
 // kernel ahead of it on the stream is still running (and must call pdl_wait

@@ -108,16 +108,17 @@ PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity, const long long* wl) {
   return __all_sync(0xffffffffu, ok);
 }
 
-// Half hf of row r of the item (query token q_begin + r / g, head kv_head * g +
-// r % g): head dims [hf * D / 2, (hf + 1) * D / 2) into this thread's
-// tensor-memory lane at q_tmem, two 16-bit values per column (the pairs are
+// Half hf of row r of the item (query token q_begin + r / g, or the listed token r / g of a
+// shared-prefix group tile; head kv_head * g + r % g): head dims [hf * D / 2, (hf + 1) * D / 2)
+// into this thread's tensor-memory lane at q_tmem, two 16-bit values per column (the pairs are
 // the row's bytes in memory order).  Rows past R are zero.
 template <int D>
 PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_tmem, int r, int hf) {
   const bool valid = r < R;
+  const int i = valid ? r / a.g : 0;
+  const int64_t token = d.pos0 <= -2 ? int64_t(__ldg(a.row_tokens + (-2 - d.pos0) + i)) : int64_t(d.q_begin) + i;
   const uint4* src = reinterpret_cast<const uint4*>(
-      static_cast<const uint16_t*>(a.q) +
-      ((int64_t(d.q_begin) + (valid ? r / a.g : 0)) * a.hq + d.kv_head * a.g + (valid ? r % a.g : 0)) * D +
+      static_cast<const uint16_t*>(a.q) + (token * a.hq + d.kv_head * a.g + (valid ? r % a.g : 0)) * D +
       hf * (D / 2));
   uint32_t w[D / 4];
 #pragma unroll
@@ -209,6 +210,10 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     s_wl = a.wait_limit;
     fence_mbar_init();
   }
+  // First on the stream after the plan staging (PKV_PLAN_TC_FIRST): nothing that work or the work
+  // before it wrote (the plan, the appended K/V, q) is read before it completes.  Behind the
+  // decode-tile kernel, whose CTAs had waited for it, this grid reads nothing that kernel writes.
+  if (a.plan_flags & PKV_PLAN_TC_FIRST) pdl_wait();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -218,6 +223,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     // ------------------------------------------------------------ producer
     // Ahead of the decode-tile kernel (PKV_PLAN_TC_FIRST): let it start at once on the SMs this
     // grid leaves free; it waits for this grid before it reads the partial states written here.
+    // (This grid itself waited for the plan staging, below the set-up.)
     if (a.plan_flags & PKV_PLAN_TC_FIRST) pdl_trigger();
     const int total_q = __ldg(a.cu_q_lens + a.num_seqs);
     const int box_rows = ta.box_rows;
@@ -255,7 +261,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       it.part_row = __shfl_sync(FULL, field, 7);
       const int rows = it.n_q * a.g;
       bool valid = it.seq >= 0 && it.seq < a.num_seqs && it.kv_head >= 0 && it.kv_head < a.hkv && it.n_q > 0 &&
-                   rows > PKV_DECODE_ROWS && rows <= T::ROWS && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q &&
+                   rows > PKV_DECODE_ROWS && rows <= T::ROWS && it.q_begin >= 0 &&
+                   (it.pos0 <= -2 || it.q_begin + it.n_q <= total_q) &&  // listed tokens: checked on the host
                    it.k_begin >= 0 && it.k_begin < it.k_end && (it.k_begin % box_rows) == 0;
       if (valid) {
         const int L = __ldg(a.seq_lens + it.seq);

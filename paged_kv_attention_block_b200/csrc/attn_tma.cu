@@ -593,6 +593,10 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     s_wl = a.wait_limit;
     fence_mbar_init();
   }
+  // Launched as a programmatic dependent of the plan staging (or of the tcgen05 kernel, which
+  // waited for it): the barriers above are set up while that runs; nothing it or the work before
+  // it wrote (the plan, the appended K/V, q) is read before this.  A no-op otherwise.
+  if (!(a.plan_flags & PKV_PLAN_TC_FIRST)) pdl_wait();
   __syncthreads();
 
   if (warp == 4) {
@@ -1046,19 +1050,15 @@ bool make_fp4_maps(const AttnArgs& a, int head_dim, int box_rows, int box_kv, CU
   return r == CUDA_SUCCESS;
 }
 
-// Behind the tcgen05 kernel (PKV_PLAN_TC_FIRST) the decode-tile kernel is a programmatic
-// dependent: its CTAs start on the SMs the tcgen05 kernel leaves free.
+// The decode-tile kernel is a programmatic dependent of the kernel ahead of it: the plan staging
+// (it waits for that before reading anything), or the tcgen05 kernel (PKV_PLAN_TC_FIRST), whose
+// free SMs its CTAs take at once.
 template <int D, int KV, bool QBF>
 cudaError_t launch_tma_grid(const AttnArgs& a, int grid, cudaStream_t st, const CUtensorMap& map,
                             const CUtensorMap& smap, const TmaArgs& ta) {
   using T = TmaCfg<D, KV, QBF>;
-  cudaError_t e;
-  if (a.plan_flags & PKV_PLAN_TC_FIRST)
-    e = launch_pdl(attn_tma_kernel<D, KV, QBF>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, smap, ta);
-  else {
-    attn_tma_kernel<D, KV, QBF><<<grid, T::THREADS, T::SMEM, st>>>(map, smap, ta);
-    e = cudaSuccess;
-  }
+  const cudaError_t e =
+      launch_pdl(attn_tma_kernel<D, KV, QBF>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, smap, ta);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

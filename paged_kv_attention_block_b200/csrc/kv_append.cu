@@ -117,6 +117,7 @@ PKV_DEVICE const int32_t* stage_cu(const AppendArgs& a, int32_t* s_cu) {
 
 template <int ELEM>
 __global__ void __launch_bounds__(256) kv_append_copy_kernel(AppendArgs a) {
+  pdl_trigger();  // a programmatic dependent (the plan staging) may start now; it waits for this grid
   __shared__ int32_t s_cu[kCuCache + 1];
   const int32_t* cu = stage_cu(a, s_cu);
   constexpr int PER = 16 / ELEM;  // elements per 16-byte chunk
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(256) kv_append_copy_kernel(AppendArgs a) {
 
 template <typename Tin>
 __global__ void __launch_bounds__(256) kv_append_e4m3_kernel(AppendArgs a) {
+  pdl_trigger();  // a programmatic dependent (the plan staging) may start now; it waits for this grid
   __shared__ int32_t s_cu[kCuCache + 1];
   const int32_t* cu = stage_cu(a, s_cu);
   const int row_chunks = a.head_dim / 8;  // 8 values -> 8 bytes
@@ -203,6 +205,7 @@ PKV_DEVICE void load4<__half>(const __half* src, float* x) {
 // lane 4j writes the group's block scale.
 template <typename Tin>
 __global__ void __launch_bounds__(256) kv_append_nvfp4_kernel(AppendArgs a) {
+  pdl_trigger();  // a programmatic dependent (the plan staging) may start now; it waits for this grid
   __shared__ int32_t s_cu[kCuCache + 1];
   const int32_t* cu = stage_cu(a, s_cu);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -63,6 +63,9 @@ struct Scratch {
   std::vector<int64_t> member_part;  // per sequence: partial row of head 0 in its group tile
   std::vector<int32_t> member_stride;
   std::vector<uint8_t> member_tc;    // per sequence: its group tile runs on the tcgen05 kernel
+  std::vector<int32_t> gmembers;     // members of every group, group after group
+  std::vector<int32_t> row_tokens;   // listed query tokens of group tiles
+  std::vector<int32_t> run_seqs, rest_seqs;
   std::vector<uint64_t> keys, tmp;
   std::vector<CostRun> runs;                       // tail check: runs of equal-cost items
   std::vector<uint64_t> loads_a, loads_b, merged;  // tail check: CTA loads
@@ -164,11 +167,19 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   const bool causal = req->causal != 0;
   auto q_len = [&](int s) { return cu[s + 1] - cu[s]; };
 
-  // 1. Shared-prefix groups.
-  struct Group { int first, last, tokens; };
+  // 1. Shared-prefix groups: sequences whose tables begin with the same physical blocks (deep
+  // dive §10: the radix tree hands the same prefix blocks to every request that shares it).  On
+  // 16-bit pools the sharers may lie anywhere in the batch (the batch is packed by request kind,
+  // not by prefix): sequences are bucketed by their first block id and each bucket is grouped
+  // greedily.  A group of consecutive sequences reads its queries as one run of tokens; any other
+  // group lists its query tokens in the plan (tensor-memory tiles only).  Other pools group runs
+  // of consecutive sequences.
+  struct Group { int mbeg, mend, tokens; bool listed; };  // members sc.gmembers[mbeg .. mend)
   std::vector<Group> groups;
   Scratch& sc = scratch();
   sc.group_of.assign(size_t(S), -1);
+  sc.gmembers.clear();
+  sc.row_tokens.clear();
   // A window would cut the shared prefix differently for every member: no groups then.
   if (req->cascade && req->block_tables && S > 1 && window == 0) {
     const int32_t* bt = req->block_tables;
@@ -176,26 +187,76 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     const int min_sh = req->min_shared_tokens > 0 ? req->min_shared_tokens : 256;
     // Blocks of a sequence every query row may see in full.
     auto usable = [&](int t) { return (causal ? L[t] - q_len(t) + 1 : L[t]) / B; };
-    int s = 0;
-    while (s < S) {
-      if (q_len(s) < 1 || q_len(s) > QT) { ++s; continue; }
-      int P = usable(s), t = s + 1;
-      while (t < S && q_len(t) >= 1 && q_len(t) <= QT) {
-        const int lim = std::min(P, usable(t));
-        int c = 0;
-        while (c < lim && bt[s * mb + c] == bt[t * mb + c]) ++c;
-        if (int64_t(c) * B < min_sh) break;
-        P = c;
-        ++t;
+    auto candidate = [&](int t) { return q_len(t) >= 1 && q_len(t) <= QT && int64_t(usable(t)) * B >= min_sh; };
+    auto common = [&](int a, int b, int lim) {
+      int c = 0;
+      while (c < lim && bt[a * mb + c] == bt[b * mb + c]) ++c;
+      return c;
+    };
+    if (!tc) {
+      int s = 0;
+      while (s < S) {
+        if (q_len(s) < 1 || q_len(s) > QT) { ++s; continue; }
+        int P = usable(s), t = s + 1;
+        while (t < S && q_len(t) >= 1 && q_len(t) <= QT) {
+          const int c = common(s, t, std::min(P, usable(t)));
+          if (int64_t(c) * B < min_sh) break;
+          P = c;
+          ++t;
+        }
+        if (t - s >= 2 && int64_t(P) * B >= min_sh) {
+          const int mbeg = int(sc.gmembers.size());
+          for (int m = s; m < t; ++m) sc.gmembers.push_back(m);
+          groups.push_back({mbeg, int(sc.gmembers.size()), P * B, false});
+          s = t;
+        } else {
+          ++s;
+        }
       }
-      if (t - s >= 2 && int64_t(P) * B >= min_sh) {
-        for (int m = s; m < t; ++m) sc.group_of[m] = int(groups.size());
-        groups.push_back({s, t - 1, P * B});
-        s = t;
-      } else {
-        ++s;
+    } else {
+      // Candidates ordered by (first block id, index); each run of one first block is grouped
+      // greedily around its first member, the rest of the run trying again.
+      std::vector<uint64_t>& keyed = sc.keys;
+      keyed.clear();
+      for (int t = 0; t < S; ++t)
+        if (candidate(t)) keyed.push_back((uint64_t(uint32_t(bt[t * mb])) << 32) | uint32_t(t));
+      std::sort(keyed.begin(), keyed.end());
+      std::vector<int32_t>& run = sc.run_seqs;
+      std::vector<int32_t>& rest = sc.rest_seqs;
+      for (size_t i = 0; i < keyed.size();) {
+        size_t j = i;
+        run.clear();
+        while (j < keyed.size() && (keyed[j] >> 32) == (keyed[i] >> 32)) run.push_back(int32_t(keyed[j++] & 0xFFFFFFFFu));
+        i = j;
+        while (run.size() >= 2) {
+          const int s0 = run[0];
+          int P = usable(s0);
+          const int mbeg = int(sc.gmembers.size());
+          sc.gmembers.push_back(s0);
+          rest.clear();
+          for (size_t k = 1; k < run.size(); ++k) {
+            const int t = run[k];
+            const int c = common(s0, t, std::min(P, usable(t)));
+            if (int64_t(c) * B >= min_sh) {
+              P = c;
+              sc.gmembers.push_back(t);
+            } else {
+              rest.push_back(t);
+            }
+          }
+          const int mend = int(sc.gmembers.size());
+          if (mend - mbeg >= 2) {
+            const bool consecutive = sc.gmembers[mend - 1] - sc.gmembers[mbeg] == mend - mbeg - 1;
+            groups.push_back({mbeg, mend, P * B, !consecutive});
+          } else {
+            sc.gmembers.resize(size_t(mbeg));
+          }
+          run.swap(rest);
+        }
       }
     }
+    for (size_t gi = 0; gi < groups.size(); ++gi)
+      for (int k = groups[gi].mbeg; k < groups[gi].mend; ++k) sc.group_of[sc.gmembers[k]] = int(gi);
   }
 
   std::vector<Piece>& pieces = sc.pieces;
@@ -210,26 +271,46 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     sc.member_tc.assign(size_t(S), 0);
   }
   bool tc_first = false;  // some decode item merges a group partial the tcgen05 kernel writes
-  // Group tiles: consecutive members packed into tiles of at most QT query tokens; the tile of
-  // head h writes its partial rows at part0 + h * n * g.
+  int n_groups = 0;
+  // Group tiles: members packed into tiles of at most QT query tokens; the tile of head h writes
+  // its partial rows at part0 + h * n * g.  A listed group keeps only tiles of more than 16 rows
+  // (tensor-memory tiles); members of a smaller tile leave the group and read their prefix
+  // themselves.
   for (const Group& G : groups) {
-    int a = G.first;
-    while (a <= G.last) {
-      int b = a, n = q_len(a);
-      while (b + 1 <= G.last && n + q_len(b + 1) <= QT) n += q_len(++b);
+    const int32_t* gm = sc.gmembers.data();
+    int a = G.mbeg;
+    bool any = false;
+    while (a < G.mend) {
+      int b = a, n = q_len(gm[a]);
+      while (b + 1 < G.mend && n + q_len(gm[b + 1]) <= QT) n += q_len(gm[++b]);
       const int rows = n * g;
       const bool t = is_tc(rows);
-      for (int m = a; m <= b; ++m) {
-        sc.member_part[m] = part_rows + int64_t(cu[m] - cu[a]) * g;
-        sc.member_stride[m] = rows;
-        sc.member_tc[m] = t;
+      if (G.listed && !t) {
+        for (int m = a; m <= b; ++m) sc.group_of[gm[m]] = -1;
+        a = b + 1;
+        continue;
       }
-      pieces.push_back({G.first, cu[a], n, 0, G.tokens, -1, int32_t(part_rows), rows,
+      int32_t pos0 = -1;  // -2 - offset: the tile's query tokens are listed at row_tokens[offset ..]
+      if (G.listed) {
+        pos0 = -2 - int32_t(sc.row_tokens.size());
+        for (int m = a; m <= b; ++m)
+          for (int tok = cu[gm[m]]; tok < cu[gm[m] + 1]; ++tok) sc.row_tokens.push_back(tok);
+      }
+      int off = 0;  // the member's first token within the tile
+      for (int m = a; m <= b; ++m) {
+        sc.member_part[gm[m]] = part_rows + int64_t(off) * g;
+        sc.member_stride[gm[m]] = rows;
+        sc.member_tc[gm[m]] = t;
+        off += q_len(gm[m]);
+      }
+      pieces.push_back({gm[a], cu[gm[a]], n, 0, G.tokens, pos0, int32_t(part_rows), rows,
                         uint64_t(G.tokens) * weight16(rows), t});
       part_rows += int64_t(rows) * Hkv;
       total_cost[t] += double(G.tokens) * double(weight16(rows)) / 16.0 * Hkv;
+      any = true;
       a = b + 1;
     }
+    n_groups += any ? 1 : 0;
   }
   const size_t n_group_pieces = pieces.size();
 
@@ -410,7 +491,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   const uint64_t tc_items_off = items_off + uint64_t(n_items - n_tc) * sizeof(PkvItem);
   const uint64_t reduce_off = items_off + uint64_t(n_items) * sizeof(PkvItem);
   const uint64_t parts_off = reduce_off + uint64_t(n_reduce) * sizeof(PkvReduce);
-  const uint64_t bytes = pkv_plan_bytes(parts_off + uint64_t(n_parts) * sizeof(int32_t));
+  const uint64_t rows_off = parts_off + uint64_t(n_parts) * sizeof(int32_t);
+  const uint64_t bytes = pkv_plan_bytes(rows_off + sc.row_tokens.size() * sizeof(int32_t));
   if (bytes > UINT32_MAX) return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: plan too large");
   info->plan_bytes = bytes;
   info->workspace_bytes = pkv_workspace_layout(bytes, part_rows, D).total;
@@ -418,7 +500,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   info->num_reduce = int32_t(n_reduce);
   info->num_parts = int32_t(n_parts);
   info->num_partial_rows = int32_t(part_rows);
-  info->num_groups = int32_t(groups.size());
+  info->num_groups = n_groups;
   info->num_ctas = num_ctas;
   info->num_tc_items = int32_t(n_tc);
   if (!plan) return PKV_OK;
@@ -452,6 +534,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.items_off = uint32_t(items_off);
   h.reduce_off = uint32_t(reduce_off);
   h.parts_off = uint32_t(parts_off);
+  h.rows_off = uint32_t(rows_off);
+  h.n_rows = int32_t(sc.row_tokens.size());
   std::memcpy(p, &h, sizeof(h));
   // Items: pieces heaviest first, each expanded over the KV heads.
   PkvItem* items = reinterpret_cast<PkvItem*>(p + items_off);
@@ -477,8 +561,10 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       *reds++ = PkvReduce{mg.q_begin, mg.n_q, hh, begin, np - begin, {0, 0, 0}};
     }
   }
-  // Zero the tail: alignment padding and the work counters.
-  const uint64_t used = parts_off + uint64_t(np) * sizeof(int32_t);
+  // The listed query tokens of group tiles, then zeros: alignment padding and the work counters.
+  if (!sc.row_tokens.empty())
+    std::memcpy(p + rows_off, sc.row_tokens.data(), sc.row_tokens.size() * sizeof(int32_t));
+  const uint64_t used = rows_off + sc.row_tokens.size() * sizeof(int32_t);
   std::memset(p + used, 0, bytes - used);
   return PKV_OK;
 }

@@ -52,7 +52,9 @@ struct PkvPlanHeader {
   int32_t wait_limit_kcycles;  // limit on every pipeline wait, thousands of SM cycles; 0 = default
   int32_t debug_flags;   // PKV_DEBUG_* (0 in normal use)
   int32_t flags;         // PKV_PLAN_* launch flags
-  int32_t pad[6];        // header is 128 bytes
+  uint32_t rows_off;     // listed query tokens of group tiles (int32 each)
+  int32_t n_rows;
+  int32_t pad[4];        // header is 128 bytes
 };
 static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 
@@ -70,7 +72,9 @@ static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 // partial rows part_row .. part_row + n_q * g - 1; part_row <= -2 (decode-tile
 // items of a PKV_PLAN_TC_FIRST plan) writes the final output after merging, row
 // by row, the partial state at partial rows -2 - part_row .. (a shared-prefix
-// group tile's rows for these queries) into its own.
+// group tile's rows for these queries) into its own.  pos0 <= -2 (shared-prefix group tiles
+// of the tensor-memory list, which are not causal): the tile's query tokens are not the run
+// q_begin .. but listed, token i at row_tokens[-2 - pos0 + i] (q_begin is the first of them).
 struct PkvItem {
   int32_t seq;
   int32_t kv_head;

@@ -85,6 +85,24 @@ __global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
   }
 }
 
+// Plan staging: each thread copies one 16-byte piece of the page-locked host plan (read through
+// its device alias) into the workspace.  The grid may start while the kernel ahead of it runs
+// (programmatic serialization) and waits for that kernel before it finishes, so the attention
+// kernels, which wait for this grid, also see everything written before it on the stream.
+__global__ void __launch_bounds__(256) plan_stage_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                         int n16) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n16) dst[i] = src[i];
+  pdl_wait();
+}
+
+cudaError_t launch_plan_stage(const void* plan_dev, void* dst, uint64_t bytes, cudaStream_t st) {
+  const int n16 = int(bytes / 16);
+  const cudaError_t e = launch_pdl(plan_stage_kernel, dim3((n16 + 255) / 256), dim3(256), 0, st,
+                                   static_cast<const uint4*>(plan_dev), static_cast<uint4*>(dst), n16);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st) {
   if (r.n_reduce <= 0) return cudaSuccess;
   const int grid = std::min(r.n_reduce, 148 * 16);

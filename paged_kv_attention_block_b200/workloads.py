@@ -16,7 +16,10 @@ blocks shared through radix-tree reuse (§10 "跨请求KV复用") and an fp8 KV 
 Recipe (all draws from numpy PCG64 streams keyed by (seed, stream id)):
 
 * lengths, block permutation, queries and every sequence's K/V come from
-  separate streams, so a sequence's K/V can be regenerated alone;
+  separate streams, so a sequence's K/V can be regenerated alone; a shared
+  prefix has a stream of its own (one per prefix group: with
+  ``prefix_groups`` = G, sequence s shares the prefix blocks and values of
+  group s mod G, so sharers need not be neighbours in the batch);
 * values are N(0, 1) float32 times ``data_scale``; bf16/f16 storage rounds
   them to nearest-even through torch's CPU conversion;
 * the physical blocks are a seeded permutation of a pool of
@@ -102,6 +105,7 @@ class Workload:
     k_scale: np.ndarray | None = None  # [num_layers][Hkv] float32, fp8 and NVFP4 only
     v_scale: np.ndarray | None = None
     window: int = 0  # limited attention window (positions); 0 = every cached key
+    prefix_groups: int = 1  # sequence s shares the prefix of group s % prefix_groups
     _kv_cache: dict = field(default_factory=dict, repr=False)
     _q: np.ndarray | None = field(default=None, repr=False)
 
@@ -163,9 +167,12 @@ class Workload:
         P = min(self.shared_prefix_tokens, L)
         parts_k, parts_v = [], []
         if P > 0:
-            if "prefix" not in self._kv_cache:
-                self._kv_cache["prefix"] = self._draw_tokens((_STREAM_PREFIX,), self.shared_prefix_tokens)
-            pk, pv = self._kv_cache["prefix"]
+            grp = s % self.prefix_groups
+            key = "prefix" if grp == 0 else f"prefix{grp}"
+            if key not in self._kv_cache:
+                stream = (_STREAM_PREFIX,) if grp == 0 else (_STREAM_PREFIX, grp)
+                self._kv_cache[key] = self._draw_tokens(stream, self.shared_prefix_tokens)
+            pk, pv = self._kv_cache[key]
             parts_k.append(pk[:P])
             parts_v.append(pv[:P])
         if L - P > 0:
@@ -264,6 +271,7 @@ def build(
     softmax_scale: float | None = None,
     table_slack: int = 0,
     threads: int | None = None,
+    prefix_groups: int = 1,
 ) -> Workload:
     """Assemble a workload; see the module docstring for the recipe."""
     seq_lens = np.asarray(seq_lens, np.int32)
@@ -281,16 +289,18 @@ def build(
     if P_blocks:
         assert all(int(L) >= shared_prefix_tokens for L in seq_lens)
     own = [n - P_blocks for n in nblk]
-    need = P_blocks + sum(own)
+    G = max(1, int(prefix_groups))
+    need = G * P_blocks + sum(own)
     if num_blocks is None:
         num_blocks = max(1, math.ceil(pool_factor * need))
     assert num_blocks >= need
     perm = _rng(seed, _STREAM_PERM).permutation(num_blocks).astype(np.int32)
     max_blocks = max(nblk + [1]) + table_slack
     bt = np.full((S, max_blocks), -1, np.int32)
-    nxt = P_blocks
+    nxt = G * P_blocks
     for s in range(S):
-        bt[s, :P_blocks] = perm[:P_blocks]
+        grp = s % G  # prefix group: its own physical prefix blocks
+        bt[s, :P_blocks] = perm[grp * P_blocks:(grp + 1) * P_blocks]
         bt[s, P_blocks:nblk[s]] = perm[nxt:nxt + own[s]]
         nxt += own[s]
     if softmax_scale is None:
@@ -300,7 +310,7 @@ def build(
         num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B,
         num_blocks=int(num_blocks), num_layers=num_layers, layer=layer, seq_lens=seq_lens,
         q_lens=q_lens, block_tables=bt, softmax_scale=float(softmax_scale), causal=causal, window=int(window),
-        data_scale=data_scale, shared_prefix_tokens=shared_prefix_tokens,
+        data_scale=data_scale, shared_prefix_tokens=shared_prefix_tokens, prefix_groups=G,
     )
     if kv_dtype in ("e4m3", "nvfp4"):
         _calibrate_fp8(w, threads or min(32, os.cpu_count() or 1), 448.0 if kv_dtype == "e4m3" else 6.0 * 448.0)

@@ -7,7 +7,7 @@ HEADER = np.dtype([("magic", "<u4"), ("bytes", "<u4"), ("n_items", "<i4"), ("n_r
                    ("causal", "<i4"), ("num_ctas", "<i4"), ("n_groups", "<i4"), ("items_off", "<u4"),
                    ("reduce_off", "<u4"), ("parts_off", "<u4"), ("n_tc_items", "<i4"), ("tc_items_off", "<u4"),
                    ("tc_num_ctas", "<i4"), ("window", "<i4"), ("wait_limit_kcycles", "<i4"), ("debug_flags", "<i4"),
-                   ("flags", "<i4"), ("pad", "<i4", 6)])
+                   ("flags", "<i4"), ("rows_off", "<u4"), ("n_rows", "<i4"), ("pad", "<i4", 4)])
 ITEM = np.dtype([("seq", "<i4"), ("kv_head", "<i4"), ("q_begin", "<i4"), ("n_q", "<i4"), ("k_begin", "<i4"),
                  ("k_end", "<i4"), ("pos0", "<i4"), ("part_row", "<i4")])
 REDUCE = np.dtype([("q_begin", "<i4"), ("n_q", "<i4"), ("kv_head", "<i4"), ("parts_begin", "<i4"),
@@ -27,7 +27,17 @@ def decode(buf) -> dict:
     items = np.concatenate([reg, tc])
     reds = np.frombuffer(b[h["reduce_off"]:h["reduce_off"] + 32 * h["n_reduce"]].tobytes(), REDUCE)
     parts = np.frombuffer(b[h["parts_off"]:h["parts_off"] + 4 * h["n_parts"]].tobytes(), "<i4")
-    return {"header": h, "items": items, "reg_items": reg, "tc_items": tc, "reduces": reds, "parts": parts}
+    rows = np.frombuffer(b[h["rows_off"]:h["rows_off"] + 4 * h["n_rows"]].tobytes(), "<i4")
+    return {"header": h, "items": items, "reg_items": reg, "tc_items": tc, "reduces": reds, "parts": parts,
+            "rows": rows}
+
+
+def item_tokens(plan: dict, it) -> np.ndarray:
+    """Query tokens of an item: the run q_begin .. q_begin + n_q, or its listed tokens (pos0 <= -2)."""
+    if it["pos0"] <= -2:
+        off = -2 - int(it["pos0"])
+        return plan["rows"][off:off + int(it["n_q"])]
+    return np.arange(int(it["q_begin"]), int(it["q_begin"]) + int(it["n_q"]))
 
 
 def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: int, causal: bool, block_tables=None,
@@ -78,6 +88,14 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
             nb = (int(src["k_end"]) + block_size - 1) // block_size
             assert (block_tables[s_own, :nb] == block_tables[s_src, :nb]).all()
 
+    # Listed items: shared-prefix group tiles of the tensor-memory list, writing partial rows.
+    listed = items[items["pos0"] <= -2]
+    for it in listed:
+        assert it["part_row"] >= 0 and it["n_q"] * g > 16 and it["k_begin"] == 0
+        tok = item_tokens(plan, it)
+        assert len(tok) == it["n_q"] and int(tok[0]) == int(it["q_begin"]) and (np.diff(tok) > 0).all()
+    for it in plan["reg_items"]:
+        assert it["pos0"] > -2
     direct = items[items["part_row"] == -1]
     for it in direct:
         for i in range(it["n_q"]):
@@ -88,9 +106,10 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
     for it in merged:
         src, off = group_source(-2 - int(it["part_row"]))
         assert src["kv_head"] == it["kv_head"] and src["n_q"] * g > 16
+        src_tok = item_tokens(plan, src)
         for i in range(it["n_q"]):
             tok = int(it["q_begin"]) + i
-            assert int(src["q_begin"]) + off + i == tok
+            assert int(src_tok[off + i]) == tok
             add(tok, int(it["kv_head"]), int(src["k_begin"]), int(src["k_end"]), "epilogue")
             add(tok, int(it["kv_head"]), int(it["k_begin"]), int(it["k_end"]), "epilogue")
         check_shared_blocks(int(it["q_begin"]), src)
@@ -99,9 +118,10 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
             # The part is either an item's first row or a row inside a group item.
             src, off = group_source(p)
             assert src["kv_head"] == r["kv_head"]
+            src_tok = item_tokens(plan, src)
             for i in range(r["n_q"]):
                 tok = int(r["q_begin"]) + i
-                assert int(src["q_begin"]) + off + i == tok
+                assert int(src_tok[off + i]) == tok
                 add(tok, int(r["kv_head"]), int(src["k_begin"]), int(src["k_end"]), "part")
             check_shared_blocks(int(r["q_begin"]), src)
     for tok in range(int(cu_q[-1])):

@@ -122,6 +122,13 @@ CASES = [
     ("prefix_split", lambda: W.prefix_reuse_bf16(n_req=11, prefix=256, suf_lo=1, suf_hi=30), {"kv_split": 64}),
     ("prefix_off", lambda: W.prefix_reuse_bf16(n_req=11, prefix=256), {"cascade": False}),
     ("tiny", lambda: W.tiny_fp32(), {}),
+    ("two_prefixes", lambda: W.build("two", seed=24, kv_dtype="bf16", num_q_heads=64, num_kv_heads=8, head_dim=128,
+                                     block_size=16, seq_lens=300 + np.arange(37) * 7, q_lens=[1] * 37,
+                                     shared_prefix_tokens=256, prefix_groups=2), {}),
+    ("two_prefixes_fp8", lambda: W.build("two8", seed=25, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32",
+                                         num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                                         seq_lens=[300] * 9, q_lens=[1] * 9, shared_prefix_tokens=256,
+                                         prefix_groups=2), {}),
 ]
 
 
@@ -296,3 +303,27 @@ def test_plan_carries_wait_limit_and_debug_flags(api):
         _plan(api, w, wait_limit_kcycles=-1)
     with pytest.raises(api.PkvError):
         _plan(api, w, debug_flags=0x2)
+
+
+def test_plan_groups_sharers_that_are_not_neighbours(api):
+    """Two prefixes alternating through the batch (sequence s shares the blocks of prefix s mod 2):
+    on a 16-bit pool both prefixes form a group, whose tensor-memory tiles list their query tokens
+    (a group tile of 16 or fewer rows would have to run on the decode tiles, so the members of such
+    a tile read their prefix themselves); an fp8 pool groups only runs of consecutive sharers, so
+    it finds none here."""
+    w = W.build("two", seed=24, kv_dtype="bf16", num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=16,
+                seq_lens=300 + np.arange(37) * 7, q_lens=[1] * 37, shared_prefix_tokens=256, prefix_groups=2)
+    p = _plan(api, w)
+    d = PD.decode(p.buffer)
+    assert p.info["num_groups"] == 2
+    listed = d["tc_items"][d["tc_items"]["pos0"] <= -2]
+    # 19 and 18 members of one token: a 16-token tile of 128 rows each, the remaining 3 and 2
+    # members (24 and 16 rows) -- the 16-row tile is dropped.
+    assert len(listed) == 3 * w.num_kv_heads
+    for it in listed[::w.num_kv_heads]:
+        tok = PD.item_tokens(d, it)
+        assert (np.diff(tok) == 2).all() and len(set(tok % 2)) == 1
+    w8 = W.build("two8", seed=25, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                 num_kv_heads=8, head_dim=128, block_size=16, seq_lens=[300] * 9, q_lens=[1] * 9,
+                 shared_prefix_tokens=256, prefix_groups=2)
+    assert _plan(api, w8).info["num_groups"] == 0

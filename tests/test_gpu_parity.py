@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import oracle.pkv_oracle as O
+import plan_decode as PD
 from gpu_common import TOL, assert_close, gpu_out_f64, oracle_out, oracle_pool, oracle_pool_bytes
 from paged_kv_attention_block_b200 import workloads as W
 
@@ -101,9 +102,10 @@ def test_prefix_reuse_bf16(pkv, cascade):
     w = W.prefix_reuse_bf16(n_req=21, prefix=512, suf_lo=1, suf_hi=300)
     plan, _ = run_case(pkv, w, cascade=cascade)
     assert (plan.info["num_groups"] > 0) == cascade
-    # With the group tiles on the tcgen05 kernel, every member's decode item merges the group's
-    # state in its own epilogue: no merge pass.
-    assert (plan.info["num_reduce"] == 0) == cascade
+    # With the group tiles on the tcgen05 kernel, the decode item of a member whose suffix is one
+    # piece merges the group's state in its own epilogue (the tcgen05 kernel runs first).
+    items = PD.decode(plan.buffer)["reg_items"]
+    assert ((items["part_row"] <= -2).sum() > 0) == cascade
 
 
 @pytest.mark.parametrize("kv", ["bf16", "f16"])
@@ -121,6 +123,24 @@ def test_prefix_reuse_member_paths(pkv, kv, split):
                 seq_lens=seq_lens, q_lens=q_lens, shared_prefix_tokens=256)
     plan, _ = run_case(pkv, w, kv_split=split)
     assert plan.info["num_groups"] >= 1
+
+
+@pytest.mark.parametrize("kv", ["bf16", "f16"])
+@pytest.mark.parametrize("split", [0, 64])
+def test_prefix_groups_not_neighbours(pkv, kv, split):
+    """Three prefixes alternating through the batch (sequence s shares the prefix blocks of group
+    s mod 3): each group's tensor-memory tiles read their listed query tokens, members of a tile
+    of 16 or fewer rows read their prefix themselves, and one- and two-token members merge the
+    group state in their epilogue or through the merge pass."""
+    r = np.random.default_rng(31)
+    n = 41
+    q_lens = r.integers(1, 3, size=n)
+    seq_lens = 256 + q_lens + r.integers(0, 300, size=n)
+    w = W.build("three", seed=32, kv_dtype=kv, num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=16,
+                seq_lens=seq_lens, q_lens=q_lens, shared_prefix_tokens=256, prefix_groups=3)
+    plan, _ = run_case(pkv, w, kv_split=split)
+    d = PD.decode(plan.buffer)
+    assert plan.info["num_groups"] == 3 and (d["tc_items"]["pos0"] <= -2).any()
 
 
 @pytest.mark.parametrize("ctas", [1, 2, 3, 5])
