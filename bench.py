@@ -412,10 +412,10 @@ def measure(w, args, dev, world, plan_opts, steps):
                                 w.causal, out=out, workspace=ws, status=dw.status)
     torch.cuda.synchronize(dev)
     # The timed steps replay one graph per step (kv_append then paged_attention), one graph per
-    # plan buffer.  A second set splits the step into an append graph and an attention graph
-    # whose library call also records events around the attention kernels: the per-phase and
-    # kernel-only times come from replaying those one step at a time after the timed run (event
-    # record nodes inside the timed graphs would add latency to the step).
+    # plan buffer.  A second set holds the paged_attention call alone, whose library call also
+    # records events around the attention kernels: the call's own time (plan staging, kernels,
+    # merge) and the kernel-only time come from replaying those one at a time after the timed run
+    # (event record nodes inside the timed graphs would add latency to the step).
     g_step = []
     for b in bufs:
         g = torch.cuda.CUDAGraph()
@@ -424,9 +424,6 @@ def measure(w, args, dev, world, plan_opts, steps):
             api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
                                 w.causal, out=out, workspace=ws, status=dw.status)
         g_step.append(g)
-    g_append = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_append, stream=stream):
-        dw.append_new()
     g_attn_ev = []
     for b in bufs:
         g = torch.cuda.CUDAGraph()
@@ -438,8 +435,8 @@ def measure(w, args, dev, world, plan_opts, steps):
     host_plan_s = 0.0
 
     def step(i, evs=None, split=False):
-        """One step; `evs` = (start, after append, end) events; split: the append and attention
-        graphs (the latter with kernel events) instead of the one-graph step."""
+        """One step; `evs` = (start, -, end) events; split: the attention call alone (its graph with
+        kernel events, no append) instead of the one-graph step."""
         nonlocal host_plan_s
         slot = i % 2
         if done[slot] is not None:
@@ -452,9 +449,6 @@ def measure(w, args, dev, world, plan_opts, steps):
             if evs:
                 evs[0].record(stream)
             if split:
-                g_append.replay()
-                if evs:
-                    evs[1].record(stream)
                 g_attn_ev[slot].replay()
             else:
                 g_step[slot].replay()
@@ -490,7 +484,7 @@ def measure(w, args, dev, world, plan_opts, steps):
         step(i, ev_split[i], split=True)
         torch.cuda.synchronize(dev)
         kern_ms.append(kev[0].elapsed_time(kev[1]))
-    attn = float(np.mean([b.elapsed_time(c) for _, b, c in ev_split]))
+    attn = float(np.mean([a_.elapsed_time(c) for a_, _, c in ev_split]))
     kern = float(np.mean(kern_ms))
     ms, attn, kern = max_over_ranks([ms, attn, kern], dev)
     assert int(dw.status.item()) == 0, "device status set during the benchmark"
@@ -500,7 +494,7 @@ def measure(w, args, dev, world, plan_opts, steps):
     for _ in range(200):
         api.plan_attention(w.cu_q_lens, w.seq_lens, buffer=bufs[0].buffer, **plan_kw)
     plan_call_us = (time.perf_counter() - t0) / 200 * 1e6
-    del g_step, g_append, g_attn_ev
+    del g_step, g_attn_ev
     read_ceiling = read_stream_gbs(flush)
     del flush
     e2e = run_e2e(args, w, dw, plan_opts, dev, api, steps)

@@ -90,19 +90,15 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
       !inside(h->parts_off, h->n_parts, sizeof(int32_t)) || h->num_ctas <= 0 || (h->n_tc_items > 0 && h->tc_num_ctas <= 0))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan sections out of range");
   if (h->n_tc_items > 0 && !tc) return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan has tcgen05 items for a pool without that kernel");
-  if (h->flags & ~PKV_PLAN_TC_FIRST) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
-  // group_merge: decode items may merge a group's partial rows (part_row <= -2) written by the
-  // tcgen05 kernel, which then runs first.
+  if (h->flags != 0) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
   if (h->n_rows < 0 || !inside(h->rows_off, h->n_rows, sizeof(int32_t)))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan token list out of range");
   const int32_t* rows_list = reinterpret_cast<const int32_t*>(base + h->rows_off);
-  auto check_items = [&](uint32_t off, int n, int lo, int hi, bool group_merge, bool tc_list,
-                         const char* what) -> pkv_status {
+  auto check_items = [&](uint32_t off, int n, int lo, int hi, bool tc_list, const char* what) -> pkv_status {
     const PkvItem* items = reinterpret_cast<const PkvItem*>(base + off);
     for (int i = 0; i < n; ++i) {
       const PkvItem& it = items[i];
       const int64_t rows = int64_t(it.n_q) * g;
-      const int64_t grow = -2 - int64_t(it.part_row);
       // Listed query tokens (shared-prefix group tiles, tensor-memory list, partial rows only).
       const bool listed = it.pos0 <= -2;
       const int64_t loff = -2 - int64_t(it.pos0);
@@ -116,16 +112,13 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
       }
       if (it.n_q <= 0 || rows < lo || rows > hi || it.kv_head < 0 || it.kv_head >= hkv || it.q_begin < 0 ||
           (!listed && int64_t(it.q_begin) + it.n_q > h->total_q) || it.k_begin < 0 || it.k_begin > it.k_end ||
-          (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows) ||
-          (it.part_row <= -2 && (!group_merge || rows > PKV_DECODE_ROWS || grow + rows > h->n_part_rows)))
+          it.part_row < -1 || (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows))
         return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d out of range", what, i);
     }
     return PKV_OK;
   };
-  const bool group_merge = (h->flags & PKV_PLAN_TC_FIRST) && h->n_tc_items > 0;
-  if (pkv_status s = check_items(h->items_off, h->n_items, 1, max_rows, group_merge, false, "item"); s != PKV_OK)
-    return s;
-  if (pkv_status s = check_items(h->tc_items_off, h->n_tc_items, PKV_DECODE_ROWS + 1, PKV_TILE_ROWS_TC, false, true,
+  if (pkv_status s = check_items(h->items_off, h->n_items, 1, max_rows, false, "item"); s != PKV_OK) return s;
+  if (pkv_status s = check_items(h->tc_items_off, h->n_tc_items, PKV_DECODE_ROWS + 1, PKV_TILE_ROWS_TC, true,
                                  "tcgen05 item");
       s != PKV_OK)
     return s;
@@ -254,7 +247,6 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   a.max_rows = k.max_rows;
   a.window = h->window;
   a.debug_flags = h->debug_flags;
-  a.plan_flags = h->flags;
   a.wait_limit = h->wait_limit_kcycles > 0 ? 1000ll * h->wait_limit_kcycles : PKV_DEFAULT_WAIT_CYCLES;
   if (kernels_begin) {
     e = record_event(static_cast<cudaEvent_t>(kernels_begin), st);
@@ -280,11 +272,10 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
       return pkv_fail(PKV_ERR_CUDA, "paged_attention: tcgen05 launch failed: %s", cudaGetErrorString(le));
     return PKV_OK;
   };
-  // Decode tiles first and the tcgen05 tiles behind them; or, when decode items merge
-  // shared-prefix group states in their epilogues, the tcgen05 kernel first.
-  const bool tc_first = (h->flags & PKV_PLAN_TC_FIRST) != 0;
-  if (pkv_status ls = tc_first ? launch_tc() : launch_reg(); ls != PKV_OK) return ls;
-  if (pkv_status ls = tc_first ? launch_reg() : launch_tc(); ls != PKV_OK) return ls;
+  // Decode tiles first, the tcgen05 tiles behind them (its CTAs take the SMs the decode-tile
+  // kernel frees as it drains).
+  if (pkv_status ls = launch_reg(); ls != PKV_OK) return ls;
+  if (pkv_status ls = launch_tc(); ls != PKV_OK) return ls;
   if (kernels_end) {
     e = record_event(static_cast<cudaEvent_t>(kernels_end), st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));

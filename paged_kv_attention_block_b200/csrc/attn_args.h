@@ -32,7 +32,6 @@ struct AttnArgs {
   int32_t max_rows;       // rows per item this kernel accepts
   int32_t window;         // limited attention window (causal rows see keys pos - window < t <= pos); 0 = none
   int32_t debug_flags;    // PKV_DEBUG_* from the plan (0 in normal use)
-  int32_t plan_flags;     // PKV_PLAN_* from the plan header
   long long wait_limit;   // SM cycles every pipeline wait may take before it gives up
 };
 

@@ -210,10 +210,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     s_wl = a.wait_limit;
     fence_mbar_init();
   }
-  // First on the stream after the plan staging (PKV_PLAN_TC_FIRST): nothing that work or the work
-  // before it wrote (the plan, the appended K/V, q) is read before it completes.  Behind the
-  // decode-tile kernel, whose CTAs had waited for it, this grid reads nothing that kernel writes.
-  if (a.plan_flags & PKV_PLAN_TC_FIRST) pdl_wait();
+  // Behind the decode-tile kernel, whose CTAs had waited for the plan staging (and so for the
+  // work before it) before triggering this launch, this grid reads nothing that kernel writes.
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -221,10 +219,6 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
 
   if (warp == T::PROD_WARP) {
     // ------------------------------------------------------------ producer
-    // Ahead of the decode-tile kernel (PKV_PLAN_TC_FIRST): let it start at once on the SMs this
-    // grid leaves free; it waits for this grid before it reads the partial states written here.
-    // (This grid itself waited for the plan staging, below the set-up.)
-    if (a.plan_flags & PKV_PLAN_TC_FIRST) pdl_trigger();
     const int total_q = __ldg(a.cu_q_lens + a.num_seqs);
     const int box_rows = ta.box_rows;
     const int lb = a.log2_block;

@@ -79,17 +79,24 @@ struct TmaCfg {
   // Four 16 KB stages (64 KB) leave room for two CTAs per SM: twice the producers and consumer
   // warps of one large-ring CTA, which measured faster than a 12-stage ring with one CTA per SM.
   static constexpr int NST = FP4 ? 8 : 4 * std::max(1, std::min(12, (64 * 1024) / STAGE_BYTES) / 4);
-  static constexpr int IR = 4;  // item descriptor slots
+  static constexpr int IR = 2;  // item descriptor slots, each with the item's query rows
+  // Query rows of a decode item, staged in shared memory with the item's descriptor: at most 16
+  // rows (8 for NVFP4) of D 16-bit values.
+  static constexpr int QROWS = FP4 ? PKV_FP4_ROWS : PKV_DECODE_ROWS;
+  static constexpr int QSLOT = QROWS * D * 2;
+  static constexpr int QBUF_BYTES = IR * QSLOT;
   static constexpr int MERGE_BYTES = 4 * 16 * D * 4 + 2 * 4 * 16 * 4;
   static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * IR + 1);
   static constexpr int DESC_BYTES = IR * 64;
   static constexpr int IDS_BYTES = 32 * 4;
-  static constexpr int SMEM = 1024 + NST * STAGE_BYTES + MERGE_BYTES + BAR_BYTES + DESC_BYTES + IDS_BYTES + 16;
+  static constexpr int SMEM =
+      1024 + NST * STAGE_BYTES + MERGE_BYTES + QBUF_BYTES + BAR_BYTES + DESC_BYTES + IDS_BYTES + 16;
   static constexpr int THREADS = 160;
   static_assert(RB == 128 || RB == 256 || (FP4 && D == 128), "TMA path takes 128- or 256-byte rows, or NVFP4 d 128");
   static_assert(STAGE_BYTES % 1024 == 0, "stages keep the swizzle atoms aligned");
   static_assert(NST % 4 == 0, "stage count must be a multiple of the consumer warp count");
-  static_assert(2 * SMEM <= 228 * 1024, "two CTAs per SM");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  static_assert(MERGE_BYTES % 16 == 0 && QSLOT % 16 == 0, "query slots 16-byte aligned for bulk copies");
 };
 
 struct ItemDesc {
@@ -168,16 +175,16 @@ PKV_DEVICE void dec_offsets(DecOffsets<D, KV, QBF>& o, int lane) {
   }
 }
 
+// The query rows of a decode item from its shared-memory slot (row r = token r / g, head r % g of
+// the item's KV head, D 16-bit values each), as the B fragments of S^T = K Q^T.
 template <int D, int KV, bool QBF, int NR>
-PKV_DEVICE void dec_load_q(const AttnArgs& a, const ItemDesc& it, int R, DecState<D, KV, QBF, NR>& st, int g4, int t4) {
+PKV_DEVICE void dec_load_q(const AttnArgs& a, uint32_t qslot, int R, DecState<D, KV, QBF, NR>& st, int g4, int t4) {
   constexpr bool MMA_BF = KV == KV_BF16;
 #pragma unroll
   for (int nr = 0; nr < NR; ++nr) {
     const int r = nr * 8 + g4;
     const bool valid = r < R;
-    const int64_t token = it.q_begin + (valid ? r / a.g : 0);
-    const int head = it.kv_head * a.g + (valid ? r % a.g : 0);
-    const uint16_t* qrow = static_cast<const uint16_t*>(a.q) + (token * a.hq + head) * D;
+    const uint32_t qrow = qslot + uint32_t(valid ? r : 0) * D * 2;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t w0 = 0, w1 = 0;
@@ -185,18 +192,18 @@ PKV_DEVICE void dec_load_q(const AttnArgs& a, const ItemDesc& it, int R, DecStat
         if constexpr (KV == KV_NVFP4) {
           // k-step 2c + h pairs dims (b + 2h, b + 2h + 4) and (b + 2h + 1, b + 2h + 5), b = 32c + 8 t4:
           // the nibble pairs (i, i + 4) of the lane's K word.
-          const uint4 x = *reinterpret_cast<const uint4*>(qrow + 32 * (ks >> 1) + 8 * t4);
+          const uint4 x = lds128(qrow + 2 * (32 * (ks >> 1) + 8 * t4));
           const uint32_t lo = (ks & 1) ? x.y : x.x, hi = (ks & 1) ? x.w : x.z;
           w0 = __byte_perm(lo, hi, 0x5410);
           w1 = __byte_perm(lo, hi, 0x7632);
         } else if constexpr (KV == KV_E4M3) {
           // dims 16 ks + 4 t4 + {0, 2} and + {1, 3}: the byte pairs (0, 2), (1, 3) of the K word.
-          const uint2 x = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * t4);
+          const uint2 x = lds64(qrow + 2 * (16 * ks + 4 * t4));
           w0 = __byte_perm(x.x, x.y, 0x5410);
           w1 = __byte_perm(x.x, x.y, 0x7632);
         } else {
-          w0 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * t4);
-          w1 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * t4);
+          w0 = lds32(qrow + 2 * (16 * ks + 2 * t4));
+          w1 = lds32(qrow + 2 * (16 * ks + 8 + 2 * t4));
         }
         if constexpr (!MMA_BF && QBF) {
           w0 = pack_f16x2(bf16_bits_to_float(uint16_t(w0 & 0xffff)), bf16_bits_to_float(uint16_t(w0 >> 16)));
@@ -566,15 +573,17 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
   float* red_o = reinterpret_cast<float*>(base_ptr + T::NST * T::STAGE_BYTES);
   float* red_m = red_o + 4 * 16 * D;
   float* red_l = red_m + 4 * 16;
-  const uint32_t bars = base + T::NST * T::STAGE_BYTES + T::MERGE_BYTES;
+  const uint32_t qbuf = base + T::NST * T::STAGE_BYTES + T::MERGE_BYTES;  // T::IR query slots
+  const uint32_t bars = qbuf + T::QBUF_BYTES;
   auto full_bar = [&](int i) { return bars + 8 * i; };
   auto empty_bar = [&](int i) { return bars + 8 * (T::NST + i); };
   auto ifull_bar = [&](int i) { return bars + 8 * (2 * T::NST + i); };
   auto iempty_bar = [&](int i) { return bars + 8 * (2 * T::NST + T::IR + i); };
   const uint32_t merge_bar = bars + 8 * (2 * T::NST + 2 * T::IR);
-  ItemDesc* descs = reinterpret_cast<ItemDesc*>(base_ptr + T::NST * T::STAGE_BYTES + T::MERGE_BYTES + T::BAR_BYTES);
+  ItemDesc* descs =
+      reinterpret_cast<ItemDesc*>(base_ptr + T::NST * T::STAGE_BYTES + T::MERGE_BYTES + T::QBUF_BYTES + T::BAR_BYTES);
   volatile int* s_ids = reinterpret_cast<volatile int*>(base_ptr + T::NST * T::STAGE_BYTES + T::MERGE_BYTES +
-                                                        T::BAR_BYTES + T::DESC_BYTES);
+                                                        T::QBUF_BYTES + T::BAR_BYTES + T::DESC_BYTES);
   __shared__ volatile int s_abort;
   __shared__ long long s_wl;  // SM cycles any one wait may take
 
@@ -593,10 +602,10 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     s_wl = a.wait_limit;
     fence_mbar_init();
   }
-  // Launched as a programmatic dependent of the plan staging (or of the tcgen05 kernel, which
-  // waited for it): the barriers above are set up while that runs; nothing it or the work before
-  // it wrote (the plan, the appended K/V, q) is read before this.  A no-op otherwise.
-  if (!(a.plan_flags & PKV_PLAN_TC_FIRST)) pdl_wait();
+  // Launched as a programmatic dependent of the plan staging: the barriers above are set up while
+  // that runs; nothing it or the work before it wrote (the plan, the appended K/V, q) is read
+  // before this.  A no-op when the kernel ahead is not a programmatic primary.
+  pdl_wait();
   __syncthreads();
 
   if (warp == 4) {
@@ -651,7 +660,19 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       if (lane == 0) {
         d.seq = it.seq; d.kv_head = it.kv_head; d.q_begin = it.q_begin; d.n_q = it.n_q; d.k_begin = it.k_begin;
         d.k_end = it.k_end; d.pos0 = it.pos0; d.part_row = it.part_row; d.ntiles = ntiles; d.state = valid ? 0 : 1;
-        mbar_arrive(ifull_bar(slot), 1);
+        const int rows = it.n_q * a.g;
+        if (valid && rows <= T::QROWS) {
+          // A decode item's query rows travel with its descriptor: for each of its tokens the g
+          // heads of the KV head are one contiguous run of g * D 16-bit values; the slot's
+          // barrier completes when they have landed.
+          const uint32_t run = uint32_t(a.g) * D * 2;
+          mbar_arrive_expect_tx(ifull_bar(slot), run * uint32_t(it.n_q));
+          const uint16_t* qsrc = static_cast<const uint16_t*>(a.q) + (int64_t(it.q_begin) * a.hq + it.kv_head * a.g) * D;
+          for (int i = 0; i < it.n_q; ++i)
+            bulk_load_1d(qbuf + slot * T::QSLOT + uint32_t(i) * run, qsrc + int64_t(i) * a.hq * D, run, ifull_bar(slot));
+        } else {
+          mbar_arrive(ifull_bar(slot), 1);
+        }
       }
       ++it_seq;
       if (ntiles == 0) continue;
@@ -743,13 +764,12 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     if (!ok && lane == 0) {
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;
-      // Let loads already issued land before the CTA's shared memory goes away.
+      // Let loads already issued land before the CTA's shared memory goes away: the last tiles
+      // and the query rows of the last published items.
       for (int k = 1; k <= T::NST && q - k >= 0; ++k) mbar_wait(full_bar((q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
+      for (int k = 1; k <= T::IR && it_seq - k >= 0; ++k)
+        mbar_wait(ifull_bar((it_seq - k) % T::IR), ((it_seq - k) / T::IR) & 1, &s_wl);
     }
-    // Launched behind the tcgen05 kernel (PKV_PLAN_TC_FIRST), this grid finishes only after it,
-    // so the merge that waits for this grid also sees that kernel's partial states.  (A no-op
-    // when this grid was launched without a programmatic dependency.)
-    if (lane == 0) pdl_wait();
     return;
   }
 
@@ -763,12 +783,14 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     const int slot = it_seq % T::IR;
     if (s_abort || !mbar_wait(ifull_bar(slot), (it_seq / T::IR) & 1, &s_wl)) { ok = false; break; }
     const ItemDesc d = descs[slot];
+    const int R = d.n_q * a.g;
+    // A decode item's slot also holds its query rows: released once they are in registers.
+    const bool q_staged = d.state == 0 && R <= T::QROWS;
     __syncwarp();
-    if (lane == 0) mbar_arrive(iempty_bar(slot), 1);
+    if (lane == 0 && !q_staged) mbar_arrive(iempty_bar(slot), 1);
     ++it_seq;
     if (d.state == 2) break;
     if (d.state == 1) continue;
-    const int R = d.n_q * a.g;
     const int ntiles = d.ntiles;
     float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
     float vscale = 1.f;
@@ -786,7 +808,9 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       auto run = [&](auto nr_tag) {
         constexpr int NR = decltype(nr_tag)::value;
         DecState<D, KV, QBF, NR> st;
-        dec_load_q<D, KV, QBF, NR>(a, d, R, st, g4, t4);
+        dec_load_q<D, KV, QBF, NR>(a, qbuf + slot * T::QSLOT, R, st, g4, t4);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(iempty_bar(slot), 1);
         int lim_min = d.k_end, lo_max = 0;
 #pragma unroll
         for (int nr = 0; nr < NR; ++nr)
@@ -868,47 +892,55 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       mbar_arrive(merge_bar, 1);
       if (!mbar_wait(merge_bar, merge_phase, &s_wl)) ok = false;
       merge_phase ^= 1;
-      // A decode row of a shared-prefix group also takes the group tile's partial state, which
-      // the tcgen05 kernel ahead of this one (PKV_PLAN_TC_FIRST) writes: wait for it first.
-      const bool group_merge = d.part_row <= -2;
-      if (group_merge) pdl_wait();
-      for (int x = tid; x < R * D; x += 128) {
-        const int r = x / D, dd = x % D;
-        float M = -INFINITY;
+      // Thread t takes row r = t / TPR and DPT consecutive head dims of it (TPR threads per row,
+      // rows rounded up to 4, 8 or 16, at most D / 4 threads per row so that DPT is a multiple of
+      // 4: every float4 and 4-element store is aligned); it computes the row's merge factors
+      // itself, so no further barrier is needed, and moves its dims as float4 reads and vector
+      // stores.  D 128: DPT 4, 8, 16 for R <= 4, 8, 16; D 64: 4, 4, 8.
+      {
+        const int Rp = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
+        const int TPR = min(128 / Rp, D / 4), DPT = D / TPR;
+        const int r = tid / TPR, d0 = (tid % TPR) * DPT;
+        if (r < R) {
+          float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * 16 + r]);
-        float o = 0.f, lsum = 0.f;
-        if (M != -INFINITY) {
+          for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * 16 + r]);
+          float f[4], lsum = 0.f;
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            const float f = fast_exp2(red_m[w * 16 + r] - M);
-            lsum += red_l[w * 16 + r] * f;
-            o += red_o[(w * 16 + r) * D + dd] * f;
+            f[w] = M == -INFINITY ? 0.f : fast_exp2(red_m[w * 16 + r] - M);
+            lsum += red_l[w * 16 + r] * f[w];
           }
-        }
-        const float inv = lsum > 0.f ? deq_undo<KV>(vscale) / lsum : 0.f;
-        float val = o * inv;
-        float lse2 = lsum > 0.f ? M + __log2f(lsum) : -INFINITY;  // log2 of the row's sum of exp2 scores
-        if (group_merge) {
-          // The shared-prefix group tile's state for this row (natural-log lse): the same merge as
-          // the split merge, M = max, w = 2^(lse - M), o = sum w o / sum w.
-          const int64_t grow = int64_t(-2 - d.part_row) + r;
-          const float lg = a.part_lse[grow] * kLog2e;
-          const float og = a.part_o[grow * D + dd];
-          const float mx = fmaxf(lse2, lg);
-          if (mx != -INFINITY) {
-            const float wo = fast_exp2(lse2 - mx), wg = fast_exp2(lg - mx);
-            val = (wo * val + wg * og) / (wo + wg);
-            lse2 = mx + __log2f(wo + wg);
+          const float inv = lsum > 0.f ? deq_undo<KV>(vscale) / lsum : 0.f;
+          const float lse2 = lsum > 0.f ? M + __log2f(lsum) : -INFINITY;  // log2 of the row's sum of exp2 scores
+#pragma unroll
+          for (int w = 0; w < 4; ++w) f[w] *= inv;
+          const int64_t orow = to_part ? int64_t(d.part_row) + r
+                                       : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
+#pragma unroll 1
+          for (int c = 0; c < DPT; c += 4) {
+            float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float4 x = *reinterpret_cast<const float4*>(red_o + (w * 16 + r) * D + d0 + c);
+              o.x = fmaf(x.x, f[w], o.x);
+              o.y = fmaf(x.y, f[w], o.y);
+              o.z = fmaf(x.z, f[w], o.z);
+              o.w = fmaf(x.w, f[w], o.w);
+            }
+            if (to_part) {
+              *reinterpret_cast<float4*>(a.part_o + orow * D + d0 + c) = o;
+            } else {
+              const uint2 pk = QBF ? make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w))
+                                   : make_uint2(pack_f16x2(o.x, o.y), pack_f16x2(o.z, o.w));
+              *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow * D + d0 + c) = pk;
+            }
           }
-        }
-        const int64_t orow = to_part ? int64_t(d.part_row) + r : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
-        if (to_part) a.part_o[orow * D + dd] = val;
-        else store_q_dtype<QBF>(a.out, orow * D + dd, val);
-        if (dd == 0) {
-          const float lse = lse2 * kLn2;
-          if (to_part) a.part_lse[orow] = lse;
-          else if (a.out_lse) a.out_lse[orow] = lse;
+          if (tid % TPR == 0) {
+            const float lse = lse2 * kLn2;
+            if (to_part) a.part_lse[orow] = lse;
+            else if (a.out_lse) a.out_lse[orow] = lse;
+          }
         }
       }
       mbar_arrive(merge_bar, 1);
@@ -1050,9 +1082,8 @@ bool make_fp4_maps(const AttnArgs& a, int head_dim, int box_rows, int box_kv, CU
   return r == CUDA_SUCCESS;
 }
 
-// The decode-tile kernel is a programmatic dependent of the kernel ahead of it: the plan staging
-// (it waits for that before reading anything), or the tcgen05 kernel (PKV_PLAN_TC_FIRST), whose
-// free SMs its CTAs take at once.
+// The decode-tile kernel is a programmatic dependent of the plan staging: its CTAs set up their
+// barriers while that runs, and wait for it before reading anything.
 template <int D, int KV, bool QBF>
 cudaError_t launch_tma_grid(const AttnArgs& a, int grid, cudaStream_t st, const CUtensorMap& map,
                             const CUtensorMap& smap, const TmaArgs& ta) {

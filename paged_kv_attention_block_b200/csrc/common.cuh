@@ -103,6 +103,12 @@ PKV_DEVICE uint4 lds128(uint32_t addr) {
   return v;
 }
 
+PKV_DEVICE uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 PKV_DEVICE uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -247,6 +253,14 @@ PKV_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, const long long* limit_
   if (mbar_try_wait(bar, parity)) return true;
   const long long limit = *static_cast<const volatile long long*>(limit_smem);
   return mbar_wait(bar, parity, limit);
+}
+
+// 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global into
+// shared memory, completion counted on `bar` (no multicast).
+PKV_DEVICE void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // 5-D tiled TMA load into shared memory, completion counted on `bar` (no multicast).

@@ -37,8 +37,7 @@ namespace {
 // keys are split or it belongs to a shared-prefix group, a merge per head).
 struct Piece {
   int32_t seq, q_begin, n_q, k_begin, k_end, pos0;
-  int32_t part0;     // partial row of head 0 (head h: part0 + h * part_stride); -1: final output;
-                     // <= -2: final output merged with a group's partial rows (the same formula)
+  int32_t part0;     // partial row of head 0 (head h: part0 + h * part_stride); -1: final output
   int32_t part_stride;
   uint64_t cost16;   // 16 x keys x max(1, rows / 16)
   bool tc;           // tensor-memory list
@@ -62,7 +61,6 @@ struct Scratch {
   std::vector<int32_t> group_of;
   std::vector<int64_t> member_part;  // per sequence: partial row of head 0 in its group tile
   std::vector<int32_t> member_stride;
-  std::vector<uint8_t> member_tc;    // per sequence: its group tile runs on the tcgen05 kernel
   std::vector<int32_t> gmembers;     // members of every group, group after group
   std::vector<int32_t> row_tokens;   // listed query tokens of group tiles
   std::vector<int32_t> run_seqs, rest_seqs;
@@ -268,9 +266,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (!groups.empty()) {
     sc.member_part.assign(size_t(S), -1);
     sc.member_stride.assign(size_t(S), 0);
-    sc.member_tc.assign(size_t(S), 0);
   }
-  bool tc_first = false;  // some decode item merges a group partial the tcgen05 kernel writes
   int n_groups = 0;
   // Group tiles: members packed into tiles of at most QT query tokens; the tile of head h writes
   // its partial rows at part0 + h * n * g.  A listed group keeps only tiles of more than 16 rows
@@ -300,7 +296,6 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       for (int m = a; m <= b; ++m) {
         sc.member_part[gm[m]] = part_rows + int64_t(off) * g;
         sc.member_stride[gm[m]] = rows;
-        sc.member_tc[gm[m]] = t;
         off += q_len(gm[m]);
       }
       pieces.push_back({gm[a], cu[gm[a]], n, 0, G.tokens, pos0, int32_t(part_rows), rows,
@@ -455,15 +450,6 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       pieces.push_back({tl.seq, tl.q_begin, tl.n_q, tl.k0, tl.ke, tl.pos0, -1, 0, uint64_t(n) * w16, t});
       continue;
     }
-    if (nseg == 1 && !t && sc.member_tc[tl.seq]) {
-      // A decode-tile member of a group whose tile runs on the tcgen05 kernel: that kernel goes
-      // first, and this item merges the group's partial state into its own in its epilogue and
-      // writes the final rows (part_row -2 - r: merge with the group partial rows r ..).
-      pieces.push_back({tl.seq, tl.q_begin, tl.n_q, tl.k0, tl.ke, tl.pos0, -2 - gp, -sc.member_stride[tl.seq],
-                        uint64_t(n) * w16, t});
-      tc_first = true;
-      continue;
-    }
     Merge mg{tl.q_begin, tl.n_q, gp, gp >= 0 ? sc.member_stride[tl.seq] : 0, int32_t(pieces.size()), nseg};
     // Partial rows of the tile's pieces: head h, piece p at base + (h * nseg + p) * rows.
     const int64_t base = part_rows;
@@ -517,7 +503,6 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.window = window;
   h.wait_limit_kcycles = req->wait_limit_kcycles;
   h.debug_flags = req->debug_flags;
-  h.flags = tc_first ? PKV_PLAN_TC_FIRST : 0;
   h.n_reduce = info->num_reduce;
   h.n_parts = info->num_parts;
   h.n_part_rows = info->num_partial_rows;

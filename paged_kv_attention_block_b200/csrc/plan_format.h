@@ -51,28 +51,20 @@ struct PkvPlanHeader {
   int32_t window;        // limited attention window in positions; 0 = none
   int32_t wait_limit_kcycles;  // limit on every pipeline wait, thousands of SM cycles; 0 = default
   int32_t debug_flags;   // PKV_DEBUG_* (0 in normal use)
-  int32_t flags;         // PKV_PLAN_* launch flags
+  int32_t flags;         // reserved (0)
   uint32_t rows_off;     // listed query tokens of group tiles (int32 each)
   int32_t n_rows;
   int32_t pad[4];        // header is 128 bytes
 };
 static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 
-// Launch flag: the tcgen05 kernel runs first (it writes shared-prefix group partial states that
-// decode items of the other kernel merge in their epilogues); the decode-tile kernel follows as a
-// programmatic dependent and waits for it before reading those states.
-#define PKV_PLAN_TC_FIRST 0x1
-
 // One CTA-sized piece of work: rows [q_begin, q_begin + n_q) x the g query
 // heads of kv_head, against keys [k_begin, k_end) read through the block-table
 // row of `seq`.  Row r of the tile is query token q_begin + r / g, head
 // kv_head * g + r % g.  With pos0 >= 0 the tile is causal: token q_begin + i
-// sits at position pos0 + i and sees keys < pos0 + i + 1.  part_row == -1
-// writes the final output; part_row >= 0 writes the normalised partial state to
-// partial rows part_row .. part_row + n_q * g - 1; part_row <= -2 (decode-tile
-// items of a PKV_PLAN_TC_FIRST plan) writes the final output after merging, row
-// by row, the partial state at partial rows -2 - part_row .. (a shared-prefix
-// group tile's rows for these queries) into its own.  pos0 <= -2 (shared-prefix group tiles
+// sits at position pos0 + i and sees keys < pos0 + i + 1.  part_row < 0 writes
+// the final output; otherwise the normalised partial state goes to partial rows
+// part_row .. part_row + n_q * g - 1.  pos0 <= -2 (shared-prefix group tiles
 // of the tensor-memory list, which are not causal): the tile's query tokens are not the run
 // q_begin .. but listed, token i at row_tokens[-2 - pos0 + i] (q_begin is the first of them).
 struct PkvItem {

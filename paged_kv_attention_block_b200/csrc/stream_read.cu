@@ -47,12 +47,6 @@ __global__ void __launch_bounds__(512) stream_read_ldg_kernel(const uint4* __res
 constexpr int kBulkChunk = 32 * 1024;
 constexpr int kBulkStages = 4;
 
-PKV_DEVICE void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
 // Chunks c = blockIdx.x, blockIdx.x + gridDim.x, ... of kBulkChunk bytes (the last one shorter).
 __global__ void __launch_bounds__(64) stream_read_bulk_kernel(const uint8_t* __restrict__ src, int64_t bytes,
                                                               uint32_t* sink, int32_t* status) {
@@ -88,7 +82,7 @@ __global__ void __launch_bounds__(64) stream_read_bulk_kernel(const uint8_t* __r
         const int64_t off = (int64_t(blockIdx.x) + k * gridDim.x) * kBulkChunk;
         const uint32_t n = uint32_t(std::min<int64_t>(kBulkChunk, bytes - off));
         mbar_arrive_expect_tx(bars + 8 * s, n);
-        bulk_load(base + s * kBulkChunk, src + off, n, bars + 8 * s);
+        bulk_load_1d(base + s * kBulkChunk, src + off, n, bars + 8 * s);
         s_issued = k + 1;
       }
     }

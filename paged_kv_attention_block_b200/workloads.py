@@ -360,6 +360,15 @@ def mixed_bf16(seed: int = 1003, n_decode: int = 120, n_prefill: int = 4, chunk:
                  block_size=block_size, seq_lens=seq_lens, q_lens=q_lens)
 
 
+def mixed_fp8(seed: int = 1003, **kw) -> Workload:
+    """The mixed in-flight batch (same lengths and values as mixed_bf16) over an fp8-e4m3 cache:
+    K/V appended from float32 with amax/448 scales per (layer, KV head, K|V), q bf16."""
+    w = mixed_bf16(seed=seed, **kw)
+    return build("mixed_fp8", seed=seed, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32",
+                 num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                 block_size=w.block_size, seq_lens=w.seq_lens, q_lens=w.q_lens)
+
+
 def llama3_8b_decode_nvfp4(seed: int = 1002, batch: int = 64, lo: int = 512, hi: int = 4096) -> Workload:
     """The Llama-3-8B decode batch (same lengths and values as the bf16 one) over an NVFP4 cache:
     Hq 32 / Hkv 8, d 128, block 64, q bf16, K/V appended from float32."""
@@ -391,4 +400,5 @@ NAMED = {
     "longctx_fp8": longctx_fp8,
     "llama3_8b_decode_nvfp4": llama3_8b_decode_nvfp4,
     "prefix_reuse_bf16": prefix_reuse_bf16,
+    "mixed_fp8": mixed_fp8,
 }

@@ -96,23 +96,11 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
         assert len(tok) == it["n_q"] and int(tok[0]) == int(it["q_begin"]) and (np.diff(tok) > 0).all()
     for it in plan["reg_items"]:
         assert it["pos0"] > -2
+    assert (items["part_row"] >= -1).all() and h["flags"] == 0
     direct = items[items["part_row"] == -1]
     for it in direct:
         for i in range(it["n_q"]):
             add(int(it["q_begin"]) + i, int(it["kv_head"]), int(it["k_begin"]), int(it["k_end"]), "direct")
-    # Items that merge a group tile's partial rows in their epilogue (after that tile's kernel).
-    merged = items[items["part_row"] <= -2]
-    assert len(merged) == 0 or h["flags"] & 1, "epilogue merges need the tcgen05 kernel first"
-    for it in merged:
-        src, off = group_source(-2 - int(it["part_row"]))
-        assert src["kv_head"] == it["kv_head"] and src["n_q"] * g > 16
-        src_tok = item_tokens(plan, src)
-        for i in range(it["n_q"]):
-            tok = int(it["q_begin"]) + i
-            assert int(src_tok[off + i]) == tok
-            add(tok, int(it["kv_head"]), int(src["k_begin"]), int(src["k_end"]), "epilogue")
-            add(tok, int(it["kv_head"]), int(it["k_begin"]), int(it["k_end"]), "epilogue")
-        check_shared_blocks(int(it["q_begin"]), src)
     for r in reds:
         for p in parts[r["parts_begin"]:r["parts_begin"] + r["n_parts"]]:
             # The part is either an item's first row or a row inside a group item.

@@ -20,6 +20,7 @@ SAMPLES = {
     "longctx_fp8": [5],
     "prefix_reuse_bf16": [0, 128, 255],
     "llama3_8b_decode_nvfp4": [0, 17, 63],
+    "mixed_fp8": [0, 3, 4, 123],
 }
 
 

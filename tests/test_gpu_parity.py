@@ -79,6 +79,16 @@ def test_mixed_bf16(pkv, aligned):
     run_case(pkv, w, num_ctas=60)
 
 
+@pytest.mark.parametrize("aligned", [True, False])
+def test_mixed_fp8(pkv, aligned):
+    """Prefill chunks over an fp8 cache (tensor-memory tiles whose fp8 K/V are widened to f16 in
+    shared memory) beside fp8 decode rows."""
+    w = W.mixed_fp8(n_decode=9, n_prefill=3, chunk=200, dec_lo=1, dec_hi=1200, cached_lo_blocks=1,
+                    cached_hi_blocks=6, aligned=aligned)
+    plan, _ = run_case(pkv, w, num_ctas=60)
+    assert plan.info["num_tc_items"] > 0
+
+
 def test_mixed_bf16_split_prefill(pkv):
     w = W.mixed_bf16(n_decode=4, n_prefill=2, chunk=150, dec_lo=100, dec_hi=900, cached_lo_blocks=2,
                      cached_hi_blocks=5, block_size=32)
@@ -102,19 +112,14 @@ def test_prefix_reuse_bf16(pkv, cascade):
     w = W.prefix_reuse_bf16(n_req=21, prefix=512, suf_lo=1, suf_hi=300)
     plan, _ = run_case(pkv, w, cascade=cascade)
     assert (plan.info["num_groups"] > 0) == cascade
-    # With the group tiles on the tcgen05 kernel, the decode item of a member whose suffix is one
-    # piece merges the group's state in its own epilogue (the tcgen05 kernel runs first).
-    items = PD.decode(plan.buffer)["reg_items"]
-    assert ((items["part_row"] <= -2).sum() > 0) == cascade
 
 
 @pytest.mark.parametrize("kv", ["bf16", "f16"])
 @pytest.mark.parametrize("split", [0, 64])
 def test_prefix_reuse_member_paths(pkv, kv, split):
-    """Shared-prefix members on every path: one-token and two-token members (8 and 16 rows, decode
-    tiles that merge the group state in their epilogue, or through the merge pass when their
-    suffix is split) and three-token members (24 rows: tcgen05 tiles merged by the merge pass);
-    Hq 64 / Hkv 8, block 16."""
+    """Shared-prefix members on every path: one-token and two-token members (8 and 16 rows: decode
+    tiles) and three-token members (24 rows: tcgen05 tiles), whole or split suffixes, all merged
+    with their group's state by the merge pass; Hq 64 / Hkv 8, block 16."""
     r = np.random.default_rng(23)
     n = 19
     q_lens = r.integers(1, 4, size=n)
@@ -129,9 +134,8 @@ def test_prefix_reuse_member_paths(pkv, kv, split):
 @pytest.mark.parametrize("split", [0, 64])
 def test_prefix_groups_not_neighbours(pkv, kv, split):
     """Three prefixes alternating through the batch (sequence s shares the prefix blocks of group
-    s mod 3): each group's tensor-memory tiles read their listed query tokens, members of a tile
-    of 16 or fewer rows read their prefix themselves, and one- and two-token members merge the
-    group state in their epilogue or through the merge pass."""
+    s mod 3): each group's tensor-memory tiles read their listed query tokens, and members of a
+    tile of 16 or fewer rows read their prefix themselves."""
     r = np.random.default_rng(31)
     n = 41
     q_lens = r.integers(1, 3, size=n)
