@@ -58,7 +58,8 @@ struct AttnKernel {
 // else the cp.async tensor-core kernel, and the CUDA-core kernel for fp32 pools.
 bool attn_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
-// tcgen05 kernel for the tiles of more than 16 rows of a 16-bit pool (attn_tc.cu).
+// tcgen05 kernel for the tiles of more than 16 rows of a 16-bit pool or of an fp8 pool of
+// head_dim 128 (attn_tc.cu).
 bool attn_tc_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k);
 // SM count x occupancy of a kernel on the current device (cached per device).
 int resident_ctas(const AttnKernel& k);

@@ -1,48 +1,50 @@
-// Paged attention for tiles of more than 16 rows on bf16 / f16 pools: the
-// sm_100a tensor cores (tcgen05.mma) with tensor-memory accumulators.
+// Paged attention for tiles of more than 16 rows on bf16 / f16 pools and on fp8
+// (E4M3) pools of head_dim 128: the sm_100a tensor cores (tcgen05.mma) with
+// tensor-memory accumulators.
 //
 // Deep dive (gentlecold.top) §6 and §8: the prefill chunks of a packed batch
 // are its compute-heavy part (and with prefix sharing, §10, so are the group
 // tiles that put many decode rows over one shared prefix).  The work list is
 // the plan's second item list; one persistent CTA per SM runs 128-row tiles,
-// one tensor-memory lane and one softmax thread per row:
+// one tensor-memory lane and two softmax threads per row:
 //
 //   warp 8     TMA producer: pulls items from its atomic counter, publishes each
 //              in a 4-slot descriptor ring and streams K and V tiles of 128 keys
 //              into two separate rings (a K stage is released as soon as S has
 //              been computed from it, a V stage once P V has), 128-byte swizzle,
 //              completion counted on mbarriers.  No load uses cluster multicast.
+//   warps 11, 12 (fp8 pools only) converters: TMA lands the one-byte codes in a
+//              raw ring; these warps widen them exactly into the f16 tiles the
+//              MMAs read.
 //   warps 9, 10 MMA issuers (one thread each): warp 10 issues S = Q K^T into one
 //              of two tensor-memory S buffers, as soon as the tile's K has landed
-//              and the softmax threads are done with the buffer's previous tile;
-//              warp 9 issues O += P V into the tensor-memory O once a tile's P is
-//              written.  Q and P are the A operands straight from tensor memory,
-//              K and V the B operands from their rings (V as an MN-major operand),
-//              so shared memory only carries K and V.  Completions are signalled
-//              with tcgen05.commit on mbarriers; with two issuers one thread's
-//              commits and waits overlap the other's MMAs.
+//              and both halves of the buffer's previous P have been consumed;
+//              warp 9 issues, for each half of the tile's keys, O_h += P_h V_h as
+//              soon as that half's P is written.  Q (staged once per item) and K
+//              come from shared memory, P from tensor memory, V from its ring as an
+//              MN-major operand.  Completions are signalled with tcgen05.commit on
+//              mbarriers; with two issuers one thread's commits and waits overlap
+//              the other's MMAs.
 //   warps 0-7  softmax, two threads per row: warps w and w + 4 share the
-//              tensor-memory lanes of rows 32 (w % 4) .. + 31 and split every row's
-//              columns in halves.  Once per item each thread writes its half of the
-//              row of Q into tensor memory; per tile it loads its half of the row
-//              of S, masks it, swaps its partial max with its partner through
-//              shared memory, keeps the running max and its partial sum in
-//              registers and writes its half of the row of P (16-bit) back to
-//              tensor memory; the epilogue reads its half of the row of O, divides
-//              by the row's sum and stores it.
+//              tensor-memory lanes of rows 32 (w % 4) .. + 31; warp w takes the low
+//              64 keys of every tile, warp w + 4 the high 64.  Each thread keeps its
+//              own running max and sum for its keys and has its own accumulator
+//              (O_lo or O_hi), so the two never wait for each other inside an item:
+//              per tile a thread loads its 64 scores, masks them, writes its 64
+//              probabilities (16-bit) back over them and signals its half's P V.
+//              Once per item the pair swaps (max, sum) through shared memory and
+//              each writes half of the row's head dims from both accumulators.
 //
-// Tensor memory (512 columns, one CTA per SM): O at 0, S buffers at 128 and
-// 256, Q at 384.  P of a tile overwrites the first half of its own S buffer
-// (both threads of every row have loaded their S by then: the max swap sits in
-// between), so P is double-buffered with S and a tile's softmax never waits for
-// the previous P V unless it has to rescale O.
+// Tensor memory (512 columns, one CTA per SM): O_lo at 0, O_hi at D, S buffers
+// at 256 and 384.  A half's P overwrites the start of that half's own S columns,
+// so P is double-buffered with S and a tile's softmax never waits for the
+// previous P V unless it has to rescale its accumulator.
 //
-// The running max of a row only moves when the row max exceeds it by more than
-// 2^8 (log2 units), so P stays <= 256 and the row of O in tensor memory is
-// rescaled rarely.  Keys past an item's end inside its last tile are masked and
-// their V rows zeroed before P V reads them.  Every wait is bounded; on a
-// timeout the CTA records PKV_DEV_TIMEOUT, drains and still frees its tensor
-// memory.
+// A thread's running max only moves when its tile max exceeds it by more than
+// 2^8 (log2 units), so P stays <= 256 and the accumulators are rescaled rarely.
+// Keys past an item's end inside its last tile are masked and their V rows
+// zeroed before P V reads them.  Every wait is bounded; on a timeout the CTA
+// records PKV_DEV_TIMEOUT, drains and still frees its tensor memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -55,37 +57,54 @@
 
 namespace pkv {
 
-template <int D>
+// F8: fp8 (E4M3) pools, d 128.  Their tiles arrive by TMA as one-byte codes in a raw ring of
+// NRAW stages per K and V, and two converter warps widen each into the f16 tile of the MMA ring
+// (value x 2^-8, exact; the power of two and the K / V scales fold into the softmax scale and
+// the output).
+template <int D, bool F8 = false>
 struct TcCfg {
   static constexpr int HALVES = D / 64;          // 64-element (128-byte) column slabs of a row
   static constexpr int TK = PKV_TC_TILE_KEYS;    // keys per tile
   static constexpr int ROWS = PKV_TILE_ROWS_TC;  // rows per item: tensor-memory lanes
   static constexpr int SLAB = TK * 128;          // one column slab of a K or V tile
   static constexpr int TILE = HALVES * SLAB;     // one K or V tile
-  static constexpr int NST = (192 * 1024) / (2 * TILE);  // stages of each ring: 3 (d 128), 6 (d 64)
+  // stages of each ring (what the Q tile leaves of 224 KB): 2 (d 128), 6 (d 64); fp8: 2 of f16
+  // tiles plus 1 of raw codes
+  static constexpr int NST = F8 ? 2 : (224 * 1024 - ROWS * D * 2 - 4096) / (2 * TILE);
+  static constexpr int RAW = F8 ? TK * D : 0;    // one fp8 K or V tile: 128 keys x D bytes
+  static constexpr int NRAW = F8 ? 1 : 0;
+  static constexpr int QBYTES = ROWS * D * 2;    // the item's Q tile (K-major, 128-byte swizzle)
   static constexpr int IR = 4;                   // item descriptor slots
   // mbarrier indices
-  // Warp roles: 0-7 softmax (two threads per row), 8 TMA producer, 9 P V issuer, 10 S issuer.
+  // Warp roles: 0-7 softmax (two threads per row), 8 TMA producer, 9 P V issuer, 10 S issuer,
+  // 11-12 fp8 converters.  Thirteen warps put four on one sub-partition, which caps registers at
+  // 128 a thread (a few bytes spill); measured, two converter warps still beat one at 170.
   static constexpr int SM_WARPS = 8, SM_THREADS = 32 * SM_WARPS, PROD_WARP = 8, PV_WARP = 9, S_WARP = 10;
-  static constexpr int CONSUMER_WARPS = SM_WARPS + 2;
+  static constexpr int CONV_WARP0 = 11, CONV_WARPS = F8 ? 2 : 0, CONV_THREADS = 32 * CONV_WARPS;
+  static constexpr int CONSUMER_WARPS = SM_WARPS + 2 + CONV_WARPS;
   static constexpr int HALF = TK / 2;  // keys of a tile per softmax thread
   // Every POLY_EVERY-th pair of a thread's scores takes its exp2 on the FMA pipe
   // (exp2_fma2), the rest on the exp unit: the split that balances the two.
   static constexpr int POLY_EVERY = 3;
-  // S, P and exchange barriers come in pairs by parity, so that a waiter is never two phases behind.
+  // S, P and exchange barriers come in pairs by parity, so that a waiter is never two phases behind;
+  // P and O barriers per half of the keys: PBAR + 2 h + parity, OBAR + 2 h + parity.
   static constexpr int KFULL = 0, KEMPTY = NST, VFULL = 2 * NST, VEMPTY = 3 * NST, IFULL = 4 * NST,
-                       IEMPTY = IFULL + IR, SBAR = IEMPTY + IR, PBAR = SBAR + 2, XBAR = PBAR + 2, OBAR = XBAR + 2,
-                       QBAR = OBAR + 2, FIN = QBAR + 1, END = FIN + 1, NBAR = END + 1;
-  // XCHG: partial row maxima / sums swapped between the two threads of a row, [2 parities][2 halves][128 rows].
-  static constexpr int K_OFF = 0, V_OFF = NST * TILE, XCHG_OFF = 2 * NST * TILE, BAR_OFF = XCHG_OFF + 2 * 2 * ROWS * 4,
+                       IEMPTY = IFULL + IR, SBAR = IEMPTY + IR, PBAR = SBAR + 2, XBAR = PBAR + 4, OBAR = XBAR + 2,
+                       QBAR = OBAR + 4, FIN = QBAR + 1, END = FIN + 1, K8FULL = END + 1, K8EMPTY = K8FULL + NRAW,
+                       V8FULL = K8EMPTY + NRAW, V8EMPTY = V8FULL + NRAW, NBAR = V8EMPTY + NRAW;
+  // XCHG: the two halves' (running max, sum) of every row, swapped once per item, [128 rows][2 halves].
+  static constexpr int K_OFF = 0, V_OFF = NST * TILE, K8_OFF = 2 * NST * TILE, V8_OFF = K8_OFF + NRAW * RAW,
+                       Q_OFF = V8_OFF + NRAW * RAW, XCHG_OFF = Q_OFF + QBYTES, BAR_OFF = XCHG_OFF + ROWS * 2 * 8,
                        DESC_OFF = BAR_OFF + (8 * NBAR + 63) / 64 * 64;
   static constexpr int SMEM = 1024 + DESC_OFF + IR * 64;
-  static constexpr int THREADS = 32 * (S_WARP + 1);
+  static constexpr int THREADS = 32 * (S_WARP + 1 + CONV_WARPS);
   static constexpr int TMEM_COLS = 512;
-  // Tensor-memory columns: O, two S buffers (fp32; P in the first half of each), Q (16-bit pairs).
-  static constexpr int O_COL = 0, S_COL = 128, Q_COL = 384;
-  static_assert(Q_COL + D / 2 <= TMEM_COLS, "tensor-memory map");
+  // Tensor-memory columns: O of the low and of the high 64 keys of every tile (D each), two S
+  // buffers (fp32; each half's P at the start of its own 64 columns).
+  static constexpr int O_COL = 0, S_COL = 256;
+  static_assert(O_COL + 2 * D <= S_COL && S_COL + 2 * TK <= TMEM_COLS, "tensor-memory map");
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(!F8 || D == 128, "fp8 tiles: head_dim 128 (128-byte rows)");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   // The CTA takes all 512 tensor-memory columns: shared memory must rule out a second CTA on the SM.
   static_assert(2 * (SMEM + 1024) > 228 * 1024, "one CTA per SM");
@@ -110,70 +129,90 @@ PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity, const long long* wl) {
 
 // Half hf of row r of the item (query token q_begin + r / g, or the listed token r / g of a
 // shared-prefix group tile; head kv_head * g + r % g): head dims [hf * D / 2, (hf + 1) * D / 2)
-// into this thread's tensor-memory lane at q_tmem, two 16-bit values per column (the pairs are
-// the row's bytes in memory order).  Rows past R are zero.
-template <int D>
-PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_tmem, int r, int hf) {
+// into the shared-memory Q tile, laid out as a K tile (64-dim column slabs of 128-byte rows,
+// 16-byte chunk c of row r at c ^ (r & 7)).  Rows past R are zero.
+template <int D, bool TO_F16 = false>
+PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_smem, int r, int hf) {
+  using T = TcCfg<D>;
   const bool valid = r < R;
   const int i = valid ? r / a.g : 0;
   const int64_t token = d.pos0 <= -2 ? int64_t(__ldg(a.row_tokens + (-2 - d.pos0) + i)) : int64_t(d.q_begin) + i;
   const uint4* src = reinterpret_cast<const uint4*>(
       static_cast<const uint16_t*>(a.q) + (token * a.hq + d.kv_head * a.g + (valid ? r % a.g : 0)) * D +
       hf * (D / 2));
-  uint32_t w[D / 4];
 #pragma unroll
-  for (int i = 0; i < D / 16; ++i) {
-    const uint4 v = valid ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
-    w[4 * i] = v.x;
-    w[4 * i + 1] = v.y;
-    w[4 * i + 2] = v.z;
-    w[4 * i + 3] = v.w;
+  for (int j = 0; j < D / 16; ++j) {
+    uint4 v = valid ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+    if constexpr (TO_F16) {
+      // bf16 queries for f16 MMAs (fp8 pools): exact for |q| in [2^-14, 65504].
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        w[k] = pack_f16x2(bf16_bits_to_float(uint16_t(w[k] & 0xffff)), bf16_bits_to_float(uint16_t(w[k] >> 16)));
+    }
+    const int dim0 = hf * (D / 2) + 8 * j;
+    const int c = (dim0 % 64) / 8;
+    sts128(q_smem + uint32_t(dim0 / 64) * T::SLAB + uint32_t(r) * 128 + (uint32_t(c ^ (r & 7)) << 4), v);
   }
-  if constexpr (D == 128) tc::st32_nowait(q_tmem, w);
-  else tc::st16_nowait(q_tmem, w);
-  tc::wait_st();
 }
 
-// S[128 x TK] = Q K^T, one thread: D/16 MMAs of K = 16.  Q comes from tensor
-// memory (8 columns per step); K is K-major with the 128-byte swizzle: 8-row
-// groups 1024 bytes apart, the k-step moving 32 bytes inside a 128-byte row,
-// then to the next 64-element column slab.
+// S[128 x TK] = Q K^T, one thread: D/16 MMAs of K = 16, A (Q) and B (K) both K-major in shared
+// memory with the 128-byte swizzle: 8-row groups 1024 bytes apart, the k-step moving 32 bytes
+// inside a 128-byte row, then to the next 64-element column slab.
 template <int D, bool BF>
-PKV_DEVICE void tc_mma_s(uint32_t s_tmem, uint32_t q_tmem, uint32_t kbase) {
+PKV_DEVICE void tc_mma_s(uint32_t s_tmem, uint32_t qbase, uint32_t kbase) {
   using T = TcCfg<D>;
   constexpr uint32_t IDESC = tc::idesc_f16(BF, 128, T::TK, false, false);
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
-    const uint64_t bd = tc::smem_desc(kbase + (ks >> 2) * T::SLAB + (ks & 3) * 32, 16, 1024, tc::SW128);
-    tc::mma_ts(s_tmem, q_tmem + 8 * ks, bd, IDESC, ks > 0);
+    const uint32_t off = (ks >> 2) * T::SLAB + (ks & 3) * 32;
+    tc::mma_ss(s_tmem, tc::smem_desc(qbase + off, 16, 1024, tc::SW128), tc::smem_desc(kbase + off, 16, 1024, tc::SW128),
+               IDESC, ks > 0);
   }
 }
 
-// O[128 x D] (+)= P V, one thread: TK/16 MMAs of K = 16.  P comes from tensor
-// memory; V is the B operand in MN-major form: 64 head dims contiguous (128
-// bytes, 128-byte swizzle), the next 64 dims one column slab further, 8 keys
-// per 1024-byte swizzle atom, so each 16-key step advances 2048 bytes.
+// O[128 x D] (+)= P V over one half of a tile (64 keys), one thread: 4 MMAs of K = 16.  P comes from
+// tensor memory; V is the B operand in MN-major form: 64 head dims contiguous (128 bytes, 128-byte
+// swizzle), the next 64 dims one column slab further, 8 keys per 1024-byte swizzle atom, so each
+// 16-key step advances 2048 bytes (vbase: the tile's first key of the half).
 template <int D, bool BF>
 PKV_DEVICE void tc_mma_o(uint32_t o_tmem, uint32_t p_tmem, uint32_t vbase, bool accumulate) {
   using T = TcCfg<D>;
   constexpr uint32_t IDESC = tc::idesc_f16(BF, 128, D, false, true);
 #pragma unroll
-  for (int ks = 0; ks < T::TK / 16; ++ks) {
+  for (int ks = 0; ks < T::HALF / 16; ++ks) {
     const uint64_t bd = tc::smem_desc(vbase + ks * 2048, T::SLAB, 1024, tc::SW128);
     tc::mma_ts(o_tmem, p_tmem + 8 * ks, bd, IDESC, accumulate || ks > 0);
   }
 }
 
-template <int D, bool BF>
-__global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcArgs ta) {
-  using T = TcCfg<D>;
+// E4M3 codes of one 16-byte chunk -> 16 f16 values (x 2^-8), in order, as two 16-byte pieces.
+PKV_DEVICE void e4m3x16_to_f16(uint4 v, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t p = __byte_perm(w[i], 0, 0x3120);  // bytes (0, 2, 1, 3): pairs (0, 1) and (2, 3)
+    o[2 * i] = e4m3_b02_f16x2(p);
+    o[2 * i + 1] = e4m3_b13_f16x2(p);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// BF: the queries are bf16 (else f16).  F8: the pool is fp8 (MMAs then run on f16 operands).
+template <int D, bool BF, bool F8>
+__global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcArgs ta) {
+  using T = TcCfg<D, F8>;
+  constexpr bool MBF = BF && !F8;  // MMA operands bf16 (else f16)
   constexpr unsigned FULL = 0xffffffffu;
   const AttnArgs& a = ta.a;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t kring = base + T::K_OFF, vring = base + T::V_OFF;
+  const uint32_t kring = base + T::K_OFF, vring = base + T::V_OFF, k8ring = base + T::K8_OFF, v8ring = base + T::V8_OFF;
   const uint32_t bars = base + T::BAR_OFF;
   auto bar = [&](int i) { return bars + 8 * i; };
   TcDesc* descs = reinterpret_cast<TcDesc*>(base_ptr + T::DESC_OFF);
@@ -185,13 +224,19 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   // This kernel may start while the decode-tile kernel ahead of it is still running: it reads
   // nothing that kernel writes (and waits for it before finishing, below).
   if (warp == 0) tc::alloc(smem_addr(&s_tmem), T::TMEM_COLS);
-  float* xchg = reinterpret_cast<float*>(base_ptr + T::XCHG_OFF);
   if (tid == 32) {
     for (int i = 0; i < T::NST; ++i) {
-      mbar_init(bar(T::KFULL + i), 1);
+      // F8: the f16 tiles are filled by the converter threads, not by TMA.
+      mbar_init(bar(T::KFULL + i), F8 ? T::CONV_THREADS : 1);
       mbar_init(bar(T::KEMPTY + i), 1);
-      mbar_init(bar(T::VFULL + i), 1);
+      mbar_init(bar(T::VFULL + i), F8 ? T::CONV_THREADS : 1);
       mbar_init(bar(T::VEMPTY + i), 1);
+    }
+    for (int i = 0; i < T::NRAW; ++i) {
+      mbar_init(bar(T::K8FULL + i), 1);
+      mbar_init(bar(T::K8EMPTY + i), T::CONV_THREADS);
+      mbar_init(bar(T::V8FULL + i), 1);
+      mbar_init(bar(T::V8EMPTY + i), T::CONV_THREADS);
     }
     for (int i = 0; i < T::IR; ++i) {
       mbar_init(bar(T::IFULL + i), 1);
@@ -199,9 +244,11 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(T::SBAR + b), 1);
-      mbar_init(bar(T::PBAR + b), T::SM_THREADS);
       mbar_init(bar(T::XBAR + b), T::SM_THREADS);
-      mbar_init(bar(T::OBAR + b), 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bar(T::PBAR + i), T::SM_THREADS / 2);  // the threads of one half
+      mbar_init(bar(T::OBAR + i), 1);
     }
     mbar_init(bar(T::QBAR), T::SM_THREADS);
     mbar_init(bar(T::FIN), 2);
@@ -287,23 +334,32 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
           }
         }
         const int row0 = box_rows == T::TK ? (key0 & bmask) : 0;
-        const int stg = q % T::NST;
-        const uint32_t par = ((q / T::NST) & 1) ^ 1;
-        const uint32_t bytes = uint32_t(nb) * T::HALVES * box_rows * 128;
+        // The ring the TMA fills: the f16 tiles, or for fp8 pools the raw tiles.
+        constexpr int NS = F8 ? T::NRAW : T::NST;
+        constexpr int FULL_K = F8 ? T::K8FULL : T::KFULL, EMPTY_K = F8 ? T::K8EMPTY : T::KEMPTY;
+        constexpr int FULL_V = F8 ? T::V8FULL : T::VFULL, EMPTY_V = F8 ? T::V8EMPTY : T::VEMPTY;
+        const int stg = q % NS;
+        const uint32_t par = ((q / NS) & 1) ^ 1;
+        const uint32_t bytes = F8 ? uint32_t(nb) * box_rows * D : uint32_t(nb) * T::HALVES * box_rows * 128;
         for (int kv = 0; kv < 2; ++kv) {  // K tile, then V tile
           int f = 1;
           if (lane == 0) {
-            f = (!s_abort && mbar_wait(bar((kv ? T::VEMPTY : T::KEMPTY) + stg), par, &s_wl)) ? 1 : 0;
-            if (f) mbar_arrive_expect_tx(bar((kv ? T::VFULL : T::KFULL) + stg), bytes);
+            f = (!s_abort && mbar_wait(bar((kv ? EMPTY_V : EMPTY_K) + stg), par, &s_wl)) ? 1 : 0;
+            if (f) mbar_arrive_expect_tx(bar((kv ? FULL_V : FULL_K) + stg), bytes);
           }
           if (!__shfl_sync(FULL, f, 0)) { ok = false; break; }
           k_armed = kv == 0;
           if (lane < nb) {
-            const uint32_t dst = (kv ? vring : kring) + stg * T::TILE + uint32_t(lane * box_rows) * 128;
+            if constexpr (F8) {
+              const uint32_t dst = (kv ? v8ring : k8ring) + stg * T::RAW + uint32_t(lane * box_rows) * D;
+              tma_load_5d(dst, &tmap, bar((kv ? FULL_V : FULL_K) + stg), 0, row0, it.kv_head, c3k + kv, phys);
+            } else {
+              const uint32_t dst = (kv ? vring : kring) + stg * T::TILE + uint32_t(lane * box_rows) * 128;
 #pragma unroll
-            for (int h = 0; h < T::HALVES; ++h)
-              tma_load_5d(dst + h * T::SLAB, &tmap, bar((kv ? T::VFULL : T::KFULL) + stg), h * 64, row0, it.kv_head,
-                          c3k + kv, phys);
+              for (int h = 0; h < T::HALVES; ++h)
+                tma_load_5d(dst + h * T::SLAB, &tmap, bar((kv ? FULL_V : FULL_K) + stg), h * 64, row0, it.kv_head,
+                            c3k + kv, phys);
+            }
           }
         }
       }
@@ -314,13 +370,71 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;
       // Let loads already issued land before the CTA's shared memory goes away.
-      if (k_armed) mbar_wait(bar(T::KFULL + q % T::NST), (q / T::NST) & 1, &s_wl);
-      for (int k = 1; k <= T::NST && q - k >= 0; ++k) {
-        mbar_wait(bar(T::KFULL + (q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
-        mbar_wait(bar(T::VFULL + (q - k) % T::NST), ((q - k) / T::NST) & 1, &s_wl);
+      constexpr int NS = F8 ? T::NRAW : T::NST;
+      constexpr int FULL_K = F8 ? T::K8FULL : T::KFULL, FULL_V = F8 ? T::V8FULL : T::VFULL;
+      if (k_armed) mbar_wait(bar(FULL_K + q % NS), (q / NS) & 1, &s_wl);
+      for (int k = 1; k <= NS && q - k >= 0; ++k) {
+        mbar_wait(bar(FULL_K + (q - k) % NS), ((q - k) / NS) & 1, &s_wl);
+        mbar_wait(bar(FULL_V + (q - k) % NS), ((q - k) / NS) & 1, &s_wl);
       }
     }
     return;
+  }
+
+  if constexpr (F8) {
+    if (warp >= T::CONV_WARP0) {
+      // ------------------------------------------- fp8 converters (warps 11, 12)
+      // Tile qq: raw stage qq % NRAW (filled by TMA) -> f16 stage qq % NST (free once the S or
+      // P V MMAs of tile qq - NST have completed).  Chunk c (16 codes: dims 16c .. 16c+15) of
+      // key row r sits at (c ^ (r & 7)) in the raw row (128-byte swizzle); its 16 f16 values go
+      // to the 16-byte chunks 2(c % 4) and +1 of column slab c / 4, swizzled the same way.
+      const int ct = tid - 32 * T::CONV_WARP0;
+      int q = 0, it_seq = 0;
+      bool ok = true;
+      for (;;) {
+        const int slot = it_seq % T::IR;
+        bool go = __all_sync(FULL, !s_abort);
+        if (go) go = warp_wait(bar(T::IFULL + slot), (it_seq / T::IR) & 1, &s_wl);
+        if (!go) { ok = false; break; }
+        const TcDesc d = descs[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(T::IEMPTY + slot), 1);
+        ++it_seq;
+        if (d.state == 2) break;
+        if (d.state == 1) continue;
+        for (int t = 0; t < d.ntiles && ok; ++t) {
+          const int qq = q + t;
+          for (int kv = 0; kv < 2 && ok; ++kv) {
+            const int s8 = qq % T::NRAW, s16 = qq % T::NST;
+            go = !s_abort && warp_wait(bar((kv ? T::V8FULL : T::K8FULL) + s8), (qq / T::NRAW) & 1, &s_wl);
+            if (go) go = warp_wait(bar((kv ? T::VEMPTY : T::KEMPTY) + s16), ((qq / T::NST) & 1) ^ 1, &s_wl);
+            if (!go) { ok = false; break; }
+            const uint32_t src = (kv ? v8ring : k8ring) + s8 * T::RAW, dst = (kv ? vring : kring) + s16 * T::TILE;
+            for (int x = ct; x < T::TK * 8; x += T::CONV_THREADS) {
+              const int r = x >> 3, c = x & 7;
+              uint4 lo, hi;
+              e4m3x16_to_f16(lds128(src + uint32_t(r) * 128 + (uint32_t(c ^ (r & 7)) << 4)), lo, hi);
+              const uint32_t row = dst + uint32_t(c >> 2) * T::SLAB + uint32_t(r) * 128;
+              const int j = (c & 3) * 2;
+              sts128(row + (uint32_t(j ^ (r & 7)) << 4), lo);
+              sts128(row + (uint32_t((j + 1) ^ (r & 7)) << 4), hi);
+            }
+            fence_proxy_async_smem();  // the f16 tile is read by the tensor core (async proxy)
+            mbar_arrive(bar((kv ? T::VFULL : T::KFULL) + s16), 1);
+            mbar_arrive(bar((kv ? T::V8EMPTY : T::K8EMPTY) + s8), 1);
+          }
+        }
+        q += d.ntiles;
+        if (!ok) break;
+      }
+      if (!ok) {
+        report(a.status, PKV_DEV_TIMEOUT);
+        s_abort = 1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(T::END), 1);
+      return;
+    }
   }
 
   if (warp > T::PROD_WARP) {
@@ -351,24 +465,32 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
           if (good) tc::fence_after_sync();
           for (int t = 0; t < n && good; ++t) {
             const int qq = q + t, stg = qq % T::NST;
-            // The buffer's previous tile: its P (in the buffer) has been read by P V.
-            if (t >= 2) good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
+            // The buffer's previous tile: both halves of its P (in the buffer) have been read by P V.
+            if (t >= 2) {
+              good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
+              if (good) good = !s_abort && mbar_wait(bar(T::OBAR + 2 + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
+            }
             if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1, &s_wl);
             if (!good) break;
             tc::fence_after_sync();
-            tc_mma_s<D, BF>(tmem + T::S_COL + (qq & 1) * T::TK, tmem + T::Q_COL, kring + stg * T::TILE);
+            tc_mma_s<D, MBF>(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, kring + stg * T::TILE);
             tc::commit(bar(T::SBAR + (qq & 1)));
             tc::commit(bar(T::KEMPTY + stg));
           }
         } else {
           for (int t = 0; t < n && good; ++t) {
-            const int qq = q + t, stg = qq % T::NST;
-            good = !s_abort && mbar_wait(bar(T::PBAR + (qq & 1)), (qq >> 1) & 1, &s_wl);
-            if (good) good = mbar_wait(bar(T::VFULL + stg), (qq / T::NST) & 1, &s_wl);
+            const int qq = q + t, stg = qq % T::NST, sb = qq & 1;
+            good = !s_abort && mbar_wait(bar(T::VFULL + stg), (qq / T::NST) & 1, &s_wl);
+            // Each half's P V as soon as that half's P is written: O_h (+)= P_h V_h.
+            for (int h = 0; h < 2 && good; ++h) {
+              good = !s_abort && mbar_wait(bar(T::PBAR + 2 * h + sb), (qq >> 1) & 1, &s_wl);
+              if (!good) break;
+              tc::fence_after_sync();
+              tc_mma_o<D, MBF>(tmem + T::O_COL + h * D, tmem + T::S_COL + sb * T::TK + h * T::HALF,
+                               vring + stg * T::TILE + h * (T::HALF / 8) * 1024, t > 0);
+              tc::commit(bar(T::OBAR + 2 * h + sb));
+            }
             if (!good) break;
-            tc::fence_after_sync();
-            tc_mma_o<D, BF>(tmem + T::O_COL, tmem + T::S_COL + (qq & 1) * T::TK, vring + stg * T::TILE, t > 0);
-            tc::commit(bar(T::OBAR + (qq & 1)));
             tc::commit(bar(T::VEMPTY + stg));
           }
         }
@@ -393,25 +515,18 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   }
 
   // ---------------------------------------------------------------- softmax
-  const int lq = warp & 3, hf = warp >> 2;  // lane quarter and column half
+  // Split O: the thread of half hf of row r owns the keys [64 hf, 64 hf + 64) of every tile, with
+  // its own running max and sum and its own accumulator O_hf, fed by the P V MMAs of those keys.
+  // The two halves of a row never wait for each other during the item; its epilogue merges them.
+  const int lq = warp & 3, hf = warp >> 2;  // lane quarter and key half
   const int r = 32 * lq + lane;             // row of the tile and tensor-memory lane
-  const int stid = tid;                     // 0 .. SM_THREADS - 1
+  const int htid = tid - hf * (T::SM_THREADS / 2);  // 0 .. 127 within the half
   const uint32_t lane_base = uint32_t(lq * 32) << 16;
-  const uint32_t o_tm = tmem + lane_base + T::O_COL + hf * (D / 2), s_tm = tmem + lane_base + T::S_COL + hf * T::HALF;
-  const uint32_t q_tm = tmem + lane_base + T::Q_COL + hf * (D / 4);
-  const uint32_t p_tm = tmem + lane_base + T::S_COL + hf * (T::HALF / 2);  // + S buffer offset
-  int q = 0, it_seq = 0, xc = 0;  // xc: exchanges so far (barrier XBAR + (xc & 1), parity (xc >> 1) & 1)
+  const uint32_t o_lo = tmem + lane_base + T::O_COL, o_hi = o_lo + D, o_own = o_lo + hf * D;
+  const uint32_t s_tm = tmem + lane_base + T::S_COL + hf * T::HALF;  // + S buffer offset: this half's S, then its P
+  float2* xchg = reinterpret_cast<float2*>(base_ptr + T::XCHG_OFF);
+  int q = 0, it_seq = 0, xc = 0;  // xc: items exchanged so far (barrier XBAR + (xc & 1), parity (xc >> 1) & 1)
   bool ok = true;
-  // Swap a value with the row's other thread through shared memory (bounded wait).
-  auto exchange = [&](float mine, float& other) -> bool {
-    float* buf = xchg + (xc & 1) * 2 * T::ROWS;
-    buf[hf * T::ROWS + r] = mine;
-    mbar_arrive(bar(T::XBAR + (xc & 1)), 1);
-    const bool done = warp_wait(bar(T::XBAR + (xc & 1)), (xc >> 1) & 1, &s_wl);
-    other = buf[(hf ^ 1) * T::ROWS + r];
-    ++xc;
-    return done;
-  };
   for (;;) {
     const int slot = it_seq % T::IR;
     bool go = __all_sync(FULL, ok && !s_abort);
@@ -425,18 +540,25 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     if (d.state == 1) continue;
     const int R = d.n_q * a.g;
     const int ntiles = d.ntiles;
-    const float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
+    float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
+    float vfac = 1.f;                    // output factor: the V scale of fp8 tiles
+    if constexpr (F8) {
+      // The widened tiles hold code values x 2^-8: the power of two goes back with the scales.
+      c *= __ldg(a.k_scale + a.layer * a.hkv + d.kv_head) * 256.f;
+      vfac = __ldg(a.v_scale + a.layer * a.hkv + d.kv_head) * 256.f;
+    }
     const bool to_part = d.part_row >= 0;
     const int last_valid = d.k_end - (d.k_begin + (ntiles - 1) * T::TK);  // keys of the last tile in range
     const int lim = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / a.g + 1) : d.k_end;
     const int lo = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / a.g : -1);
 
-    // The previous item's MMAs are complete (its epilogue waited for the last P V): Q is free.
-    tc_stage_q<D>(a, d, R, q_tm, r, hf);
-    tc::fence_before_sync();
+    // The previous item's MMAs are complete (its epilogue waited for its last P V): Q is free.
+    tc_stage_q<D, F8 && BF>(a, d, R, base + T::Q_OFF, r, hf);
+    fence_proxy_async_smem();  // read by the tensor core
+    tc::fence_before_sync();   // the previous item's tensor-memory reads, before its next MMAs
     mbar_arrive(bar(T::QBAR), 1);
 
-    float m_run = -INFINITY, l_run = 0.f;  // running max of the row (log2 units), sum of this half
+    float m_run = -INFINITY, l_run = 0.f;  // running max (log2 units) and sum of this half's keys
     for (int t = 0; t < ntiles; ++t) {
       const int qq = q + t, stg = qq % T::NST, sb = qq & 1;
       go = __all_sync(FULL, ok && !s_abort);
@@ -457,23 +579,19 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         for (int j = 0; j < T::HALF; ++j)
           if (key0 + j >= lim || key0 + j < lo) s[j] = -INFINITY;
       }
-      // Max of this half over 8 independent chains, then of the row with the partner's.
+      // Max of this half over 8 independent chains.
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
       for (int j = 8; j < T::HALF; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      float mx_other;
-      if (!exchange(mx, mx_other)) { ok = false; continue; }
-      mx = fmaxf(mx, mx_other);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mnew = mx * c;
-      // Both threads of the row take the same decisions from the same values.
       float alpha = 1.f;
       bool rescale = false;
       if (mnew > m_run + 8.f) {
-        alpha = fast_exp2(m_run - mnew);  // 0 while the row has seen no key
+        alpha = fast_exp2(m_run - mnew);  // 0 while this half has seen no key
         rescale = t > 0 && m_run != -INFINITY;
         m_run = mnew;
         l_run *= alpha;
@@ -492,12 +610,15 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       }
       acc[0] = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
       l_run += acc[0].x + acc[0].y;
-      if (t == ntiles - 1 && last_valid < T::TK) {
-        // Keys past the item's end: zero their V rows before P V reads them (0 * NaN would leak).
+      // Keys of this half past the item's end: zero their V rows before this half's P V reads them
+      // (0 * NaN would leak).
+      const int zrow0 = max(last_valid, hf * T::HALF), nz = (hf + 1) * T::HALF - zrow0;
+      const bool zero_tail = t == ntiles - 1 && nz > 0;
+      if (zero_tail) {
         if (warp_wait(bar(T::VFULL + stg), (qq / T::NST) & 1, &s_wl)) {
           const uint32_t vt = vring + stg * T::TILE;
-          for (int x = stid; x < (T::TK - last_valid) * T::HALVES * 8; x += T::SM_THREADS) {
-            const int row = last_valid + x / (T::HALVES * 8), h = (x / 8) % T::HALVES, ch = x % 8;
+          for (int x = htid; x < nz * T::HALVES * 8; x += T::SM_THREADS / 2) {
+            const int row = zrow0 + x / (T::HALVES * 8), h = (x / 8) % T::HALVES, ch = x % 8;
             sts128(vt + h * T::SLAB + row * 128 + (uint32_t(ch ^ (row & 7)) << 4), make_uint4(0, 0, 0, 0));
           }
         } else {
@@ -505,71 +626,87 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         }
       }
       if (__any_sync(FULL, rescale)) {
-        // O must hold the previous tile's P V before it is rescaled (t > 0 here).
-        if (!warp_wait(bar(T::OBAR + ((qq - 1) & 1)), ((qq - 1) >> 1) & 1, &s_wl)) { ok = false; continue; }
+        // O_hf must hold this half's previous P V before it is rescaled (t > 0 here).
+        if (!warp_wait(bar(T::OBAR + 2 * hf + ((qq - 1) & 1)), ((qq - 1) >> 1) & 1, &s_wl)) { ok = false; continue; }
         tc::fence_after_sync();
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        for (int c0 = 0; c0 < D; c0 += 32) {
           float o[32];
-          tc::ld32(o_tm + c0, o);
+          tc::ld32(o_own + c0, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= f;
-          tc::st32(o_tm + c0, o);
+          tc::st32(o_own + c0, o);
         }
       }
-      // This half of the row of P (16-bit pairs) into tensor memory for the P V step.
+      // This half's P (16-bit pairs) at the start of its own S columns, for its P V.
       {
         uint32_t w[T::HALF / 2];
 #pragma unroll
         for (int i = 0; i < T::HALF / 2; ++i)
-          w[i] = BF ? pack_bf16x2(s[2 * i], s[2 * i + 1]) : pack_f16x2(s[2 * i], s[2 * i + 1]);
-        tc::st32_nowait(p_tm + sb * T::TK, w);
+          w[i] = MBF ? pack_bf16x2(s[2 * i], s[2 * i + 1]) : pack_f16x2(s[2 * i], s[2 * i + 1]);
+        tc::st32_nowait(s_tm + sb * T::TK, w);
       }
       tc::wait_st();
-      if (t == ntiles - 1 && last_valid < T::TK) fence_proxy_async_smem();  // the zeroed V rows
+      if (zero_tail) fence_proxy_async_smem();  // the zeroed V rows
       tc::fence_before_sync();
-      mbar_arrive(bar(T::PBAR + sb), 1);
+      mbar_arrive(bar(T::PBAR + 2 * hf + sb), 1);
     }
-    // Epilogue: this half of O / l, straight from tensor memory; l is the sum of both halves.
+    // Epilogue: once this half's last P V is done, the halves swap (max, sum); each thread writes
+    // half of the row's head dims from both accumulators:
+    //   o = (O_lo 2^(m_lo - M) + O_hi 2^(m_hi - M)) / (l_lo 2^(m_lo - M) + l_hi 2^(m_hi - M)).
     go = __all_sync(FULL, ok);
-    float l_other = 0.f;
-    if (go) go = exchange(l_run, l_other);
-    if (go) go = warp_wait(bar(T::OBAR + ((q + ntiles - 1) & 1)), ((q + ntiles - 1) >> 1) & 1, &s_wl);
+    const int qlast = q + ntiles - 1;
+    if (go) go = warp_wait(bar(T::OBAR + 2 * hf + (qlast & 1)), (qlast >> 1) & 1, &s_wl);
+    float2 other = make_float2(-INFINITY, 0.f);
+    if (go) {
+      xchg[r * 2 + hf] = make_float2(m_run, l_run);
+      tc::fence_before_sync();
+      mbar_arrive(bar(T::XBAR + (xc & 1)), 1);
+      go = warp_wait(bar(T::XBAR + (xc & 1)), (xc >> 1) & 1, &s_wl);
+      other = xchg[r * 2 + (hf ^ 1)];
+      ++xc;
+    }
     if (go) {
       tc::fence_after_sync();
-      const float l = l_run + l_other;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float M = fmaxf(m_run, other.x);
+      const float f_own = m_run == -INFINITY ? 0.f : fast_exp2(m_run - M);
+      const float f_oth = other.x == -INFINITY ? 0.f : fast_exp2(other.x - M);
+      const float l = l_run * f_own + other.y * f_oth;
+      const float inv = l > 0.f ? vfac / l : 0.f;
+      const float f_lo = (hf == 0 ? f_own : f_oth) * inv, f_hi = (hf == 0 ? f_oth : f_own) * inv;
       const int64_t orow = to_part ? int64_t(d.part_row) + r
                                    : (int64_t(d.q_begin) + r / a.g) * a.hq + d.kv_head * a.g + r % a.g;
 #pragma unroll 1
       for (int c0 = 0; c0 < D / 2; c0 += 32) {
-        float o[32];
-        tc::ld32(o_tm + c0, o);
         const int col = hf * (D / 2) + c0;
+        float o[32], oh[32];
+        tc::ld32(o_lo + col, o);
+        tc::ld32(o_hi + col, oh);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = o[i] * f_lo + oh[i] * f_hi;
         if (r < R) {
           if (to_part) {
             float4* dst = reinterpret_cast<float4*>(a.part_o + orow * D + col);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float* x = o + 8 * i;
-              if constexpr (BF)
-                dst[i] = make_uint4(pack_bf16x2(x[0] * inv, x[1] * inv), pack_bf16x2(x[2] * inv, x[3] * inv),
-                                    pack_bf16x2(x[4] * inv, x[5] * inv), pack_bf16x2(x[6] * inv, x[7] * inv));
+              if constexpr (BF)  // the output in q's dtype
+                dst[i] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                    pack_bf16x2(x[6], x[7]));
               else
-                dst[i] = make_uint4(pack_f16x2(x[0] * inv, x[1] * inv), pack_f16x2(x[2] * inv, x[3] * inv),
-                                    pack_f16x2(x[4] * inv, x[5] * inv), pack_f16x2(x[6] * inv, x[7] * inv));
+                dst[i] = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]), pack_f16x2(x[4], x[5]),
+                                    pack_f16x2(x[6], x[7]));
             }
           }
         }
       }
       if (r < R && hf == 0) {
-        const float lse = l > 0.f ? (m_run + __log2f(l)) * kLn2 : -INFINITY;
+        const float lse = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
         if (to_part) a.part_lse[orow] = lse;
         else if (a.out_lse) a.out_lse[orow] = lse;
       }
@@ -601,24 +738,24 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
 
 // ---- host side -------------------------------------------------------------
 
-template <int D, bool BF>
+template <int D, bool BF, bool F8>
 cudaError_t launch_tc(const AttnArgs& a, int grid, cudaStream_t st) {
-  using T = TcCfg<D>;
+  using T = TcCfg<D, F8>;
   CUtensorMap map;
   const int box_rows = std::min(1 << a.log2_block, T::TK);
-  if (!make_pool_map(a, D, 2, BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, box_rows, 1,
-                     &map))
-    return cudaErrorInvalidValue;
-  const cudaError_t e = launch_pdl(attn_tc_kernel<D, BF>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map,
+  const CUtensorMapDataType dt = F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                    : (BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  if (!make_pool_map(a, D, F8 ? 1 : 2, dt, box_rows, 1, &map)) return cudaErrorInvalidValue;
+  const cudaError_t e = launch_pdl(attn_tc_kernel<D, BF, F8>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map,
                                    TcArgs{a, box_rows});
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int D, bool BF>
+template <int D, bool BF, bool F8 = false>
 AttnKernel tc_kernel() {
-  using T = TcCfg<D>;
-  return AttnKernel{reinterpret_cast<const void*>(&attn_tc_kernel<D, BF>), T::THREADS, T::SMEM, &launch_tc<D, BF>,
-                    T::ROWS};
+  using T = TcCfg<D, F8>;
+  return AttnKernel{reinterpret_cast<const void*>(&attn_tc_kernel<D, BF, F8>), T::THREADS, T::SMEM,
+                    &launch_tc<D, BF, F8>, T::ROWS};
 }
 
 bool attn_tc_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {
@@ -632,17 +769,23 @@ bool attn_tc_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size,
     *k = d128 ? tc_kernel<128, false>() : tc_kernel<64, false>();
     return true;
   }
+  if (kv_dtype == PKV_FP8_E4M3 && d128 && (q_dtype == PKV_BF16 || q_dtype == PKV_F16)) {
+    *k = q_dtype == PKV_BF16 ? tc_kernel<128, true, true>() : tc_kernel<128, false, true>();
+    return true;
+  }
   return false;
 }
 
 }  // namespace pkv
 
 bool pkv_tc_capable(int kv_dtype, int head_dim, int block_size) {
+  if (kv_dtype == PKV_FP8_E4M3) return head_dim == 128 && block_size >= 8;
   return (kv_dtype == PKV_BF16 || kv_dtype == PKV_F16) && (head_dim == 64 || head_dim == 128) && block_size >= 8;
 }
 
 int pkv_tc_resident_ctas(int kv_dtype, int head_dim, int block_size) {
   pkv::AttnKernel k;
-  if (!pkv::attn_tc_kernel_for(kv_dtype, kv_dtype, head_dim, block_size, &k)) return -1;
+  const int q_dtype = kv_dtype == PKV_F16 ? PKV_F16 : PKV_BF16;
+  if (!pkv::attn_tc_kernel_for(kv_dtype, q_dtype, head_dim, block_size, &k)) return -1;
   return pkv::resident_ctas(k);
 }

@@ -24,9 +24,8 @@
 //     MMA through movmatrix.  Fragment addresses are fixed per lane; masking
 //     runs only on tiles that reach past a row's limit.  The four warps merge
 //     their softmax states at the end of the item.
-//   * Prefill tiles (> 16 rows; fp8 pools, since 16-bit pools send them to the
-//     tcgen05 kernel of attn_tc.cu): every warp reads every tile and owns 16
-//     rows (the row-split step of attn_tile.cuh).
+//   * Tiles of more than 16 rows (prefill chunks, shared-prefix group tiles) go to
+//     the tcgen05 kernel of attn_tc.cu; this kernel takes decode-sized items only.
 //   * fp8 and NVFP4 tiles widen to f16 in registers with integer operations
 //     (exact; values times a power of two taken back in the score and output
 //     scales).  NVFP4 tiles arrive as two TMA boxes, E2M1 codes (64-byte rows,
@@ -74,8 +73,7 @@ struct TmaCfg {
   // A multiple of 4: decode tiles go round-robin to the 4 consumer warps by tile
   // index within the item, so within an item every tile that lands in a given
   // stage belongs to the same warp and the stage's phases are consumed in order;
-  // across items, the end-of-item merge barrier (decode) or every warp reading
-  // every tile (prefill) orders them.
+  // across items, the end-of-item merge barrier orders them.
   // Four 16 KB stages (64 KB) leave room for two CTAs per SM: twice the producers and consumer
   // warps of one large-ring CTA, which measured faster than a 12-stage ring with one CTA per SM.
   static constexpr int NST = FP4 ? 8 : 4 * std::max(1, std::min(12, (64 * 1024) / STAGE_BYTES) / 4);
@@ -946,68 +944,6 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       mbar_arrive(merge_bar, 1);
       if (!mbar_wait(merge_bar, merge_phase, &s_wl)) ok = false;
       merge_phase ^= 1;
-    } else if constexpr (KV == KV_E4M3) {
-      // ---- prefill tile (fp8 pools; 16-bit pools send these to the tcgen05 kernel):
-      // every warp reads every tile, 16 rows per warp.
-      ItemCtx<D, KV, QBF> cx;
-      cx.g = a.g;
-      cx.R = R;
-      cx.row_base = 16 * warp;
-      const bool active = cx.row_base < R;
-      PkvItem it{d.seq, d.kv_head, d.q_begin, d.n_q, d.k_begin, d.k_end, d.pos0, d.part_row};
-      load_q<D, KV, QBF>(a, it, cx, g4, t4);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int r = cx.row_base + g4 + 8 * hh;
-        cx.lim[hh] = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / cx.g + 1) : d.k_end;
-        cx.lo[hh] = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / cx.g : -1);
-        cx.m[hh] = -INFINITY;
-        cx.l[hh] = 0.f;
-      }
-#pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) cx.acc[nt][0] = cx.acc[nt][1] = cx.acc[nt][2] = cx.acc[nt][3] = 0.f;
-      for (int t = 0; t < ntiles; ++t) {
-        const int qq = q + t;
-        const int stg = qq % T::NST;
-        if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1, &s_wl)) { ok = false; continue; }
-        const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::TK * 128;
-        if (t == ntiles - 1 && last_valid < T::TK) {
-          zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);  // each warp writes the same zeros
-          fence_proxy_async_smem();
-        }
-        if (active)
-          compute_keys<T::TK / 16, D, KV, QBF, T::TK, T::SLAB>(a, cx, kb, vb, 0, d.k_begin + t * T::TK, g4, t4, lane, c);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(stg), 1);
-      }
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        cx.l[hh] += __shfl_xor_sync(0xffffffffu, cx.l[hh], 1);
-        cx.l[hh] += __shfl_xor_sync(0xffffffffu, cx.l[hh], 2);
-      }
-      if (active) {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int r = cx.row_base + g4 + 8 * hh;
-          if (r >= R) continue;
-          const float inv = cx.l[hh] > 0.f ? vscale / cx.l[hh] : 0.f;
-          const float lse = cx.l[hh] > 0.f ? (cx.m[hh] + __log2f(cx.l[hh])) * kLn2 : -INFINITY;
-          const int64_t orow = to_part ? int64_t(d.part_row) + r : (int64_t(d.q_begin) + r / cx.g) * a.hq + d.kv_head * cx.g + r % cx.g;
-#pragma unroll
-          for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-            for (int e = 2 * hh; e < 2 * hh + 2; ++e) {
-              const int dd = acc_dim<KV>(nt, e, t4);
-              const float v = cx.acc[nt][e] * inv;
-              if (to_part) a.part_o[orow * D + dd] = v;
-              else store_q_dtype<QBF>(a.out, orow * D + dd, v);
-            }
-          if (t4 == 0) {
-            if (to_part) a.part_lse[orow] = lse;
-            else if (a.out_lse) a.out_lse[orow] = lse;
-          }
-        }
-      }
     }
     q += ntiles;
     if (!ok) break;
@@ -1118,10 +1054,10 @@ cudaError_t launch_tma(const AttnArgs& a, int grid, cudaStream_t st) {
 template <int D, int KV, bool QBF>
 AttnKernel tma_kernel() {
   using T = TmaCfg<D, KV, QBF>;
-  // 16-bit pools: only decode-sized tiles (larger ones are tcgen05 items); fp8: up to 64 rows.
+  // Decode-sized tiles only (larger ones are tcgen05 items).
   return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF>), T::THREADS, T::SMEM,
                     &launch_tma<D, KV, QBF>,
-                    KV == KV_E4M3 ? PKV_TILE_ROWS : (KV == KV_NVFP4 ? PKV_FP4_ROWS : PKV_DECODE_ROWS)};
+                    KV == KV_NVFP4 ? PKV_FP4_ROWS : PKV_DECODE_ROWS};
 }
 
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {

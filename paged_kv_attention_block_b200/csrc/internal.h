@@ -8,7 +8,8 @@
 pkv_status pkv_fail(pkv_status s, const char* fmt, ...);
 
 // True when tiles of more than PKV_DECODE_ROWS rows of these shapes run on the
-// tcgen05 kernel (16-bit pools, head_dim 64 or 128, block size >= 8).
+// tcgen05 kernel (16-bit pools of head_dim 64 or 128, fp8 pools of head_dim 128;
+// block size >= 8).
 bool pkv_tc_capable(int kv_dtype, int head_dim, int block_size);
 // CTAs of the tcgen05 kernel resident on the current device, or -1.
 int pkv_tc_resident_ctas(int kv_dtype, int head_dim, int block_size);

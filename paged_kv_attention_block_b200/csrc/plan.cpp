@@ -12,8 +12,8 @@
 //      persistent CTAs finish together, weighting a tile by its rows (compute)
 //      and keys (bytes); every KV head of a tile gets the same pieces;
 //   3. emits the merges that combine split ranges (and group tiles) per row.
-// On 16-bit pools tiles of more than 16 rows (prefill chunks, shared-prefix
-// groups) go to a second list served by the tcgen05 kernel, 128 rows a tile,
+// On 16-bit pools (and fp8 pools of head_dim 128) tiles of more than 16 rows
+// (prefill chunks, shared-prefix groups) go to a second list served by the tcgen05 kernel, 128 rows a tile,
 // and are split and balanced over that kernel's CTAs on their own.  Items are
 // ordered heaviest first within each list; CTAs pull them from an atomic
 // counter.
@@ -167,7 +167,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
 
   // 1. Shared-prefix groups: sequences whose tables begin with the same physical blocks (deep
   // dive §10: the radix tree hands the same prefix blocks to every request that shares it).  On
-  // 16-bit pools the sharers may lie anywhere in the batch (the batch is packed by request kind,
+  // tensor-memory pools the sharers may lie anywhere in the batch (the batch is packed by request kind,
   // not by prefix): sequences are bucketed by their first block id and each bucket is grouped
   // greedily.  A group of consecutive sequences reads its queries as one run of tokens; any other
   // group lists its query tokens in the plan (tensor-memory tiles only).  Other pools group runs

@@ -14,7 +14,7 @@
 #define PKV_TILE_ROWS 64
 // Keys per pipeline stage of the register-tile kernels.
 #define PKV_TILE_KEYS 64
-// Tensor-memory items (16-bit pools): more than PKV_DECODE_ROWS and at most
+// Tensor-memory items (16-bit pools; fp8 pools of head_dim 128): more than PKV_DECODE_ROWS and at most
 // PKV_TILE_ROWS_TC rows (one tensor-memory lane per row), keys in tiles of
 // PKV_TC_TILE_KEYS; a split key range starts on a multiple of that.
 #define PKV_DECODE_ROWS 16

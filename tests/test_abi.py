@@ -147,8 +147,8 @@ def test_plan_covers_every_key_once(api, name, make, opts):
 
 
 def test_plan_routes_prefill_tiles_to_tensor_memory_list(api):
-    """16-bit pools: tiles of more than 16 rows go to the tcgen05 list in 128-row tiles;
-    fp8 pools keep 64-row tiles in the register-tile list."""
+    """16-bit pools and fp8 pools of head_dim 128: tiles of more than 16 rows go to the tcgen05
+    list in 128-row tiles; fp8 pools of head_dim 64 keep 64-row tiles in the register-tile list."""
     w = W.mixed_bf16(n_decode=6, n_prefill=2, chunk=300, block_size=16, cached_lo_blocks=1, cached_hi_blocks=20)
     d = PD.decode(_plan(api, w).buffer)
     g = w.num_q_heads // w.num_kv_heads
@@ -158,7 +158,12 @@ def test_plan_routes_prefill_tiles_to_tensor_memory_list(api):
     w8 = W.build("f8", seed=2, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32, num_kv_heads=8,
                  head_dim=128, block_size=16, seq_lens=[400, 50], q_lens=[200, 1])
     d8 = PD.decode(_plan(api, w8).buffer)
-    assert d8["header"]["n_tc_items"] == 0 and (d8["items"]["n_q"] * 4).max() == 64
+    assert d8["header"]["n_tc_items"] > 0 and (d8["tc_items"]["n_q"] * 4).max() == 128
+    assert (d8["reg_items"]["n_q"] * 4 <= 16).all()
+    w64 = W.build("f8d64", seed=2, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
+                  num_kv_heads=8, head_dim=64, block_size=16, seq_lens=[400, 50], q_lens=[200, 1])
+    d64 = PD.decode(_plan(api, w64).buffer)
+    assert d64["header"]["n_tc_items"] == 0 and (d64["items"]["n_q"] * 4).max() == 64
 
 
 @pytest.mark.parametrize("window", [1, 5, 64, 200, 100000])
@@ -309,8 +314,8 @@ def test_plan_groups_sharers_that_are_not_neighbours(api):
     """Two prefixes alternating through the batch (sequence s shares the blocks of prefix s mod 2):
     on a 16-bit pool both prefixes form a group, whose tensor-memory tiles list their query tokens
     (a group tile of 16 or fewer rows would have to run on the decode tiles, so the members of such
-    a tile read their prefix themselves); an fp8 pool groups only runs of consecutive sharers, so
-    it finds none here."""
+    a tile read their prefix themselves); an fp8 pool of head_dim 64 (register tiles only) groups
+    only runs of consecutive sharers, so it finds none here."""
     w = W.build("two", seed=24, kv_dtype="bf16", num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=16,
                 seq_lens=300 + np.arange(37) * 7, q_lens=[1] * 37, shared_prefix_tokens=256, prefix_groups=2)
     p = _plan(api, w)
@@ -324,6 +329,6 @@ def test_plan_groups_sharers_that_are_not_neighbours(api):
         tok = PD.item_tokens(d, it)
         assert (np.diff(tok) == 2).all() and len(set(tok % 2)) == 1
     w8 = W.build("two8", seed=25, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32,
-                 num_kv_heads=8, head_dim=128, block_size=16, seq_lens=[300] * 9, q_lens=[1] * 9,
+                 num_kv_heads=8, head_dim=64, block_size=16, seq_lens=[300] * 9, q_lens=[1] * 9,
                  shared_prefix_tokens=256, prefix_groups=2)
     assert _plan(api, w8).info["num_groups"] == 0

@@ -130,7 +130,7 @@ def test_prefix_reuse_member_paths(pkv, kv, split):
     assert plan.info["num_groups"] >= 1
 
 
-@pytest.mark.parametrize("kv", ["bf16", "f16"])
+@pytest.mark.parametrize("kv", ["bf16", "f16", "e4m3"])
 @pytest.mark.parametrize("split", [0, 64])
 def test_prefix_groups_not_neighbours(pkv, kv, split):
     """Three prefixes alternating through the batch (sequence s shares the prefix blocks of group
@@ -140,8 +140,9 @@ def test_prefix_groups_not_neighbours(pkv, kv, split):
     n = 41
     q_lens = r.integers(1, 3, size=n)
     seq_lens = 256 + q_lens + r.integers(0, 300, size=n)
+    fp8 = dict(q_dtype="bf16", kv_in_dtype="f32") if kv == "e4m3" else {}
     w = W.build("three", seed=32, kv_dtype=kv, num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=16,
-                seq_lens=seq_lens, q_lens=q_lens, shared_prefix_tokens=256, prefix_groups=3)
+                seq_lens=seq_lens, q_lens=q_lens, shared_prefix_tokens=256, prefix_groups=3, **fp8)
     plan, _ = run_case(pkv, w, kv_split=split)
     d = PD.decode(plan.buffer)
     assert plan.info["num_groups"] == 3 and (d["tc_items"]["pos0"] <= -2).any()
@@ -159,6 +160,16 @@ def test_few_ctas_many_items(pkv, ctas):
 @pytest.mark.parametrize("ctas", [1, 3])
 def test_few_ctas_decode_fp8(pkv, ctas):
     run_case(pkv, W.longctx_fp8(batch=5, seq_len=2000), num_ctas=ctas, kv_split=192)
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 5])
+def test_few_ctas_prefill_fp8(pkv, ctas):
+    """fp8 prefill tiles on the tcgen05 kernel with few CTAs: the raw-code and f16 rings and the
+    converter warps wrap many times, across items of ragged last tiles (block 16)."""
+    w = W.mixed_fp8(n_decode=9, n_prefill=3, chunk=200, dec_lo=1, dec_hi=700, cached_lo_blocks=1,
+                    cached_hi_blocks=30, block_size=16, aligned=False)
+    plan, _ = run_case(pkv, w, num_ctas=ctas, kv_split=256)
+    assert plan.info["num_tc_items"] > 0
 
 
 # ---- shapes and dtypes ----------------------------------------------------
