@@ -540,7 +540,7 @@ def summarise(w, r, world, peak, peak_kind):
                 "ms_per_step": r["e2e"]["ms"]},
         "clocks": r["clocks"],
         "plan": {k: r["plan"][k] for k in ("num_items", "num_tc_items", "num_reduce", "num_partial_rows",
-                                           "num_groups", "num_ctas")},
+                                           "num_groups", "num_ctas", "tc_num_ctas", "side_by_side")},
         "launches_per_step": 1 + (r["plan"]["num_items"] > n_tc) + (n_tc > 0) + (r["plan"]["num_reduce"] > 0),
     }
 

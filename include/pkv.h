@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define PKV_ABI_VERSION 2
+#define PKV_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define PKV_API __attribute__((visibility("default")))
@@ -224,6 +224,17 @@ typedef struct pkv_plan_request {
                                    test the timeout path (with a short wait_limit_kcycles) without a
                                    fault.  Outputs are then incomplete.  Kernels without a TMA producer
                                    (block sizes below 8, 64-byte fp8 rows, fp32 pools) ignore it. */
+  int32_t tc_num_ctas;          /* side by side: tiles of more than 16 rows (the tcgen05 kernel, deep dive
+                                   §6/§8 prefill chunks and §10 shared-prefix group tiles) and the
+                                   decode-sized tiles (the HBM stream) in one call run at the same time on
+                                   disjoint SMs, the tcgen05 kernel on tc_num_ctas CTAs (one an SM) and the
+                                   decode-tile kernel on num_ctas CTAs, instead of one after the other.
+                                   > 0: side by side on these counts whenever the batch has both kinds of
+                                   tile (num_ctas must then be > 0 too; both are capped at what fits).
+                                   0: automatic, with num_ctas = 0 only: side by side when the planner's
+                                   estimate of the two kernels' times says it pays, splitting the SMs of
+                                   the current device between them.  < 0: never.  Plans are the same for
+                                   every layer either way. */
 } pkv_plan_request;
 
 #define PKV_DEBUG_WITHHOLD_LOADS 0x1
@@ -238,6 +249,9 @@ typedef struct pkv_plan_info {
   int32_t num_groups;           /* shared-prefix groups found */
   int32_t num_ctas;             /* CTAs planned for */
   int32_t num_tc_items;         /* of num_items: tiles of more than 16 rows for the tcgen05 kernel */
+  int32_t tc_num_ctas;          /* CTAs planned for the tcgen05 kernel */
+  int32_t side_by_side;         /* 1: the two kernels run at the same time on disjoint SMs (num_ctas
+                                   and tc_num_ctas CTAs); 0: one after the other */
 } pkv_plan_info;
 
 /*
@@ -270,9 +284,11 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  * launch serves a packed mix of prefill and decode requests), §8 (chunked
  * prefill with causal masking).  One call enqueues one persistent attention
  * kernel for the decode-sized tiles, one tcgen05 kernel for the tiles of more
- * than 16 rows of a bf16/f16 pool (when the plan has such tiles) and, when the
- * plan split a key range, one merge kernel (the same merge
- * pkv_split_kv_reduce performs), in that order on `stream`.
+ * than 16 rows of a bf16/f16 pool or an fp8 pool of head_dim 128 (when the plan
+ * has such tiles) and, when the plan split a key range, one merge kernel (the
+ * same merge pkv_split_kv_reduce performs), in that order on `stream`; a plan
+ * made side by side (pkv_plan_info.side_by_side) enqueues the tcgen05 kernel
+ * first and the decode-tile kernel beside it, on the SMs it leaves free.
  *
  * q: device [total_q][num_q_heads][head_dim], q_dtype F32 (F32 pools only),
  *   BF16 (BF16, FP8 or NVFP4 pools) or F16 (F16, FP8 or NVFP4 pools).

@@ -90,7 +90,9 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
       !inside(h->parts_off, h->n_parts, sizeof(int32_t)) || h->num_ctas <= 0 || (h->n_tc_items > 0 && h->tc_num_ctas <= 0))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan sections out of range");
   if (h->n_tc_items > 0 && !tc) return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan has tcgen05 items for a pool without that kernel");
-  if (h->flags != 0) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
+  if ((h->flags & ~PKV_PLAN_CORUN) != 0) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
+  if ((h->flags & PKV_PLAN_CORUN) != 0 && (h->n_items == 0 || h->n_tc_items == 0))
+    return pkv_fail(PKV_ERR_PLAN, "paged_attention: side-by-side plan without both item lists");
   if (h->n_rows < 0 || !inside(h->rows_off, h->n_rows, sizeof(int32_t)))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan token list out of range");
   const int32_t* rows_list = reinterpret_cast<const int32_t*>(base + h->rows_off);
@@ -252,10 +254,13 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
     e = record_event(static_cast<cudaEvent_t>(kernels_begin), st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));
   }
+  const bool corun = (h->flags & PKV_PLAN_CORUN) != 0;
   auto launch_reg = [&]() -> pkv_status {
     if (h->n_items == 0) return PKV_OK;
     const int grid = std::max(1, std::min(std::min(resident, h->num_ctas), h->n_items));
-    const cudaError_t le = k.launch(a, grid, st);
+    pkv::AttnArgs r = a;
+    r.pdl_role = corun ? 1 : 0;  // side by side: launched beside the tcgen05 kernel
+    const cudaError_t le = k.launch(r, grid, st);
     if (le != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: launch failed: %s", cudaGetErrorString(le));
     return PKV_OK;
   };
@@ -266,16 +271,23 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
     t.n_items = h->n_tc_items;
     t.counter = a.counter + 32;  // 128 bytes on
     t.max_rows = ktc.max_rows;
+    t.pdl_role = corun ? 0 : 1;
     const int grid = std::max(1, std::min(std::min(tc_resident, h->tc_num_ctas), h->n_tc_items));
     const cudaError_t le = ktc.launch(t, grid, st);
     if (le != cudaSuccess)
       return pkv_fail(PKV_ERR_CUDA, "paged_attention: tcgen05 launch failed: %s", cudaGetErrorString(le));
     return PKV_OK;
   };
-  // Decode tiles first, the tcgen05 tiles behind them (its CTAs take the SMs the decode-tile
-  // kernel frees as it drains).
-  if (pkv_status ls = launch_reg(); ls != PKV_OK) return ls;
-  if (pkv_status ls = launch_tc(); ls != PKV_OK) return ls;
+  // Side by side: the tcgen05 tiles first on their share of the SMs, the decode tiles beside
+  // them.  Otherwise the decode tiles first and the tcgen05 tiles behind them (its CTAs take the
+  // SMs the decode-tile kernel frees as it drains).
+  if (corun) {
+    if (pkv_status ls = launch_tc(); ls != PKV_OK) return ls;
+    if (pkv_status ls = launch_reg(); ls != PKV_OK) return ls;
+  } else {
+    if (pkv_status ls = launch_reg(); ls != PKV_OK) return ls;
+    if (pkv_status ls = launch_tc(); ls != PKV_OK) return ls;
+  }
   if (kernels_end) {
     e = record_event(static_cast<cudaEvent_t>(kernels_end), st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));

@@ -257,8 +257,14 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     s_wl = a.wait_limit;
     fence_mbar_init();
   }
-  // Behind the decode-tile kernel, whose CTAs had waited for the plan staging (and so for the
-  // work before it) before triggering this launch, this grid reads nothing that kernel writes.
+  // Second (behind the decode-tile kernel, whose CTAs had waited for the plan staging, and so
+  // for the work before it, before triggering this launch): this grid reads nothing that kernel
+  // writes.  First: wait for the plan staging, then let the decode-tile kernel launch beside
+  // this one on the SMs it leaves free.
+  if (a.pdl_role == 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -730,8 +736,8 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     __syncwarp();
     tc::fence_after_sync();
     tc::dealloc(tmem, T::TMEM_COLS);
-    // The grid finishes only after the kernel ahead of it, so the merge that waits for this
-    // grid also sees that kernel's partial states.
+    // Second: the grid finishes only after the kernel ahead of it, so the merge that waits for
+    // this grid also sees that kernel's partial states.  (First: returns at once.)
     if (lane == 0) pdl_wait();
   }
 }

@@ -600,10 +600,12 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     s_wl = a.wait_limit;
     fence_mbar_init();
   }
-  // Launched as a programmatic dependent of the plan staging: the barriers above are set up while
-  // that runs; nothing it or the work before it wrote (the plan, the appended K/V, q) is read
-  // before this.  A no-op when the kernel ahead is not a programmatic primary.
-  pdl_wait();
+  // First: launched as a programmatic dependent of the plan staging, the barriers above are set
+  // up while that runs; nothing it or the work before it wrote (the plan, the appended K/V, q)
+  // is read before this.  A no-op when the kernel ahead is not a programmatic primary.  Second
+  // (beside the tcgen05 kernel): that kernel waited for the plan staging before it let this
+  // launch.
+  if (a.pdl_role == 0) pdl_wait();
   __syncthreads();
 
   if (warp == 4) {
@@ -952,6 +954,9 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     report(a.status, PKV_DEV_TIMEOUT);
     s_abort = 1;
   }
+  // Second: the grid finishes only after the tcgen05 kernel beside it, so the merge that waits
+  // for this grid also sees that kernel's partial states.
+  if (a.pdl_role == 1 && tid == 0) pdl_wait();
 }
 
 // ---- host side -------------------------------------------------------------

@@ -33,6 +33,13 @@
 
 namespace {
 
+// Side-by-side estimate, measured on B200: the tensor-memory tiles' rate per CTA (16-bit and fp8
+// pools, causal chunks), the decode-tile kernel's stream rate per SM (16-bit, fp8 pools) and the whole HBM stream, the
+// fixed cost of a decode item per CTA, and the least gain that makes the plan run side by side.
+constexpr double kTcFlopsPerSm = 4.5e12, kTcFp8FlopsPerSm = 2.3e12;
+constexpr double kRegBytesPerSm = 75e9, kRegFp8BytesPerSm = 45e9, kHbmBytes = 6.0e12, kRegItemSec = 1.5e-6;
+constexpr double kCorunGain = 0.92;
+
 // One (query tile, key piece): every KV head h of it becomes an item (and, when the tile's
 // keys are split or it belongs to a shared-prefix group, a merge per head).
 struct Piece {
@@ -139,6 +146,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (req->wait_limit_kcycles < 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: wait_limit_kcycles < 0");
   if (req->debug_flags & ~PKV_DEBUG_WITHHOLD_LOADS)
     return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: unknown debug_flags 0x%x", req->debug_flags);
+  if (req->tc_num_ctas > 0 && req->num_ctas <= 0)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: tc_num_ctas > 0 needs num_ctas > 0");
   const int32_t* cu = req->cu_q_lens;
   const int32_t* L = req->seq_lens;
   if (S > 0 && cu[0] != 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: cu_q_lens[0] != 0");
@@ -329,6 +338,47 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     }
   }
 
+  // 2b. Side by side.  With both decode-sized tiles (HBM-bound) and tensor-memory tiles
+  // (tensor-bound) in the batch, the tcgen05 kernel may take k SMs and the decode-tile kernel the
+  // others at the same time instead of one after the other.  Estimated times: the tensor-memory
+  // list at kTcFlopsPerSm a CTA, the decode-tile list at the smaller of the HBM stream rate and
+  // kRegBytesPerSm an SM, plus kRegItemSec per item and CTA.  Only for automatic CTA counts.
+  bool corun = false;
+  if (req->tc_num_ctas > 0) {
+    if (tc && total_cost[0] > 0 && total_cost[1] > 0) {
+      corun = true;
+      tc_ctas = req->tc_num_ctas;
+    }
+  } else if (req->tc_num_ctas == 0 && req->num_ctas <= 0 && tc && total_cost[0] > 0 && total_cost[1] > 0) {
+    const int sms = tc_ctas;  // one tcgen05 CTA an SM
+    const int per_sm = std::max(1, num_ctas / std::max(1, sms));
+    const bool f8 = req->kv_dtype == PKV_FP8_E4M3;
+    const double flops = total_cost[1] * 16.0 * 4.0 * D;           // rows x keys x 4 head_dim
+    const double bytes = total_cost[0] * 2.0 * D * (f8 ? 1.0 : 2.0);  // K and V rows of every key
+    int64_t n_reg_pieces = 0;  // decode-tile items before any key split
+    for (size_t i = 0; i < n_group_pieces; ++i) n_reg_pieces += pieces[i].tc ? 0 : 1;
+    for (const Tile& t : tiles) n_reg_pieces += is_tc(t.n_q * g) ? 0 : 1;
+    const double reg_items = double(n_reg_pieces) * Hkv;
+    const double tc_rate = f8 ? kTcFp8FlopsPerSm : kTcFlopsPerSm;
+    auto t_tc = [&](int k) { return flops / (double(k) * tc_rate); };
+    auto t_reg = [&](int n) {
+      return bytes / std::min(kHbmBytes, double(n) * (f8 ? kRegFp8BytesPerSm : kRegBytesPerSm)) +
+             reg_items * kRegItemSec / double(n * per_sm);
+    };
+    const double serial = t_tc(sms) + t_reg(sms);
+    double best = serial;
+    int best_k = 0;
+    for (int k = 1; k < sms; ++k) {
+      const double t = std::max(t_tc(k), t_reg(sms - k));
+      if (t < best) { best = t; best_k = k; }
+    }
+    if (best_k > 0 && best < kCorunGain * serial) {
+      corun = true;
+      tc_ctas = best_k;
+      num_ctas = (sms - best_k) * per_sm;
+    }
+  }
+
   // 3. Key-range split and merges.
   const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 2.0)};
   // Longest key range of one item of a tile's list; the automatic length (about two items per
@@ -489,6 +539,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   info->num_groups = n_groups;
   info->num_ctas = num_ctas;
   info->num_tc_items = int32_t(n_tc);
+  info->tc_num_ctas = tc_ctas;
+  info->side_by_side = corun ? 1 : 0;
   if (!plan) return PKV_OK;
   if (capacity < bytes) return pkv_fail(PKV_ERR_WORKSPACE, "attention_plan: capacity %zu < %llu", capacity, (unsigned long long)bytes);
 
@@ -500,6 +552,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.n_tc_items = int32_t(n_tc);
   h.tc_items_off = uint32_t(tc_items_off);
   h.tc_num_ctas = tc_ctas;
+  h.flags = corun ? PKV_PLAN_CORUN : 0;
   h.window = window;
   h.wait_limit_kcycles = req->wait_limit_kcycles;
   h.debug_flags = req->debug_flags;

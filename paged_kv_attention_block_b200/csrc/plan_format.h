@@ -51,12 +51,16 @@ struct PkvPlanHeader {
   int32_t window;        // limited attention window in positions; 0 = none
   int32_t wait_limit_kcycles;  // limit on every pipeline wait, thousands of SM cycles; 0 = default
   int32_t debug_flags;   // PKV_DEBUG_* (0 in normal use)
-  int32_t flags;         // reserved (0)
+  int32_t flags;         // PKV_PLAN_* bits
   uint32_t rows_off;     // listed query tokens of group tiles (int32 each)
   int32_t n_rows;
   int32_t pad[4];        // header is 128 bytes
 };
 static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
+// The two item lists run side by side: the tcgen05 kernel is launched first on tc_num_ctas CTAs
+// (one an SM) and the decode-tile kernel beside it on num_ctas CTAs (the other SMs).  Without it
+// the decode-tile kernel runs first and the tcgen05 kernel takes the SMs it frees.
+#define PKV_PLAN_CORUN 0x1
 
 // One CTA-sized piece of work: rows [q_begin, q_begin + n_q) x the g query
 // heads of kv_head, against keys [k_begin, k_end) read through the block-table

@@ -96,7 +96,9 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
         assert len(tok) == it["n_q"] and int(tok[0]) == int(it["q_begin"]) and (np.diff(tok) > 0).all()
     for it in plan["reg_items"]:
         assert it["pos0"] > -2
-    assert (items["part_row"] >= -1).all() and h["flags"] == 0
+    assert (items["part_row"] >= -1).all() and h["flags"] in (0, 1)
+    if h["flags"] == 1:  # side by side: both lists run at once
+        assert len(plan["reg_items"]) > 0 and len(plan["tc_items"]) > 0
     direct = items[items["part_row"] == -1]
     for it in direct:
         for i in range(it["n_q"]):

@@ -39,7 +39,7 @@ def test_exports_match_header(api):
 
 
 def test_version_and_strings(api):
-    assert api._lib.pkv_abi_version() == 2
+    assert api._lib.pkv_abi_version() == 3
     assert api.status_string(0) == "ok" and api.status_string(4) == "buffer too small"
 
 
@@ -308,6 +308,24 @@ def test_plan_carries_wait_limit_and_debug_flags(api):
         _plan(api, w, wait_limit_kcycles=-1)
     with pytest.raises(api.PkvError):
         _plan(api, w, debug_flags=0x2)
+
+
+def test_plan_side_by_side(api):
+    """tc_num_ctas > 0: a batch with both kinds of tile is planned side by side (header flag, the
+    two CTA counts as given, every row covered once); a decode-only batch, tc_num_ctas < 0, or an
+    explicit num_ctas alone is not; tc_num_ctas > 0 without num_ctas is refused."""
+    w = W.mixed_bf16(n_decode=30, n_prefill=2, chunk=300, block_size=16, cached_lo_blocks=1, cached_hi_blocks=20)
+    d = PD.decode(_plan(api, w, num_ctas=200, tc_num_ctas=48).buffer)
+    h = d["header"]
+    assert h["flags"] == 1 and h["num_ctas"] == 200 and h["tc_num_ctas"] == 48
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
+                      w.block_size)
+    assert PD.decode(_plan(api, w, num_ctas=200, tc_num_ctas=-1).buffer)["header"]["flags"] == 0
+    assert PD.decode(_plan(api, w, num_ctas=200).buffer)["header"]["flags"] == 0
+    wd = W.llama3_8b_decode_bf16(batch=9, lo=10, hi=900)
+    assert PD.decode(_plan(api, wd, num_ctas=200, tc_num_ctas=48).buffer)["header"]["flags"] == 0
+    with pytest.raises(api.PkvError):
+        _plan(api, w, num_ctas=0, tc_num_ctas=48)
 
 
 def test_plan_groups_sharers_that_are_not_neighbours(api):

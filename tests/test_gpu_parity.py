@@ -162,6 +162,25 @@ def test_few_ctas_decode_fp8(pkv, ctas):
     run_case(pkv, W.longctx_fp8(batch=5, seq_len=2000), num_ctas=ctas, kv_split=192)
 
 
+SIDE_CASES = {
+    "mixed_bf16": lambda: W.mixed_bf16(n_decode=20, n_prefill=3, chunk=200, dec_lo=1, dec_hi=1500, cached_lo_blocks=1,
+                                       cached_hi_blocks=8, block_size=32, aligned=False),
+    "mixed_fp8": lambda: W.mixed_fp8(n_decode=20, n_prefill=3, chunk=200, dec_lo=1, dec_hi=1500, cached_lo_blocks=1,
+                                     cached_hi_blocks=8, block_size=32, aligned=False),
+    "prefix_bf16": lambda: W.prefix_reuse_bf16(n_req=21, prefix=512, suf_lo=1, suf_hi=300),
+}
+
+
+@pytest.mark.parametrize("ctas", [(40, 4), (7, 2), (200, 60)])
+@pytest.mark.parametrize("kind", list(SIDE_CASES))
+def test_side_by_side(pkv, kind, ctas):
+    """The tcgen05 tiles (prefill chunks, shared-prefix group tiles) and the decode tiles running
+    at the same time on disjoint SMs, with forced CTA counts (rings wrapping in both kernels)."""
+    w = SIDE_CASES[kind]()
+    plan, _ = run_case(pkv, w, num_ctas=ctas[0], tc_num_ctas=ctas[1])
+    assert PD.decode(plan.buffer)["header"]["flags"] == 1
+
+
 @pytest.mark.parametrize("ctas", [1, 2, 5])
 def test_few_ctas_prefill_fp8(pkv, ctas):
     """fp8 prefill tiles on the tcgen05 kernel with few CTAs: the raw-code and f16 rings and the
@@ -442,6 +461,9 @@ TIMEOUT_CASES = {
     # a prefill chunk (tcgen05 kernel) beside decode rows
     "mixed_bf16": lambda: W.mixed_bf16(n_decode=3, n_prefill=1, chunk=150, dec_lo=50, dec_hi=900, cached_lo_blocks=1,
                                        cached_hi_blocks=3),
+    # the same batch with the two kernels side by side
+    "mixed_bf16_side_by_side": lambda: W.mixed_bf16(n_decode=3, n_prefill=1, chunk=150, dec_lo=50, dec_hi=900,
+                                                    cached_lo_blocks=1, cached_hi_blocks=3),
 }
 
 
@@ -455,14 +477,17 @@ def test_wait_timeout_is_reported(pkv, kind):
     w = TIMEOUT_CASES[kind]()
     dw = runner.DeviceWorkload(w)
     dw.append_new()
-    plan = dw.plan(num_ctas=16, wait_limit_kcycles=200, debug_flags=api.PKV_DEBUG_WITHHOLD_LOADS)
+    side = {"tc_num_ctas": 4} if kind.endswith("side_by_side") else {}
+    plan = dw.plan(num_ctas=16, wait_limit_kcycles=200, debug_flags=api.PKV_DEBUG_WITHHOLD_LOADS, **side)
+    if side:
+        assert PD.decode(plan.buffer)["header"]["flags"] == 1
     out = torch.zeros_like(dw.q)
     dw.attention(plan, out=out)
     torch.cuda.synchronize()
     assert int(dw.status.item()) & 0x10, "PKV_DEV_TIMEOUT not reported"
     dw.status.zero_()
     out = torch.full_like(dw.q, float("nan"))
-    dw.attention(dw.plan(num_ctas=16), out=out)
+    dw.attention(dw.plan(num_ctas=16, **side), out=out)
     torch.cuda.synchronize()
     assert int(dw.status.item()) == 0
     ref, _ = oracle_out(w, oracle_pool(w))
