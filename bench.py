@@ -412,10 +412,10 @@ def measure(w, args, dev, world, plan_opts, steps):
                                 w.causal, out=out, workspace=ws, status=dw.status)
     torch.cuda.synchronize(dev)
     # The timed steps replay one graph per step (kv_append then paged_attention), one graph per
-    # plan buffer.  A second set holds the paged_attention call alone, whose library call also
-    # records events around the attention kernels: the call's own time (plan staging, kernels,
-    # merge) and the kernel-only time come from replaying those one at a time after the timed run
-    # (event record nodes inside the timed graphs would add latency to the step).
+    # plan buffer.  A second set holds the paged_attention call alone (plan staging, kernels,
+    # merge), timed back to back like the steps; a third the same call with events recorded by
+    # the library around the attention kernels, replayed one at a time for the kernel-only time
+    # (event record nodes inside the timed graphs would add latency).
     g_step = []
     for b in bufs:
         g = torch.cuda.CUDAGraph()
@@ -424,6 +424,13 @@ def measure(w, args, dev, world, plan_opts, steps):
             api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
                                 w.causal, out=out, workspace=ws, status=dw.status)
         g_step.append(g)
+    g_attn = []
+    for b in bufs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            api.paged_attention(dw.cache, dw.q, dw.cu_q, dw.seq_lens, dw.block_tables, b, w.softmax_scale,
+                                w.causal, out=out, workspace=ws, status=dw.status)
+        g_attn.append(g)
     g_attn_ev = []
     for b in bufs:
         g = torch.cuda.CUDAGraph()
@@ -434,9 +441,9 @@ def measure(w, args, dev, world, plan_opts, steps):
     done = [None, None]
     host_plan_s = 0.0
 
-    def step(i, evs=None, split=False):
-        """One step; `evs` = (start, -, end) events; split: the attention call alone (its graph with
-        kernel events, no append) instead of the one-graph step."""
+    def step(i, evs=None, split=None):
+        """One step; `evs` = (start, -, end) events; split: "attn" the attention call alone (no
+        append), "attn_ev" the same with kernel events, instead of the one-graph step."""
         nonlocal host_plan_s
         slot = i % 2
         if done[slot] is not None:
@@ -448,7 +455,9 @@ def measure(w, args, dev, world, plan_opts, steps):
             flush.sum()
             if evs:
                 evs[0].record(stream)
-            if split:
+            if split == "attn":
+                g_attn[slot].replay()
+            elif split == "attn_ev":
                 g_attn_ev[slot].replay()
             else:
                 g_step[slot].replay()
@@ -477,14 +486,17 @@ def measure(w, args, dev, world, plan_opts, steps):
     host_plan_us = host_plan_s / steps * 1e6
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     ms = float(np.mean(step_ms))
-    # Per phase and the attention kernels' own duration: the same steps from the split graphs,
-    # one at a time, each read back after it ran.
+    # The attention call alone, back to back like the steps; then the attention kernels' own
+    # duration from the graphs with kernel events, one at a time, each read back after it ran.
+    for i in range(nsplit):
+        step(i, ev_split[i], split="attn")
+    torch.cuda.synchronize(dev)
+    attn = float(np.mean([a_.elapsed_time(c) for a_, _, c in ev_split]))
     kern_ms = []
     for i in range(nsplit):
-        step(i, ev_split[i], split=True)
+        step(i, split="attn_ev")
         torch.cuda.synchronize(dev)
         kern_ms.append(kev[0].elapsed_time(kev[1]))
-    attn = float(np.mean([a_.elapsed_time(c) for a_, _, c in ev_split]))
     kern = float(np.mean(kern_ms))
     ms, attn, kern = max_over_ranks([ms, attn, kern], dev)
     assert int(dw.status.item()) == 0, "device status set during the benchmark"
@@ -494,7 +506,7 @@ def measure(w, args, dev, world, plan_opts, steps):
     for _ in range(200):
         api.plan_attention(w.cu_q_lens, w.seq_lens, buffer=bufs[0].buffer, **plan_kw)
     plan_call_us = (time.perf_counter() - t0) / 200 * 1e6
-    del g_step, g_attn_ev
+    del g_step, g_attn, g_attn_ev
     read_ceiling = read_stream_gbs(flush)
     del flush
     e2e = run_e2e(args, w, dw, plan_opts, dev, api, steps)
@@ -541,7 +553,9 @@ def summarise(w, r, world, peak, peak_kind):
         "clocks": r["clocks"],
         "plan": {k: r["plan"][k] for k in ("num_items", "num_tc_items", "num_reduce", "num_partial_rows",
                                            "num_groups", "num_ctas", "tc_num_ctas", "side_by_side")},
-        "launches_per_step": 1 + (r["plan"]["num_items"] > n_tc) + (n_tc > 0) + (r["plan"]["num_reduce"] > 0),
+        # kv_append, the plan staging kernel (the plans are page-locked), the attention kernels present
+        # in the plan, the merge when the plan has one.
+        "launches_per_step": 2 + (r["plan"]["num_items"] > n_tc) + (n_tc > 0) + (r["plan"]["num_reduce"] > 0),
     }
 
 
