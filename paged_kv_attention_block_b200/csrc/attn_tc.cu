@@ -13,9 +13,10 @@
 //              into two separate rings (a K stage is released as soon as S has
 //              been computed from it, a V stage once P V has), 128-byte swizzle,
 //              completion counted on mbarriers.  No load uses cluster multicast.
-//   warps 11, 12 (fp8 pools only) converters: TMA lands the one-byte codes in a
-//              raw ring; these warps widen them exactly into the f16 tiles the
-//              MMAs read.
+//   warps 11, 12 (fp8 pools only) converters: TMA lands the one-byte codes in
+//              raw rings; S reads the K codes as they are (kind::f8f6f4, with Q
+//              split into high and low E4M3 parts), and these warps widen the V
+//              codes exactly into the f16 tiles the P V MMAs read.
 //   warps 9, 10 MMA issuers (one thread each): warp 10 issues S = Q K^T into one
 //              of two tensor-memory S buffers, as soon as the tile's K has landed
 //              and both halves of the buffer's previous P have been consumed;
@@ -57,10 +58,12 @@
 
 namespace pkv {
 
-// F8: fp8 (E4M3) pools, d 128.  Their tiles arrive by TMA as one-byte codes in a raw ring of
-// NRAW stages per K and V, and two converter warps widen each into the f16 tile of the MMA ring
-// (value x 2^-8, exact; the power of two and the K / V scales fold into the softmax scale and
-// the output).
+// F8: fp8 (E4M3) pools, d 128.  Their tiles arrive by TMA as one-byte codes in raw rings (NRK
+// stages of K, NRV of V).  S = Q K^T runs on kind::f8f6f4 straight from the raw K tiles, with Q
+// split per row into a high and a low E4M3 part after a power-of-two row scale (together they
+// hold Q's 8 significant bits); two converter warps widen each V tile into the f16 tile of the
+// P V ring (value x 2^-8, exact).  The row scale and the K scale fold into the softmax scale, the
+// power of two and the V scale into the output.
 template <int D, bool F8 = false>
 struct TcCfg {
   static constexpr int HALVES = D / 64;          // 64-element (128-byte) column slabs of a row
@@ -71,8 +74,9 @@ struct TcCfg {
   // stages of each ring (what the Q tile leaves of 224 KB): 2 (d 128), 6 (d 64); fp8: 2 of f16
   // tiles plus 1 of raw codes
   static constexpr int NST = F8 ? 2 : (224 * 1024 - ROWS * D * 2 - 4096) / (2 * TILE);
+  static constexpr int NSK = F8 ? 0 : NST;       // f16 K stages (fp8: S reads the raw codes)
   static constexpr int RAW = F8 ? TK * D : 0;    // one fp8 K or V tile: 128 keys x D bytes
-  static constexpr int NRAW = F8 ? 1 : 0;
+  static constexpr int NRK = F8 ? 4 : 0, NRV = F8 ? 2 : 0;  // raw K and V stages
   static constexpr int QBYTES = ROWS * D * 2;    // the item's Q tile (K-major, 128-byte swizzle)
   static constexpr int IR = 4;                   // item descriptor slots
   // mbarrier indices
@@ -88,13 +92,16 @@ struct TcCfg {
   static constexpr int POLY_EVERY = 3;
   // S, P and exchange barriers come in pairs by parity, so that a waiter is never two phases behind;
   // P and O barriers per half of the keys: PBAR + 2 h + parity, OBAR + 2 h + parity.
-  static constexpr int KFULL = 0, KEMPTY = NST, VFULL = 2 * NST, VEMPTY = 3 * NST, IFULL = 4 * NST,
+  static constexpr int KFULL = 0, KEMPTY = NSK, VFULL = 2 * NSK, VEMPTY = 2 * NSK + NST, IFULL = 2 * NSK + 2 * NST,
                        IEMPTY = IFULL + IR, SBAR = IEMPTY + IR, PBAR = SBAR + 2, XBAR = PBAR + 4, OBAR = XBAR + 2,
-                       QBAR = OBAR + 4, FIN = QBAR + 1, END = FIN + 1, K8FULL = END + 1, K8EMPTY = K8FULL + NRAW,
-                       V8FULL = K8EMPTY + NRAW, V8EMPTY = V8FULL + NRAW, NBAR = V8EMPTY + NRAW;
+                       QBAR = OBAR + 4, QMX = QBAR + 1, FIN = QMX + 1, END = FIN + 1, K8FULL = END + 1,
+                       K8EMPTY = K8FULL + NRK, V8FULL = K8EMPTY + NRK, V8EMPTY = V8FULL + NRV, NBAR = V8EMPTY + NRV;
   // XCHG: the two halves' (running max, sum) of every row, swapped once per item, [128 rows][2 halves].
-  static constexpr int K_OFF = 0, V_OFF = NST * TILE, K8_OFF = 2 * NST * TILE, V8_OFF = K8_OFF + NRAW * RAW,
-                       Q_OFF = V8_OFF + NRAW * RAW, XCHG_OFF = Q_OFF + QBYTES, BAR_OFF = XCHG_OFF + ROWS * 2 * 8,
+  // QMX (fp8): the two halves' Q row maxima, [128 rows][2 halves].  fp8 Q: the high E4M3 part at
+  // Q_OFF, the low part at Q_OFF + ROWS * 128 (one 128-byte row per query row).
+  static constexpr int K_OFF = 0, V_OFF = NSK * TILE, K8_OFF = (NSK + NST) * TILE, V8_OFF = K8_OFF + NRK * RAW,
+                       Q_OFF = V8_OFF + NRV * RAW, XCHG_OFF = Q_OFF + QBYTES, QMX_OFF = XCHG_OFF + ROWS * 2 * 8,
+                       BAR_OFF = QMX_OFF + (F8 ? ROWS * 2 * 4 : 0),
                        DESC_OFF = BAR_OFF + (8 * NBAR + 63) / 64 * 64;
   static constexpr int SMEM = 1024 + DESC_OFF + IR * 64;
   static constexpr int THREADS = 32 * (S_WARP + 1 + CONV_WARPS);
@@ -131,7 +138,7 @@ PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity, const long long* wl) {
 // shared-prefix group tile; head kv_head * g + r % g): head dims [hf * D / 2, (hf + 1) * D / 2)
 // into the shared-memory Q tile, laid out as a K tile (64-dim column slabs of 128-byte rows,
 // 16-byte chunk c of row r at c ^ (r & 7)).  Rows past R are zero.
-template <int D, bool TO_F16 = false>
+template <int D>
 PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_smem, int r, int hf) {
   using T = TcCfg<D>;
   const bool valid = r < R;
@@ -142,21 +149,14 @@ PKV_DEVICE void tc_stage_q(const AttnArgs& a, const TcDesc& d, int R, uint32_t q
       hf * (D / 2));
 #pragma unroll
   for (int j = 0; j < D / 16; ++j) {
-    uint4 v = valid ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
-    if constexpr (TO_F16) {
-      // bf16 queries for f16 MMAs (fp8 pools): exact for |q| in [2^-14, 65504].
-      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        w[k] = pack_f16x2(bf16_bits_to_float(uint16_t(w[k] & 0xffff)), bf16_bits_to_float(uint16_t(w[k] >> 16)));
-    }
+    const uint4 v = valid ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
     const int dim0 = hf * (D / 2) + 8 * j;
     const int c = (dim0 % 64) / 8;
     sts128(q_smem + uint32_t(dim0 / 64) * T::SLAB + uint32_t(r) * 128 + (uint32_t(c ^ (r & 7)) << 4), v);
   }
 }
 
-// S[128 x TK] = Q K^T, one thread: D/16 MMAs of K = 16, A (Q) and B (K) both K-major in shared
+// S[128 x TK] = Q K^T (16-bit pools), one thread: D/16 MMAs of K = 16, A (Q) and B (K) both K-major in shared
 // memory with the 128-byte swizzle: 8-row groups 1024 bytes apart, the k-step moving 32 bytes
 // inside a 128-byte row, then to the next 64-element column slab.
 template <int D, bool BF>
@@ -184,6 +184,75 @@ PKV_DEVICE void tc_mma_o(uint32_t o_tmem, uint32_t p_tmem, uint32_t vbase, bool 
     const uint64_t bd = tc::smem_desc(vbase + ks * 2048, T::SLAB, 1024, tc::SW128);
     tc::mma_ts(o_tmem, p_tmem + 8 * ks, bd, IDESC, accumulate || ks > 0);
   }
+}
+
+// S[128 x TK] = (Q_hi + Q_lo) K^T for fp8 pools, one thread: kind::f8f6f4 MMAs of K = 32, A (the
+// high, then the low E4M3 part of Q) and B (the raw K codes) K-major in shared memory with the
+// 128-byte swizzle (one 128-byte row per query row / key), the k-step moving 32 bytes.
+PKV_DEVICE void tc_mma_s_f8(uint32_t s_tmem, uint32_t qhi, uint32_t qlo, uint32_t kbase) {
+  constexpr uint32_t IDESC = tc::idesc_f8(128, PKV_TC_TILE_KEYS);
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const uint64_t bd = tc::smem_desc(kbase + ks * 32, 16, 1024, tc::SW128);
+    tc::mma_ss_f8(s_tmem, tc::smem_desc(qhi + ks * 32, 16, 1024, tc::SW128), bd, IDESC, ks > 0);
+    tc::mma_ss_f8(s_tmem, tc::smem_desc(qlo + ks * 32, 16, 1024, tc::SW128), bd, IDESC, true);
+  }
+}
+
+// fp8 pools: half hf of row r of the item's Q (64 of the 128 head dims, bf16 or f16) into the high
+// and low E4M3 tiles.  The two halves swap their maxima (barrier QMX, bounded wait) and both use
+// the row scale 2^(7 - e), e = floor(log2 max|q|), which puts the row maximum in [128, 256);
+// high = E4M3(q s), low = E4M3(q s - high), each with round to nearest.  qs_inv = 1 / s.  Rows past
+// R are zero.  Returns false when the wait runs out.
+template <bool BF>
+PKV_DEVICE bool tc_stage_q_f8(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_smem, float* qmx, uint32_t qmx_bar,
+                              int qm, int r, int hf, const long long* wl, float& qs_inv) {
+  const bool valid = r < R;
+  const int i = valid ? r / a.g : 0;
+  const int64_t token = d.pos0 <= -2 ? int64_t(__ldg(a.row_tokens + (-2 - d.pos0) + i)) : int64_t(d.q_begin) + i;
+  const uint4* src = reinterpret_cast<const uint4*>(
+      static_cast<const uint16_t*>(a.q) + (token * a.hq + d.kv_head * a.g + (valid ? r % a.g : 0)) * 128 + hf * 64);
+  float x[64];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint4 v = valid ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint16_t lo = uint16_t(w[k] & 0xffff), hi = uint16_t(w[k] >> 16);
+      x[8 * j + 2 * k] = BF ? bf16_bits_to_float(lo) : __half2float(__ushort_as_half(lo));
+      x[8 * j + 2 * k + 1] = BF ? bf16_bits_to_float(hi) : __half2float(__ushort_as_half(hi));
+    }
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int j = 0; j < 64; ++j) m = fmaxf(m, fabsf(x[j]));
+  qmx[r * 2 + hf] = m;
+  mbar_arrive(qmx_bar, 1);
+  if (!mbar_wait(qmx_bar, uint32_t(qm & 1), wl)) return false;
+  m = fmaxf(m, qmx[r * 2 + (hf ^ 1)]);
+  int e = m > 0.f ? int((__float_as_uint(m) >> 23) & 0xff) - 127 : 7;  // floor(log2 m) for normal m
+  e = max(-119, min(e, 134));  // 2^(7 - e) and its inverse stay normal floats
+  const float sc = __uint_as_float(uint32_t(127 + 7 - e) << 23);
+  qs_inv = __uint_as_float(uint32_t(127 - 7 + e) << 23);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {  // 16-dim chunk 4 hf + c of the 128-byte row
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float* v = x + 16 * c + 4 * k;
+      const uint32_t h01 = e4m3x2_rn(v[0] * sc, v[1] * sc), h23 = e4m3x2_rn(v[2] * sc, v[3] * sc);
+      const float2 b01 = e4m3x2_to_float2(h01), b23 = e4m3x2_to_float2(h23);
+      const uint32_t l01 = e4m3x2_rn(v[0] * sc - b01.x, v[1] * sc - b01.y);
+      const uint32_t l23 = e4m3x2_rn(v[2] * sc - b23.x, v[3] * sc - b23.y);
+      hw[k] = h01 | (h23 << 16);
+      lw[k] = l01 | (l23 << 16);
+    }
+    const uint32_t off = uint32_t(r) * 128 + (uint32_t((4 * hf + c) ^ (r & 7)) << 4);
+    sts128(q_smem + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+    sts128(q_smem + 128 * 128 + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+  }
+  return true;
 }
 
 // E4M3 codes of one 16-byte chunk -> 16 f16 values (x 2^-8), in order, as two 16-byte pieces.
@@ -225,19 +294,24 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
   // nothing that kernel writes (and waits for it before finishing, below).
   if (warp == 0) tc::alloc(smem_addr(&s_tmem), T::TMEM_COLS);
   if (tid == 32) {
-    for (int i = 0; i < T::NST; ++i) {
-      // F8: the f16 tiles are filled by the converter threads, not by TMA.
-      mbar_init(bar(T::KFULL + i), F8 ? T::CONV_THREADS : 1);
+    for (int i = 0; i < T::NSK; ++i) {
+      mbar_init(bar(T::KFULL + i), 1);
       mbar_init(bar(T::KEMPTY + i), 1);
+    }
+    for (int i = 0; i < T::NST; ++i) {
+      // F8: the f16 V tiles are filled by the converter threads, not by TMA.
       mbar_init(bar(T::VFULL + i), F8 ? T::CONV_THREADS : 1);
       mbar_init(bar(T::VEMPTY + i), 1);
     }
-    for (int i = 0; i < T::NRAW; ++i) {
+    for (int i = 0; i < T::NRK; ++i) {
       mbar_init(bar(T::K8FULL + i), 1);
-      mbar_init(bar(T::K8EMPTY + i), T::CONV_THREADS);
+      mbar_init(bar(T::K8EMPTY + i), 1);  // released by the S MMAs' commit
+    }
+    for (int i = 0; i < T::NRV; ++i) {
       mbar_init(bar(T::V8FULL + i), 1);
       mbar_init(bar(T::V8EMPTY + i), T::CONV_THREADS);
     }
+    mbar_init(bar(T::QMX), T::SM_THREADS);
     for (int i = 0; i < T::IR; ++i) {
       mbar_init(bar(T::IFULL + i), 1);
       mbar_init(bar(T::IEMPTY + i), T::CONSUMER_WARPS);
@@ -341,13 +415,13 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
         }
         const int row0 = box_rows == T::TK ? (key0 & bmask) : 0;
         // The ring the TMA fills: the f16 tiles, or for fp8 pools the raw tiles.
-        constexpr int NS = F8 ? T::NRAW : T::NST;
+        constexpr int NSKR = F8 ? T::NRK : T::NSK, NSVR = F8 ? T::NRV : T::NST;
         constexpr int FULL_K = F8 ? T::K8FULL : T::KFULL, EMPTY_K = F8 ? T::K8EMPTY : T::KEMPTY;
         constexpr int FULL_V = F8 ? T::V8FULL : T::VFULL, EMPTY_V = F8 ? T::V8EMPTY : T::VEMPTY;
-        const int stg = q % NS;
-        const uint32_t par = ((q / NS) & 1) ^ 1;
         const uint32_t bytes = F8 ? uint32_t(nb) * box_rows * D : uint32_t(nb) * T::HALVES * box_rows * 128;
         for (int kv = 0; kv < 2; ++kv) {  // K tile, then V tile
+          const int ns = kv ? NSVR : NSKR, stg = q % ns;
+          const uint32_t par = ((q / ns) & 1) ^ 1;
           int f = 1;
           if (lane == 0) {
             f = (!s_abort && mbar_wait(bar((kv ? EMPTY_V : EMPTY_K) + stg), par, &s_wl)) ? 1 : 0;
@@ -376,13 +450,11 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
       report(a.status, PKV_DEV_TIMEOUT);
       s_abort = 1;
       // Let loads already issued land before the CTA's shared memory goes away.
-      constexpr int NS = F8 ? T::NRAW : T::NST;
+      constexpr int NSKR = F8 ? T::NRK : T::NSK, NSVR = F8 ? T::NRV : T::NST;
       constexpr int FULL_K = F8 ? T::K8FULL : T::KFULL, FULL_V = F8 ? T::V8FULL : T::VFULL;
-      if (k_armed) mbar_wait(bar(FULL_K + q % NS), (q / NS) & 1, &s_wl);
-      for (int k = 1; k <= NS && q - k >= 0; ++k) {
-        mbar_wait(bar(FULL_K + (q - k) % NS), ((q - k) / NS) & 1, &s_wl);
-        mbar_wait(bar(FULL_V + (q - k) % NS), ((q - k) / NS) & 1, &s_wl);
-      }
+      if (k_armed) mbar_wait(bar(FULL_K + q % NSKR), (q / NSKR) & 1, &s_wl);
+      for (int k = 1; k <= NSKR && q - k >= 0; ++k) mbar_wait(bar(FULL_K + (q - k) % NSKR), ((q - k) / NSKR) & 1, &s_wl);
+      for (int k = 1; k <= NSVR && q - k >= 0; ++k) mbar_wait(bar(FULL_V + (q - k) % NSVR), ((q - k) / NSVR) & 1, &s_wl);
     }
     return;
   }
@@ -390,8 +462,8 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
   if constexpr (F8) {
     if (warp >= T::CONV_WARP0) {
       // ------------------------------------------- fp8 converters (warps 11, 12)
-      // Tile qq: raw stage qq % NRAW (filled by TMA) -> f16 stage qq % NST (free once the S or
-      // P V MMAs of tile qq - NST have completed).  Chunk c (16 codes: dims 16c .. 16c+15) of
+      // V of tile qq: raw stage qq % NRV (filled by TMA) -> f16 stage qq % NST (free once the P V
+      // MMAs of tile qq - NST have completed).  Chunk c (16 codes: dims 16c .. 16c+15) of
       // key row r sits at (c ^ (r & 7)) in the raw row (128-byte swizzle); its 16 f16 values go
       // to the 16-byte chunks 2(c % 4) and +1 of column slab c / 4, swizzled the same way.
       const int ct = tid - 32 * T::CONV_WARP0;
@@ -410,9 +482,9 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
         if (d.state == 1) continue;
         for (int t = 0; t < d.ntiles && ok; ++t) {
           const int qq = q + t;
-          for (int kv = 0; kv < 2 && ok; ++kv) {
-            const int s8 = qq % T::NRAW, s16 = qq % T::NST;
-            go = !s_abort && warp_wait(bar((kv ? T::V8FULL : T::K8FULL) + s8), (qq / T::NRAW) & 1, &s_wl);
+          for (int kv = 1; kv < 2 && ok; ++kv) {  // V only: S reads the raw K codes
+            const int s8 = qq % T::NRV, s16 = qq % T::NST;
+            go = !s_abort && warp_wait(bar((kv ? T::V8FULL : T::K8FULL) + s8), (qq / T::NRV) & 1, &s_wl);
             if (go) go = warp_wait(bar((kv ? T::VEMPTY : T::KEMPTY) + s16), ((qq / T::NST) & 1) ^ 1, &s_wl);
             if (!go) { ok = false; break; }
             const uint32_t src = (kv ? v8ring : k8ring) + s8 * T::RAW, dst = (kv ? vring : kring) + s16 * T::TILE;
@@ -476,12 +548,23 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
               good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
               if (good) good = !s_abort && mbar_wait(bar(T::OBAR + 2 + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
             }
-            if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1, &s_wl);
-            if (!good) break;
-            tc::fence_after_sync();
-            tc_mma_s<D, MBF>(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, kring + stg * T::TILE);
-            tc::commit(bar(T::SBAR + (qq & 1)));
-            tc::commit(bar(T::KEMPTY + stg));
+            if constexpr (F8) {
+              const int s8 = qq % T::NRK;
+              if (good) good = !s_abort && mbar_wait(bar(T::K8FULL + s8), (qq / T::NRK) & 1, &s_wl);
+              if (!good) break;
+              tc::fence_after_sync();
+              tc_mma_s_f8(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, base + T::Q_OFF + T::ROWS * 128,
+                          k8ring + s8 * T::RAW);
+              tc::commit(bar(T::SBAR + (qq & 1)));
+              tc::commit(bar(T::K8EMPTY + s8));
+            } else {
+              if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1, &s_wl);
+              if (!good) break;
+              tc::fence_after_sync();
+              tc_mma_s<D, MBF>(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, kring + stg * T::TILE);
+              tc::commit(bar(T::SBAR + (qq & 1)));
+              tc::commit(bar(T::KEMPTY + stg));
+            }
           }
         } else {
           for (int t = 0; t < n && good; ++t) {
@@ -532,6 +615,7 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
   const uint32_t s_tm = tmem + lane_base + T::S_COL + hf * T::HALF;  // + S buffer offset: this half's S, then its P
   float2* xchg = reinterpret_cast<float2*>(base_ptr + T::XCHG_OFF);
   int q = 0, it_seq = 0, xc = 0;  // xc: items exchanged so far (barrier XBAR + (xc & 1), parity (xc >> 1) & 1)
+  int qm = 0;                     // fp8: Q row maxima swapped so far (barrier QMX, parity qm & 1)
   bool ok = true;
   for (;;) {
     const int slot = it_seq % T::IR;
@@ -549,8 +633,9 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
     float vfac = 1.f;                    // output factor: the V scale of fp8 tiles
     if constexpr (F8) {
-      // The widened tiles hold code values x 2^-8: the power of two goes back with the scales.
-      c *= __ldg(a.k_scale + a.layer * a.hkv + d.kv_head) * 256.f;
+      // S comes from the raw K codes (times the row scale of Q, taken back below); the widened V
+      // tiles hold code values x 2^-8, whose power of two goes back with the V scale.
+      c *= __ldg(a.k_scale + a.layer * a.hkv + d.kv_head);
       vfac = __ldg(a.v_scale + a.layer * a.hkv + d.kv_head) * 256.f;
     }
     const bool to_part = d.part_row >= 0;
@@ -559,7 +644,18 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     const int lo = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / a.g : -1);
 
     // The previous item's MMAs are complete (its epilogue waited for its last P V): Q is free.
-    tc_stage_q<D, F8 && BF>(a, d, R, base + T::Q_OFF, r, hf);
+    if constexpr (F8) {
+      float qs_inv = 1.f;
+      if (!tc_stage_q_f8<BF>(a, d, R, base + T::Q_OFF, reinterpret_cast<float*>(base_ptr + T::QMX_OFF), bar(T::QMX),
+                             qm, r, hf, &s_wl, qs_inv)) {
+        ok = false;
+        break;
+      }
+      ++qm;
+      c *= qs_inv;
+    } else {
+      tc_stage_q<D>(a, d, R, base + T::Q_OFF, r, hf);
+    }
     fence_proxy_async_smem();  // read by the tensor core
     tc::fence_before_sync();   // the previous item's tensor-memory reads, before its next MMAs
     mbar_arrive(bar(T::QBAR), 1);
