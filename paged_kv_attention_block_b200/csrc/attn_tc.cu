@@ -15,7 +15,7 @@
 //              completion counted on mbarriers.  No load uses cluster multicast.
 //   warps 11, 12 (fp8 pools only) converters: TMA lands the one-byte codes in
 //              raw rings; S reads the K codes as they are (kind::f8f6f4, with Q
-//              split into high and low E4M3 parts), and these warps widen the V
+//              split into a high E4M3 and a low E5M2 part), and these warps widen the V
 //              codes exactly into the f16 tiles the P V MMAs read.
 //   warps 9, 10 MMA issuers (one thread each): warp 10 issues S = Q K^T into one
 //              of two tensor-memory S buffers, as soon as the tile's K has landed
@@ -60,8 +60,7 @@ namespace pkv {
 
 // F8: fp8 (E4M3) pools, d 128.  Their tiles arrive by TMA as one-byte codes in raw rings (NRK
 // stages of K, NRV of V).  S = Q K^T runs on kind::f8f6f4 straight from the raw K tiles, with Q
-// split per row into a high and a low E4M3 part after a power-of-two row scale (together they
-// hold Q's 8 significant bits); two converter warps widen each V tile into the f16 tile of the
+// split per row into a high E4M3 and a low E5M2 part after a power-of-two row scale; two converter warps widen each V tile into the f16 tile of the
 // P V ring (value x 2^-8, exact).  The row scale and the K scale fold into the softmax scale, the
 // power of two and the V scale into the output.
 template <int D, bool F8 = false>
@@ -77,7 +76,8 @@ struct TcCfg {
   static constexpr int NSK = F8 ? 0 : NST;       // f16 K stages (fp8: S reads the raw codes)
   static constexpr int RAW = F8 ? TK * D : 0;    // one fp8 K or V tile: 128 keys x D bytes
   static constexpr int NRK = F8 ? 4 : 0, NRV = F8 ? 2 : 0;  // raw K and V stages
-  static constexpr int QBYTES = ROWS * D * 2;    // the item's Q tile (K-major, 128-byte swizzle)
+  // the item's Q tile (K-major, 128-byte swizzle); fp8: up to three one-byte parts of it
+  static constexpr int QBYTES = F8 ? 3 * ROWS * D : ROWS * D * 2;
   static constexpr int IR = 4;                   // item descriptor slots
   // mbarrier indices
   // Warp roles: 0-7 softmax (two threads per row), 8 TMA producer, 9 P V issuer, 10 S issuer,
@@ -98,7 +98,8 @@ struct TcCfg {
                        K8EMPTY = K8FULL + NRK, V8FULL = K8EMPTY + NRK, V8EMPTY = V8FULL + NRV, NBAR = V8EMPTY + NRV;
   // XCHG: the two halves' (running max, sum) of every row, swapped once per item, [128 rows][2 halves].
   // QMX (fp8): the two halves' Q row maxima, [128 rows][2 halves].  fp8 Q: the high E4M3 part at
-  // Q_OFF, the low part at Q_OFF + ROWS * 128 (one 128-byte row per query row).
+  // Q_OFF, the low E5M2 part at Q_OFF + ROWS * 128 and (f16 queries) the middle E4M3 part at
+  // Q_OFF + 2 * ROWS * 128 (one 128-byte row per query row each).
   static constexpr int K_OFF = 0, V_OFF = NSK * TILE, K8_OFF = (NSK + NST) * TILE, V8_OFF = K8_OFF + NRK * RAW,
                        Q_OFF = V8_OFF + NRV * RAW, XCHG_OFF = Q_OFF + QBYTES, QMX_OFF = XCHG_OFF + ROWS * 2 * 8,
                        BAR_OFF = QMX_OFF + (F8 ? ROWS * 2 * 4 : 0),
@@ -186,23 +187,33 @@ PKV_DEVICE void tc_mma_o(uint32_t o_tmem, uint32_t p_tmem, uint32_t vbase, bool 
   }
 }
 
-// S[128 x TK] = (Q_hi + Q_lo) K^T for fp8 pools, one thread: kind::f8f6f4 MMAs of K = 32, A (the
-// high, then the low E4M3 part of Q) and B (the raw K codes) K-major in shared memory with the
-// 128-byte swizzle (one 128-byte row per query row / key), the k-step moving 32 bytes.
-PKV_DEVICE void tc_mma_s_f8(uint32_t s_tmem, uint32_t qhi, uint32_t qlo, uint32_t kbase) {
-  constexpr uint32_t IDESC = tc::idesc_f8(128, PKV_TC_TILE_KEYS);
+// S[128 x TK] = (Q_hi + Q_lo [+ Q_mid]) K^T for fp8 pools, one thread: kind::f8f6f4 MMAs of K = 32,
+// A (the high E4M3, the low E5M2 and, for f16 queries, the middle E4M3 part of Q) and B (the raw K
+// codes) K-major in shared memory with the 128-byte swizzle (one 128-byte row per query row / key),
+// the k-step moving 32 bytes.
+template <bool BF>
+PKV_DEVICE void tc_mma_s_f8(uint32_t s_tmem, uint32_t qbase, uint32_t kbase) {
+  constexpr uint32_t IDESC_E4 = tc::idesc_f8(128, PKV_TC_TILE_KEYS, 0), IDESC_E5 = tc::idesc_f8(128, PKV_TC_TILE_KEYS, 1);
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
     const uint64_t bd = tc::smem_desc(kbase + ks * 32, 16, 1024, tc::SW128);
-    tc::mma_ss_f8(s_tmem, tc::smem_desc(qhi + ks * 32, 16, 1024, tc::SW128), bd, IDESC, ks > 0);
-    tc::mma_ss_f8(s_tmem, tc::smem_desc(qlo + ks * 32, 16, 1024, tc::SW128), bd, IDESC, true);
+    tc::mma_ss_f8(s_tmem, tc::smem_desc(qbase + ks * 32, 16, 1024, tc::SW128), bd, IDESC_E4, ks > 0);
+    tc::mma_ss_f8(s_tmem, tc::smem_desc(qbase + 128 * 128 + ks * 32, 16, 1024, tc::SW128), bd, IDESC_E5, true);
+    if constexpr (!BF)
+      tc::mma_ss_f8(s_tmem, tc::smem_desc(qbase + 2 * 128 * 128 + ks * 32, 16, 1024, tc::SW128), bd, IDESC_E4, true);
   }
 }
 
-// fp8 pools: half hf of row r of the item's Q (64 of the 128 head dims, bf16 or f16) into the high
-// and low E4M3 tiles.  The two halves swap their maxima (barrier QMX, bounded wait) and both use
-// the row scale 2^(7 - e), e = floor(log2 max|q|), which puts the row maximum in [128, 256);
-// high = E4M3(q s), low = E4M3(q s - high), each with round to nearest.  qs_inv = 1 / s.  Rows past
+// fp8 pools: half hf of row r of the item's Q (64 of the 128 head dims, bf16 or f16) into its
+// one-byte parts.  The two halves swap their maxima (barrier QMX, bounded wait) and both use the row
+// scale 2^(7 - e), e = floor(log2 max|q|), which puts the row maximum in [128, 256).  bf16: high =
+// E4M3(q s), low = E5M2(q s - high); f16: high = E4M3(q s), middle = E4M3(q s - high), low =
+// E5M2(q s - high - middle); every rounding to nearest.  The parts sum to q s exactly: after the
+// high part (4 significant bits) the residual of a bf16 q is an integer of at most 8 in units of its
+// last place, which E5M2 holds; an f16 q leaves up to 64 units, of which the middle part takes all
+// but at most 2.  That holds for entries down to 2^-16 of the row maximum, and the low part's
+// subnormals still carry entries down to 2^-23 (an E4M3 low part stops at 2^-16: on rows spanning
+// many binades that moved the log-sum-exp by 1e-2, and a two-part f16 q moved it by 2).  qs_inv = 1 / s.  Rows past
 // R are zero.  Returns false when the wait runs out.
 template <bool BF>
 PKV_DEVICE bool tc_stage_q_f8(const AttnArgs& a, const TcDesc& d, int R, uint32_t q_smem, float* qmx, uint32_t qmx_bar,
@@ -237,20 +248,29 @@ PKV_DEVICE bool tc_stage_q_f8(const AttnArgs& a, const TcDesc& d, int R, uint32_
   qs_inv = __uint_as_float(uint32_t(127 - 7 + e) << 23);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {  // 16-dim chunk 4 hf + c of the 128-byte row
-    uint32_t hw[4], lw[4];
+    uint32_t hw[4], lw[4], mw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float* v = x + 16 * c + 4 * k;
-      const uint32_t h01 = e4m3x2_rn(v[0] * sc, v[1] * sc), h23 = e4m3x2_rn(v[2] * sc, v[3] * sc);
-      const float2 b01 = e4m3x2_to_float2(h01), b23 = e4m3x2_to_float2(h23);
-      const uint32_t l01 = e4m3x2_rn(v[0] * sc - b01.x, v[1] * sc - b01.y);
-      const uint32_t l23 = e4m3x2_rn(v[2] * sc - b23.x, v[3] * sc - b23.y);
+      const uint32_t h01 = tc::e4m3x2_rn(v[0] * sc, v[1] * sc), h23 = tc::e4m3x2_rn(v[2] * sc, v[3] * sc);
+      const float2 b01 = tc::e4m3x2_to_float2(h01), b23 = tc::e4m3x2_to_float2(h23);
+      float r0 = v[0] * sc - b01.x, r1 = v[1] * sc - b01.y, r2 = v[2] * sc - b23.x, r3 = v[3] * sc - b23.y;
+      if constexpr (!BF) {
+        const uint32_t m01 = tc::e4m3x2_rn(r0, r1), m23 = tc::e4m3x2_rn(r2, r3);
+        const float2 c01 = tc::e4m3x2_to_float2(m01), c23 = tc::e4m3x2_to_float2(m23);
+        r0 -= c01.x;
+        r1 -= c01.y;
+        r2 -= c23.x;
+        r3 -= c23.y;
+        mw[k] = m01 | (m23 << 16);
+      }
       hw[k] = h01 | (h23 << 16);
-      lw[k] = l01 | (l23 << 16);
+      lw[k] = tc::e5m2x2_rn(r0, r1) | (tc::e5m2x2_rn(r2, r3) << 16);
     }
     const uint32_t off = uint32_t(r) * 128 + (uint32_t((4 * hf + c) ^ (r & 7)) << 4);
     sts128(q_smem + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
     sts128(q_smem + 128 * 128 + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+    if constexpr (!BF) sts128(q_smem + 2 * 128 * 128 + off, make_uint4(mw[0], mw[1], mw[2], mw[3]));
   }
   return true;
 }
@@ -553,8 +573,7 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
               if (good) good = !s_abort && mbar_wait(bar(T::K8FULL + s8), (qq / T::NRK) & 1, &s_wl);
               if (!good) break;
               tc::fence_after_sync();
-              tc_mma_s_f8(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, base + T::Q_OFF + T::ROWS * 128,
-                          k8ring + s8 * T::RAW);
+              tc_mma_s_f8<BF>(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, k8ring + s8 * T::RAW);
               tc::commit(bar(T::SBAR + (qq & 1)));
               tc::commit(bar(T::K8EMPTY + s8));
             } else {

@@ -60,18 +60,6 @@ PKV_DEVICE uint32_t e2m1_pair_f16x2_dyn(uint32_t w, int I) {
   const uint32_t x = w << (12 - 4 * I);
   return ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
 }
-// (x0, x1) -> two E4M3 codes, round to nearest, saturating at +-448; x0 in the low byte.
-PKV_DEVICE uint32_t e4m3x2_rn(float x0, float x1) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(x1), "f"(x0));
-  return r;
-}
-// Two E4M3 codes (low byte first) -> their values.
-PKV_DEVICE float2 e4m3x2_to_float2(uint32_t codes) {
-  uint32_t h2;
-  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(h2) : "r"(codes));
-  return make_float2(__half2float(__ushort_as_half(uint16_t(h2 & 0xffff))), __half2float(__ushort_as_half(uint16_t(h2 >> 16))));
-}
 constexpr uint32_t kF16Pow2_15x2 = 0x78007800u;  // f16x2 (2^15, 2^15)
 // f16x2 product, round to nearest (exact for the scaled E2M1 and E4M3 values multiplied here).
 PKV_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {

@@ -41,9 +41,28 @@ PKV_DEVICE void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_
       : "memory");
 }
 
-// kind::f8f6f4 instruction descriptor: f32 accumulate, A and B both E4M3 (format 0), K-major.
-__host__ __device__ constexpr uint32_t idesc_f8(int M, int N) {
-  return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+// (x0, x1) -> two E4M3 codes, round to nearest, saturating at +-448; x0 in the low byte.
+PKV_DEVICE uint32_t e4m3x2_rn(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+// (x0, x1) -> two E5M2 codes, round to nearest, saturating at +-57344; x0 in the low byte.
+PKV_DEVICE uint32_t e5m2x2_rn(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+// Two E4M3 codes (low byte first) -> their values.
+PKV_DEVICE float2 e4m3x2_to_float2(uint32_t codes) {
+  uint32_t h2;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(h2) : "r"(codes));
+  return make_float2(__half2float(__ushort_as_half(uint16_t(h2 & 0xffff))), __half2float(__ushort_as_half(uint16_t(h2 >> 16))));
+}
+// kind::f8f6f4 instruction descriptor: f32 accumulate, B E4M3 (format 0), A E4M3 (0) or E5M2 (1),
+// both K-major.
+__host__ __device__ constexpr uint32_t idesc_f8(int M, int N, uint32_t a_format = 0) {
+  return (1u << 4) | (a_format << 7) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T on 8-bit operands (kind::f8f6f4, K = 32), issued by one thread.

@@ -181,6 +181,24 @@ def test_side_by_side(pkv, kind, ctas):
     assert PD.decode(plan.buffer)["header"]["flags"] == 1
 
 
+@pytest.mark.parametrize("q_dtype", ["bf16", "f16"])
+def test_fp8_prefill_wide_query_rows(pkv, q_dtype):
+    """fp8 prefill tiles (S on kind::f8f6f4 with each query row scaled by a power of two and split
+    into high and low E4M3 parts): rows whose entries span many binades (a few large, most small,
+    some exactly zero, whole rows zero) still match the oracle, and so does their LSE."""
+    w = W.build("wideq", seed=41, kv_dtype="e4m3", q_dtype=q_dtype, kv_in_dtype="f32", num_q_heads=32,
+                num_kv_heads=8, head_dim=128, block_size=16, seq_lens=[700, 300, 90], q_lens=[160, 300, 1])
+    r = np.random.default_rng(42)
+    x = r.standard_normal((w.total_q, w.num_q_heads, w.head_dim)).astype(np.float32)
+    x *= np.float32(2.0) ** r.integers(-12, 4, size=x.shape).astype(np.float32)  # 16 binades per row
+    x[r.random(x.shape) < 0.1] = 0.0
+    x[::7, 3] = 0.0  # whole rows of zeros
+    x[::5, :, 17] *= 200.0  # a large entry sets the row scale
+    w._q = W.to_storage(x, q_dtype)
+    plan, _ = run_case(pkv, w)
+    assert plan.info["num_tc_items"] > 0
+
+
 @pytest.mark.parametrize("ctas", [1, 2, 5])
 def test_few_ctas_prefill_fp8(pkv, ctas):
     """fp8 prefill tiles on the tcgen05 kernel with few CTAs: the raw-code and f16 rings and the
