@@ -580,6 +580,10 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
     builder = W.NAMED[args.config]
     w = builder(seed=builder.__defaults__[0] + 1000 * rank) if rank else builder()
     plan_opts = {"kv_split": args.kv_split} if args.kv_split else {}
+    if args.num_ctas:
+        plan_opts["num_ctas"] = args.num_ctas
+    if args.tc_num_ctas:
+        plan_opts["tc_num_ctas"] = args.tc_num_ctas
     peak, peak_kind = peaks()
     r = measure(w, args, dev, world, plan_opts, args.steps)
     head = summarise(w, r, world, peak, peak_kind)
@@ -713,6 +717,9 @@ def main():
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--config", default="llama3_8b_decode_bf16")
     ap.add_argument("--kv-split", type=int, default=0)
+    ap.add_argument("--num-ctas", type=int, default=0, help="decode-tile kernel CTAs (0: all that fit)")
+    ap.add_argument("--tc-num-ctas", type=int, default=0,
+                    help="> 0: the tcgen05 kernel side by side on this many CTAs (needs --num-ctas); < 0: never")
     ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference sample")
     ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample (default all)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline oracle timing")

@@ -36,9 +36,9 @@ namespace {
 // Side-by-side estimate, measured on B200: the tensor-memory tiles' rate per CTA (16-bit and fp8
 // pools, causal chunks), the decode-tile kernel's stream rate per SM (16-bit, fp8 pools) and the whole HBM stream, the
 // fixed cost of a decode item per CTA, and the least gain that makes the plan run side by side.
-constexpr double kTcFlopsPerSm = 4.5e12, kTcFp8FlopsPerSm = 3.3e12;
+constexpr double kTcFlopsPerSm = 4.5e12, kTcFp8FlopsPerSm = 3.6e12;
 constexpr double kRegBytesPerSm = 75e9, kRegFp8BytesPerSm = 45e9, kHbmBytes = 6.0e12, kRegItemSec = 1.5e-6;
-constexpr double kCorunGain = 0.92;
+constexpr double kCorunGain = 0.95;
 
 // One (query tile, key piece): every KV head h of it becomes an item (and, when the tile's
 // keys are split or it belongs to a shared-prefix group, a merge per head).
