@@ -250,6 +250,7 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   a.window = h->window;
   a.debug_flags = h->debug_flags;
   a.wait_limit = h->wait_limit_kcycles > 0 ? 1000ll * h->wait_limit_kcycles : PKV_DEFAULT_WAIT_CYCLES;
+  a.total_q = h->total_q;
   if (kernels_begin) {
     e = record_event(static_cast<cudaEvent_t>(kernels_begin), st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));

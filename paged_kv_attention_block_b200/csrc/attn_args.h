@@ -33,6 +33,7 @@ struct AttnArgs {
   int32_t window;         // limited attention window (causal rows see keys pos - window < t <= pos); 0 = none
   int32_t debug_flags;    // PKV_DEBUG_* from the plan (0 in normal use)
   long long wait_limit;   // SM cycles every pipeline wait may take before it gives up
+  int32_t total_q;        // query tokens of the batch (rows of q / Hq)
   // Place among the attention kernels launched as programmatic dependents: 0 = first (waits for
   // the work ahead at its start, then lets the next kernel launch), 1 = second (launched beside
   // the first, which waited for the work ahead before letting it launch; it waits for the first

@@ -12,7 +12,11 @@
 //              in a 4-slot descriptor ring and streams K and V tiles of 128 keys
 //              into two separate rings (a K stage is released as soon as S has
 //              been computed from it, a V stage once P V has), 128-byte swizzle,
-//              completion counted on mbarriers.  No load uses cluster multicast.
+//              completion counted on mbarriers.  For 16-bit pools it also loads
+//              each item's Q tile, ahead of the item, into one of two Q buffers
+//              (a TMA box per column slab; plain copies for listed tokens), so
+//              the next item's S runs during the previous item's epilogue.  No
+//              load uses cluster multicast.
 //   warps 11, 12 (fp8 pools only) converters: TMA lands the one-byte codes in
 //              raw rings; S reads the K codes as they are (kind::f8f6f4, with Q
 //              split into a high E4M3 and a low E5M2 part), and these warps widen the V
@@ -21,7 +25,7 @@
 //              of two tensor-memory S buffers, as soon as the tile's K has landed
 //              and both halves of the buffer's previous P have been consumed;
 //              warp 9 issues, for each half of the tile's keys, O_h += P_h V_h as
-//              soon as that half's P is written.  Q (staged once per item) and K
+//              soon as that half's P is written.  Q (one tile per item) and K
 //              come from shared memory, P from tensor memory, V from its ring as an
 //              MN-major operand.  Completions are signalled with tcgen05.commit on
 //              mbarriers; with two issuers one thread's commits and waits overlap
@@ -49,7 +53,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "attn_args.h"
 #include "common.cuh"
@@ -72,12 +79,14 @@ struct TcCfg {
   static constexpr int TILE = HALVES * SLAB;     // one K or V tile
   // stages of each ring (what the Q tile leaves of 224 KB): 2 (d 128), 6 (d 64); fp8: 2 of f16
   // tiles plus 1 of raw codes
-  static constexpr int NST = F8 ? 2 : (224 * 1024 - ROWS * D * 2 - 4096) / (2 * TILE);
+  static constexpr int NST = F8 ? 2 : (224 * 1024 - 2 * ROWS * D * 2 - 4096) / (2 * TILE);
   static constexpr int NSK = F8 ? 0 : NST;       // f16 K stages (fp8: S reads the raw codes)
   static constexpr int RAW = F8 ? TK * D : 0;    // one fp8 K or V tile: 128 keys x D bytes
   static constexpr int NRK = F8 ? 4 : 0, NRV = F8 ? 2 : 0;  // raw K and V stages
   // the item's Q tile (K-major, 128-byte swizzle); fp8: up to three one-byte parts of it
   static constexpr int QBYTES = F8 ? 3 * ROWS * D : ROWS * D * 2;
+  // 16-bit pools: two Q buffers, filled by the producer ahead of the item that uses them.
+  static constexpr int NQB = F8 ? 1 : 2;
   static constexpr int IR = 4;                   // item descriptor slots
   // mbarrier indices
   // Warp roles: 0-7 softmax (two threads per row), 8 TMA producer, 9 P V issuer, 10 S issuer,
@@ -94,14 +103,14 @@ struct TcCfg {
   // P and O barriers per half of the keys: PBAR + 2 h + parity, OBAR + 2 h + parity.
   static constexpr int KFULL = 0, KEMPTY = NSK, VFULL = 2 * NSK, VEMPTY = 2 * NSK + NST, IFULL = 2 * NSK + 2 * NST,
                        IEMPTY = IFULL + IR, SBAR = IEMPTY + IR, PBAR = SBAR + 2, XBAR = PBAR + 4, OBAR = XBAR + 2,
-                       QBAR = OBAR + 4, QMX = QBAR + 1, FIN = QMX + 1, END = FIN + 1, K8FULL = END + 1,
+                       QBAR = OBAR + 4, QMX = QBAR + 1, QFULL = QMX + 1, QEMPTY = QFULL + 2, FIN = QEMPTY + 2, END = FIN + 1, K8FULL = END + 1,
                        K8EMPTY = K8FULL + NRK, V8FULL = K8EMPTY + NRK, V8EMPTY = V8FULL + NRV, NBAR = V8EMPTY + NRV;
   // XCHG: the two halves' (running max, sum) of every row, swapped once per item, [128 rows][2 halves].
   // QMX (fp8): the two halves' Q row maxima, [128 rows][2 halves].  fp8 Q: the high E4M3 part at
   // Q_OFF, the low E5M2 part at Q_OFF + ROWS * 128 and (f16 queries) the middle E4M3 part at
   // Q_OFF + 2 * ROWS * 128 (one 128-byte row per query row each).
   static constexpr int K_OFF = 0, V_OFF = NSK * TILE, K8_OFF = (NSK + NST) * TILE, V8_OFF = K8_OFF + NRK * RAW,
-                       Q_OFF = V8_OFF + NRV * RAW, XCHG_OFF = Q_OFF + QBYTES, QMX_OFF = XCHG_OFF + ROWS * 2 * 8,
+                       Q_OFF = V8_OFF + NRV * RAW, XCHG_OFF = Q_OFF + NQB * QBYTES, QMX_OFF = XCHG_OFF + ROWS * 2 * 8,
                        BAR_OFF = QMX_OFF + (F8 ? ROWS * 2 * 4 : 0),
                        DESC_OFF = BAR_OFF + (8 * NBAR + 63) / 64 * 64;
   static constexpr int SMEM = 1024 + DESC_OFF + IR * 64;
@@ -127,7 +136,16 @@ static_assert(sizeof(TcDesc) == 64, "descriptor slot");
 struct TcArgs {
   AttnArgs a;
   int32_t box_rows;  // rows per TMA box: the block size, capped at one tile
+  int32_t q_tokens;  // 16-bit pools: tokens per Q box (128 / g)
 };
+
+// 3-D tiled TMA load into shared memory, completion counted on `bar` (no multicast).
+PKV_DEVICE void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 
 // Every lane waits; the warp agrees on the outcome (tcgen05.ld / st are warp-wide).
 PKV_DEVICE bool warp_wait(uint32_t bar, uint32_t parity, const long long* wl) {
@@ -292,7 +310,7 @@ PKV_DEVICE void e4m3x16_to_f16(uint4 v, uint4& lo, uint4& hi) {
 // BF: the queries are bf16 (else f16).  F8: the pool is fp8 (MMAs then run on f16 operands).
 template <int D, bool BF, bool F8>
 __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcArgs ta) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap qmap, const TcArgs ta) {
   using T = TcCfg<D, F8>;
   constexpr bool MBF = BF && !F8;  // MMA operands bf16 (else f16)
   constexpr unsigned FULL = 0xffffffffu;
@@ -345,11 +363,24 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
       mbar_init(bar(T::OBAR + i), 1);
     }
     mbar_init(bar(T::QBAR), T::SM_THREADS);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(T::QFULL + b), 1);   // the producer's arrival (with the TMA bytes, or after its copies)
+      mbar_init(bar(T::QEMPTY + b), 1);  // the S issuer's commit after the item's last S
+    }
     mbar_init(bar(T::FIN), 2);
     mbar_init(bar(T::END), T::CONSUMER_WARPS);
     s_abort = 0;
     s_wl = a.wait_limit;
     fence_mbar_init();
+  }
+  if constexpr (!F8) {
+    // Rows past the last whole group of g heads are never loaded: keep them zero (finite S).
+    const int rows_loaded = (T::ROWS / a.g) * a.g;
+    if (tid < T::ROWS && tid >= rows_loaded)
+      for (int b = 0; b < T::NQB; ++b)
+        for (int h = 0; h < T::HALVES; ++h)
+          for (int c = 0; c < 8; ++c) sts128(base + T::Q_OFF + b * T::QBYTES + h * T::SLAB + tid * 128 + c * 16, make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
   }
   // Second (behind the decode-tile kernel, whose CTAs had waited for the plan staging, and so
   // for the work before it, before triggering this launch): this grid reads nothing that kernel
@@ -373,6 +404,7 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     const int c3k = 2 * a.layer;
     int q = 0, it_seq = 0;
     bool ok = true, k_armed = false;  // k_armed: K of tile q issued, its V not yet
+    int qi = 0;                       // 16-bit pools: items whose Q this warp loaded
     int next_idx = blockIdx.x;  // first item: the CTA's own index; later ones from the counter
     for (;;) {
       const int slot = it_seq % T::IR;
@@ -411,9 +443,44 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
       }
       if (!valid && lane == 0) report(a.status, PKV_DEV_PLAN_MISMATCH);
       const int ntiles = valid ? (it.k_end - it.k_begin + T::TK - 1) / T::TK : 0;
+      int qb = 0;
+      if constexpr (!F8) {
+        if (valid) {
+          // The item's Q into buffer qi % 2, once the S MMAs of the item that used it last are
+          // done: one TMA box (TOKB tokens x g heads x 64 dims) per column slab for a run of
+          // tokens; plain copies for listed tokens.  Rows r = token r / g, head r % g.
+          qb = qi & 1;
+          int f = 1;
+          if (lane == 0) f = (!s_abort && mbar_wait(bar(T::QEMPTY + qb), ((qi >> 1) & 1) ^ 1, &s_wl)) ? 1 : 0;
+          if (!__shfl_sync(FULL, f, 0)) { ok = false; break; }
+          const uint32_t qdst = base + T::Q_OFF + qb * T::QBYTES;
+          if (it.pos0 > -2) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(bar(T::QFULL + qb), uint32_t(T::HALVES * 128 * a.g * ta.q_tokens));
+#pragma unroll
+              for (int h = 0; h < T::HALVES; ++h)
+                tma_load_3d(qdst + h * T::SLAB, &qmap, bar(T::QFULL + qb), h * 64, it.kv_head * a.g, it.q_begin);
+            }
+          } else {
+            const int R = it.n_q * a.g;
+            for (int x = lane; x < R * (D / 8); x += 32) {
+              const int r = x / (D / 8), ch = x % (D / 8), i = r / a.g;
+              const int64_t tok = __ldg(a.row_tokens + (-2 - it.pos0) + i);
+              const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+                  static_cast<const uint16_t*>(a.q) + (tok * a.hq + it.kv_head * a.g + r % a.g) * D + ch * 8));
+              sts128(qdst + uint32_t(ch / 8) * T::SLAB + uint32_t(r) * 128 + (uint32_t((ch % 8) ^ (r & 7)) << 4), v);
+            }
+            fence_proxy_async_smem();  // read by the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(T::QFULL + qb), 1);
+          }
+          ++qi;
+        }
+      }
       if (lane == 0) {
         d.seq = it.seq; d.kv_head = it.kv_head; d.q_begin = it.q_begin; d.n_q = it.n_q; d.k_begin = it.k_begin;
         d.k_end = it.k_end; d.pos0 = it.pos0; d.part_row = it.part_row; d.ntiles = ntiles; d.state = valid ? 0 : 1;
+        d.pad[0] = qb;
         mbar_arrive(bar(T::IFULL + slot), 1);
       }
       ++it_seq;
@@ -540,7 +607,7 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     // Tile qq (counted over the CTA's items) uses ring stage qq % NST, S buffer and
     // S / P / O barriers qq & 1, whose phases for that tile have parity (qq >> 1) & 1.
     const bool s_side = warp == T::S_WARP;
-    int q = 0, it_seq = 0;
+    int q = 0, it_seq = 0, qi_s = 0;  // qi_s: 16-bit items whose S this warp issued
     uint32_t q_ph = 0;
     bool ok = true;
     for (;;) {
@@ -558,13 +625,17 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
       if (lane == 0) {
         bool good = true;
         if (s_side) {
-          // Q staged means every earlier item is finished (its epilogue waited for its last P V).
-          good = !s_abort && mbar_wait(bar(T::QBAR), q_ph, &s_wl);
+          // fp8: Q staged by the softmax threads means every earlier item is finished (its
+          // epilogue waited for its last P V).  16-bit: the item's Q buffer is full.
+          if constexpr (F8) good = !s_abort && mbar_wait(bar(T::QBAR), q_ph, &s_wl);
+          else good = !s_abort && mbar_wait(bar(T::QFULL + (qi_s & 1)), (qi_s >> 1) & 1, &s_wl);
           if (good) tc::fence_after_sync();
           for (int t = 0; t < n && good; ++t) {
             const int qq = q + t, stg = qq % T::NST;
             // The buffer's previous tile: both halves of its P (in the buffer) have been read by P V.
-            if (t >= 2) {
+            // fp8: the previous item is finished (Q staged after its epilogue); 16-bit: the previous
+            // item's last tiles may still be in flight, so the wait counts tiles over items.
+            if (F8 ? t >= 2 : qq >= 2) {
               good = !s_abort && mbar_wait(bar(T::OBAR + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
               if (good) good = !s_abort && mbar_wait(bar(T::OBAR + 2 + (qq & 1)), ((qq - 2) >> 1) & 1, &s_wl);
             }
@@ -580,9 +651,11 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
               if (good) good = !s_abort && mbar_wait(bar(T::KFULL + stg), (qq / T::NST) & 1, &s_wl);
               if (!good) break;
               tc::fence_after_sync();
-              tc_mma_s<D, MBF>(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF, kring + stg * T::TILE);
+              tc_mma_s<D, MBF>(tmem + T::S_COL + (qq & 1) * T::TK, base + T::Q_OFF + (qi_s & 1) * T::QBYTES,
+                               kring + stg * T::TILE);
               tc::commit(bar(T::SBAR + (qq & 1)));
               tc::commit(bar(T::KEMPTY + stg));
+              if (t == n - 1) tc::commit(bar(T::QEMPTY + (qi_s & 1)));  // the item's Q is no longer read
             }
           }
         } else {
@@ -608,6 +681,7 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
         }
       }
       q_ph ^= 1;
+      ++qi_s;
       q += n;
       if (!__shfl_sync(FULL, ok ? 1 : 0, 0)) break;
     }
@@ -662,7 +736,8 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
     const int lim = (d.pos0 >= 0 && r < R) ? min(d.k_end, d.pos0 + r / a.g + 1) : d.k_end;
     const int lo = window_start(a.window, (d.pos0 >= 0 && r < R) ? d.pos0 + r / a.g : -1);
 
-    // The previous item's MMAs are complete (its epilogue waited for its last P V): Q is free.
+    // fp8: the previous item's MMAs are complete (its epilogue waited for its last P V): Q is
+    // free.  16-bit pools: the producer loaded Q already.
     if constexpr (F8) {
       float qs_inv = 1.f;
       if (!tc_stage_q_f8<BF>(a, d, R, base + T::Q_OFF, reinterpret_cast<float*>(base_ptr + T::QMX_OFF), bar(T::QMX),
@@ -672,12 +747,12 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
       }
       ++qm;
       c *= qs_inv;
-    } else {
-      tc_stage_q<D>(a, d, R, base + T::Q_OFF, r, hf);
     }
-    fence_proxy_async_smem();  // read by the tensor core
-    tc::fence_before_sync();   // the previous item's tensor-memory reads, before its next MMAs
-    mbar_arrive(bar(T::QBAR), 1);
+    if constexpr (F8) {
+      fence_proxy_async_smem();  // read by the tensor core
+      tc::fence_before_sync();   // the previous item's tensor-memory reads, before its next MMAs
+      mbar_arrive(bar(T::QBAR), 1);
+    }
 
     float m_run = -INFINITY, l_run = 0.f;  // running max (log2 units) and sum of this half's keys
     for (int t = 0; t < ntiles; ++t) {
@@ -859,6 +934,35 @@ __global__ void __launch_bounds__(TcCfg<D, F8>::THREADS, 1)
 
 // ---- host side -------------------------------------------------------------
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult res;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &res) == cudaSuccess &&
+        res == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// q [total_q][Hq][D] (16-bit) as a 3-D tensor (dim, head, token); boxes of 64 dims x g heads x
+// q_tokens tokens; tokens past total_q read as zeros.
+bool make_q_map(const AttnArgs& a, int head_dim, CUtensorMapDataType dt, int q_tokens, CUtensorMap* map) {
+  auto fn = q_encode_fn();
+  if (!fn || a.total_q <= 0 || q_tokens < 1 || q_tokens > 256 || a.g > 256) return false;
+  cuuint64_t dims[3] = {cuuint64_t(head_dim), cuuint64_t(a.hq), cuuint64_t(a.total_q)};
+  cuuint64_t strides[2] = {cuuint64_t(head_dim) * 2, cuuint64_t(head_dim) * 2 * a.hq};
+  cuuint32_t box[3] = {64, cuuint32_t(a.g), cuuint32_t(q_tokens)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, dt, 3, const_cast<void*>(a.q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+}  // namespace
+
 template <int D, bool BF, bool F8>
 cudaError_t launch_tc(const AttnArgs& a, int grid, cudaStream_t st) {
   using T = TcCfg<D, F8>;
@@ -867,8 +971,15 @@ cudaError_t launch_tc(const AttnArgs& a, int grid, cudaStream_t st) {
   const CUtensorMapDataType dt = F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                     : (BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   if (!make_pool_map(a, D, F8 ? 1 : 2, dt, box_rows, 1, &map)) return cudaErrorInvalidValue;
-  const cudaError_t e = launch_pdl(attn_tc_kernel<D, BF, F8>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map,
-                                   TcArgs{a, box_rows});
+  // Q as (dim, head, token), boxes of 64 dims x g heads x 128 / g tokens, 128-byte swizzle: one box
+  // lands a column slab of an item's Q tile in the layout the S MMAs read.
+  CUtensorMap qmap{};
+  const int q_tokens = T::ROWS / a.g;
+  if constexpr (!F8) {
+    if (!make_q_map(a, D, dt, q_tokens, &qmap)) return cudaErrorInvalidValue;
+  }
+  const cudaError_t e = launch_pdl(attn_tc_kernel<D, BF, F8>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, qmap,
+                                   TcArgs{a, box_rows, q_tokens});
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
