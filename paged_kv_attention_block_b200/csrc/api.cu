@@ -78,7 +78,8 @@ extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, i
 // Structural check of a host plan: every index the kernels follow stays inside
 // the plan and the workspace (lengths are checked against the device arrays by
 // the kernels themselves).
-static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_rows, bool tc) {
+// merge_rows receives the most rows of any one merge (the merge grid's y extent in 16-row chunks).
+static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_rows, bool tc, int* merge_rows) {
   const char* base = reinterpret_cast<const char*>(h);
   const uint64_t bytes = h->bytes;
   if (bytes < sizeof(PkvPlanHeader) + PKV_PLAN_COUNTER_BYTES || (bytes & 255))
@@ -126,9 +127,11 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
     return s;
   const PkvReduce* reds = reinterpret_cast<const PkvReduce*>(base + h->reduce_off);
   const int32_t* parts = reinterpret_cast<const int32_t*>(base + h->parts_off);
+  *merge_rows = 0;
   for (int i = 0; i < h->n_reduce; ++i) {
     const PkvReduce& r = reds[i];
     const int64_t rows = int64_t(r.n_q) * g;
+    *merge_rows = std::max(*merge_rows, int(std::min<int64_t>(rows, PKV_TILE_ROWS_TC)));
     if (r.n_q <= 0 || rows > PKV_TILE_ROWS_TC || r.kv_head < 0 || r.kv_head >= hkv || r.q_begin < 0 ||
         int64_t(r.q_begin) + r.n_q > h->total_q || r.parts_begin < 0 || r.n_parts < 0 ||
         int64_t(r.parts_begin) + r.n_parts > h->n_parts)
@@ -184,7 +187,9 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
     return pkv_fail(PKV_ERR_INVALID_ARG, "paged_attention: softmax_scale must be positive and finite");
   pkv::AttnKernel ktc{};
   const bool tc = pkv::attn_tc_kernel_for(c.kv_dtype, q_dtype, c.head_dim, c.block_size, &ktc);
-  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads, k.max_rows, tc); vs != PKV_OK)
+  int merge_rows = 0;
+  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads, k.max_rows, tc, &merge_rows);
+      vs != PKV_OK)
     return vs;
   const PkvWorkspaceLayout L = pkv_workspace_layout(h->bytes, h->n_part_rows, c.head_dim);
   if (h->n_items == 0 && h->n_tc_items == 0) return PKV_OK;
@@ -306,7 +311,7 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
     r.hq = num_q_heads;
     r.g = a.g;
     r.head_dim = c.head_dim;
-    e = pkv::launch_plan_reduce(r, st);
+    e = pkv::launch_plan_reduce(r, merge_rows, st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: merge launch failed: %s", cudaGetErrorString(e));
   }
   return PKV_OK;

@@ -73,7 +73,9 @@ int resident_ctas(const AttnKernel& k);
 // boxes of 128 bytes x box_rows slots x 1 head x box_kv x 1 block, 128-byte swizzle.
 bool make_pool_map(const AttnArgs& a, int head_dim, int elem, CUtensorMapDataType dt, int box_rows, int box_kv,
                    CUtensorMap* map);
-cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st);
+// The plan's merges (reduce.cu); max_rows = the most rows of any one merge, which sizes the
+// grid's y dimension in chunks of 16 rows.
+cudaError_t launch_plan_reduce(const ReduceArgs& r, int max_rows, cudaStream_t st);
 // Copy `bytes` (a multiple of 16) of a page-locked host plan, addressed through its device
 // alias, into the workspace (reduce.cu).  Launched as a programmatic dependent; the grid
 // completes only after the work ahead of it on the stream.

@@ -380,9 +380,10 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   }
 
   // 3. Key-range split and merges.
-  const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 2.0)};
+  const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 3.0)};
   // Longest key range of one item of a tile's list; the automatic length (about two items per
-  // CTA) is scaled by `mult`.
+  // CTA on the decode kernel, three on the tcgen05 kernel, whose CTAs take items in turn
+  // from a longer queue and whose merges spread over 16-row chunks) is scaled by `mult`.
   auto max_keys_for = [&](int rows, bool t, double mult) -> int32_t {
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     int64_t max_keys;

@@ -30,9 +30,11 @@ __global__ void __launch_bounds__(256) dense_reduce_kernel(const float* __restri
   }
 }
 
-// One warp per output row of a merge (a merge covers n_q tokens x g heads);
-// lane j merges head dims [VEC j, VEC (j + 1)) with the same per-element
-// arithmetic as merge_elem, so each lane issues VEC-wide loads of the parts.
+// One warp per output row of a merge (a merge covers n_q tokens x g heads; the
+// CTA at blockIdx.y takes its rows 16 y .. 16 y + 15, four a warp, so a merge of
+// 128-row partials spreads over 8 CTAs); lane j merges head dims [VEC j, VEC (j + 1))
+// with the same per-element arithmetic as merge_elem, so each lane issues VEC-wide
+// loads of the parts.
 template <int D>
 __global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
   constexpr int VEC = D / 32;
@@ -43,7 +45,8 @@ __global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
     const int R = red.n_q * a.g;
     const int32_t* parts = a.parts + red.parts_begin;
     const int n = red.n_parts;
-    for (int r = warp; r < R; r += 4) {
+    const int r_end = min(R, int(blockIdx.y) * 16 + 16);
+    for (int r = int(blockIdx.y) * 16 + warp; r < r_end; r += 4) {
       float M = -INFINITY;
       for (int i = 0; i < n; ++i) M = fmaxf(M, __ldg(a.part_lse + int64_t(__ldg(parts + i)) + r));
       float o[VEC], lse;
@@ -103,11 +106,11 @@ cudaError_t launch_plan_stage(const void* plan_dev, void* dst, uint64_t bytes, c
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_plan_reduce(const ReduceArgs& r, cudaStream_t st) {
+cudaError_t launch_plan_reduce(const ReduceArgs& r, int max_rows, cudaStream_t st) {
   if (r.n_reduce <= 0) return cudaSuccess;
-  const int grid = std::min(r.n_reduce, 148 * 16);
-  const cudaError_t e = r.head_dim == 128 ? launch_pdl(plan_reduce_kernel<128>, dim3(grid), dim3(128), 0, st, r)
-                                           : launch_pdl(plan_reduce_kernel<64>, dim3(grid), dim3(128), 0, st, r);
+  const dim3 grid(std::min(r.n_reduce, 148 * 16), std::max(1, (max_rows + 15) / 16));
+  const cudaError_t e = r.head_dim == 128 ? launch_pdl(plan_reduce_kernel<128>, grid, dim3(128), 0, st, r)
+                                           : launch_pdl(plan_reduce_kernel<64>, grid, dim3(128), 0, st, r);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
