@@ -552,7 +552,8 @@ def summarise(w, r, world, peak, peak_kind):
                 "ms_per_step": r["e2e"]["ms"]},
         "clocks": r["clocks"],
         "plan": {k: r["plan"][k] for k in ("num_items", "num_tc_items", "num_reduce", "num_partial_rows",
-                                           "num_groups", "num_ctas", "tc_num_ctas", "side_by_side")},
+                                           "num_groups", "num_ctas", "tc_num_ctas", "side_by_side",
+                                           "heads_per_item")},
         # kv_append, the plan staging kernel (the plans are page-locked), the attention kernels present
         # in the plan, the merge when the plan has one.
         "launches_per_step": 2 + (r["plan"]["num_items"] > n_tc) + (n_tc > 0) + (r["plan"]["num_reduce"] > 0),
@@ -584,6 +585,8 @@ def run_pkv(args, rank: int, world: int, local_rank: int):
         plan_opts["num_ctas"] = args.num_ctas
     if args.tc_num_ctas:
         plan_opts["tc_num_ctas"] = args.tc_num_ctas
+    if args.heads_per_item:
+        plan_opts["heads_per_item"] = args.heads_per_item
     peak, peak_kind = peaks()
     r = measure(w, args, dev, world, plan_opts, args.steps)
     head = summarise(w, r, world, peak, peak_kind)
@@ -720,6 +723,8 @@ def main():
     ap.add_argument("--num-ctas", type=int, default=0, help="decode-tile kernel CTAs (0: all that fit)")
     ap.add_argument("--tc-num-ctas", type=int, default=0,
                     help="> 0: the tcgen05 kernel side by side on this many CTAs (needs --num-ctas); < 0: never")
+    ap.add_argument("--heads-per-item", type=int, default=0,
+                    help="KV heads per decode-sized work item: 1 or 4 (0: the planner decides)")
     ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference sample")
     ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample (default all)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline oracle timing")

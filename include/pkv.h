@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define PKV_ABI_VERSION 3
+#define PKV_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define PKV_API __attribute__((visibility("default")))
@@ -235,6 +235,19 @@ typedef struct pkv_plan_request {
                                    estimate of the two kernels' times says it pays, splitting the SMs of
                                    the current device between them.  < 0: never.  Plans are the same for
                                    every layer either way. */
+  int32_t heads_per_item;       /* KV heads one decode-sized work item covers.  4: each item of the
+                                   decode-tile list takes four consecutive KV heads of one query tile
+                                   and key range, one head per consumer warp of the TMA-fed decode
+                                   kernel, so a warp runs its head over the whole range and no warps'
+                                   states are merged at the item's end (short key ranges: many small
+                                   decode requests, shared-prefix members' own suffixes).  Needs
+                                   num_kv_heads a multiple of 4, a pool the TMA-fed kernel serves
+                                   (16-bit pools with block_size >= 8, fp8 pools of head_dim 128 with
+                                   block_size >= 8, NVFP4 pools) and at most 8 rows per decode tile
+                                   (query tokens x Hq/Hkv); else UNSUPPORTED.  1: one KV head per item.
+                                   0: automatic, 4 where it applies on NVFP4 pools (instruction-bound
+                                   tiles) and, on the others, where the decode tiles' key ranges are
+                                   short against the per-CTA share of the batch. */
 } pkv_plan_request;
 
 #define PKV_DEBUG_WITHHOLD_LOADS 0x1
@@ -252,6 +265,7 @@ typedef struct pkv_plan_info {
   int32_t tc_num_ctas;          /* CTAs planned for the tcgen05 kernel */
   int32_t side_by_side;         /* 1: the two kernels run at the same time on disjoint SMs (num_ctas
                                    and tc_num_ctas CTAs); 0: one after the other */
+  int32_t heads_per_item;       /* KV heads per item of the decode-tile list (1 or 4) */
 } pkv_plan_info;
 
 /*

@@ -58,7 +58,8 @@ class _PlanRequest(C.Structure):
                 ("num_ctas", C.c_int32), ("kv_split", C.c_int32), ("cascade", C.c_int32),
                 ("min_shared_tokens", C.c_int32), ("max_blocks", C.c_int32), ("cu_q_lens", C.c_void_p),
                 ("seq_lens", C.c_void_p), ("block_tables", C.c_void_p), ("window", C.c_int32),
-                ("wait_limit_kcycles", C.c_int32), ("debug_flags", C.c_int32), ("tc_num_ctas", C.c_int32)]
+                ("wait_limit_kcycles", C.c_int32), ("debug_flags", C.c_int32), ("tc_num_ctas", C.c_int32),
+                ("heads_per_item", C.c_int32)]
 
 PKV_DEBUG_WITHHOLD_LOADS = 0x1
 
@@ -67,7 +68,7 @@ class _PlanInfo(C.Structure):
     _fields_ = [("plan_bytes", C.c_size_t), ("workspace_bytes", C.c_size_t), ("num_items", C.c_int32),
                 ("num_reduce", C.c_int32), ("num_parts", C.c_int32), ("num_partial_rows", C.c_int32),
                 ("num_groups", C.c_int32), ("num_ctas", C.c_int32), ("num_tc_items", C.c_int32),
-                ("tc_num_ctas", C.c_int32), ("side_by_side", C.c_int32)]
+                ("tc_num_ctas", C.c_int32), ("side_by_side", C.c_int32), ("heads_per_item", C.c_int32)]
 
 
 _P, _I32, _I64, _SZ, _F = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t, C.c_float
@@ -218,12 +219,16 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
                    kv_dtype: int | str, causal: bool = True, block_tables=None, max_blocks: int | None = None,
                    num_ctas: int = 0, kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0,
                    pin: bool = True, buffer: torch.Tensor | None = None, window: int = 0,
-                   wait_limit_kcycles: int = 0, debug_flags: int = 0, tc_num_ctas: int = 0) -> Plan:
+                   wait_limit_kcycles: int = 0, debug_flags: int = 0, tc_num_ctas: int = 0,
+                   heads_per_item: int = 0) -> Plan:
     """Build the work list for one paged_attention call from host copies of the lengths.
 
     ``tc_num_ctas`` > 0 runs the tcgen05 tiles side by side with the decode tiles on that many
     CTAs (``num_ctas`` > 0 then counts the decode-tile kernel's); 0 lets the planner decide
     (with ``num_ctas`` = 0); < 0 never.
+
+    ``heads_per_item`` 4 makes every decode-sized item cover four consecutive KV heads (one per
+    consumer warp of the TMA-fed decode kernel); 1 one head; 0 lets the planner decide.
 
     ``window`` > 0 limits every (causal) row to its ``window`` most recent positions; the
     plan carries it to ``paged_attention``, as it does ``wait_limit_kcycles`` (limit of every
@@ -242,7 +247,7 @@ def plan_attention(cu_q_lens, seq_lens, *, num_q_heads: int, num_kv_heads: int, 
     req = _PlanRequest(sl.shape[0], num_q_heads, num_kv_heads, head_dim, block_size, code, int(bool(causal)), num_ctas,
                        kv_split, int(bool(cascade)), min_shared_tokens, max_blocks, cu.ctypes.data, sl.ctypes.data,
                        None if bt is None else bt.ctypes.data, int(window), int(wait_limit_kcycles), int(debug_flags),
-                       int(tc_num_ctas))
+                       int(tc_num_ctas), int(heads_per_item))
     info = _PlanInfo()
     # With a buffer given, plan straight into it (one call); only a buffer too small costs a
     # size query and a new buffer.
@@ -274,7 +279,7 @@ class Planner:
                  head_dim: int, block_size: int, kv_dtype: int | str, causal: bool = True, num_ctas: int = 0,
                  kv_split: int = 0, cascade: bool = True, min_shared_tokens: int = 0, window: int = 0,
                  max_blocks: int | None = None, wait_limit_kcycles: int = 0, debug_flags: int = 0,
-                 tc_num_ctas: int = 0):
+                 tc_num_ctas: int = 0, heads_per_item: int = 0):
         self.cu_q_lens = self._host(cu_q_lens)
         self.seq_lens = self._host(seq_lens)
         self.block_tables = None if block_tables is None else self._host(block_tables)
@@ -285,7 +290,8 @@ class Planner:
                                  int(bool(causal)), num_ctas, kv_split, int(bool(cascade)), min_shared_tokens,
                                  max_blocks, self.cu_q_lens.ctypes.data, self.seq_lens.ctypes.data,
                                  None if self.block_tables is None else self.block_tables.ctypes.data, int(window),
-                                 int(wait_limit_kcycles), int(debug_flags), int(tc_num_ctas))
+                                 int(wait_limit_kcycles), int(debug_flags), int(tc_num_ctas),
+                                 int(heads_per_item))
         self._req_ref = C.byref(self._req)
         self._info = _PlanInfo()
         self._info_ref = C.byref(self._info)
@@ -425,7 +431,7 @@ class GraphStep:
 
     _FIELDS = ("q", "k_new", "v_new", "cu_q", "seq_lens", "start_pos", "block_tables")
     _SHAPE_KEYS = ("plan_bytes", "workspace_bytes", "num_items", "num_tc_items", "num_reduce", "num_parts",
-                   "num_partial_rows", "num_ctas", "tc_num_ctas", "side_by_side")
+                   "num_partial_rows", "num_ctas", "tc_num_ctas", "side_by_side", "heads_per_item")
 
     def __init__(self, cache: Cache, like: dict, plan_kwargs: dict, softmax_scale: float, causal: bool = True,
                  slots: int = 2, stream=None):

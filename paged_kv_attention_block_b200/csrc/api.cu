@@ -55,6 +55,8 @@ int resident_ctas(const AttnKernel& k) {
   cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess && k.smem > 48 * 1024)
     e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+  if (e == cudaSuccess && k.smem > 48 * 1024 && k.fn_heads4)
+    e = cudaFuncSetAttribute(k.fn_heads4, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
   if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, k.smem);
   if (e != cudaSuccess) return -1;
   const int n = std::max(1, sms * std::max(1, per_sm));
@@ -79,7 +81,9 @@ extern "C" pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, i
 // the plan and the workspace (lengths are checked against the device arrays by
 // the kernels themselves).
 // merge_rows receives the most rows of any one merge (the merge grid's y extent in 16-row chunks).
-static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_rows, bool tc, int* merge_rows) {
+// heads4_ok: the decode-tile kernel of this pool takes four-head items.
+static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_rows, bool tc, bool heads4_ok,
+                                int* merge_rows) {
   const char* base = reinterpret_cast<const char*>(h);
   const uint64_t bytes = h->bytes;
   if (bytes < sizeof(PkvPlanHeader) + PKV_PLAN_COUNTER_BYTES || (bytes & 255))
@@ -91,7 +95,10 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
       !inside(h->parts_off, h->n_parts, sizeof(int32_t)) || h->num_ctas <= 0 || (h->n_tc_items > 0 && h->tc_num_ctas <= 0))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan sections out of range");
   if (h->n_tc_items > 0 && !tc) return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan has tcgen05 items for a pool without that kernel");
-  if ((h->flags & ~PKV_PLAN_CORUN) != 0) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
+  if ((h->flags & ~(PKV_PLAN_CORUN | PKV_PLAN_HEADS4)) != 0) return pkv_fail(PKV_ERR_PLAN, "paged_attention: unknown plan flags");
+  const bool heads4 = (h->flags & PKV_PLAN_HEADS4) != 0;
+  if (heads4 && (!heads4_ok || hkv % 4 != 0))
+    return pkv_fail(PKV_ERR_PLAN, "paged_attention: four-head plan for a pool or head count without that kernel");
   if ((h->flags & PKV_PLAN_CORUN) != 0 && (h->n_items == 0 || h->n_tc_items == 0))
     return pkv_fail(PKV_ERR_PLAN, "paged_attention: side-by-side plan without both item lists");
   if (h->n_rows < 0 || !inside(h->rows_off, h->n_rows, sizeof(int32_t)))
@@ -113,9 +120,14 @@ static pkv_status validate_plan(const PkvPlanHeader* h, int g, int hkv, int max_
           if (tok < 0 || tok >= h->total_q) return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d lists bad tokens", what, i);
         }
       }
-      if (it.n_q <= 0 || rows < lo || rows > hi || it.kv_head < 0 || it.kv_head >= hkv || it.q_begin < 0 ||
+      // A four-head item (decode-tile list of a PKV_PLAN_HEADS4 plan) spans heads kv_head .. + 3
+      // and their partial rows.
+      const int nh = heads4 && !tc_list ? 4 : 1;
+      if (nh == 4 && (rows > PKV_HEADS4_ROWS || it.kv_head % 4 != 0))
+        return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d is not a four-head item", what, i);
+      if (it.n_q <= 0 || rows < lo || rows > hi || it.kv_head < 0 || it.kv_head + nh > hkv || it.q_begin < 0 ||
           (!listed && int64_t(it.q_begin) + it.n_q > h->total_q) || it.k_begin < 0 || it.k_begin > it.k_end ||
-          it.part_row < -1 || (it.part_row >= 0 && int64_t(it.part_row) + rows > h->n_part_rows))
+          it.part_row < -1 || (it.part_row >= 0 && int64_t(it.part_row) + nh * rows > h->n_part_rows))
         return pkv_fail(PKV_ERR_PLAN, "paged_attention: plan %s %d out of range", what, i);
     }
     return PKV_OK;
@@ -188,7 +200,8 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   pkv::AttnKernel ktc{};
   const bool tc = pkv::attn_tc_kernel_for(c.kv_dtype, q_dtype, c.head_dim, c.block_size, &ktc);
   int merge_rows = 0;
-  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads, k.max_rows, tc, &merge_rows);
+  if (pkv_status vs = validate_plan(h, num_q_heads / c.num_kv_heads, c.num_kv_heads, k.max_rows, tc,
+                                    pkv_heads4_capable(c.kv_dtype, c.head_dim, c.block_size), &merge_rows);
       vs != PKV_OK)
     return vs;
   const PkvWorkspaceLayout L = pkv_workspace_layout(h->bytes, h->n_part_rows, c.head_dim);
@@ -256,6 +269,7 @@ extern "C" pkv_status pkv_paged_attention_timed(const pkv_cache* cache, const vo
   a.debug_flags = h->debug_flags;
   a.wait_limit = h->wait_limit_kcycles > 0 ? 1000ll * h->wait_limit_kcycles : PKV_DEFAULT_WAIT_CYCLES;
   a.total_q = h->total_q;
+  a.heads4 = (h->flags & PKV_PLAN_HEADS4) ? 1 : 0;
   if (kernels_begin) {
     e = record_event(static_cast<cudaEvent_t>(kernels_begin), st);
     if (e != cudaSuccess) return pkv_fail(PKV_ERR_CUDA, "paged_attention: event record: %s", cudaGetErrorString(e));

@@ -39,6 +39,9 @@ struct AttnArgs {
   // the first, which waited for the work ahead before letting it launch; it waits for the first
   // before it finishes, so the merge after it sees both).
   int32_t pdl_role;
+  // 1: the plan's decode-tile items each cover four KV heads, kv_head .. kv_head + 3
+  // (PKV_PLAN_HEADS4); consumer warp w runs head kv_head + w.
+  int32_t heads4;
 };
 
 struct ReduceArgs {
@@ -59,6 +62,9 @@ struct AttnKernel {
   int smem;
   cudaError_t (*launch)(const AttnArgs&, int grid, cudaStream_t);
   int max_rows;  // rows per item the kernel accepts
+  // The variant for four-head plans (same threads and shared memory), launched by `launch`
+  // when AttnArgs::heads4 is set; null where there is none.
+  const void* fn_heads4 = nullptr;
 };
 // Picks the TMA kernel where it applies (block size >= 8, 128/256-byte rows),
 // else the cp.async tensor-core kernel, and the CUDA-core kernel for fp32 pools.

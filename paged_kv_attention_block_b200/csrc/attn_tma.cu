@@ -24,6 +24,12 @@
 //     MMA through movmatrix.  Fragment addresses are fixed per lane; masking
 //     runs only on tiles that reach past a row's limit.  The four warps merge
 //     their softmax states at the end of the item.
+//   * Four-head plans: each decode item covers KV heads kv_head .. kv_head + 3
+//     of one query tile and key range, and warp w runs head kv_head + w over
+//     the whole range (tile t: key tile t / 4, head t % 4).  A warp then holds
+//     its head's complete state: it normalises and writes its rows itself,
+//     with no merge between warps and no end-of-item barrier; the producer
+//     reads the item's fields and block ids once for four heads.
 //   * Tiles of more than 16 rows (prefill chunks, shared-prefix group tiles) go to
 //     the tcgen05 kernel of attn_tc.cu; this kernel takes decode-sized items only.
 //   * fp8 and NVFP4 tiles widen to f16 in registers with integer operations
@@ -73,7 +79,10 @@ struct TmaCfg {
   // A multiple of 4: decode tiles go round-robin to the 4 consumer warps by tile
   // index within the item, so within an item every tile that lands in a given
   // stage belongs to the same warp and the stage's phases are consumed in order;
-  // across items, the end-of-item merge barrier orders them.
+  // across items, the end-of-item merge barrier orders them.  Four-head items have
+  // no such barrier: every item has a multiple of 4 tiles, so the running tile
+  // count q stays a multiple of 4 and warp w always takes the tiles q + w + 4k,
+  // whose stages (q + w + 4k) mod NST no other warp uses.
   // Four 16 KB stages (64 KB) leave room for two CTAs per SM: twice the producers and consumer
   // warps of one large-ring CTA, which measured faster than a 12-stage ring with one CTA per SM.
   static constexpr int NST = FP4 ? 8 : 4 * std::max(1, std::min(12, (64 * 1024) / STAGE_BYTES) / 4);
@@ -84,6 +93,12 @@ struct TmaCfg {
   static constexpr int QSLOT = QROWS * D * 2;
   static constexpr int QBUF_BYTES = IR * QSLOT;
   static constexpr int MERGE_BYTES = 4 * 16 * D * 4 + 2 * 4 * 16 * 4;
+  // Four-head plans never merge warps' states: their query slots (four heads' rows, IR of them)
+  // and each warp's output staging (PKV_HEADS4_ROWS rows of D floats, padded so that the rows
+  // 2 t4 + b a store instruction touches fall in distinct banks) live in the merge region.
+  static constexpr int Q4SLOT = 4 * PKV_HEADS4_ROWS * D * 2;
+  static constexpr int OSTRIDE = D + 4;
+  static constexpr int OWARP = PKV_HEADS4_ROWS * OSTRIDE * 4;
   static constexpr int BAR_BYTES = 8 * (2 * NST + 2 * IR + 1);
   static constexpr int DESC_BYTES = IR * 64;
   static constexpr int IDS_BYTES = 32 * 4;
@@ -95,6 +110,7 @@ struct TmaCfg {
   static_assert(NST % 4 == 0, "stage count must be a multiple of the consumer warp count");
   static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
   static_assert(MERGE_BYTES % 16 == 0 && QSLOT % 16 == 0, "query slots 16-byte aligned for bulk copies");
+  static_assert(IR * Q4SLOT + 4 * OWARP <= MERGE_BYTES && OWARP % 16 == 0, "four-head slots fit the merge region");
 };
 
 struct ItemDesc {
@@ -175,14 +191,18 @@ PKV_DEVICE void dec_offsets(DecOffsets<D, KV, QBF>& o, int lane) {
 
 // The query rows of a decode item from its shared-memory slot (row r = token r / g, head r % g of
 // the item's KV head, D 16-bit values each), as the B fragments of S^T = K Q^T.
+// w4 >= 0: a four-head slot, whose token i holds the 4 g rows of the item's four heads; the rows
+// of head w4 are token r / g, slot row 4 g (r / g) + g w4 + r % g.
 template <int D, int KV, bool QBF, int NR>
-PKV_DEVICE void dec_load_q(const AttnArgs& a, uint32_t qslot, int R, DecState<D, KV, QBF, NR>& st, int g4, int t4) {
+PKV_DEVICE void dec_load_q(const AttnArgs& a, uint32_t qslot, int R, DecState<D, KV, QBF, NR>& st, int g4, int t4,
+                           int w4) {
   constexpr bool MMA_BF = KV == KV_BF16;
 #pragma unroll
   for (int nr = 0; nr < NR; ++nr) {
     const int r = nr * 8 + g4;
     const bool valid = r < R;
-    const uint32_t qrow = qslot + uint32_t(valid ? r : 0) * D * 2;
+    const int sr = w4 < 0 ? r : (r / a.g) * 4 * a.g + w4 * a.g + r % a.g;
+    const uint32_t qrow = qslot + uint32_t(valid ? sr : 0) * D * 2;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t w0 = 0, w1 = 0;
@@ -558,7 +578,48 @@ PKV_DEVICE void zero_v_tail(uint32_t vbase, int from, int lane) {
   __syncwarp();
 }
 
+// Four-head items: one warp writes its head's R (<= 8) rows from its staging rows (row r: D
+// unnormalised dims, then the row's max and sum in scaled-log2 units), TPR lanes a row and DPT
+// consecutive dims each.  part_row >= 0: float32 partial rows part_row + r; else output rows of
+// token q_begin + r / g, head head * g + r % g.
 template <int D, int KV, bool QBF>
+PKV_DEVICE void h4_write_rows(const float* ob, int R, int lane, int g, int hq, int q_begin, int head,
+                                           int part_row, float vscale, void* out, float* out_lse, float* part_o,
+                                           float* part_lse) {
+  using T = TmaCfg<D, KV, QBF>;
+  const int Rp = R <= 4 ? 4 : 8;
+  const int TPR = 32 / Rp, DPT = D / TPR;
+  const int r = lane / TPR, d0 = (lane % TPR) * DPT;
+  if (r >= R) return;
+  const float M = ob[r * T::OSTRIDE + D], lsum = ob[r * T::OSTRIDE + D + 1];
+  const float inv = lsum > 0.f ? vscale / lsum : 0.f;
+  const float lse2 = lsum > 0.f ? M + __log2f(lsum) : -INFINITY;
+  const bool to_part = part_row >= 0;
+  const int64_t orow = to_part ? int64_t(part_row) + r : (int64_t(q_begin) + r / g) * hq + head * g + r % g;
+#pragma unroll 1
+  for (int c = 0; c < DPT; c += 4) {
+    float4 o = *reinterpret_cast<const float4*>(ob + r * T::OSTRIDE + d0 + c);
+    o.x *= inv;
+    o.y *= inv;
+    o.z *= inv;
+    o.w *= inv;
+    if (to_part) {
+      *reinterpret_cast<float4*>(part_o + orow * D + d0 + c) = o;
+    } else {
+      const uint2 pk = QBF ? make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w))
+                           : make_uint2(pack_f16x2(o.x, o.y), pack_f16x2(o.z, o.w));
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow * D + d0 + c) = pk;
+    }
+  }
+  if (lane % TPR == 0) {
+    const float lse = lse2 * kLn2;
+    if (to_part) part_lse[orow] = lse;
+    else if (out_lse) out_lse[orow] = lse;
+  }
+}
+
+// H4: the four-head variant, launched for plans whose decode items cover four KV heads each.
+template <int D, int KV, bool QBF, bool H4>
 __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                           const __grid_constant__ CUtensorMap smap, const TmaArgs ta) {
   using T = TmaCfg<D, KV, QBF>;
@@ -572,6 +633,10 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
   float* red_m = red_o + 4 * 16 * D;
   float* red_l = red_m + 4 * 16;
   const uint32_t qbuf = base + T::NST * T::STAGE_BYTES + T::MERGE_BYTES;  // T::IR query slots
+  // Four-head plans: T::IR query slots at the start of the merge region, the warps' output
+  // staging after them.
+  const uint32_t q4buf = base + T::NST * T::STAGE_BYTES;
+  constexpr bool h4 = H4;  // every decode item covers four KV heads
   const uint32_t bars = qbuf + T::QBUF_BYTES;
   auto full_bar = [&](int i) { return bars + 8 * i; };
   auto empty_bar = [&](int i) { return bars + 8 * (T::NST + i); };
@@ -650,26 +715,29 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       it.part_row = __shfl_sync(0xffffffffu, field, 7);
       bool valid = it.seq >= 0 && it.seq < a.num_seqs && it.kv_head >= 0 && it.kv_head < a.hkv && it.n_q > 0 &&
                    it.n_q * a.g <= a.max_rows && it.q_begin >= 0 && it.q_begin + it.n_q <= total_q &&
-                   it.k_begin >= 0 && it.k_begin < it.k_end && (it.k_begin % box_rows) == 0;
+                   it.k_begin >= 0 && it.k_begin < it.k_end && (it.k_begin % box_rows) == 0 &&
+                   (!h4 || (it.kv_head % 4 == 0 && it.kv_head + 4 <= a.hkv && it.n_q * a.g <= PKV_HEADS4_ROWS));
       if (valid) {
         const int L = __ldg(a.seq_lens + it.seq);
         valid = it.k_end <= L && ((it.k_end - 1) >> a.log2_block) < a.max_blocks && (it.pos0 < 0 || it.pos0 + it.n_q <= L);
       }
       if (!valid && lane == 0) report(a.status, PKV_DEV_PLAN_MISMATCH);
-      const int ntiles = valid ? (it.k_end - it.k_begin + T::TK - 1) / T::TK : 0;
+      // Four-head items: 4 tiles per key tile, tile t of head kv_head + t % 4.
+      const int ntiles = valid ? ((it.k_end - it.k_begin + T::TK - 1) / T::TK) * (h4 ? 4 : 1) : 0;
       if (lane == 0) {
         d.seq = it.seq; d.kv_head = it.kv_head; d.q_begin = it.q_begin; d.n_q = it.n_q; d.k_begin = it.k_begin;
         d.k_end = it.k_end; d.pos0 = it.pos0; d.part_row = it.part_row; d.ntiles = ntiles; d.state = valid ? 0 : 1;
         const int rows = it.n_q * a.g;
         if (valid && rows <= T::QROWS) {
           // A decode item's query rows travel with its descriptor: for each of its tokens the g
-          // heads of the KV head are one contiguous run of g * D 16-bit values; the slot's
-          // barrier completes when they have landed.
-          const uint32_t run = uint32_t(a.g) * D * 2;
+          // heads of the KV head (4 g of the four KV heads) are one contiguous run of 16-bit
+          // values; the slot's barrier completes when they have landed.
+          const uint32_t run = uint32_t(a.g) * D * 2 * (h4 ? 4u : 1u);
+          const uint32_t qdst = h4 ? q4buf + slot * T::Q4SLOT : qbuf + slot * T::QSLOT;
           mbar_arrive_expect_tx(ifull_bar(slot), run * uint32_t(it.n_q));
           const uint16_t* qsrc = static_cast<const uint16_t*>(a.q) + (int64_t(it.q_begin) * a.hq + it.kv_head * a.g) * D;
           for (int i = 0; i < it.n_q; ++i)
-            bulk_load_1d(qbuf + slot * T::QSLOT + uint32_t(i) * run, qsrc + int64_t(i) * a.hq * D, run, ifull_bar(slot));
+            bulk_load_1d(qdst + uint32_t(i) * run, qsrc + int64_t(i) * a.hq * D, run, ifull_bar(slot));
         } else {
           mbar_arrive(ifull_bar(slot), 1);
         }
@@ -689,7 +757,8 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
           // Tiles whose first block lies in this chunk (a tile never straddles chunks:
           // 32 is a multiple of the blocks per tile).
           for (; t < ntiles; ++t, ++q) {
-            const int key0 = it.k_begin + t * T::TK;
+            const int key0 = it.k_begin + (h4 ? t >> 2 : t) * T::TK;
+            const int head = it.kv_head + (h4 ? t & 3 : 0);
             const int rel = (key0 >> a.log2_block) - first_blk - chunk;
             if (rel >= 32) break;
             const int stg = q % T::NST;
@@ -709,14 +778,14 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
                   phys = int(a.num_blocks);  // out of the tensor: the loads fill zeros
                 }
                 if (merged) {
-                  tma_load_5d(sdst, &tmap, full_bar(stg), 0, key0 & bmask, it.kv_head, c3k, phys);
-                  tma_load_5d(sdst + T::KS_OFF, &smap, full_bar(stg), 0, (key0 & bmask) >> 1, it.kv_head, c3k, phys);
+                  tma_load_5d(sdst, &tmap, full_bar(stg), 0, key0 & bmask, head, c3k, phys);
+                  tma_load_5d(sdst + T::KS_OFF, &smap, full_bar(stg), 0, (key0 & bmask) >> 1, head, c3k, phys);
                 } else {
                   const uint32_t r0 = uint32_t(j * box_rows);
-                  tma_load_5d(sdst + r0 * T::RB, &tmap, full_bar(stg), 0, 0, it.kv_head, c3k, phys);
-                  tma_load_5d(sdst + T::V_OFF + r0 * T::RB, &tmap, full_bar(stg), 0, 0, it.kv_head, c3k + 1, phys);
-                  tma_load_5d(sdst + T::KS_OFF + r0 * T::SCALE_ROW, &smap, full_bar(stg), 0, 0, it.kv_head, c3k, phys);
-                  tma_load_5d(sdst + T::VS_OFF + r0 * T::SCALE_ROW, &smap, full_bar(stg), 0, 0, it.kv_head, c3k + 1,
+                  tma_load_5d(sdst + r0 * T::RB, &tmap, full_bar(stg), 0, 0, head, c3k, phys);
+                  tma_load_5d(sdst + T::V_OFF + r0 * T::RB, &tmap, full_bar(stg), 0, 0, head, c3k + 1, phys);
+                  tma_load_5d(sdst + T::KS_OFF + r0 * T::SCALE_ROW, &smap, full_bar(stg), 0, 0, head, c3k, phys);
+                  tma_load_5d(sdst + T::VS_OFF + r0 * T::SCALE_ROW, &smap, full_bar(stg), 0, 0, head, c3k + 1,
                               phys);
                 }
               }
@@ -729,7 +798,7 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
               mbar_arrive_expect_tx(full_bar(stg), T::HALVES * 2 * T::TK * 128);
 #pragma unroll
               for (int h = 0; h < T::HALVES; ++h)
-                tma_load_5d(sdst + h * T::SLAB, &tmap, full_bar(stg), h * (128 / T::ELEM), key0 & bmask, it.kv_head,
+                tma_load_5d(sdst + h * T::SLAB, &tmap, full_bar(stg), h * (128 / T::ELEM), key0 & bmask, head,
                             c3k, phys);
             } else {
               int nb = 0;
@@ -744,8 +813,8 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
 #pragma unroll
                 for (int h = 0; h < T::HALVES; ++h) {
                   const uint32_t dst = sdst + h * T::SLAB + uint32_t(j * box_rows) * 128;
-                  tma_load_5d(dst, &tmap, full_bar(stg), h * (128 / T::ELEM), 0, it.kv_head, c3k, phys);
-                  tma_load_5d(dst + T::TK * 128, &tmap, full_bar(stg), h * (128 / T::ELEM), 0, it.kv_head, c3k + 1,
+                  tma_load_5d(dst, &tmap, full_bar(stg), h * (128 / T::ELEM), 0, head, c3k, phys);
+                  tma_load_5d(dst + T::TK * 128, &tmap, full_bar(stg), h * (128 / T::ELEM), 0, head, c3k + 1,
                               phys);
                 }
               }
@@ -795,11 +864,11 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
     float c = a.softmax_scale * kLog2e;  // raw score -> log2 units
     float vscale = 1.f;
     if constexpr (KV == KV_E4M3 || KV == KV_NVFP4) {
-      c *= __ldg(a.k_scale + a.layer * a.hkv + d.kv_head);
-      vscale = __ldg(a.v_scale + a.layer * a.hkv + d.kv_head);
+      const int sh = d.kv_head + (h4 ? warp : 0);  // scales are per (layer, KV head): the warp's head
+      c *= __ldg(a.k_scale + a.layer * a.hkv + sh);
+      vscale = __ldg(a.v_scale + a.layer * a.hkv + sh);
     }
     const bool to_part = d.part_row >= 0;
-    const int last_valid = d.k_end - (d.k_begin + (ntiles - 1) * T::TK);  // rows of the last tile in range
 
     if (R <= 16) {
       // ---- decode: warps take whole tiles round-robin, S^T / O^T formulation.
@@ -808,7 +877,11 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       auto run = [&](auto nr_tag) {
         constexpr int NR = decltype(nr_tag)::value;
         DecState<D, KV, QBF, NR> st;
-        dec_load_q<D, KV, QBF, NR>(a, qbuf + slot * T::QSLOT, R, st, g4, t4);
+        const bool hw = NR == 1 && h4;  // four-head items have at most 8 rows: one row group
+        const int nkt = hw ? ntiles >> 2 : ntiles;                         // key tiles of the item
+        const int last_valid = d.k_end - (d.k_begin + (nkt - 1) * T::TK);  // rows of the last key tile in range
+        if (hw) dec_load_q<D, KV, QBF, NR>(a, q4buf + slot * T::Q4SLOT, R, st, g4, t4, warp);
+        else dec_load_q<D, KV, QBF, NR>(a, qbuf + slot * T::QSLOT, R, st, g4, t4, -1);
         __syncwarp();
         if (lane == 0) mbar_arrive(iempty_bar(slot), 1);
         int lim_min = d.k_end, lo_max = 0;
@@ -837,12 +910,13 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
           const int stg = qq % T::NST;
           if (!ok || s_abort || !mbar_wait(full_bar(stg), (qq / T::NST) & 1, &s_wl)) { ok = false; continue; }
           const uint32_t kb = stages + stg * T::STAGE_BYTES, vb = kb + T::V_OFF;
-          if (t == ntiles - 1 && last_valid < T::TK) {
+          const int kt = hw ? t >> 2 : t;  // key tile (four-head items: head kv_head + warp)
+          if (kt == nkt - 1 && last_valid < T::TK) {
             if constexpr (T::FP4) zero_v_tail_fp4<T::TK, T::SCALE_ROW>(vb, kb + T::VS_OFF, last_valid, lane);
             else zero_v_tail<T::RB, T::TK, T::SLAB>(vb, last_valid, lane);
             fence_proxy_async_smem();
           }
-          const int key0 = d.k_begin + t * T::TK;
+          const int key0 = d.k_begin + kt * T::TK;
           if constexpr (T::FP4)
             dec_tile_fp4<D, QBF>(st, offs, kb, vb, kb + T::KS_OFF, kb + T::VS_OFF, key0, lane, deq_undo<KV>(c),
                                  key0 + T::TK > lim_min || key0 < lo_max);
@@ -863,6 +937,26 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
             x += __shfl_xor_sync(0xffffffffu, x, 16);
             st.l[nr][b] = x;
           }
+        if (hw) {
+          // The warp's head is complete: its rows (R <= 8) go to the warp's own staging rows,
+          // max and sum in the row's first two padding floats; written out below.
+          float* ob = red_o + (T::IR * T::Q4SLOT + warp * T::OWARP) / 4;
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int r = 2 * t4 + (e & 1);
+              if (r < R) ob[r * T::OSTRIDE + dec_dim<KV>(mt, e, g4)] = st.acc[0][mt][e];
+            }
+          if (g4 == 0) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              ob[(2 * t4 + b) * T::OSTRIDE + D] = st.m[0][b];
+              ob[(2 * t4 + b) * T::OSTRIDE + D + 1] = st.l[0][b];
+            }
+          }
+          return;
+        }
 #pragma unroll
         for (int nr = 0; nr < NR; ++nr)
 #pragma unroll
@@ -886,8 +980,18 @@ __global__ void __launch_bounds__(160, 2) attn_tma_kernel(const __grid_constant_
       if constexpr (T::FP4) {
         run(std::integral_constant<int, 1>{});  // NVFP4 items carry at most 8 rows
       } else {
-        if (R <= 8) run(std::integral_constant<int, 1>{});
-        else run(std::integral_constant<int, 2>{});
+        if (h4 || R <= 8) run(std::integral_constant<int, 1>{});  // four-head items: at most 8 rows
+        else if constexpr (!H4) run(std::integral_constant<int, 2>{});
+      }
+      if constexpr (H4) {
+        __syncwarp();
+        h4_write_rows<D, KV, QBF>(red_o + (T::IR * T::Q4SLOT + warp * T::OWARP) / 4, R, lane, a.g, a.hq,
+                                  d.q_begin, d.kv_head + warp, to_part ? d.part_row + warp * R : -1,
+                                  deq_undo<KV>(vscale), a.out, a.out_lse, a.part_o, a.part_lse);
+        __syncwarp();  // the staging rows are rewritten by the warp's next item
+        q += ntiles;
+        if (!ok) break;
+        continue;
       }
       mbar_arrive(merge_bar, 1);
       if (!mbar_wait(merge_bar, merge_phase, &s_wl)) ok = false;
@@ -1030,7 +1134,8 @@ cudaError_t launch_tma_grid(const AttnArgs& a, int grid, cudaStream_t st, const 
                             const CUtensorMap& smap, const TmaArgs& ta) {
   using T = TmaCfg<D, KV, QBF>;
   const cudaError_t e =
-      launch_pdl(attn_tma_kernel<D, KV, QBF>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, smap, ta);
+      a.heads4 ? launch_pdl(attn_tma_kernel<D, KV, QBF, true>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, smap, ta)
+               : launch_pdl(attn_tma_kernel<D, KV, QBF, false>, dim3(grid), dim3(T::THREADS), T::SMEM, st, map, smap, ta);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1060,9 +1165,9 @@ template <int D, int KV, bool QBF>
 AttnKernel tma_kernel() {
   using T = TmaCfg<D, KV, QBF>;
   // Decode-sized tiles only (larger ones are tcgen05 items).
-  return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF>), T::THREADS, T::SMEM,
-                    &launch_tma<D, KV, QBF>,
-                    KV == KV_NVFP4 ? PKV_FP4_ROWS : PKV_DECODE_ROWS};
+  return AttnKernel{reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF, false>), T::THREADS, T::SMEM,
+                    &launch_tma<D, KV, QBF>, KV == KV_NVFP4 ? PKV_FP4_ROWS : PKV_DECODE_ROWS,
+                    reinterpret_cast<const void*>(&attn_tma_kernel<D, KV, QBF, true>)};
 }
 
 bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size, AttnKernel* k) {
@@ -1097,3 +1202,10 @@ bool attn_tma_kernel_for(int kv_dtype, int q_dtype, int head_dim, int block_size
 }
 
 }  // namespace pkv
+
+bool pkv_heads4_capable(int kv_dtype, int head_dim, int block_size) {
+  // The pools' own query dtype (fp8 and NVFP4 pools take either 16-bit query on this kernel).
+  const int q_dtype = kv_dtype == PKV_F16 ? PKV_F16 : PKV_BF16;
+  pkv::AttnKernel k;
+  return pkv::attn_tma_kernel_for(kv_dtype, q_dtype, head_dim, block_size, &k);
+}

@@ -44,7 +44,10 @@ constexpr double kCorunGain = 0.95;
 // keys are split or it belongs to a shared-prefix group, a merge per head).
 struct Piece {
   int32_t seq, q_begin, n_q, k_begin, k_end, pos0;
-  int32_t part0;     // partial row of head 0 (head h: part0 + h * part_stride); -1: final output
+  // Partial rows, -1: final output.  With h heads an item (4 for decode pieces of a four-head plan,
+  // else 1), head hh's rows start at part0 + (hh / h) * part_stride + (hh % h) * n_q * g, so the
+  // four heads of an item own consecutive row runs.
+  int32_t part0;
   int32_t part_stride;
   uint64_t cost16;   // 16 x keys x max(1, rows / 16)
   bool tc;           // tensor-memory list
@@ -148,6 +151,13 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: unknown debug_flags 0x%x", req->debug_flags);
   if (req->tc_num_ctas > 0 && req->num_ctas <= 0)
     return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: tc_num_ctas > 0 needs num_ctas > 0");
+  if (req->heads_per_item != 0 && req->heads_per_item != 1 && req->heads_per_item != 4)
+    return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: heads_per_item %d (0, 1 or 4)", req->heads_per_item);
+  // Four-head decode items: the TMA-fed decode kernel, KV heads in fours.
+  const bool h4_capable = Hkv % 4 == 0 && pkv_heads4_capable(req->kv_dtype, D, B);
+  if (req->heads_per_item == 4 && !h4_capable)
+    return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: four-head items need num_kv_heads a multiple of 4 and a "
+                    "pool the TMA-fed decode kernel serves");
   const int32_t* cu = req->cu_q_lens;
   const int32_t* L = req->seq_lens;
   if (S > 0 && cu[0] != 0) return pkv_fail(PKV_ERR_INVALID_ARG, "attention_plan: cu_q_lens[0] != 0");
@@ -338,6 +348,46 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     }
   }
 
+  // 2a. KV heads per decode-tile item.  A one-head item's keys are split over the kernel's four
+  // consumer warps, whose states merge at the item's end, and each item costs its CTA a fixed
+  // setup; items of four heads give each warp one head for the whole range, with no merge and a
+  // quarter of the items.  Automatic choice: four heads on NVFP4 pools (instruction-bound tiles,
+  // where the warps' merge and its barrier cost more than the extra partial rows of shorter
+  // pieces) and, on the others, when the decode tiles' key ranges average at most half the
+  // per-CTA share of the decode list (short ranges, where the fixed cost per item counts); long
+  // ranges keep one head an item, which splits them less.
+  int hpi = 1;
+  {
+    bool fits = h4_capable;  // every decode-sized tile of at most PKV_HEADS4_ROWS rows
+    int64_t dec_tiles = 0;
+    double dec_keys = 0;
+    for (size_t i = 0; i < n_group_pieces; ++i)
+      if (!pieces[i].tc) {
+        fits = fits && pieces[i].n_q * g <= PKV_HEADS4_ROWS;
+        ++dec_tiles;
+        dec_keys += double(pieces[i].k_end - pieces[i].k_begin);
+      }
+    for (const Tile& t : tiles)
+      if (!is_tc(t.n_q * g)) {
+        fits = fits && t.n_q * g <= PKV_HEADS4_ROWS;
+        ++dec_tiles;
+        dec_keys += double(std::max(0, t.ke - t.k0));
+      }
+    if (req->heads_per_item == 4) {
+      if (!fits)
+        return pkv_fail(PKV_ERR_UNSUPPORTED, "attention_plan: four-head items take decode tiles of at most %d rows",
+                        PKV_HEADS4_ROWS);
+      hpi = dec_tiles > 0 ? 4 : 1;
+    } else if (req->heads_per_item == 0 && fits && dec_tiles > 0) {
+      const double share = total_cost[0] / (double(num_ctas) * 2.0);  // keys x heads per item, one head
+      if (fp4 || 2.0 * dec_keys / double(dec_tiles) <= share) hpi = 4;
+    }
+    if (hpi == 4)
+      for (size_t i = 0; i < n_group_pieces; ++i)
+        if (!pieces[i].tc) pieces[i].part_stride *= 4;  // part0 + hh * rows for every head hh
+  }
+  auto heads_of = [&](bool t) { return t ? 1 : hpi; };  // KV heads per item of a list
+
   // 2b. Side by side.  With both decode-sized tiles (HBM-bound) and tensor-memory tiles
   // (tensor-bound) in the batch, the tcgen05 kernel may take k SMs and the decode-tile kernel the
   // others at the same time instead of one after the other.  Estimated times: the tensor-memory
@@ -358,7 +408,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     int64_t n_reg_pieces = 0;  // decode-tile items before any key split
     for (size_t i = 0; i < n_group_pieces; ++i) n_reg_pieces += pieces[i].tc ? 0 : 1;
     for (const Tile& t : tiles) n_reg_pieces += is_tc(t.n_q * g) ? 0 : 1;
-    const double reg_items = double(n_reg_pieces) * Hkv;
+    const double reg_items = double(n_reg_pieces) * Hkv / hpi;
     const double tc_rate = f8 ? kTcFp8FlopsPerSm : kTcFlopsPerSm;
     auto t_tc = [&](int k) { return flops / (double(k) * tc_rate); };
     auto t_reg = [&](int n) {
@@ -383,14 +433,16 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   const double target[2] = {total_cost[0] / (double(num_ctas) * 2.0), total_cost[1] / (double(tc_ctas) * 3.0)};
   // Longest key range of one item of a tile's list; the automatic length (about two items per
   // CTA on the decode kernel, three on the tcgen05 kernel, whose CTAs take items in turn
-  // from a longer queue and whose merges spread over 16-row chunks) is scaled by `mult`.
+  // from a longer queue and whose merges spread over 16-row chunks; a four-head item a quarter
+  // of a one-head item's keys) is scaled by `mult`.
   auto max_keys_for = [&](int rows, bool t, double mult) -> int32_t {
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     int64_t max_keys;
     if (req->kv_split < 0) max_keys = INT32_MAX;
     else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
     else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
-                                      round_up(int64_t(std::ceil(target[t] * mult * 16.0 / double(weight16(rows)))),
+                                      round_up(int64_t(std::ceil(target[t] * mult * 16.0 /
+                                                                 (double(weight16(rows)) * heads_of(t)))),
                                                tile_keys));
     return int32_t(std::min<int64_t>(max_keys, INT32_MAX / 2));
   };
@@ -409,7 +461,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   if (req->kv_split == 0) {
     auto count_items = [&](double mult) {
       size_t n_items = 0;
-      for (size_t i = 0; i < n_group_pieces; ++i) n_items += pieces[i].tc ? 0 : size_t(Hkv);
+      for (size_t i = 0; i < n_group_pieces; ++i) n_items += pieces[i].tc ? 0 : size_t(Hkv / hpi);
       int last = -1;
       int32_t m = 0;
       for (const Tile& t : tiles) {
@@ -419,7 +471,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
         int32_t nseg;
         int64_t seg;
         split(std::max(0, t.ke - t.k0), m, PKV_TILE_KEYS, nseg, seg);
-        n_items += size_t(nseg) * size_t(Hkv);
+        n_items += size_t(nseg) * size_t(Hkv / hpi);
       }
       return n_items;
     };
@@ -435,7 +487,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       auto makespan = [&](double mult) {
         runs.clear();
         for (size_t i = 0; i < n_group_pieces; ++i)  // shared-prefix group items, never split
-          if (!pieces[i].tc) runs.push_back({pieces[i].cost16, uint32_t(Hkv)});
+          if (!pieces[i].tc) runs.push_back({pieces[i].cost16 * uint64_t(hpi), uint32_t(Hkv / hpi)});
         int last = -1;
         int32_t m = 0;
         for (const Tile& t : tiles) {
@@ -447,9 +499,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
           int64_t seg;
           split(n, m, PKV_TILE_KEYS, nseg, seg);
           if (nseg == 0) continue;
-          const uint64_t w16 = weight16(rows);
-          if (nseg > 1) runs.push_back({uint64_t(seg) * w16, uint32_t(nseg - 1) * uint32_t(Hkv)});
-          runs.push_back({uint64_t(n - (nseg - 1) * seg) * w16, uint32_t(Hkv)});
+          const uint64_t w16 = weight16(rows) * uint64_t(hpi);
+          if (nseg > 1) runs.push_back({uint64_t(seg) * w16, uint32_t(nseg - 1) * uint32_t(Hkv / hpi)});
+          runs.push_back({uint64_t(n - (nseg - 1) * seg) * w16, uint32_t(Hkv / hpi)});
         }
         std::sort(runs.begin(), runs.end(), [](const CostRun& x, const CostRun& y) { return x.cost16 > y.cost16; });
         A.assign(size_t(num_ctas), 0);
@@ -502,13 +554,14 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       continue;
     }
     Merge mg{tl.q_begin, tl.n_q, gp, gp >= 0 ? sc.member_stride[tl.seq] : 0, int32_t(pieces.size()), nseg};
-    // Partial rows of the tile's pieces: head h, piece p at base + (h * nseg + p) * rows.
-    const int64_t base = part_rows;
+    // Partial rows of the tile's pieces, h heads an item: head hh, piece p at
+    // base + ((hh / h) * nseg + p) * h * rows + (hh % h) * rows.
+    const int64_t base = part_rows, hr = int64_t(heads_of(t)) * rows;
     int p = 0;
     for (int64_t k0 = tl.k0; k0 < tl.ke; k0 += seg, ++p) {
       const int k1 = int(std::min<int64_t>(tl.ke, k0 + seg));
-      pieces.push_back({tl.seq, tl.q_begin, tl.n_q, int32_t(k0), k1, tl.pos0, int32_t(base + int64_t(p) * rows),
-                        int32_t(int64_t(nseg) * rows), uint64_t(k1 - k0) * w16, t});
+      pieces.push_back({tl.seq, tl.q_begin, tl.n_q, int32_t(k0), k1, tl.pos0, int32_t(base + int64_t(p) * hr),
+                        int32_t(int64_t(nseg) * hr), uint64_t(k1 - k0) * w16, t});
     }
     part_rows += int64_t(nseg) * rows * Hkv;
     n_parts += int64_t(nseg + (gp >= 0 ? 1 : 0)) * Hkv;
@@ -521,7 +574,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
 
   size_t n_tc_pieces = 0;
   for (const Piece& pc : pieces) n_tc_pieces += pc.tc ? 1 : 0;
-  const int64_t n_items = int64_t(pieces.size()) * Hkv, n_tc = int64_t(n_tc_pieces) * Hkv;
+  const int64_t n_tc = int64_t(n_tc_pieces) * Hkv;
+  const int64_t n_items = n_tc + int64_t(pieces.size() - n_tc_pieces) * (Hkv / hpi);
   const int64_t n_reduce = int64_t(merges.size()) * Hkv;
 
   const uint64_t items_off = sizeof(PkvPlanHeader);
@@ -542,6 +596,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   info->num_tc_items = int32_t(n_tc);
   info->tc_num_ctas = tc_ctas;
   info->side_by_side = corun ? 1 : 0;
+  info->heads_per_item = hpi;
   if (!plan) return PKV_OK;
   if (capacity < bytes) return pkv_fail(PKV_ERR_WORKSPACE, "attention_plan: capacity %zu < %llu", capacity, (unsigned long long)bytes);
 
@@ -553,7 +608,7 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.n_tc_items = int32_t(n_tc);
   h.tc_items_off = uint32_t(tc_items_off);
   h.tc_num_ctas = tc_ctas;
-  h.flags = corun ? PKV_PLAN_CORUN : 0;
+  h.flags = (corun ? PKV_PLAN_CORUN : 0) | (hpi == 4 ? PKV_PLAN_HEADS4 : 0);
   h.window = window;
   h.wait_limit_kcycles = req->wait_limit_kcycles;
   h.debug_flags = req->debug_flags;
@@ -576,14 +631,16 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   h.rows_off = uint32_t(rows_off);
   h.n_rows = int32_t(sc.row_tokens.size());
   std::memcpy(p, &h, sizeof(h));
-  // Items: pieces heaviest first, each expanded over the KV heads.
+  // Items: pieces heaviest first, each expanded over the KV heads (in fours on a four-head plan's
+  // decode-tile list: item j takes heads 4j .. 4j + 3 and the rows of head 4j).
   PkvItem* items = reinterpret_cast<PkvItem*>(p + items_off);
   order_pieces(pieces, sc.keys, sc.tmp);
   for (size_t i = 0; i < pieces.size(); ++i) {
     const Piece& pc = pieces[size_t(sc.keys[i] & 0xFFFFF)];
-    for (int hh = 0; hh < Hkv; ++hh)
-      *items++ = PkvItem{pc.seq, hh, pc.q_begin, pc.n_q, pc.k_begin, pc.k_end, pc.pos0,
-                         pc.part0 == -1 ? -1 : pc.part0 + hh * pc.part_stride};
+    const int nh = heads_of(pc.tc);
+    for (int j = 0; j < Hkv / nh; ++j)
+      *items++ = PkvItem{pc.seq, j * nh, pc.q_begin, pc.n_q, pc.k_begin, pc.k_end, pc.pos0,
+                         pc.part0 == -1 ? -1 : pc.part0 + j * pc.part_stride};
   }
   // Merges and their part lists, per tile and KV head: the group part first, then the pieces.
   PkvReduce* reds = reinterpret_cast<PkvReduce*>(p + reduce_off);
@@ -595,7 +652,8 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       if (mg.group_part0 >= 0) parts[np++] = mg.group_part0 + hh * mg.group_stride;
       for (int k = 0; k < mg.n_pieces; ++k) {
         const Piece& pc = pieces[size_t(mg.first_piece + k)];
-        parts[np++] = pc.part0 + hh * pc.part_stride;
+        const int nh = heads_of(pc.tc);
+        parts[np++] = pc.part0 + (hh / nh) * pc.part_stride + (hh % nh) * pc.n_q * g;
       }
       *reds++ = PkvReduce{mg.q_begin, mg.n_q, hh, begin, np - begin, {0, 0, 0}};
     }

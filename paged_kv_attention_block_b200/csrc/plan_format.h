@@ -61,6 +61,12 @@ static_assert(sizeof(PkvPlanHeader) == 128, "plan header size");
 // (one an SM) and the decode-tile kernel beside it on num_ctas CTAs (the other SMs).  Without it
 // the decode-tile kernel runs first and the tcgen05 kernel takes the SMs it frees.
 #define PKV_PLAN_CORUN 0x1
+// Every item of the decode-tile list covers four consecutive KV heads, kv_head .. kv_head + 3
+// (kv_head a multiple of 4), with at most PKV_HEADS4_ROWS rows per head; head kv_head + w of it
+// writes its partial rows at part_row + w * n_q * g.  Only the TMA-fed decode kernel takes such
+// plans: each of its four consumer warps runs one of the heads over the whole key range.
+#define PKV_PLAN_HEADS4 0x2
+#define PKV_HEADS4_ROWS 8
 
 // One CTA-sized piece of work: rows [q_begin, q_begin + n_q) x the g query
 // heads of kv_head, against keys [k_begin, k_end) read through the block-table

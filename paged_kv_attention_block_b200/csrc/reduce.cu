@@ -34,27 +34,82 @@ __global__ void __launch_bounds__(256) dense_reduce_kernel(const float* __restri
 // CTA at blockIdx.y takes its rows 16 y .. 16 y + 15, four a warp, so a merge of
 // 128-row partials spreads over 8 CTAs); lane j merges head dims [VEC j, VEC (j + 1))
 // with the same per-element arithmetic as merge_elem, so each lane issues VEC-wide
-// loads of the parts.
+// loads of the parts.  Latency, not bandwidth, sets this kernel's time: the merges and
+// their part lists (staged before the attention kernels started, which waited for the
+// staging) are read before the wait for the attention kernels, and a row of two parts
+// loads both at once.  40 registers: 12 CTAs an SM (1,776 on a B200) hold most plans' merges at once.
 template <int D>
-__global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
+PKV_DEVICE void load_part(const float* part_o, int64_t prow, int lane, float (&x)[D / 32]) {
+  constexpr int VEC = D / 32;
+  const float* src = part_o + prow * D + lane * VEC;
+  if constexpr (VEC == 4) {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(src));
+    x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+  } else {
+    const float2 f = __ldg(reinterpret_cast<const float2*>(src));
+    x[0] = f.x; x[1] = f.y;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128, 12) plan_reduce_kernel(const ReduceArgs a) {
   constexpr int VEC = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int e = blockIdx.x;
+  PkvReduce red{};
+  int32_t my_part = 0;  // lane i: the merge's part i (i < 32)
+  auto fetch = [&](int m) {
+    red = a.reduces[m];
+    my_part = lane < red.n_parts ? __ldg(a.parts + red.parts_begin + lane) : 0;
+  };
+  if (e < a.n_reduce) fetch(e);
   pdl_wait();  // launched as a dependent of the attention kernels: their partial states are complete
-  for (int e = blockIdx.x; e < a.n_reduce; e += gridDim.x) {
-    const PkvReduce red = a.reduces[e];
+  for (; e < a.n_reduce; e += gridDim.x) {
+    if (e != int(blockIdx.x)) fetch(e);
     const int R = red.n_q * a.g;
-    const int32_t* parts = a.parts + red.parts_begin;
     const int n = red.n_parts;
     const int r_end = min(R, int(blockIdx.y) * 16 + 16);
     for (int r = int(blockIdx.y) * 16 + warp; r < r_end; r += 4) {
-      float M = -INFINITY;
-      for (int i = 0; i < n; ++i) M = fmaxf(M, __ldg(a.part_lse + int64_t(__ldg(parts + i)) + r));
       float o[VEC], lse;
-      if (M == -INFINITY) {
+      if (n <= 2) {
+        // The usual case (a split in two, or a shared-prefix group part and a member's own part):
+        // both parts' sums and rows are loaded at once.
+        const int64_t p0 = int64_t(__shfl_sync(0xffffffffu, my_part, 0)) + r;
+        const int64_t p1 = int64_t(__shfl_sync(0xffffffffu, my_part, 1)) + r;
+        const float l0 = n > 0 ? __ldg(a.part_lse + p0) : -INFINITY;
+        const float l1 = n > 1 ? __ldg(a.part_lse + p1) : -INFINITY;
+        float x0[VEC], x1[VEC];
+        if (n > 0) load_part<D>(a.part_o, p0, lane, x0);
+        if (n > 1) load_part<D>(a.part_o, p1, lane, x1);
+        const float M = fmaxf(l0, l1);
+        if (M == -INFINITY) {
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) o[v] = 0.f;
-        lse = -INFINITY;
+          for (int v = 0; v < VEC; ++v) o[v] = 0.f;
+          lse = -INFINITY;
+        } else {
+          float num[VEC], den = 0.f;
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) num[v] = 0.f;
+          if (l0 != -INFINITY) {
+            const float w = expf(l0 - M);
+            den += w;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) num[v] = fmaf(w, x0[v], num[v]);
+          }
+          if (l1 != -INFINITY) {
+            const float w = expf(l1 - M);
+            den += w;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) num[v] = fmaf(w, x1[v], num[v]);
+          }
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) o[v] = num[v] / den;
+          lse = M + logf(den);
+        }
       } else {
+        const int32_t* parts = a.parts + red.parts_begin;
+        float M = -INFINITY;
+        for (int i = 0; i < n; ++i) M = fmaxf(M, __ldg(a.part_lse + int64_t(__ldg(parts + i)) + r));
         float num[VEC], den = 0.f;
 #pragma unroll
         for (int v = 0; v < VEC; ++v) num[v] = 0.f;
@@ -64,21 +119,15 @@ __global__ void __launch_bounds__(128) plan_reduce_kernel(const ReduceArgs a) {
           if (li == -INFINITY) continue;
           const float w = expf(li - M);
           den += w;
-          const float* src = a.part_o + prow * D + lane * VEC;
           float x[VEC];
-          if constexpr (VEC == 4) {
-            const float4 f = __ldg(reinterpret_cast<const float4*>(src));
-            x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
-          } else {
-            const float2 f = __ldg(reinterpret_cast<const float2*>(src));
-            x[0] = f.x; x[1] = f.y;
-          }
+          load_part<D>(a.part_o, prow, lane, x);
 #pragma unroll
           for (int v = 0; v < VEC; ++v) num[v] = fmaf(w, x[v], num[v]);
         }
+        // M = -inf leaves den = 0: o = 0, lse = -inf, as merge_elem gives.
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) o[v] = num[v] / den;
-        lse = M + logf(den);
+        for (int v = 0; v < VEC; ++v) o[v] = M == -INFINITY ? 0.f : num[v] / den;
+        lse = M == -INFINITY ? -INFINITY : M + logf(den);
       }
       const int64_t orow = (int64_t(red.q_begin) + r / a.g) * a.hq + red.kv_head * a.g + r % a.g;
 #pragma unroll

@@ -16,6 +16,7 @@ assert HEADER.itemsize == 128 and ITEM.itemsize == 32 and REDUCE.itemsize == 32
 
 
 TILE_ROWS, DECODE_ROWS, TILE_ROWS_TC, TC_TILE_KEYS = 64, 16, 128, 128
+PLAN_CORUN, PLAN_HEADS4, HEADS4_ROWS = 0x1, 0x2, 8
 
 
 def decode(buf) -> dict:
@@ -24,12 +25,28 @@ def decode(buf) -> dict:
     h = np.frombuffer(b[:128].tobytes(), HEADER)[0]
     reg = np.frombuffer(b[h["items_off"]:h["items_off"] + 32 * h["n_items"]].tobytes(), ITEM)
     tc = np.frombuffer(b[h["tc_items_off"]:h["tc_items_off"] + 32 * h["n_tc_items"]].tobytes(), ITEM)
-    items = np.concatenate([reg, tc])
+    if h["flags"] & PLAN_HEADS4:
+        reg_heads = _expand_heads4(reg, int(h["num_q_heads"]) // int(h["num_kv_heads"]))
+    else:
+        reg_heads = reg
+    items = np.concatenate([reg_heads, tc])
     reds = np.frombuffer(b[h["reduce_off"]:h["reduce_off"] + 32 * h["n_reduce"]].tobytes(), REDUCE)
     parts = np.frombuffer(b[h["parts_off"]:h["parts_off"] + 4 * h["n_parts"]].tobytes(), "<i4")
     rows = np.frombuffer(b[h["rows_off"]:h["rows_off"] + 4 * h["n_rows"]].tobytes(), "<i4")
     return {"header": h, "items": items, "reg_items": reg, "tc_items": tc, "reduces": reds, "parts": parts,
             "rows": rows}
+
+
+def _expand_heads4(reg, g: int) -> np.ndarray:
+    """The decode-tile items of a four-head plan as one record per KV head: item (kv_head h, part_row p)
+    stands for heads h .. h + 3, head h + w writing partial rows p + w * n_q * g."""
+    assert (reg["kv_head"] % 4 == 0).all() and (reg["n_q"] * g <= HEADS4_ROWS).all()
+    out = np.repeat(reg, 4)
+    w = np.tile(np.arange(4, dtype=np.int32), len(reg))
+    out["kv_head"] += w
+    part = out["part_row"] >= 0
+    out["part_row"][part] += (w * out["n_q"] * g)[part]
+    return out
 
 
 def item_tokens(plan: dict, it) -> np.ndarray:
@@ -96,8 +113,8 @@ def check_coverage(plan: dict, cu_q, seq_lens, num_q_heads: int, num_kv_heads: i
         assert len(tok) == it["n_q"] and int(tok[0]) == int(it["q_begin"]) and (np.diff(tok) > 0).all()
     for it in plan["reg_items"]:
         assert it["pos0"] > -2
-    assert (items["part_row"] >= -1).all() and h["flags"] in (0, 1)
-    if h["flags"] == 1:  # side by side: both lists run at once
+    assert (items["part_row"] >= -1).all() and h["flags"] in (0, 1, 2, 3)
+    if h["flags"] & PLAN_CORUN:  # side by side: both lists run at once
         assert len(plan["reg_items"]) > 0 and len(plan["tc_items"]) > 0
     direct = items[items["part_row"] == -1]
     for it in direct:

@@ -39,7 +39,7 @@ def test_exports_match_header(api):
 
 
 def test_version_and_strings(api):
-    assert api._lib.pkv_abi_version() == 3
+    assert api._lib.pkv_abi_version() == 4
     assert api.status_string(0) == "ok" and api.status_string(4) == "buffer too small"
 
 
@@ -317,13 +317,13 @@ def test_plan_side_by_side(api):
     w = W.mixed_bf16(n_decode=30, n_prefill=2, chunk=300, block_size=16, cached_lo_blocks=1, cached_hi_blocks=20)
     d = PD.decode(_plan(api, w, num_ctas=200, tc_num_ctas=48).buffer)
     h = d["header"]
-    assert h["flags"] == 1 and h["num_ctas"] == 200 and h["tc_num_ctas"] == 48
+    assert h["flags"] & PD.PLAN_CORUN and h["num_ctas"] == 200 and h["tc_num_ctas"] == 48
     PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
                       w.block_size)
-    assert PD.decode(_plan(api, w, num_ctas=200, tc_num_ctas=-1).buffer)["header"]["flags"] == 0
-    assert PD.decode(_plan(api, w, num_ctas=200).buffer)["header"]["flags"] == 0
+    assert not PD.decode(_plan(api, w, num_ctas=200, tc_num_ctas=-1).buffer)["header"]["flags"] & PD.PLAN_CORUN
+    assert not PD.decode(_plan(api, w, num_ctas=200).buffer)["header"]["flags"] & PD.PLAN_CORUN
     wd = W.llama3_8b_decode_bf16(batch=9, lo=10, hi=900)
-    assert PD.decode(_plan(api, wd, num_ctas=200, tc_num_ctas=48).buffer)["header"]["flags"] == 0
+    assert not PD.decode(_plan(api, wd, num_ctas=200, tc_num_ctas=48).buffer)["header"]["flags"] & PD.PLAN_CORUN
     with pytest.raises(api.PkvError):
         _plan(api, w, num_ctas=0, tc_num_ctas=48)
 
@@ -350,3 +350,69 @@ def test_plan_groups_sharers_that_are_not_neighbours(api):
                  num_kv_heads=8, head_dim=64, block_size=16, seq_lens=[300] * 9, q_lens=[1] * 9,
                  shared_prefix_tokens=256, prefix_groups=2)
     assert _plan(api, w8).info["num_groups"] == 0
+
+
+H4_OK = [c for c in CASES if c[0] not in ("tiny",)]
+
+
+@pytest.mark.parametrize("name,make,opts", H4_OK, ids=[c[0] for c in H4_OK])
+def test_plan_four_head_items_cover_every_key_once(api, name, make, opts):
+    """heads_per_item = 4: every decode-tile item covers KV heads 4j .. 4j + 3 of one query tile and
+    key range, at most 8 rows a head, its heads' partial rows consecutive; expanded per head, the
+    plan still covers every (token, KV head) key range once.  The tcgen05 list keeps one head an
+    item, and the item count is the tensor-memory items plus a quarter of the one-head decode items
+    for the same split."""
+    w = make()
+    if w.kv_dtype == "e4m3" and w.head_dim != 128:
+        pytest.skip("fp8 pools of head_dim 64 run on the cp.async kernel")
+    g = w.num_q_heads // w.num_kv_heads
+    if any(q * g > PD.HEADS4_ROWS and q * g <= PD.DECODE_ROWS for q in np.diff(w.cu_q_lens)):
+        with pytest.raises(api.PkvError):
+            _plan(api, w, heads_per_item=4, **opts)
+        return
+    p = _plan(api, w, heads_per_item=4, **opts)
+    d = PD.decode(p.buffer)
+    h = d["header"]
+    assert p.info["heads_per_item"] == 4 and h["flags"] & PD.PLAN_HEADS4
+    reg = d["reg_items"]
+    assert (reg["kv_head"] % 4 == 0).all() and (reg["n_q"] * g <= PD.HEADS4_ROWS).all()
+    assert (d["tc_items"]["n_q"] * g > PD.DECODE_ROWS).all()
+    PD.check_coverage(d, w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal, w.block_tables,
+                      w.block_size)
+    one = _plan(api, w, heads_per_item=1, **opts)
+    if opts.get("kv_split", 0) != 0:  # the same pieces: a quarter of the decode items
+        d1 = PD.decode(one.buffer)
+        assert len(reg) * 4 == len(d1["reg_items"]) and len(d["tc_items"]) == len(d1["tc_items"])
+    assert one.info["heads_per_item"] == 1 and not PD.decode(one.buffer)["header"]["flags"] & PD.PLAN_HEADS4
+
+
+def test_plan_four_head_choice_and_rules(api):
+    """Automatic: four-head items for short decode ranges (the shared-prefix batch's suffixes) and
+    on NVFP4 pools, one head for long ranges on the others (the 8B decode batch, the long-context
+    batch).  Refused: other values,
+    KV heads not a multiple of 4, pools without the TMA-fed decode kernel, decode tiles of more
+    than 8 rows."""
+    assert _plan(api, W.prefix_reuse_bf16()).info["heads_per_item"] == 4
+    assert _plan(api, W.llama3_8b_decode_bf16()).info["heads_per_item"] == 1
+    assert _plan(api, W.longctx_fp8()).info["heads_per_item"] == 1
+    assert _plan(api, W.llama3_8b_decode_nvfp4()).info["heads_per_item"] == 4
+    w = W.llama3_8b_decode_bf16(batch=9, lo=10, hi=900)
+    for bad in (2, 3, 8, -1):
+        with pytest.raises(api.PkvError):
+            _plan(api, w, heads_per_item=bad)
+    cases = [
+        W.build("h6", seed=3, kv_dtype="bf16", num_q_heads=12, num_kv_heads=6, head_dim=128, block_size=16,
+                seq_lens=[40, 70], q_lens=[1, 1]),                           # 6 KV heads
+        W.build("b4", seed=3, kv_dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=4,
+                seq_lens=[40, 70], q_lens=[1, 1]),                           # cp.async kernel
+        W.build("f8", seed=3, kv_dtype="e4m3", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32, num_kv_heads=8,
+                head_dim=64, block_size=16, seq_lens=[40, 70], q_lens=[1, 1]),  # 64-byte fp8 rows
+        W.build("f32", seed=3, kv_dtype="f32", num_q_heads=8, num_kv_heads=4, head_dim=64, block_size=16,
+                seq_lens=[40, 70], q_lens=[1, 1]),                           # fp32 kernel
+        W.build("r12", seed=3, kv_dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                seq_lens=[40, 70], q_lens=[3, 1]),                           # a 12-row decode tile
+    ]
+    for bad in cases:
+        with pytest.raises(api.PkvError):
+            _plan(api, bad, heads_per_item=4)
+        assert _plan(api, bad).info["heads_per_item"] == 1

@@ -171,14 +171,17 @@ SIDE_CASES = {
 }
 
 
+@pytest.mark.parametrize("heads", [1, 0])
 @pytest.mark.parametrize("ctas", [(40, 4), (7, 2), (200, 60)])
 @pytest.mark.parametrize("kind", list(SIDE_CASES))
-def test_side_by_side(pkv, kind, ctas):
+def test_side_by_side(pkv, kind, ctas, heads):
     """The tcgen05 tiles (prefill chunks, shared-prefix group tiles) and the decode tiles running
-    at the same time on disjoint SMs, with forced CTA counts (rings wrapping in both kernels)."""
+    at the same time on disjoint SMs, with forced CTA counts (rings wrapping in both kernels), with
+    one-head decode items and with the planner's choice (four-head items where it takes them)."""
     w = SIDE_CASES[kind]()
-    plan, _ = run_case(pkv, w, num_ctas=ctas[0], tc_num_ctas=ctas[1])
-    assert PD.decode(plan.buffer)["header"]["flags"] == 1
+    plan, _ = run_case(pkv, w, num_ctas=ctas[0], tc_num_ctas=ctas[1], heads_per_item=heads)
+    flags = PD.decode(plan.buffer)["header"]["flags"]
+    assert flags & PD.PLAN_CORUN and (heads == 0 or not flags & PD.PLAN_HEADS4)
 
 
 @pytest.mark.parametrize("q_dtype", ["bf16", "f16"])
@@ -434,6 +437,56 @@ def test_unowned_slots_do_not_reach_the_output(pkv, kv):
     assert_close(gpu_out_f64(outs[0]), ref, w.kv_dtype)
 
 
+# ---- four-head decode items --------------------------------------------------
+
+def _h4_decode(name, seed, kv, hq, hkv, D, B, n, hi, q_len=1, q_dtype=None):
+    r = np.random.default_rng(seed)
+    extra = {} if q_dtype is None else {"q_dtype": q_dtype, "kv_in_dtype": "f32"}
+    return W.build(name, seed=seed, kv_dtype=kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=D, block_size=B,
+                   seq_lens=r.integers(q_len, hi, size=n), q_lens=[q_len] * n, **extra)
+
+
+H4_CASES = {
+    "bf16_g4": lambda: W.llama3_8b_decode_bf16(batch=7, lo=1, hi=1500),
+    "f16_d64_g2": lambda: _h4_decode("h4a", 41, "f16", 32, 16, 64, 16, 9, 2000),
+    "bf16_g8_block8": lambda: _h4_decode("h4b", 42, "bf16", 64, 8, 128, 8, 6, 900),
+    "bf16_two_tokens": lambda: _h4_decode("h4c", 43, "bf16", 32, 8, 128, 32, 5, 700, q_len=2),
+    "fp8_g4": lambda: _h4_decode("h4d", 44, "e4m3", 32, 8, 128, 64, 6, 3000, q_dtype="bf16"),
+    "fp8_f16q_block16": lambda: _h4_decode("h4e", 45, "e4m3", 32, 8, 128, 16, 5, 1200, q_dtype="f16"),
+    "nvfp4_g4": lambda: _h4_decode("h4f", 46, "nvfp4", 32, 8, 128, 64, 6, 2500, q_dtype="bf16"),
+    "nvfp4_g8_block16": lambda: _h4_decode("h4g", 47, "nvfp4", 64, 8, 128, 16, 4, 900, q_dtype="f16"),
+    "prefix_g8": lambda: W.prefix_reuse_bf16(n_req=37, prefix=512, suf_lo=1, suf_hi=300),
+}
+
+
+@pytest.mark.parametrize("split", [0, -1, 64])
+@pytest.mark.parametrize("kind", list(H4_CASES))
+def test_four_head_items(pkv, kind, split):
+    """Plans whose decode items cover four KV heads (one consumer warp a head, no merge between
+    warps): every pool kind of the TMA-fed decode kernel, g 2 to 8, one and two query tokens,
+    blocks smaller than a tile, split and unsplit key ranges, shared-prefix members' suffixes."""
+    w = H4_CASES[kind]()
+    plan, _ = run_case(pkv, w, heads_per_item=4, kv_split=split, num_ctas=40)
+    assert plan.info["heads_per_item"] == 4
+    d = PD.decode(plan.buffer)
+    assert d["header"]["flags"] & PD.PLAN_HEADS4 and (d["reg_items"]["kv_head"] % 4 == 0).all()
+
+
+@pytest.mark.parametrize("ctas", [1, 3])
+@pytest.mark.parametrize("kind", ["bf16_g4", "nvfp4_g4"])
+def test_four_head_items_few_ctas(pkv, kind, ctas):
+    """Few CTAs run many four-head items in turn: the warps' stage rings and staging rows carry
+    from item to item without an end-of-item barrier."""
+    run_case(pkv, H4_CASES[kind](), check_pool=False, heads_per_item=4, num_ctas=ctas)
+
+
+@pytest.mark.parametrize("window", [1, 100])
+def test_four_head_items_window(pkv, window):
+    w = _h4_decode("h4w", 48, "bf16", 32, 8, 128, 16, 7, 2000)
+    w.window = window
+    run_case(pkv, w, heads_per_item=4, num_ctas=40)
+
+
 @pytest.mark.parametrize("kv", ["e4m3", "nvfp4"])
 def test_bad_block_id_in_quantised_pools(pkv, kv):
     """fp8 and NVFP4 decode tiles: a block id outside the pool inside a sequence's range is
@@ -482,6 +535,8 @@ TIMEOUT_CASES = {
     # the same batch with the two kernels side by side
     "mixed_bf16_side_by_side": lambda: W.mixed_bf16(n_decode=3, n_prefill=1, chunk=150, dec_lo=50, dec_hi=900,
                                                     cached_lo_blocks=1, cached_hi_blocks=3),
+    # four-head decode items (no end-of-item barrier between the warps)
+    "decode_bf16_heads4": lambda: W.llama3_8b_decode_bf16(batch=5, lo=100, hi=2000),
 }
 
 
@@ -496,9 +551,12 @@ def test_wait_timeout_is_reported(pkv, kind):
     dw = runner.DeviceWorkload(w)
     dw.append_new()
     side = {"tc_num_ctas": 4} if kind.endswith("side_by_side") else {}
+    if kind.endswith("heads4"):
+        side = {"heads_per_item": 4}
     plan = dw.plan(num_ctas=16, wait_limit_kcycles=200, debug_flags=api.PKV_DEBUG_WITHHOLD_LOADS, **side)
     if side:
-        assert PD.decode(plan.buffer)["header"]["flags"] == 1
+        flag = PD.PLAN_HEADS4 if kind.endswith("heads4") else PD.PLAN_CORUN
+        assert PD.decode(plan.buffer)["header"]["flags"] == flag
     out = torch.zeros_like(dw.q)
     dw.attention(plan, out=out)
     torch.cuda.synchronize()
