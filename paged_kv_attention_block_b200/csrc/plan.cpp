@@ -391,8 +391,9 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   // 2b. Side by side.  With both decode-sized tiles (HBM-bound) and tensor-memory tiles
   // (tensor-bound) in the batch, the tcgen05 kernel may take k SMs and the decode-tile kernel the
   // others at the same time instead of one after the other.  Estimated times: the tensor-memory
-  // list at kTcFlopsPerSm a CTA, the decode-tile list at the smaller of the HBM stream rate and
-  // kRegBytesPerSm an SM, plus kRegItemSec per item and CTA.  Only for automatic CTA counts.
+  // list at kTcFlopsPerSm a CTA (in whole rounds of its unsplit group tiles), the decode-tile list
+  // at the smaller of the HBM stream rate and kRegBytesPerSm an SM, plus kRegItemSec per item and
+  // CTA.  Only for automatic CTA counts.
   bool corun = false;
   if (req->tc_num_ctas > 0) {
     if (tc && total_cost[0] > 0 && total_cost[1] > 0) {
@@ -410,7 +411,17 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
     for (const Tile& t : tiles) n_reg_pieces += is_tc(t.n_q * g) ? 0 : 1;
     const double reg_items = double(n_reg_pieces) * Hkv / hpi;
     const double tc_rate = f8 ? kTcFp8FlopsPerSm : kTcFlopsPerSm;
-    auto t_tc = [&](int k) { return flops / (double(k) * tc_rate); };
+    // Shared-prefix group tiles are never split: k CTAs take them in ceil(G / k) rounds of the
+    // largest one at least (128 tiles: 64 CTAs finish in two rounds, 63 need three).
+    double g_items = 0, g_flops = 0;
+    for (size_t i = 0; i < n_group_pieces; ++i)
+      if (pieces[i].tc) {
+        g_items += Hkv;
+        g_flops = std::max(g_flops, double(pieces[i].cost16) * 4.0 * D);
+      }
+    auto t_tc = [&](int k) {
+      return std::max(flops / double(k), std::ceil(g_items / double(k)) * g_flops) / tc_rate;
+    };
     auto t_reg = [&](int n) {
       return bytes / std::min(kHbmBytes, double(n) * (f8 ? kRegFp8BytesPerSm : kRegBytesPerSm)) +
              reg_items * kRegItemSec / double(n * per_sm);
@@ -434,13 +445,14 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
   // Longest key range of one item of a tile's list; the automatic length (about two items per
   // CTA on the decode kernel, three on the tcgen05 kernel, whose CTAs take items in turn
   // from a longer queue and whose merges spread over 16-row chunks; a four-head item a quarter
-  // of a one-head item's keys) is scaled by `mult`.
+  // of a one-head item's keys, but at least 512, so that short ranges such as shared-prefix
+  // members' suffixes stay whole and merge two parts) is scaled by `mult`.
   auto max_keys_for = [&](int rows, bool t, double mult) -> int32_t {
     const int64_t tile_keys = t ? PKV_TC_TILE_KEYS : PKV_TILE_KEYS;
     int64_t max_keys;
     if (req->kv_split < 0) max_keys = INT32_MAX;
     else if (req->kv_split > 0) max_keys = round_up(req->kv_split, tile_keys);
-    else max_keys = std::max<int64_t>(std::max<int64_t>(256, 2 * tile_keys),
+    else max_keys = std::max<int64_t>(std::max<int64_t>(heads_of(t) == 4 ? 512 : 256, 2 * tile_keys),
                                       round_up(int64_t(std::ceil(target[t] * mult * 16.0 /
                                                                  (double(weight16(rows)) * heads_of(t)))),
                                                tile_keys));
