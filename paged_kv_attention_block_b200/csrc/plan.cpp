@@ -25,6 +25,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <functional>
 #include <iterator>
 #include <vector>
 
@@ -76,7 +77,7 @@ struct Scratch {
   std::vector<int32_t> run_seqs, rest_seqs;
   std::vector<uint64_t> keys, tmp;
   std::vector<CostRun> runs;                       // tail check: runs of equal-cost items
-  std::vector<uint64_t> loads_a, loads_b, merged;  // tail check: CTA loads
+  std::vector<uint64_t> loads_a;                   // tail check: CTA loads (a min-heap)
 };
 
 Scratch& scratch() {
@@ -488,14 +489,16 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
       return n_items;
     };
     const size_t N = count_items(1.0), C = size_t(num_ctas);
-    if (N > C && N < 4 * C && (N % C) * 4 < C) {
-      // The counter's greedy assignment, simulated over runs of equal-cost items: items come
-      // heaviest first and each goes to the least loaded CTA.  Within a run the loads an item
-      // lands on only grow, so the updated loads form a second ascending queue beside the
-      // untouched ones; a run is O(items) and the two queues are merged between runs.
+    // A longer piece length that leaves the item count unchanged leaves every tile's piece count,
+    // and so the plan, unchanged (piece counts only fall as the length grows): nothing to try
+    // when even the longest candidate gives N items (shared-prefix suffixes, already whole).
+    if (N > C && N < 4 * C && (N % C) * 4 < C && count_items(1.5) != N) {
+      // The counter's greedy assignment, simulated: items come heaviest first and each goes to
+      // the least loaded CTA (a min-heap of the CTAs' loads; which of equally loaded CTAs takes
+      // an item does not change the loads).  This branch has fewer than 4 items a CTA, so a
+      // simulation is O(items log CTAs) whatever the number of distinct item costs.
       std::vector<CostRun>& runs = sc.runs;
       std::vector<uint64_t>& A = sc.loads_a;
-      std::vector<uint64_t>& Bq = sc.loads_b;
       auto makespan = [&](double mult) {
         runs.clear();
         for (size_t i = 0; i < n_group_pieces; ++i)  // shared-prefix group items, never split
@@ -516,25 +519,19 @@ extern "C" pkv_status pkv_attention_plan(const pkv_plan_request* req, void* plan
           runs.push_back({uint64_t(n - (nseg - 1) * seg) * w16, uint32_t(Hkv / hpi)});
         }
         std::sort(runs.begin(), runs.end(), [](const CostRun& x, const CostRun& y) { return x.cost16 > y.cost16; });
-        A.assign(size_t(num_ctas), 0);
-        for (size_t r = 0; r < runs.size();) {
-          const uint64_t c = runs[r].cost16;
-          uint64_t cnt = 0;
-          for (; r < runs.size() && runs[r].cost16 == c; ++r) cnt += runs[r].count;
-          Bq.clear();
-          size_t ia = 0, ib = 0;
-          for (uint64_t k = 0; k < cnt; ++k) {
-            const bool from_a = ia < A.size() && (ib >= Bq.size() || A[ia] <= Bq[ib]);
-            Bq.push_back((from_a ? A[ia++] : Bq[ib++]) + c);
+        A.assign(size_t(num_ctas), 0);  // all zero: already a heap
+        const auto later = std::greater<uint64_t>();
+        for (const CostRun& run : runs)
+          for (uint32_t k = 0; k < run.count; ++k) {
+            std::pop_heap(A.begin(), A.end(), later);
+            A.back() += run.cost16;
+            std::push_heap(A.begin(), A.end(), later);
           }
-          sc.merged.clear();
-          std::merge(A.begin() + long(ia), A.end(), Bq.begin() + long(ib), Bq.end(), std::back_inserter(sc.merged));
-          A.swap(sc.merged);
-        }
-        return A.empty() ? 0.0 : double(A.back());
+        return A.empty() ? 0.0 : double(*std::max_element(A.begin(), A.end()));
       };
       double best = makespan(1.0);
       for (double mult : {1.125, 1.25, 1.375, 1.5}) {
+        if (count_items(mult) == N) continue;  // the same plan as mult 1
         const double t = makespan(mult);
         if (t < best * 0.98) {
           best = t;
