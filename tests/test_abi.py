@@ -416,3 +416,21 @@ def test_plan_four_head_choice_and_rules(api):
         with pytest.raises(api.PkvError):
             _plan(api, bad, heads_per_item=4)
         assert _plan(api, bad).info["heads_per_item"] == 1
+
+
+def test_plan_tail_check_stays_cheap(api):
+    """The tail check's schedule simulation is O(items log CTAs): the shared-prefix batch on 168
+    decode CTAs (512 four-head items of 256 distinct lengths, just past three rounds, where no longer
+    piece length changes the item count) plans in well under a millisecond (about 70 us on a
+    desktop core; 580 us with a per-distinct-cost merge of all CTA loads)."""
+    import time
+    w = W.prefix_reuse_bf16()
+    pl = api.Planner(w.cu_q_lens, w.seq_lens, w.block_tables, num_q_heads=w.num_q_heads,
+                     num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype,
+                     causal=w.causal, num_ctas=168)
+    p = pl.plan()
+    assert p.info["heads_per_item"] == 4 and p.info["num_items"] == 640
+    t0 = time.perf_counter()
+    for _ in range(50):
+        pl.plan()
+    assert (time.perf_counter() - t0) / 50 < 1e-3
