@@ -9,7 +9,7 @@
 //
 //   * Two persistent CTAs per SM: warp 4 is the producer, warps 0-3 consume.
 //     The producer pulls items from the atomic counter (one item ahead),
-//     publishes each item in a 4-slot descriptor ring, and streams the item's
+//     publishes each item in a 2-slot descriptor ring, and streams the item's
 //     K/V tiles (TK keys: 32 for 256-byte rows, 64 for 128-byte rows) into an
 //     NST-stage shared-memory ring with 5-D TMA loads, 128-byte swizzle,
 //     completion counted on an mbarrier.  Block ids arrive 32 at a time through
