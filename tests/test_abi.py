@@ -386,6 +386,20 @@ def test_plan_four_head_items_cover_every_key_once(api, name, make, opts):
     assert one.info["heads_per_item"] == 1 and not PD.decode(one.buffer)["header"]["flags"] & PD.PLAN_HEADS4
 
 
+def test_plan_four_head_group_items_on_nvfp4(api):
+    """On an NVFP4 pool a run of sharers reads its prefix as decode-tile group items; with four heads
+    an item, head hh of a group item still writes member m's rows at part0 + hh * rows + offset, where
+    the members' merges look for them."""
+    w = W.build("nvp", seed=49, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32, num_kv_heads=8,
+                head_dim=128, block_size=16, seq_lens=300 + np.arange(9) * 13, q_lens=[1] * 9,
+                shared_prefix_tokens=256)
+    for heads in (1, 4):
+        p = _plan(api, w, heads_per_item=heads, num_ctas=40)
+        assert p.info["num_groups"] == 1 and p.info["heads_per_item"] == heads
+        PD.check_coverage(PD.decode(p.buffer), w.cu_q_lens, w.seq_lens, w.num_q_heads, w.num_kv_heads, w.causal,
+                          w.block_tables, w.block_size)
+
+
 def test_plan_four_head_choice_and_rules(api):
     """Automatic: four-head items for short decode ranges (the shared-prefix batch's suffixes) and
     on NVFP4 pools, one head for long ranges on the others (the 8B decode batch, the long-context

@@ -472,6 +472,17 @@ def test_four_head_items(pkv, kind, split):
     assert d["header"]["flags"] & PD.PLAN_HEADS4 and (d["reg_items"]["kv_head"] % 4 == 0).all()
 
 
+@pytest.mark.parametrize("heads", [1, 4])
+def test_nvfp4_shared_prefix_groups(pkv, heads):
+    """NVFP4 pools have no tcgen05 kernel: a run of sharers reads its prefix as decode-tile group
+    items (at most 8 rows), one or four KV heads an item, merged with each member's own suffix."""
+    w = W.build("nvp", seed=49, kv_dtype="nvfp4", q_dtype="bf16", kv_in_dtype="f32", num_q_heads=32, num_kv_heads=8,
+                head_dim=128, block_size=16, seq_lens=300 + np.arange(9) * 13, q_lens=[1] * 9,
+                shared_prefix_tokens=256)
+    plan, _ = run_case(pkv, w, heads_per_item=heads, num_ctas=40)
+    assert plan.info["num_groups"] == 1 and plan.info["heads_per_item"] == heads
+
+
 @pytest.mark.parametrize("ctas", [1, 3])
 @pytest.mark.parametrize("kind", ["bf16_g4", "nvfp4_g4"])
 def test_four_head_items_few_ctas(pkv, kind, ctas):
