@@ -472,11 +472,11 @@ PKV_DEVICE void dec_tile_fp4(DecState<D, KV_NVFP4, QBF, 1>& st, const DecOffsets
           const uint32_t sel = (b << 4) | (b << 12);
           const uint32_t sg = hmul2(e4m3_b13_f16x2(__byte_perm(w0, 0, sel)), kF16Pow2_15x2);
           const uint32_t sg8 = hmul2(e4m3_b13_f16x2(__byte_perm(w1, 0, sel)), kF16Pow2_15x2);
-          const uint32_t lo = r[2 * cc], hi = r[2 * cc + 1];
-          const uint32_t k0[4] = {hmul2(e2m1_pair_f16x2<0>(lo), sg), hmul2(e2m1_pair_f16x2<0>(hi), sg8),
-                                  hmul2(e2m1_pair_f16x2<1>(lo), sg), hmul2(e2m1_pair_f16x2<1>(hi), sg8)};
-          const uint32_t k1[4] = {hmul2(e2m1_pair_f16x2<2>(lo), sg), hmul2(e2m1_pair_f16x2<2>(hi), sg8),
-                                  hmul2(e2m1_pair_f16x2<3>(lo), sg), hmul2(e2m1_pair_f16x2<3>(hi), sg8)};
+          uint32_t pl[4], ph[4];  // nibble pairs (i, i+4) of the lo and hi words
+          e2m1_word_f16x2(r[2 * cc], pl);
+          e2m1_word_f16x2(r[2 * cc + 1], ph);
+          const uint32_t k0[4] = {hmul2(pl[0], sg), hmul2(ph[0], sg8), hmul2(pl[1], sg), hmul2(ph[1], sg8)};
+          const uint32_t k1[4] = {hmul2(pl[2], sg), hmul2(ph[2], sg8), hmul2(pl[3], sg), hmul2(ph[3], sg8)};
           const int ks = 2 * (2 * p + cc);
           mma16816<false>(s4, k0, st.qb[0][ks][0], st.qb[0][ks][1]);
           mma16816<false>(s4, k1, st.qb[0][ks + 1][0], st.qb[0][ks + 1][1]);
@@ -541,14 +541,14 @@ PKV_DEVICE void dec_tile_fp4(DecState<D, KV_NVFP4, QBF, 1>& st, const DecOffsets
                               hmul2(e4m3_b13_f16x2(__byte_perm(a0w, a1w, selB)), kF16Pow2_15x2),
                               hmul2(e4m3_b13_f16x2(__byte_perm(b0w, b1w, selA)), kF16Pow2_15x2),
                               hmul2(e4m3_b13_f16x2(__byte_perm(b0w, b1w, selB)), kF16Pow2_15x2)};
+      uint32_t px[4][4];  // word k's nibble pairs (i, i+4)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) e2m1_word_f16x2(x[k], px[k]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         // m-tile 4p + i: rows g4 -> dim 64p + 4 g4 + i, rows g4 + 8 -> dim 64p + 32 + 4 g4 + i.
-        uint32_t a[4];
-        a[0] = hmul2(e2m1_pair_f16x2_dyn(x[0], i), sc[0]);
-        a[1] = hmul2(e2m1_pair_f16x2_dyn(x[1], i), sc[1]);
-        a[2] = hmul2(e2m1_pair_f16x2_dyn(x[2], i), sc[2]);
-        a[3] = hmul2(e2m1_pair_f16x2_dyn(x[3], i), sc[3]);
+        const uint32_t a[4] = {hmul2(px[0][i], sc[0]), hmul2(px[1][i], sc[1]), hmul2(px[2][i], sc[2]),
+                               hmul2(px[3][i], sc[3])};
         mma16816<false>(st.acc[0][4 * p + i], a, pb0, pb1);
       }
     }

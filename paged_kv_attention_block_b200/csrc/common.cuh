@@ -55,10 +55,17 @@ PKV_DEVICE uint32_t e2m1_pair_f16x2(uint32_t w) {
   const uint32_t x = w << (12 - 4 * I);  // nibble I -> bits 12..15, nibble I+4 -> bits 28..31
   return ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
 }
-// The same for a pair index known only at run time (I in 0..3).
-PKV_DEVICE uint32_t e2m1_pair_f16x2_dyn(uint32_t w, int I) {
-  const uint32_t x = w << (12 - 4 * I);
-  return ((x >> 3) & 0x0E000E00u) | (x & 0x80008000u);
+// All four nibble pairs (i, i + 4) of w at once, p[i] = e2m1_pair_f16x2<i>(w), in 13 integer
+// operations instead of 15: in every byte of the even and of the odd nibbles one multiply-add
+// (n + 7 (n & 8)) moves the sign from bit 3 to bit 6, leaving the magnitude in bits 0-2 with three
+// zero bits between (the f16 pattern); after a shift by one, byte permutes place the bytes.
+PKV_DEVICE void e2m1_word_f16x2(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t e = w & 0x0F0F0F0Fu, o = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t es = (e + 7u * (e & 0x08080808u)) << 1, os = (o + 7u * (o & 0x08080808u)) << 1;
+  p[0] = __byte_perm(es, 0, 0x2404);  // nibbles 0, 4 (bytes 0, 2 of the even nibbles)
+  p[2] = __byte_perm(es, 0, 0x3414);  // nibbles 2, 6
+  p[1] = __byte_perm(os, 0, 0x2404);  // nibbles 1, 5
+  p[3] = __byte_perm(os, 0, 0x3414);  // nibbles 3, 7
 }
 constexpr uint32_t kF16Pow2_15x2 = 0x78007800u;  // f16x2 (2^15, 2^15)
 // f16x2 product, round to nearest (exact for the scaled E2M1 and E4M3 values multiplied here).
