@@ -302,7 +302,9 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  * has such tiles) and, when the plan split a key range, one merge kernel (the
  * same merge pkv_split_kv_reduce performs), in that order on `stream`; a plan
  * made side by side (pkv_plan_info.side_by_side) enqueues the tcgen05 kernel
- * first and the decode-tile kernel beside it, on the SMs it leaves free.
+ * first and the decode-tile kernel beside it, on the SMs it leaves free.  A plan
+ * with four-head items (pkv_plan_info.heads_per_item 4) runs the decode-tile
+ * kernel's four-head variant: one consumer warp per KV head of an item.
  *
  * q: device [total_q][num_q_heads][head_dim], q_dtype F32 (F32 pools only),
  *   BF16 (BF16, FP8 or NVFP4 pools) or F16 (F16, FP8 or NVFP4 pools).
@@ -312,9 +314,11 @@ PKV_API pkv_status pkv_default_num_ctas(int32_t kv_dtype, int32_t head_dim, int3
  * block_tables: device int32 [num_seqs][max_blocks].
  * softmax_scale: scale on q.k (typically 1/sqrt(head_dim)), positive and finite;
  *   causal as planned.  fp8 and NVFP4 scales must be positive.
- * plan: host buffer from pkv_attention_plan for these shapes.  It is copied to
- *   the workspace with cudaMemcpyAsync; use page-locked memory for an
- *   asynchronous copy and keep it unchanged until the copy has run.
+ * plan: host buffer from pkv_attention_plan for these shapes.  It is staged in
+ *   the workspace on `stream`: a page-locked plan by a kernel that reads it
+ *   through its device alias (launched as a programmatic dependent of the work
+ *   ahead of it), any other plan by cudaMemcpyAsync.  Keep it unchanged until
+ *   the staging has run.
  * out: device [total_q][num_q_heads][head_dim] in q_dtype.
  * out_lse: device float32 [total_q][num_q_heads] natural-log sum of exp(scores)
  *   per row, or NULL.
