@@ -448,3 +448,41 @@ def test_plan_tail_check_stays_cheap(api):
     for _ in range(50):
         pl.plan()
     assert (time.perf_counter() - t0) / 50 < 1e-3
+
+
+def _attention_status(api, w, plan_buf):
+    """pkv_paged_attention's synchronous status for a (possibly edited) host plan, with placeholder
+    device pointers: plan validation comes before any CUDA call."""
+    c = _cache(num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=w.block_size,
+               kv_dtype=api.DTYPE_CODES[w.kv_dtype], num_blocks=w.num_blocks)
+    fake = 0x10000
+    return api._lib.pkv_paged_attention(C.byref(c), fake, api.PKV_BF16, w.num_q_heads, fake, fake, fake,
+                                        w.block_tables.shape[1], w.num_seqs, 0.1, int(w.causal),
+                                        plan_buf.data_ptr(), fake, None, fake, 1 << 30, None, None)
+
+
+def test_paged_attention_refuses_broken_four_head_plans(api):
+    """A four-head plan is checked before anything is enqueued: a decode item whose first KV head is not a
+    multiple of 4 or that carries more than 8 rows a head, and the four-head flag on a pool whose
+    decode tiles run on a kernel without four-head items, return PKV_ERR_PLAN (5)."""
+    w = W.llama3_8b_decode_bf16(batch=9, lo=10, hi=900)
+    good = _plan(api, w, heads_per_item=4, num_ctas=40)
+    base = good.buffer.clone()
+    h = PD.decode(base)["header"]
+    off = int(h["items_off"])
+    for field, value in (("kv_head", 1), ("n_q", 3)):  # kv_head 1; 3 tokens x 4 heads = 12 rows
+        bad = base.clone()
+        items = np.frombuffer(bad.numpy(), dtype=PD.ITEM, count=int(h["n_items"]), offset=off).copy()
+        items[0][field] = value
+        bad[off:off + items.nbytes] = torch.from_numpy(items.view(np.uint8))
+        assert _attention_status(api, w, bad) == 5, (field, api._lib.pkv_last_error())
+    w4 = W.build("b4", seed=3, kv_dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=4,
+                 seq_lens=[40, 70], q_lens=[1, 1])
+    p4 = _plan(api, w4, num_ctas=40)
+    assert p4.info["heads_per_item"] == 1
+    flagged = p4.buffer.clone()
+    hdr = np.frombuffer(flagged.numpy()[:128].tobytes(), PD.HEADER).copy()
+    hdr["flags"] |= PD.PLAN_HEADS4
+    flagged[:128] = torch.from_numpy(hdr.view(np.uint8).copy())
+    assert _attention_status(api, w4, flagged) == 5
+    assert b"four-head" in api._lib.pkv_last_error()
