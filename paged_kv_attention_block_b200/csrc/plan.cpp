@@ -20,7 +20,9 @@
 //
 // The work is done once per (query tile, key piece) -- a "piece" below -- and
 // expanded over the KV heads only when the items are written: a decode batch of
-// S sequences plans S tiles, not S x Hkv.  Scratch vectors live per thread and
+// S sequences plans S tiles, not S x Hkv.  A piece of the decode-tile list becomes
+// one item per KV head, or, in a four-head plan, one item per four KV heads (each
+// of the TMA-fed kernel's consumer warps then runs one head's whole key range).  Scratch vectors live per thread and
 // keep their capacity across calls, so a steady-state plan allocates nothing.
 #include <algorithm>
 #include <cmath>
